@@ -1,0 +1,406 @@
+"""Benchmark of the block-sparse attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one pass of the prefill hot path over the video-DiT workload
+(B=1, H=12, N=32768 on an 8x64x64 grid, d=128, bf16, block 128, dot router,
+keep 10% of KV blocks, zero-order tail): block statistics -> router ->
+sparse attention.  Inputs (302 MB) are larger than L2 (126 MB) and are
+generated on the device before timing.  Rank 0 prints one JSON line.
+
+With N > 1 (torchrun, one process per GPU) every rank runs its own,
+independently seeded problem of the same size: the path shards by (batch,
+head) with no exchange, so the scaling is weak and no collective touches the
+data path (NCCL only carries the timing max).
+
+--impl reference times the CPU oracle (float64 numpy) on a bounded sample of
+the same workload on the host cores (rank 0 only).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from block_sparse_approximate_b200 import workloads as wl  # noqa: E402
+
+WORKLOAD = "video_dit"
+METRIC = "sparse-attn prefill dense-equivalent TFLOPS (block_pool+route+sparse_attn_fwd step)"
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p["bf16_tflops_sustained"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def dense_flops(w) -> float:
+    return 4.0 * w.B * w.H * float(w.N) * w.N * w.d
+
+
+def algorithmic_attn_flops(w) -> float:
+    """FLOPs the method performs in the attention kernel: every query row takes
+    4·d FLOPs (QKᵀ and PV) per exact key (k blocks × block tokens) and per
+    zero-order pseudo-key (nb − k unselected blocks)."""
+    keys = w.k * w.block + ((w.nb - w.k) if w.tail == "zero_order" else 0)
+    return 4.0 * w.d * keys * w.B * w.H * float(w.N)
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 100 ms."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.f = tempfile.NamedTemporaryFile(mode="w+", suffix=".csv", delete=False)
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--id={index}", f"--query-gpu={self.FIELDS}",
+                                       "--format=csv,noheader,nounits", "-lms", "100"],
+                                      stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.p = None
+        self.marks = []
+
+    def mark(self):
+        self.marks.append(time.time())
+
+    def stop(self):
+        if self.p is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except Exception:
+            self.p.kill()
+        self.f.flush()
+        self.f.seek(0)
+        rows = [r.split(", ") for r in self.f.read().strip().splitlines() if r.strip()]
+        os.unlink(self.f.name)
+        sm = [float(r[1]) for r in rows if len(r) >= 9 and r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if len(r) >= 9 and r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in rows:
+            if len(r) >= 9:
+                for n, v in zip(names, r[5:9]):
+                    if v.strip() == "Active":
+                        reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def _dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def _max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], device="cuda", dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# --------------------------------------------------------------------------
+# CPU oracle timing (cpu_baseline leg and the reference arm)
+# --------------------------------------------------------------------------
+
+def oracle_sample(w, inp_cpu: dict, n_blocks: int, seed: int = 0):
+    """Runs the oracle's full path (stats of one head, route scores, top-k,
+    attention) for n_blocks query blocks of one head; returns (seconds,
+    dense-equivalent FLOPs of those query blocks)."""
+    import oracle
+    rng = np.random.default_rng(seed)
+    h = int(rng.integers(w.H))
+    Q = inp_cpu["Q"][:, h:h + 1].float().numpy()
+    K = inp_cpu["K"][:, h:h + 1].float().numpy()
+    V = inp_cpu["V"][:, h:h + 1].float().numpy()
+    blocks = sorted(rng.choice(w.nb, n_blocks, replace=False).tolist())
+    t0 = time.perf_counter()
+    st = oracle.block_pool(Q, K, V, w.block)
+    sc = oracle.route_scores(st["qmean"][:, :, blocks], st["kmean"], "dot")
+    idx_sel = oracle.topk_from_scores(sc, w.k)                  # [1,1,n,k]
+    idx = np.zeros((1, 1, w.nb, w.k), dtype=np.int64)
+    idx[0, 0, blocks] = idx_sel[0, 0]
+    oracle.sparse_attention(Q, K, V, idx, w.block, w.tail, w.scale,
+                            qblocks=[(0, 0, i) for i in blocks])
+    dt = time.perf_counter() - t0
+    # the stats of one head serve all its query blocks: charge them pro rata
+    return dt, 4.0 * w.block * n_blocks * float(w.N) * w.d
+
+
+def cpu_baseline(w, inp_cpu: dict, budget_s: float = 15.0) -> dict:
+    import oracle  # noqa: F401  (test infrastructure: only this leg runs it)
+    n = 2
+    dt, fl = oracle_sample(w, inp_cpu, n)
+    while dt < budget_s / 4 and n < w.nb:
+        n = min(w.nb, n * 2)
+        dt, fl = oracle_sample(w, inp_cpu, n, seed=n)
+    return {"value": fl / dt / 1e12, "unit": "TFLOPS", "cores": torch.get_num_threads(),
+            "kind": "oracle",
+            "sample": f"{n} query blocks of one head of {w.name} (of {w.H * w.nb}), full oracle path "
+                      f"(stats, route, top-k, float64 attention), {dt:.1f} s; value = dense-equivalent "
+                      f"FLOPs of the sample / time"}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return 0
+    w = wl.WORKLOADS[WORKLOAD]
+    inp = wl.prefill_inputs(w, "cpu")
+    per_step = []
+    flops = 0.0
+    for i in range(args.warmup + args.steps):
+        dt, fl = oracle_sample(w, inp, 2, seed=i)
+        if i >= args.warmup:
+            per_step.append(dt)
+            flops += fl
+    tot = sum(per_step)
+    val = flops / tot / 1e12
+    cores = torch.get_num_threads()
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOPS", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+                                            "block": w.block, "route": w.route, "keep_pct": w.keep_pct,
+                                            "tail": w.tail, "sample_per_step": "2 query blocks"},
+            "cpu_baseline": {"value": val, "unit": "TFLOPS", "cores": cores, "kind": "oracle",
+                             "sample": "each step: the oracle's full path for 2 query blocks of one head"},
+            "e2e": {"value": val, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------
+# GPU arm
+# --------------------------------------------------------------------------
+
+def time_decode(steps: int = 50, warmup: int = 5):
+    """Decode workload timing (separate from the prefill step): GB/s of the
+    bytes the method moves per decode step."""
+    from block_sparse_approximate_b200 import binding as bd
+    from block_sparse_approximate_b200.pipeline import DecodeStep
+    w = wl.WORKLOADS["decode"]
+    inp = wl.decode_inputs(w, "cuda")
+    st = bd.block_pool(None, inp["Kcache"], inp["Vcache"], w.block, variance=True)
+    step = DecodeStep(w, inp, st)
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(steps):
+        step()
+    e.record()
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e) / steps
+    B, Hkv, nb, d = w.B, w.Hkv, w.nb, w.d
+    kv = 2.0 * B * Hkv * w.k * w.block * d * 2          # selected K and V, bf16
+    stats = 3.0 * B * Hkv * nb * d * 4                    # kmean, kvar, vsum fp32 (read once each)
+    qo = 2.0 * B * w.H * d * 2
+    byts = kv + stats + qo
+    hbm, _, _, src = _peaks()
+    del inp, st, step
+    torch.cuda.empty_cache()
+    return {"workload": "decode", "ms": ms, "bytes_per_step": byts, "gbs": byts / ms / 1e6,
+            "hbm_peak_gbs": hbm, "frac": byts / ms / 1e6 / hbm, "peak_source": src}
+
+
+def run_ours(args, world, rank, local):
+    from block_sparse_approximate_b200 import binding as bd
+    from block_sparse_approximate_b200.pipeline import PrefillStep
+    torch.cuda.set_device(local)
+    bd.load()
+    w = wl.WORKLOADS[WORKLOAD]
+    wr = wl.Workload(**{**w.__dict__, "seed": w.seed + 1000 * rank}) if rank else w
+    inp = wl.prefill_inputs(wr, "cuda")
+    step = PrefillStep(wr, inp)
+    clocks = ClockSampler(local) if rank == 0 else None
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    # timed region: K steps, attention kernel bracketed by events on the
+    # launching stream (torch's current stream, which the step launches on)
+    stream = torch.cuda.current_stream()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    lib = step.lib
+
+    def attn_only():
+        import ctypes
+        buf = step.buf
+        bd._check("sa_sparse_attn_fwd",
+                  lib.sa_sparse_attn_fwd(inp["Q"].data_ptr(), inp["K"].data_ptr(), inp["V"].data_ptr(),
+                                         step.dtype, step.shape, buf.block_idx.data_ptr(), int(wr.k),
+                                         bd.TAIL[wr.tail], None, ctypes.byref(step.cst),
+                                         float(wr.scale), buf.out.data_ptr(), stream.cuda_stream))
+
+    def pool_route():
+        import ctypes
+        buf = step.buf
+        s = stream.cuda_stream
+        bd._check("sa_block_pool", lib.sa_block_pool(inp["Q"].data_ptr(), inp["K"].data_ptr(),
+                                                     inp["V"].data_ptr(), step.dtype, step.shape,
+                                                     ctypes.byref(step.cst), s))
+        bd._check("sa_route", lib.sa_route(ctypes.byref(step.cst), step.shape, bd.ROUTE[wr.route],
+                                           None, None, float(wr.scale), int(wr.k),
+                                           buf.block_idx.data_ptr(), None, s))
+
+    _barrier(world)
+    torch.cuda.synchronize()
+    if clocks:
+        clocks.mark()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(args.steps):
+        pool_route()
+        ev[i][0].record(stream)
+        attn_only()
+        ev[i][1].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    _barrier(world)
+    if clocks:
+        clocks.mark()
+    ms_total = t0.elapsed_time(t1)
+    ms_total = _max_over_ranks(ms_total, world)
+    attn_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    ms_step = ms_total / args.steps
+
+    # end to end: pinned host inputs -> device, step, output -> host
+    e2e = None
+    if not args.no_e2e:
+        hostQ, hostK, hostV = (inp[n].cpu().pin_memory() for n in ("Q", "K", "V"))
+        hostO = torch.empty(step.buf.out.shape, dtype=step.buf.out.dtype).pin_memory()
+        for _ in range(2):
+            inp["Q"].copy_(hostQ, non_blocking=True)
+            inp["K"].copy_(hostK, non_blocking=True)
+            inp["V"].copy_(hostV, non_blocking=True)
+            step()
+            hostO.copy_(step.buf.out, non_blocking=True)
+        torch.cuda.synchronize()
+        _barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_e2e = max(3, min(args.steps, 10))
+        e0.record(stream)
+        for _ in range(n_e2e):
+            inp["Q"].copy_(hostQ, non_blocking=True)
+            inp["K"].copy_(hostK, non_blocking=True)
+            inp["V"].copy_(hostV, non_blocking=True)
+            step()
+            hostO.copy_(step.buf.out, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = _max_over_ranks(e0.elapsed_time(e1) / n_e2e, world)
+        e2e = {"value": world * dense_flops(w) / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS",
+               "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": sum(inp[n].numel() * inp[n].element_size() for n in ("Q", "K", "V")),
+               "d2h_bytes_per_step": step.buf.out.numel() * step.buf.out.element_size()}
+
+    decode = None
+    if rank == 0 and not args.no_decode:
+        del step
+        torch.cuda.empty_cache()
+        decode = time_decode()
+    ck = clocks.stop() if clocks else None
+
+    if rank != 0:
+        return 0
+    hbm, bf16, bf16_sus, src = _peaks()
+    attn_flops = algorithmic_attn_flops(w)
+    achieved = attn_flops / (attn_ms * 1e-3) / 1e12
+    cpu = None
+    if not args.no_cpu:
+        inp_cpu = {n: inp[n].cpu() for n in ("Q", "K", "V")}
+        cpu = cpu_baseline(w, inp_cpu)
+    line = {
+        "metric": METRIC, "value": world * dense_flops(w) / (ms_step * 1e-3) / 1e12, "unit": "TFLOPS",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "grid": list(w.grid), "d": w.d,
+                   "block": w.block, "route": w.route, "keep_pct": w.keep_pct, "topk": w.k,
+                   "tail": w.tail, "parallelism": f"replicas x{world} (independent problems)",
+                   "l2": "inputs larger than L2 (302 MB vs 126 MB)"},
+        "attn_ms": attn_ms,
+        "executed_tflops": achieved,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": bf16, "unit": "TFLOP/s",
+                     "frac": achieved / bf16, "traffic": None,
+                     "kernel": "sparse_attn_fwd", "peak_source": f"{src} bf16 dense (burst)"},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": args.steps * PrefillStepLaunches(w),
+        "clocks": ck,
+        "decode": decode,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def PrefillStepLaunches(w) -> int:
+    return 3 + (1 if w.tail == "linear_mix" else 0)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    world, rank, local = _dist()
+    if args.impl == "reference":
+        return run_reference(args, world, rank)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        return run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

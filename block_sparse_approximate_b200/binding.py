@@ -1,0 +1,205 @@
+"""ctypes binding of libsparseattn (argument marshalling only).
+
+Every function here validates tensor placement, allocates the outputs with
+torch on the inputs' device, passes raw device pointers and the current CUDA
+stream to the C entry point of the same name, and raises ``SparseAttnError``
+on a non-OK status.  All computation happens in the library's CUDA kernels;
+there is no fallback: if ``libsparseattn.so`` has not been built, ``load()``
+raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsparseattn.so")
+
+SA_OK, SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED, SA_ERR_ALIGNMENT, SA_ERR_CUDA, SA_ERR_WORKSPACE = range(6)
+SA_FP32, SA_BF16 = 0, 1
+ROUTE = {"dot": 0, "proj": 1, "taylor2": 2}
+TAIL = {"drop": 0, "zero_order": 1, "linear_mix": 2}
+
+# every entry point declared in include/sparseattn.h
+EXPORTS = ("sa_block_pool", "sa_route", "sa_sparse_attn_fwd", "sa_decode_workspace_size",
+           "sa_decode_fwd", "sa_last_error", "sa_version")
+
+
+class SparseAttnError(RuntimeError):
+    def __init__(self, fn: str, status: int, msg: str):
+        super().__init__(f"{fn} failed with status {status}: {msg}")
+        self.status = status
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("N", ctypes.c_int32),
+                ("d", ctypes.c_int32), ("block", ctypes.c_int32)]
+
+
+class DecodeShape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32),
+                ("N", ctypes.c_int32), ("d", ctypes.c_int32), ("block", ctypes.c_int32)]
+
+
+_STAT_FIELDS = ("qmean", "kmean", "vsum", "kvar", "zrelu", "htot", "ztot", "kmean_bf16", "vmean_bf16")
+
+
+class BlockStats(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in _STAT_FIELDS]
+
+
+_lib = None
+
+
+def load():
+    """Loads libsparseattn.so (built in-tree) and declares its signatures."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: run `python -m block_sparse_approximate_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i32, f32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
+    lib.sa_block_pool.argtypes = [vp, vp, vp, ctypes.c_int, Shape, ctypes.POINTER(BlockStats), vp]
+    lib.sa_route.argtypes = [ctypes.POINTER(BlockStats), Shape, ctypes.c_int, vp, vp, f32, i32, vp, vp, vp]
+    lib.sa_sparse_attn_fwd.argtypes = [vp, vp, vp, ctypes.c_int, Shape, vp, i32, ctypes.c_int, vp,
+                                       ctypes.POINTER(BlockStats), f32, vp, vp]
+    lib.sa_decode_workspace_size.argtypes = [DecodeShape, i32]
+    lib.sa_decode_workspace_size.restype = sz
+    lib.sa_decode_fwd.argtypes = [vp, vp, vp, ctypes.c_int, DecodeShape, ctypes.POINTER(BlockStats),
+                                  i32, f32, ctypes.c_int, vp, vp, vp, vp, sz, vp]
+    for fn in ("sa_block_pool", "sa_route", "sa_sparse_attn_fwd", "sa_decode_fwd"):
+        getattr(lib, fn).restype = ctypes.c_int
+    lib.sa_last_error.restype = ctypes.c_char_p
+    lib.sa_version.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def _check(fn: str, status: int):
+    if status != SA_OK:
+        raise SparseAttnError(fn, status, load().sa_last_error().decode())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream=None) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return SA_FP32
+    if t.dtype == torch.bfloat16:
+        return SA_BF16
+    raise ValueError(f"unsupported dtype {t.dtype}")
+
+
+def _stats_struct(stats: dict) -> BlockStats:
+    return BlockStats(*[_ptr(stats.get(n)) for n in _STAT_FIELDS])
+
+
+def version() -> str:
+    return load().sa_version().decode()
+
+
+def block_pool(Q: Optional[torch.Tensor], K: torch.Tensor, V: torch.Tensor, block: int, *,
+               variance: bool = False, linear: bool = False, centroids_bf16: bool = False,
+               stream=None) -> dict:
+    """Block statistics of (Q,) K, V [B,H,N,d]; returns a dict of float32 tensors."""
+    lib = load()
+    Bsz, H, N, d = K.shape
+    nb = N // block
+    dev = K.device
+    f = dict(device=dev, dtype=torch.float32)
+    st = {"kmean": torch.empty(Bsz, H, nb, d, **f), "vsum": torch.empty(Bsz, H, nb, d, **f)}
+    if Q is not None:
+        st["qmean"] = torch.empty(Bsz, H, nb, d, **f)
+    if variance:
+        st["kvar"] = torch.empty(Bsz, H, nb, d, **f)
+    if linear:
+        st["zrelu"] = torch.empty(Bsz, H, nb, d, **f)
+        st["htot"] = torch.empty(Bsz, H, d, d, **f)
+        st["ztot"] = torch.empty(Bsz, H, d, **f)
+    if centroids_bf16:
+        st["kmean_bf16"] = torch.empty(Bsz, H, nb, d, device=dev, dtype=torch.bfloat16)
+        st["vmean_bf16"] = torch.empty(Bsz, H, nb, d, device=dev, dtype=torch.bfloat16)
+    cst = _stats_struct(st)
+    _check("sa_block_pool", lib.sa_block_pool(_ptr(Q), _ptr(K), _ptr(V), _dtype_code(K),
+                                              Shape(Bsz, H, N, d, block), ctypes.byref(cst),
+                                              _stream(stream)))
+    return st
+
+
+def route(stats: dict, shape, mode: str, topk: int, *, proj_q=None, proj_k=None,
+          scale: float = 1.0, want_scores: bool = False, stream=None):
+    """Top-k KV blocks per query block: returns (block_idx int32 [B,H,nqb,topk], scores or None)."""
+    lib = load()
+    Bsz, H, N, d, block = shape
+    nb = N // block
+    dev = stats["kmean"].device
+    idx = torch.empty(Bsz, H, nb, topk, device=dev, dtype=torch.int32)
+    sc = torch.empty(Bsz, H, nb, nb, device=dev, dtype=torch.float32) if want_scores else None
+    cst = _stats_struct(stats)
+    _check("sa_route", lib.sa_route(ctypes.byref(cst), Shape(Bsz, H, N, d, block), ROUTE[mode],
+                                    _ptr(proj_q), _ptr(proj_k), float(scale), int(topk),
+                                    _ptr(idx), _ptr(sc), _stream(stream)))
+    return idx, sc
+
+
+def sparse_attn_fwd(Q, K, V, block_idx, block: int, tail: str, stats: dict, scale: float, *,
+                    alpha=None, out=None, stream=None) -> torch.Tensor:
+    """Sparse prefill forward; returns O with the shape and dtype of Q."""
+    lib = load()
+    Bsz, H, N, d = Q.shape
+    O = out if out is not None else torch.empty_like(Q)
+    topk = block_idx.shape[-1] if block_idx is not None else 0
+    cst = _stats_struct(stats or {})
+    _check("sa_sparse_attn_fwd",
+           lib.sa_sparse_attn_fwd(_ptr(Q), _ptr(K), _ptr(V), _dtype_code(Q),
+                                  Shape(Bsz, H, N, d, block),
+                                  _ptr(block_idx) if topk > 0 else None, int(topk), TAIL[tail],
+                                  _ptr(alpha), ctypes.byref(cst), float(scale), _ptr(O),
+                                  _stream(stream)))
+    return O
+
+
+def decode_workspace_size(B: int, Hq: int, Hkv: int, N: int, d: int, block: int, topk: int) -> int:
+    return int(load().sa_decode_workspace_size(DecodeShape(B, Hq, Hkv, N, d, block), int(topk)))
+
+
+def decode_fwd(q, Kcache, Vcache, stats: dict, block: int, topk: int, scale: float, *,
+               tail: str = "zero_order", workspace=None, want_route: bool = True, out=None,
+               stream=None):
+    """GQA decode; returns (o [B,Hq,d], block_idx [B,Hkv,topk] or None, scores [B,Hkv,nb] or None)."""
+    lib = load()
+    Bsz, Hq, d = q.shape
+    Hkv, N = Kcache.shape[1], Kcache.shape[2]
+    nb = N // block
+    dev = q.device
+    ws_bytes = decode_workspace_size(Bsz, Hq, Hkv, N, d, block, topk)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 256), device=dev, dtype=torch.uint8)
+    o = out if out is not None else torch.empty_like(q)
+    idx = torch.empty(Bsz, Hkv, topk, device=dev, dtype=torch.int32) if want_route else None
+    sc = torch.empty(Bsz, Hkv, nb, device=dev, dtype=torch.float32) if want_route else None
+    cst = _stats_struct(stats)
+    _check("sa_decode_fwd",
+           lib.sa_decode_fwd(_ptr(q), _ptr(Kcache), _ptr(Vcache), _dtype_code(q),
+                             DecodeShape(Bsz, Hq, Hkv, N, d, block), ctypes.byref(cst), int(topk),
+                             float(scale), TAIL[tail], _ptr(idx), _ptr(sc), _ptr(o),
+                             _ptr(workspace), workspace.numel(), _stream(stream)))
+    return o, idx, sc

@@ -1,0 +1,249 @@
+// Block statistics: the pre-computation step of PISA ("Implementação de
+// Hardware": block centroids and value sums), the mean pooling of SLA2's
+// router (§2B) and the block mean / diagonal covariance of SPLA's score
+// (§2.1).  HBM-bound: every input element is read once with 16-byte loads.
+#include "common.cuh"
+
+namespace sa {
+namespace {
+
+constexpr int kPoolThreads = 256;
+
+// One CTA per (block j, head h, batch b).  Thread t covers the 8 channels
+// [8*(t % COLS), +8) of rows t / COLS, t / COLS + RPP, ...  Means are reduced
+// through shared memory; the key variance is the exact two-pass form over the
+// register-resident block.
+template <typename T, int D, int BLK>
+__global__ void __launch_bounds__(kPoolThreads)
+block_pool_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __restrict__ V,
+                  int H, int N, sa_block_stats st) {
+  constexpr int COLS = D / 8;                 // 16-byte vectors per row
+  constexpr int RPP = kPoolThreads / COLS;    // rows per pass
+  constexpr int ROWS = BLK / RPP;             // rows per thread
+  static_assert(BLK % RPP == 0, "block must be a multiple of rows per pass");
+  const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int nb = N / BLK;
+  const int tid = threadIdx.x;
+  const int col = tid % COLS, r0 = tid / COLS;
+  const size_t head_off = ((size_t)b * H + h) * (size_t)N * D;
+  const size_t row0 = (size_t)j * BLK;
+  const size_t stat_off = (((size_t)b * H + h) * nb + j) * D;
+
+  __shared__ float red[RPP][D];
+  __shared__ float mean_sh[D];
+
+  auto reduce_rows = [&](float acc[8]) {
+    // sums acc over the RPP threads that share a column; result for channel
+    // c is left in red[0][c]
+#pragma unroll
+    for (int i = 0; i < 8; ++i) red[r0][col * 8 + i] = acc[i];
+    __syncthreads();
+    if (tid < D) {
+      float s = 0.f;
+#pragma unroll 8
+      for (int r = 0; r < RPP; ++r) s += red[r][tid];
+      mean_sh[tid] = s;
+    }
+    __syncthreads();
+  };
+
+  float x[ROWS][8];
+  // ---- keys: mean, variance, relu sums
+  {
+#pragma unroll
+    for (int r = 0; r < ROWS; ++r)
+      load8<T>(K + head_off + (row0 + r0 + r * RPP) * D + col * 8, x[r]);
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      float s = 0.f;
+#pragma unroll
+      for (int r = 0; r < ROWS; ++r) s += x[r][i];
+      acc[i] = s;
+    }
+    reduce_rows(acc);
+    const float inv = 1.0f / BLK;
+    float mu[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) mu[i] = mean_sh[col * 8 + i] * inv;
+    if (tid < D) {
+      const float m = mean_sh[tid] * inv;
+      st.kmean[stat_off + tid] = m;
+      if (st.kmean_bf16)
+        reinterpret_cast<__nv_bfloat16*>(st.kmean_bf16)[stat_off + tid] = __float2bfloat16_rn(m);
+    }
+    __syncthreads();
+    if (st.kvar) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float s = 0.f;
+#pragma unroll
+        for (int r = 0; r < ROWS; ++r) {
+          const float dlt = x[r][i] - mu[i];
+          s = fmaf(dlt, dlt, s);
+        }
+        acc[i] = s;
+      }
+      reduce_rows(acc);
+      if (tid < D) st.kvar[stat_off + tid] = mean_sh[tid] * inv;
+      __syncthreads();
+    }
+    if (st.zrelu) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float s = 0.f;
+#pragma unroll
+        for (int r = 0; r < ROWS; ++r) s += fmaxf(x[r][i], 0.f);
+        acc[i] = s;
+      }
+      reduce_rows(acc);
+      if (tid < D) st.zrelu[stat_off + tid] = mean_sh[tid];
+      __syncthreads();
+    }
+  }
+  // ---- values: block sums
+  {
+#pragma unroll
+    for (int r = 0; r < ROWS; ++r)
+      load8<T>(V + head_off + (row0 + r0 + r * RPP) * D + col * 8, x[r]);
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      float s = 0.f;
+#pragma unroll
+      for (int r = 0; r < ROWS; ++r) s += x[r][i];
+      acc[i] = s;
+    }
+    reduce_rows(acc);
+    if (tid < D) {
+      st.vsum[stat_off + tid] = mean_sh[tid];
+      if (st.vmean_bf16)
+        reinterpret_cast<__nv_bfloat16*>(st.vmean_bf16)[stat_off + tid] =
+            __float2bfloat16_rn(mean_sh[tid] * (1.0f / BLK));
+    }
+    __syncthreads();
+  }
+  // ---- queries: block means (query blocks have the same size as KV blocks)
+  if (Q != nullptr && st.qmean != nullptr) {
+#pragma unroll
+    for (int r = 0; r < ROWS; ++r)
+      load8<T>(Q + head_off + (row0 + r0 + r * RPP) * D + col * 8, x[r]);
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      float s = 0.f;
+#pragma unroll
+      for (int r = 0; r < ROWS; ++r) s += x[r][i];
+      acc[i] = s;
+    }
+    reduce_rows(acc);
+    if (tid < D) st.qmean[stat_off + tid] = mean_sh[tid] * (1.0f / BLK);
+  }
+}
+
+// htot[b,h] += Σ_{n in chunk} relu(k_n) v_nᵀ and ztot[b,h] += Σ relu(k_n) for
+// one chunk of tokens per CTA (the totals of the SLA2/SALAD linear branch).
+// Thread t owns row c = t / (256/D) of the d×d sum and D*D/256 of its columns.
+constexpr int kLinChunk = 1024;
+constexpr int kLinTile = 32;
+
+template <typename T, int D>
+__global__ void __launch_bounds__(256)
+linear_totals_kernel(const T* __restrict__ K, const T* __restrict__ V, int H, int N,
+                     float* __restrict__ htot, float* __restrict__ ztot) {
+  constexpr int TPR = 256 / D;       // threads per output row
+  constexpr int CPT = D / TPR;       // columns per thread
+  const int chunk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const size_t head_off = ((size_t)b * H + h) * (size_t)N * D;
+  const int tid = threadIdx.x;
+  const int c = tid / TPR, e0 = (tid % TPR) * CPT;
+  __shared__ float ks[kLinTile][D];
+  __shared__ float vs[kLinTile][D];
+  float acc[CPT];
+#pragma unroll
+  for (int i = 0; i < CPT; ++i) acc[i] = 0.f;
+  float z = 0.f;
+  const int n_begin = chunk * kLinChunk;
+  const int n_end = min(N, n_begin + kLinChunk);
+  for (int n0 = n_begin; n0 < n_end; n0 += kLinTile) {
+    __syncthreads();
+    for (int idx = tid; idx < kLinTile * D; idx += 256) {
+      const int r = idx / D, cc = idx % D;
+      const int n = n0 + r;
+      float kv = 0.f, vv = 0.f;
+      if (n < n_end) {
+        kv = to_f<T>(K[head_off + (size_t)n * D + cc]);
+        vv = to_f<T>(V[head_off + (size_t)n * D + cc]);
+      }
+      ks[r][cc] = fmaxf(kv, 0.f);
+      vs[r][cc] = vv;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int r = 0; r < kLinTile; ++r) {
+      const float kr = ks[r][c];
+      if (e0 == 0) z += kr;
+#pragma unroll
+      for (int i = 0; i < CPT; ++i) acc[i] = fmaf(kr, vs[r][e0 + i], acc[i]);
+    }
+  }
+  float* hp = htot + ((size_t)b * H + h) * D * D + (size_t)c * D + e0;
+#pragma unroll
+  for (int i = 0; i < CPT; ++i) atomicAdd(hp + i, acc[i]);
+  if (e0 == 0) atomicAdd(ztot + ((size_t)b * H + h) * D + c, z);
+}
+
+template <typename T, int D, int BLK>
+sa_status launch_pool(const void* Q, const void* K, const void* V, const sa_shape& s,
+                      const sa_block_stats& st, cudaStream_t stream) {
+  dim3 grid(s.N / BLK, s.H, s.B);
+  block_pool_kernel<T, D, BLK><<<grid, kPoolThreads, 0, stream>>>(
+      static_cast<const T*>(Q), static_cast<const T*>(K), static_cast<const T*>(V), s.H, s.N, st);
+  sa_status r = launch_status("block_pool_kernel");
+  if (r != SA_OK) return r;
+  if (st.htot || st.ztot) {
+    const size_t hbytes = (size_t)s.B * s.H * s.d * s.d * sizeof(float);
+    const size_t zbytes = (size_t)s.B * s.H * s.d * sizeof(float);
+    if (cudaMemsetAsync(st.htot, 0, hbytes, stream) != cudaSuccess ||
+        cudaMemsetAsync(st.ztot, 0, zbytes, stream) != cudaSuccess)
+      return launch_status("cudaMemsetAsync(htot/ztot)");
+    dim3 g2((s.N + kLinChunk - 1) / kLinChunk, s.H, s.B);
+    linear_totals_kernel<T, D><<<g2, 256, 0, stream>>>(
+        static_cast<const T*>(K), static_cast<const T*>(V), s.H, s.N, st.htot, st.ztot);
+    r = launch_status("linear_totals_kernel");
+  }
+  return r;
+}
+
+template <typename T>
+sa_status dispatch_pool(const void* Q, const void* K, const void* V, const sa_shape& s,
+                        const sa_block_stats& st, cudaStream_t stream) {
+  if (s.d == 128 && s.block == 128) return launch_pool<T, 128, 128>(Q, K, V, s, st, stream);
+  if (s.d == 128 && s.block == 64) return launch_pool<T, 128, 64>(Q, K, V, s, st, stream);
+  if (s.d == 64 && s.block == 128) return launch_pool<T, 64, 128>(Q, K, V, s, st, stream);
+  if (s.d == 64 && s.block == 64) return launch_pool<T, 64, 64>(Q, K, V, s, st, stream);
+  return fail(SA_ERR_UNSUPPORTED, "sa_block_pool: d and block must be 64 or 128");
+}
+
+}  // namespace
+}  // namespace sa
+
+extern "C" sa_status sa_block_pool(const void* Q, const void* K, const void* V, sa_dtype dtype,
+                                   sa_shape shape, const sa_block_stats* stats, void* stream) {
+  using namespace sa;
+  sa_status r = check_shape(shape, "sa_block_pool");
+  if (r != SA_OK) return r;
+  if (!K || !V || !stats || !stats->kmean || !stats->vsum)
+    return fail(SA_ERR_INVALID_ARG, "sa_block_pool: K, V, stats, stats->kmean and stats->vsum are required");
+  if ((stats->htot == nullptr) != (stats->ztot == nullptr))
+    return fail(SA_ERR_INVALID_ARG, "sa_block_pool: htot and ztot go together");
+  const void* ptrs[] = {Q, K, V, stats->qmean, stats->kmean, stats->vsum, stats->kvar,
+                        stats->zrelu, stats->htot, stats->ztot, stats->kmean_bf16, stats->vmean_bf16};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(SA_ERR_ALIGNMENT, "sa_block_pool: pointers must be 16-byte aligned");
+  if (shape.N == 0 || shape.B == 0 || shape.H == 0) return SA_OK;
+  cudaStream_t s = as_stream(stream);
+  if (dtype == SA_BF16) return dispatch_pool<__nv_bfloat16>(Q, K, V, shape, *stats, s);
+  if (dtype == SA_FP32) return dispatch_pool<float>(Q, K, V, shape, *stats, s);
+  return fail(SA_ERR_UNSUPPORTED, "sa_block_pool: dtype must be SA_FP32 or SA_BF16");
+}

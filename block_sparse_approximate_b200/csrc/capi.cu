@@ -1,0 +1,67 @@
+// C-ABI plumbing of libsparseattn: error reporting, shape checks and the
+// sparse prefill entry point (which picks the tensor-core or the CUDA-core
+// kernel for the request).
+#include <string>
+
+#include "attn_simt.cuh"
+
+namespace sa {
+
+namespace {
+thread_local std::string g_last_error;
+}
+
+void set_error(const std::string& msg) { g_last_error = msg; }
+
+sa_status check_shape(const sa_shape& s, const char* fn) {
+  if (s.B < 0 || s.H < 0 || s.N < 0 || s.d <= 0 || s.block <= 0)
+    return fail(SA_ERR_INVALID_ARG, std::string(fn) + ": negative or zero size");
+  if (s.d != 64 && s.d != 128) return fail(SA_ERR_UNSUPPORTED, std::string(fn) + ": d must be 64 or 128");
+  if (s.block != 64 && s.block != 128)
+    return fail(SA_ERR_UNSUPPORTED, std::string(fn) + ": block must be 64 or 128");
+  if (s.N % s.block) return fail(SA_ERR_INVALID_ARG, std::string(fn) + ": N must be a multiple of block");
+  return SA_OK;
+}
+
+}  // namespace sa
+
+extern "C" const char* sa_last_error(void) { return sa::g_last_error.c_str(); }
+
+extern "C" const char* sa_version(void) { return "libsparseattn 0.1 (sm_100a)"; }
+
+extern "C" sa_status sa_sparse_attn_fwd(const void* Q, const void* K, const void* V,
+                                        sa_dtype dtype, sa_shape shape,
+                                        const int32_t* block_idx, int32_t topk,
+                                        sa_tail_mode tail, const float* alpha,
+                                        const sa_block_stats* stats, float scale, void* O,
+                                        void* stream) {
+  using namespace sa;
+  sa_status r = check_shape(shape, "sa_sparse_attn_fwd");
+  if (r != SA_OK) return r;
+  const int nb = shape.N / shape.block;
+  if (dtype != SA_FP32 && dtype != SA_BF16)
+    return fail(SA_ERR_UNSUPPORTED, "sa_sparse_attn_fwd: dtype must be SA_FP32 or SA_BF16");
+  if (tail != SA_TAIL_DROP && tail != SA_TAIL_ZERO_ORDER && tail != SA_TAIL_LINEAR_MIX)
+    return fail(SA_ERR_INVALID_ARG, "sa_sparse_attn_fwd: unknown tail mode");
+  if (!Q || !K || !V || !O) return fail(SA_ERR_INVALID_ARG, "sa_sparse_attn_fwd: Q, K, V and O are required");
+  if (topk < 0 || topk > nb) return fail(SA_ERR_INVALID_ARG, "sa_sparse_attn_fwd: topk must be in [0, N/block]");
+  if (topk > 0 && !block_idx) return fail(SA_ERR_INVALID_ARG, "sa_sparse_attn_fwd: block_idx is required");
+  if (nb > kMaxAttnBlocks) return fail(SA_ERR_UNSUPPORTED, "sa_sparse_attn_fwd: at most 4096 blocks per head");
+  sa_block_stats st{};
+  if (stats) st = *stats;
+  if (tail == SA_TAIL_ZERO_ORDER && (!st.kmean || !st.vsum))
+    return fail(SA_ERR_INVALID_ARG, "sa_sparse_attn_fwd: SA_TAIL_ZERO_ORDER needs stats->kmean and stats->vsum");
+  if (tail == SA_TAIL_LINEAR_MIX && (!alpha || !st.zrelu || !st.htot || !st.ztot))
+    return fail(SA_ERR_INVALID_ARG,
+                "sa_sparse_attn_fwd: SA_TAIL_LINEAR_MIX needs alpha and stats->zrelu, htot, ztot");
+  const void* ptrs[] = {Q, K, V, O, block_idx, alpha, st.kmean, st.vsum, st.zrelu, st.htot, st.ztot,
+                        st.kmean_bf16, st.vmean_bf16};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(SA_ERR_ALIGNMENT, "sa_sparse_attn_fwd: pointers must be 16-byte aligned");
+  if (shape.B == 0 || shape.H == 0 || shape.N == 0) return SA_OK;
+  cudaStream_t s = as_stream(stream);
+  if (attn_tc_supports(dtype, shape, tail) &&
+      (tail != SA_TAIL_ZERO_ORDER || (st.kmean_bf16 && st.vmean_bf16)))
+    return attn_tc(Q, K, V, shape, block_idx, topk, tail, alpha, st, scale, O, s);
+  return attn_simt(Q, K, V, dtype, shape, block_idx, topk, tail, alpha, st, scale, O, s);
+}

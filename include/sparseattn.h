@@ -1,0 +1,176 @@
+/*
+ * libsparseattn — block-sparse attention with in-softmax block approximation,
+ * for NVIDIA B200 (sm_100a).
+ *
+ * The method (sources, by page title):
+ *   [PISA]  "PISA - Atenção Esparsa por Partes para Transformers de Difusão
+ *            Eficientes", §2 "Algoritmo Central" and "Implementação de Hardware"
+ *   [SLA2]  "SLA2: Sparse-Linear Attention with Learnable Routing and QAT",
+ *            §2A (mixture), §2B (router), §2C (low-precision sparse branch)
+ *   [SALAD] "SALAD: Achieve High-Sparsity Attention via Efficient Linear
+ *            Attention Tuning for Video Diffusion Transformer", §2 (ReLU
+ *            linear branch in parallel with the sparse one)
+ *   [SPLA]  "SPLA - Block Sparse Plus Linear Attention para Modelagem de
+ *            Contexto Longo", §2.1 (second-order block score), §2.2
+ *            (subtraction form of the residual linear term; decode is bound
+ *            by KV loading)
+ *
+ * Conventions for every entry point
+ *   - All tensor pointers are DEVICE pointers to memory the caller owns; the
+ *     library allocates nothing and frees nothing.  Dense activations are
+ *     row-major and contiguous: [B, H, N, d] means d is the fastest axis.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
+ *     NULL is the legacy default stream).  The return value reports host-side
+ *     argument validation and the launch; a fault inside a kernel surfaces at
+ *     the caller's next synchronisation as usual.
+ *   - On any status other than SA_OK nothing has been launched, except for
+ *     SA_ERR_CUDA (a launch failed; earlier launches of the same call may have
+ *     run).  sa_last_error() then returns a message for the calling thread.
+ *   - Supported: d in {64, 128}; block in {64, 128}; N a multiple of block;
+ *     0 <= topk <= N/block; pointers 16-byte aligned.
+ *   - Nothing is thrown across this interface.
+ */
+#ifndef SPARSEATTN_H
+#define SPARSEATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SA_OK = 0,
+  SA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, topk out of range */
+  SA_ERR_UNSUPPORTED = 2,   /* valid request this build does not implement */
+  SA_ERR_ALIGNMENT = 3,     /* a pointer is not 16-byte aligned */
+  SA_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
+  SA_ERR_WORKSPACE = 5      /* workspace missing or smaller than required */
+} sa_status;
+
+typedef enum { SA_FP32 = 0, SA_BF16 = 1 } sa_dtype;
+
+typedef enum {
+  SA_ROUTE_DOT = 0,      /* q̄_i · k̄_j on mean-pooled blocks [SLA2 §2B] */
+  SA_ROUTE_PROJ = 1,     /* (q̄_i P_q) · (k̄_j P_k), learnable router [SLA2 §2B] */
+  SA_ROUTE_TAYLOR2 = 2   /* s q̄·k̄_j + log1p(½ s² Σ_c q̄_c² var_jc), the log of
+                            exp(q·k̄)(1 + ½ qᵀ diag(Var k) q) [SPLA §2.1] */
+} sa_route_mode;
+
+typedef enum {
+  SA_TAIL_DROP = 0,        /* unselected blocks contribute nothing */
+  SA_TAIL_ZERO_ORDER = 1,  /* PISA zero-order block term inside numerator
+                              and denominator [PISA §2 "Algoritmo Central"] */
+  SA_TAIL_LINEAR_MIX = 2   /* O = α⊙O_s + (1−α)⊙O_l, O_l = ReLU linear
+                              attention over the unselected blocks
+                              [SLA2 §2A, SALAD §2, SPLA §2.2] */
+} sa_tail_mode;
+
+/* Shape of a prefill problem: Q, K, V, O are [B, H, N, d]; query blocks and
+ * KV blocks both hold `block` consecutive tokens (nb = N / block of each). */
+typedef struct {
+  int32_t B, H, N, d, block;
+} sa_shape;
+
+/* Shape of a GQA decode problem: q and o are [B, Hq, d] (one token per
+ * sequence), the caches are [B, Hkv, N, d]; query head h reads KV head
+ * h / (Hq / Hkv). */
+typedef struct {
+  int32_t B, Hq, Hkv, N, d, block;
+} sa_decode_shape;
+
+/* Block statistics, float32 device arrays owned by the caller.  A NULL field
+ * is not computed by sa_block_pool and must not be needed by a later call.
+ * nqb = nb = N / block.  [PISA "Implementação de Hardware", pre-computation;
+ * SLA2 §2B pooling; SPLA §2.1 block mean and diagonal covariance] */
+typedef struct {
+  float* qmean;     /* [B,H,nqb,d] mean of each query block                 */
+  float* kmean;     /* [B,H,nb,d]  mean of each key block (centroid k̄_j)    */
+  float* vsum;      /* [B,H,nb,d]  sum of each value block Σ_n v_{j,n}       */
+  float* kvar;      /* [B,H,nb,d]  per-channel population variance of keys */
+  float* zrelu;     /* [B,H,nb,d]  Σ_{n∈j} relu(k_n)                         */
+  float* htot;      /* [B,H,d,d]   Σ_n relu(k_n) v_nᵀ over all tokens        */
+  float* ztot;      /* [B,H,d]     Σ_n relu(k_n) over all tokens             */
+  uint16_t* kmean_bf16;  /* [B,H,nb,d] bf16 copy of kmean (tensor-core tail) */
+  uint16_t* vmean_bf16;  /* [B,H,nb,d] bf16 of vsum / block (tensor-core tail) */
+} sa_block_stats;
+
+/* Block statistics of Q (optional), K and V.
+ * Q: [B,H,N,d] or NULL (then stats->qmean is ignored); K, V: [B,H,N,d];
+ * dtype: element type of Q, K, V.  Every non-NULL field of *stats is written;
+ * kmean and vsum are required.  htot and ztot are sums over all tokens of a
+ * head and are overwritten (no accumulation across calls).
+ * Errors: SA_ERR_INVALID_ARG (null K/V/stats/kmean/vsum, bad shape),
+ *         SA_ERR_UNSUPPORTED (d or block not supported), SA_ERR_ALIGNMENT. */
+sa_status sa_block_pool(const void* Q, const void* K, const void* V, sa_dtype dtype,
+                        sa_shape shape, const sa_block_stats* stats, void* stream);
+
+/* Router: scores every (query block i, KV block j) pair and keeps the topk
+ * best KV blocks per query block [SLA2 §2B; PISA S_i; SPLA §2.1].
+ * stats: needs qmean and kmean (+ kvar for TAYLOR2).  proj_q, proj_k: [d,d]
+ * float32 row-major (x P means Σ_r x_r P[r][c]); required for PROJ, ignored
+ * otherwise.  scale: softmax scale s (used by TAYLOR2 only).
+ * block_idx: [B,H,nqb,topk] int32 output, ascending; a tie in score goes to
+ * the smaller block index.  scores: [B,H,nqb,nb] float32 output or NULL.
+ * Errors: SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED (nb > 4096), SA_ERR_ALIGNMENT. */
+sa_status sa_route(const sa_block_stats* stats, sa_shape shape, sa_route_mode mode,
+                   const float* proj_q, const float* proj_k, float scale, int32_t topk,
+                   int32_t* block_idx, float* scores, void* stream);
+
+/* Sparse prefill forward [PISA §2; SLA2 §2A]:
+ * for query row t of block i with selected set S_i = block_idx[b,h,i,:] and
+ * unselected set U_i,
+ *   DROP:        o_t = Σ_{n∈S} e^{s q·k_n} v_n / Σ_{n∈S} e^{s q·k_n}  (0 if S empty)
+ *   ZERO_ORDER:  o_t = (Σ_{n∈S} e^{s q·k_n} v_n + Σ_{j∈U} e^{s q·k̄_j} vsum_j)
+ *                    / (Σ_{n∈S} e^{s q·k_n}     + Σ_{j∈U} block·e^{s q·k̄_j})
+ *   LINEAR_MIX:  o_t = α_h ⊙ O_s + (1−α_h) ⊙ O_l,  O_s the DROP output,
+ *                O_l = relu(q)ᵀ(H_tot − Σ_{j∈S} h_j) / (relu(q)·(z_tot − Σ_{j∈S} z_j) + 1e-6),
+ *                h_j = Σ_{n∈j} relu(k_n) v_nᵀ (accumulated from the tiles the
+ *                kernel already loads, SPLA §2.2's subtraction form).
+ * Q, K, V, O: [B,H,N,d] of `dtype` (O has the same dtype).  block_idx:
+ * [B,H,nqb,topk] int32, each row ascending without repeats, entries in
+ * [0, nb).  alpha: [H,d] float32 (LINEAR_MIX only).  stats: ZERO_ORDER needs
+ * kmean, vsum (and kmean_bf16, vmean_bf16 for the bf16 tensor-core path);
+ * LINEAR_MIX needs zrelu, htot, ztot.
+ * Errors: SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED, SA_ERR_ALIGNMENT. */
+sa_status sa_sparse_attn_fwd(const void* Q, const void* K, const void* V, sa_dtype dtype,
+                             sa_shape shape, const int32_t* block_idx, int32_t topk,
+                             sa_tail_mode tail, const float* alpha,
+                             const sa_block_stats* stats, float scale, void* O,
+                             void* stream);
+
+/* Bytes of workspace sa_decode_fwd needs for this shape and topk (0 on bad
+ * arguments). */
+size_t sa_decode_workspace_size(sa_decode_shape shape, int32_t topk);
+
+/* GQA decode of one query token per sequence [SPLA §2.1, §2.2; PISA §2]:
+ * routes each (sequence, KV head) group with the TAYLOR2 score summed over the
+ * group's query heads (a logsumexp of the log scores), keeps topk blocks, and
+ * evaluates ZERO_ORDER (or DROP) attention for every query head of the group.
+ * Split over the KV axis; partial (max, sum, acc) states are merged.
+ * q: [B,Hq,d]; Kcache, Vcache: [B,Hkv,N,d], all of `dtype` (bf16 only).
+ * stats: kmean, kvar, vsum of the caches (sa_block_pool with Q = NULL).
+ * block_idx_out: [B,Hkv,topk] int32 or NULL; scores_out: [B,Hkv,nb] float32
+ * or NULL.  O: [B,Hq,d] of `dtype`.  workspace: device scratch of at least
+ * sa_decode_workspace_size() bytes, 256-byte aligned; its contents on entry
+ * do not matter.
+ * Errors: SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED, SA_ERR_ALIGNMENT,
+ *         SA_ERR_WORKSPACE. */
+sa_status sa_decode_fwd(const void* q, const void* Kcache, const void* Vcache, sa_dtype dtype,
+                        sa_decode_shape shape, const sa_block_stats* stats, int32_t topk,
+                        float scale, sa_tail_mode tail, int32_t* block_idx_out,
+                        float* scores_out, void* O, void* workspace, size_t workspace_bytes,
+                        void* stream);
+
+/* Message for the last non-SA_OK status returned on the calling thread. */
+const char* sa_last_error(void);
+
+/* Library version string. */
+const char* sa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPARSEATTN_H */

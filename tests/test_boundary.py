@@ -1,0 +1,103 @@
+"""The C-ABI library: it loads, exports every declared entry point, and its
+host-side argument validation returns the documented status codes (these
+checks run before any CUDA call, so no GPU is needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from block_sparse_approximate_b200 import binding as bd
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", fn)).read()
+            names |= set(re.findall(r"^\S.*?\b(sa_\w+)\s*\(", txt, flags=re.M))
+    return names
+
+
+def test_exports_every_declared_symbol(lib):
+    declared = _declared()
+    assert {"sa_block_pool", "sa_route", "sa_sparse_attn_fwd", "sa_decode_fwd"} <= declared
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert set(bd.EXPORTS) <= declared
+
+
+def test_version(lib):
+    assert "sm_100a" in bd.version()
+
+
+def _stats(**kw):
+    return bd.BlockStats(*[kw.get(n) for n in bd._STAT_FIELDS])
+
+
+FAKE = 0x10000  # never dereferenced: validation fails (or returns) before any launch
+
+
+def test_block_pool_validation(lib):
+    st = _stats(kmean=FAKE, vsum=FAKE)
+    assert lib.sa_block_pool(None, None, FAKE, 1, bd.Shape(1, 1, 256, 128, 128), ctypes.byref(st), None) \
+        == bd.SA_ERR_INVALID_ARG
+    assert lib.sa_block_pool(None, FAKE, FAKE, 1, bd.Shape(1, 1, 256, 96, 128), ctypes.byref(st), None) \
+        == bd.SA_ERR_UNSUPPORTED
+    assert lib.sa_block_pool(None, FAKE, FAKE, 1, bd.Shape(1, 1, 250, 128, 128), ctypes.byref(st), None) \
+        == bd.SA_ERR_INVALID_ARG
+    assert lib.sa_block_pool(None, FAKE + 4, FAKE, 1, bd.Shape(1, 1, 256, 128, 128), ctypes.byref(st), None) \
+        == bd.SA_ERR_ALIGNMENT
+    assert "16-byte" in lib.sa_last_error().decode()
+    # empty problem: nothing to launch
+    assert lib.sa_block_pool(None, FAKE, FAKE, 1, bd.Shape(1, 1, 0, 128, 128), ctypes.byref(st), None) == bd.SA_OK
+
+
+def test_route_validation(lib):
+    st = _stats(qmean=FAKE, kmean=FAKE)
+    sh = bd.Shape(1, 1, 1024, 128, 128)
+    assert lib.sa_route(ctypes.byref(st), sh, 0, None, None, 1.0, 9, FAKE, None, None) == bd.SA_ERR_INVALID_ARG
+    assert lib.sa_route(ctypes.byref(st), sh, 1, None, None, 1.0, 2, FAKE, None, None) == bd.SA_ERR_INVALID_ARG
+    assert lib.sa_route(ctypes.byref(st), sh, 2, None, None, 1.0, 2, FAKE, None, None) == bd.SA_ERR_INVALID_ARG
+    assert lib.sa_route(ctypes.byref(st), sh, 7, None, None, 1.0, 2, FAKE, None, None) == bd.SA_ERR_INVALID_ARG
+    big = bd.Shape(1, 1, 8192 * 64, 128, 64)
+    assert lib.sa_route(ctypes.byref(st), big, 0, None, None, 1.0, 2, FAKE, None, None) == bd.SA_ERR_UNSUPPORTED
+
+
+def test_sparse_attn_validation(lib):
+    sh = bd.Shape(1, 1, 1024, 128, 128)
+    none = _stats()
+    f = lib.sa_sparse_attn_fwd
+    assert f(FAKE, FAKE, FAKE, 1, sh, FAKE, 2, 1, None, ctypes.byref(none), 0.1, FAKE, None) \
+        == bd.SA_ERR_INVALID_ARG            # zero_order without kmean / vsum
+    assert f(FAKE, FAKE, FAKE, 1, sh, FAKE, 2, 2, None, ctypes.byref(none), 0.1, FAKE, None) \
+        == bd.SA_ERR_INVALID_ARG            # linear_mix without alpha and totals
+    assert f(FAKE, FAKE, FAKE, 1, sh, None, 2, 0, None, ctypes.byref(none), 0.1, FAKE, None) \
+        == bd.SA_ERR_INVALID_ARG            # topk > 0 without block_idx
+    assert f(FAKE, FAKE, FAKE, 1, sh, FAKE, 9, 0, None, ctypes.byref(none), 0.1, FAKE, None) \
+        == bd.SA_ERR_INVALID_ARG            # topk > nb
+    assert f(FAKE, FAKE, FAKE, 5, sh, FAKE, 2, 0, None, ctypes.byref(none), 0.1, FAKE, None) \
+        == bd.SA_ERR_UNSUPPORTED            # unknown dtype
+    assert f(FAKE, FAKE + 8, FAKE, 1, sh, FAKE, 2, 0, None, ctypes.byref(none), 0.1, FAKE, None) \
+        == bd.SA_ERR_ALIGNMENT
+
+
+def test_decode_validation_and_workspace(lib):
+    sh = bd.DecodeShape(16, 32, 8, 131072, 128, 64)
+    ws = lib.sa_decode_workspace_size(sh, 64)
+    assert ws > 16 * 32 * 128 * 4
+    assert lib.sa_decode_workspace_size(bd.DecodeShape(1, 6, 4, 1024, 128, 64), 4) == 0   # Hq % Hkv
+    st = _stats(kmean=FAKE, kvar=FAKE, vsum=FAKE)
+    f = lib.sa_decode_fwd
+    assert f(FAKE, FAKE, FAKE, 1, sh, ctypes.byref(st), 64, 0.1, 1, None, None, FAKE, FAKE, ws - 1, None) \
+        == bd.SA_ERR_WORKSPACE
+    assert f(FAKE, FAKE, FAKE, 0, sh, ctypes.byref(st), 64, 0.1, 1, None, None, FAKE, FAKE, ws, None) \
+        == bd.SA_ERR_UNSUPPORTED            # fp32 caches
+    assert f(FAKE, FAKE, FAKE, 1, sh, ctypes.byref(st), 64, 0.1, 2, None, None, FAKE, FAKE, ws, None) \
+        == bd.SA_ERR_UNSUPPORTED            # linear_mix decode
+    assert f(FAKE, FAKE, FAKE, 1, sh, ctypes.byref(st), 5000, 0.1, 1, None, None, FAKE, FAKE, ws, None) \
+        == bd.SA_ERR_INVALID_ARG
+    assert f(FAKE, FAKE, FAKE, 1, sh, ctypes.byref(st), 64, 0.1, 1, None, None, FAKE, FAKE + 16, ws, None) \
+        == bd.SA_ERR_ALIGNMENT              # workspace must be 256-byte aligned

@@ -1,0 +1,195 @@
+"""GPU parity: every step of the path through the C-ABI against the CPU oracle
+on the same seeded inputs (small sizes spanning several tiles and ragged
+tails, plus edge cases).  Full-size workloads are in test_parity_full_gpu.py."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from block_sparse_approximate_b200 import binding as bd
+from block_sparse_approximate_b200 import workloads as wl
+from tests._parity import (BF16_TOL, FP32_TOL, assert_stats_close, assert_tol, check_topk_exact,
+                           np64, selection_agreement)
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _gauss(B, H, N, d, dtype, seed):
+    g = torch.Generator(device=DEV)
+    g.manual_seed(seed)
+    return [torch.randn(B, H, N, d, generator=g, device=DEV).to(dtype).contiguous() for _ in range(3)]
+
+
+# --------------------------------------------------------------------------
+# block statistics
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dtype,d,block,N", [(torch.float32, 64, 64, 1024), (torch.bfloat16, 128, 128, 4736),
+                                             (torch.bfloat16, 128, 64, 2048), (torch.bfloat16, 64, 128, 1024)])
+def test_block_pool(lib, dtype, d, block, N):
+    Q, K, V = _gauss(2, 3, N, d, dtype, 1)
+    st = bd.block_pool(Q, K, V, block, variance=True, linear=True, centroids_bf16=True)
+    ref = oracle.block_pool(np64(Q), np64(K), np64(V), block, variance=True, linear=True)
+    for n in ("qmean", "kmean", "vsum", "kvar", "zrelu", "ztot"):
+        assert_stats_close(st[n], ref[n], n)
+    assert_stats_close(st["htot"], ref["htot"], "htot", rtol=1e-4)
+    assert_stats_close(st["kmean_bf16"].float(), ref["kmean"], "kmean_bf16", rtol=1e-2)
+    assert_stats_close(st["vmean_bf16"].float(), ref["vsum"] / block, "vmean_bf16", rtol=1e-2)
+
+
+def test_block_pool_large_offset_variance(lib):
+    # two-pass variance: a large common offset must not destroy the variance
+    Q, K, V = _gauss(1, 2, 2048, 128, torch.float32, 2)
+    K = (K + 1000.0).contiguous()
+    st = bd.block_pool(None, K, V, 128, variance=True)
+    ref = oracle.block_pool(None, np64(K), np64(V), 128, variance=True)
+    np.testing.assert_allclose(np64(st["kvar"]), ref["kvar"], rtol=2e-3, atol=2e-3)
+
+
+# --------------------------------------------------------------------------
+# router
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("mode", ["dot", "proj", "taylor2"])
+@pytest.mark.parametrize("nb,k", [(37, 5), (256, 26), (16, 0), (16, 16)])
+def test_route(lib, mode, nb, k):
+    d, block = 128, 128
+    w = wl.WORKLOADS["video_dit"]
+    if nb == 256:
+        inp = wl.prefill_inputs(w, DEV, H=2, N=nb * block)
+        Q, K, V = inp["Q"], inp["K"], inp["V"]
+    else:
+        Q, K, V = _gauss(1, 2, nb * block, d, torch.bfloat16, 3)
+    g = torch.Generator(device=DEV)
+    g.manual_seed(5)
+    Pq = (torch.randn(d, d, generator=g, device=DEV) / math.sqrt(d)).contiguous()
+    Pk = (torch.randn(d, d, generator=g, device=DEV) / math.sqrt(d)).contiguous()
+    st = bd.block_pool(Q, K, V, block, variance=True)
+    s = 1 / math.sqrt(d)
+    shape = (1, 2, nb * block, d, block)
+    idx, sc = bd.route(st, shape, mode, k, proj_q=Pq, proj_k=Pk, scale=s, want_scores=True)
+    ref = oracle.route_scores(np64(st["qmean"]), np64(st["kmean"]), mode, proj_q=np64(Pq),
+                              proj_k=np64(Pk), kvar=np64(st["kvar"]), scale=s)
+    assert_stats_close(sc, ref, f"{mode} scores", rtol=2e-5)
+    check_topk_exact(idx, sc, k)
+    frac = selection_agreement(np64(sc), ref, k)
+    assert frac >= 0.95
+
+
+def test_route_ties_pick_smaller_index(lib):
+    # identical key blocks: every score ties, the smallest indices win
+    d, block, nb = 128, 128, 12
+    Q, K, V = _gauss(1, 1, nb * block, d, torch.float32, 6)
+    K = K[:, :, :block].repeat(1, 1, nb, 1).contiguous()
+    st = bd.block_pool(Q, K, V, block)
+    idx, sc = bd.route(st, (1, 1, nb * block, d, block), "dot", 5, want_scores=True)
+    assert (idx.cpu().numpy() == np.arange(5)).all()
+
+
+# --------------------------------------------------------------------------
+# sparse prefill
+# --------------------------------------------------------------------------
+
+def _prefill_case(Q, K, V, block, k, tail, mode="dot", alpha=None, seed=0, tol=BF16_TOL):
+    B, H, N, d = Q.shape
+    s = 1 / math.sqrt(d)
+    st = bd.block_pool(Q, K, V, block, linear=(tail == "linear_mix"),
+                       centroids_bf16=(Q.dtype == torch.bfloat16))
+    idx, sc = bd.route(st, (B, H, N, d, block), mode, k, want_scores=True)
+    check_topk_exact(idx, sc, k)
+    O = bd.sparse_attn_fwd(Q, K, V, idx, block, tail, st, s, alpha=alpha)
+    torch.cuda.synchronize()
+    ref = oracle.sparse_attention(np64(Q), np64(K), np64(V), idx.cpu().numpy(), block, tail, s,
+                                  alpha=None if alpha is None else np64(alpha))
+    return assert_tol(np64(O), ref, tol, f"{tail} k={k}")
+
+
+@pytest.mark.parametrize("tail", ["zero_order", "drop", "linear_mix"])
+def test_tiny_fp32(lib, tail):
+    w = wl.WORKLOADS["tiny"]
+    inp = wl.prefill_inputs(w, DEV)
+    alpha = torch.rand(w.H, w.d, device=DEV) * 0.7 + 0.2 if tail == "linear_mix" else None
+    _prefill_case(inp["Q"], inp["K"], inp["V"], w.block, w.k, tail, alpha=alpha, tol=FP32_TOL)
+
+
+@pytest.mark.parametrize("tail", ["zero_order", "drop", "linear_mix"])
+@pytest.mark.parametrize("k", [0, 1, 4, 32])
+def test_video_small_bf16(lib, tail, k):
+    w = wl.WORKLOADS["video_dit"]
+    inp = wl.prefill_inputs(w, DEV, H=2, N=4096)        # 1x64x64 grid, 32 blocks
+    alpha = torch.rand(2, w.d, device=DEV) * 0.7 + 0.2 if tail == "linear_mix" else None
+    _prefill_case(inp["Q"], inp["K"], inp["V"], w.block, k, tail, alpha=alpha)
+
+
+@pytest.mark.parametrize("tail", ["zero_order", "drop", "linear_mix"])
+@pytest.mark.parametrize("dtype,d,block,nb,k", [
+    (torch.bfloat16, 128, 128, 37, 5),     # ragged centroid tiles
+    (torch.bfloat16, 128, 128, 133, 13),   # more than one 128-centroid tile, ragged
+    (torch.bfloat16, 128, 64, 40, 6),
+    (torch.bfloat16, 64, 128, 20, 3),
+    (torch.float32, 128, 128, 9, 2),
+    (torch.float32, 64, 64, 1, 1),         # a single block
+])
+def test_shapes(lib, tail, dtype, d, block, nb, k):
+    Q, K, V = _gauss(2, 2, nb * block, d, dtype, 7 + nb)
+    alpha = torch.rand(2, d, device=DEV) * 0.7 + 0.2 if tail == "linear_mix" else None
+    tol = FP32_TOL if dtype == torch.float32 else BF16_TOL
+    _prefill_case(Q, K, V, block, k, tail, alpha=alpha, tol=tol)
+
+
+def test_empty_problem_is_a_no_op(lib):
+    Q = torch.empty(1, 2, 0, 128, device=DEV, dtype=torch.bfloat16)
+    st = {"kmean": torch.empty(1, 2, 0, 128, device=DEV), "vsum": torch.empty(1, 2, 0, 128, device=DEV)}
+    idx = torch.empty(1, 2, 0, 0, device=DEV, dtype=torch.int32)
+    O = bd.sparse_attn_fwd(Q, Q, Q, idx, 128, "zero_order", st, 0.1)
+    assert O.shape == Q.shape
+
+
+def test_value_shift_on_gpu(lib):
+    # V + c shifts every output row by c (row normalisation, PISA §2)
+    Q, K, V = _gauss(1, 2, 4096, 128, torch.float32, 11)
+    c = torch.linspace(-1, 1, 128, device=DEV)
+    for tail in ("zero_order", "drop"):
+        st1 = bd.block_pool(Q, K, V, 128)
+        idx, _ = bd.route(st1, (1, 2, 4096, 128, 128), "dot", 4)
+        O1 = bd.sparse_attn_fwd(Q, K, V, idx, 128, tail, st1, 0.088)
+        V2 = (V + c).contiguous()
+        st2 = bd.block_pool(Q, K, V2, 128)
+        O2 = bd.sparse_attn_fwd(Q, K, V2, idx, 128, tail, st2, 0.088)
+        assert (O2 - O1 - c).abs().max().item() < 1e-4
+
+
+# --------------------------------------------------------------------------
+# decode
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("tail", ["zero_order", "drop"])
+@pytest.mark.parametrize("B,Hq,Hkv,N,d,block,k", [
+    (2, 8, 2, 8192, 128, 64, 16),
+    (1, 4, 4, 4096, 128, 128, 5),
+    (2, 8, 1, 2048, 64, 64, 0),
+    (1, 4, 2, 2048, 128, 64, 32),           # every block selected
+    (3, 6, 3, 64 * 77, 128, 64, 7),         # ragged split ranges
+])
+def test_decode(lib, tail, B, Hq, Hkv, N, d, block, k):
+    w = wl.WORKLOADS["decode"]
+    g = torch.Generator(device=DEV)
+    g.manual_seed(100 + N + k)
+    q = torch.randn(B, Hq, d, generator=g, device=DEV).to(torch.bfloat16)
+    Kc = (torch.randn(B, Hkv, N // block, block, d, generator=g, device=DEV)
+          + 0.7 * torch.randn(B, Hkv, N // block, 1, d, generator=g, device=DEV)).reshape(B, Hkv, N, d).to(torch.bfloat16)
+    Vc = torch.randn(B, Hkv, N, d, generator=g, device=DEV).to(torch.bfloat16)
+    st = bd.block_pool(None, Kc, Vc, block, variance=True)
+    s = 1 / math.sqrt(d)
+    o, idx, sc = bd.decode_fwd(q, Kc, Vc, st, block, k, s, tail=tail)
+    torch.cuda.synchronize()
+    check_topk_exact(idx, sc, k)
+    ref_sc = oracle.decode_route_scores(np64(q), np64(st["kmean"]), np64(st["kvar"]), s)
+    assert_stats_close(sc, ref_sc, "decode scores", rtol=2e-5)
+    ref_o, _, _ = oracle.decode_attention(np64(q), np64(Kc), np64(Vc), block, k, s, tail=tail,
+                                          block_idx=idx.cpu().numpy())
+    assert_tol(np64(o), ref_o, BF16_TOL, f"decode {tail}")
+    del w
