@@ -26,7 +26,7 @@ TAIL = {"drop": 0, "zero_order": 1, "linear_mix": 2}
 
 # every entry point declared in include/sparseattn.h
 EXPORTS = ("sa_block_pool", "sa_route", "sa_sparse_attn_fwd", "sa_decode_workspace_size",
-           "sa_decode_fwd", "sa_last_error", "sa_version")
+           "sa_decode_fwd", "sa_device_error", "sa_last_error", "sa_version")
 
 
 class SparseAttnError(RuntimeError):
@@ -74,6 +74,8 @@ def load():
                                   i32, f32, ctypes.c_int, vp, vp, vp, vp, sz, vp]
     for fn in ("sa_block_pool", "sa_route", "sa_sparse_attn_fwd", "sa_decode_fwd"):
         getattr(lib, fn).restype = ctypes.c_int
+    lib.sa_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
+    lib.sa_device_error.restype = ctypes.c_int
     lib.sa_last_error.restype = ctypes.c_char_p
     lib.sa_version.restype = ctypes.c_char_p
     _lib = lib
@@ -110,6 +112,13 @@ def _dtype_code(t: torch.Tensor) -> int:
 
 def _stats_struct(stats: dict) -> BlockStats:
     return BlockStats(*[_ptr(stats.get(n)) for n in _STAT_FIELDS])
+
+
+def device_error() -> int:
+    """Reads and clears the device-side error word (0 = no kernel gave up)."""
+    v = ctypes.c_uint32(0)
+    _check("sa_device_error", load().sa_device_error(ctypes.byref(v)))
+    return int(v.value)
 
 
 def version() -> str:

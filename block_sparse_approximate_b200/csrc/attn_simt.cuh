@@ -12,8 +12,8 @@ sa_status attn_simt(const void* Q, const void* K, const void* V, sa_dtype dtype,
                     const int32_t* block_idx, int topk, sa_tail_mode tail, const float* alpha,
                     const sa_block_stats& st, float scale, void* O, cudaStream_t stream);
 
-// Tensor-core path (tcgen05 + TMEM + TMA): bf16, block 128, d 128.  Returns
-// SA_ERR_UNSUPPORTED for anything else.
+// Tensor-core path (tcgen05 + TMEM + TMA): bf16, block 128, d 128, tails
+// drop and zero-order (attn_tc_supports says which requests it takes).
 sa_status attn_tc(const void* Q, const void* K, const void* V, const sa_shape& s,
                   const int32_t* block_idx, int topk, sa_tail_mode tail, const float* alpha,
                   const sa_block_stats& st, float scale, void* O, cudaStream_t stream);

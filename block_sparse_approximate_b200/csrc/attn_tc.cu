@@ -1,13 +1,407 @@
-// Tensor-core sparse prefill (tcgen05 + TMEM + TMA), bf16, block 128.
+// Sparse prefill on the 5th-generation tensor cores (tcgen05 + TMEM + TMA),
+// bf16 Q/K/V, 128-token blocks, d = 128, tails drop and zero-order.
+//
+// PISA's fused kernel ("Implementação de Hardware") interleaves the exact
+// scan over the selected blocks and the approximate scan over the block
+// aggregates inside one online softmax.  Here both scans are the same tile
+// loop: a CTA owns one 128-row query block and walks a list of 128-key tiles,
+//   tiles 0..k-1      the selected KV blocks (exact, PISA "Fase 1"),
+//   tiles k..k+c-1    the block centroids k̄_j with values vsum_j / B in
+//                     groups of 128 blocks (PISA "Fase 2"): logit bias log2 B
+//                     and the selected blocks masked out, which adds
+//                     e^{s q·k̄_j}·vsum_j to the numerator and B·e^{s q·k̄_j}
+//                     to the denominator,
+// so the tail costs 1/B of the dense work and no N×N matrix exists.
+//
+// Warp roles (192 threads, one CTA per SM):
+//   warps 0-3  softmax: thread r owns query row r (TMEM lane r); reads S from
+//              TMEM, keeps (max, sum) in registers, writes P back into TMEM as
+//              bf16 over the S columns, rescales O in TMEM when the running
+//              max grows by more than 2^8, and writes the output;
+//   warp 4     TMA producer: Q once, then K/V tiles into a 3-stage ring;
+//   warp 5     MMA issuer: S = Q·Kᵀ (both operands K-major in shared memory)
+//              into a double-buffered S in TMEM, then O += P·V with P read
+//              from TMEM and V as an MN-major shared-memory operand.
+// TMEM: S0 cols [0,128), S1 [128,256), O [256,384) of a 512-column allocation.
+#include <mutex>
+
 #include "attn_simt.cuh"
+#include "tc_util.cuh"
 
 namespace sa {
+namespace {
 
-bool attn_tc_supports(sa_dtype, const sa_shape&, sa_tail_mode) { return false; }
+using namespace tc;
 
-sa_status attn_tc(const void*, const void*, const void*, const sa_shape&, const int32_t*, int,
-                  sa_tail_mode, const float*, const sa_block_stats&, float, void*, cudaStream_t) {
-  return fail(SA_ERR_UNSUPPORTED, "sa_sparse_attn_fwd: tensor-core path not built");
+constexpr int TB = 128;                        // rows per tile (queries and keys)
+constexpr int TD = 128;                        // head dim
+constexpr int NS = 3;                          // K/V pipeline stages
+constexpr int kTcThreads = 192;
+constexpr int kTmaWarp = 4, kMmaWarp = 5;
+constexpr uint32_t kHalfTile = TB * 64 * 2;    // 128 rows x 64 bf16 (one 128-byte swizzle span)
+constexpr uint32_t kTile = 2 * kHalfTile;      // 128 x 128 bf16
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColO = 256;
+constexpr float kLazyRescale = 8.0f;           // log2 units
+
+// barrier slots
+constexpr int B_Q = 0;
+constexpr int B_KF = 1;                 // NS
+constexpr int B_VF = B_KF + NS;         // NS
+constexpr int B_KE = B_VF + NS;         // NS
+constexpr int B_SF = B_KE + NS;         // 2
+constexpr int B_PR = B_SF + 2;          // 2
+constexpr int B_OD = B_PR + 2;          // 1
+constexpr int B_FIN = B_OD + 1;         // 1
+constexpr int NBAR = B_FIN + 1;
+
+constexpr uint32_t kBarOff = kTile * (1 + 2 * NS);
+constexpr uint32_t kSlotOff = kBarOff + 8 * NBAR;     // tmem base, abort flag
+constexpr uint32_t kMaskOff = kSlotOff + 16;
+
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity) {
+  // used only on the abort path, where no other role can release us
+  const long long t0 = clock64();
+  for (;;) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    if (done) return true;
+    if (clock64() - t0 > kWaitCycles / 8) return false;
+  }
+}
+
+template <bool ZO>
+__global__ void __launch_bounds__(kTcThreads, 1)
+attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKb,
+               const __grid_constant__ CUtensorMap tmVb, const int32_t* __restrict__ block_idx, int nb,
+               int topk, float scale2, __nv_bfloat16* __restrict__ O, int N) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(smem);
+  const int i = blockIdx.x, bh = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kSlotOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kSlotOff + 4);
+  uint32_t* selmask = reinterpret_cast<uint32_t*>(smem + kMaskOff);
+  auto bar = [&](int k) { return sb + kBarOff + 8u * k; };
+
+  const int nwords = (nb + 31) >> 5;
+  const int ntail = (ZO && topk < nb) ? (nb + TB - 1) / TB : 0;
+  const int T = topk + ntail;
+  const int32_t* sel = block_idx + ((size_t)bh * nb + i) * topk;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(B_Q), 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(bar(B_KF + s), 1);
+      mbar_init(bar(B_VF + s), 1);
+      mbar_init(bar(B_KE + s), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(B_SF + s), 1);
+      mbar_init(bar(B_PR + s), 128);
+    }
+    mbar_init(bar(B_OD), 1);
+    mbar_init(bar(B_FIN), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  for (int w = threadIdx.x; w < nwords; w += kTcThreads) selmask[w] = 0u;
+  if (warp == 0) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+  __syncthreads();
+  for (int s = threadIdx.x; s < topk; s += kTcThreads) {
+    const int j = sel[s];
+    atomicOr(&selmask[j >> 5], 1u << (j & 31));
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+
+  if (warp == kTmaWarp) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && T > 0) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      if (ZO) {
+        prefetch_tmap(&tmKb);
+        prefetch_tmap(&tmVb);
+      }
+      mbar_expect_tx(bar(B_Q), kTile);
+      tma_load_3d(sb, &tmQ, 0, i * TB, bh, bar(B_Q));
+      tma_load_3d(sb + kHalfTile, &tmQ, 64, i * TB, bh, bar(B_Q));
+      int issued = 0;
+      for (int t = 0; t < T; ++t) {
+        const int s = t % NS;
+        if (t >= NS && !mbar_wait(bar(B_KE + s), ((t / NS) - 1) & 1, abort_flag)) break;
+        const bool exact = t < topk;
+        const CUtensorMap* mk = exact ? &tmK : &tmKb;
+        const CUtensorMap* mv = exact ? &tmV : &tmVb;
+        const int row = exact ? sel[t] * TB : (t - topk) * TB;
+        const uint32_t ka = sb + kTile * (1 + 2 * s), va = ka + kTile;
+        mbar_expect_tx(bar(B_KF + s), kTile);
+        tma_load_3d(ka, mk, 0, row, bh, bar(B_KF + s));
+        tma_load_3d(ka + kHalfTile, mk, 64, row, bh, bar(B_KF + s));
+        mbar_expect_tx(bar(B_VF + s), kTile);
+        tma_load_3d(va, mv, 0, row, bh, bar(B_VF + s));
+        tma_load_3d(va + kHalfTile, mv, 64, row, bh, bar(B_VF + s));
+        issued = t + 1;
+      }
+      if (*abort_flag) {
+        // let the loads already in flight land before the CTA goes away
+        wait_bounded(bar(B_Q), 0);
+        for (int t = issued > NS ? issued - NS : 0; t < issued; ++t) {
+          wait_bounded(bar(B_KF + t % NS), (t / NS) & 1);
+          wait_bounded(bar(B_VF + t % NS), (t / NS) & 1);
+        }
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && T > 0) {
+      constexpr uint32_t idS = idesc_bf16_f32(TB, TB, 0, 0);
+      constexpr uint32_t idO = idesc_bf16_f32(TB, TD, 0, 1);
+      bool ok = mbar_wait(bar(B_Q), 0, abort_flag);
+      for (int t = 0; ok && t <= T; ++t) {
+        if (t < T) {
+          const int s = t % NS;
+          if (!mbar_wait(bar(B_KF + s), (t / NS) & 1, abort_flag)) break;
+          tc_fence_after();
+          const uint32_t ka = sb + kTile * (1 + 2 * s);
+          const uint32_t d = tbase + (uint32_t)(t & 1) * TB;
+#pragma unroll
+          for (int k = 0; k < TD / 16; ++k) {
+            const uint32_t koff = (k >> 2) * kHalfTile + (k & 3) * 32;
+            mma_ss(d, desc_sw128(sb + koff, 16, 1024), desc_sw128(ka + koff, 16, 1024), idS, k > 0);
+          }
+          mma_commit(bar(B_SF + (t & 1)));
+        }
+        if (t >= 1) {
+          const int u = t - 1, su = u % NS;
+          if (!mbar_wait(bar(B_PR + (u & 1)), (u >> 1) & 1, abort_flag)) break;
+          if (!mbar_wait(bar(B_VF + su), (u / NS) & 1, abort_flag)) break;
+          tc_fence_after();
+          const uint32_t va = sb + kTile * (2 + 2 * su);
+          const uint32_t pa = tbase + (uint32_t)(u & 1) * TB;
+#pragma unroll
+          for (int k = 0; k < TB / 16; ++k)
+            mma_ts(tbase + kColO, pa + k * 8, desc_sw128(va + k * 16 * 128, kHalfTile, 1024), idO,
+                   (u > 0 || k > 0));
+          mma_commit(bar(B_KE + su));
+          mma_commit(bar(B_OD));
+        }
+      }
+      // every MMA issued above has completed before TMEM is released
+      mma_commit(bar(B_FIN));
+      wait_bounded(bar(B_FIN), 0);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int r = warp * 32 + lane;
+    const uint32_t lrow = tbase + ((uint32_t)(warp * 32) << 16);
+    float m_used = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int t = 0; t < T; ++t) {
+      const int sbuf = t & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_SF + sbuf), (t >> 1) & 1, abort_flag))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t v[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        tmem_ld32(lrow + sbuf * TB + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * c]));
+      tmem_wait_ld();
+      float mx = -INFINITY;
+      if (t < topk) {
+#pragma unroll
+        for (int n = 0; n < TB; ++n) {
+          const float x = __uint_as_float(v[n]) * scale2;
+          v[n] = __float_as_uint(x);
+          mx = fmaxf(mx, x);
+        }
+      } else {
+        const int jb = (t - topk) * TB;
+#pragma unroll
+        for (int n = 0; n < TB; ++n) {
+          const int j = jb + n;
+          const bool valid = j < nb && !((selmask[j >> 5] >> (j & 31)) & 1u);
+          const float x = valid ? fmaf(__uint_as_float(v[n]), scale2, 7.0f) : -INFINITY;  // + log2(128)
+          v[n] = __float_as_uint(x);
+          mx = fmaxf(mx, x);
+        }
+      }
+      const float m_new = fmaxf(m_used, mx);
+      const bool need = m_new > m_used + kLazyRescale;
+      float factor = 1.f;
+      if (need) {
+        factor = fast_exp2(m_used - m_new);
+        m_used = m_new;
+      }
+      const bool live = m_used != -INFINITY;
+      float sum = 0.f;
+      uint32_t pk[64];
+#pragma unroll
+      for (int n = 0; n < 64; ++n) {
+        const float p0 = live ? fast_exp2(__uint_as_float(v[2 * n]) - m_used) : 0.f;
+        const float p1 = live ? fast_exp2(__uint_as_float(v[2 * n + 1]) - m_used) : 0.f;
+        sum += p0 + p1;
+        pk[n] = pack_bf16(p0, p1);
+      }
+      l = l * factor + sum;
+      tmem_st32(lrow + sbuf * TB, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+      tmem_st32(lrow + sbuf * TB + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+      tmem_wait_st();
+      if (t >= 1) {
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(B_OD), (t - 1) & 1, abort_flag))) {
+          ok = false;
+          break;
+        }
+        if (__any_sync(0xffffffffu, need)) {
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t o[32];
+            tmem_ld32(lrow + kColO + 32 * c, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
+            tmem_st32(lrow + kColO + 32 * c, o);
+          }
+          tmem_wait_st();
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(B_PR + sbuf));
+    }
+    if (ok && T > 0) {
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_OD), (T - 1) & 1, abort_flag));
+      tc_fence_after();
+    }
+    if (ok) {
+      const float inv = l > 0.f ? 1.0f / l : 0.f;
+      uint4* orow = reinterpret_cast<uint4*>(O + ((size_t)bh * N + (size_t)i * TB + r) * TD);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t o[32];
+        if (T > 0) {
+          tmem_ld32(lrow + kColO + 32 * c, o);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = 0u;
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint4 w;
+          w.x = pack_bf16(__uint_as_float(o[8 * q + 0]) * inv, __uint_as_float(o[8 * q + 1]) * inv);
+          w.y = pack_bf16(__uint_as_float(o[8 * q + 2]) * inv, __uint_as_float(o[8 * q + 3]) * inv);
+          w.z = pack_bf16(__uint_as_float(o[8 * q + 4]) * inv, __uint_as_float(o[8 * q + 5]) * inv);
+          w.w = pack_bf16(__uint_as_float(o[8 * q + 6]) * inv, __uint_as_float(o[8 * q + 7]) * inv);
+          orow[4 * c + q] = w;
+        }
+      }
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tbase, kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+size_t tc_smem_bytes(int nb) {
+  return 1024 + kMaskOff + 4 * (size_t)((nb + 31) / 32) + 16;
+}
+
+}  // namespace
+
+bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows, uint64_t outer,
+                       uint32_t box_cols, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {cols, rows, outer};
+  cuuint64_t strides[2] = {cols * 2, cols * rows * 2};
+  cuuint32_t box[3] = {box_cols, box_rows, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool attn_tc_supports(sa_dtype dtype, const sa_shape& s, sa_tail_mode tail) {
+  return dtype == SA_BF16 && s.block == TB && s.d == TD &&
+         (tail == SA_TAIL_DROP || tail == SA_TAIL_ZERO_ORDER);
+}
+
+sa_status attn_tc(const void* Q, const void* K, const void* V, const sa_shape& s, const int32_t* block_idx,
+                  int topk, sa_tail_mode tail, const float* alpha, const sa_block_stats& st, float scale,
+                  void* O, cudaStream_t stream) {
+  (void)alpha;
+  const int nb = s.N / TB;
+  const uint64_t BH = (uint64_t)s.B * s.H;
+  CUtensorMap mq, mk, mv, mkb, mvb;
+  if (!make_tmap_bf16_3d(&mq, Q, TD, s.N, BH, 64, TB) || !make_tmap_bf16_3d(&mk, K, TD, s.N, BH, 64, TB) ||
+      !make_tmap_bf16_3d(&mv, V, TD, s.N, BH, 64, TB))
+    return fail(SA_ERR_CUDA, "sa_sparse_attn_fwd: cuTensorMapEncodeTiled failed for Q/K/V");
+  const bool zo = tail == SA_TAIL_ZERO_ORDER;
+  if (zo) {
+    if (!make_tmap_bf16_3d(&mkb, st.kmean_bf16, TD, nb, BH, 64, TB) ||
+        !make_tmap_bf16_3d(&mvb, st.vmean_bf16, TD, nb, BH, 64, TB))
+      return fail(SA_ERR_CUDA, "sa_sparse_attn_fwd: cuTensorMapEncodeTiled failed for the block centroids");
+  } else {
+    mkb = mk;
+    mvb = mv;
+  }
+  const size_t smem = tc_smem_bytes(nb);
+  auto kern = zo ? attn_tc_kernel<true> : attn_tc_kernel<false>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return launch_status("cudaFuncSetAttribute(attn_tc_kernel)");
+  dim3 grid(nb, (unsigned)BH);
+  kern<<<grid, kTcThreads, smem, stream>>>(mq, mk, mv, mkb, mvb, block_idx, nb, topk, scale * kLog2e,
+                                           static_cast<__nv_bfloat16*>(O), s.N);
+  return launch_status("attn_tc_kernel");
 }
 
 }  // namespace sa
+
+extern "C" sa_status sa_device_error(uint32_t* code) {
+  using namespace sa;
+  if (!code) return fail(SA_ERR_INVALID_ARG, "sa_device_error: code is required");
+  unsigned int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, tc::g_device_error, sizeof(v)) != cudaSuccess ||
+      cudaMemcpyToSymbol(tc::g_device_error, &zero, sizeof(zero)) != cudaSuccess)
+    return launch_status("sa_device_error");
+  *code = v;
+  return SA_OK;
+}

@@ -101,7 +101,7 @@ extern "C" sa_status sa_route(const sa_block_stats* stats, sa_shape shape, sa_ro
   sa_status r = check_shape(shape, "sa_route");
   if (r != SA_OK) return r;
   const int nb = shape.N / shape.block;
-  if (!stats || !stats->qmean || !stats->kmean || !block_idx)
+  if (!stats || !stats->qmean || !stats->kmean || (topk > 0 && !block_idx))
     return fail(SA_ERR_INVALID_ARG, "sa_route: stats->qmean, stats->kmean and block_idx are required");
   if (mode != SA_ROUTE_DOT && mode != SA_ROUTE_PROJ && mode != SA_ROUTE_TAYLOR2)
     return fail(SA_ERR_INVALID_ARG, "sa_route: unknown route mode");

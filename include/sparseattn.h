@@ -112,7 +112,7 @@ sa_status sa_block_pool(const void* Q, const void* K, const void* V, sa_dtype dt
  * float32 row-major (x P means Σ_r x_r P[r][c]); required for PROJ, ignored
  * otherwise.  scale: softmax scale s (used by TAYLOR2 only).
  * block_idx: [B,H,nqb,topk] int32 output, ascending; a tie in score goes to
- * the smaller block index.  scores: [B,H,nqb,nb] float32 output or NULL.
+ * the smaller block index (may be NULL when topk == 0).  scores: [B,H,nqb,nb] float32 output or NULL.
  * Errors: SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED (nb > 4096), SA_ERR_ALIGNMENT. */
 sa_status sa_route(const sa_block_stats* stats, sa_shape shape, sa_route_mode mode,
                    const float* proj_q, const float* proj_k, float scale, int32_t topk,
@@ -162,6 +162,13 @@ sa_status sa_decode_fwd(const void* q, const void* Kcache, const void* Vcache, s
                         float scale, sa_tail_mode tail, int32_t* block_idx_out,
                         float* scores_out, void* O, void* workspace, size_t workspace_bytes,
                         void* stream);
+
+/* Reads and clears the library's device-side error word (synchronous: waits
+ * for work already queued on the legacy default stream).  Non-zero means a
+ * kernel gave up on an internal wait (bit 0: a bounded barrier wait timed
+ * out, about two seconds) and returned without writing its output; the CUDA
+ * context stays usable.  Kernels never trap on their own errors. */
+sa_status sa_device_error(uint32_t* code);
 
 /* Message for the last non-SA_OK status returned on the calling thread. */
 const char* sa_last_error(void);

@@ -17,6 +17,10 @@ def np64(t: torch.Tensor) -> np.ndarray:
     return t.detach().to("cpu", torch.float64).numpy()
 
 
+def assert_no_device_error():
+    assert bd.device_error() == 0, "a kernel gave up on a bounded wait"
+
+
 def assert_tol(got, ref, tol, what=""):
     got = np.asarray(got, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)

@@ -11,7 +11,8 @@ import oracle
 from block_sparse_approximate_b200 import binding as bd
 from block_sparse_approximate_b200 import workloads as wl
 from block_sparse_approximate_b200.pipeline import DecodeStep, PrefillStep
-from tests._parity import BF16_TOL, assert_tol, check_topk_exact, np64, selection_agreement
+from tests._parity import (BF16_TOL, assert_no_device_error, assert_tol, check_topk_exact, np64,
+                           selection_agreement)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -32,6 +33,7 @@ def test_prefill_full_size_sampled(lib, name):
     step = PrefillStep(w, inp, want_scores=True)
     O = step()
     torch.cuda.synchronize()
+    assert_no_device_error()
     buf = step.buf
     check_topk_exact(buf.block_idx, buf.scores, w.k)
     ref_sc = oracle.route_scores(np64(buf.stats["qmean"]), np64(buf.stats["kmean"]), w.route,

@@ -10,8 +10,8 @@ import torch
 import oracle
 from block_sparse_approximate_b200 import binding as bd
 from block_sparse_approximate_b200 import workloads as wl
-from tests._parity import (BF16_TOL, FP32_TOL, assert_stats_close, assert_tol, check_topk_exact,
-                           np64, selection_agreement)
+from tests._parity import (BF16_TOL, FP32_TOL, assert_no_device_error, assert_stats_close, assert_tol,
+                           check_topk_exact, np64, selection_agreement)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -102,6 +102,7 @@ def _prefill_case(Q, K, V, block, k, tail, mode="dot", alpha=None, seed=0, tol=B
     check_topk_exact(idx, sc, k)
     O = bd.sparse_attn_fwd(Q, K, V, idx, block, tail, st, s, alpha=alpha)
     torch.cuda.synchronize()
+    assert_no_device_error()
     ref = oracle.sparse_attention(np64(Q), np64(K), np64(V), idx.cpu().numpy(), block, tail, s,
                                   alpha=None if alpha is None else np64(alpha))
     return assert_tol(np64(O), ref, tol, f"{tail} k={k}")
