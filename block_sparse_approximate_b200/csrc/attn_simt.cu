@@ -190,7 +190,18 @@ attn_simt_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __re
       for (int c = 0; c < PER; ++c) orow[lane * PER + c] = from_f<T>(acc[r * D + lane * PER + c] * inv_l);
       continue;
     }
-    // linear branch over the unselected blocks, then the SLA2 mixture
+    // linear branch over the unselected blocks, then the SLA2 mixture; with
+    // every block selected the unselected set is empty and O_l is 0 (the
+    // subtraction H_tot - A_i would only leave rounding noise)
+    const float* al = alpha + (size_t)h * D;
+    if (topk == nb) {
+#pragma unroll
+      for (int e = 0; e < PER; ++e) {
+        const int ee = lane * PER + e;
+        orow[ee] = from_f<T>(al[ee] * acc[r * D + ee] * inv_l);
+      }
+      continue;
+    }
     const float* qr = qs + r * D;
     const float* zt = st.ztot + bh * D;
     float dp = 0.f;
@@ -212,7 +223,6 @@ attn_simt_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __re
         num[e] = fmaf(fq, Ht[(size_t)c * D + ee] - A[c * D + ee], num[e]);
       }
     }
-    const float* al = alpha + (size_t)h * D;
 #pragma unroll
     for (int e = 0; e < PER; ++e) {
       const int ee = lane * PER + e;

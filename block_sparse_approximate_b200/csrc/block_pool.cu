@@ -233,6 +233,7 @@ extern "C" sa_status sa_block_pool(const void* Q, const void* K, const void* V, 
   using namespace sa;
   sa_status r = check_shape(shape, "sa_block_pool");
   if (r != SA_OK) return r;
+  if (shape.N == 0 || shape.B == 0 || shape.H == 0) return SA_OK;  // nothing to compute
   if (!K || !V || !stats || !stats->kmean || !stats->vsum)
     return fail(SA_ERR_INVALID_ARG, "sa_block_pool: K, V, stats, stats->kmean and stats->vsum are required");
   if ((stats->htot == nullptr) != (stats->ztot == nullptr))
@@ -241,7 +242,6 @@ extern "C" sa_status sa_block_pool(const void* Q, const void* K, const void* V, 
                         stats->zrelu, stats->htot, stats->ztot, stats->kmean_bf16, stats->vmean_bf16};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return fail(SA_ERR_ALIGNMENT, "sa_block_pool: pointers must be 16-byte aligned");
-  if (shape.N == 0 || shape.B == 0 || shape.H == 0) return SA_OK;
   cudaStream_t s = as_stream(stream);
   if (dtype == SA_BF16) return dispatch_pool<__nv_bfloat16>(Q, K, V, shape, *stats, s);
   if (dtype == SA_FP32) return dispatch_pool<float>(Q, K, V, shape, *stats, s);

@@ -43,6 +43,7 @@ extern "C" sa_status sa_sparse_attn_fwd(const void* Q, const void* K, const void
     return fail(SA_ERR_UNSUPPORTED, "sa_sparse_attn_fwd: dtype must be SA_FP32 or SA_BF16");
   if (tail != SA_TAIL_DROP && tail != SA_TAIL_ZERO_ORDER && tail != SA_TAIL_LINEAR_MIX)
     return fail(SA_ERR_INVALID_ARG, "sa_sparse_attn_fwd: unknown tail mode");
+  if (shape.B == 0 || shape.H == 0 || shape.N == 0) return SA_OK;  // nothing to compute
   if (!Q || !K || !V || !O) return fail(SA_ERR_INVALID_ARG, "sa_sparse_attn_fwd: Q, K, V and O are required");
   if (topk < 0 || topk > nb) return fail(SA_ERR_INVALID_ARG, "sa_sparse_attn_fwd: topk must be in [0, N/block]");
   if (topk > 0 && !block_idx) return fail(SA_ERR_INVALID_ARG, "sa_sparse_attn_fwd: block_idx is required");
@@ -58,7 +59,6 @@ extern "C" sa_status sa_sparse_attn_fwd(const void* Q, const void* K, const void
                         st.kmean_bf16, st.vmean_bf16};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return fail(SA_ERR_ALIGNMENT, "sa_sparse_attn_fwd: pointers must be 16-byte aligned");
-  if (shape.B == 0 || shape.H == 0 || shape.N == 0) return SA_OK;
   cudaStream_t s = as_stream(stream);
   if (attn_tc_supports(dtype, shape, tail) &&
       (tail != SA_TAIL_ZERO_ORDER || (st.kmean_bf16 && st.vmean_bf16)))

@@ -101,6 +101,7 @@ extern "C" sa_status sa_route(const sa_block_stats* stats, sa_shape shape, sa_ro
   sa_status r = check_shape(shape, "sa_route");
   if (r != SA_OK) return r;
   const int nb = shape.N / shape.block;
+  if (shape.N == 0 || shape.B == 0 || shape.H == 0) return SA_OK;  // nothing to compute
   if (!stats || !stats->qmean || !stats->kmean || (topk > 0 && !block_idx))
     return fail(SA_ERR_INVALID_ARG, "sa_route: stats->qmean, stats->kmean and block_idx are required");
   if (mode != SA_ROUTE_DOT && mode != SA_ROUTE_PROJ && mode != SA_ROUTE_TAYLOR2)
@@ -114,7 +115,6 @@ extern "C" sa_status sa_route(const sa_block_stats* stats, sa_shape shape, sa_ro
   const void* ptrs[] = {stats->qmean, stats->kmean, stats->kvar, proj_q, proj_k, block_idx, scores};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return fail(SA_ERR_ALIGNMENT, "sa_route: pointers must be 16-byte aligned");
-  if (shape.N == 0 || shape.B == 0 || shape.H == 0) return SA_OK;
   const size_t smem = route_smem_bytes(nb, shape.d);
   dim3 grid(nb, shape.H, shape.B);
   cudaStream_t s = as_stream(stream);

@@ -127,7 +127,8 @@ sa_status sa_route(const sa_block_stats* stats, sa_shape shape, sa_route_mode mo
  *   LINEAR_MIX:  o_t = α_h ⊙ O_s + (1−α_h) ⊙ O_l,  O_s the DROP output,
  *                O_l = relu(q)ᵀ(H_tot − Σ_{j∈S} h_j) / (relu(q)·(z_tot − Σ_{j∈S} z_j) + 1e-6),
  *                h_j = Σ_{n∈j} relu(k_n) v_nᵀ (accumulated from the tiles the
- *                kernel already loads, SPLA §2.2's subtraction form).
+ *                kernel already loads, SPLA §2.2's subtraction form);
+ *                O_l = 0 when every block is selected (U_i empty).
  * Q, K, V, O: [B,H,N,d] of `dtype` (O has the same dtype).  block_idx:
  * [B,H,nqb,topk] int32, each row ascending without repeats, entries in
  * [0, nb).  alpha: [H,d] float32 (LINEAR_MIX only).  stats: ZERO_ORDER needs
