@@ -26,7 +26,7 @@ TAIL = {"drop": 0, "zero_order": 1, "linear_mix": 2}
 
 # every entry point declared in include/sparseattn.h
 EXPORTS = ("sa_block_pool", "sa_route", "sa_sparse_attn_fwd", "sa_decode_workspace_size",
-           "sa_decode_fwd", "sa_device_error", "sa_last_error", "sa_version")
+           "sa_decode_fwd", "sa_decode_fwd_static", "sa_device_error", "sa_last_error", "sa_version")
 
 
 class SparseAttnError(RuntimeError):
@@ -72,7 +72,9 @@ def load():
     lib.sa_decode_workspace_size.restype = sz
     lib.sa_decode_fwd.argtypes = [vp, vp, vp, ctypes.c_int, DecodeShape, ctypes.POINTER(BlockStats),
                                   i32, f32, ctypes.c_int, vp, vp, vp, vp, sz, vp]
-    for fn in ("sa_block_pool", "sa_route", "sa_sparse_attn_fwd", "sa_decode_fwd"):
+    lib.sa_decode_fwd_static.argtypes = [vp, vp, vp, ctypes.c_int, DecodeShape, ctypes.POINTER(BlockStats),
+                                         i32, f32, ctypes.c_int, vp, vp, vp, vp]
+    for fn in ("sa_block_pool", "sa_route", "sa_sparse_attn_fwd", "sa_decode_fwd", "sa_decode_fwd_static"):
         getattr(lib, fn).restype = ctypes.c_int
     lib.sa_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
     lib.sa_device_error.restype = ctypes.c_int
@@ -211,4 +213,25 @@ def decode_fwd(q, Kcache, Vcache, stats: dict, block: int, topk: int, scale: flo
                              DecodeShape(Bsz, Hq, Hkv, N, d, block), ctypes.byref(cst), int(topk),
                              float(scale), TAIL[tail], _ptr(idx), _ptr(sc), _ptr(o),
                              _ptr(workspace), workspace.numel(), _stream(stream)))
+    return o, idx, sc
+
+
+def decode_fwd_static(q, Kcache, Vcache, stats: dict, block: int, topk: int, scale: float, *,
+                      tail: str = "zero_order", out=None, stream=None):
+    """decode_fwd with the library's static scratch instead of a workspace
+    (see sa_decode_fwd_static); returns (o, block_idx, scores)."""
+    lib = load()
+    Bsz, Hq, d = q.shape
+    Hkv, N = Kcache.shape[1], Kcache.shape[2]
+    nb = N // block
+    dev = q.device
+    o = out if out is not None else torch.empty_like(q)
+    idx = torch.empty(Bsz, Hkv, topk, device=dev, dtype=torch.int32)
+    sc = torch.empty(Bsz, Hkv, nb, device=dev, dtype=torch.float32)
+    cst = _stats_struct(stats)
+    _check("sa_decode_fwd_static",
+           lib.sa_decode_fwd_static(_ptr(q), _ptr(Kcache), _ptr(Vcache), _dtype_code(q),
+                                    DecodeShape(Bsz, Hq, Hkv, N, d, block), ctypes.byref(cst), int(topk),
+                                    float(scale), TAIL[tail], _ptr(idx), _ptr(sc), _ptr(o),
+                                    _stream(stream)))
     return o, idx, sc

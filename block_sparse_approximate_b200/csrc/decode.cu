@@ -13,6 +13,8 @@
 //                           PISA zero-order pseudo-keys of this split's share of
 //                           the unselected blocks -> partial (max, sum, acc)
 //   4. decode_combine_kernel  merges the partial states -> o
+#include <mutex>
+
 #include "topk.cuh"
 
 namespace sa {
@@ -441,4 +443,61 @@ extern "C" sa_status sa_decode_fwd(const void* q, const void* Kcache, const void
                               scores_out, O, ws, s);
   return launch_decode<64>(q, Kcache, Vcache, shape, *stats, topk, scale, tail, block_idx_out,
                            scores_out, O, ws, s);
+}
+
+// ---- decode with library-owned scratch ---------------------------------------
+// sa_decode_fwd_static runs the same kernels as sa_decode_fwd, with its
+// scratch (route scores, selected indices, per-split partial states) in this
+// file-scope device array instead of a caller workspace.  The array exists
+// once per device that loads the library and stays allocated until the
+// process exits.  Host code must not hand `g_decode_scratch` itself to a
+// kernel (on the host it names a shadow variable, not device memory); the
+// device address is looked up once per device with cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_decode_scratch[SA_DECODE_STATIC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_addr[kMaxDevices] = {};
+
+// Device address of g_decode_scratch on the current device (looked up on the
+// first call per device, with that device current).
+sa_status static_scratch(void** out) {
+  using namespace sa;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return launch_status("sa_decode_fwd_static: cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(SA_ERR_UNSUPPORTED, "sa_decode_fwd_static: device index above 63");
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_addr[dev] == nullptr) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
+    if (e != cudaSuccess || p == nullptr)
+      return fail(SA_ERR_CUDA, std::string("sa_decode_fwd_static: cudaGetSymbolAddress failed: ") +
+                                   cudaGetErrorString(e));
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return SA_OK;
+}
+}  // namespace
+
+extern "C" sa_status sa_decode_fwd_static(const void* q, const void* Kcache, const void* Vcache,
+                                          sa_dtype dtype, sa_decode_shape shape,
+                                          const sa_block_stats* stats, int32_t topk, float scale,
+                                          sa_tail_mode tail, int32_t* block_idx_out,
+                                          float* scores_out, void* O, void* stream) {
+  using namespace sa;
+  const size_t need = sa_decode_workspace_size(shape, topk);
+  if (need > SA_DECODE_STATIC_SCRATCH_BYTES)
+    return fail(SA_ERR_WORKSPACE, "sa_decode_fwd_static: this problem needs " + std::to_string(need) +
+                                      " bytes of scratch; the library's static scratch holds " +
+                                      std::to_string((size_t)SA_DECODE_STATIC_SCRATCH_BYTES) +
+                                      " bytes (use sa_decode_fwd with a workspace)");
+  void* scratch = nullptr;
+  sa_status r = static_scratch(&scratch);
+  if (r != SA_OK) return r;
+  // every scratch entry the kernels read is written earlier in the same call,
+  // so the contents left by a previous call need no clearing
+  return sa_decode_fwd(q, Kcache, Vcache, dtype, shape, stats, topk, scale, tail, block_idx_out,
+                       scores_out, O, scratch, SA_DECODE_STATIC_SCRATCH_BYTES, stream);
 }

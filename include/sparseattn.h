@@ -164,6 +164,41 @@ sa_status sa_decode_fwd(const void* q, const void* Kcache, const void* Vcache, s
                         float* scores_out, void* O, void* workspace, size_t workspace_bytes,
                         void* stream);
 
+/* Size of the scratch array that sa_decode_fwd_static uses: 8 MiB.  It holds
+ * the route scores, the kept indices and the per-split partial states of one
+ * call; the 16-sequence x 8-KV-head x 131072-token decode with topk 64 needs
+ * about 7.1 MiB. */
+#define SA_DECODE_STATIC_SCRATCH_BYTES (8u << 20)
+
+/* sa_decode_fwd for callers that cannot allocate device memory.
+ * Not part of the method: the pages have no counterpart to it.
+ *
+ * Some callers have no device allocator they may use: a plugin or
+ * foreign-function host that only passes the tensors it was given and has no
+ * way to request a workspace, or a serving loop that must not call cudaMalloc
+ * because it can synchronise the whole device.  This entry point takes the
+ * same arguments as sa_decode_fwd minus the workspace and allocates nothing:
+ * its scratch is a static device array of SA_DECODE_STATIC_SCRATCH_BYTES that
+ * every GPU loading the library holds until the process exits.  Inputs and
+ * outputs are still the caller's.
+ *   - A problem whose sa_decode_workspace_size() exceeds
+ *     SA_DECODE_STATIC_SCRATCH_BYTES is rejected with SA_ERR_WORKSPACE before
+ *     anything runs.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture.  Later calls do no set-up.
+ *   - Every call on a device shares the one array and it keeps the last
+ *     call's contents (nothing in it needs clearing: each call writes every
+ *     entry before reading it).  Calls whose executions overlap on the GPU
+ *     (different streams, no ordering between them) race on the array and
+ *     corrupt each other's results: serialise them.
+ * Errors: as sa_decode_fwd, plus SA_ERR_WORKSPACE for a problem too large for
+ * the static scratch and SA_ERR_CUDA if the symbol lookup fails. */
+sa_status sa_decode_fwd_static(const void* q, const void* Kcache, const void* Vcache, sa_dtype dtype,
+                               sa_decode_shape shape, const sa_block_stats* stats, int32_t topk,
+                               float scale, sa_tail_mode tail, int32_t* block_idx_out,
+                               float* scores_out, void* O, void* stream);
+
 /* Reads and clears the library's device-side error word (synchronous: waits
  * for work already queued on the legacy default stream).  Non-zero means a
  * kernel gave up on an internal wait (bit 0: a bounded barrier wait timed
