@@ -205,12 +205,15 @@ def run_reference(args, world, rank):
 # GPU arm
 # --------------------------------------------------------------------------
 
-def time_decode(steps: int = 50, warmup: int = 5):
+def time_decode(steps: int = 50, warmup: int = 5, batch=None):
     """Decode workload timing (separate from the prefill step): GB/s of the
-    bytes the method moves per decode step."""
+    bytes the method moves per decode step.  ``batch`` shrinks the number of
+    sequences (for bounded profiler captures)."""
     from block_sparse_approximate_b200 import binding as bd
     from block_sparse_approximate_b200.pipeline import DecodeStep
     w = wl.WORKLOADS["decode"]
+    if batch:
+        w = wl.Workload(**{**w.__dict__, "B": int(batch)})
     inp = wl.decode_inputs(w, "cuda")
     st = bd.block_pool(None, inp["Kcache"], inp["Vcache"], w.block, variance=True)
     step = DecodeStep(w, inp, st)
@@ -241,6 +244,10 @@ def run_ours(args, world, rank, local):
     from block_sparse_approximate_b200.pipeline import PrefillStep
     torch.cuda.set_device(local)
     bd.load()
+    if args.only == "decode":
+        if rank == 0:
+            print(json.dumps({"decode": time_decode(args.steps, args.warmup, args.decode_batch)}), flush=True)
+        return 0
     w = wl.WORKLOADS[WORKLOAD]
     wr = wl.Workload(**{**w.__dict__, "seed": w.seed + 1000 * rank}) if rank else w
     inp = wl.prefill_inputs(wr, "cuda")
@@ -330,10 +337,10 @@ def run_ours(args, world, rank, local):
                "d2h_bytes_per_step": step.buf.out.numel() * step.buf.out.element_size()}
 
     decode = None
-    if rank == 0 and not args.no_decode:
+    if rank == 0 and args.only == "all" and not args.no_decode:
         del step
         torch.cuda.empty_cache()
-        decode = time_decode()
+        decode = time_decode(batch=args.decode_batch)
     ck = clocks.stop() if clocks else None
 
     if rank != 0:
@@ -382,6 +389,10 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
+                    help="prefill: the timed step only; decode: only the decode timing")
+    ap.add_argument("--decode-batch", type=int, default=None,
+                    help="sequences in the decode workload (default: the full 16)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
