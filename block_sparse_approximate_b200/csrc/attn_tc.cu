@@ -13,16 +13,21 @@
 //                     to the denominator,
 // so the tail costs 1/B of the dense work and no N×N matrix exists.
 //
-// Warp roles (192 threads, one CTA per SM):
-//   warps 0-3  softmax: thread r owns query row r (TMEM lane r); reads S from
-//              TMEM, keeps (max, sum) in registers, writes P back into TMEM as
-//              bf16 over the S columns, rescales O in TMEM when the running
-//              max grows by more than 2^8, and writes the output;
-//   warp 4     TMA producer: Q once, then K/V tiles into a 3-stage ring;
-//   warp 5     MMA issuer: S = Q·Kᵀ (both operands K-major in shared memory)
-//              into a double-buffered S in TMEM, then O += P·V with P read
-//              from TMEM and V as an MN-major shared-memory operand.
-// TMEM: S0 cols [0,128), S1 [128,256), O [256,384) of a 512-column allocation.
+// Warp roles (320 threads, one CTA per SM):
+//   warps 0-3, 4-7  two softmax warpgroups ("streams"): stream s takes the
+//              tiles t with t % 2 == s, so the two halves of the tile list are
+//              reduced concurrently and merged at the end (the same merge as
+//              split-KV decoding).  Thread r of a group owns query row r (TMEM
+//              lane r): it reads its S row from TMEM, keeps (max, sum) in
+//              registers, writes P back into TMEM as bf16 over the S columns,
+//              and rescales its O row in TMEM only when the running max grows
+//              by more than 2^8;
+//   warp 8     TMA producer: Q once, then K/V tiles into a 3-stage ring;
+//   warp 9     MMA issuer: S = Q·Kᵀ (both operands K-major in shared memory)
+//              into the stream's S, and O_s += P·V with P read from TMEM and V
+//              as an MN-major shared-memory operand, alternating the streams
+//              so one group's softmax overlaps the other group's MMAs.
+// TMEM (512 columns): S_0 [0,128), S_1 [128,256), O_0 [256,384), O_1 [384,512).
 #include <mutex>
 
 #include "attn_simt.cuh"
@@ -36,8 +41,8 @@ using namespace tc;
 constexpr int TB = 128;                        // rows per tile (queries and keys)
 constexpr int TD = 128;                        // head dim
 constexpr int NS = 3;                          // K/V pipeline stages
-constexpr int kTcThreads = 192;
-constexpr int kTmaWarp = 4, kMmaWarp = 5;
+constexpr int kTcThreads = 320;
+constexpr int kTmaWarp = 8, kMmaWarp = 9;
 constexpr uint32_t kHalfTile = TB * 64 * 2;    // 128 rows x 64 bf16 (one 128-byte swizzle span)
 constexpr uint32_t kTile = 2 * kHalfTile;      // 128 x 128 bf16
 constexpr uint32_t kTmemCols = 512;
@@ -49,10 +54,10 @@ constexpr int B_Q = 0;
 constexpr int B_KF = 1;                 // NS
 constexpr int B_VF = B_KF + NS;         // NS
 constexpr int B_KE = B_VF + NS;         // NS
-constexpr int B_SF = B_KE + NS;         // 2
-constexpr int B_PR = B_SF + 2;          // 2
-constexpr int B_OD = B_PR + 2;          // 1
-constexpr int B_FIN = B_OD + 1;         // 1
+constexpr int B_SF = B_KE + NS;         // 2 (per stream)
+constexpr int B_PR = B_SF + 2;          // 2 (per stream)
+constexpr int B_OD = B_PR + 2;          // 2 (per stream)
+constexpr int B_FIN = B_OD + 2;         // 1
 constexpr int NBAR = B_FIN + 1;
 
 constexpr uint32_t kBarOff = kTile * (1 + 2 * NS);
@@ -74,6 +79,11 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity) {
     if (done) return true;
     if (clock64() - t0 > kWaitCycles / 8) return false;
   }
+}
+
+__device__ __forceinline__ void named_bar_softmax() {
+  // barrier 1 over the two softmax warpgroups (256 threads)
+  asm volatile("bar.sync 1, 256;" ::: "memory");
 }
 
 template <bool ZO>
@@ -107,13 +117,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(B_SF + s), 1);
       mbar_init(bar(B_PR + s), 128);
+      mbar_init(bar(B_OD + s), 1);
     }
-    mbar_init(bar(B_OD), 1);
     mbar_init(bar(B_FIN), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  for (int w = threadIdx.x; w < nwords; w += kTcThreads) selmask[w] = 0u;
+  // selection bitmap, padded with 4 zero words so a tile's 4 words never run past it
+  for (int w = threadIdx.x; w < nwords + 4; w += kTcThreads) selmask[w] = 0u;
   if (warp == 0) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
   __syncthreads();
   for (int s = threadIdx.x; s < topk; s += kTcThreads) {
@@ -169,35 +180,38 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     if (lane == 0 && T > 0) {
       constexpr uint32_t idS = idesc_bf16_f32(TB, TB, 0, 0);
       constexpr uint32_t idO = idesc_bf16_f32(TB, TD, 0, 1);
+      // S(t) = Q K_tᵀ into the S columns of stream t % 2
+      auto issue_s = [&](int t) -> bool {
+        const int s = t % NS;
+        if (!mbar_wait(bar(B_KF + s), (t / NS) & 1, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t ka = sb + kTile * (1 + 2 * s);
+        const uint32_t d = tbase + (uint32_t)(t & 1) * TB;
+#pragma unroll
+        for (int k = 0; k < TD / 16; ++k) {
+          const uint32_t koff = (k >> 2) * kHalfTile + (k & 3) * 32;
+          mma_ss(d, desc_sw128(sb + koff, 16, 1024), desc_sw128(ka + koff, 16, 1024), idS, k > 0);
+        }
+        mma_commit(bar(B_SF + (t & 1)));
+        return true;
+      };
       bool ok = mbar_wait(bar(B_Q), 0, abort_flag);
-      for (int t = 0; ok && t <= T; ++t) {
-        if (t < T) {
-          const int s = t % NS;
-          if (!mbar_wait(bar(B_KF + s), (t / NS) & 1, abort_flag)) break;
-          tc_fence_after();
-          const uint32_t ka = sb + kTile * (1 + 2 * s);
-          const uint32_t d = tbase + (uint32_t)(t & 1) * TB;
+      if (ok) ok = issue_s(0);
+      if (ok && T > 1) ok = issue_s(1);
+      for (int t = 0; ok && t < T; ++t) {
+        const int st = t & 1, u = t >> 1, su = t % NS;
+        if (!mbar_wait(bar(B_PR + st), u & 1, abort_flag)) break;
+        if (!mbar_wait(bar(B_VF + su), (t / NS) & 1, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t va = sb + kTile * (2 + 2 * su);
+        const uint32_t pa = tbase + (uint32_t)st * TB;
+        const uint32_t od = tbase + kColO + (uint32_t)st * TD;
 #pragma unroll
-          for (int k = 0; k < TD / 16; ++k) {
-            const uint32_t koff = (k >> 2) * kHalfTile + (k & 3) * 32;
-            mma_ss(d, desc_sw128(sb + koff, 16, 1024), desc_sw128(ka + koff, 16, 1024), idS, k > 0);
-          }
-          mma_commit(bar(B_SF + (t & 1)));
-        }
-        if (t >= 1) {
-          const int u = t - 1, su = u % NS;
-          if (!mbar_wait(bar(B_PR + (u & 1)), (u >> 1) & 1, abort_flag)) break;
-          if (!mbar_wait(bar(B_VF + su), (u / NS) & 1, abort_flag)) break;
-          tc_fence_after();
-          const uint32_t va = sb + kTile * (2 + 2 * su);
-          const uint32_t pa = tbase + (uint32_t)(u & 1) * TB;
-#pragma unroll
-          for (int k = 0; k < TB / 16; ++k)
-            mma_ts(tbase + kColO, pa + k * 8, desc_sw128(va + k * 16 * 128, kHalfTile, 1024), idO,
-                   (u > 0 || k > 0));
-          mma_commit(bar(B_KE + su));
-          mma_commit(bar(B_OD));
-        }
+        for (int k = 0; k < TB / 16; ++k)
+          mma_ts(od, pa + k * 8, desc_sw128(va + k * 16 * 128, kHalfTile, 1024), idO, (u > 0 || k > 0));
+        mma_commit(bar(B_KE + su));
+        mma_commit(bar(B_OD + st));
+        if (t + 2 < T && !issue_s(t + 2)) break;
       }
       // every MMA issued above has completed before TMEM is released
       mma_commit(bar(B_FIN));
@@ -205,13 +219,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     }
   } else {
     // ------------------------------------------------------------ softmax
-    const int r = warp * 32 + lane;
-    const uint32_t lrow = tbase + ((uint32_t)(warp * 32) << 16);
+    const int st = warp >> 2;                   // stream
+    const int wq = warp & 3;                    // TMEM lane quarter
+    const int r = wq * 32 + lane;               // query row
+    const uint32_t lrow = tbase + ((uint32_t)(wq * 32) << 16);
+    const uint32_t s_col = (uint32_t)st * TB;
+    const uint32_t o_col = kColO + (uint32_t)st * TD;
+    const int U = T > st ? (T - st + 1) / 2 : 0;   // tiles of this stream
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int t = 0; t < T; ++t) {
-      const int sbuf = t & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_SF + sbuf), (t >> 1) & 1, abort_flag))) {
+    for (int u = 0; u < U; ++u) {
+      const int t = 2 * u + st;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_SF + st), u & 1, abort_flag))) {
         ok = false;
         break;
       }
@@ -219,28 +238,34 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       uint32_t v[128];
 #pragma unroll
       for (int c = 0; c < 4; ++c)
-        tmem_ld32(lrow + sbuf * TB + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * c]));
+        tmem_ld32(lrow + s_col + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * c]));
       tmem_wait_ld();
-      float mx = -INFINITY;
-      if (t < topk) {
-#pragma unroll
-        for (int n = 0; n < TB; ++n) {
-          const float x = __uint_as_float(v[n]) * scale2;
-          v[n] = __float_as_uint(x);
-          mx = fmaxf(mx, x);
-        }
-      } else {
+      const bool centroid = t >= topk;
+      float bias = 0.f;
+      if (centroid) {
+        // validity of the 128 pseudo-keys: inside the head and not selected
         const int jb = (t - topk) * TB;
+        bias = 7.0f;   // log2 of the block size 128
 #pragma unroll
-        for (int n = 0; n < TB; ++n) {
-          const int j = jb + n;
-          const bool valid = j < nb && !((selmask[j >> 5] >> (j & 31)) & 1u);
-          const float x = valid ? fmaf(__uint_as_float(v[n]), scale2, 7.0f) : -INFINITY;  // + log2(128)
-          v[n] = __float_as_uint(x);
-          mx = fmaxf(mx, x);
+        for (int c = 0; c < 4; ++c) {
+          const int w0 = (jb >> 5) + c;
+          const int lim = nb - (jb + 32 * c);
+          const uint32_t range = lim >= 32 ? 0xffffffffu : (lim <= 0 ? 0u : ((1u << lim) - 1u));
+          const uint32_t valid = ~selmask[w0] & range;
+#pragma unroll
+          for (int n = 0; n < 32; ++n)
+            if (!((valid >> n) & 1u)) v[32 * c + n] = __float_as_uint(-INFINITY);
         }
       }
-      const float m_new = fmaxf(m_used, mx);
+      float mx8[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) mx8[k] = -INFINITY;
+#pragma unroll
+      for (int n = 0; n < TB; ++n) mx8[n & 7] = fmaxf(mx8[n & 7], __uint_as_float(v[n]));
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      const float m_tile = mx == -INFINITY ? -INFINITY : fmaf(mx, scale2, bias);
+      const float m_new = fmaxf(m_used, m_tile);
       const bool need = m_new > m_used + kLazyRescale;
       float factor = 1.f;
       if (need) {
@@ -248,21 +273,24 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         m_used = m_new;
       }
       const bool live = m_used != -INFINITY;
-      float sum = 0.f;
-      uint32_t pk[64];
+      const float neg = bias - m_used;
+      float sm8[8];
 #pragma unroll
-      for (int n = 0; n < 64; ++n) {
-        const float p0 = live ? fast_exp2(__uint_as_float(v[2 * n]) - m_used) : 0.f;
-        const float p1 = live ? fast_exp2(__uint_as_float(v[2 * n + 1]) - m_used) : 0.f;
-        sum += p0 + p1;
-        pk[n] = pack_bf16(p0, p1);
+      for (int k = 0; k < 8; ++k) sm8[k] = 0.f;
+#pragma unroll
+      for (int n = 0; n < TB / 2; ++n) {
+        const float p0 = live ? fast_exp2(fmaf(__uint_as_float(v[2 * n]), scale2, neg)) : 0.f;
+        const float p1 = live ? fast_exp2(fmaf(__uint_as_float(v[2 * n + 1]), scale2, neg)) : 0.f;
+        sm8[n & 7] += p0 + p1;
+        v[n] = pack_bf16(p0, p1);
       }
+      const float sum = ((sm8[0] + sm8[1]) + (sm8[2] + sm8[3])) + ((sm8[4] + sm8[5]) + (sm8[6] + sm8[7]));
       l = l * factor + sum;
-      tmem_st32(lrow + sbuf * TB, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-      tmem_st32(lrow + sbuf * TB + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+      tmem_st32(lrow + s_col, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+      tmem_st32(lrow + s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
       tmem_wait_st();
-      if (t >= 1) {
-        if (!__all_sync(0xffffffffu, mbar_wait(bar(B_OD), (t - 1) & 1, abort_flag))) {
+      if (u >= 1) {
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(B_OD + st), (u - 1) & 1, abort_flag))) {
           ok = false;
           break;
         }
@@ -271,42 +299,67 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             uint32_t o[32];
-            tmem_ld32(lrow + kColO + 32 * c, o);
+            tmem_ld32(lrow + o_col + 32 * c, o);
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
-            tmem_st32(lrow + kColO + 32 * c, o);
+            tmem_st32(lrow + o_col + 32 * c, o);
           }
           tmem_wait_st();
         }
       }
       tc_fence_before();
-      mbar_arrive(bar(B_PR + sbuf));
+      mbar_arrive(bar(B_PR + st));
     }
-    if (ok && T > 0) {
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_OD), (T - 1) & 1, abort_flag));
-      tc_fence_after();
-    }
+    if (ok && U > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_OD + st), (U - 1) & 1, abort_flag));
+    // both groups past their last PV: every MMA that reads Q has completed,
+    // so the Q tile's shared memory can carry the (max, sum) exchange
+    named_bar_softmax();
+    float* ex = reinterpret_cast<float*>(smem);   // [2 streams][2][128]
+    ex[st * 256 + r] = (U > 0) ? m_used : -INFINITY;
+    ex[st * 256 + 128 + r] = l;
+    named_bar_softmax();
+    const float m0 = ex[r], l0 = ex[128 + r], m1 = ex[256 + r], l1 = ex[384 + r];
+    const int U0 = T > 0 ? (T + 1) / 2 : 0, U1 = T > 1 ? T / 2 : 0;
+    const float M = fmaxf(m0, m1);
+    const float f0 = (U0 > 0 && m0 != -INFINITY) ? fast_exp2(m0 - M) : 0.f;
+    const float f1 = (U1 > 0 && m1 != -INFINITY) ? fast_exp2(m1 - M) : 0.f;
+    const float L = l0 * f0 + l1 * f1;
+    const float inv = L > 0.f ? 1.0f / L : 0.f;
+    ok = __all_sync(0xffffffffu, ok) && !*abort_flag;
     if (ok) {
-      const float inv = l > 0.f ? 1.0f / l : 0.f;
-      uint4* orow = reinterpret_cast<uint4*>(O + ((size_t)bh * N + (size_t)i * TB + r) * TD);
+      tc_fence_after();
+      // stream st writes output columns [64 st, 64 st + 64) of its rows
+      uint4* orow = reinterpret_cast<uint4*>(O + ((size_t)bh * N + (size_t)i * TB + r) * TD + 64 * st);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t o[32];
-        if (T > 0) {
-          tmem_ld32(lrow + kColO + 32 * c, o);
-          tmem_wait_ld();
-        } else {
+      for (int c = 0; c < 2; ++c) {
+        uint32_t a[32], b[32];
+        if (U0 > 0) {
+          tmem_ld32(lrow + kColO + 64 * st + 32 * c, a);
+        }
+        if (U1 > 0) {
+          tmem_ld32(lrow + kColO + TD + 64 * st + 32 * c, b);
+        }
+        tmem_wait_ld();
+        if (U0 == 0) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = 0u;
+          for (int e = 0; e < 32; ++e) a[e] = 0u;
+        }
+        if (U1 == 0) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) b[e] = 0u;
         }
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
+          float y[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            y[e] = (__uint_as_float(a[8 * q + e]) * f0 + __uint_as_float(b[8 * q + e]) * f1) * inv;
           uint4 w;
-          w.x = pack_bf16(__uint_as_float(o[8 * q + 0]) * inv, __uint_as_float(o[8 * q + 1]) * inv);
-          w.y = pack_bf16(__uint_as_float(o[8 * q + 2]) * inv, __uint_as_float(o[8 * q + 3]) * inv);
-          w.z = pack_bf16(__uint_as_float(o[8 * q + 4]) * inv, __uint_as_float(o[8 * q + 5]) * inv);
-          w.w = pack_bf16(__uint_as_float(o[8 * q + 6]) * inv, __uint_as_float(o[8 * q + 7]) * inv);
+          w.x = pack_bf16(y[0], y[1]);
+          w.y = pack_bf16(y[2], y[3]);
+          w.z = pack_bf16(y[4], y[5]);
+          w.w = pack_bf16(y[6], y[7]);
           orow[4 * c + q] = w;
         }
       }
@@ -341,7 +394,7 @@ EncodeTiledFn encode_fn() {
 }
 
 size_t tc_smem_bytes(int nb) {
-  return 1024 + kMaskOff + 4 * (size_t)((nb + 31) / 32) + 16;
+  return 1024 + kMaskOff + 4 * (size_t)((nb + 31) / 32 + 4);
 }
 
 }  // namespace
