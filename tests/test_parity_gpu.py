@@ -54,7 +54,7 @@ def test_block_pool_large_offset_variance(lib):
 # --------------------------------------------------------------------------
 
 @pytest.mark.parametrize("mode", ["dot", "proj", "taylor2"])
-@pytest.mark.parametrize("nb,k", [(37, 5), (256, 26), (16, 0), (16, 16)])
+@pytest.mark.parametrize("nb,k", [(37, 5), (256, 26), (16, 0), (16, 16), (97, 64), (97, 65), (300, 100)])
 def test_route(lib, mode, nb, k):
     d, block = 128, 128
     w = wl.WORKLOADS["video_dit"]
