@@ -38,6 +38,27 @@ def _headers():
     return sorted(glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(INCLUDE, "*.h")))
 
 
+# attn_tc_kernel reallocates registers with setmaxnreg: its launch register
+# count times 384 threads must cover 256 x 216 + 128 x 40 (see attn_tc.cu), or
+# setmaxnreg.inc would wait for registers that never come.
+TC_MIN_LAUNCH_REGS = 158
+
+
+def _check_tc_registers(ptxas_log: str):
+    import re
+    lines = ptxas_log.splitlines()
+    for k, line in enumerate(lines):
+        if "Compiling entry function" in line and "attn_tc_kernel" in line:
+            for nxt in lines[k + 1:k + 4]:
+                m = re.search(r"Used (\d+) registers", nxt)
+                if m:
+                    regs = int(m.group(1))
+                    if regs < TC_MIN_LAUNCH_REGS:
+                        raise RuntimeError(f"attn_tc_kernel launches with {regs} registers per thread; "
+                                           f"the setmaxnreg split needs >= {TC_MIN_LAUNCH_REGS}")
+                    break
+
+
 def _stale(target, deps):
     if not os.path.exists(target):
         return True
@@ -53,7 +74,10 @@ def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
         obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
         objs.append(obj)
         if force or _stale(obj, [src] + headers):
-            cmd = [NVCC, *ARCH, *FLAGS, *extra_flags, "-c", src, "-o", obj]
+            extra = list(extra_flags)
+            if os.path.basename(src) == "attn_tc.cu" and "-v" not in extra:
+                extra += ["-Xptxas", "-v"]
+            cmd = [NVCC, *ARCH, *FLAGS, *extra, "-c", src, "-o", obj]
             jobs.append(cmd)
 
     def run(cmd):
@@ -68,6 +92,8 @@ def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
                 print(r.stdout + r.stderr, flush=True)
             if r.returncode != 0:
                 raise RuntimeError("nvcc failed:\n" + " ".join(cmd) + "\n" + r.stdout + r.stderr)
+            if cmd[-3].endswith("attn_tc.cu"):
+                _check_tc_registers(r.stdout + r.stderr)
     if force or jobs or _stale(LIB, objs):
         cmd = [NVCC, *ARCH, "-shared", "-o", LIB, *objs]
         r = subprocess.run(cmd, capture_output=True, text=True)

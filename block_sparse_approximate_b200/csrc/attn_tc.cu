@@ -13,7 +13,8 @@
 //                     to the denominator,
 // so the tail costs 1/B of the dense work and no N×N matrix exists.
 //
-// Warp roles (320 threads, one CTA per SM):
+// Warp roles (384 threads, one CTA per SM; the producer warpgroup gives its
+// registers to the softmax warpgroups with setmaxnreg):
 //   warps 0-3, 4-7  two softmax warpgroups ("streams"): stream s takes the
 //              tiles t with t % 2 == s, so the two halves of the tile list are
 //              reduced concurrently and merged at the end (the same merge as
@@ -23,6 +24,7 @@
 //              and rescales its O row in TMEM only when the running max grows
 //              by more than 2^8;
 //   warp 8     TMA producer: Q once, then K/V tiles into a 3-stage ring;
+//   warps 10-11 idle (they complete the producer warpgroup);
 //   warp 9     MMA issuer: S = Q·Kᵀ (both operands K-major in shared memory)
 //              into the stream's S, and O_s += P·V with P read from TMEM and V
 //              as an MN-major shared-memory operand, alternating the streams
@@ -41,8 +43,11 @@ using namespace tc;
 constexpr int TB = 128;                        // rows per tile (queries and keys)
 constexpr int TD = 128;                        // head dim
 constexpr int NS = 3;                          // K/V pipeline stages
-constexpr int kTcThreads = 320;
+constexpr int kTcThreads = 384;
 constexpr int kTmaWarp = 8, kMmaWarp = 9;
+// register split: 256 softmax threads x 216 + 128 producer threads x 40 =
+// 60416 <= 384 x (launch registers); build.py checks ptxas reports >= 158
+constexpr int kSoftmaxRegs = 216, kProducerRegs = 40;
 constexpr uint32_t kHalfTile = TB * 64 * 2;    // 128 rows x 64 bf16 (one 128-byte swizzle span)
 constexpr uint32_t kTile = 2 * kHalfTile;      // 128 x 128 bf16
 constexpr uint32_t kTmemCols = 512;
@@ -138,6 +143,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 
   if (warp == kTmaWarp) {
     // ------------------------------------------------------------ producer
+    regs_dec<kProducerRegs>();
     if (lane == 0 && T > 0) {
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
@@ -177,6 +183,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
+    regs_dec<kProducerRegs>();
     if (lane == 0 && T > 0) {
       constexpr uint32_t idS = idesc_bf16_f32(TB, TB, 0, 0);
       constexpr uint32_t idO = idesc_bf16_f32(TB, TD, 0, 1);
@@ -217,8 +224,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       mma_commit(bar(B_FIN));
       wait_bounded(bar(B_FIN), 0);
     }
+  } else if (warp >= 8) {
+    regs_dec<kProducerRegs>();                  // idle warps of the producer warpgroup
   } else {
     // ------------------------------------------------------------ softmax
+    regs_inc<kSoftmaxRegs>();
     const int st = warp >> 2;                   // stream
     const int wq = warp & 3;                    // TMEM lane quarter
     const int r = wq * 32 + lane;               // query row
@@ -261,9 +271,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
       for (int k = 0; k < 8; ++k) mx8[k] = -INFINITY;
 #pragma unroll
-      for (int n = 0; n < TB; ++n) mx8[n & 7] = fmaxf(mx8[n & 7], __uint_as_float(v[n]));
-      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      for (int n = 0; n < TB / 2; ++n)
+        mx8[n & 7] = fmax3(mx8[n & 7], __uint_as_float(v[2 * n]), __uint_as_float(v[2 * n + 1]));
+      const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                             fmaxf(mx8[6], mx8[7]));
       const float m_tile = mx == -INFINITY ? -INFINITY : fmaf(mx, scale2, bias);
       const float m_new = fmaxf(m_used, m_tile);
       const bool need = m_new > m_used + kLazyRescale;
@@ -277,11 +288,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       float sm8[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) sm8[k] = 0.f;
+      const float sc2 = live ? scale2 : 0.f, ng = live ? neg : -INFINITY;   // dead row: p = 0
 #pragma unroll
       for (int n = 0; n < TB / 2; ++n) {
-        const float p0 = live ? fast_exp2(fmaf(__uint_as_float(v[2 * n]), scale2, neg)) : 0.f;
-        const float p1 = live ? fast_exp2(fmaf(__uint_as_float(v[2 * n + 1]), scale2, neg)) : 0.f;
-        sm8[n & 7] += p0 + p1;
+        float a0, a1;
+        ffma2(a0, a1, __uint_as_float(v[2 * n]), __uint_as_float(v[2 * n + 1]), sc2, sc2, ng, ng);
+        const float p0 = fast_exp2(a0), p1 = fast_exp2(a1);
+        fadd2(sm8[2 * (n & 3)], sm8[2 * (n & 3) + 1], p0, p1);
         v[n] = pack_bf16(p0, p1);
       }
       const float sum = ((sm8[0] + sm8[1]) + (sm8[2] + sm8[3])) + ((sm8[4] + sm8[5]) + (sm8[6] + sm8[7]));
