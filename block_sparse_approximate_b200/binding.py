@@ -26,7 +26,8 @@ TAIL = {"drop": 0, "zero_order": 1, "linear_mix": 2}
 
 # every entry point declared in include/sparseattn.h
 EXPORTS = ("sa_block_pool", "sa_route", "sa_sparse_attn_fwd", "sa_decode_workspace_size",
-           "sa_decode_fwd", "sa_decode_fwd_static", "sa_device_error", "sa_last_error", "sa_version")
+           "sa_decode_fwd", "sa_decode_fwd_static", "sa_quantize_e4m3", "sa_sparse_attn_fwd_fp8",
+           "sa_device_error", "sa_last_error", "sa_version")
 
 
 class SparseAttnError(RuntimeError):
@@ -52,6 +53,14 @@ class BlockStats(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in _STAT_FIELDS]
 
 
+_FP8_FIELDS = ("q", "k", "v", "q_scale", "k_scale", "v_scale", "v_scale_max", "kbar", "vbar",
+               "kbar_scale", "vbar_scale")
+
+
+class Fp8Operands(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in _FP8_FIELDS]
+
+
 _lib = None
 
 
@@ -74,7 +83,10 @@ def load():
                                   i32, f32, ctypes.c_int, vp, vp, vp, vp, sz, vp]
     lib.sa_decode_fwd_static.argtypes = [vp, vp, vp, ctypes.c_int, DecodeShape, ctypes.POINTER(BlockStats),
                                          i32, f32, ctypes.c_int, vp, vp, vp, vp]
-    for fn in ("sa_block_pool", "sa_route", "sa_sparse_attn_fwd", "sa_decode_fwd", "sa_decode_fwd_static"):
+    lib.sa_quantize_e4m3.argtypes = [vp, ctypes.c_int64, i32, i32, i32, vp, vp, vp, vp]
+    lib.sa_sparse_attn_fwd_fp8.argtypes = [ctypes.POINTER(Fp8Operands), Shape, vp, i32, ctypes.c_int, f32, vp, vp]
+    for fn in ("sa_block_pool", "sa_route", "sa_sparse_attn_fwd", "sa_decode_fwd", "sa_decode_fwd_static",
+               "sa_quantize_e4m3", "sa_sparse_attn_fwd_fp8"):
         getattr(lib, fn).restype = ctypes.c_int
     lib.sa_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
     lib.sa_device_error.restype = ctypes.c_int
@@ -235,3 +247,45 @@ def decode_fwd_static(q, Kcache, Vcache, stats: dict, block: int, topk: int, sca
                                     float(scale), TAIL[tail], _ptr(idx), _ptr(sc), _ptr(o),
                                     _stream(stream)))
     return o, idx, sc
+
+
+def quantize_e4m3(X: torch.Tensor, block: int = 128, *, want_max: bool = False, stream=None):
+    """Per-block e4m3 codes of a bf16 tensor [B,H,N,d]: returns (codes uint8
+    [B,H,N,d], scales float32 [B,H,ceil(N/block)], scale_max [B,H] or None)."""
+    lib = load()
+    Bsz, H, N, d = X.shape
+    nblk = (N + block - 1) // block
+    codes = torch.empty(X.shape, device=X.device, dtype=torch.uint8)
+    scales = torch.empty(Bsz, H, nblk, device=X.device, dtype=torch.float32)
+    smax = torch.empty(Bsz, H, device=X.device, dtype=torch.float32) if want_max else None
+    _check("sa_quantize_e4m3", lib.sa_quantize_e4m3(_ptr(X), Bsz * H, N, d, block, _ptr(codes), _ptr(scales),
+                                                    _ptr(smax), _stream(stream)))
+    return codes, scales, smax
+
+
+def fp8_operands(Q, K, V, stats: dict, block: int = 128, stream=None) -> dict:
+    """Quantises Q, K, V and (if present) the bf16 centroid tiles of ``stats``."""
+    q, qs, _ = quantize_e4m3(Q, block, stream=stream)
+    k, ks, _ = quantize_e4m3(K, block, stream=stream)
+    v, vs, vmax = quantize_e4m3(V, block, want_max=True, stream=stream)
+    ops = {"q": q, "k": k, "v": v, "q_scale": qs, "k_scale": ks, "v_scale": vs, "v_scale_max": vmax}
+    if stats.get("kmean_bf16") is not None:
+        ops["kbar"], ops["kbar_scale"], _ = quantize_e4m3(stats["kmean_bf16"].view(torch.bfloat16), 128,
+                                                          stream=stream)
+        ops["vbar"], ops["vbar_scale"], _ = quantize_e4m3(stats["vmean_bf16"].view(torch.bfloat16), 128,
+                                                          stream=stream)
+    return ops
+
+
+def sparse_attn_fwd_fp8(ops: dict, shape, block_idx, tail: str, scale: float, *, out=None, stream=None):
+    """e4m3 sparse prefill; ``ops`` from fp8_operands; returns bf16 O [B,H,N,d]."""
+    lib = load()
+    Bsz, H, N, d, block = shape
+    O = out if out is not None else torch.empty(Bsz, H, N, d, device=ops["q"].device, dtype=torch.bfloat16)
+    topk = block_idx.shape[-1] if block_idx is not None else 0
+    cops = Fp8Operands(*[_ptr(ops.get(n)) for n in _FP8_FIELDS])
+    _check("sa_sparse_attn_fwd_fp8",
+           lib.sa_sparse_attn_fwd_fp8(ctypes.byref(cops), Shape(Bsz, H, N, d, block),
+                                      _ptr(block_idx) if topk > 0 else None, int(topk), TAIL[tail],
+                                      float(scale), _ptr(O), _stream(stream)))
+    return O

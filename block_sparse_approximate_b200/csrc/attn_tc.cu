@@ -1,5 +1,7 @@
 // Sparse prefill on the 5th-generation tensor cores (tcgen05 + TMEM + TMA),
-// bf16 Q/K/V, 128-token blocks, d = 128, tails drop and zero-order.
+// 128-token blocks, d = 128, tails drop and zero-order, with bf16 operands
+// (kind::f16) or per-block-scaled e4m3 operands (kind::f8f6f4, SLA2 §2C's
+// low-precision sparse branch).
 //
 // PISA's fused kernel ("Implementação de Hardware") interleaves the exact
 // scan over the selected blocks and the approximate scan over the block
@@ -30,9 +32,18 @@
 //              as an MN-major shared-memory operand, alternating the streams
 //              so one group's softmax overlaps the other group's MMAs.
 // TMEM (512 columns): S_0 [0,128), S_1 [128,256), O_0 [256,384), O_1 [384,512).
+//
+// e4m3 variant: Q, K, V (and the centroid tiles) are e4m3 codes with one
+// scale per 128-row block; S = σ_Q σ_K (Q̂·K̂ᵀ).  P is quantised to e4m3 as
+// P · 448 · σ_V(tile) / σ_Vmax (P ≤ 1: the running max is applied at once,
+// not lazily), so the MMA accumulates Σ P σ_V V̂ · 448 / σ_Vmax across tiles of
+// different V scales; the row sum uses the unquantised P.  σ_Vmax is the
+// largest V scale of the head (exact and centroid tiles).
 #include <mutex>
 
 #include "attn_simt.cuh"
+#include <cuda_fp8.h>
+
 #include "tc_util.cuh"
 
 namespace sa {
@@ -42,32 +53,55 @@ using namespace tc;
 
 constexpr int TB = 128;                        // rows per tile (queries and keys)
 constexpr int TD = 128;                        // head dim
-constexpr int NS = 3;                          // K/V pipeline stages
 constexpr int kTcThreads = 384;
 constexpr int kTmaWarp = 8, kMmaWarp = 9;
 // register split: 256 softmax threads x 216 + 128 producer threads x 40 =
 // 60416 <= 384 x (launch registers); build.py checks ptxas reports >= 158
 constexpr int kSoftmaxRegs = 216, kProducerRegs = 40;
-constexpr uint32_t kHalfTile = TB * 64 * 2;    // 128 rows x 64 bf16 (one 128-byte swizzle span)
-constexpr uint32_t kTile = 2 * kHalfTile;      // 128 x 128 bf16
+constexpr uint32_t kSpan = TB * 128;           // 128 rows x one 128-byte swizzle span = 16 KB
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 256;
-constexpr float kLazyRescale = 8.0f;           // log2 units
 
-// barrier slots
-constexpr int B_Q = 0;
-constexpr int B_KF = 1;                 // NS
-constexpr int B_VF = B_KF + NS;         // NS
-constexpr int B_KE = B_VF + NS;         // NS
-constexpr int B_SF = B_KE + NS;         // 2 (per stream)
-constexpr int B_PR = B_SF + 2;          // 2 (per stream)
-constexpr int B_OD = B_PR + 2;          // 2 (per stream)
-constexpr int B_FIN = B_OD + 2;         // 1
-constexpr int NBAR = B_FIN + 1;
+// Operand format of the kernel: spans per 128x128 tile, pipeline depth, MMA
+// K step (in elements), lazy-rescale threshold.
+template <bool F8>
+struct Fmt;
+template <>
+struct Fmt<false> {   // bf16
+  static constexpr int kSpans = 2;             // 256 bytes per row
+  static constexpr int NS = 3;
+  static constexpr int kK = 16;                // K per MMA instruction
+  static constexpr float kLazy = 8.0f;
+};
+template <>
+struct Fmt<true> {    // e4m3
+  static constexpr int kSpans = 1;             // 128 bytes per row
+  static constexpr int NS = 6;
+  static constexpr int kK = 32;
+  static constexpr float kLazy = 0.0f;         // P <= 1 so that P·448 stays in range
+};
 
-constexpr uint32_t kBarOff = kTile * (1 + 2 * NS);
-constexpr uint32_t kSlotOff = kBarOff + 8 * NBAR;     // tmem base, abort flag
-constexpr uint32_t kMaskOff = kSlotOff + 16;
+template <bool F8>
+struct Layout {
+  static constexpr int NS = Fmt<F8>::NS;
+  static constexpr uint32_t kTile = kSpan * Fmt<F8>::kSpans;
+  static constexpr int B_Q = 0, B_KF = 1, B_VF = B_KF + NS, B_KE = B_VF + NS, B_SF = B_KE + NS,
+                       B_PR = B_SF + 2, B_OD = B_PR + 2, B_FIN = B_OD + 2, NBAR = B_FIN + 1;
+  static constexpr uint32_t kBarOff = kTile * (1 + 2 * NS);
+  static constexpr uint32_t kSlotOff = kBarOff + 8 * NBAR;   // tmem base, abort flag
+  static constexpr uint32_t kMaskOff = kSlotOff + 16;
+  static size_t smem_bytes(int nb) { return 1024 + kMaskOff + 4 * (size_t)((nb + 31) / 32 + 4); }
+};
+
+// Scales of the e4m3 operands (all null for bf16).
+struct F8Scales {
+  const float* q;       // [BH][nqb]
+  const float* k;       // [BH][nb]
+  const float* v;       // [BH][nb]
+  const float* v_max;   // [BH]  max over the head's V blocks
+  const float* kbar;    // [BH][ceil(nb/128)]  centroid key tiles
+  const float* vbar;    // [BH][ceil(nb/128)]  centroid value tiles
+};
 
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity) {
   // used only on the abort path, where no other role can release us
@@ -91,21 +125,57 @@ __device__ __forceinline__ void named_bar_softmax() {
   asm volatile("bar.sync 1, 256;" ::: "memory");
 }
 
-template <bool ZO>
+__device__ __forceinline__ void mma_ss_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, {%5, %5, %5, %5}, p;\n\t}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0u)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_ts_f8(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, {%5, %5, %5, %5}, p;\n\t}"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0u)
+      : "memory");
+}
+
+// Instruction descriptor of kind::f8f6f4 with e4m3 A/B and fp32 accumulation.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N, int b_mn_major) {
+  return (1u << 4) | ((uint32_t)b_mn_major << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float d) {
+  const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+  const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(c, d), __NV_SATFINITE, __NV_E4M3);
+  return lo | (hi << 16);
+}
+
+template <bool ZO, bool F8>
 __global__ void __launch_bounds__(kTcThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKb,
                const __grid_constant__ CUtensorMap tmVb, const int32_t* __restrict__ block_idx, int nb,
-               int topk, float scale2, __nv_bfloat16* __restrict__ O, int N) {
+               int topk, float scale2, F8Scales f8, __nv_bfloat16* __restrict__ O, int N) {
+  using L = Layout<F8>;
+  constexpr int NS = L::NS;
+  constexpr uint32_t kTile = L::kTile;
+  constexpr int kSpans = Fmt<F8>::kSpans;
+  constexpr int kK = Fmt<F8>::kK;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
   const int i = blockIdx.x, bh = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kSlotOff);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kSlotOff + 4);
-  uint32_t* selmask = reinterpret_cast<uint32_t*>(smem + kMaskOff);
-  auto bar = [&](int k) { return sb + kBarOff + 8u * k; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kSlotOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kSlotOff + 4);
+  uint32_t* selmask = reinterpret_cast<uint32_t*>(smem + L::kMaskOff);
+  auto bar = [&](int k) { return sb + L::kBarOff + 8u * k; };
 
   const int nwords = (nb + 31) >> 5;
   const int ntail = (ZO && topk < nb) ? (nb + TB - 1) / TB : 0;
@@ -113,18 +183,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const int32_t* sel = block_idx + ((size_t)bh * nb + i) * topk;
 
   if (threadIdx.x == 0) {
-    mbar_init(bar(B_Q), 1);
+    mbar_init(bar(L::B_Q), 1);
     for (int s = 0; s < NS; ++s) {
-      mbar_init(bar(B_KF + s), 1);
-      mbar_init(bar(B_VF + s), 1);
-      mbar_init(bar(B_KE + s), 1);
+      mbar_init(bar(L::B_KF + s), 1);
+      mbar_init(bar(L::B_VF + s), 1);
+      mbar_init(bar(L::B_KE + s), 1);
     }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(bar(B_SF + s), 1);
-      mbar_init(bar(B_PR + s), 128);
-      mbar_init(bar(B_OD + s), 1);
+      mbar_init(bar(L::B_SF + s), 1);
+      mbar_init(bar(L::B_PR + s), 128);
+      mbar_init(bar(L::B_OD + s), 1);
     }
-    mbar_init(bar(B_FIN), 1);
+    mbar_init(bar(L::B_FIN), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -152,32 +222,32 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         prefetch_tmap(&tmKb);
         prefetch_tmap(&tmVb);
       }
-      mbar_expect_tx(bar(B_Q), kTile);
-      tma_load_3d(sb, &tmQ, 0, i * TB, bh, bar(B_Q));
-      tma_load_3d(sb + kHalfTile, &tmQ, 64, i * TB, bh, bar(B_Q));
+      mbar_expect_tx(bar(L::B_Q), kTile);
+#pragma unroll
+      for (int h = 0; h < kSpans; ++h) tma_load_3d(sb + h * kSpan, &tmQ, 64 * h, i * TB, bh, bar(L::B_Q));
       int issued = 0;
       for (int t = 0; t < T; ++t) {
         const int s = t % NS;
-        if (t >= NS && !mbar_wait(bar(B_KE + s), ((t / NS) - 1) & 1, abort_flag)) break;
+        if (t >= NS && !mbar_wait(bar(L::B_KE + s), ((t / NS) - 1) & 1, abort_flag)) break;
         const bool exact = t < topk;
         const CUtensorMap* mk = exact ? &tmK : &tmKb;
         const CUtensorMap* mv = exact ? &tmV : &tmVb;
         const int row = exact ? sel[t] * TB : (t - topk) * TB;
         const uint32_t ka = sb + kTile * (1 + 2 * s), va = ka + kTile;
-        mbar_expect_tx(bar(B_KF + s), kTile);
-        tma_load_3d(ka, mk, 0, row, bh, bar(B_KF + s));
-        tma_load_3d(ka + kHalfTile, mk, 64, row, bh, bar(B_KF + s));
-        mbar_expect_tx(bar(B_VF + s), kTile);
-        tma_load_3d(va, mv, 0, row, bh, bar(B_VF + s));
-        tma_load_3d(va + kHalfTile, mv, 64, row, bh, bar(B_VF + s));
+        mbar_expect_tx(bar(L::B_KF + s), kTile);
+#pragma unroll
+        for (int h = 0; h < kSpans; ++h) tma_load_3d(ka + h * kSpan, mk, 64 * h, row, bh, bar(L::B_KF + s));
+        mbar_expect_tx(bar(L::B_VF + s), kTile);
+#pragma unroll
+        for (int h = 0; h < kSpans; ++h) tma_load_3d(va + h * kSpan, mv, 64 * h, row, bh, bar(L::B_VF + s));
         issued = t + 1;
       }
       if (*abort_flag) {
         // let the loads already in flight land before the CTA goes away
-        wait_bounded(bar(B_Q), 0);
+        wait_bounded(bar(L::B_Q), 0);
         for (int t = issued > NS ? issued - NS : 0; t < issued; ++t) {
-          wait_bounded(bar(B_KF + t % NS), (t / NS) & 1);
-          wait_bounded(bar(B_VF + t % NS), (t / NS) & 1);
+          wait_bounded(bar(L::B_KF + t % NS), (t / NS) & 1);
+          wait_bounded(bar(L::B_VF + t % NS), (t / NS) & 1);
         }
       }
     }
@@ -185,44 +255,51 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     // ------------------------------------------------------------ MMA issuer
     regs_dec<kProducerRegs>();
     if (lane == 0 && T > 0) {
-      constexpr uint32_t idS = idesc_bf16_f32(TB, TB, 0, 0);
-      constexpr uint32_t idO = idesc_bf16_f32(TB, TD, 0, 1);
+      constexpr uint32_t idS = F8 ? idesc_e4m3_f32(TB, TB, 0) : idesc_bf16_f32(TB, TB, 0, 0);
+      constexpr uint32_t idO = F8 ? idesc_e4m3_f32(TB, TD, 1) : idesc_bf16_f32(TB, TD, 0, 1);
       // S(t) = Q K_tᵀ into the S columns of stream t % 2
       auto issue_s = [&](int t) -> bool {
         const int s = t % NS;
-        if (!mbar_wait(bar(B_KF + s), (t / NS) & 1, abort_flag)) return false;
+        if (!mbar_wait(bar(L::B_KF + s), (t / NS) & 1, abort_flag)) return false;
         tc_fence_after();
         const uint32_t ka = sb + kTile * (1 + 2 * s);
         const uint32_t d = tbase + (uint32_t)(t & 1) * TB;
 #pragma unroll
-        for (int k = 0; k < TD / 16; ++k) {
-          const uint32_t koff = (k >> 2) * kHalfTile + (k & 3) * 32;
-          mma_ss(d, desc_sw128(sb + koff, 16, 1024), desc_sw128(ka + koff, 16, 1024), idS, k > 0);
+        for (int k = 0; k < TD / kK; ++k) {
+          // K step k: 32 bytes further along the row, next span every 4 steps
+          const uint32_t koff = (k >> 2) * kSpan + (k & 3) * 32;
+          const uint64_t a = desc_sw128(sb + koff, 16, 1024), b = desc_sw128(ka + koff, 16, 1024);
+          if (F8) mma_ss_f8(d, a, b, idS, k > 0);
+          else mma_ss(d, a, b, idS, k > 0);
         }
-        mma_commit(bar(B_SF + (t & 1)));
+        mma_commit(bar(L::B_SF + (t & 1)));
         return true;
       };
-      bool ok = mbar_wait(bar(B_Q), 0, abort_flag);
+      bool ok = mbar_wait(bar(L::B_Q), 0, abort_flag);
       if (ok) ok = issue_s(0);
       if (ok && T > 1) ok = issue_s(1);
       for (int t = 0; ok && t < T; ++t) {
         const int st = t & 1, u = t >> 1, su = t % NS;
-        if (!mbar_wait(bar(B_PR + st), u & 1, abort_flag)) break;
-        if (!mbar_wait(bar(B_VF + su), (t / NS) & 1, abort_flag)) break;
+        if (!mbar_wait(bar(L::B_PR + st), u & 1, abort_flag)) break;
+        if (!mbar_wait(bar(L::B_VF + su), (t / NS) & 1, abort_flag)) break;
         tc_fence_after();
         const uint32_t va = sb + kTile * (2 + 2 * su);
         const uint32_t pa = tbase + (uint32_t)st * TB;
         const uint32_t od = tbase + kColO + (uint32_t)st * TD;
 #pragma unroll
-        for (int k = 0; k < TB / 16; ++k)
-          mma_ts(od, pa + k * 8, desc_sw128(va + k * 16 * 128, kHalfTile, 1024), idO, (u > 0 || k > 0));
-        mma_commit(bar(B_KE + su));
-        mma_commit(bar(B_OD + st));
+        for (int k = 0; k < TB / kK; ++k) {
+          // K step k: kK keys = kK rows of 128 bytes further into V; 8 TMEM columns of P
+          const uint64_t b = desc_sw128(va + k * kK * 128, kSpan, 1024);
+          if (F8) mma_ts_f8(od, pa + k * 8, b, idO, (u > 0 || k > 0));
+          else mma_ts(od, pa + k * 8, b, idO, (u > 0 || k > 0));
+        }
+        mma_commit(bar(L::B_KE + su));
+        mma_commit(bar(L::B_OD + st));
         if (t + 2 < T && !issue_s(t + 2)) break;
       }
       // every MMA issued above has completed before TMEM is released
-      mma_commit(bar(B_FIN));
-      wait_bounded(bar(B_FIN), 0);
+      mma_commit(bar(L::B_FIN));
+      wait_bounded(bar(L::B_FIN), 0);
     }
   } else if (warp >= 8) {
     regs_dec<kProducerRegs>();                  // idle warps of the producer warpgroup
@@ -236,11 +313,20 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const uint32_t s_col = (uint32_t)st * TB;
     const uint32_t o_col = kColO + (uint32_t)st * TD;
     const int U = T > st ? (T - st + 1) / 2 : 0;   // tiles of this stream
+    // e4m3: the head's largest V scale and this query block's Q scale
+    float vmax = 1.f, qs = 1.f;
+    if (F8) {
+      const int ntiles = (nb + TB - 1) / TB;
+      vmax = f8.v_max[bh];
+      if (ZO)
+        for (int c = 0; c < ntiles; ++c) vmax = fmaxf(vmax, f8.vbar[(size_t)bh * ntiles + c]);
+      qs = f8.q[(size_t)bh * nb + i];
+    }
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     for (int u = 0; u < U; ++u) {
       const int t = 2 * u + st;
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_SF + st), u & 1, abort_flag))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_SF + st), u & 1, abort_flag))) {
         ok = false;
         break;
       }
@@ -252,6 +338,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       tmem_wait_ld();
       const bool centroid = t >= topk;
       float bias = 0.f;
+      float tscale = scale2, pscale = 1.f;
+      if (F8) {
+        const int ntiles = (nb + TB - 1) / TB;
+        if (centroid) {
+          const int c = t - topk;
+          tscale = scale2 * qs * f8.kbar[(size_t)bh * ntiles + c];
+          pscale = 448.0f * f8.vbar[(size_t)bh * ntiles + c] / vmax;
+        } else {
+          const int j = sel[t];
+          tscale = scale2 * qs * f8.k[(size_t)bh * nb + j];
+          pscale = 448.0f * f8.v[(size_t)bh * nb + j] / vmax;
+        }
+      }
       if (centroid) {
         // validity of the 128 pseudo-keys: inside the head and not selected
         const int jb = (t - topk) * TB;
@@ -275,9 +374,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         mx8[n & 7] = fmax3(mx8[n & 7], __uint_as_float(v[2 * n]), __uint_as_float(v[2 * n + 1]));
       const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
                              fmaxf(mx8[6], mx8[7]));
-      const float m_tile = mx == -INFINITY ? -INFINITY : fmaf(mx, scale2, bias);
+      const float m_tile = mx == -INFINITY ? -INFINITY : fmaf(mx, tscale, bias);
       const float m_new = fmaxf(m_used, m_tile);
-      const bool need = m_new > m_used + kLazyRescale;
+      const bool need = m_new > m_used + Fmt<F8>::kLazy;
       float factor = 1.f;
       if (need) {
         factor = fast_exp2(m_used - m_new);
@@ -288,22 +387,34 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       float sm8[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) sm8[k] = 0.f;
-      const float sc2 = live ? scale2 : 0.f, ng = live ? neg : -INFINITY;   // dead row: p = 0
+      const float sc2 = live ? tscale : 0.f, ng = live ? neg : -INFINITY;   // dead row: p = 0
+      if (F8) {
 #pragma unroll
-      for (int n = 0; n < TB / 2; ++n) {
-        float a0, a1;
-        ffma2(a0, a1, __uint_as_float(v[2 * n]), __uint_as_float(v[2 * n + 1]), sc2, sc2, ng, ng);
-        const float p0 = fast_exp2(a0), p1 = fast_exp2(a1);
-        fadd2(sm8[2 * (n & 3)], sm8[2 * (n & 3) + 1], p0, p1);
-        v[n] = pack_bf16(p0, p1);
+        for (int n = 0; n < TB / 4; ++n) {
+          float a0, a1, a2, a3;
+          ffma2(a0, a1, __uint_as_float(v[4 * n]), __uint_as_float(v[4 * n + 1]), sc2, sc2, ng, ng);
+          ffma2(a2, a3, __uint_as_float(v[4 * n + 2]), __uint_as_float(v[4 * n + 3]), sc2, sc2, ng, ng);
+          const float p0 = fast_exp2(a0), p1 = fast_exp2(a1), p2 = fast_exp2(a2), p3 = fast_exp2(a3);
+          fadd2(sm8[2 * (n & 3)], sm8[2 * (n & 3) + 1], p0 + p2, p1 + p3);
+          v[n] = pack_e4m3x4(p0 * pscale, p1 * pscale, p2 * pscale, p3 * pscale);
+        }
+      } else {
+#pragma unroll
+        for (int n = 0; n < TB / 2; ++n) {
+          float a0, a1;
+          ffma2(a0, a1, __uint_as_float(v[2 * n]), __uint_as_float(v[2 * n + 1]), sc2, sc2, ng, ng);
+          const float p0 = fast_exp2(a0), p1 = fast_exp2(a1);
+          fadd2(sm8[2 * (n & 3)], sm8[2 * (n & 3) + 1], p0, p1);
+          v[n] = pack_bf16(p0, p1);
+        }
       }
       const float sum = ((sm8[0] + sm8[1]) + (sm8[2] + sm8[3])) + ((sm8[4] + sm8[5]) + (sm8[6] + sm8[7]));
       l = l * factor + sum;
       tmem_st32(lrow + s_col, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-      tmem_st32(lrow + s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+      if (!F8) tmem_st32(lrow + s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
       tmem_wait_st();
       if (u >= 1) {
-        if (!__all_sync(0xffffffffu, mbar_wait(bar(B_OD + st), (u - 1) & 1, abort_flag))) {
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_OD + st), (u - 1) & 1, abort_flag))) {
           ok = false;
           break;
         }
@@ -322,9 +433,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
       }
       tc_fence_before();
-      mbar_arrive(bar(B_PR + st));
+      mbar_arrive(bar(L::B_PR + st));
     }
-    if (ok && U > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_OD + st), (U - 1) & 1, abort_flag));
+    if (ok && U > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_OD + st), (U - 1) & 1, abort_flag));
     // both groups past their last PV: every MMA that reads Q has completed,
     // so the Q tile's shared memory can carry the (max, sum) exchange
     named_bar_softmax();
@@ -337,8 +448,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const float M = fmaxf(m0, m1);
     const float f0 = (U0 > 0 && m0 != -INFINITY) ? fast_exp2(m0 - M) : 0.f;
     const float f1 = (U1 > 0 && m1 != -INFINITY) ? fast_exp2(m1 - M) : 0.f;
-    const float L = l0 * f0 + l1 * f1;
-    const float inv = L > 0.f ? 1.0f / L : 0.f;
+    const float L_ = l0 * f0 + l1 * f1;
+    // e4m3: O accumulated Σ P σ_V V̂ · 448 / σ_Vmax
+    const float inv = L_ > 0.f ? (F8 ? vmax / 448.0f : 1.0f) / L_ : 0.f;
     ok = __all_sync(0xffffffffu, ok) && !*abort_flag;
     if (ok) {
       tc_fence_after();
@@ -406,24 +518,37 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-size_t tc_smem_bytes(int nb) {
-  return 1024 + kMaskOff + 4 * (size_t)((nb + 31) / 32 + 4);
-}
-
-}  // namespace
-
-bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows, uint64_t outer,
-                       uint32_t box_cols, uint32_t box_rows) {
+// 3-D tensor map [outer][rows][cols] (cols innermost) with a box of
+// {128 bytes, 128 rows, 1} and 128-byte swizzle; elem = 2 (bf16) or 1 (e4m3).
+bool make_tmap_3d(CUtensorMap* map, const void* base, int elem, uint64_t cols, uint64_t rows, uint64_t outer) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {cols, rows, outer};
-  cuuint64_t strides[2] = {cols * 2, cols * rows * 2};
-  cuuint32_t box[3] = {box_cols, box_rows, 1};
+  cuuint64_t strides[2] = {cols * elem, cols * rows * elem};
+  cuuint32_t box[3] = {128u / (cuuint32_t)elem, (cuuint32_t)TB, 1};
   cuuint32_t es[3] = {1, 1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+  return fn(map, elem == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 3,
+            const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
+template <bool F8>
+sa_status launch_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mkb,
+                    const CUtensorMap& mvb, bool zo, const sa_shape& s, const int32_t* block_idx, int topk,
+                    float scale, const F8Scales& f8, void* O, cudaStream_t stream) {
+  const int nb = s.N / TB;
+  const size_t smem = Layout<F8>::smem_bytes(nb);
+  auto kern = zo ? attn_tc_kernel<true, F8> : attn_tc_kernel<false, F8>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return launch_status("cudaFuncSetAttribute(attn_tc_kernel)");
+  dim3 grid(nb, (unsigned)((uint64_t)s.B * s.H));
+  kern<<<grid, kTcThreads, smem, stream>>>(mq, mk, mv, mkb, mvb, block_idx, nb, topk, scale * kLog2e, f8,
+                                           static_cast<__nv_bfloat16*>(O), s.N);
+  return launch_status("attn_tc_kernel");
+}
+
+}  // namespace
 
 bool attn_tc_supports(sa_dtype dtype, const sa_shape& s, sa_tail_mode tail) {
   return dtype == SA_BF16 && s.block == TB && s.d == TD &&
@@ -437,29 +562,61 @@ sa_status attn_tc(const void* Q, const void* K, const void* V, const sa_shape& s
   const int nb = s.N / TB;
   const uint64_t BH = (uint64_t)s.B * s.H;
   CUtensorMap mq, mk, mv, mkb, mvb;
-  if (!make_tmap_bf16_3d(&mq, Q, TD, s.N, BH, 64, TB) || !make_tmap_bf16_3d(&mk, K, TD, s.N, BH, 64, TB) ||
-      !make_tmap_bf16_3d(&mv, V, TD, s.N, BH, 64, TB))
+  if (!make_tmap_3d(&mq, Q, 2, TD, s.N, BH) || !make_tmap_3d(&mk, K, 2, TD, s.N, BH) ||
+      !make_tmap_3d(&mv, V, 2, TD, s.N, BH))
     return fail(SA_ERR_CUDA, "sa_sparse_attn_fwd: cuTensorMapEncodeTiled failed for Q/K/V");
   const bool zo = tail == SA_TAIL_ZERO_ORDER;
   if (zo) {
-    if (!make_tmap_bf16_3d(&mkb, st.kmean_bf16, TD, nb, BH, 64, TB) ||
-        !make_tmap_bf16_3d(&mvb, st.vmean_bf16, TD, nb, BH, 64, TB))
+    if (!make_tmap_3d(&mkb, st.kmean_bf16, 2, TD, nb, BH) || !make_tmap_3d(&mvb, st.vmean_bf16, 2, TD, nb, BH))
       return fail(SA_ERR_CUDA, "sa_sparse_attn_fwd: cuTensorMapEncodeTiled failed for the block centroids");
   } else {
     mkb = mk;
     mvb = mv;
   }
-  const size_t smem = tc_smem_bytes(nb);
-  auto kern = zo ? attn_tc_kernel<true> : attn_tc_kernel<false>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-    return launch_status("cudaFuncSetAttribute(attn_tc_kernel)");
-  dim3 grid(nb, (unsigned)BH);
-  kern<<<grid, kTcThreads, smem, stream>>>(mq, mk, mv, mkb, mvb, block_idx, nb, topk, scale * kLog2e,
-                                           static_cast<__nv_bfloat16*>(O), s.N);
-  return launch_status("attn_tc_kernel");
+  return launch_tc<false>(mq, mk, mv, mkb, mvb, zo, s, block_idx, topk, scale, F8Scales{}, O, stream);
 }
 
 }  // namespace sa
+
+extern "C" sa_status sa_sparse_attn_fwd_fp8(const sa_fp8_operands* ops, sa_shape shape,
+                                            const int32_t* block_idx, int32_t topk, sa_tail_mode tail,
+                                            float scale, void* O, void* stream) {
+  using namespace sa;
+  sa_status r = check_shape(shape, "sa_sparse_attn_fwd_fp8");
+  if (r != SA_OK) return r;
+  if (shape.d != TD || shape.block != TB)
+    return fail(SA_ERR_UNSUPPORTED, "sa_sparse_attn_fwd_fp8: d and block must be 128");
+  if (tail != SA_TAIL_DROP && tail != SA_TAIL_ZERO_ORDER)
+    return fail(SA_ERR_UNSUPPORTED, "sa_sparse_attn_fwd_fp8: tail must be SA_TAIL_DROP or SA_TAIL_ZERO_ORDER");
+  if (shape.B == 0 || shape.H == 0 || shape.N == 0) return SA_OK;
+  const int nb = shape.N / TB;
+  if (!ops || !ops->q || !ops->k || !ops->v || !ops->q_scale || !ops->k_scale || !ops->v_scale ||
+      !ops->v_scale_max || !O)
+    return fail(SA_ERR_INVALID_ARG, "sa_sparse_attn_fwd_fp8: codes, scales, v_scale_max and O are required");
+  const bool zo = tail == SA_TAIL_ZERO_ORDER;
+  if (zo && (!ops->kbar || !ops->vbar || !ops->kbar_scale || !ops->vbar_scale))
+    return fail(SA_ERR_INVALID_ARG, "sa_sparse_attn_fwd_fp8: SA_TAIL_ZERO_ORDER needs the centroid codes and scales");
+  if (topk < 0 || topk > nb) return fail(SA_ERR_INVALID_ARG, "sa_sparse_attn_fwd_fp8: topk must be in [0, N/block]");
+  if (topk > 0 && !block_idx) return fail(SA_ERR_INVALID_ARG, "sa_sparse_attn_fwd_fp8: block_idx is required");
+  if (nb > kMaxAttnBlocks) return fail(SA_ERR_UNSUPPORTED, "sa_sparse_attn_fwd_fp8: at most 4096 blocks per head");
+  const void* ptrs[] = {ops->q, ops->k, ops->v, ops->kbar, ops->vbar, O, block_idx};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(SA_ERR_ALIGNMENT, "sa_sparse_attn_fwd_fp8: pointers must be 16-byte aligned");
+  const uint64_t BH = (uint64_t)shape.B * shape.H;
+  CUtensorMap mq, mk, mv, mkb, mvb;
+  if (!make_tmap_3d(&mq, ops->q, 1, TD, shape.N, BH) || !make_tmap_3d(&mk, ops->k, 1, TD, shape.N, BH) ||
+      !make_tmap_3d(&mv, ops->v, 1, TD, shape.N, BH))
+    return fail(SA_ERR_CUDA, "sa_sparse_attn_fwd_fp8: cuTensorMapEncodeTiled failed for Q/K/V");
+  if (zo) {
+    if (!make_tmap_3d(&mkb, ops->kbar, 1, TD, nb, BH) || !make_tmap_3d(&mvb, ops->vbar, 1, TD, nb, BH))
+      return fail(SA_ERR_CUDA, "sa_sparse_attn_fwd_fp8: cuTensorMapEncodeTiled failed for the centroids");
+  } else {
+    mkb = mk;
+    mvb = mv;
+  }
+  F8Scales f8{ops->q_scale, ops->k_scale, ops->v_scale, ops->v_scale_max, ops->kbar_scale, ops->vbar_scale};
+  return launch_tc<true>(mq, mk, mv, mkb, mvb, zo, shape, block_idx, topk, scale, f8, O, as_stream(stream));
+}
 
 extern "C" sa_status sa_device_error(uint32_t* code) {
   using namespace sa;

@@ -115,3 +115,33 @@ class DecodeStep:
 
     def launches(self) -> int:
         return 4
+
+
+class Fp8PrefillStep:
+    """One step of the e4m3 sparse branch: block statistics (bf16 inputs) ->
+    router -> per-block e4m3 quantisation of Q, K, V and of the centroid tiles
+    -> e4m3 sparse attention."""
+
+    def __init__(self, w: Workload, inputs: dict):
+        self.w = w
+        self.inp = inputs
+        Q = inputs["Q"]
+        self.buf = alloc_prefill(w, Q)
+        B, H, N, d = Q.shape
+        self.shape = (B, H, N, d, w.block)
+        self.ops = None
+
+    def __call__(self, stream=None):
+        w, inp, buf = self.w, self.inp, self.buf
+        bd._check("sa_block_pool", bd.load().sa_block_pool(
+            inp["Q"].data_ptr(), inp["K"].data_ptr(), inp["V"].data_ptr(), bd.SA_BF16, bd.Shape(*self.shape),
+            ctypes.byref(bd._stats_struct(buf.stats)), bd._stream(stream)))
+        bd._check("sa_route", bd.load().sa_route(
+            ctypes.byref(bd._stats_struct(buf.stats)), bd.Shape(*self.shape), bd.ROUTE[w.route], None, None,
+            float(w.scale), int(w.k), buf.block_idx.data_ptr(), None, bd._stream(stream)))
+        self.ops = bd.fp8_operands(inp["Q"], inp["K"], inp["V"], buf.stats, stream=stream)
+        return bd.sparse_attn_fwd_fp8(self.ops, self.shape, buf.block_idx, w.tail, w.scale, out=buf.out,
+                                      stream=stream)
+
+    def launches(self) -> int:
+        return 2 + 5 + 1

@@ -141,6 +141,42 @@ sa_status sa_sparse_attn_fwd(const void* Q, const void* K, const void* V, sa_dty
                              const sa_block_stats* stats, float scale, void* O,
                              void* stream);
 
+/* Per-block e4m3 quantisation [SLA2 §2C, low-precision sparse branch]:
+ * X: bf16 [BH][N][d] (BH = batch x heads); codes: uint8 [BH][N][d] e4m3fn bit
+ * patterns; scales: float [BH][ceil(N/block)] with σ = absmax/448 of each block
+ * of `block` rows (1 for an all-zero block; the last block may be ragged);
+ * scale_max: float [BH] (max of the head's σ) or NULL.  code = e4m3(x / σ)
+ * with the correctly rounded fp32 division, round-to-nearest-even and
+ * saturation to ±448.  d and block in {64, 128}.
+ * Errors: SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED, SA_ERR_ALIGNMENT. */
+sa_status sa_quantize_e4m3(const void* X, int64_t BH, int32_t N, int32_t d, int32_t block, uint8_t* codes,
+                           float* scales, float* scale_max, void* stream);
+
+/* e4m3 operands of sa_sparse_attn_fwd_fp8 (all device pointers; block 128). */
+typedef struct {
+  const uint8_t* q;            /* [B,H,N,d] codes of Q                          */
+  const uint8_t* k;            /* [B,H,N,d] codes of K                          */
+  const uint8_t* v;            /* [B,H,N,d] codes of V                          */
+  const float* q_scale;        /* [B,H,N/128]                                   */
+  const float* k_scale;        /* [B,H,N/128]                                   */
+  const float* v_scale;        /* [B,H,N/128]                                   */
+  const float* v_scale_max;    /* [B,H] max of v_scale over the head            */
+  const uint8_t* kbar;         /* [B,H,nb,d] codes of kmean_bf16 (ZERO_ORDER)   */
+  const uint8_t* vbar;         /* [B,H,nb,d] codes of vmean_bf16 (ZERO_ORDER)   */
+  const float* kbar_scale;     /* [B,H,ceil(nb/128)] scales of 128-centroid tiles */
+  const float* vbar_scale;     /* [B,H,ceil(nb/128)]                            */
+} sa_fp8_operands;
+
+/* Sparse prefill with the SLA2 §2C low-precision sparse branch: the same
+ * DROP / ZERO_ORDER attention as sa_sparse_attn_fwd with e4m3 Q, K, V (and
+ * centroid tiles, produced by sa_quantize_e4m3 from kmean_bf16 / vmean_bf16),
+ * logits σ_Q σ_K (Q̂·K̂ᵀ), P quantised to e4m3 on the tensor cores, fp32
+ * accumulation, row sums from the unquantised P.  O: bf16 [B,H,N,d].
+ * d = block = 128.
+ * Errors: SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED, SA_ERR_ALIGNMENT, SA_ERR_CUDA. */
+sa_status sa_sparse_attn_fwd_fp8(const sa_fp8_operands* ops, sa_shape shape, const int32_t* block_idx,
+                                 int32_t topk, sa_tail_mode tail, float scale, void* O, void* stream);
+
 /* Bytes of workspace sa_decode_fwd needs for this shape and topk (0 on bad
  * arguments). */
 size_t sa_decode_workspace_size(sa_decode_shape shape, int32_t topk);

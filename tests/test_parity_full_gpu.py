@@ -10,7 +10,7 @@ import torch
 import oracle
 from block_sparse_approximate_b200 import binding as bd
 from block_sparse_approximate_b200 import workloads as wl
-from block_sparse_approximate_b200.pipeline import DecodeStep, PrefillStep
+from block_sparse_approximate_b200.pipeline import DecodeStep, Fp8PrefillStep, PrefillStep
 from tests._parity import (BF16_TOL, assert_no_device_error, assert_tol, check_topk_exact, np64,
                            selection_agreement)
 
@@ -71,3 +71,22 @@ def test_decode_full_size_sampled(lib):
                                                    block_idx=step.idx[b:b + 1, kh:kh + 1].cpu().numpy())
         selection_agreement(np64(step.scores[b, kh]), ref_sc[0, 0], w.k)  # asserts on clear gaps
         assert_tol(np64(o[b, kh * g:(kh + 1) * g]), ref_o[0], BF16_TOL, f"decode b={b} g={kh}")
+
+
+def test_fp8_full_size_sampled(lib):
+    # e4m3 sparse branch against the float64 oracle on the unquantised inputs
+    w = wl.WORKLOADS["fp8"]
+    inp = wl.prefill_inputs(w, DEV)
+    step = Fp8PrefillStep(w, inp)
+    O = step()
+    torch.cuda.synchronize()
+    assert_no_device_error()
+    picks = _sample_blocks(w.H, w.nb, 12, 3)
+    heads = sorted({h for _, h, _ in picks})
+    hmap = {h: r for r, h in enumerate(heads)}
+    idx = step.buf.block_idx[:, heads].cpu().numpy()
+    sub = {n: inp[n][:, heads].cpu().float().numpy() for n in ("Q", "K", "V")}
+    ref = oracle.sparse_attention(sub["Q"], sub["K"], sub["V"], idx, w.block, w.tail, w.scale,
+                                  qblocks=[(b, hmap[h], i) for b, h, i in picks])
+    got = np.stack([np64(O[b, h, i * w.block:(i + 1) * w.block]) for b, h, i in picks])
+    assert_tol(got, ref, (6e-2, 6e-3), "fp8 full size")

@@ -194,3 +194,60 @@ def test_decode(lib, tail, B, Hq, Hkv, N, d, block, k):
                                           block_idx=idx.cpu().numpy())
     assert_tol(np64(o), ref_o, BF16_TOL, f"decode {tail}")
     del w
+
+
+# --------------------------------------------------------------------------
+# FP8 e4m3 sparse branch
+# --------------------------------------------------------------------------
+
+FP8_TOL = (6e-2, 6e-3)
+
+
+def _e4m3_values(codes: torch.Tensor) -> np.ndarray:
+    return codes.cpu().view(torch.float8_e4m3fn).to(torch.float64).numpy()
+
+
+@pytest.mark.parametrize("N,block", [(4096, 128), (4736, 128), (1000, 128), (2048, 64)])
+def test_quantize_e4m3_bit_exact(lib, N, block):
+    g = torch.Generator(device=DEV)
+    g.manual_seed(N)
+    X = (torch.randn(2, 3, N, 128, generator=g, device=DEV) * 3).to(torch.bfloat16)
+    X[0, 1, :block] = 0          # an all-zero block gets scale 1
+    codes, scales, smax = bd.quantize_e4m3(X, block, want_max=True)
+    torch.cuda.synchronize()
+    Xn = np64(X)
+    nblk = (N + block - 1) // block
+    pad = nblk * block - N
+    Xp = np.concatenate([Xn, np.zeros((2, 3, pad, 128))], axis=2) if pad else Xn
+    deq, ref_codes, ref_sigma = oracle.quantise_blocks_e4m3(Xp, block)
+    np.testing.assert_array_equal(scales.cpu().numpy(), ref_sigma)
+    np.testing.assert_array_equal(_e4m3_values(codes), ref_codes[:, :, :N])
+    np.testing.assert_array_equal(smax.cpu().numpy(), ref_sigma.max(axis=2))
+
+
+def _fp8_case(Q, K, V, k, tail):
+    B, H, N, d = Q.shape
+    s = 1 / math.sqrt(d)
+    st = bd.block_pool(Q, K, V, 128, centroids_bf16=True)
+    idx, sc = bd.route(st, (B, H, N, d, 128), "dot", k, want_scores=True)
+    ops = bd.fp8_operands(Q, K, V, st)
+    O = bd.sparse_attn_fwd_fp8(ops, (B, H, N, d, 128), idx, tail, s)
+    torch.cuda.synchronize()
+    assert_no_device_error()
+    ref = oracle.sparse_attention(np64(Q), np64(K), np64(V), idx.cpu().numpy(), 128, tail, s)
+    return assert_tol(np64(O), ref, FP8_TOL, f"fp8 {tail} k={k}")
+
+
+@pytest.mark.parametrize("tail", ["zero_order", "drop"])
+@pytest.mark.parametrize("k", [0, 1, 4, 32])
+def test_fp8_video_small(lib, tail, k):
+    w = wl.WORKLOADS["fp8"]
+    inp = wl.prefill_inputs(w, DEV, H=2, N=4096)
+    _fp8_case(inp["Q"], inp["K"], inp["V"], k, tail)
+
+
+@pytest.mark.parametrize("tail", ["zero_order", "drop"])
+@pytest.mark.parametrize("nb,k", [(37, 5), (133, 13)])
+def test_fp8_ragged(lib, tail, nb, k):
+    Q, K, V = _gauss(2, 2, nb * 128, 128, torch.bfloat16, 70 + nb)
+    _fp8_case(Q, K, V, k, tail)
