@@ -30,4 +30,5 @@ from .sparse_attention import (  # noqa: F401
     decode_attention,
     e4m3_round,
     quantise_blocks_e4m3,
+    fp8_attention,
 )

@@ -41,6 +41,8 @@ Pins (the tests under ``tests/test_oracle_*.py``):
   e4m3_round          every one of the 256 e4m3 codes and random values
                       against torch.float8_e4m3fn
   quantise_blocks_e4m3  bounds of the format (|error| <= half an ulp)
+  fp8_attention       on inputs already e4m3-exact per block the quantised
+                      forward equals sparse_attention (drop tail)
 """
 
 from __future__ import annotations
@@ -203,7 +205,8 @@ def _block_tokens(blocks: Sequence[int], block: int) -> np.ndarray:
 
 
 def _attend_rows(q, K, V, sel: Sequence[int], nb: int, block: int, tail: str,
-                 scale: float, alpha_h=None, eps: float = EPS_LINEAR) -> np.ndarray:
+                 scale: float, alpha_h=None, eps: float = EPS_LINEAR,
+                 centroids=None) -> np.ndarray:
     """Output rows o_t for query rows q [R, d] against one head's K, V [N, d].
 
     PISA "Algoritmo Central":  o_t = N_t / D_t with
@@ -222,8 +225,12 @@ def _attend_rows(q, K, V, sel: Sequence[int], nb: int, block: int, tail: str,
     R, d = q.shape
     a = scale * (q @ Ks.T)                      # exact logits [R, |S|B]
     if tail == "zero_order":
-        kbar = K.reshape(nb, block, d).mean(axis=1)[uns]      # [|U|, d]
-        vsum = V.reshape(nb, block, d).sum(axis=1)[uns]       # [|U|, d]
+        if centroids is None:
+            kbar = K.reshape(nb, block, d).mean(axis=1)[uns]      # [|U|, d]
+            vsum = V.reshape(nb, block, d).sum(axis=1)[uns]       # [|U|, d]
+        else:   # given block centroids k̄_j and value means v̄_j = vsum_j / B
+            kbar = centroids[0][uns]
+            vsum = block * centroids[1][uns]
         c = scale * (q @ kbar.T)                               # [R, |U|]
         m = np.full(R, -np.inf)
         if a.shape[1]:
@@ -385,21 +392,65 @@ def quantise_blocks_e4m3(X, block: int = 128):
     """Per-(batch, head, token block) absmax-scaled e4m3 quantisation.
 
     SLA2 §2C quantises the sparse branch to 8 bits; the scale layout is a
-    reading: one float32 scale per block of ``block`` tokens,
-    σ = absmax / 448 (σ = 1 for an all-zero block), codes = e4m3(x / σ) with the
-    division done in float32.  Returns (dequantised float64 X̂, codes as float64,
+    reading: one float32 scale per block of ``block`` tokens (a ragged last
+    block has its own scale), σ = absmax / 448 (σ = 1 for an all-zero block),
+    codes = e4m3(x / σ) with the division done in float32.  Returns (dequantised float64 X̂, codes as float64,
     σ [B,H,N/block] float32).
     """
     X32 = np.asarray(X, dtype=np.float32)
     Bsz, H, N, d = X32.shape
-    nb = N // block
+    nb = -(-N // block)
+    if nb * block != N:   # a ragged last block: zero rows do not change its absmax
+        X32 = np.concatenate([X32, np.zeros((Bsz, H, nb * block - N, d), np.float32)], axis=2)
     Xb = X32.reshape(Bsz, H, nb, block, d)
     amax = np.abs(Xb).max(axis=(3, 4))
     sigma = np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
     scaled = (Xb / sigma[:, :, :, None, None]).astype(np.float32)
     codes = e4m3_round(scaled)
     deq = codes * sigma[:, :, :, None, None].astype(np.float64)
-    return deq.reshape(Bsz, H, N, d), codes.reshape(Bsz, H, N, d), sigma
+    return (deq.reshape(Bsz, H, nb * block, d)[:, :, :N], codes.reshape(Bsz, H, nb * block, d)[:, :, :N],
+            sigma)
+
+
+def _bf16(x) -> np.ndarray:
+    """Round to bfloat16 (nearest, ties to even) and back to float64."""
+    import torch
+    return torch.as_tensor(np.asarray(x, dtype=np.float32)).to(torch.bfloat16).to(torch.float64).numpy()
+
+
+def fp8_attention(Q, K, V, block_idx, block: int, tail: str, scale: float, *,
+                  qblocks: Optional[Iterable[Tuple[int, int, int]]] = None):
+    """The e4m3 quantised forward of the sparse branch, float64 (P unquantised).
+
+    SLA2 §2C runs the sparse branch in 8 bits; reading: Q, K, V are replaced by
+    their per-(batch, head, block) e4m3 values (``quantise_blocks_e4m3``), and
+    the zero-order tail uses the block centroids k̄_j and value means vsum_j/B
+    of the unquantised inputs, stored in bfloat16 and quantised to e4m3 with one
+    scale per group of 128 blocks.  The attention itself is PISA's N_t / D_t in
+    float64.  Same return convention as ``sparse_attention``.
+    """
+    Qd = quantise_blocks_e4m3(Q, block)[0]
+    Kd = quantise_blocks_e4m3(K, block)[0]
+    Vd = quantise_blocks_e4m3(V, block)[0]
+    Bsz, H, N, d = np.asarray(K).shape
+    nb = N // block
+    idx = np.asarray(block_idx)
+    cent = None
+    if tail == "zero_order":
+        K64, V64 = _f64(K), _f64(V)
+        kb = _bf16(K64.reshape(Bsz, H, nb, block, d).mean(axis=3))
+        vb = _bf16(V64.reshape(Bsz, H, nb, block, d).sum(axis=3) / block)
+        cent = (quantise_blocks_e4m3(kb, 128)[0], quantise_blocks_e4m3(vb, 128)[0])
+    todo = list(qblocks) if qblocks is not None else [
+        (b, h, i) for b in range(Bsz) for h in range(H) for i in range(N // block)]
+    out = np.empty((len(todo), block, d))
+    for r, (b, h, i) in enumerate(todo):
+        c = None if cent is None else (cent[0][b, h], cent[1][b, h])
+        out[r] = _attend_rows(Qd[b, h, i * block:(i + 1) * block], Kd[b, h], Vd[b, h], idx[b, h, i], nb,
+                              block, tail, scale, centroids=c)
+    if qblocks is not None:
+        return out
+    return out.reshape(Bsz, H, N // block, block, d).reshape(Bsz, H, N, d)
 
 
 def dense_equivalent_flops(Bsz: int, H: int, N: int, d: int) -> float:
@@ -410,6 +461,6 @@ def dense_equivalent_flops(Bsz: int, H: int, N: int, d: int) -> float:
 __all__ = [
     "block_pool", "route_scores", "decode_route_scores", "k_from_percent",
     "topk_from_scores", "sparse_attention", "decode_attention", "e4m3_round",
-    "quantise_blocks_e4m3", "dense_equivalent_flops", "EPS_LINEAR", "E4M3_MAX",
+    "quantise_blocks_e4m3", "fp8_attention", "dense_equivalent_flops", "EPS_LINEAR", "E4M3_MAX",
 ]
 

@@ -436,3 +436,30 @@ def test_quantise_blocks_error_bound():
     ulp = 2.0 ** (e - 3)
     assert np.all(np.abs(codes - xs) <= ulp / 2 + 1e-6 * ulp)
     assert np.all(np.abs(deq - X) <= (ulp / 2 + 1e-6 * ulp) * sigma.max())
+
+
+def test_fp8_attention_is_exact_on_e4m3_representable_blocks():
+    # build per-block inputs whose absmax is 448 * sigma and whose values are
+    # e4m3 values times sigma: quantisation is then lossless, so the quantised
+    # forward equals the float64 attention (drop tail has no centroids)
+    rng = np.random.default_rng(70)
+    Bsz, H, N, d, blk = 1, 2, 256, 16, 128
+    vals = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    vals = vals[np.isfinite(vals) & (np.abs(vals) <= 64)]
+    def make():
+        X = rng.choice(vals, size=(Bsz, H, N, d))
+        X[:, :, ::blk, 0] = 448.0          # pins each block's absmax to 448
+        return X * 2.0 ** -10              # a power-of-two scale keeps x / sigma exact
+    Q, K, V = make(), make(), make()
+    idx = _rand_idx(np.random.default_rng(71), Bsz, H, N // blk, N // blk, 1)
+    np.testing.assert_array_equal(oracle.quantise_blocks_e4m3(Q, blk)[0], Q)
+    a = oracle.fp8_attention(Q, K, V, idx, blk, "drop", 0.3)
+    b = oracle.sparse_attention(Q, K, V, idx, blk, "drop", 0.3)
+    np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-14)
+
+
+def test_quantise_blocks_ragged_last_block():
+    X = _rand((1, 1, 300, 8), 72)
+    deq, codes, sigma = oracle.quantise_blocks_e4m3(X, 128)
+    assert deq.shape == X.shape and sigma.shape == (1, 1, 3)
+    np.testing.assert_allclose(sigma[0, 0, 2], np.float32(np.abs(X[0, 0, 256:]).max()) / np.float32(448.0))

@@ -74,7 +74,9 @@ def test_decode_full_size_sampled(lib):
 
 
 def test_fp8_full_size_sampled(lib):
-    # e4m3 sparse branch against the float64 oracle on the unquantised inputs
+    # e4m3 sparse branch against the oracle's quantised forward (the pin, at
+    # the FP8 tolerance); its distance to the unquantised float64 oracle is
+    # the format's own error on these inputs and is only bounded loosely here
     w = wl.WORKLOADS["fp8"]
     inp = wl.prefill_inputs(w, DEV)
     step = Fp8PrefillStep(w, inp)
@@ -86,7 +88,11 @@ def test_fp8_full_size_sampled(lib):
     hmap = {h: r for r, h in enumerate(heads)}
     idx = step.buf.block_idx[:, heads].cpu().numpy()
     sub = {n: inp[n][:, heads].cpu().float().numpy() for n in ("Q", "K", "V")}
-    ref = oracle.sparse_attention(sub["Q"], sub["K"], sub["V"], idx, w.block, w.tail, w.scale,
-                                  qblocks=[(b, hmap[h], i) for b, h, i in picks])
+    qb = [(b, hmap[h], i) for b, h, i in picks]
     got = np.stack([np64(O[b, h, i * w.block:(i + 1) * w.block]) for b, h, i in picks])
-    assert_tol(got, ref, (6e-2, 6e-3), "fp8 full size")
+    emu = oracle.fp8_attention(sub["Q"], sub["K"], sub["V"], idx, w.block, w.tail, w.scale, qblocks=qb)
+    assert_tol(got, emu, (6e-2, 6e-3), "fp8 full size vs quantised forward")
+    ref = oracle.sparse_attention(sub["Q"], sub["K"], sub["V"], idx, w.block, w.tail, w.scale, qblocks=qb)
+    err = np.abs(got - ref)
+    print(f"fp8 vs unquantised float64 oracle: max-abs {err.max():.3e} mean-abs {err.mean():.3e}")
+    assert err.mean() < 4e-2 and err.max() < 0.8

@@ -226,6 +226,9 @@ def test_quantize_e4m3_bit_exact(lib, N, block):
 
 
 def _fp8_case(Q, K, V, k, tail):
+    """The e4m3 kernel against the oracle's quantised forward (SLA2 §2C: Q, K,
+    V and the centroid tiles quantised per block, float64 attention); the only
+    kernel-side difference left is the e4m3 rounding of P and fp32 sums."""
     B, H, N, d = Q.shape
     s = 1 / math.sqrt(d)
     st = bd.block_pool(Q, K, V, 128, centroids_bf16=True)
@@ -234,7 +237,7 @@ def _fp8_case(Q, K, V, k, tail):
     O = bd.sparse_attn_fwd_fp8(ops, (B, H, N, d, 128), idx, tail, s)
     torch.cuda.synchronize()
     assert_no_device_error()
-    ref = oracle.sparse_attention(np64(Q), np64(K), np64(V), idx.cpu().numpy(), 128, tail, s)
+    ref = oracle.fp8_attention(np64(Q), np64(K), np64(V), idx.cpu().numpy(), 128, tail, s)
     return assert_tol(np64(O), ref, FP8_TOL, f"fp8 {tail} k={k}")
 
 
