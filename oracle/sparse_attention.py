@@ -419,7 +419,8 @@ def _bf16(x) -> np.ndarray:
 
 
 def fp8_attention(Q, K, V, block_idx, block: int, tail: str, scale: float, *,
-                  qblocks: Optional[Iterable[Tuple[int, int, int]]] = None):
+                  qblocks: Optional[Iterable[Tuple[int, int, int]]] = None,
+                  absolute_values: bool = False):
     """The e4m3 quantised forward of the sparse branch, float64 (P unquantised).
 
     SLA2 §2C runs the sparse branch in 8 bits; reading: Q, K, V are replaced by
@@ -428,10 +429,16 @@ def fp8_attention(Q, K, V, block_idx, block: int, tail: str, scale: float, *,
     of the unquantised inputs, stored in bfloat16 and quantised to e4m3 with one
     scale per group of 128 blocks.  The attention itself is PISA's N_t / D_t in
     float64.  Same return convention as ``sparse_attention``.
+
+    With ``absolute_values`` the values (and value means) are replaced by their
+    absolute values, which gives Σ_n p_n |v_n| / l per output element: the
+    scale of the error that rounding each p_n to e4m3 can cause.
     """
     Qd = quantise_blocks_e4m3(Q, block)[0]
     Kd = quantise_blocks_e4m3(K, block)[0]
     Vd = quantise_blocks_e4m3(V, block)[0]
+    if absolute_values:
+        Vd = np.abs(Vd)
     Bsz, H, N, d = np.asarray(K).shape
     nb = N // block
     idx = np.asarray(block_idx)
@@ -441,6 +448,8 @@ def fp8_attention(Q, K, V, block_idx, block: int, tail: str, scale: float, *,
         kb = _bf16(K64.reshape(Bsz, H, nb, block, d).mean(axis=3))
         vb = _bf16(V64.reshape(Bsz, H, nb, block, d).sum(axis=3) / block)
         cent = (quantise_blocks_e4m3(kb, 128)[0], quantise_blocks_e4m3(vb, 128)[0])
+        if absolute_values:
+            cent = (cent[0], np.abs(cent[1]))
     todo = list(qblocks) if qblocks is not None else [
         (b, h, i) for b in range(Bsz) for h in range(H) for i in range(N // block)]
     out = np.empty((len(todo), block, d))

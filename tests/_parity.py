@@ -65,3 +65,20 @@ def selection_agreement(scores_gpu: np.ndarray, scores_ref: np.ndarray, k: int, 
             assert a == b, f"row {r}: selections differ although the score gap is {gap:.3e}"
         agree += a == b
     return agree / sr.shape[0]
+
+
+# e4m3 rounds to nearest even with 3 mantissa bits: the relative error of a
+# rounded normal value is at most 2^-4
+E4M3_REL = 2.0 ** -4
+
+
+def assert_fp8_bound(got, emu, emu_abs, what=""):
+    """|got - emu| <= 2^-4 Σp|v|/l (P rounded to e4m3) + 2^-8 |emu| (bf16
+    output) + 2e-3 (fp32 sums, e4m3 subnormals of tiny p), elementwise."""
+    got = np.asarray(got, dtype=np.float64)
+    bound = E4M3_REL * np.asarray(emu_abs) + 2.0 ** -8 * np.abs(emu) + 2e-3
+    err = np.abs(got - emu)
+    worst = float((err / bound).max())
+    assert np.all(np.isfinite(got)), f"{what}: non-finite output"
+    assert worst <= 1.0, f"{what}: error reaches {worst:.2f} of the e4m3 rounding bound (max-abs {err.max():.3e})"
+    return float(err.max()), float(err.mean())

@@ -11,8 +11,8 @@ import oracle
 from block_sparse_approximate_b200 import binding as bd
 from block_sparse_approximate_b200 import workloads as wl
 from block_sparse_approximate_b200.pipeline import DecodeStep, Fp8PrefillStep, PrefillStep
-from tests._parity import (BF16_TOL, assert_no_device_error, assert_tol, check_topk_exact, np64,
-                           selection_agreement)
+from tests._parity import (BF16_TOL, assert_fp8_bound, assert_no_device_error, assert_tol, check_topk_exact,
+                           np64, selection_agreement)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -74,9 +74,10 @@ def test_decode_full_size_sampled(lib):
 
 
 def test_fp8_full_size_sampled(lib):
-    # e4m3 sparse branch against the oracle's quantised forward (the pin, at
-    # the FP8 tolerance); its distance to the unquantised float64 oracle is
-    # the format's own error on these inputs and is only bounded loosely here
+    # e4m3 sparse branch against the oracle's quantised forward within the
+    # bound of P's e4m3 rounding (the pin); its distance to the unquantised
+    # float64 oracle is the format's own error on these inputs (reported, and
+    # only bounded loosely here)
     w = wl.WORKLOADS["fp8"]
     inp = wl.prefill_inputs(w, DEV)
     step = Fp8PrefillStep(w, inp)
@@ -90,8 +91,10 @@ def test_fp8_full_size_sampled(lib):
     sub = {n: inp[n][:, heads].cpu().float().numpy() for n in ("Q", "K", "V")}
     qb = [(b, hmap[h], i) for b, h, i in picks]
     got = np.stack([np64(O[b, h, i * w.block:(i + 1) * w.block]) for b, h, i in picks])
-    emu = oracle.fp8_attention(sub["Q"], sub["K"], sub["V"], idx, w.block, w.tail, w.scale, qblocks=qb)
-    assert_tol(got, emu, (6e-2, 6e-3), "fp8 full size vs quantised forward")
+    args = (sub["Q"], sub["K"], sub["V"], idx, w.block, w.tail, w.scale)
+    emu = oracle.fp8_attention(*args, qblocks=qb)
+    emu_abs = oracle.fp8_attention(*args, qblocks=qb, absolute_values=True)
+    assert_fp8_bound(got, emu, emu_abs, "fp8 full size vs quantised forward")
     ref = oracle.sparse_attention(sub["Q"], sub["K"], sub["V"], idx, w.block, w.tail, w.scale, qblocks=qb)
     err = np.abs(got - ref)
     print(f"fp8 vs unquantised float64 oracle: max-abs {err.max():.3e} mean-abs {err.mean():.3e}")
