@@ -239,6 +239,87 @@ def time_decode(steps: int = 50, warmup: int = 5, batch=None):
             "hbm_peak_gbs": hbm, "frac": byts / ms / 1e6 / hbm, "peak_source": src}
 
 
+def _time_prefill_variant(step, attn_call, steps: int, warmup: int):
+    """Times ``step`` (whole step) and ``attn_call`` (the attention launch alone)."""
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(steps):
+        step()
+    e.record()
+    torch.cuda.synchronize()
+    ms_step = s.elapsed_time(e) / steps
+    s.record()
+    for _ in range(steps):
+        attn_call()
+    e.record()
+    torch.cuda.synchronize()
+    return ms_step, s.elapsed_time(e) / steps
+
+
+def time_fp8(steps: int = 10, warmup: int = 3):
+    """The e4m3 sparse branch on the fp8 workload (video_dit shapes, seed 3)."""
+    from block_sparse_approximate_b200 import binding as bd
+    from block_sparse_approximate_b200.pipeline import Fp8PrefillStep
+    w = wl.WORKLOADS["fp8"]
+    inp = wl.prefill_inputs(w, "cuda")
+    step = Fp8PrefillStep(w, inp)
+    step()
+    attn = lambda: bd.sparse_attn_fwd_fp8(step.ops, step.shape, step.buf.block_idx, w.tail, w.scale,
+                                          out=step.buf.out)
+    ms_step, attn_ms = _time_prefill_variant(step, attn, steps, warmup)
+    _, bf16, _, src = _peaks()
+    fl = algorithmic_attn_flops(w)
+    ach = fl / (attn_ms * 1e-3) / 1e12
+    out = {"workload": w.name, "ms_per_step": ms_step, "attn_ms": attn_ms, "executed_tflops": ach,
+           "dense_equiv_tflops": dense_flops(w) / (ms_step * 1e-3) / 1e12,
+           "peak_tflops": 2 * bf16, "frac": ach / (2 * bf16),
+           "peak_source": f"2 x {src} bf16 burst (e4m3 dense rate is twice bf16)",
+           "step": "block_pool + route + e4m3 quantisation of Q, K, V and centroids + sparse_attn_fwd_fp8"}
+    del inp, step
+    torch.cuda.empty_cache()
+    return out
+
+
+def linear_mix_flops(w) -> float:
+    """Per query block: exact softmax part 4·d·(k·B)·B, the A_i accumulation
+    2·d²·(k·B) and the final relu(Q)(H_tot − A_i) 2·d²·B."""
+    per_qblk = 4.0 * w.d * w.k * w.block * w.block + 2.0 * w.d * w.d * w.k * w.block + 2.0 * w.d * w.d * w.block
+    return per_qblk * w.B * w.H * w.nb
+
+
+def time_sla2(steps: int = 2, warmup: int = 1):
+    """The SLA2 mix workload (H=40, N=65536, proj router, linear mix)."""
+    from block_sparse_approximate_b200 import binding as bd
+    from block_sparse_approximate_b200.pipeline import PrefillStep
+    w = wl.WORKLOADS["sla2_mix"]
+    inp = wl.prefill_inputs(w, "cuda")
+    step = PrefillStep(w, inp)
+    step()
+
+    def attn():
+        import ctypes
+        buf = step.buf
+        bd._check("sa_sparse_attn_fwd",
+                  step.lib.sa_sparse_attn_fwd(inp["Q"].data_ptr(), inp["K"].data_ptr(), inp["V"].data_ptr(),
+                                              step.dtype, step.shape, buf.block_idx.data_ptr(), int(w.k),
+                                              bd.TAIL[w.tail], inp["alpha"].data_ptr(), ctypes.byref(step.cst),
+                                              float(w.scale), buf.out.data_ptr(),
+                                              torch.cuda.current_stream().cuda_stream))
+    ms_step, attn_ms = _time_prefill_variant(step, attn, steps, warmup)
+    _, bf16, _, src = _peaks()
+    fl = linear_mix_flops(w)
+    ach = fl / (attn_ms * 1e-3) / 1e12
+    out = {"workload": w.name, "ms_per_step": ms_step, "attn_ms": attn_ms, "executed_tflops": ach,
+           "dense_equiv_tflops": dense_flops(w) / (ms_step * 1e-3) / 1e12,
+           "peak_tflops": bf16, "frac": ach / bf16, "peak_source": f"{src} bf16 burst"}
+    del inp, step
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args, world, rank, local):
     from block_sparse_approximate_b200 import binding as bd
     from block_sparse_approximate_b200.pipeline import PrefillStep
@@ -247,6 +328,14 @@ def run_ours(args, world, rank, local):
     if args.only == "decode":
         if rank == 0:
             print(json.dumps({"decode": time_decode(args.steps, args.warmup, args.decode_batch)}), flush=True)
+        return 0
+    if args.only == "fp8":
+        if rank == 0:
+            print(json.dumps({"fp8": time_fp8(args.steps, args.warmup)}), flush=True)
+        return 0
+    if args.only == "sla2":
+        if rank == 0:
+            print(json.dumps({"sla2_mix": time_sla2(args.steps, args.warmup)}), flush=True)
         return 0
     w = wl.WORKLOADS[WORKLOAD]
     wr = wl.Workload(**{**w.__dict__, "seed": w.seed + 1000 * rank}) if rank else w
@@ -336,11 +425,13 @@ def run_ours(args, world, rank, local):
                "h2d_bytes_per_step": sum(inp[n].numel() * inp[n].element_size() for n in ("Q", "K", "V")),
                "d2h_bytes_per_step": step.buf.out.numel() * step.buf.out.element_size()}
 
-    decode = None
+    decode = fp8 = sla2 = None
     if rank == 0 and args.only == "all" and not args.no_decode:
         del step
         torch.cuda.empty_cache()
         decode = time_decode(batch=args.decode_batch)
+        fp8 = time_fp8()
+        sla2 = time_sla2()
     ck = clocks.stop() if clocks else None
 
     if rank != 0:
@@ -371,6 +462,8 @@ def run_ours(args, world, rank, local):
         "gpu_launches": args.steps * PrefillStepLaunches(w),
         "clocks": ck,
         "decode": decode,
+        "fp8": fp8,
+        "sla2_mix": sla2,
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -389,8 +482,8 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
-    ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
-                    help="prefill: the timed step only; decode: only the decode timing")
+    ap.add_argument("--only", choices=["all", "prefill", "decode", "fp8", "sla2"], default="all",
+                    help="prefill: the timed step only; decode / fp8 / sla2: only that workload's timing")
     ap.add_argument("--decode-batch", type=int, default=None,
                     help="sequences in the decode workload (default: the full 16)")
     args = ap.parse_args(argv)
