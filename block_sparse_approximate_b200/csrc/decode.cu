@@ -1,18 +1,25 @@
 // GQA decode with block routing and the zero-order tail.
 //
-// SPLA §2 notes that decoding is bound by loading the KV cache and keeps the
-// IO profile of sparse decoding: only the selected blocks are read token by
-// token; every other block is represented by its precomputed statistics.
-// Steps (all on the caller's stream):
-//   1. decode_score_kernel  the SPLA §2.1 block score (log form) of every KV
-//                           block for each query head, summed over the GQA group
-//                           (logsumexp) -> scores[b, g, j]
-//   2. decode_topk_kernel   top-k per (sequence, KV head) -> block_idx
-//   3. decode_attn_kernel   split over the KV axis: exact online softmax over
-//                           this split's share of the selected blocks plus the
-//                           PISA zero-order pseudo-keys of this split's share of
-//                           the unselected blocks -> partial (max, sum, acc)
-//   4. decode_combine_kernel  merges the partial states -> o
+// SPLA §1-2 notes that decoding is bound by loading the KV cache and keeps
+// the IO profile of sparse decoding: only the selected blocks are read token
+// by token; every other block is represented by its precomputed statistics.
+// Four launches on the caller's stream:
+//   A. decode_stats_kernel  one pass over the block statistics (kmean, kvar,
+//        vsum, each read once): the SPLA §2.1 score of every block for each
+//        query head, summed over the GQA group (logsumexp) -> scores, and the
+//        PISA zero-order term of EVERY block -> per-segment partial states
+//        (max, sum, acc) per query head;
+//   B. decode_topk_kernel   top-k per (sequence, KV head) -> block_idx;
+//   C. decode_exact_kernel  the selected blocks token by token (exact online
+//        softmax), and for each selected block its own zero-order term with
+//        weight -1, so that A + C hold the zero-order term of the unselected
+//        blocks only (the subtraction form of SPLA §2.2 applied to PISA's
+//        tail; it cannot cancel below zero because Σ_n e^{x_n} ≥ B e^{mean x}
+//        for every block) -> per-segment partial states;
+//   D. decode_combine_kernel  merges the partial states -> o.
+// A and C are persistent streaming kernels: each CTA walks a list of
+// 48 KB / 32 KB stages staged into shared memory with cp.async, three or four
+// stages deep, so the HBM stays busy while the previous stage is reduced.
 #include <mutex>
 
 #include "topk.cuh"
@@ -23,321 +30,575 @@ namespace {
 constexpr int kDecThreads = 256;
 constexpr int kDecWarps = kDecThreads / 32;
 constexpr int kMaxGroup = 8;
-constexpr int kScoreChunk = 64;   // KV blocks per CTA of the score kernel
-constexpr int kTok = 32;          // tokens (or centroids) per warp step
+constexpr int kTok = 32;
+
+// A: a stage is 32 blocks of statistics (kmean, kvar, vsum rows); a segment
+// is kSegA stages (one partial state per segment and query head)
+constexpr int kStageBlocksA = 32;
+constexpr int kSegA = 8;
+constexpr int kRingA = 3;
+// C: a stage is 64 tokens of K and V; a segment is kSegC stages
+constexpr int kStageTokC = 64;
+constexpr int kSegC = 8;
+constexpr int kRingC = 4;
 
 struct DecodeLayout {
-  size_t scores_off, idx_off, part_off, total;
-  int nsplit;
+  size_t scores_off, idx_off, parta_off, partc_off, total;
+  int nsegA, nsegC;
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-int decode_splits(const sa_decode_shape& s, int topk) {
-  const int nb = s.N / s.block;
-  const long chunks = (long)topk * (s.block / kTok) + (nb + kTok - 1) / kTok;
-  long ns = (chunks + kDecWarps - 1) / kDecWarps;
-  if (ns < 1) ns = 1;
-  if (ns > 64) ns = 64;
-  return (int)ns;
-}
-
 DecodeLayout decode_layout(const sa_decode_shape& s, int topk) {
   DecodeLayout L;
   const int nb = s.N / s.block;
-  L.nsplit = decode_splits(s, topk);
+  L.nsegA = (nb + kStageBlocksA * kSegA - 1) / (kStageBlocksA * kSegA);
+  L.nsegC = (int)(((long)topk * s.block + kStageTokC * kSegC - 1) / (kStageTokC * kSegC));
+  const size_t part = (size_t)(s.d + 2) * sizeof(float);
   L.scores_off = 0;
   L.idx_off = align256((size_t)s.B * s.Hkv * nb * sizeof(float));
-  L.part_off = L.idx_off + align256((size_t)s.B * s.Hkv * (topk > 0 ? topk : 1) * sizeof(int32_t));
-  L.total = L.part_off + align256((size_t)s.B * s.Hq * L.nsplit * (s.d + 2) * sizeof(float));
+  L.parta_off = L.idx_off + align256((size_t)s.B * s.Hkv * (topk > 0 ? topk : 1) * sizeof(int32_t));
+  L.partc_off = L.parta_off + align256((size_t)s.B * s.Hq * (L.nsegA > 0 ? L.nsegA : 1) * part);
+  L.total = L.partc_off + align256((size_t)s.B * s.Hq * (L.nsegC > 0 ? L.nsegC : 1) * part);
   return L;
 }
 
-// ---- 1. scores -----------------------------------------------------------
-template <int D>
-__global__ void __launch_bounds__(kDecThreads)
-decode_score_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int Hq, int Hkv,
-                    int nb, float scale, float* __restrict__ scores) {
-  constexpr int PER = D / 32;
-  const int chunk = blockIdx.x, kh = blockIdx.y, b = blockIdx.z;
-  const int g = Hq / Hkv;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  __shared__ float qs[kMaxGroup][D];
-  __shared__ float ws[kMaxGroup][D];
-  for (int idx = threadIdx.x; idx < g * D; idx += kDecThreads) {
-    const int hh = idx / D, c = idx % D;
-    const float x = __bfloat162float(q[((size_t)b * Hq + kh * g + hh) * D + c]);
-    qs[hh][c] = scale * x;
-    ws[hh][c] = 0.5f * scale * scale * x * x;
-  }
-  __syncthreads();
-  const size_t base = ((size_t)b * Hkv + kh) * nb;
-  const int j_end = min(nb, (chunk + 1) * kScoreChunk);
-  for (int j = chunk * kScoreChunk + warp; j < j_end; j += kDecWarps) {
-    float km[PER], kv[PER];
-#pragma unroll
-    for (int p = 0; p < PER; ++p) {
-      km[p] = st.kmean[(base + j) * D + lane * PER + p];
-      kv[p] = st.kvar[(base + j) * D + lane * PER + p];
-    }
-    float L[kMaxGroup];
-    float mx = -INFINITY;
-#pragma unroll
-    for (int hh = 0; hh < kMaxGroup; ++hh) {
-      if (hh < g) {
-        float s1 = 0.f, s2 = 0.f;
-#pragma unroll
-        for (int p = 0; p < PER; ++p) {
-          s1 = fmaf(qs[hh][lane * PER + p], km[p], s1);
-          s2 = fmaf(ws[hh][lane * PER + p], kv[p], s2);
-        }
-        s1 = warp_sum(s1);
-        s2 = warp_sum(s2);
-        L[hh] = s1 + log1pf(s2);
-        mx = fmaxf(mx, L[hh]);
-      }
-    }
-    float sum = 0.f;
-#pragma unroll
-    for (int hh = 0; hh < kMaxGroup; ++hh)
-      if (hh < g) sum += expf(L[hh] - mx);
-    if (lane == 0) scores[base + j] = mx + logf(sum);
-  }
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(smem_dst)),
+               "l"(gsrc)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// ---- 2. top-k ------------------------------------------------------------
-__global__ void __launch_bounds__(kDecThreads)
-decode_topk_kernel(const float* __restrict__ scores, int Hkv, int nb, int topk,
-                   int32_t* __restrict__ idx) {
-  const int kh = blockIdx.x, b = blockIdx.y;
-  extern __shared__ unsigned long long smem_u64[];
-  int n2 = 1;
-  while (n2 < nb) n2 <<= 1;
-  float* sc = reinterpret_cast<float*>(smem_u64 + n2);
-  const size_t base = ((size_t)b * Hkv + kh);
-  for (int j = threadIdx.x; j < nb; j += kDecThreads) sc[j] = scores[base * nb + j];
-  __syncthreads();
-  block_topk_ascending(sc, nb, topk, smem_u64, idx + base * topk);
-}
-
-// ---- 3. split attention --------------------------------------------------
-// Warp step over kTok keys: lane t computes the logits of key t for the g
-// heads (lane = key); the accumulators are then updated with lane = channel,
-// the probabilities broadcast by shuffles.
-template <int D>
-struct WarpState {
-  float m[kMaxGroup], l[kMaxGroup], acc[kMaxGroup][D / 32];
+// Partial online-softmax state of one query head in a warp: log2-domain max,
+// lane-partial sum, and the lane's 4 channels (lane = channel group).
+struct HeadState {
+  float m, l, acc[4];
 };
 
+__device__ __forceinline__ void head_reset(HeadState& S) {
+  S.m = -INFINITY;
+  S.l = 0.f;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) S.acc[c] = 0.f;
+}
+
+// Adds keys with lane-held log2 logits x (lane = key, -inf = absent) to S;
+// returns the lane's probability (relative to the new max) for the caller to
+// fold values in with lane = channel.
+__device__ __forceinline__ float head_add_logits(HeadState& S, float x) {
+  const float tmax = warp_max(x);
+  if (tmax == -INFINITY) return 0.f;
+  const float m_new = fmaxf(S.m, tmax);
+  const float corr = fast_exp2(S.m - m_new);
+  const float p = fast_exp2(x - m_new);
+  S.l = S.l * corr + p;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) S.acc[c] *= corr;
+  S.m = m_new;
+  return p;
+}
+
+// Writes the warp's state (lane sums reduced) to out[0..D+2) (D = 128: 4
+// channels per lane; D = 64: lanes 0..15 hold 4 channels each).
 template <int D>
-__global__ void __launch_bounds__(kDecThreads)
-decode_attn_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ Kc,
-                   const __nv_bfloat16* __restrict__ Vc, sa_block_stats st, int Hq, int Hkv, int N,
-                   int blk, const int32_t* __restrict__ idx, int topk, int tail, float scale,
-                   int nsplit, float* __restrict__ partial) {
-  constexpr int PER = D / 32;
-  const int split = blockIdx.x, kh = blockIdx.y, b = blockIdx.z;
+__device__ __forceinline__ void head_store(const HeadState& S, float* out, int lane) {
+  const float l = warp_sum(S.l);
+  if (lane == 0) {
+    out[0] = S.m;
+    out[1] = l;
+  }
+  if (lane * 4 < D) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) out[2 + lane * 4 + c] = S.acc[c];
+  }
+}
+
+// ---- A. statistics pass --------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(kDecThreads, 1)
+decode_stats_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int Hq, int Hkv, int nb, int blk,
+                    float scale, int nsegA, int npairs, float* __restrict__ scores, float* __restrict__ parta) {
+  constexpr int CH = D / 4;                          // float4 chunks per row
+  constexpr uint32_t kRowB = D * 4;                  // bytes per stats row
+  constexpr uint32_t kArrB = kStageBlocksA * kRowB;  // one array of one stage
+  constexpr uint32_t kStageB = 3 * kArrB;
+  extern __shared__ __align__(16) uint8_t dsm[];
+  float* qs = reinterpret_cast<float*>(dsm);                 // [g][D]  s q log2e
+  float* ws = qs + kMaxGroup * D;                            // [g][D]  ½ s² q²
+  float* lsm = ws + kMaxGroup * D;                           // [g][32] per-head log scores
+  uint8_t* ring = reinterpret_cast<uint8_t*>(lsm + kMaxGroup * kStageBlocksA);
   const int g = Hq / Hkv;
-  const int nb = N / blk;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const size_t kv_base = ((size_t)b * Hkv + kh) * (size_t)N * D;
-  const size_t st_base = ((size_t)b * Hkv + kh) * (size_t)nb;
-  const int32_t* sel = idx + ((size_t)b * Hkv + kh) * topk;
-
-  extern __shared__ float dsm[];
-  float* qs = dsm;                                             // kMaxGroup * D
-  uint32_t* selmask = reinterpret_cast<uint32_t*>(qs + kMaxGroup * D);
-  const int nwords = (nb + 31) / 32;
-  float* red = reinterpret_cast<float*>(selmask + ((nwords + 3) & ~3));  // warps*g*(D+2)
-
-  const float scale2 = scale * kLog2e;
-  for (int i = threadIdx.x; i < g * D; i += kDecThreads) {
-    const int hh = i / D, c = i % D;
-    qs[hh * D + c] = scale2 * __bfloat162float(q[((size_t)b * Hq + kh * g + hh) * D + c]);
-  }
-  for (int w = threadIdx.x; w < nwords; w += kDecThreads) selmask[w] = 0u;
-  __syncthreads();
-  for (int s = threadIdx.x; s < topk; s += kDecThreads) {
-    const int j = sel[s];
-    atomicOr(&selmask[j >> 5], 1u << (j & 31));
-  }
-  __syncthreads();
-
-  WarpState<D> S;
-#pragma unroll
-  for (int hh = 0; hh < kMaxGroup; ++hh) {
-    S.m[hh] = -INFINITY;
-    S.l[hh] = 0.f;
-#pragma unroll
-    for (int c = 0; c < PER; ++c) S.acc[hh][c] = 0.f;
-  }
-
-  // this split's share of the selected blocks and of the block range
-  const int s0 = (int)(((long)topk * split) / nsplit), s1 = (int)(((long)topk * (split + 1)) / nsplit);
-  const int j0 = (int)(((long)nb * split) / nsplit), j1 = (int)(((long)nb * (split + 1)) / nsplit);
-  const int steps_per_block = blk / kTok;
-  const int n_exact = (s1 - s0) * steps_per_block;
-  const int n_tail = tail == SA_TAIL_ZERO_ORDER ? (j1 - j0 + kTok - 1) / kTok : 0;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int stages_per_seg_full = kSegA;
+  const int nstage_pair = (nb + kStageBlocksA - 1) / kStageBlocksA;
+  const long total_segs = (long)npairs * nsegA;
   const float bias2 = log2f((float)blk);
   const float inv_blk = 1.0f / blk;
 
-  for (int step = warp; step < n_exact + n_tail; step += kDecWarps) {
-    const bool exact = step < n_exact;
-    float lg[kMaxGroup];
-    bool valid = true;
-    int tok0 = 0, jbase = 0;
-    if (exact) {
-      const int j = sel[s0 + step / steps_per_block];
-      tok0 = j * blk + (step % steps_per_block) * kTok;
-      // lane = token: logits over the full key row
-      const __nv_bfloat16* krow = Kc + kv_base + (size_t)(tok0 + lane) * D;
-#pragma unroll
-      for (int hh = 0; hh < kMaxGroup; ++hh) lg[hh] = 0.f;
-#pragma unroll 4
-      for (int c8 = 0; c8 < D; c8 += 8) {
-        float kx[8];
-        load8<__nv_bfloat16>(krow + c8, kx);
-#pragma unroll
-        for (int hh = 0; hh < kMaxGroup; ++hh) {
-          if (hh < g) {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) lg[hh] = fmaf(qs[hh * D + c8 + e], kx[e], lg[hh]);
-          }
-        }
-      }
-    } else {
-      jbase = j0 + (step - n_exact) * kTok;
-      const int jj = jbase + lane;   // lane = centroid of an unselected block
-      valid = jj < j1 && !((selmask[jj >> 5] >> (jj & 31)) & 1u);
-#pragma unroll
-      for (int hh = 0; hh < kMaxGroup; ++hh) lg[hh] = bias2;
-      if (jj < j1) {
-        const float* kmr = st.kmean + (st_base + jj) * D;
-#pragma unroll 4
-        for (int c4 = 0; c4 < D; c4 += 4) {
-          const float4 k4 = __ldg(reinterpret_cast<const float4*>(kmr + c4));
-#pragma unroll
-          for (int hh = 0; hh < kMaxGroup; ++hh) {
-            if (hh < g) {
-              lg[hh] = fmaf(qs[hh * D + c4 + 0], k4.x, lg[hh]);
-              lg[hh] = fmaf(qs[hh * D + c4 + 1], k4.y, lg[hh]);
-              lg[hh] = fmaf(qs[hh * D + c4 + 2], k4.z, lg[hh]);
-              lg[hh] = fmaf(qs[hh * D + c4 + 3], k4.w, lg[hh]);
-            }
-          }
-        }
-      }
+  // the CTA's stage sequence: its segments in order, each segment's stages
+  auto seg_of = [&](long k_seg) { return (long)blockIdx.x + k_seg * gridDim.x; };
+  auto stages_in = [&](long seg) {
+    const int sseg = (int)(seg % nsegA);
+    const int first = sseg * stages_per_seg_full;
+    return min(stages_per_seg_full, nstage_pair - first);
+  };
+  // issue the copies of stage `sub` of segment `seg` into ring slot `slot`
+  auto issue = [&](long seg, int sub, int slot) {
+    const int pair = (int)(seg / nsegA), sseg = (int)(seg % nsegA);
+    const int j0 = (sseg * stages_per_seg_full + sub) * kStageBlocksA;
+    const int rows = min(kStageBlocksA, nb - j0);
+    const size_t goff = ((size_t)pair * nb + j0) * D;
+    uint8_t* dst = ring + slot * kStageB;
+    const int n16 = rows * (int)(kRowB / 16);
+    for (int x = tid; x < 3 * n16; x += kDecThreads) {
+      const int a = x / n16, o = x % n16;
+      const float* src = (a == 0 ? st.kmean : a == 1 ? st.kvar : st.vsum) + goff;
+      cp_async16(dst + a * kArrB + o * 16, reinterpret_cast<const uint8_t*>(src) + o * 16);
     }
-    // online-softmax bookkeeping per head (lane-local probabilities)
-    float p[kMaxGroup];
-    bool any = false;
-#pragma unroll
-    for (int hh = 0; hh < kMaxGroup; ++hh) {
-      p[hh] = 0.f;
-      if (hh < g) {
-        const float x = valid ? lg[hh] : -INFINITY;
-        const float tmax = warp_max(x);
-        if (tmax != -INFINITY) {
-          any = true;
-          const float m_new = fmaxf(S.m[hh], tmax);
-          const float corr = fast_exp2(S.m[hh] - m_new);
-          p[hh] = fast_exp2(x - m_new);
-          S.l[hh] = S.l[hh] * corr + p[hh];   // lane-partial sum
-#pragma unroll
-          for (int c = 0; c < PER; ++c) S.acc[hh][c] *= corr;
-          S.m[hh] = m_new;
-        }
-      }
+  };
+
+  // flat iteration over (segment, stage) pairs of this CTA
+  long cur_seg_k = 0;
+  if (seg_of(0) >= total_segs) return;
+  int cur_sub = 0;
+  // lookahead cursor for prefetching
+  long pf_seg_k = 0;
+  int pf_sub = 0;
+  auto pf_valid = [&]() { return seg_of(pf_seg_k) < total_segs; };
+  auto pf_advance = [&]() {
+    if (++pf_sub >= stages_in(seg_of(pf_seg_k))) {
+      pf_sub = 0;
+      ++pf_seg_k;
     }
-    if (!any) continue;
-    // lane = channel: accumulate the kTok value rows
-#pragma unroll 4
-    for (int t = 0; t < kTok; ++t) {
-      float v[PER];
-      if (exact) {
-        const __nv_bfloat16* vrow = Vc + kv_base + (size_t)(tok0 + t) * D + lane * PER;
-        if constexpr (PER == 4) {
-          const uint2 u = __ldg(reinterpret_cast<const uint2*>(vrow));
-          const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
-          const float2 c = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
-          v[0] = a.x; v[1] = a.y; v[2] = c.x; v[3] = c.y;
-        } else {
-          const unsigned u = __ldg(reinterpret_cast<const unsigned*>(vrow));
-          const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u));
-          v[0] = a.x; v[1] = a.y;
-        }
-      } else {
-        const int jt = jbase + t;
-        if (jt < j1) {
-          const float* vr = st.vsum + (st_base + jt) * D + lane * PER;
-#pragma unroll
-          for (int c = 0; c < PER; ++c) v[c] = __ldg(vr + c) * inv_blk;
-        } else {
-#pragma unroll
-          for (int c = 0; c < PER; ++c) v[c] = 0.f;
-        }
-      }
-#pragma unroll
-      for (int hh = 0; hh < kMaxGroup; ++hh) {
-        if (hh < g) {
-          const float pt = __shfl_sync(0xffffffffu, p[hh], t);
-#pragma unroll
-          for (int c = 0; c < PER; ++c) S.acc[hh][c] = fmaf(pt, v[c], S.acc[hh][c]);
-        }
-      }
+  };
+  int pf_slot = 0;
+  for (int r = 0; r < kRingA - 1; ++r) {
+    if (pf_valid()) {
+      issue(seg_of(pf_seg_k), pf_sub, pf_slot);
+      pf_advance();
     }
+    cp_async_commit();
+    pf_slot = (pf_slot + 1) % kRingA;
   }
 
-  // merge the warps' states, then write this split's partial state
-  float* my = red + (size_t)warp * kMaxGroup * (D + 2);
-#pragma unroll
-  for (int hh = 0; hh < kMaxGroup; ++hh) {
-    if (hh < g) {
-      const float lsum = warp_sum(S.l[hh]);
-      if (lane == 0) {
-        my[hh * (D + 2) + 0] = S.m[hh];
-        my[hh * (D + 2) + 1] = lsum;
+  HeadState S;
+  int cur_pair = -1;
+  int slot = 0;
+  while (seg_of(cur_seg_k) < total_segs) {
+    const long seg = seg_of(cur_seg_k);
+    const int pair = (int)(seg / nsegA), sseg = (int)(seg % nsegA);
+    const int b = pair / Hkv, kh = pair % Hkv;
+    if (cur_sub == 0) {
+      if (pair != cur_pair) {
+        // this pair's query vectors
+        __syncthreads();
+        for (int x = tid; x < g * D; x += kDecThreads) {
+          const int hh = x / D, c = x % D;
+          const float v = __bfloat162float(q[((size_t)b * Hq + kh * g + hh) * D + c]);
+          qs[hh * D + c] = scale * kLog2e * v;
+          ws[hh * D + c] = 0.5f * scale * scale * v * v;
+        }
+        cur_pair = pair;
       }
-#pragma unroll
-      for (int c = 0; c < PER; ++c) my[hh * (D + 2) + 2 + lane * PER + c] = S.acc[hh][c];
+      head_reset(S);
+    }
+    // prefetch one more stage, then wait for the current one
+    if (pf_valid()) {
+      issue(seg_of(pf_seg_k), pf_sub, pf_slot);
+      pf_advance();
+    }
+    cp_async_commit();
+    pf_slot = (pf_slot + 1) % kRingA;
+    cp_async_wait<kRingA - 1>();
+    __syncthreads();
+
+    const uint8_t* stg = ring + slot * kStageB;
+    const float* km = reinterpret_cast<const float*>(stg);
+    const float* kv = reinterpret_cast<const float*>(stg + kArrB);
+    const float* vs = reinterpret_cast<const float*>(stg + 2 * kArrB);
+    const int j0 = (sseg * stages_per_seg_full + cur_sub) * kStageBlocksA;
+    const int rows = min(kStageBlocksA, nb - j0);
+    if (warp < g) {
+      // lane = block: dot products over rotated float4 chunks (conflict free)
+      const int hh = warp;
+      float d1 = 0.f, d2 = 0.f;
+      if (lane < rows) {
+        const float4* kr = reinterpret_cast<const float4*>(km + lane * D);
+        const float4* vr = reinterpret_cast<const float4*>(kv + lane * D);
+        const float4* qr = reinterpret_cast<const float4*>(qs + hh * D);
+        const float4* wr = reinterpret_cast<const float4*>(ws + hh * D);
+#pragma unroll 8
+        for (int c = 0; c < CH; ++c) {
+          const int cc = (c + lane) % CH;
+          const float4 a = kr[cc], qv = qr[cc], vv = vr[cc], wv = wr[cc];
+          d1 = fmaf(a.x, qv.x, fmaf(a.y, qv.y, fmaf(a.z, qv.z, fmaf(a.w, qv.w, d1))));
+          d2 = fmaf(vv.x, wv.x, fmaf(vv.y, wv.y, fmaf(vv.z, wv.z, fmaf(vv.w, wv.w, d2))));
+        }
+      }
+      // d1 = s log2e q·k̄: natural log score s q·k̄ + log1p(½ s² Σ q² var)
+      const float lnat = d1 * kLn2 + log1pf(d2);
+      lsm[hh * kStageBlocksA + lane] = lnat;
+      // zero-order term of every block of the stage (log2 domain)
+      const float x = lane < rows ? d1 + bias2 : -INFINITY;
+      const float p = head_add_logits(S, x);
+      for (int t = 0; t < rows; ++t) {
+        const float pt = __shfl_sync(0xffffffffu, p, t);
+        if (lane * 4 < D) {
+          const float4 v4 = *reinterpret_cast<const float4*>(vs + t * D + lane * 4);
+          S.acc[0] = fmaf(pt, v4.x * inv_blk, S.acc[0]);
+          S.acc[1] = fmaf(pt, v4.y * inv_blk, S.acc[1]);
+          S.acc[2] = fmaf(pt, v4.z * inv_blk, S.acc[2]);
+          S.acc[3] = fmaf(pt, v4.w * inv_blk, S.acc[3]);
+        }
+      }
+    }
+    __syncthreads();
+    // group score of the stage's blocks: logsumexp over the g heads
+    if (warp == 0 && lane < rows) {
+      float mx = -INFINITY;
+      for (int hh = 0; hh < g; ++hh) mx = fmaxf(mx, lsm[hh * kStageBlocksA + lane]);
+      float sum = 0.f;
+      for (int hh = 0; hh < g; ++hh) sum += expf(lsm[hh * kStageBlocksA + lane] - mx);
+      scores[(size_t)pair * nb + j0 + lane] = mx + logf(sum);
+    }
+    slot = (slot + 1) % kRingA;
+    // end of segment: write this segment's partial state for each head
+    if (++cur_sub >= stages_in(seg)) {
+      if (warp < g)
+        head_store<D>(S, parta + (((size_t)b * Hq + kh * g + warp) * nsegA + sseg) * (D + 2), lane);
+      cur_sub = 0;
+      ++cur_seg_k;
     }
   }
+  cp_async_wait<0>();
+}
+
+// ---- B. top-k ------------------------------------------------------------
+// k <= 64: each warp takes the k best of its share of the scores by repeated
+// warp arg-max over (score desc, index asc) keys, then warp 0 takes the k best
+// of the candidates the same way, and the winners are emitted in ascending
+// order.  Larger k: a bitonic sort of the whole row.
+constexpr int kTopkWarpMax = 64;
+
+__device__ __forceinline__ unsigned long long rank_key_d(float score, int j) {
+  return ((unsigned long long)(~order_key(score)) << 32) | (unsigned)j;
+}
+
+__device__ __forceinline__ unsigned long long warp_min_u64d(unsigned long long v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const unsigned long long w = __shfl_xor_sync(0xffffffffu, v, o);
+    v = w < v ? w : v;
+  }
+  return v;
+}
+
+__global__ void __launch_bounds__(kDecThreads)
+decode_topk_kernel(const float* __restrict__ scores, int nb, int topk, int32_t* __restrict__ idx) {
+  const int pair = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  extern __shared__ unsigned long long tk_smem[];
+  const float* sc = scores + (size_t)pair * nb;
+  int32_t* out = idx + (size_t)pair * topk;
+  if (topk > kTopkWarpMax) {
+    int n2 = 1;
+    while (n2 < nb) n2 <<= 1;
+    float* scs = reinterpret_cast<float*>(tk_smem + n2);
+    for (int j = tid; j < nb; j += kDecThreads) scs[j] = sc[j];
+    __syncthreads();
+    block_topk_ascending(scs, nb, topk, tk_smem, out);
+    return;
+  }
+  unsigned long long* cand = tk_smem;                       // [warps][topk]
+  const int nwords = (nb + 31) / 32;
+  uint32_t* bits = reinterpret_cast<uint32_t*>(cand + kDecWarps * kTopkWarpMax);
+  for (int x = tid; x < nwords; x += kDecThreads) bits[x] = 0u;
+  // stage 1: per warp, the k best of scores j = warp*32 + lane + 256 i
+  unsigned long long prev = 0ull;
+  for (int r = 0; r < topk; ++r) {
+    unsigned long long mine = ~0ull;
+    for (int j = warp * 32 + lane; j < nb; j += kDecThreads) {
+      const unsigned long long k = rank_key_d(sc[j], j);
+      if ((r == 0 || k > prev) && k < mine) mine = k;
+    }
+    const unsigned long long best = warp_min_u64d(mine);
+    if (lane == 0) cand[warp * kTopkWarpMax + r] = best;
+    prev = best;
+  }
   __syncthreads();
-  for (int i = threadIdx.x; i < g * D; i += kDecThreads) {
-    const int hh = i / D, c = i % D;
-    float M = -INFINITY;
-    for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, red[(w * kMaxGroup + hh) * (D + 2)]);
-    float L = 0.f, A = 0.f;
-    if (M != -INFINITY) {
-      for (int w = 0; w < kDecWarps; ++w) {
-        const float* r = red + (w * kMaxGroup + hh) * (D + 2);
+  // stage 2: the k best of the warps' candidates (absent ones are all ones)
+  if (warp == 0) {
+    prev = 0ull;
+    const int ncand = kDecWarps * topk;
+    for (int r = 0; r < topk; ++r) {
+      unsigned long long mine = ~0ull;
+      for (int x = lane; x < ncand; x += 32) {
+        const unsigned long long k = cand[(x / topk) * kTopkWarpMax + (x % topk)];
+        if ((r == 0 || k > prev) && k < mine) mine = k;
+      }
+      const unsigned long long best = warp_min_u64d(mine);
+      if (lane == 0 && best != ~0ull) {
+        const int jb = (int)(best & 0xffffffffu);
+        bits[jb >> 5] |= 1u << (jb & 31);
+      }
+      prev = best;
+    }
+    __syncwarp();
+    int base = 0;
+    for (int x0 = 0; x0 < nwords; x0 += 32) {
+      const int x = x0 + lane;
+      const uint32_t word = x < nwords ? bits[x] : 0u;
+      const int cnt = __popc(word);
+      int pre = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, pre, o);
+        if (lane >= o) pre += y;
+      }
+      int pos = base + pre - cnt;
+      uint32_t m = word;
+      while (m) {
+        const int bpos = __ffs(m) - 1;
+        out[pos++] = x * 32 + bpos;
+        m &= m - 1;
+      }
+      base += __shfl_sync(0xffffffffu, pre, 31);
+    }
+  }
+}
+
+// ---- C. exact pass over the selected blocks --------------------------------
+template <int D>
+__global__ void __launch_bounds__(kDecThreads, 1)
+decode_exact_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ Kc,
+                    const __nv_bfloat16* __restrict__ Vc, sa_block_stats st, int Hq, int Hkv, int N, int blk,
+                    const int32_t* __restrict__ idx, int topk, int zero_order, float scale, int nsegC, int npairs,
+                    float* __restrict__ partc) {
+  constexpr int CH = D / 8;                         // 16-byte chunks per bf16 row
+  constexpr int QST = 12;                           // padded floats per q chunk of 8
+  constexpr uint32_t kRowB = D * 2;
+  constexpr uint32_t kArrB = kStageTokC * kRowB;    // K (or V) of one stage
+  constexpr uint32_t kStageB = 2 * kArrB;
+  extern __shared__ __align__(16) uint8_t dsm[];
+  float* qs = reinterpret_cast<float*>(dsm);                         // [g][CH][QST]
+  float* xs = qs + kMaxGroup * CH * QST;                             // merge scratch [8 warps][D+2]
+  uint8_t* ring = reinterpret_cast<uint8_t*>(xs + kDecWarps * (D + 2));
+  const int g = Hq / Hkv;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nb = N / blk;
+  const int tok_pair = topk * blk;                  // exact tokens of one (sequence, KV head)
+  const int nstage_pair = (tok_pair + kStageTokC - 1) / kStageTokC;
+  const long total_segs = (long)npairs * nsegC;
+  const float scale2 = scale * kLog2e;
+  const float bias2 = log2f((float)blk);
+  const float inv_blk = 1.0f / blk;
+  // warp w: token half (w & 1) of the stage, heads hh with hh % 4 == w >> 1
+  const int half = warp & 1, hsel = warp >> 1;
+
+  auto seg_of = [&](long k_seg) { return (long)blockIdx.x + k_seg * gridDim.x; };
+  auto stages_in = [&](long seg) {
+    const int sseg = (int)(seg % nsegC);
+    return min(kSegC, nstage_pair - sseg * kSegC);
+  };
+  auto issue = [&](long seg, int sub, int slot) {
+    const int pair = (int)(seg / nsegC), sseg = (int)(seg % nsegC);
+    const int t0 = (sseg * kSegC + sub) * kStageTokC;     // first exact token of the stage
+    const int32_t* sel = idx + (size_t)pair * topk;
+    uint8_t* dst = ring + slot * kStageB;
+    const size_t base = (size_t)pair * N * D;
+    const int rows = min(kStageTokC, tok_pair - t0);
+    const int n16 = rows * CH;
+    for (int x = tid; x < 2 * n16; x += kDecThreads) {
+      const int a = x / n16, o = x % n16;
+      const int r = o / CH, c = o % CH;
+      const int t = t0 + r;
+      const int tok = sel[t / blk] * blk + (t % blk);
+      const __nv_bfloat16* src = (a == 0 ? Kc : Vc) + base + (size_t)tok * D + c * 8;
+      cp_async16(dst + a * kArrB + r * kRowB + c * 16, src);
+    }
+  };
+
+  if (seg_of(0) >= total_segs) return;
+  long pf_seg_k = 0;
+  int pf_sub = 0;
+  auto pf_valid = [&]() { return seg_of(pf_seg_k) < total_segs; };
+  auto pf_advance = [&]() {
+    if (++pf_sub >= stages_in(seg_of(pf_seg_k))) {
+      pf_sub = 0;
+      ++pf_seg_k;
+    }
+  };
+  int pf_slot = 0;
+  for (int r = 0; r < kRingC - 1; ++r) {
+    if (pf_valid()) {
+      issue(seg_of(pf_seg_k), pf_sub, pf_slot);
+      pf_advance();
+    }
+    cp_async_commit();
+    pf_slot = (pf_slot + 1) % kRingC;
+  }
+
+  HeadState S[2];
+  long cur_seg_k = 0;
+  int cur_sub = 0, cur_pair = -1, slot = 0;
+  while (seg_of(cur_seg_k) < total_segs) {
+    const long seg = seg_of(cur_seg_k);
+    const int pair = (int)(seg / nsegC), sseg = (int)(seg % nsegC);
+    const int b = pair / Hkv, kh = pair % Hkv;
+    if (cur_sub == 0) {
+      if (pair != cur_pair) {
+        __syncthreads();
+        for (int x = tid; x < g * D; x += kDecThreads) {
+          const int hh = x / D, c = x % D;
+          qs[(hh * CH + c / 8) * QST + (c % 8)] =
+              scale2 * __bfloat162float(q[((size_t)b * Hq + kh * g + hh) * D + c]);
+        }
+        cur_pair = pair;
+      }
+      head_reset(S[0]);
+      head_reset(S[1]);
+    }
+    if (pf_valid()) {
+      issue(seg_of(pf_seg_k), pf_sub, pf_slot);
+      pf_advance();
+    }
+    cp_async_commit();
+    pf_slot = (pf_slot + 1) % kRingC;
+    cp_async_wait<kRingC - 1>();
+    __syncthreads();
+
+    const uint8_t* stg = ring + slot * kStageB;
+    const int t0 = (sseg * kSegC + cur_sub) * kStageTokC;
+    const int rows = min(kStageTokC, tok_pair - t0);
+    const int r = half * kTok + lane;                    // this lane's token in the stage
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int hh = hsel + 4 * e;
+      if (hh >= g) break;
+      // lane = token: q·k over rotated 16-byte chunks of the K row
+      float x = -INFINITY;
+      if (r < rows) {
+        const uint8_t* krow = stg + r * kRowB;
+        const float* qh = qs + hh * CH * QST;
+        float acc = 0.f;
+#pragma unroll 4
+        for (int c = 0; c < CH; ++c) {
+          const int cc = (c + lane) % CH;
+          const uint4 u = *reinterpret_cast<const uint4*>(krow + cc * 16);
+          const float4 qa = *reinterpret_cast<const float4*>(qh + cc * QST);
+          const float4 qb = *reinterpret_cast<const float4*>(qh + cc * QST + 4);
+          const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+          const float2 k0 = __bfloat1622float2(h2[0]), k1 = __bfloat1622float2(h2[1]);
+          const float2 k2 = __bfloat1622float2(h2[2]), k3 = __bfloat1622float2(h2[3]);
+          acc = fmaf(k0.x, qa.x, fmaf(k0.y, qa.y, fmaf(k1.x, qa.z, fmaf(k1.y, qa.w, acc))));
+          acc = fmaf(k2.x, qb.x, fmaf(k2.y, qb.y, fmaf(k3.x, qb.z, fmaf(k3.y, qb.w, acc))));
+        }
+        x = acc;
+      }
+      const float p = head_add_logits(S[e], x);
+      // lane = channel group: fold in the value rows of the warp's 32 tokens
+      const uint8_t* vbase = stg + kArrB + (half * kTok) * kRowB;
+      const int nt = min(kTok, rows - half * kTok);
+      for (int t = 0; t < nt; ++t) {
+        const float pt = __shfl_sync(0xffffffffu, p, t);
+        if (lane * 4 < D) {
+          const uint2 u = *reinterpret_cast<const uint2*>(vbase + t * kRowB + lane * 8);
+          const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+          const float2 c2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+          S[e].acc[0] = fmaf(pt, a.x, S[e].acc[0]);
+          S[e].acc[1] = fmaf(pt, a.y, S[e].acc[1]);
+          S[e].acc[2] = fmaf(pt, c2.x, S[e].acc[2]);
+          S[e].acc[3] = fmaf(pt, c2.y, S[e].acc[3]);
+        }
+      }
+    }
+    __syncthreads();
+    slot = (slot + 1) % kRingC;
+    if (++cur_sub >= stages_in(seg)) {
+      // end of segment: merge the two token halves of each head, subtract the
+      // zero-order terms of the segment's blocks, write the partial state
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int hh = hsel + 4 * e;
+        if (hh < g) head_store<D>(S[e], xs + warp * (D + 2), lane);
+        __syncthreads();
+        if (hh < g && half == 0) {
+          const float* o0 = xs + warp * (D + 2);
+          const float* o1 = xs + (warp + 1) * (D + 2);
+          HeadState T;
+          const float M = fmaxf(o0[0], o1[0]);
+          const float f0 = o0[0] == -INFINITY ? 0.f : fast_exp2(o0[0] - M);
+          const float f1 = o1[0] == -INFINITY ? 0.f : fast_exp2(o1[0] - M);
+          T.m = M;
+          T.l = lane == 0 ? o0[1] * f0 + o1[1] * f1 : 0.f;   // lane-partial sum: lane 0 holds it
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            T.acc[c] = lane * 4 < D ? o0[2 + lane * 4 + c] * f0 + o1[2 + lane * 4 + c] * f1 : 0.f;
+          if (zero_order) {
+            const int32_t* sel = idx + (size_t)pair * topk;
+            const int tb = sseg * kSegC * kStageTokC;
+            const int te = min(tok_pair, tb + kSegC * kStageTokC);
+            const float* qh = qs + hh * CH * QST;
+            for (int sidx = tb / blk; sidx * blk < te; ++sidx) {
+              if (sidx * blk < tb) continue;   // a block belongs to the segment holding its first token
+              const int j = sel[sidx];
+              const float* kr = st.kmean + ((size_t)pair * nb + j) * D;
+              float d = 0.f;
+              for (int c = lane; c < D; c += 32) d = fmaf(qh[(c / 8) * QST + (c % 8)], kr[c], d);
+              d = warp_sum(d);
+              const float cl = d + bias2;                  // the block's zero-order log2 weight
+              const float m_new = fmaxf(T.m, cl);
+              const float corr = T.m == -INFINITY ? 0.f : fast_exp2(T.m - m_new);
+              const float w = fast_exp2(cl - m_new);
+              T.l = T.l * corr - (lane == 0 ? w : 0.f);
+              const float* vr = st.vsum + ((size_t)pair * nb + j) * D;
+#pragma unroll
+              for (int c = 0; c < 4; ++c) {
+                const float vv = lane * 4 < D ? vr[lane * 4 + c] * inv_blk : 0.f;
+                T.acc[c] = T.acc[c] * corr - w * vv;
+              }
+              T.m = m_new;
+            }
+          }
+          head_store<D>(T, partc + (((size_t)b * Hq + kh * g + hh) * nsegC + sseg) * (D + 2), lane);
+        }
+        __syncthreads();
+      }
+      cur_sub = 0;
+      ++cur_seg_k;
+    }
+  }
+  cp_async_wait<0>();
+}
+
+// ---- D. merge ------------------------------------------------------------
+template <int D>
+__global__ void decode_combine_kernel(const float* __restrict__ parta, int nsegA, const float* __restrict__ partc,
+                                      int nsegC, int use_tail, int Hq, __nv_bfloat16* __restrict__ O) {
+  const int h = blockIdx.x, b = blockIdx.y, c = threadIdx.x;
+  const float* pa = parta + ((size_t)b * Hq + h) * nsegA * (D + 2);
+  const float* pc = partc + ((size_t)b * Hq + h) * nsegC * (D + 2);
+  float M = -INFINITY;
+  if (use_tail)
+    for (int s = 0; s < nsegA; ++s) M = fmaxf(M, pa[s * (D + 2)]);
+  for (int s = 0; s < nsegC; ++s) M = fmaxf(M, pc[s * (D + 2)]);
+  float L = 0.f, A = 0.f;
+  if (M != -INFINITY) {
+    if (use_tail)
+      for (int s = 0; s < nsegA; ++s) {
+        const float* r = pa + s * (D + 2);
         if (r[0] == -INFINITY) continue;
         const float f = fast_exp2(r[0] - M);
         L = fmaf(r[1], f, L);
         A = fmaf(r[2 + c], f, A);
       }
-    }
-    float* out = partial + (((size_t)b * Hq + kh * g + hh) * nsplit + split) * (D + 2);
-    if (c == 0) {
-      out[0] = M;
-      out[1] = L;
-    }
-    out[2 + c] = A;
-  }
-}
-
-// ---- 4. combine ----------------------------------------------------------
-template <int D>
-__global__ void decode_combine_kernel(const float* __restrict__ partial, int Hq, int nsplit,
-                                      __nv_bfloat16* __restrict__ O) {
-  const int h = blockIdx.x, b = blockIdx.y, c = threadIdx.x;
-  const float* p = partial + ((size_t)b * Hq + h) * nsplit * (D + 2);
-  float M = -INFINITY;
-  for (int s = 0; s < nsplit; ++s) M = fmaxf(M, p[s * (D + 2)]);
-  float L = 0.f, A = 0.f;
-  if (M != -INFINITY) {
-    for (int s = 0; s < nsplit; ++s) {
-      const float* r = p + s * (D + 2);
+    for (int s = 0; s < nsegC; ++s) {
+      const float* r = pc + s * (D + 2);
       if (r[0] == -INFINITY) continue;
       const float f = fast_exp2(r[0] - M);
       L = fmaf(r[1], f, L);
@@ -347,6 +608,17 @@ __global__ void decode_combine_kernel(const float* __restrict__ partial, int Hq,
   O[((size_t)b * Hq + h) * D + c] = __float2bfloat16_rn(L > 0.f ? A / L : 0.f);
 }
 
+int sm_count() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
 template <int D>
 sa_status launch_decode(const void* q, const void* Kc, const void* Vc, const sa_decode_shape& s,
                         const sa_block_stats& st, int topk, float scale, sa_tail_mode tail,
@@ -354,39 +626,65 @@ sa_status launch_decode(const void* q, const void* Kc, const void* Vc, const sa_
                         cudaStream_t stream) {
   const DecodeLayout L = decode_layout(s, topk);
   const int nb = s.N / s.block;
+  const int npairs = s.B * s.Hkv;
   float* scores = scores_out ? scores_out : reinterpret_cast<float*>(ws + L.scores_off);
   int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(ws + L.idx_off);
-  float* part = reinterpret_cast<float*>(ws + L.part_off);
+  float* parta = reinterpret_cast<float*>(ws + L.parta_off);
+  float* partc = reinterpret_cast<float*>(ws + L.partc_off);
   const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(q);
+  const int sms = sm_count();
 
-  dim3 g1((nb + kScoreChunk - 1) / kScoreChunk, s.Hkv, s.B);
-  decode_score_kernel<D><<<g1, kDecThreads, 0, stream>>>(qb, st, s.Hq, s.Hkv, nb, scale, scores);
-  sa_status r = launch_status("decode_score_kernel");
+  // A
+  const size_t smemA = sizeof(float) * (2 * kMaxGroup * D + kMaxGroup * kStageBlocksA) +
+                       (size_t)kRingA * 3 * kStageBlocksA * D * 4;
+  if (cudaFuncSetAttribute(decode_stats_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smemA) !=
+      cudaSuccess)
+    return launch_status("cudaFuncSetAttribute(decode_stats_kernel)");
+  const long segsA = (long)npairs * L.nsegA;
+  const int gridA = (int)(segsA < sms ? segsA : sms);
+  decode_stats_kernel<D><<<gridA, kDecThreads, smemA, stream>>>(qb, st, s.Hq, s.Hkv, nb, s.block, scale,
+                                                                 L.nsegA, npairs, scores, parta);
+  sa_status r = launch_status("decode_stats_kernel");
   if (r != SA_OK) return r;
 
-  int n2 = 1;
-  while (n2 < nb) n2 <<= 1;
-  const size_t smem2 = (size_t)n2 * 8 + (size_t)nb * 4;
-  if (smem2 > 48 * 1024 &&
-      cudaFuncSetAttribute(decode_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2) != cudaSuccess)
-    return launch_status("cudaFuncSetAttribute(decode_topk_kernel)");
-  decode_topk_kernel<<<dim3(s.Hkv, s.B), kDecThreads, smem2, stream>>>(scores, s.Hkv, nb, topk, idx);
-  r = launch_status("decode_topk_kernel");
-  if (r != SA_OK) return r;
+  // B
+  if (topk > 0) {
+    size_t smemB;
+    if (topk > kTopkWarpMax) {
+      int n2 = 1;
+      while (n2 < nb) n2 <<= 1;
+      smemB = (size_t)n2 * 8 + (size_t)nb * 4;
+    } else {
+      smemB = (size_t)kDecWarps * kTopkWarpMax * 8 + (size_t)((nb + 31) / 32) * 4;
+    }
+    if (smemB > 48 * 1024 &&
+        cudaFuncSetAttribute(decode_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smemB) !=
+            cudaSuccess)
+      return launch_status("cudaFuncSetAttribute(decode_topk_kernel)");
+    decode_topk_kernel<<<npairs, kDecThreads, smemB, stream>>>(scores, nb, topk, idx);
+    r = launch_status("decode_topk_kernel");
+    if (r != SA_OK) return r;
+  }
 
-  const int nwords = (nb + 31) / 32;
-  const size_t smem3 = sizeof(float) * kMaxGroup * D + sizeof(uint32_t) * ((nwords + 3) & ~3) +
-                       sizeof(float) * kDecWarps * kMaxGroup * (D + 2);
-  if (smem3 > 48 * 1024 &&
-      cudaFuncSetAttribute(decode_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem3) != cudaSuccess)
-    return launch_status("cudaFuncSetAttribute(decode_attn_kernel)");
-  decode_attn_kernel<D><<<dim3(L.nsplit, s.Hkv, s.B), kDecThreads, smem3, stream>>>(
-      qb, static_cast<const __nv_bfloat16*>(Kc), static_cast<const __nv_bfloat16*>(Vc), st, s.Hq,
-      s.Hkv, s.N, s.block, idx, topk, (int)tail, scale, L.nsplit, part);
-  r = launch_status("decode_attn_kernel");
-  if (r != SA_OK) return r;
+  // C
+  if (topk > 0) {
+    const size_t smemC = sizeof(float) * (kMaxGroup * (D / 8) * 12 + kDecWarps * (D + 2)) +
+                         (size_t)kRingC * 2 * kStageTokC * D * 2;
+    if (cudaFuncSetAttribute(decode_exact_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smemC) !=
+        cudaSuccess)
+      return launch_status("cudaFuncSetAttribute(decode_exact_kernel)");
+    const long segsC = (long)npairs * L.nsegC;
+    const int gridC = (int)(segsC < sms ? segsC : sms);
+    decode_exact_kernel<D><<<gridC, kDecThreads, smemC, stream>>>(
+        qb, static_cast<const __nv_bfloat16*>(Kc), static_cast<const __nv_bfloat16*>(Vc), st, s.Hq, s.Hkv, s.N,
+        s.block, idx, topk, tail == SA_TAIL_ZERO_ORDER, scale, L.nsegC, npairs, partc);
+    r = launch_status("decode_exact_kernel");
+    if (r != SA_OK) return r;
+  }
 
-  decode_combine_kernel<D><<<dim3(s.Hq, s.B), D, 0, stream>>>(part, s.Hq, L.nsplit,
+  // D
+  decode_combine_kernel<D><<<dim3(s.Hq, s.B), D, 0, stream>>>(parta, L.nsegA, partc, topk > 0 ? L.nsegC : 0,
+                                                             tail == SA_TAIL_ZERO_ORDER, s.Hq,
                                                              static_cast<__nv_bfloat16*>(O));
   return launch_status("decode_combine_kernel");
 }
