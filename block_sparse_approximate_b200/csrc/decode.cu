@@ -134,40 +134,37 @@ decode_stats_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int 
   uint8_t* ring = reinterpret_cast<uint8_t*>(lsm + kMaxGroup * kStageBlocksA);
   const int g = Hq / Hkv;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int stages_per_seg_full = kSegA;
   const int nstage_pair = (nb + kStageBlocksA - 1) / kStageBlocksA;
-  const long total_segs = (long)npairs * nsegA;
+  const int total_segs = npairs * nsegA;
   const float bias2 = log2f((float)blk);
   const float inv_blk = 1.0f / blk;
 
   // the CTA's stage sequence: its segments in order, each segment's stages
-  auto seg_of = [&](long k_seg) { return (long)blockIdx.x + k_seg * gridDim.x; };
-  auto stages_in = [&](long seg) {
-    const int sseg = (int)(seg % nsegA);
-    const int first = sseg * stages_per_seg_full;
-    return min(stages_per_seg_full, nstage_pair - first);
-  };
+  auto seg_of = [&](int k_seg) { return (int)blockIdx.x + k_seg * (int)gridDim.x; };
+  auto stages_in = [&](int seg) { return min(kSegA, nstage_pair - (seg % nsegA) * kSegA); };
   // issue the copies of stage `sub` of segment `seg` into ring slot `slot`
-  auto issue = [&](long seg, int sub, int slot) {
-    const int pair = (int)(seg / nsegA), sseg = (int)(seg % nsegA);
-    const int j0 = (sseg * stages_per_seg_full + sub) * kStageBlocksA;
-    const int rows = min(kStageBlocksA, nb - j0);
+  auto issue = [&](int seg, int sub, int slot) {
+    const int pair = seg / nsegA, sseg = seg % nsegA;
+    const int j0 = (sseg * kSegA + sub) * kStageBlocksA;
+    const int n16 = min(kStageBlocksA, nb - j0) * (int)(kRowB / 16);
     const size_t goff = ((size_t)pair * nb + j0) * D;
     uint8_t* dst = ring + slot * kStageB;
-    const int n16 = rows * (int)(kRowB / 16);
-    for (int x = tid; x < 3 * n16; x += kDecThreads) {
-      const int a = x / n16, o = x % n16;
-      const float* src = (a == 0 ? st.kmean : a == 1 ? st.kvar : st.vsum) + goff;
-      cp_async16(dst + a * kArrB + o * 16, reinterpret_cast<const uint8_t*>(src) + o * 16);
+    const uint8_t* src0 = reinterpret_cast<const uint8_t*>(st.kmean + goff);
+    const uint8_t* src1 = reinterpret_cast<const uint8_t*>(st.kvar + goff);
+    const uint8_t* src2 = reinterpret_cast<const uint8_t*>(st.vsum + goff);
+    for (int o = tid; o < n16; o += kDecThreads) {
+      cp_async16(dst + o * 16, src0 + o * 16);
+      cp_async16(dst + kArrB + o * 16, src1 + o * 16);
+      cp_async16(dst + 2 * kArrB + o * 16, src2 + o * 16);
     }
   };
 
   // flat iteration over (segment, stage) pairs of this CTA
-  long cur_seg_k = 0;
+  int cur_seg_k = 0;
   if (seg_of(0) >= total_segs) return;
   int cur_sub = 0;
   // lookahead cursor for prefetching
-  long pf_seg_k = 0;
+  int pf_seg_k = 0;
   int pf_sub = 0;
   auto pf_valid = [&]() { return seg_of(pf_seg_k) < total_segs; };
   auto pf_advance = [&]() {
@@ -190,8 +187,8 @@ decode_stats_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int 
   int cur_pair = -1;
   int slot = 0;
   while (seg_of(cur_seg_k) < total_segs) {
-    const long seg = seg_of(cur_seg_k);
-    const int pair = (int)(seg / nsegA), sseg = (int)(seg % nsegA);
+    const int seg = seg_of(cur_seg_k);
+    const int pair = seg / nsegA, sseg = seg % nsegA;
     const int b = pair / Hkv, kh = pair % Hkv;
     if (cur_sub == 0) {
       if (pair != cur_pair) {
@@ -221,7 +218,7 @@ decode_stats_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int 
     const float* km = reinterpret_cast<const float*>(stg);
     const float* kv = reinterpret_cast<const float*>(stg + kArrB);
     const float* vs = reinterpret_cast<const float*>(stg + 2 * kArrB);
-    const int j0 = (sseg * stages_per_seg_full + cur_sub) * kStageBlocksA;
+    const int j0 = (sseg * kSegA + cur_sub) * kStageBlocksA;
     const int rows = min(kStageBlocksA, nb - j0);
     if (warp < g) {
       // lane = block: dot products over rotated float4 chunks (conflict free)
@@ -232,13 +229,22 @@ decode_stats_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int 
         const float4* vr = reinterpret_cast<const float4*>(kv + lane * D);
         const float4* qr = reinterpret_cast<const float4*>(qs + hh * D);
         const float4* wr = reinterpret_cast<const float4*>(ws + hh * D);
+        float a1[4] = {0.f, 0.f, 0.f, 0.f}, a2[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 8
         for (int c = 0; c < CH; ++c) {
           const int cc = (c + lane) % CH;
           const float4 a = kr[cc], qv = qr[cc], vv = vr[cc], wv = wr[cc];
-          d1 = fmaf(a.x, qv.x, fmaf(a.y, qv.y, fmaf(a.z, qv.z, fmaf(a.w, qv.w, d1))));
-          d2 = fmaf(vv.x, wv.x, fmaf(vv.y, wv.y, fmaf(vv.z, wv.z, fmaf(vv.w, wv.w, d2))));
+          a1[0] = fmaf(a.x, qv.x, a1[0]);
+          a1[1] = fmaf(a.y, qv.y, a1[1]);
+          a1[2] = fmaf(a.z, qv.z, a1[2]);
+          a1[3] = fmaf(a.w, qv.w, a1[3]);
+          a2[0] = fmaf(vv.x, wv.x, a2[0]);
+          a2[1] = fmaf(vv.y, wv.y, a2[1]);
+          a2[2] = fmaf(vv.z, wv.z, a2[2]);
+          a2[3] = fmaf(vv.w, wv.w, a2[3]);
         }
+        d1 = (a1[0] + a1[1]) + (a1[2] + a1[3]);
+        d2 = (a2[0] + a2[1]) + (a2[2] + a2[3]);
       }
       // d1 = s log2e q·k̄: natural log score s q·k̄ + log1p(½ s² Σ q² var)
       const float lnat = d1 * kLn2 + log1pf(d2);
@@ -318,14 +324,21 @@ decode_topk_kernel(const float* __restrict__ scores, int nb, int topk, int32_t* 
   const int nwords = (nb + 31) / 32;
   uint32_t* bits = reinterpret_cast<uint32_t*>(cand + kDecWarps * kTopkWarpMax);
   for (int x = tid; x < nwords; x += kDecThreads) bits[x] = 0u;
-  // stage 1: per warp, the k best of scores j = warp*32 + lane + 256 i
+  // stage 1: per warp, the k best of scores j = warp*32 + lane + 256 i (the
+  // row is at most 4096 long: 16 keys per lane, held in registers)
+  constexpr int KPL = kMaxRouteBlocks / kDecThreads;
+  unsigned long long key[KPL];
+#pragma unroll
+  for (int e = 0; e < KPL; ++e) {
+    const int j = warp * 32 + lane + e * kDecThreads;
+    key[e] = j < nb ? rank_key_d(sc[j], j) : ~0ull;
+  }
   unsigned long long prev = 0ull;
   for (int r = 0; r < topk; ++r) {
     unsigned long long mine = ~0ull;
-    for (int j = warp * 32 + lane; j < nb; j += kDecThreads) {
-      const unsigned long long k = rank_key_d(sc[j], j);
-      if ((r == 0 || k > prev) && k < mine) mine = k;
-    }
+#pragma unroll
+    for (int e = 0; e < KPL; ++e)
+      if ((r == 0 || key[e] > prev) && key[e] < mine) mine = key[e];
     const unsigned long long best = warp_min_u64d(mine);
     if (lane == 0) cand[warp * kTopkWarpMax + r] = best;
     prev = best;
@@ -333,14 +346,18 @@ decode_topk_kernel(const float* __restrict__ scores, int nb, int topk, int32_t* 
   __syncthreads();
   // stage 2: the k best of the warps' candidates (absent ones are all ones)
   if (warp == 0) {
+    unsigned long long ck[kDecWarps * kTopkWarpMax / 32];
+#pragma unroll
+    for (int e = 0; e < kDecWarps * kTopkWarpMax / 32; ++e) {
+      const int x = lane + 32 * e;                      // candidate x = (warp x / 64, rank x % 64)
+      ck[e] = (x % kTopkWarpMax) < topk ? cand[x] : ~0ull;
+    }
     prev = 0ull;
-    const int ncand = kDecWarps * topk;
     for (int r = 0; r < topk; ++r) {
       unsigned long long mine = ~0ull;
-      for (int x = lane; x < ncand; x += 32) {
-        const unsigned long long k = cand[(x / topk) * kTopkWarpMax + (x % topk)];
-        if ((r == 0 || k > prev) && k < mine) mine = k;
-      }
+#pragma unroll
+      for (int e = 0; e < kDecWarps * kTopkWarpMax / 32; ++e)
+        if ((r == 0 || ck[e] > prev) && ck[e] < mine) mine = ck[e];
       const unsigned long long best = warp_min_u64d(mine);
       if (lane == 0 && best != ~0ull) {
         const int jb = (int)(best & 0xffffffffu);
@@ -387,44 +404,61 @@ decode_exact_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
   extern __shared__ __align__(16) uint8_t dsm[];
   float* qs = reinterpret_cast<float*>(dsm);                         // [g][CH][QST]
   float* xs = qs + kMaxGroup * CH * QST;                             // merge scratch [8 warps][D+2]
-  uint8_t* ring = reinterpret_cast<uint8_t*>(xs + kDecWarps * (D + 2));
+  // centroid rows of the segments in flight: [kCenSlots][segment blocks][kmean, vsum][D]
+  // (prefetching runs at most kRingC - 1 stages, hence segments, ahead)
+  float* cen = xs + kDecWarps * (D + 2);
+  constexpr int kSegBlocksMax = kSegC * kStageTokC / 64;             // blocks of a segment (blk >= 64)
+  constexpr int kCenSlots = kRingC;
+  uint8_t* ring = reinterpret_cast<uint8_t*>(cen + kCenSlots * kSegBlocksMax * 2 * D);
   const int g = Hq / Hkv;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nb = N / blk;
   const int tok_pair = topk * blk;                  // exact tokens of one (sequence, KV head)
   const int nstage_pair = (tok_pair + kStageTokC - 1) / kStageTokC;
-  const long total_segs = (long)npairs * nsegC;
+  const int total_segs = npairs * nsegC;
   const float scale2 = scale * kLog2e;
   const float bias2 = log2f((float)blk);
   const float inv_blk = 1.0f / blk;
   // warp w: token half (w & 1) of the stage, heads hh with hh % 4 == w >> 1
   const int half = warp & 1, hsel = warp >> 1;
 
-  auto seg_of = [&](long k_seg) { return (long)blockIdx.x + k_seg * gridDim.x; };
-  auto stages_in = [&](long seg) {
-    const int sseg = (int)(seg % nsegC);
-    return min(kSegC, nstage_pair - sseg * kSegC);
-  };
-  auto issue = [&](long seg, int sub, int slot) {
-    const int pair = (int)(seg / nsegC), sseg = (int)(seg % nsegC);
+  auto seg_of = [&](int k_seg) { return (int)blockIdx.x + k_seg * (int)gridDim.x; };
+  auto stages_in = [&](int seg) { return min(kSegC, nstage_pair - (seg % nsegC) * kSegC); };
+  // a stage is 64 consecutive tokens of one selected block (64 divides blk)
+  auto issue = [&](int seg, int sub, int slot) {
+    const int pair = seg / nsegC, sseg = seg % nsegC;
     const int t0 = (sseg * kSegC + sub) * kStageTokC;     // first exact token of the stage
-    const int32_t* sel = idx + (size_t)pair * topk;
+    const int tok0 = __ldg(idx + (size_t)pair * topk + t0 / blk) * blk + (t0 % blk);
+    const size_t off = ((size_t)pair * N + tok0) * D;
+    const uint8_t* ks = reinterpret_cast<const uint8_t*>(Kc + off);
+    const uint8_t* vsrc = reinterpret_cast<const uint8_t*>(Vc + off);
     uint8_t* dst = ring + slot * kStageB;
-    const size_t base = (size_t)pair * N * D;
-    const int rows = min(kStageTokC, tok_pair - t0);
-    const int n16 = rows * CH;
-    for (int x = tid; x < 2 * n16; x += kDecThreads) {
-      const int a = x / n16, o = x % n16;
-      const int r = o / CH, c = o % CH;
-      const int t = t0 + r;
-      const int tok = sel[t / blk] * blk + (t % blk);
-      const __nv_bfloat16* src = (a == 0 ? Kc : Vc) + base + (size_t)tok * D + c * 8;
-      cp_async16(dst + a * kArrB + r * kRowB + c * 16, src);
+    const int n16 = min(kStageTokC, tok_pair - t0) * CH;
+    for (int o = tid; o < n16; o += kDecThreads) {
+      cp_async16(dst + o * 16, ks + o * 16);
+      cp_async16(dst + kArrB + o * 16, vsrc + o * 16);
+    }
+  };
+  // the kmean and vsum rows of a segment's selected blocks (zero-order only),
+  // into centroid slot `cslot`; issued with the segment's first stage, so the
+  // wait for that stage also covers them
+  auto issue_centroids = [&](int seg, int cslot) {
+    float* cb = cen + cslot * kSegBlocksMax * 2 * D;
+    const int pair = seg / nsegC, sseg = seg % nsegC;
+    const int s0 = sseg * kSegC * kStageTokC / blk;
+    const int s1 = min(topk, ((sseg + 1) * kSegC * kStageTokC) / blk);
+    constexpr int R16 = D * 4 / 16;
+    for (int o = tid; o < (s1 - s0) * R16; o += kDecThreads) {
+      const int sidx = s0 + o / R16, c = o % R16;
+      const int j = __ldg(idx + (size_t)pair * topk + sidx);
+      const size_t row = ((size_t)pair * nb + j) * D;
+      cp_async16(cb + ((sidx - s0) * 2 + 0) * D + c * 4, st.kmean + row + c * 4);
+      cp_async16(cb + ((sidx - s0) * 2 + 1) * D + c * 4, st.vsum + row + c * 4);
     }
   };
 
   if (seg_of(0) >= total_segs) return;
-  long pf_seg_k = 0;
+  int pf_seg_k = 0;
   int pf_sub = 0;
   auto pf_valid = [&]() { return seg_of(pf_seg_k) < total_segs; };
   auto pf_advance = [&]() {
@@ -434,21 +468,23 @@ decode_exact_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
     }
   };
   int pf_slot = 0;
-  for (int r = 0; r < kRingC - 1; ++r) {
+  auto prefetch = [&]() {
     if (pf_valid()) {
+      if (zero_order && pf_sub == 0) issue_centroids(seg_of(pf_seg_k), pf_seg_k % kCenSlots);
       issue(seg_of(pf_seg_k), pf_sub, pf_slot);
       pf_advance();
     }
     cp_async_commit();
     pf_slot = (pf_slot + 1) % kRingC;
-  }
+  };
+  for (int r = 0; r < kRingC - 1; ++r) prefetch();
 
   HeadState S[2];
-  long cur_seg_k = 0;
+  int cur_seg_k = 0;
   int cur_sub = 0, cur_pair = -1, slot = 0;
   while (seg_of(cur_seg_k) < total_segs) {
-    const long seg = seg_of(cur_seg_k);
-    const int pair = (int)(seg / nsegC), sseg = (int)(seg % nsegC);
+    const int seg = seg_of(cur_seg_k);
+    const int pair = seg / nsegC, sseg = seg % nsegC;
     const int b = pair / Hkv, kh = pair % Hkv;
     if (cur_sub == 0) {
       if (pair != cur_pair) {
@@ -463,12 +499,7 @@ decode_exact_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
       head_reset(S[0]);
       head_reset(S[1]);
     }
-    if (pf_valid()) {
-      issue(seg_of(pf_seg_k), pf_sub, pf_slot);
-      pf_advance();
-    }
-    cp_async_commit();
-    pf_slot = (pf_slot + 1) % kRingC;
+    prefetch();
     cp_async_wait<kRingC - 1>();
     __syncthreads();
 
@@ -485,7 +516,7 @@ decode_exact_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
       if (r < rows) {
         const uint8_t* krow = stg + r * kRowB;
         const float* qh = qs + hh * CH * QST;
-        float acc = 0.f;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 4
         for (int c = 0; c < CH; ++c) {
           const int cc = (c + lane) % CH;
@@ -495,10 +526,12 @@ decode_exact_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
           const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
           const float2 k0 = __bfloat1622float2(h2[0]), k1 = __bfloat1622float2(h2[1]);
           const float2 k2 = __bfloat1622float2(h2[2]), k3 = __bfloat1622float2(h2[3]);
-          acc = fmaf(k0.x, qa.x, fmaf(k0.y, qa.y, fmaf(k1.x, qa.z, fmaf(k1.y, qa.w, acc))));
-          acc = fmaf(k2.x, qb.x, fmaf(k2.y, qb.y, fmaf(k3.x, qb.z, fmaf(k3.y, qb.w, acc))));
+          acc[0] = fmaf(k0.x, qa.x, fmaf(k0.y, qa.y, acc[0]));
+          acc[1] = fmaf(k1.x, qa.z, fmaf(k1.y, qa.w, acc[1]));
+          acc[2] = fmaf(k2.x, qb.x, fmaf(k2.y, qb.y, acc[2]));
+          acc[3] = fmaf(k3.x, qb.z, fmaf(k3.y, qb.w, acc[3]));
         }
-        x = acc;
+        x = (acc[0] + acc[1]) + (acc[2] + acc[3]);
       }
       const float p = head_add_logits(S[e], x);
       // lane = channel group: fold in the value rows of the warp's 32 tokens
@@ -540,14 +573,13 @@ decode_exact_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
           for (int c = 0; c < 4; ++c)
             T.acc[c] = lane * 4 < D ? o0[2 + lane * 4 + c] * f0 + o1[2 + lane * 4 + c] * f1 : 0.f;
           if (zero_order) {
-            const int32_t* sel = idx + (size_t)pair * topk;
             const int tb = sseg * kSegC * kStageTokC;
             const int te = min(tok_pair, tb + kSegC * kStageTokC);
             const float* qh = qs + hh * CH * QST;
             for (int sidx = tb / blk; sidx * blk < te; ++sidx) {
-              if (sidx * blk < tb) continue;   // a block belongs to the segment holding its first token
-              const int j = sel[sidx];
-              const float* kr = st.kmean + ((size_t)pair * nb + j) * D;
+              // rows staged by issue_centroids with the segment's first stage
+              const float* cb = cen + (cur_seg_k % kCenSlots) * kSegBlocksMax * 2 * D;
+              const float* kr = cb + ((sidx - tb / blk) * 2 + 0) * D;
               float d = 0.f;
               for (int c = lane; c < D; c += 32) d = fmaf(qh[(c / 8) * QST + (c % 8)], kr[c], d);
               d = warp_sum(d);
@@ -556,7 +588,7 @@ decode_exact_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
               const float corr = T.m == -INFINITY ? 0.f : fast_exp2(T.m - m_new);
               const float w = fast_exp2(cl - m_new);
               T.l = T.l * corr - (lane == 0 ? w : 0.f);
-              const float* vr = st.vsum + ((size_t)pair * nb + j) * D;
+              const float* vr = cb + ((sidx - tb / blk) * 2 + 1) * D;
 #pragma unroll
               for (int c = 0; c < 4; ++c) {
                 const float vv = lane * 4 < D ? vr[lane * 4 + c] * inv_blk : 0.f;
@@ -668,12 +700,13 @@ sa_status launch_decode(const void* q, const void* Kc, const void* Vc, const sa_
 
   // C
   if (topk > 0) {
-    const size_t smemC = sizeof(float) * (kMaxGroup * (D / 8) * 12 + kDecWarps * (D + 2)) +
+    const size_t smemC = sizeof(float) * (kMaxGroup * (D / 8) * 12 + kDecWarps * (D + 2) +
+                                          kRingC * (kSegC * kStageTokC / 64) * 2 * D) +
                          (size_t)kRingC * 2 * kStageTokC * D * 2;
     if (cudaFuncSetAttribute(decode_exact_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smemC) !=
         cudaSuccess)
       return launch_status("cudaFuncSetAttribute(decode_exact_kernel)");
-    const long segsC = (long)npairs * L.nsegC;
+    const long segsC = (long)npairs * L.nsegC;   // < 2^31 for any supported shape
     const int gridC = (int)(segsC < sms ? segsC : sms);
     decode_exact_kernel<D><<<gridC, kDecThreads, smemC, stream>>>(
         qb, static_cast<const __nv_bfloat16*>(Kc), static_cast<const __nv_bfloat16*>(Vc), st, s.Hq, s.Hkv, s.N,
