@@ -38,9 +38,10 @@ def _headers():
     return sorted(glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(INCLUDE, "*.h")))
 
 
-# attn_tc_kernel reallocates registers with setmaxnreg: its launch register
-# count times 384 threads must cover 256 x 216 + 128 x 40 (see attn_tc.cu), or
-# setmaxnreg.inc would wait for registers that never come.
+# attn_tc_kernel and attn_tc_linmix_kernel reallocate registers with
+# setmaxnreg: their launch register count times 384 threads must cover the
+# split (256 x 216 + 128 x 40, and 128 x 216 + 128 x 96 + 128 x 40; see
+# attn_tc.cu), or setmaxnreg.inc would wait for registers that never come.
 TC_MIN_LAUNCH_REGS = 158
 
 
@@ -48,7 +49,7 @@ def _check_tc_registers(ptxas_log: str):
     import re
     lines = ptxas_log.splitlines()
     for k, line in enumerate(lines):
-        if "Compiling entry function" in line and "attn_tc_kernel" in line:
+        if "Compiling entry function" in line and ("attn_tc_kernel" in line or "attn_tc_linmix_kernel" in line):
             for nxt in lines[k + 1:k + 4]:
                 m = re.search(r"Used (\d+) registers", nxt)
                 if m:

@@ -548,23 +548,417 @@ sa_status launch_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensor
   return launch_status("attn_tc_kernel");
 }
 
+// ---------------------------------------------------------------- linear mix
+// SLA2 §2A mixture O = α⊙O_s + (1−α)⊙O_l on the tensor cores.  O_s is the
+// exact softmax over the selected blocks; O_l is the ReLU linear attention
+// (SALAD §2) over the unselected blocks in SPLA §2.2's subtraction form:
+//   O_l = relu(q)ᵀ (H_tot − A_i) / (relu(q)·(z_tot − ζ_i) + eps),
+//   A_i = Σ_{j∈S_i} relu(K_j)ᵀ V_j,  ζ_i = Σ_{j∈S_i} z_j,
+// with A_i accumulated by the MMA warp from the K/V tiles already in shared
+// memory (unselected blocks are never read).  TMEM (512 columns): S0, S1 (the
+// double-buffered score tile), O (the softmax accumulator), A (A_i, d×d).
+// Warps 0-3 run the softmax of every tile; warps 4-7 apply ReLU in place to
+// each K tile once its S MMA has finished with it, then build the epilogue's
+// operands (relu(Q) in place, D = H_tot − A_i as a bf16 tile, ζ_i); warp 8 is
+// the TMA producer, warp 9 the MMA issuer.
+struct LinLayout {
+  static constexpr int NS = 3;
+  static constexpr uint32_t kTile = 2 * kSpan;
+  static constexpr int B_Q = 0, B_KF = 1, B_VF = B_KF + NS, B_KE = B_VF + NS, B_SF = B_KE + NS,
+                       B_PR = B_SF + 2, B_RL = B_PR + 2, B_OD = B_RL + 2, B_LAST = B_OD + 1,
+                       B_EPI_IN = B_LAST + 1, B_EPI = B_EPI_IN + 1, B_FIN = B_EPI + 1, NBAR = B_FIN + 1;
+  static constexpr uint32_t kBarOff = kTile * (1 + 2 * NS);
+  static constexpr uint32_t kSlotOff = kBarOff + 8 * NBAR;   // tmem base, abort flag
+  static constexpr uint32_t kZetaOff = kSlotOff + 16;        // ζ_i: TD floats
+  static constexpr uint32_t kEnd = kZetaOff + TD * 4;
+  static size_t smem_bytes() { return 1024 + kEnd; }
+};
+constexpr uint32_t kColA = 384;
+constexpr int kReluRegs = 96;
+
+__global__ void __launch_bounds__(kTcThreads, 1)
+attn_tc_linmix_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                      const __grid_constant__ CUtensorMap tmV, const int32_t* __restrict__ block_idx, int nb,
+                      int topk, float scale2, const float* __restrict__ alpha, const float* __restrict__ zrelu,
+                      const float* __restrict__ htot, const float* __restrict__ ztot, int H,
+                      __nv_bfloat16* __restrict__ O, int N) {
+  using L = LinLayout;
+  constexpr int NS = L::NS;
+  constexpr uint32_t kTile = L::kTile;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(smem);
+  const int i = blockIdx.x, bh = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kSlotOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kSlotOff + 4);
+  float* zeta = reinterpret_cast<float*>(smem + L::kZetaOff);
+  auto bar = [&](int k) { return sb + L::kBarOff + 8u * k; };
+  const int T = topk;
+  const int32_t* sel = block_idx + ((size_t)bh * nb + i) * topk;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(L::B_Q), 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(bar(L::B_KF + s), 1);
+      mbar_init(bar(L::B_VF + s), 1);
+      mbar_init(bar(L::B_KE + s), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(L::B_SF + s), 1);
+      mbar_init(bar(L::B_PR + s), 128);
+      mbar_init(bar(L::B_RL + s), 128);
+    }
+    mbar_init(bar(L::B_OD), 1);
+    mbar_init(bar(L::B_LAST), 1);
+    mbar_init(bar(L::B_EPI_IN), 256);
+    mbar_init(bar(L::B_EPI), 1);
+    mbar_init(bar(L::B_FIN), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+
+  if (warp == kTmaWarp) {
+    // ------------------------------------------------------------ producer
+    regs_dec<kProducerRegs>();
+    if (lane == 0) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      mbar_expect_tx(bar(L::B_Q), kTile);
+      tma_load_3d(sb, &tmQ, 0, i * TB, bh, bar(L::B_Q));
+      tma_load_3d(sb + kSpan, &tmQ, 64, i * TB, bh, bar(L::B_Q));
+      int issued = 0;
+      for (int t = 0; t < T; ++t) {
+        const int s = t % NS;
+        if (t >= NS && !mbar_wait(bar(L::B_KE + s), ((t / NS) - 1) & 1, abort_flag)) break;
+        const int row = sel[t] * TB;
+        const uint32_t ka = sb + kTile * (1 + 2 * s), va = ka + kTile;
+        mbar_expect_tx(bar(L::B_KF + s), kTile);
+        tma_load_3d(ka, &tmK, 0, row, bh, bar(L::B_KF + s));
+        tma_load_3d(ka + kSpan, &tmK, 64, row, bh, bar(L::B_KF + s));
+        mbar_expect_tx(bar(L::B_VF + s), kTile);
+        tma_load_3d(va, &tmV, 0, row, bh, bar(L::B_VF + s));
+        tma_load_3d(va + kSpan, &tmV, 64, row, bh, bar(L::B_VF + s));
+        issued = t + 1;
+      }
+      if (*abort_flag) {
+        wait_bounded(bar(L::B_Q), 0);
+        for (int t = issued > NS ? issued - NS : 0; t < issued; ++t) {
+          wait_bounded(bar(L::B_KF + t % NS), (t / NS) & 1);
+          wait_bounded(bar(L::B_VF + t % NS), (t / NS) & 1);
+        }
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    regs_dec<kProducerRegs>();
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16_f32(TB, TB, 0, 0);
+      constexpr uint32_t idO = idesc_bf16_f32(TB, TD, 0, 1);
+      constexpr uint32_t idA = idesc_bf16_f32(TD, TD, 1, 1);   // relu(K)ᵀ (MN-major) · V (MN-major)
+      const uint32_t colO = tbase + 256, colA = tbase + kColA;
+      auto issue_s = [&](int t) -> bool {
+        const int s = t % NS;
+        if (!mbar_wait(bar(L::B_KF + s), (t / NS) & 1, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t ka = sb + kTile * (1 + 2 * s);
+        const uint32_t d = tbase + (uint32_t)(t & 1) * TB;
+#pragma unroll
+        for (int k = 0; k < TD / 16; ++k) {
+          const uint32_t koff = (k >> 2) * kSpan + (k & 3) * 32;
+          mma_ss(d, desc_sw128(sb + koff, 16, 1024), desc_sw128(ka + koff, 16, 1024), idS, k > 0);
+        }
+        mma_commit(bar(L::B_SF + (t & 1)));
+        return true;
+      };
+      bool ok = mbar_wait(bar(L::B_Q), 0, abort_flag);
+      if (ok && T > 0) ok = issue_s(0);
+      if (ok && T > 1) ok = issue_s(1);
+      for (int t = 0; ok && t < T; ++t) {
+        const int su = t % NS, b2 = t & 1;
+        const uint32_t ka = sb + kTile * (1 + 2 * su), va = ka + kTile;
+        // A_i += relu(K_t)ᵀ V_t once warps 4-7 have applied the ReLU
+        if (!mbar_wait(bar(L::B_RL + b2), (t >> 1) & 1, abort_flag)) break;
+        if (!mbar_wait(bar(L::B_VF + su), (t / NS) & 1, abort_flag)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < TB / 16; ++k)
+          mma_ss(colA, desc_sw128(ka + k * 16 * 128, kSpan, 1024), desc_sw128(va + k * 16 * 128, kSpan, 1024),
+                 idA, (t > 0 || k > 0));
+        // O += P_t V_t
+        if (!mbar_wait(bar(L::B_PR + b2), (t >> 1) & 1, abort_flag)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < TB / 16; ++k)
+          mma_ts(colO, tbase + (uint32_t)b2 * TB + k * 8, desc_sw128(va + k * 16 * 128, kSpan, 1024), idO,
+                 (t > 0 || k > 0));
+        mma_commit(bar(L::B_KE + su));
+        mma_commit(bar(L::B_OD));
+        if (t + 2 < T && !issue_s(t + 2)) break;
+      }
+      mma_commit(bar(L::B_LAST));   // every MMA of the tile loop (or none) has completed
+      // epilogue: S0 = relu(Q) · (H_tot − A_i), operands prepared by warps 0-7
+      if (ok && mbar_wait(bar(L::B_EPI_IN), 0, abort_flag)) {
+        tc_fence_after();
+        const uint32_t dbase = sb + kTile;   // D tile in stage 0's K slot
+#pragma unroll
+        for (int k = 0; k < TD / 16; ++k) {
+          const uint32_t koff = (k >> 2) * kSpan + (k & 3) * 32;
+          mma_ss(tbase, desc_sw128(sb + koff, 16, 1024), desc_sw128(dbase + k * 16 * 128, kSpan, 1024),
+                 idO, k > 0);
+        }
+        mma_commit(bar(L::B_EPI));
+      }
+      mma_commit(bar(L::B_FIN));
+      wait_bounded(bar(L::B_FIN), 0);
+    }
+  } else if (warp >= 8) {
+    regs_dec<kProducerRegs>();
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ ReLU warps
+    regs_dec<kReluRegs>();
+    const int tr = threadIdx.x - 128;          // 0..127
+    bool ok = true;
+    for (int t = 0; t < T; ++t) {
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_SF + (t & 1)), (t >> 1) & 1, abort_flag))) {
+        ok = false;
+        break;
+      }
+      // the S MMA has read K_t: replace it by relu(K_t) in place (layout-free)
+      uint4* kt = reinterpret_cast<uint4*>(smem + kTile * (1 + 2 * (t % NS)));
+      const __nv_bfloat162 zero = __float2bfloat162_rn(0.f);
+#pragma unroll 4
+      for (int x = tr; x < (int)(kTile / 16); x += 128) {
+        uint4 u = kt[x];
+        __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) h[e] = __hmax2(h[e], zero);
+        kt[x] = u;
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_arrive(bar(L::B_RL + (t & 1)));
+    }
+    // ζ_i = Σ_{j∈S_i} z_j (channel tr)
+    float z = 0.f;
+    for (int s2 = 0; s2 < T; ++s2) z += zrelu[((size_t)bh * nb + sel[s2]) * TD + tr];
+    zeta[tr] = z;
+    // after the last MMA reading Q: relu(Q) in place
+    ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(L::B_LAST), 0, abort_flag));
+    if (ok) {
+      uint4* qt = reinterpret_cast<uint4*>(smem);
+      const __nv_bfloat162 zero = __float2bfloat162_rn(0.f);
+      for (int x = tr; x < (int)(kTile / 16); x += 128) {
+        uint4 u = qt[x];
+        __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) h[e] = __hmax2(h[e], zero);
+        qt[x] = u;
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    named_bar_softmax();          // zeta visible to warps 0-3
+    mbar_arrive(bar(L::B_EPI_IN));
+  } else {
+    // ------------------------------------------------------------ softmax
+    regs_inc<kSoftmaxRegs>();
+    const int r = warp * 32 + lane;
+    const uint32_t lrow = tbase + ((uint32_t)(warp * 32) << 16);
+    float m_used = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int t = 0; t < T; ++t) {
+      const int b2 = t & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_SF + b2), (t >> 1) & 1, abort_flag))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t v[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        tmem_ld32(lrow + b2 * TB + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * c]));
+      tmem_wait_ld();
+      float mx8[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) mx8[k] = -INFINITY;
+#pragma unroll
+      for (int n = 0; n < TB / 2; ++n)
+        mx8[n & 7] = fmax3(mx8[n & 7], __uint_as_float(v[2 * n]), __uint_as_float(v[2 * n + 1]));
+      const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                             fmaxf(mx8[6], mx8[7]));
+      const float m_tile = mx * scale2;
+      const float m_new = fmaxf(m_used, m_tile);
+      const bool need = m_new > m_used + Fmt<false>::kLazy;
+      float factor = 1.f;
+      if (need) {
+        factor = fast_exp2(m_used - m_new);
+        m_used = m_new;
+      }
+      const float neg = -m_used;
+      float sm8[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) sm8[k] = 0.f;
+#pragma unroll
+      for (int n = 0; n < TB / 2; ++n) {
+        float a0, a1;
+        ffma2(a0, a1, __uint_as_float(v[2 * n]), __uint_as_float(v[2 * n + 1]), scale2, scale2, neg, neg);
+        const float p0 = fast_exp2(a0), p1 = fast_exp2(a1);
+        fadd2(sm8[2 * (n & 3)], sm8[2 * (n & 3) + 1], p0, p1);
+        v[n] = pack_bf16(p0, p1);
+      }
+      l = l * factor + (((sm8[0] + sm8[1]) + (sm8[2] + sm8[3])) + ((sm8[4] + sm8[5]) + (sm8[6] + sm8[7])));
+      tmem_st32(lrow + b2 * TB, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+      tmem_st32(lrow + b2 * TB + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+      tmem_wait_st();
+      if (t >= 1) {
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_OD), (t - 1) & 1, abort_flag))) {
+          ok = false;
+          break;
+        }
+        if (__any_sync(0xffffffffu, need)) {
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t o[32];
+            tmem_ld32(lrow + 256 + 32 * c, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
+            tmem_st32(lrow + 256 + 32 * c, o);
+          }
+          tmem_wait_st();
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(L::B_PR + b2));
+    }
+    ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(L::B_LAST), 0, abort_flag));
+    // D = H_tot − A_i (row c = this thread's TMEM lane) as a bf16 MN-major tile
+    // in stage 0's K slot: span e/64, row c, 16-byte chunk (e%64)/8 xor (c%8)
+    if (ok) {
+      tc_fence_after();
+      const float* hrow = htot + ((size_t)bh * TD + r) * TD;
+      uint8_t* dt = smem + kTile;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t a[32];
+        if (T > 0) {
+          tmem_ld32(lrow + kColA + 32 * c, a);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) a[e] = 0u;
+        }
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const int e0 = 32 * c + 8 * q4;                  // first of 8 output channels
+          uint4 w;
+          w.x = pack_bf16(hrow[e0 + 0] - __uint_as_float(a[8 * q4 + 0]), hrow[e0 + 1] - __uint_as_float(a[8 * q4 + 1]));
+          w.y = pack_bf16(hrow[e0 + 2] - __uint_as_float(a[8 * q4 + 2]), hrow[e0 + 3] - __uint_as_float(a[8 * q4 + 3]));
+          w.z = pack_bf16(hrow[e0 + 4] - __uint_as_float(a[8 * q4 + 4]), hrow[e0 + 5] - __uint_as_float(a[8 * q4 + 5]));
+          w.w = pack_bf16(hrow[e0 + 6] - __uint_as_float(a[8 * q4 + 6]), hrow[e0 + 7] - __uint_as_float(a[8 * q4 + 7]));
+          const int span = e0 >> 6, chunk = (e0 & 63) >> 3;
+          *reinterpret_cast<uint4*>(dt + span * kSpan + r * 128 + ((chunk ^ (r & 7)) << 4)) = w;
+        }
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    named_bar_softmax();          // zeta ready (warps 4-7)
+    mbar_arrive(bar(L::B_EPI_IN));
+    ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(L::B_EPI), 0, abort_flag)) && !*abort_flag;
+    if (ok) {
+      tc_fence_after();
+      // relu(q_r)·(z_tot − ζ_i) from this row of the (now relu'd) Q tile
+      float den = kLinearEps;
+      const float* zt = ztot + (size_t)bh * TD;
+#pragma unroll 4
+      for (int ch = 0; ch < 16; ++ch) {            // 16-byte chunks of the 128 channels
+        const int span = ch >> 3, cc = ch & 7;
+        const uint4 u = *reinterpret_cast<const uint4*>(smem + span * kSpan + r * 128 + ((cc ^ (r & 7)) << 4));
+        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(h2[e]);
+          const int c0 = ch * 8 + 2 * e;
+          den = fmaf(f.x, zt[c0] - zeta[c0], den);
+          den = fmaf(f.y, zt[c0 + 1] - zeta[c0 + 1], den);
+        }
+      }
+      const bool u_empty = (topk == nb);            // no unselected block: O_l = 0
+      const float inv_den = u_empty ? 0.f : 1.0f / den;
+      const float inv_l = l > 0.f ? 1.0f / l : 0.f;
+      const float* al = alpha + (size_t)(bh % H) * TD;
+      uint4* orow = reinterpret_cast<uint4*>(O + ((size_t)bh * N + (size_t)i * TB + r) * TD);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t os[32], ol[32];
+        if (T > 0) tmem_ld32(lrow + 256 + 32 * c, os);
+        tmem_ld32(lrow + 32 * c, ol);
+        tmem_wait_ld();
+        if (T == 0) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) os[e] = 0u;
+        }
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          float y[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int ee = 32 * c + 8 * q4 + e;
+            const float a = al[ee];
+            y[e] = a * __uint_as_float(os[8 * q4 + e]) * inv_l + (1.0f - a) * __uint_as_float(ol[8 * q4 + e]) * inv_den;
+          }
+          uint4 w;
+          w.x = pack_bf16(y[0], y[1]);
+          w.y = pack_bf16(y[2], y[3]);
+          w.z = pack_bf16(y[4], y[5]);
+          w.w = pack_bf16(y[6], y[7]);
+          orow[4 * c + q4] = w;
+        }
+      }
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tbase, kTmemCols);
+  }
+}
+
 }  // namespace
 
 bool attn_tc_supports(sa_dtype dtype, const sa_shape& s, sa_tail_mode tail) {
   return dtype == SA_BF16 && s.block == TB && s.d == TD &&
-         (tail == SA_TAIL_DROP || tail == SA_TAIL_ZERO_ORDER);
+         (tail == SA_TAIL_DROP || tail == SA_TAIL_ZERO_ORDER || tail == SA_TAIL_LINEAR_MIX);
 }
 
 sa_status attn_tc(const void* Q, const void* K, const void* V, const sa_shape& s, const int32_t* block_idx,
                   int topk, sa_tail_mode tail, const float* alpha, const sa_block_stats& st, float scale,
                   void* O, cudaStream_t stream) {
-  (void)alpha;
   const int nb = s.N / TB;
   const uint64_t BH = (uint64_t)s.B * s.H;
   CUtensorMap mq, mk, mv, mkb, mvb;
   if (!make_tmap_3d(&mq, Q, 2, TD, s.N, BH) || !make_tmap_3d(&mk, K, 2, TD, s.N, BH) ||
       !make_tmap_3d(&mv, V, 2, TD, s.N, BH))
     return fail(SA_ERR_CUDA, "sa_sparse_attn_fwd: cuTensorMapEncodeTiled failed for Q/K/V");
+  if (tail == SA_TAIL_LINEAR_MIX) {
+    const size_t smem = LinLayout::smem_bytes();
+    if (cudaFuncSetAttribute(attn_tc_linmix_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+      return launch_status("cudaFuncSetAttribute(attn_tc_linmix_kernel)");
+    dim3 grid(nb, (unsigned)BH);
+    attn_tc_linmix_kernel<<<grid, kTcThreads, smem, stream>>>(mq, mk, mv, block_idx, nb, topk, scale * kLog2e,
+                                                              alpha, st.zrelu, st.htot, st.ztot, s.H,
+                                                              static_cast<__nv_bfloat16*>(O), s.N);
+    return launch_status("attn_tc_linmix_kernel");
+  }
   const bool zo = tail == SA_TAIL_ZERO_ORDER;
   if (zo) {
     if (!make_tmap_3d(&mkb, st.kmean_bf16, 2, TD, nb, BH) || !make_tmap_3d(&mvb, st.vmean_bf16, 2, TD, nb, BH))
