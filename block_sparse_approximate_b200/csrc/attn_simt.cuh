@@ -20,4 +20,9 @@ sa_status attn_tc(const void* Q, const void* K, const void* V, const sa_shape& s
 
 bool attn_tc_supports(sa_dtype dtype, const sa_shape& s, sa_tail_mode tail);
 
+// H_tot = Σ_n relu(k_n) v_nᵀ per head on the tensor cores (bf16, d = 128, N a
+// multiple of 128); adds into htot, which the caller zeroes first.  Returns
+// SA_ERR_UNSUPPORTED (without setting an error) for other shapes.
+sa_status htot_tc(const void* K, const void* V, const sa_shape& s, float* htot, cudaStream_t stream);
+
 }  // namespace sa

@@ -932,7 +932,166 @@ attn_tc_linmix_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
   }
 }
 
+// ---------------------------------------------------------------- H_tot
+// H_tot = Σ_n relu(k_n) v_nᵀ of one head (the total of SLA2's ReLU linear
+// branch, SALAD §2) on the tensor cores: a CTA takes a chunk of 128-token
+// tiles of one head, warps 2-5 apply ReLU in place to each K tile, warp 1
+// accumulates relu(K)ᵀ V in TMEM (MN-major × MN-major MMA), and the chunk's
+// d×d sum is added to htot with vector atomics.  Warp 0 is the TMA producer.
+constexpr int kHtThreads = 192;
+constexpr int kHtTiles = 32;          // tiles (of 128 tokens) per CTA
+struct HtLayout {
+  static constexpr int NS = 3;
+  static constexpr uint32_t kTile = 2 * kSpan;
+  static constexpr int B_KF = 0, B_VF = B_KF + NS, B_KE = B_VF + NS, B_RL = B_KE + NS, B_DONE = B_RL + NS,
+                       NBAR = B_DONE + 1;
+  static constexpr uint32_t kBarOff = 2 * kTile * NS;
+  static constexpr uint32_t kSlotOff = kBarOff + 8 * NBAR;
+  static size_t smem_bytes() { return 1024 + kSlotOff + 16; }
+};
+
+__global__ void __launch_bounds__(kHtThreads, 1)
+htot_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, int N,
+               float* __restrict__ htot) {
+  using L = HtLayout;
+  constexpr int NS = L::NS;
+  constexpr uint32_t kTile = L::kTile;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(smem);
+  const int chunk = blockIdx.x, bh = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kSlotOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kSlotOff + 4);
+  auto bar = [&](int k) { return sb + L::kBarOff + 8u * k; };
+  const int ntile_head = N / TB;
+  const int t0 = chunk * kHtTiles;
+  const int T = min(kHtTiles, ntile_head - t0);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(bar(L::B_KF + s), 1);
+      mbar_init(bar(L::B_VF + s), 1);
+      mbar_init(bar(L::B_KE + s), 1);
+      mbar_init(bar(L::B_RL + s), 128);
+    }
+    mbar_init(bar(L::B_DONE), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) tmem_alloc(smem_u32(tmem_slot), 128);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int issued = 0;
+      for (int t = 0; t < T; ++t) {
+        const int s = t % NS;
+        if (t >= NS && !mbar_wait(bar(L::B_KE + s), ((t / NS) - 1) & 1, abort_flag)) break;
+        const int row = (t0 + t) * TB;
+        const uint32_t ka = sb + 2 * kTile * s, va = ka + kTile;
+        mbar_expect_tx(bar(L::B_KF + s), kTile);
+        tma_load_3d(ka, &tmK, 0, row, bh, bar(L::B_KF + s));
+        tma_load_3d(ka + kSpan, &tmK, 64, row, bh, bar(L::B_KF + s));
+        mbar_expect_tx(bar(L::B_VF + s), kTile);
+        tma_load_3d(va, &tmV, 0, row, bh, bar(L::B_VF + s));
+        tma_load_3d(va + kSpan, &tmV, 64, row, bh, bar(L::B_VF + s));
+        issued = t + 1;
+      }
+      if (*abort_flag)
+        for (int t = issued > NS ? issued - NS : 0; t < issued; ++t) {
+          wait_bounded(bar(L::B_KF + t % NS), (t / NS) & 1);
+          wait_bounded(bar(L::B_VF + t % NS), (t / NS) & 1);
+        }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idA = idesc_bf16_f32(TD, TD, 1, 1);
+      for (int t = 0; t < T; ++t) {
+        const int s = t % NS;
+        if (!mbar_wait(bar(L::B_RL + s), (t / NS) & 1, abort_flag)) break;
+        if (!mbar_wait(bar(L::B_VF + s), (t / NS) & 1, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t ka = sb + 2 * kTile * s, va = ka + kTile;
+#pragma unroll
+        for (int k = 0; k < TB / 16; ++k)
+          mma_ss(tbase, desc_sw128(ka + k * 16 * 128, kSpan, 1024), desc_sw128(va + k * 16 * 128, kSpan, 1024),
+                 idA, (t > 0 || k > 0));
+        mma_commit(bar(L::B_KE + s));
+      }
+      mma_commit(bar(L::B_DONE));
+      wait_bounded(bar(L::B_DONE), 0);
+    }
+  } else {
+    // warps 2-5: ReLU of each K tile, then the epilogue (TMEM lane quarter w % 4)
+    const int tr = threadIdx.x - 64;
+    bool ok = true;
+    for (int t = 0; t < T; ++t) {
+      const int s = t % NS;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_KF + s), (t / NS) & 1, abort_flag))) {
+        ok = false;
+        break;
+      }
+      uint4* kt = reinterpret_cast<uint4*>(smem + 2 * kTile * s);
+      const __nv_bfloat162 zero = __float2bfloat162_rn(0.f);
+#pragma unroll 4
+      for (int x = tr; x < (int)(kTile / 16); x += 128) {
+        uint4 u = kt[x];
+        __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) h[e] = __hmax2(h[e], zero);
+        kt[x] = u;
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_arrive(bar(L::B_RL + s));
+    }
+    ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(L::B_DONE), 0, abort_flag)) && !*abort_flag;
+    if (ok && T > 0) {
+      tc_fence_after();
+      const int wq = warp & 3;
+      const int c = wq * 32 + lane;                  // row c of relu(K)ᵀ V
+      const uint32_t lrow = tbase + ((uint32_t)(wq * 32) << 16);
+      float4* hrow = reinterpret_cast<float4*>(htot + ((size_t)bh * TD + c) * TD);
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t a[32];
+        tmem_ld32(lrow + 32 * cc, a);
+        tmem_wait_ld();
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4)
+          atomicAdd(hrow + 8 * cc + q4, make_float4(__uint_as_float(a[4 * q4]), __uint_as_float(a[4 * q4 + 1]),
+                                                    __uint_as_float(a[4 * q4 + 2]), __uint_as_float(a[4 * q4 + 3])));
+      }
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 128);
+  }
+}
+
 }  // namespace
+
+sa_status htot_tc(const void* K, const void* V, const sa_shape& s, float* htot, cudaStream_t stream) {
+  if (s.d != TD || (s.N % TB)) return SA_ERR_UNSUPPORTED;
+  const uint64_t BH = (uint64_t)s.B * s.H;
+  CUtensorMap mk, mv;
+  if (!make_tmap_3d(&mk, K, 2, TD, s.N, BH) || !make_tmap_3d(&mv, V, 2, TD, s.N, BH))
+    return fail(SA_ERR_CUDA, "sa_block_pool: cuTensorMapEncodeTiled failed for K/V");
+  const size_t smem = HtLayout::smem_bytes();
+  if (cudaFuncSetAttribute(htot_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return launch_status("cudaFuncSetAttribute(htot_tc_kernel)");
+  const int nt = s.N / TB;
+  dim3 grid((nt + kHtTiles - 1) / kHtTiles, (unsigned)BH);
+  htot_tc_kernel<<<grid, kHtThreads, smem, stream>>>(mk, mv, s.N, htot);
+  return launch_status("htot_tc_kernel");
+}
 
 bool attn_tc_supports(sa_dtype dtype, const sa_shape& s, sa_tail_mode tail) {
   return dtype == SA_BF16 && s.block == TB && s.d == TD &&

@@ -2,7 +2,7 @@
 // Hardware": block centroids and value sums), the mean pooling of SLA2's
 // router (§2B) and the block mean / diagonal covariance of SPLA's score
 // (§2.1).  HBM-bound: every input element is read once with 16-byte loads.
-#include "common.cuh"
+#include "attn_simt.cuh"
 
 namespace sa {
 namespace {
@@ -193,6 +193,16 @@ linear_totals_kernel(const T* __restrict__ K, const T* __restrict__ V, int H, in
   if (e0 == 0) atomicAdd(ztot + ((size_t)b * H + h) * D + c, z);
 }
 
+// z_tot = Σ_j zrelu_j over the head's blocks (one thread per channel).
+template <int D>
+__global__ void ztot_from_blocks_kernel(const float* __restrict__ zrelu, int H, int nb, float* __restrict__ ztot) {
+  const int h = blockIdx.x, b = blockIdx.y, c = threadIdx.x;
+  const float* z = zrelu + ((size_t)b * H + h) * nb * D + c;
+  float acc = 0.f;
+  for (int j = 0; j < nb; ++j) acc += z[(size_t)j * D];
+  ztot[((size_t)b * H + h) * D + c] = acc;
+}
+
 template <typename T, int D, int BLK>
 sa_status launch_pool(const void* Q, const void* K, const void* V, const sa_shape& s,
                       const sa_block_stats& st, cudaStream_t stream) {
@@ -207,6 +217,12 @@ sa_status launch_pool(const void* Q, const void* K, const void* V, const sa_shap
     if (cudaMemsetAsync(st.htot, 0, hbytes, stream) != cudaSuccess ||
         cudaMemsetAsync(st.ztot, 0, zbytes, stream) != cudaSuccess)
       return launch_status("cudaMemsetAsync(htot/ztot)");
+    // bf16, d = 128: H_tot on the tensor cores and z_tot from the block sums
+    if (sizeof(T) == 2 && D == 128 && st.zrelu &&
+        htot_tc(K, V, s, st.htot, stream) == SA_OK) {
+      ztot_from_blocks_kernel<D><<<dim3(s.H, s.B), D, 0, stream>>>(st.zrelu, s.H, s.N / BLK, st.ztot);
+      return launch_status("ztot_from_blocks_kernel");
+    }
     dim3 g2((s.N + kLinChunk - 1) / kLinChunk, s.H, s.B);
     linear_totals_kernel<T, D><<<g2, 256, 0, stream>>>(
         static_cast<const T*>(K), static_cast<const T*>(V), s.H, s.N, st.htot, st.ztot);
