@@ -74,6 +74,11 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
+__device__ __forceinline__ uint32_t pack2bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
 // Partial online-softmax state of one query head in a warp: log2-domain max,
 // lane-partial sum, and the lane's 4 channels (lane = channel group).
 struct HeadState {
@@ -390,6 +395,41 @@ decode_topk_kernel(const float* __restrict__ scores, int nb, int topk, int32_t* 
 }
 
 // ---- C. exact pass over the selected blocks --------------------------------
+// A stage is 64 consecutive tokens of one selected block (K and V rows staged
+// by cp.async with the 16-byte chunks of row r stored at chunk ^ (r & 7), so
+// ldmatrix reads are free of bank conflicts).  Warp w takes tokens
+// [8w, 8w + 8) of each stage and runs the small contractions on mma.sync
+// (m16n8k16, bf16 in, fp32 accumulate): S = Q Kᵀ with the group's g <= 8
+// query heads as the MMA rows, then O += P V.  Each warp keeps an online
+// softmax state per head; at the end of a segment the eight warps' states are
+// merged, the zero-order terms of the segment's blocks are subtracted, and one
+// partial state per head is written.
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a2, uint32_t b0) {
+  // rows 8-15 of A and k 8-15 of B are zero (a1 = a3 = b1 = 0)
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(0u));
+}
+__device__ __forceinline__ void mma16816_full(float (&d)[4], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
 template <int D>
 __global__ void __launch_bounds__(kDecThreads, 1)
 decode_exact_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ Kc,
@@ -397,51 +437,48 @@ decode_exact_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
                     const int32_t* __restrict__ idx, int topk, int zero_order, float scale, int nsegC, int npairs,
                     float* __restrict__ partc) {
   constexpr int CH = D / 8;                         // 16-byte chunks per bf16 row
-  constexpr int QST = 12;                           // padded floats per q chunk of 8
+  constexpr int NT = D / 8;                         // n-tiles of 8 channels
+  constexpr int KS = D / 16;                        // k steps of 16 channels
   constexpr uint32_t kRowB = D * 2;
   constexpr uint32_t kArrB = kStageTokC * kRowB;    // K (or V) of one stage
   constexpr uint32_t kStageB = 2 * kArrB;
+  constexpr int kSegBlocksMax = kSegC * kStageTokC / 64;   // blocks of a segment (blk >= 64)
+  constexpr int kCenSlots = kRingC;                         // prefetch runs < kRingC segments ahead
   extern __shared__ __align__(16) uint8_t dsm[];
-  float* qs = reinterpret_cast<float*>(dsm);                         // [g][CH][QST]
-  float* xs = qs + kMaxGroup * CH * QST;                             // merge scratch [8 warps][D+2]
-  // centroid rows of the segments in flight: [kCenSlots][segment blocks][kmean, vsum][D]
-  // (prefetching runs at most kRingC - 1 stages, hence segments, ahead)
-  float* cen = xs + kDecWarps * (D + 2);
-  constexpr int kSegBlocksMax = kSegC * kStageTokC / 64;             // blocks of a segment (blk >= 64)
-  constexpr int kCenSlots = kRingC;
+  float* qs = reinterpret_cast<float*>(dsm);                         // [g][D]  s log2e q
+  float* mg = qs + kMaxGroup * D;                                    // [8 warps][g][D + 2] merge
+  float* cen = mg + kDecWarps * kMaxGroup * (D + 2);                 // [slots][blocks][kmean, vsum][D]
   uint8_t* ring = reinterpret_cast<uint8_t*>(cen + kCenSlots * kSegBlocksMax * 2 * D);
+  const uint32_t ring_s = (uint32_t)__cvta_generic_to_shared(ring);
   const int g = Hq / Hkv;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nb = N / blk;
   const int tok_pair = topk * blk;                  // exact tokens of one (sequence, KV head)
-  const int nstage_pair = (tok_pair + kStageTokC - 1) / kStageTokC;
+  const int nstage_pair = tok_pair / kStageTokC;    // blk is a multiple of 64
   const int total_segs = npairs * nsegC;
   const float scale2 = scale * kLog2e;
   const float bias2 = log2f((float)blk);
   const float inv_blk = 1.0f / blk;
-  // warp w: token half (w & 1) of the stage, heads hh with hh % 4 == w >> 1
-  const int half = warp & 1, hsel = warp >> 1;
+  const int hrow = lane >> 2;                       // MMA row of this thread = query head
+  const bool hvalid = hrow < g;
 
   auto seg_of = [&](int k_seg) { return (int)blockIdx.x + k_seg * (int)gridDim.x; };
   auto stages_in = [&](int seg) { return min(kSegC, nstage_pair - (seg % nsegC) * kSegC); };
-  // a stage is 64 consecutive tokens of one selected block (64 divides blk)
   auto issue = [&](int seg, int sub, int slot) {
     const int pair = seg / nsegC, sseg = seg % nsegC;
-    const int t0 = (sseg * kSegC + sub) * kStageTokC;     // first exact token of the stage
+    const int t0 = (sseg * kSegC + sub) * kStageTokC;
     const int tok0 = __ldg(idx + (size_t)pair * topk + t0 / blk) * blk + (t0 % blk);
     const size_t off = ((size_t)pair * N + tok0) * D;
-    const uint8_t* ks = reinterpret_cast<const uint8_t*>(Kc + off);
+    const uint8_t* ksrc = reinterpret_cast<const uint8_t*>(Kc + off);
     const uint8_t* vsrc = reinterpret_cast<const uint8_t*>(Vc + off);
     uint8_t* dst = ring + slot * kStageB;
-    const int n16 = min(kStageTokC, tok_pair - t0) * CH;
-    for (int o = tid; o < n16; o += kDecThreads) {
-      cp_async16(dst + o * 16, ks + o * 16);
-      cp_async16(dst + kArrB + o * 16, vsrc + o * 16);
+    for (int o = tid; o < kStageTokC * CH; o += kDecThreads) {
+      const int r = o / CH, c = o % CH;
+      const uint32_t sw = r * kRowB + ((c ^ (r & 7)) << 4);
+      cp_async16(dst + sw, ksrc + o * 16);
+      cp_async16(dst + kArrB + sw, vsrc + o * 16);
     }
   };
-  // the kmean and vsum rows of a segment's selected blocks (zero-order only),
-  // into centroid slot `cslot`; issued with the segment's first stage, so the
-  // wait for that stage also covers them
   auto issue_centroids = [&](int seg, int cslot) {
     float* cb = cen + cslot * kSegBlocksMax * 2 * D;
     const int pair = seg / nsegC, sseg = seg % nsegC;
@@ -458,149 +495,163 @@ decode_exact_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
   };
 
   if (seg_of(0) >= total_segs) return;
-  int pf_seg_k = 0;
-  int pf_sub = 0;
+  int pf_seg_k = 0, pf_sub = 0, pf_slot = 0;
   auto pf_valid = [&]() { return seg_of(pf_seg_k) < total_segs; };
-  auto pf_advance = [&]() {
-    if (++pf_sub >= stages_in(seg_of(pf_seg_k))) {
-      pf_sub = 0;
-      ++pf_seg_k;
-    }
-  };
-  int pf_slot = 0;
   auto prefetch = [&]() {
     if (pf_valid()) {
       if (zero_order && pf_sub == 0) issue_centroids(seg_of(pf_seg_k), pf_seg_k % kCenSlots);
       issue(seg_of(pf_seg_k), pf_sub, pf_slot);
-      pf_advance();
+      if (++pf_sub >= stages_in(seg_of(pf_seg_k))) {
+        pf_sub = 0;
+        ++pf_seg_k;
+      }
     }
     cp_async_commit();
     pf_slot = (pf_slot + 1) % kRingC;
   };
   for (int r = 0; r < kRingC - 1; ++r) prefetch();
 
-  HeadState S[2];
-  int cur_seg_k = 0;
-  int cur_sub = 0, cur_pair = -1, slot = 0;
+  uint32_t qa0[KS], qa2[KS];                  // Q A-fragments (rows = heads)
+  float m_run = -INFINITY, l_run = 0.f;
+  float o[NT][4];
+  int cur_seg_k = 0, cur_sub = 0, cur_pair = -1, slot = 0;
   while (seg_of(cur_seg_k) < total_segs) {
     const int seg = seg_of(cur_seg_k);
     const int pair = seg / nsegC, sseg = seg % nsegC;
     const int b = pair / Hkv, kh = pair % Hkv;
     if (cur_sub == 0) {
       if (pair != cur_pair) {
-        __syncthreads();
-        for (int x = tid; x < g * D; x += kDecThreads) {
-          const int hh = x / D, c = x % D;
-          qs[(hh * CH + c / 8) * QST + (c % 8)] =
-              scale2 * __bfloat162float(q[((size_t)b * Hq + kh * g + hh) * D + c]);
+        const __nv_bfloat16* qrow = q + ((size_t)b * Hq + kh * g + (hvalid ? hrow : 0)) * D;
+#pragma unroll
+        for (int kk = 0; kk < KS; ++kk) {
+          const uint32_t lo = *reinterpret_cast<const uint32_t*>(qrow + 16 * kk + 2 * (lane & 3));
+          const uint32_t hi = *reinterpret_cast<const uint32_t*>(qrow + 16 * kk + 8 + 2 * (lane & 3));
+          qa0[kk] = hvalid ? lo : 0u;
+          qa2[kk] = hvalid ? hi : 0u;
         }
+        __syncthreads();   // the previous pair's merge is done with qs
+        for (int x = tid; x < g * D; x += kDecThreads)
+          qs[x] = scale2 * __bfloat162float(q[((size_t)b * Hq + kh * g) * D + x]);
         cur_pair = pair;
       }
-      head_reset(S[0]);
-      head_reset(S[1]);
+      m_run = -INFINITY;
+      l_run = 0.f;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[nt][e] = 0.f;
     }
     prefetch();
     cp_async_wait<kRingC - 1>();
     __syncthreads();
 
-    const uint8_t* stg = ring + slot * kStageB;
-    const int t0 = (sseg * kSegC + cur_sub) * kStageTokC;
-    const int rows = min(kStageTokC, tok_pair - t0);
-    const int r = half * kTok + lane;                    // this lane's token in the stage
+    const uint32_t kbase = ring_s + slot * kStageB, vbase = kbase + kArrB;
+    const int tokr = 8 * warp + (lane & 7);     // the row this lane addresses for ldmatrix
+    // S = Q Kᵀ for tokens [8 warp, 8 warp + 8)
+    float sacc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int hh = hsel + 4 * e;
-      if (hh >= g) break;
-      // lane = token: q·k over rotated 16-byte chunks of the K row
-      float x = -INFINITY;
-      if (r < rows) {
-        const uint8_t* krow = stg + r * kRowB;
-        const float* qh = qs + hh * CH * QST;
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-        for (int c = 0; c < CH; ++c) {
-          const int cc = (c + lane) % CH;
-          const uint4 u = *reinterpret_cast<const uint4*>(krow + cc * 16);
-          const float4 qa = *reinterpret_cast<const float4*>(qh + cc * QST);
-          const float4 qb = *reinterpret_cast<const float4*>(qh + cc * QST + 4);
-          const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
-          const float2 k0 = __bfloat1622float2(h2[0]), k1 = __bfloat1622float2(h2[1]);
-          const float2 k2 = __bfloat1622float2(h2[2]), k3 = __bfloat1622float2(h2[3]);
-          acc[0] = fmaf(k0.x, qa.x, fmaf(k0.y, qa.y, acc[0]));
-          acc[1] = fmaf(k1.x, qa.z, fmaf(k1.y, qa.w, acc[1]));
-          acc[2] = fmaf(k2.x, qb.x, fmaf(k2.y, qb.y, acc[2]));
-          acc[3] = fmaf(k3.x, qb.z, fmaf(k3.y, qb.w, acc[3]));
-        }
-        x = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-      }
-      const float p = head_add_logits(S[e], x);
-      // lane = channel group: fold in the value rows of the warp's 32 tokens
-      const uint8_t* vbase = stg + kArrB + (half * kTok) * kRowB;
-      const int nt = min(kTok, rows - half * kTok);
-      for (int t = 0; t < nt; ++t) {
-        const float pt = __shfl_sync(0xffffffffu, p, t);
-        if (lane * 4 < D) {
-          const uint2 u = *reinterpret_cast<const uint2*>(vbase + t * kRowB + lane * 8);
-          const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
-          const float2 c2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
-          S[e].acc[0] = fmaf(pt, a.x, S[e].acc[0]);
-          S[e].acc[1] = fmaf(pt, a.y, S[e].acc[1]);
-          S[e].acc[2] = fmaf(pt, c2.x, S[e].acc[2]);
-          S[e].acc[3] = fmaf(pt, c2.y, S[e].acc[3]);
-        }
+    for (int kp = 0; kp < KS / 2; ++kp) {
+      uint32_t kf[4];
+      const int chunk = 4 * kp + (lane >> 3);
+      ldsm_x4(kf, kbase + tokr * kRowB + ((chunk ^ (tokr & 7)) << 4));
+      mma16816_full(sacc, qa0[2 * kp], qa2[2 * kp], kf[0], kf[1]);
+      mma16816_full(sacc, qa0[2 * kp + 1], qa2[2 * kp + 1], kf[2], kf[3]);
+    }
+    // online softmax of this warp's 8 tokens for head hrow
+    const float x0 = sacc[0] * scale2, x1 = sacc[1] * scale2;
+    float tmax = fmaxf(x0, x1);
+    tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 1));
+    tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 2));
+    const float m_new = fmaxf(m_run, tmax);
+    const float corr = fast_exp2(m_run - m_new);
+    const float p0 = hvalid ? fast_exp2(x0 - m_new) : 0.f;
+    const float p1 = hvalid ? fast_exp2(x1 - m_new) : 0.f;
+    l_run = l_run * corr + p0 + p1;
+    m_run = m_new;
+    const uint32_t pa = pack2bf16(p0, p1);
+    // O += P V for the 8 tokens (k 8-15 of the MMA are zero)
+#pragma unroll
+    for (int nq = 0; nq < NT / 4; ++nq) {
+      uint32_t vf[4];
+      const int chunk = 4 * nq + (lane >> 3);
+      ldsm_x4_t(vf, vbase + tokr * kRowB + ((chunk ^ (tokr & 7)) << 4));
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        float* oo = o[4 * nq + e];
+        oo[0] *= corr;
+        oo[1] *= corr;
+        mma16816(o[4 * nq + e], pa, 0u, vf[e]);
       }
     }
     __syncthreads();
     slot = (slot + 1) % kRingC;
+
     if (++cur_sub >= stages_in(seg)) {
-      // end of segment: merge the two token halves of each head, subtract the
-      // zero-order terms of the segment's blocks, write the partial state
+      // ---- end of segment: merge the warps' states per head
+      float lq = l_run;
+      lq += __shfl_xor_sync(0xffffffffu, lq, 1);
+      lq += __shfl_xor_sync(0xffffffffu, lq, 2);
+      if (hvalid) {
+        float* mw = mg + ((size_t)warp * kMaxGroup + hrow) * (D + 2);
+        if ((lane & 3) == 0) {
+          mw[0] = m_run;
+          mw[1] = lq;
+        }
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int hh = hsel + 4 * e;
-        if (hh < g) head_store<D>(S[e], xs + warp * (D + 2), lane);
-        __syncthreads();
-        if (hh < g && half == 0) {
-          const float* o0 = xs + warp * (D + 2);
-          const float* o1 = xs + (warp + 1) * (D + 2);
-          HeadState T;
-          const float M = fmaxf(o0[0], o1[0]);
-          const float f0 = o0[0] == -INFINITY ? 0.f : fast_exp2(o0[0] - M);
-          const float f1 = o1[0] == -INFINITY ? 0.f : fast_exp2(o1[0] - M);
-          T.m = M;
-          T.l = lane == 0 ? o0[1] * f0 + o1[1] * f1 : 0.f;   // lane-partial sum: lane 0 holds it
+        for (int nt = 0; nt < NT; ++nt) {
+          mw[2 + 8 * nt + 2 * (lane & 3)] = o[nt][0];
+          mw[2 + 8 * nt + 2 * (lane & 3) + 1] = o[nt][1];
+        }
+      }
+      __syncthreads();
+      for (int hh = warp; hh < g; hh += kDecWarps) {
+        HeadState T;
+        float M = -INFINITY;
+        for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, mg[((size_t)w * kMaxGroup + hh) * (D + 2)]);
+        T.m = M;
+        T.l = 0.f;
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
-            T.acc[c] = lane * 4 < D ? o0[2 + lane * 4 + c] * f0 + o1[2 + lane * 4 + c] * f1 : 0.f;
-          if (zero_order) {
-            const int tb = sseg * kSegC * kStageTokC;
-            const int te = min(tok_pair, tb + kSegC * kStageTokC);
-            const float* qh = qs + hh * CH * QST;
-            for (int sidx = tb / blk; sidx * blk < te; ++sidx) {
-              // rows staged by issue_centroids with the segment's first stage
-              const float* cb = cen + (cur_seg_k % kCenSlots) * kSegBlocksMax * 2 * D;
-              const float* kr = cb + ((sidx - tb / blk) * 2 + 0) * D;
-              float d = 0.f;
-              for (int c = lane; c < D; c += 32) d = fmaf(qh[(c / 8) * QST + (c % 8)], kr[c], d);
-              d = warp_sum(d);
-              const float cl = d + bias2;                  // the block's zero-order log2 weight
-              const float m_new = fmaxf(T.m, cl);
-              const float corr = T.m == -INFINITY ? 0.f : fast_exp2(T.m - m_new);
-              const float w = fast_exp2(cl - m_new);
-              T.l = T.l * corr - (lane == 0 ? w : 0.f);
-              const float* vr = cb + ((sidx - tb / blk) * 2 + 1) * D;
+        for (int c = 0; c < 4; ++c) T.acc[c] = 0.f;
+        if (M != -INFINITY) {
+          for (int w = 0; w < kDecWarps; ++w) {
+            const float* mw = mg + ((size_t)w * kMaxGroup + hh) * (D + 2);
+            if (mw[0] == -INFINITY) continue;
+            const float f = fast_exp2(mw[0] - M);
+            if (lane == 0) T.l = fmaf(mw[1], f, T.l);
+            if (lane * 4 < D) {
 #pragma unroll
-              for (int c = 0; c < 4; ++c) {
-                const float vv = lane * 4 < D ? vr[lane * 4 + c] * inv_blk : 0.f;
-                T.acc[c] = T.acc[c] * corr - w * vv;
-              }
-              T.m = m_new;
+              for (int c = 0; c < 4; ++c) T.acc[c] = fmaf(mw[2 + lane * 4 + c], f, T.acc[c]);
             }
           }
-          head_store<D>(T, partc + (((size_t)b * Hq + kh * g + hh) * nsegC + sseg) * (D + 2), lane);
         }
-        __syncthreads();
+        if (zero_order) {
+          // subtract the zero-order term of each block of the segment
+          const int tb = sseg * kSegC * kStageTokC;
+          const int te = min(tok_pair, tb + kSegC * kStageTokC);
+          const float* qh = qs + hh * D;
+          const float* cb = cen + (cur_seg_k % kCenSlots) * kSegBlocksMax * 2 * D;
+          for (int sidx = tb / blk; sidx * blk < te; ++sidx) {
+            const float* kr = cb + ((sidx - tb / blk) * 2 + 0) * D;
+            const float* vr = cb + ((sidx - tb / blk) * 2 + 1) * D;
+            float d = 0.f;
+            for (int c = lane; c < D; c += 32) d = fmaf(qh[c], kr[c], d);
+            d = warp_sum(d);
+            const float cl = d + bias2;
+            const float m_new2 = fmaxf(T.m, cl);
+            const float corr2 = T.m == -INFINITY ? 0.f : fast_exp2(T.m - m_new2);
+            const float w = fast_exp2(cl - m_new2);
+            T.l = T.l * corr2 - (lane == 0 ? w : 0.f);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const float vv = lane * 4 < D ? vr[lane * 4 + c] * inv_blk : 0.f;
+              T.acc[c] = T.acc[c] * corr2 - w * vv;
+            }
+            T.m = m_new2;
+          }
+        }
+        head_store<D>(T, partc + (((size_t)b * Hq + kh * g + hh) * nsegC + sseg) * (D + 2), lane);
       }
+      __syncthreads();
       cur_sub = 0;
       ++cur_seg_k;
     }
@@ -700,7 +751,7 @@ sa_status launch_decode(const void* q, const void* Kc, const void* Vc, const sa_
 
   // C
   if (topk > 0) {
-    const size_t smemC = sizeof(float) * (kMaxGroup * (D / 8) * 12 + kDecWarps * (D + 2) +
+    const size_t smemC = sizeof(float) * (kMaxGroup * D + kDecWarps * kMaxGroup * (D + 2) +
                                           kRingC * (kSegC * kStageTokC / 64) * 2 * D) +
                          (size_t)kRingC * 2 * kStageTokC * D * 2;
     if (cudaFuncSetAttribute(decode_exact_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smemC) !=
