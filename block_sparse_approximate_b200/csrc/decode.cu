@@ -124,6 +124,13 @@ __device__ __forceinline__ void head_store(const HeadState& S, float* out, int l
 }
 
 // ---- A. statistics pass --------------------------------------------------
+// Per stage (32 blocks of kmean, kvar, vsum rows in shared memory) the 8 warps
+// work in three phases: (1) warp w takes head w % g and channel slice w / g of
+// the dot products q·k̄_j and (½ s² q²)·var_j (lane = block j, rotated 16-byte
+// chunks so the row reads are free of bank conflicts); (2) one warp per head
+// sums the slices, forms the block score and the zero-order logit, and takes
+// the online-softmax step; (3) warp w folds the blocks' value means into head
+// w % g's accumulator for its channel slice.
 template <int D>
 __global__ void __launch_bounds__(kDecThreads, 1)
 decode_stats_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int Hq, int Hkv, int nb, int blk,
@@ -133,21 +140,27 @@ decode_stats_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int 
   constexpr uint32_t kArrB = kStageBlocksA * kRowB;  // one array of one stage
   constexpr uint32_t kStageB = 3 * kArrB;
   extern __shared__ __align__(16) uint8_t dsm[];
-  float* qs = reinterpret_cast<float*>(dsm);                 // [g][D]  s q log2e
+  float* qs = reinterpret_cast<float*>(dsm);                 // [g][D]  s log2e q
   float* ws = qs + kMaxGroup * D;                            // [g][D]  ½ s² q²
-  float* lsm = ws + kMaxGroup * D;                           // [g][32] per-head log scores
-  uint8_t* ring = reinterpret_cast<uint8_t*>(lsm + kMaxGroup * kStageBlocksA);
+  float* lsm = ws + kMaxGroup * D;                           // [g][32] natural log scores
+  float* part = lsm + kMaxGroup * kStageBlocksA;             // [8 warps][2][32] slice dots
+  float* pp = part + kDecWarps * 2 * kStageBlocksA;          // [g][32] probabilities
+  float* cr = pp + kMaxGroup * kStageBlocksA;                // [g] rescale factors (+pad)
+  uint8_t* ring = reinterpret_cast<uint8_t*>(cr + 16);
   const int g = Hq / Hkv;
+  const int P = kDecWarps / g;                       // channel slices per head
+  const int CS = CH / P;                             // float4 chunks per slice
+  const int CPL = (D / P) >= 32 ? (D / P) / 32 : 1;  // channels per lane in the fold
+  const int FL = (D / P) / CPL;                      // lanes active in the fold
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int hw = warp % g, sl = warp / g;            // this warp's head and channel slice
   const int nstage_pair = (nb + kStageBlocksA - 1) / kStageBlocksA;
   const int total_segs = npairs * nsegA;
   const float bias2 = log2f((float)blk);
   const float inv_blk = 1.0f / blk;
 
-  // the CTA's stage sequence: its segments in order, each segment's stages
   auto seg_of = [&](int k_seg) { return (int)blockIdx.x + k_seg * (int)gridDim.x; };
   auto stages_in = [&](int seg) { return min(kSegA, nstage_pair - (seg % nsegA) * kSegA); };
-  // issue the copies of stage `sub` of segment `seg` into ring slot `slot`
   auto issue = [&](int seg, int sub, int slot) {
     const int pair = seg / nsegA, sseg = seg % nsegA;
     const int j0 = (sseg * kSegA + sub) * kStageBlocksA;
@@ -164,40 +177,32 @@ decode_stats_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int 
     }
   };
 
-  // flat iteration over (segment, stage) pairs of this CTA
-  int cur_seg_k = 0;
   if (seg_of(0) >= total_segs) return;
-  int cur_sub = 0;
-  // lookahead cursor for prefetching
-  int pf_seg_k = 0;
-  int pf_sub = 0;
-  auto pf_valid = [&]() { return seg_of(pf_seg_k) < total_segs; };
-  auto pf_advance = [&]() {
-    if (++pf_sub >= stages_in(seg_of(pf_seg_k))) {
-      pf_sub = 0;
-      ++pf_seg_k;
-    }
-  };
-  int pf_slot = 0;
-  for (int r = 0; r < kRingA - 1; ++r) {
-    if (pf_valid()) {
+  int pf_seg_k = 0, pf_sub = 0, pf_slot = 0;
+  auto prefetch = [&]() {
+    if (seg_of(pf_seg_k) < total_segs) {
       issue(seg_of(pf_seg_k), pf_sub, pf_slot);
-      pf_advance();
+      if (++pf_sub >= stages_in(seg_of(pf_seg_k))) {
+        pf_sub = 0;
+        ++pf_seg_k;
+      }
     }
     cp_async_commit();
     pf_slot = (pf_slot + 1) % kRingA;
-  }
+  };
+  for (int r = 0; r < kRingA - 1; ++r) prefetch();
 
-  HeadState S;
-  int cur_pair = -1;
-  int slot = 0;
+  // per warp: the fold accumulator of (head hw, slice sl); the phase-2 warp of
+  // each head (sl == 0) also owns the head's running max and sum
+  float acc[4];
+  float m_run = -INFINITY, l_run = 0.f;
+  int cur_seg_k = 0, cur_sub = 0, cur_pair = -1, slot = 0;
   while (seg_of(cur_seg_k) < total_segs) {
     const int seg = seg_of(cur_seg_k);
     const int pair = seg / nsegA, sseg = seg % nsegA;
     const int b = pair / Hkv, kh = pair % Hkv;
     if (cur_sub == 0) {
       if (pair != cur_pair) {
-        // this pair's query vectors
         __syncthreads();
         for (int x = tid; x < g * D; x += kDecThreads) {
           const int hh = x / D, c = x % D;
@@ -207,15 +212,12 @@ decode_stats_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int 
         }
         cur_pair = pair;
       }
-      head_reset(S);
+      m_run = -INFINITY;
+      l_run = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[c] = 0.f;
     }
-    // prefetch one more stage, then wait for the current one
-    if (pf_valid()) {
-      issue(seg_of(pf_seg_k), pf_sub, pf_slot);
-      pf_advance();
-    }
-    cp_async_commit();
-    pf_slot = (pf_slot + 1) % kRingA;
+    prefetch();
     cp_async_wait<kRingA - 1>();
     __syncthreads();
 
@@ -225,51 +227,55 @@ decode_stats_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int 
     const float* vs = reinterpret_cast<const float*>(stg + 2 * kArrB);
     const int j0 = (sseg * kSegA + cur_sub) * kStageBlocksA;
     const int rows = min(kStageBlocksA, nb - j0);
-    if (warp < g) {
-      // lane = block: dot products over rotated float4 chunks (conflict free)
-      const int hh = warp;
-      float d1 = 0.f, d2 = 0.f;
+
+    // phase 1: slice dot products (lane = block)
+    {
+      float a1[4] = {0.f, 0.f, 0.f, 0.f}, a2[4] = {0.f, 0.f, 0.f, 0.f};
       if (lane < rows) {
         const float4* kr = reinterpret_cast<const float4*>(km + lane * D);
         const float4* vr = reinterpret_cast<const float4*>(kv + lane * D);
-        const float4* qr = reinterpret_cast<const float4*>(qs + hh * D);
-        const float4* wr = reinterpret_cast<const float4*>(ws + hh * D);
-        float a1[4] = {0.f, 0.f, 0.f, 0.f}, a2[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 8
-        for (int c = 0; c < CH; ++c) {
-          const int cc = (c + lane) % CH;
-          const float4 a = kr[cc], qv = qr[cc], vv = vr[cc], wv = wr[cc];
-          a1[0] = fmaf(a.x, qv.x, a1[0]);
-          a1[1] = fmaf(a.y, qv.y, a1[1]);
-          a1[2] = fmaf(a.z, qv.z, a1[2]);
-          a1[3] = fmaf(a.w, qv.w, a1[3]);
-          a2[0] = fmaf(vv.x, wv.x, a2[0]);
-          a2[1] = fmaf(vv.y, wv.y, a2[1]);
-          a2[2] = fmaf(vv.z, wv.z, a2[2]);
-          a2[3] = fmaf(vv.w, wv.w, a2[3]);
-        }
-        d1 = (a1[0] + a1[1]) + (a1[2] + a1[3]);
-        d2 = (a2[0] + a2[1]) + (a2[2] + a2[3]);
-      }
-      // d1 = s log2e q·k̄: natural log score s q·k̄ + log1p(½ s² Σ q² var)
-      const float lnat = d1 * kLn2 + log1pf(d2);
-      lsm[hh * kStageBlocksA + lane] = lnat;
-      // zero-order term of every block of the stage (log2 domain)
-      const float x = lane < rows ? d1 + bias2 : -INFINITY;
-      const float p = head_add_logits(S, x);
-      for (int t = 0; t < rows; ++t) {
-        const float pt = __shfl_sync(0xffffffffu, p, t);
-        if (lane * 4 < D) {
-          const float4 v4 = *reinterpret_cast<const float4*>(vs + t * D + lane * 4);
-          S.acc[0] = fmaf(pt, v4.x * inv_blk, S.acc[0]);
-          S.acc[1] = fmaf(pt, v4.y * inv_blk, S.acc[1]);
-          S.acc[2] = fmaf(pt, v4.z * inv_blk, S.acc[2]);
-          S.acc[3] = fmaf(pt, v4.w * inv_blk, S.acc[3]);
+        const float4* qr = reinterpret_cast<const float4*>(qs + hw * D);
+        const float4* wr = reinterpret_cast<const float4*>(ws + hw * D);
+        for (int c = 0; c < CS; ++c) {
+          const int cc = sl * CS + (c + lane) % CS;
+          const float4 ka = kr[cc], qv = qr[cc], va = vr[cc], wv = wr[cc];
+          a1[0] = fmaf(ka.x, qv.x, a1[0]);
+          a1[1] = fmaf(ka.y, qv.y, a1[1]);
+          a1[2] = fmaf(ka.z, qv.z, a1[2]);
+          a1[3] = fmaf(ka.w, qv.w, a1[3]);
+          a2[0] = fmaf(va.x, wv.x, a2[0]);
+          a2[1] = fmaf(va.y, wv.y, a2[1]);
+          a2[2] = fmaf(va.z, wv.z, a2[2]);
+          a2[3] = fmaf(va.w, wv.w, a2[3]);
         }
       }
+      part[(warp * 2 + 0) * kStageBlocksA + lane] = (a1[0] + a1[1]) + (a1[2] + a1[3]);
+      part[(warp * 2 + 1) * kStageBlocksA + lane] = (a2[0] + a2[1]) + (a2[2] + a2[3]);
     }
     __syncthreads();
-    // group score of the stage's blocks: logsumexp over the g heads
+    // phase 2: one warp per head (slice 0): score, zero-order logit, softmax step
+    if (sl == 0) {
+      float d1 = 0.f, d2 = 0.f;
+      for (int t = 0; t < P; ++t) {   // slices of head hw are warps hw + t g
+        d1 += part[((hw + t * g) * 2 + 0) * kStageBlocksA + lane];
+        d2 += part[((hw + t * g) * 2 + 1) * kStageBlocksA + lane];
+      }
+      lsm[hw * kStageBlocksA + lane] = d1 * kLn2 + log1pf(d2);
+      const float x = lane < rows ? d1 + bias2 : -INFINITY;
+      const float tmax = warp_max(x);
+      float corr = 1.f, p = 0.f;
+      if (tmax != -INFINITY) {
+        const float m_new = fmaxf(m_run, tmax);
+        corr = fast_exp2(m_run - m_new);
+        p = fast_exp2(x - m_new);
+        l_run = l_run * corr + p;
+        m_run = m_new;
+      }
+      pp[hw * kStageBlocksA + lane] = p;
+      if (lane == 0) cr[hw] = corr;
+    }
+    __syncthreads();
+    // group score of the stage's blocks (warp 0), then phase 3: the fold
     if (warp == 0 && lane < rows) {
       float mx = -INFINITY;
       for (int hh = 0; hh < g; ++hh) mx = fmaxf(mx, lsm[hh * kStageBlocksA + lane]);
@@ -277,11 +283,39 @@ decode_stats_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int 
       for (int hh = 0; hh < g; ++hh) sum += expf(lsm[hh * kStageBlocksA + lane] - mx);
       scores[(size_t)pair * nb + j0 + lane] = mx + logf(sum);
     }
+    {
+      const float corr = cr[hw];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[c] *= corr;
+      if (lane < FL) {
+        const int c0 = sl * (D / P) + lane * CPL;
+        const float* ph = pp + hw * kStageBlocksA;
+        for (int t = 0; t < rows; ++t) {
+          const float pt = ph[t] * inv_blk;
+          const float* vr = vs + t * D + c0;
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            if (c < CPL) acc[c] = fmaf(pt, vr[c], acc[c]);
+        }
+      }
+    }
+    __syncthreads();
     slot = (slot + 1) % kRingA;
-    // end of segment: write this segment's partial state for each head
     if (++cur_sub >= stages_in(seg)) {
-      if (warp < g)
-        head_store<D>(S, parta + (((size_t)b * Hq + kh * g + warp) * nsegA + sseg) * (D + 2), lane);
+      float* out = parta + (((size_t)b * Hq + kh * g + hw) * nsegA + sseg) * (D + 2);
+      if (sl == 0) {
+        const float l = warp_sum(l_run);
+        if (lane == 0) {
+          out[0] = m_run;
+          out[1] = l;
+        }
+      }
+      if (lane < FL) {
+        const int c0 = sl * (D / P) + lane * CPL;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          if (c < CPL) out[2 + c0 + c] = acc[c];
+      }
       cur_sub = 0;
       ++cur_seg_k;
     }
@@ -718,7 +752,8 @@ sa_status launch_decode(const void* q, const void* Kc, const void* Vc, const sa_
   const int sms = sm_count();
 
   // A
-  const size_t smemA = sizeof(float) * (2 * kMaxGroup * D + kMaxGroup * kStageBlocksA) +
+  const size_t smemA = sizeof(float) * (2 * kMaxGroup * D + kMaxGroup * kStageBlocksA +
+                                        kDecWarps * 2 * kStageBlocksA + kMaxGroup * kStageBlocksA + 16) +
                        (size_t)kRingA * 3 * kStageBlocksA * D * 4;
   if (cudaFuncSetAttribute(decode_stats_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smemA) !=
       cudaSuccess)
@@ -777,7 +812,8 @@ sa_status check_decode_shape(const sa_decode_shape& s, int topk) {
   if (s.B < 0 || s.Hq <= 0 || s.Hkv <= 0 || s.N < 0)
     return fail(SA_ERR_INVALID_ARG, "sa_decode_fwd: negative or zero size");
   if (s.Hq % s.Hkv) return fail(SA_ERR_INVALID_ARG, "sa_decode_fwd: Hq must be a multiple of Hkv");
-  if (s.Hq / s.Hkv > kMaxGroup) return fail(SA_ERR_UNSUPPORTED, "sa_decode_fwd: at most 8 query heads per KV head");
+  if (s.Hq / s.Hkv > kMaxGroup || (kMaxGroup % (s.Hq / s.Hkv)))
+    return fail(SA_ERR_UNSUPPORTED, "sa_decode_fwd: the GQA group (Hq / Hkv) must be 1, 2, 4 or 8");
   if (s.d != 64 && s.d != 128) return fail(SA_ERR_UNSUPPORTED, "sa_decode_fwd: d must be 64 or 128");
   if (s.block != 64 && s.block != 128) return fail(SA_ERR_UNSUPPORTED, "sa_decode_fwd: block must be 64 or 128");
   if (s.N % s.block) return fail(SA_ERR_INVALID_ARG, "sa_decode_fwd: N must be a multiple of block");

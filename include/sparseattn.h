@@ -186,7 +186,8 @@ size_t sa_decode_workspace_size(sa_decode_shape shape, int32_t topk);
  * group's query heads (a logsumexp of the log scores), keeps topk blocks, and
  * evaluates ZERO_ORDER (or DROP) attention for every query head of the group.
  * Split over the KV axis; partial (max, sum, acc) states are merged.
- * q: [B,Hq,d]; Kcache, Vcache: [B,Hkv,N,d], all of `dtype` (bf16 only).
+ * q: [B,Hq,d]; Kcache, Vcache: [B,Hkv,N,d], all of `dtype` (bf16 only);
+ * the group Hq / Hkv is 1, 2, 4 or 8.
  * stats: kmean, kvar, vsum of the caches (sa_block_pool with Q = NULL).
  * block_idx_out: [B,Hkv,topk] int32 or NULL; scores_out: [B,Hkv,nb] float32
  * or NULL.  O: [B,Hq,d] of `dtype`.  workspace: device scratch of at least
