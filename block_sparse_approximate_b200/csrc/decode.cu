@@ -30,7 +30,6 @@ namespace {
 constexpr int kDecThreads = 256;
 constexpr int kDecWarps = kDecThreads / 32;
 constexpr int kMaxGroup = 8;
-constexpr int kTok = 32;
 
 // A: a stage is 32 blocks of statistics (kmean, kvar, vsum rows); a segment
 // is kSegA stages (one partial state per segment and query head)
@@ -72,6 +71,15 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// (d0, d1) += (a0, a1) * (b0, b1) on two fp32 lanes at once (sm_100 packed FMA)
+__device__ __forceinline__ void ffma2x(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rd, {%0, %1};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rd;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "+f"(d0), "+f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
 
 __device__ __forceinline__ uint32_t pack2bf16(float lo, float hi) {
@@ -124,13 +132,6 @@ __device__ __forceinline__ void head_store(const HeadState& S, float* out, int l
 }
 
 // ---- A. statistics pass --------------------------------------------------
-// Per stage (32 blocks of kmean, kvar, vsum rows in shared memory) the 8 warps
-// work in three phases: (1) warp w takes head w % g and channel slice w / g of
-// the dot products q·k̄_j and (½ s² q²)·var_j (lane = block j, rotated 16-byte
-// chunks so the row reads are free of bank conflicts); (2) one warp per head
-// sums the slices, forms the block score and the zero-order logit, and takes
-// the online-softmax step; (3) warp w folds the blocks' value means into head
-// w % g's accumulator for its channel slice.
 template <int D>
 __global__ void __launch_bounds__(kDecThreads, 1)
 decode_stats_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int Hq, int Hkv, int nb, int blk,
@@ -140,27 +141,21 @@ decode_stats_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int 
   constexpr uint32_t kArrB = kStageBlocksA * kRowB;  // one array of one stage
   constexpr uint32_t kStageB = 3 * kArrB;
   extern __shared__ __align__(16) uint8_t dsm[];
-  float* qs = reinterpret_cast<float*>(dsm);                 // [g][D]  s log2e q
+  float* qs = reinterpret_cast<float*>(dsm);                 // [g][D]  s q log2e
   float* ws = qs + kMaxGroup * D;                            // [g][D]  ½ s² q²
-  float* lsm = ws + kMaxGroup * D;                           // [g][32] natural log scores
-  float* part = lsm + kMaxGroup * kStageBlocksA;             // [8 warps][2][32] slice dots
-  float* pp = part + kDecWarps * 2 * kStageBlocksA;          // [g][32] probabilities
-  float* cr = pp + kMaxGroup * kStageBlocksA;                // [g] rescale factors (+pad)
-  uint8_t* ring = reinterpret_cast<uint8_t*>(cr + 16);
+  float* lsm = ws + kMaxGroup * D;                           // [g][32] per-head log scores
+  uint8_t* ring = reinterpret_cast<uint8_t*>(lsm + kMaxGroup * kStageBlocksA);
   const int g = Hq / Hkv;
-  const int P = kDecWarps / g;                       // channel slices per head
-  const int CS = CH / P;                             // float4 chunks per slice
-  const int CPL = (D / P) >= 32 ? (D / P) / 32 : 1;  // channels per lane in the fold
-  const int FL = (D / P) / CPL;                      // lanes active in the fold
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int hw = warp % g, sl = warp / g;            // this warp's head and channel slice
   const int nstage_pair = (nb + kStageBlocksA - 1) / kStageBlocksA;
   const int total_segs = npairs * nsegA;
   const float bias2 = log2f((float)blk);
   const float inv_blk = 1.0f / blk;
 
+  // the CTA's stage sequence: its segments in order, each segment's stages
   auto seg_of = [&](int k_seg) { return (int)blockIdx.x + k_seg * (int)gridDim.x; };
   auto stages_in = [&](int seg) { return min(kSegA, nstage_pair - (seg % nsegA) * kSegA); };
+  // issue the copies of stage `sub` of segment `seg` into ring slot `slot`
   auto issue = [&](int seg, int sub, int slot) {
     const int pair = seg / nsegA, sseg = seg % nsegA;
     const int j0 = (sseg * kSegA + sub) * kStageBlocksA;
@@ -177,32 +172,40 @@ decode_stats_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int 
     }
   };
 
+  // flat iteration over (segment, stage) pairs of this CTA
+  int cur_seg_k = 0;
   if (seg_of(0) >= total_segs) return;
-  int pf_seg_k = 0, pf_sub = 0, pf_slot = 0;
-  auto prefetch = [&]() {
-    if (seg_of(pf_seg_k) < total_segs) {
+  int cur_sub = 0;
+  // lookahead cursor for prefetching
+  int pf_seg_k = 0;
+  int pf_sub = 0;
+  auto pf_valid = [&]() { return seg_of(pf_seg_k) < total_segs; };
+  auto pf_advance = [&]() {
+    if (++pf_sub >= stages_in(seg_of(pf_seg_k))) {
+      pf_sub = 0;
+      ++pf_seg_k;
+    }
+  };
+  int pf_slot = 0;
+  for (int r = 0; r < kRingA - 1; ++r) {
+    if (pf_valid()) {
       issue(seg_of(pf_seg_k), pf_sub, pf_slot);
-      if (++pf_sub >= stages_in(seg_of(pf_seg_k))) {
-        pf_sub = 0;
-        ++pf_seg_k;
-      }
+      pf_advance();
     }
     cp_async_commit();
     pf_slot = (pf_slot + 1) % kRingA;
-  };
-  for (int r = 0; r < kRingA - 1; ++r) prefetch();
+  }
 
-  // per warp: the fold accumulator of (head hw, slice sl); the phase-2 warp of
-  // each head (sl == 0) also owns the head's running max and sum
-  float acc[4];
-  float m_run = -INFINITY, l_run = 0.f;
-  int cur_seg_k = 0, cur_sub = 0, cur_pair = -1, slot = 0;
+  HeadState S;
+  int cur_pair = -1;
+  int slot = 0;
   while (seg_of(cur_seg_k) < total_segs) {
     const int seg = seg_of(cur_seg_k);
     const int pair = seg / nsegA, sseg = seg % nsegA;
     const int b = pair / Hkv, kh = pair % Hkv;
     if (cur_sub == 0) {
       if (pair != cur_pair) {
+        // this pair's query vectors
         __syncthreads();
         for (int x = tid; x < g * D; x += kDecThreads) {
           const int hh = x / D, c = x % D;
@@ -212,12 +215,15 @@ decode_stats_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int 
         }
         cur_pair = pair;
       }
-      m_run = -INFINITY;
-      l_run = 0.f;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) acc[c] = 0.f;
+      head_reset(S);
     }
-    prefetch();
+    // prefetch one more stage, then wait for the current one
+    if (pf_valid()) {
+      issue(seg_of(pf_seg_k), pf_sub, pf_slot);
+      pf_advance();
+    }
+    cp_async_commit();
+    pf_slot = (pf_slot + 1) % kRingA;
     cp_async_wait<kRingA - 1>();
     __syncthreads();
 
@@ -227,55 +233,47 @@ decode_stats_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int 
     const float* vs = reinterpret_cast<const float*>(stg + 2 * kArrB);
     const int j0 = (sseg * kSegA + cur_sub) * kStageBlocksA;
     const int rows = min(kStageBlocksA, nb - j0);
-
-    // phase 1: slice dot products (lane = block)
-    {
-      float a1[4] = {0.f, 0.f, 0.f, 0.f}, a2[4] = {0.f, 0.f, 0.f, 0.f};
+    if (warp < g) {
+      // lane = block: dot products over rotated float4 chunks (conflict free)
+      const int hh = warp;
+      float d1 = 0.f, d2 = 0.f;
       if (lane < rows) {
         const float4* kr = reinterpret_cast<const float4*>(km + lane * D);
         const float4* vr = reinterpret_cast<const float4*>(kv + lane * D);
-        const float4* qr = reinterpret_cast<const float4*>(qs + hw * D);
-        const float4* wr = reinterpret_cast<const float4*>(ws + hw * D);
-        for (int c = 0; c < CS; ++c) {
-          const int cc = sl * CS + (c + lane) % CS;
-          const float4 ka = kr[cc], qv = qr[cc], va = vr[cc], wv = wr[cc];
-          a1[0] = fmaf(ka.x, qv.x, a1[0]);
-          a1[1] = fmaf(ka.y, qv.y, a1[1]);
-          a1[2] = fmaf(ka.z, qv.z, a1[2]);
-          a1[3] = fmaf(ka.w, qv.w, a1[3]);
-          a2[0] = fmaf(va.x, wv.x, a2[0]);
-          a2[1] = fmaf(va.y, wv.y, a2[1]);
-          a2[2] = fmaf(va.z, wv.z, a2[2]);
-          a2[3] = fmaf(va.w, wv.w, a2[3]);
+        const float4* qr = reinterpret_cast<const float4*>(qs + hh * D);
+        const float4* wr = reinterpret_cast<const float4*>(ws + hh * D);
+        float a1[4] = {0.f, 0.f, 0.f, 0.f}, a2[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+        for (int c = 0; c < CH; ++c) {
+          const int cc = (c + lane) % CH;
+          const float4 a = kr[cc], qv = qr[cc], vv = vr[cc], wv = wr[cc];
+          ffma2x(a1[0], a1[1], a.x, a.y, qv.x, qv.y);
+          ffma2x(a1[2], a1[3], a.z, a.w, qv.z, qv.w);
+          ffma2x(a2[0], a2[1], vv.x, vv.y, wv.x, wv.y);
+          ffma2x(a2[2], a2[3], vv.z, vv.w, wv.z, wv.w);
+        }
+        d1 = (a1[0] + a1[1]) + (a1[2] + a1[3]);
+        d2 = (a2[0] + a2[1]) + (a2[2] + a2[3]);
+      }
+      // d1 = s log2e q·k̄: natural log score s q·k̄ + log1p(½ s² Σ q² var)
+      const float lnat = d1 * kLn2 + log1pf(d2);
+      lsm[hh * kStageBlocksA + lane] = lnat;
+      // zero-order term of every block of the stage (log2 domain)
+      const float x = lane < rows ? d1 + bias2 : -INFINITY;
+      // the value of a pseudo-key is vsum / B: fold 1/B into its probability
+      const float p = head_add_logits(S, x) * inv_blk;
+#pragma unroll 4
+      for (int t = 0; t < rows; ++t) {
+        const float pt = __shfl_sync(0xffffffffu, p, t);
+        if (lane * 4 < D) {
+          const float4 v4 = *reinterpret_cast<const float4*>(vs + t * D + lane * 4);
+          ffma2x(S.acc[0], S.acc[1], pt, pt, v4.x, v4.y);
+          ffma2x(S.acc[2], S.acc[3], pt, pt, v4.z, v4.w);
         }
       }
-      part[(warp * 2 + 0) * kStageBlocksA + lane] = (a1[0] + a1[1]) + (a1[2] + a1[3]);
-      part[(warp * 2 + 1) * kStageBlocksA + lane] = (a2[0] + a2[1]) + (a2[2] + a2[3]);
     }
     __syncthreads();
-    // phase 2: one warp per head (slice 0): score, zero-order logit, softmax step
-    if (sl == 0) {
-      float d1 = 0.f, d2 = 0.f;
-      for (int t = 0; t < P; ++t) {   // slices of head hw are warps hw + t g
-        d1 += part[((hw + t * g) * 2 + 0) * kStageBlocksA + lane];
-        d2 += part[((hw + t * g) * 2 + 1) * kStageBlocksA + lane];
-      }
-      lsm[hw * kStageBlocksA + lane] = d1 * kLn2 + log1pf(d2);
-      const float x = lane < rows ? d1 + bias2 : -INFINITY;
-      const float tmax = warp_max(x);
-      float corr = 1.f, p = 0.f;
-      if (tmax != -INFINITY) {
-        const float m_new = fmaxf(m_run, tmax);
-        corr = fast_exp2(m_run - m_new);
-        p = fast_exp2(x - m_new);
-        l_run = l_run * corr + p;
-        m_run = m_new;
-      }
-      pp[hw * kStageBlocksA + lane] = p;
-      if (lane == 0) cr[hw] = corr;
-    }
-    __syncthreads();
-    // group score of the stage's blocks (warp 0), then phase 3: the fold
+    // group score of the stage's blocks: logsumexp over the g heads
     if (warp == 0 && lane < rows) {
       float mx = -INFINITY;
       for (int hh = 0; hh < g; ++hh) mx = fmaxf(mx, lsm[hh * kStageBlocksA + lane]);
@@ -283,39 +281,11 @@ decode_stats_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int 
       for (int hh = 0; hh < g; ++hh) sum += expf(lsm[hh * kStageBlocksA + lane] - mx);
       scores[(size_t)pair * nb + j0 + lane] = mx + logf(sum);
     }
-    {
-      const float corr = cr[hw];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) acc[c] *= corr;
-      if (lane < FL) {
-        const int c0 = sl * (D / P) + lane * CPL;
-        const float* ph = pp + hw * kStageBlocksA;
-        for (int t = 0; t < rows; ++t) {
-          const float pt = ph[t] * inv_blk;
-          const float* vr = vs + t * D + c0;
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-            if (c < CPL) acc[c] = fmaf(pt, vr[c], acc[c]);
-        }
-      }
-    }
-    __syncthreads();
     slot = (slot + 1) % kRingA;
+    // end of segment: write this segment's partial state for each head
     if (++cur_sub >= stages_in(seg)) {
-      float* out = parta + (((size_t)b * Hq + kh * g + hw) * nsegA + sseg) * (D + 2);
-      if (sl == 0) {
-        const float l = warp_sum(l_run);
-        if (lane == 0) {
-          out[0] = m_run;
-          out[1] = l;
-        }
-      }
-      if (lane < FL) {
-        const int c0 = sl * (D / P) + lane * CPL;
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          if (c < CPL) out[2 + c0 + c] = acc[c];
-      }
+      if (warp < g)
+        head_store<D>(S, parta + (((size_t)b * Hq + kh * g + warp) * nsegA + sseg) * (D + 2), lane);
       cur_sub = 0;
       ++cur_seg_k;
     }
@@ -324,87 +294,114 @@ decode_stats_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int 
 }
 
 // ---- B. top-k ------------------------------------------------------------
-// k <= 64: each warp takes the k best of its share of the scores by repeated
-// warp arg-max over (score desc, index asc) keys, then warp 0 takes the k best
-// of the candidates the same way, and the winners are emitted in ascending
-// order.  Larger k: a bitonic sort of the whole row.
-constexpr int kTopkWarpMax = 64;
-
-__device__ __forceinline__ unsigned long long rank_key_d(float score, int j) {
-  return ((unsigned long long)(~order_key(score)) << 32) | (unsigned)j;
-}
-
-__device__ __forceinline__ unsigned long long warp_min_u64d(unsigned long long v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const unsigned long long w = __shfl_xor_sync(0xffffffffu, v, o);
-    v = w < v ? w : v;
-  }
-  return v;
-}
+// Radix select over the 32-bit order keys of the scores (higher score =
+// smaller key): four 8-bit histogram passes find the key T of the k-th best
+// block; every block with a smaller key is kept, and of the blocks whose key
+// equals T the ones with the smallest indices fill the remaining places.  The
+// kept indices are emitted in ascending order from a bitmap.
+constexpr int kTopkKPT = kMaxRouteBlocks / kDecThreads;   // keys per thread
 
 __global__ void __launch_bounds__(kDecThreads)
 decode_topk_kernel(const float* __restrict__ scores, int nb, int topk, int32_t* __restrict__ idx) {
   const int pair = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  extern __shared__ unsigned long long tk_smem[];
+  __shared__ unsigned hist[256];
+  __shared__ uint32_t bits[kMaxRouteBlocks / 32];
+  __shared__ unsigned sh_prefix, sh_rank, sh_eq;
   const float* sc = scores + (size_t)pair * nb;
   int32_t* out = idx + (size_t)pair * topk;
-  if (topk > kTopkWarpMax) {
-    int n2 = 1;
-    while (n2 < nb) n2 <<= 1;
-    float* scs = reinterpret_cast<float*>(tk_smem + n2);
-    for (int j = tid; j < nb; j += kDecThreads) scs[j] = sc[j];
-    __syncthreads();
-    block_topk_ascending(scs, nb, topk, tk_smem, out);
-    return;
-  }
-  unsigned long long* cand = tk_smem;                       // [warps][topk]
   const int nwords = (nb + 31) / 32;
-  uint32_t* bits = reinterpret_cast<uint32_t*>(cand + kDecWarps * kTopkWarpMax);
-  for (int x = tid; x < nwords; x += kDecThreads) bits[x] = 0u;
-  // stage 1: per warp, the k best of scores j = warp*32 + lane + 256 i (the
-  // row is at most 4096 long: 16 keys per lane, held in registers)
-  constexpr int KPL = kMaxRouteBlocks / kDecThreads;
-  unsigned long long key[KPL];
+
+  uint32_t key[kTopkKPT];
 #pragma unroll
-  for (int e = 0; e < KPL; ++e) {
-    const int j = warp * 32 + lane + e * kDecThreads;
-    key[e] = j < nb ? rank_key_d(sc[j], j) : ~0ull;
+  for (int e = 0; e < kTopkKPT; ++e) {
+    const int j = tid + e * kDecThreads;
+    key[e] = j < nb ? ~order_key(sc[j]) : 0xffffffffu;
   }
-  unsigned long long prev = 0ull;
-  for (int r = 0; r < topk; ++r) {
-    unsigned long long mine = ~0ull;
+  for (int x = tid; x < nwords; x += kDecThreads) bits[x] = 0u;
+  if (tid == 0) {
+    sh_prefix = 0u;
+    sh_rank = (unsigned)topk;
+  }
+  unsigned mask = 0u;
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    for (int x = tid; x < 256; x += kDecThreads) hist[x] = 0u;
+    __syncthreads();
+    const unsigned prefix = sh_prefix;
 #pragma unroll
-    for (int e = 0; e < KPL; ++e)
-      if ((r == 0 || key[e] > prev) && key[e] < mine) mine = key[e];
-    const unsigned long long best = warp_min_u64d(mine);
-    if (lane == 0) cand[warp * kTopkWarpMax + r] = best;
-    prev = best;
+    for (int e = 0; e < kTopkKPT; ++e) {
+      const int j = tid + e * kDecThreads;
+      if (j < nb && (key[e] & mask) == prefix) atomicAdd(&hist[(key[e] >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    if (warp == 0) {
+      // bucket holding the rank-th smallest key among those matching prefix
+      unsigned c[8], tot = 0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        c[e] = hist[lane * 8 + e];
+        tot += c[e];
+      }
+      unsigned incl = tot;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const unsigned rank = sh_rank;
+      const unsigned excl = incl - tot;
+      if (excl < rank && rank <= incl) {
+        unsigned run = excl;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          if (run < rank && rank <= run + c[e]) {
+            sh_prefix = prefix | ((unsigned)(lane * 8 + e) << shift);
+            sh_rank = rank - run;
+          }
+          run += c[e];
+        }
+      }
+    }
+    mask |= 255u << shift;
+    __syncthreads();
+  }
+  const unsigned T = sh_prefix;         // key of the k-th best block
+  const unsigned need_eq = sh_rank;     // how many blocks with key T are kept
+  if (tid == 0) sh_eq = 0u;
+  __syncthreads();
+  unsigned my_eq = 0;
+#pragma unroll
+  for (int e = 0; e < kTopkKPT; ++e) {
+    const int j = tid + e * kDecThreads;
+    if (j < nb) {
+      if (key[e] < T) atomicOr(&bits[j >> 5], 1u << (j & 31));
+      else if (key[e] == T) ++my_eq;
+    }
+  }
+  if (my_eq) atomicAdd(&sh_eq, my_eq);
+  __syncthreads();
+  if (sh_eq == need_eq) {
+#pragma unroll
+    for (int e = 0; e < kTopkKPT; ++e) {
+      const int j = tid + e * kDecThreads;
+      if (j < nb && key[e] == T) atomicOr(&bits[j >> 5], 1u << (j & 31));
+    }
+  } else if (warp == 0) {
+    // ties at the threshold: the smallest indices first
+    unsigned left = need_eq;
+    for (int j0 = 0; j0 < nb && left > 0; j0 += 32) {
+      const int j = j0 + lane;
+      const bool eq = j < nb && ~order_key(sc[j]) == T;
+      const unsigned bal = __ballot_sync(0xffffffffu, eq);
+      const unsigned before = __popc(bal & ((1u << lane) - 1u));
+      if (eq && before < left) atomicOr(&bits[j >> 5], 1u << (j & 31));
+      const unsigned n = __popc(bal);
+      left = n >= left ? 0u : left - n;
+    }
   }
   __syncthreads();
-  // stage 2: the k best of the warps' candidates (absent ones are all ones)
   if (warp == 0) {
-    unsigned long long ck[kDecWarps * kTopkWarpMax / 32];
-#pragma unroll
-    for (int e = 0; e < kDecWarps * kTopkWarpMax / 32; ++e) {
-      const int x = lane + 32 * e;                      // candidate x = (warp x / 64, rank x % 64)
-      ck[e] = (x % kTopkWarpMax) < topk ? cand[x] : ~0ull;
-    }
-    prev = 0ull;
-    for (int r = 0; r < topk; ++r) {
-      unsigned long long mine = ~0ull;
-#pragma unroll
-      for (int e = 0; e < kDecWarps * kTopkWarpMax / 32; ++e)
-        if ((r == 0 || ck[e] > prev) && ck[e] < mine) mine = ck[e];
-      const unsigned long long best = warp_min_u64d(mine);
-      if (lane == 0 && best != ~0ull) {
-        const int jb = (int)(best & 0xffffffffu);
-        bits[jb >> 5] |= 1u << (jb & 31);
-      }
-      prev = best;
-    }
-    __syncwarp();
     int base = 0;
     for (int x0 = 0; x0 < nwords; x0 += 32) {
       const int x = x0 + lane;
@@ -752,8 +749,7 @@ sa_status launch_decode(const void* q, const void* Kc, const void* Vc, const sa_
   const int sms = sm_count();
 
   // A
-  const size_t smemA = sizeof(float) * (2 * kMaxGroup * D + kMaxGroup * kStageBlocksA +
-                                        kDecWarps * 2 * kStageBlocksA + kMaxGroup * kStageBlocksA + 16) +
+  const size_t smemA = sizeof(float) * (2 * kMaxGroup * D + kMaxGroup * kStageBlocksA) +
                        (size_t)kRingA * 3 * kStageBlocksA * D * 4;
   if (cudaFuncSetAttribute(decode_stats_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smemA) !=
       cudaSuccess)
@@ -767,19 +763,7 @@ sa_status launch_decode(const void* q, const void* Kc, const void* Vc, const sa_
 
   // B
   if (topk > 0) {
-    size_t smemB;
-    if (topk > kTopkWarpMax) {
-      int n2 = 1;
-      while (n2 < nb) n2 <<= 1;
-      smemB = (size_t)n2 * 8 + (size_t)nb * 4;
-    } else {
-      smemB = (size_t)kDecWarps * kTopkWarpMax * 8 + (size_t)((nb + 31) / 32) * 4;
-    }
-    if (smemB > 48 * 1024 &&
-        cudaFuncSetAttribute(decode_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smemB) !=
-            cudaSuccess)
-      return launch_status("cudaFuncSetAttribute(decode_topk_kernel)");
-    decode_topk_kernel<<<npairs, kDecThreads, smemB, stream>>>(scores, nb, topk, idx);
+    decode_topk_kernel<<<npairs, kDecThreads, 0, stream>>>(scores, nb, topk, idx);
     r = launch_status("decode_topk_kernel");
     if (r != SA_OK) return r;
   }
