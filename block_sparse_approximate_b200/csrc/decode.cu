@@ -35,7 +35,7 @@ constexpr int kMaxGroup = 8;
 // is kSegA stages (one partial state per segment and query head)
 constexpr int kStageBlocksA = 32;
 constexpr int kSegA = 8;
-constexpr int kRingA = 3;
+constexpr int kRingA = 2;
 // C: a stage is 64 tokens of K and V; a segment is kSegC stages
 constexpr int kStageTokC = 64;
 constexpr int kSegC = 8;
@@ -132,8 +132,10 @@ __device__ __forceinline__ void head_store(const HeadState& S, float* out, int l
 }
 
 // ---- A. statistics pass --------------------------------------------------
+constexpr int kThrA = 128;   // 4 warps; two CTAs share an SM
+
 template <int D>
-__global__ void __launch_bounds__(kDecThreads, 1)
+__global__ void __launch_bounds__(kThrA, 2)
 decode_stats_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int Hq, int Hkv, int nb, int blk,
                     float scale, int nsegA, int npairs, float* __restrict__ scores, float* __restrict__ parta) {
   constexpr int CH = D / 4;                          // float4 chunks per row
@@ -165,7 +167,7 @@ decode_stats_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int 
     const uint8_t* src0 = reinterpret_cast<const uint8_t*>(st.kmean + goff);
     const uint8_t* src1 = reinterpret_cast<const uint8_t*>(st.kvar + goff);
     const uint8_t* src2 = reinterpret_cast<const uint8_t*>(st.vsum + goff);
-    for (int o = tid; o < n16; o += kDecThreads) {
+    for (int o = tid; o < n16; o += kThrA) {
       cp_async16(dst + o * 16, src0 + o * 16);
       cp_async16(dst + kArrB + o * 16, src1 + o * 16);
       cp_async16(dst + 2 * kArrB + o * 16, src2 + o * 16);
@@ -196,7 +198,7 @@ decode_stats_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int 
     pf_slot = (pf_slot + 1) % kRingA;
   }
 
-  HeadState S;
+  HeadState S[2];   // heads warp and warp + 4 (a group has at most 8 heads)
   int cur_pair = -1;
   int slot = 0;
   while (seg_of(cur_seg_k) < total_segs) {
@@ -207,7 +209,7 @@ decode_stats_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int 
       if (pair != cur_pair) {
         // this pair's query vectors
         __syncthreads();
-        for (int x = tid; x < g * D; x += kDecThreads) {
+        for (int x = tid; x < g * D; x += kThrA) {
           const int hh = x / D, c = x % D;
           const float v = __bfloat162float(q[((size_t)b * Hq + kh * g + hh) * D + c]);
           qs[hh * D + c] = scale * kLog2e * v;
@@ -215,7 +217,8 @@ decode_stats_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int 
         }
         cur_pair = pair;
       }
-      head_reset(S);
+      head_reset(S[0]);
+      head_reset(S[1]);
     }
     // prefetch one more stage, then wait for the current one
     if (pf_valid()) {
@@ -233,9 +236,11 @@ decode_stats_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int 
     const float* vs = reinterpret_cast<const float*>(stg + 2 * kArrB);
     const int j0 = (sseg * kSegA + cur_sub) * kStageBlocksA;
     const int rows = min(kStageBlocksA, nb - j0);
-    if (warp < g) {
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int hh = warp + 4 * e;
+      if (hh >= g) break;
       // lane = block: dot products over rotated float4 chunks (conflict free)
-      const int hh = warp;
       float d1 = 0.f, d2 = 0.f;
       if (lane < rows) {
         const float4* kr = reinterpret_cast<const float4*>(km + lane * D);
@@ -256,19 +261,18 @@ decode_stats_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int 
         d2 = (a2[0] + a2[1]) + (a2[2] + a2[3]);
       }
       // d1 = s log2e q·k̄: natural log score s q·k̄ + log1p(½ s² Σ q² var)
-      const float lnat = d1 * kLn2 + log1pf(d2);
-      lsm[hh * kStageBlocksA + lane] = lnat;
+      lsm[hh * kStageBlocksA + lane] = d1 * kLn2 + log1pf(d2);
       // zero-order term of every block of the stage (log2 domain)
       const float x = lane < rows ? d1 + bias2 : -INFINITY;
       // the value of a pseudo-key is vsum / B: fold 1/B into its probability
-      const float p = head_add_logits(S, x) * inv_blk;
+      const float p = head_add_logits(S[e], x) * inv_blk;
 #pragma unroll 4
       for (int t = 0; t < rows; ++t) {
         const float pt = __shfl_sync(0xffffffffu, p, t);
         if (lane * 4 < D) {
           const float4 v4 = *reinterpret_cast<const float4*>(vs + t * D + lane * 4);
-          ffma2x(S.acc[0], S.acc[1], pt, pt, v4.x, v4.y);
-          ffma2x(S.acc[2], S.acc[3], pt, pt, v4.z, v4.w);
+          ffma2x(S[e].acc[0], S[e].acc[1], pt, pt, v4.x, v4.y);
+          ffma2x(S[e].acc[2], S[e].acc[3], pt, pt, v4.z, v4.w);
         }
       }
     }
@@ -284,8 +288,10 @@ decode_stats_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int 
     slot = (slot + 1) % kRingA;
     // end of segment: write this segment's partial state for each head
     if (++cur_sub >= stages_in(seg)) {
-      if (warp < g)
-        head_store<D>(S, parta + (((size_t)b * Hq + kh * g + warp) * nsegA + sseg) * (D + 2), lane);
+#pragma unroll
+      for (int e = 0; e < 2; ++e)
+        if (warp + 4 * e < g)
+          head_store<D>(S[e], parta + (((size_t)b * Hq + kh * g + warp + 4 * e) * nsegA + sseg) * (D + 2), lane);
       cur_sub = 0;
       ++cur_seg_k;
     }
@@ -755,8 +761,8 @@ sa_status launch_decode(const void* q, const void* Kc, const void* Vc, const sa_
       cudaSuccess)
     return launch_status("cudaFuncSetAttribute(decode_stats_kernel)");
   const long segsA = (long)npairs * L.nsegA;
-  const int gridA = (int)(segsA < sms ? segsA : sms);
-  decode_stats_kernel<D><<<gridA, kDecThreads, smemA, stream>>>(qb, st, s.Hq, s.Hkv, nb, s.block, scale,
+  const int gridA = (int)(segsA < 2 * sms ? segsA : 2 * sms);
+  decode_stats_kernel<D><<<gridA, kThrA, smemA, stream>>>(qb, st, s.Hq, s.Hkv, nb, s.block, scale,
                                                                  L.nsegA, npairs, scores, parta);
   sa_status r = launch_status("decode_stats_kernel");
   if (r != SA_OK) return r;
