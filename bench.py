@@ -50,6 +50,28 @@ def _peaks():
         return 6650.0, 1590.0, 1400.0, "fallback"
 
 
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one
+# attn_tc_kernel launch on the video_dit workload, from an ncu capture, keyed by
+# the SHA-256 of the attention kernel's sources at capture time.  When the
+# sources change the figure no longer describes the kernel and is reported as
+# null until it is captured again.
+ATTN_TRAFFIC = {"sources": ("csrc/attn_tc.cu", "csrc/tc_util.cuh", "csrc/common.cuh"),
+                "sha256": "c07cde26 b0dc92cc 33ab5e2b", "bytes": 389.77e6}
+
+
+def attn_traffic_bytes():
+    import hashlib
+    pkg = os.path.join(ROOT, "block_sparse_approximate_b200")
+    got = []
+    for rel in ATTN_TRAFFIC["sources"]:
+        try:
+            with open(os.path.join(pkg, rel), "rb") as f:
+                got.append(hashlib.sha256(f.read()).hexdigest()[:8])
+        except OSError:
+            return None
+    return ATTN_TRAFFIC["bytes"] if " ".join(got) == ATTN_TRAFFIC["sha256"] else None
+
+
 def dense_flops(w) -> float:
     return 4.0 * w.B * w.H * float(w.N) * w.N * w.d
 
@@ -455,7 +477,8 @@ def run_ours(args, world, rank, local):
         "attn_ms": attn_ms,
         "executed_tflops": achieved,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": bf16, "unit": "TFLOP/s",
-                     "frac": achieved / bf16, "traffic": None,
+                     "frac": achieved / bf16, "traffic": attn_traffic_bytes(),
+                     "traffic_unit": "bytes per launch",
                      "kernel": "sparse_attn_fwd", "peak_source": f"{src} bf16 dense (burst)"},
         "cpu_baseline": cpu,
         "e2e": e2e,
