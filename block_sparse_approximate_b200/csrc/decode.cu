@@ -34,7 +34,7 @@ constexpr int kMaxGroup = 8;
 // A: a stage is 32 blocks of statistics (kmean, kvar, vsum rows); a segment
 // is kSegA stages (one partial state per segment and query head)
 constexpr int kStageBlocksA = 32;
-constexpr int kSegA = 8;
+constexpr int kSegA = 4;
 constexpr int kRingA = 2;
 // C: a stage is 64 tokens of K and V; a segment is kSegC stages
 constexpr int kStageTokC = 64;
@@ -93,29 +93,6 @@ struct HeadState {
   float m, l, acc[4];
 };
 
-__device__ __forceinline__ void head_reset(HeadState& S) {
-  S.m = -INFINITY;
-  S.l = 0.f;
-#pragma unroll
-  for (int c = 0; c < 4; ++c) S.acc[c] = 0.f;
-}
-
-// Adds keys with lane-held log2 logits x (lane = key, -inf = absent) to S;
-// returns the lane's probability (relative to the new max) for the caller to
-// fold values in with lane = channel.
-__device__ __forceinline__ float head_add_logits(HeadState& S, float x) {
-  const float tmax = warp_max(x);
-  if (tmax == -INFINITY) return 0.f;
-  const float m_new = fmaxf(S.m, tmax);
-  const float corr = fast_exp2(S.m - m_new);
-  const float p = fast_exp2(x - m_new);
-  S.l = S.l * corr + p;
-#pragma unroll
-  for (int c = 0; c < 4; ++c) S.acc[c] *= corr;
-  S.m = m_new;
-  return p;
-}
-
 // Writes the warp's state (lane sums reduced) to out[0..D+2) (D = 128: 4
 // channels per lane; D = 64: lanes 0..15 hold 4 channels each).
 template <int D>
@@ -132,27 +109,58 @@ __device__ __forceinline__ void head_store(const HeadState& S, float* out, int l
 }
 
 // ---- A. statistics pass --------------------------------------------------
-constexpr int kThrA = 128;   // 4 warps; two CTAs share an SM
+// Two CTAs of 4 warps per SM.  A stage (32 blocks of kmean, kvar and vsum
+// rows, 48 KB for d = 128) lands in shared memory by cp.async; warp w takes
+// blocks [8w, 8w + 8) of it.  Lane = a group of d/32 channels: it holds
+// s log2e q and ½ s² q² of the group's channels for all G heads in
+// registers and reads each stats row as one contiguous 512-byte row, so a
+// row costs four shared-memory wavefronts and is read by one warp only.
+// A batch of 16/G blocks gives each lane 32 partial sums (q·k̄ and
+// ½ s² Σ q² Var for each (block, head)); a reduce-scatter over the warp
+// (31 shuffles) leaves value v in lane v, fully summed.  The zero-order
+// terms of the batch then enter the warp's online state of each head
+// (max, sum, numerator channels of the lane); the four warps' states are
+// merged once per segment.
+constexpr int kThrA = 128;
 
-template <int D>
+// channels [lane CPL, lane CPL + CPL) of a shared-memory row, or zeros
+template <int CPL>
+__device__ __forceinline__ void load_lane(float (&r)[CPL], const float* row, int lane, bool ok) {
+  if constexpr (CPL == 4) {
+    const float4 x = ok ? *reinterpret_cast<const float4*>(row + lane * 4) : make_float4(0.f, 0.f, 0.f, 0.f);
+    r[0] = x.x;
+    r[1] = x.y;
+    r[2] = x.z;
+    r[3] = x.w;
+  } else {
+    const float2 x = ok ? *reinterpret_cast<const float2*>(row + lane * 2) : make_float2(0.f, 0.f);
+    r[0] = x.x;
+    r[1] = x.y;
+  }
+}
+
+constexpr int kWarpBlocksA = kStageBlocksA / (kThrA / 32);   // blocks of a stage per warp
+
+template <int D, int G>
 __global__ void __launch_bounds__(kThrA, 2)
 decode_stats_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int Hq, int Hkv, int nb, int blk,
                     float scale, int nsegA, int npairs, float* __restrict__ scores, float* __restrict__ parta) {
-  constexpr int CH = D / 4;                          // float4 chunks per row
+  constexpr int CPL = D / 32;                        // channels per lane
+  constexpr int NBT = 16 / G;                        // blocks per batch: NBT x G x 2 = 32 sums
+  constexpr int kBatches = (kWarpBlocksA + NBT - 1) / NBT;
   constexpr uint32_t kRowB = D * 4;                  // bytes per stats row
   constexpr uint32_t kArrB = kStageBlocksA * kRowB;  // one array of one stage
   constexpr uint32_t kStageB = 3 * kArrB;
+  constexpr int kWarps = kThrA / 32;
   extern __shared__ __align__(16) uint8_t dsm[];
-  float* qs = reinterpret_cast<float*>(dsm);                 // [g][D]  s q log2e
-  float* ws = qs + kMaxGroup * D;                            // [g][D]  ½ s² q²
-  float* lsm = ws + kMaxGroup * D;                           // [g][32] per-head log scores
-  uint8_t* ring = reinterpret_cast<uint8_t*>(lsm + kMaxGroup * kStageBlocksA);
-  const int g = Hq / Hkv;
+  float* mg = reinterpret_cast<float*>(dsm);                 // [warps][G][D + 2] segment merge
+  uint8_t* ring = dsm + sizeof(float) * kWarps * G * (D + 2);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nstage_pair = (nb + kStageBlocksA - 1) / kStageBlocksA;
   const int total_segs = npairs * nsegA;
   const float bias2 = log2f((float)blk);
   const float inv_blk = 1.0f / blk;
+  const int hl = (lane >> 1) % G, jbl = (lane >> 1) / G;   // the (block, head) of the sum lane ends with
 
   // the CTA's stage sequence: its segments in order, each segment's stages
   auto seg_of = [&](int k_seg) { return (int)blockIdx.x + k_seg * (int)gridDim.x; };
@@ -174,13 +182,9 @@ decode_stats_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int 
     }
   };
 
-  // flat iteration over (segment, stage) pairs of this CTA
-  int cur_seg_k = 0;
   if (seg_of(0) >= total_segs) return;
-  int cur_sub = 0;
-  // lookahead cursor for prefetching
-  int pf_seg_k = 0;
-  int pf_sub = 0;
+  int cur_seg_k = 0, cur_sub = 0;
+  int pf_seg_k = 0, pf_sub = 0, pf_slot = 0;
   auto pf_valid = [&]() { return seg_of(pf_seg_k) < total_segs; };
   auto pf_advance = [&]() {
     if (++pf_sub >= stages_in(seg_of(pf_seg_k))) {
@@ -188,7 +192,6 @@ decode_stats_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int 
       ++pf_seg_k;
     }
   };
-  int pf_slot = 0;
   for (int r = 0; r < kRingA - 1; ++r) {
     if (pf_valid()) {
       issue(seg_of(pf_seg_k), pf_sub, pf_slot);
@@ -198,7 +201,8 @@ decode_stats_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int 
     pf_slot = (pf_slot + 1) % kRingA;
   }
 
-  HeadState S[2];   // heads warp and warp + 4 (a group has at most 8 heads)
+  float qv[G][CPL], wv[G][CPL];   // s log2e q and ½ s² q² of this lane's channels
+  float m[G], l[G], acc[G][CPL];  // the warp's online state per head (m, l replicated in all lanes)
   int cur_pair = -1;
   int slot = 0;
   while (seg_of(cur_seg_k) < total_segs) {
@@ -207,18 +211,23 @@ decode_stats_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int 
     const int b = pair / Hkv, kh = pair % Hkv;
     if (cur_sub == 0) {
       if (pair != cur_pair) {
-        // this pair's query vectors
-        __syncthreads();
-        for (int x = tid; x < g * D; x += kThrA) {
-          const int hh = x / D, c = x % D;
-          const float v = __bfloat162float(q[((size_t)b * Hq + kh * g + hh) * D + c]);
-          qs[hh * D + c] = scale * kLog2e * v;
-          ws[hh * D + c] = 0.5f * scale * scale * v * v;
-        }
+#pragma unroll
+        for (int h = 0; h < G; ++h)
+#pragma unroll
+          for (int c = 0; c < CPL; ++c) {
+            const float v = __bfloat162float(q[((size_t)b * Hq + kh * G + h) * D + lane * CPL + c]);
+            qv[h][c] = scale * kLog2e * v;
+            wv[h][c] = 0.5f * scale * scale * v * v;
+          }
         cur_pair = pair;
       }
-      head_reset(S[0]);
-      head_reset(S[1]);
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        m[h] = -INFINITY;
+        l[h] = 0.f;
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) acc[h][c] = 0.f;
+      }
     }
     // prefetch one more stage, then wait for the current one
     if (pf_valid()) {
@@ -236,62 +245,138 @@ decode_stats_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int 
     const float* vs = reinterpret_cast<const float*>(stg + 2 * kArrB);
     const int j0 = (sseg * kSegA + cur_sub) * kStageBlocksA;
     const int rows = min(kStageBlocksA, nb - j0);
+
 #pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int hh = warp + 4 * e;
-      if (hh >= g) break;
-      // lane = block: dot products over rotated float4 chunks (conflict free)
-      float d1 = 0.f, d2 = 0.f;
-      if (lane < rows) {
-        const float4* kr = reinterpret_cast<const float4*>(km + lane * D);
-        const float4* vr = reinterpret_cast<const float4*>(kv + lane * D);
-        const float4* qr = reinterpret_cast<const float4*>(qs + hh * D);
-        const float4* wr = reinterpret_cast<const float4*>(ws + hh * D);
-        float a1[4] = {0.f, 0.f, 0.f, 0.f}, a2[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 8
-        for (int c = 0; c < CH; ++c) {
-          const int cc = (c + lane) % CH;
-          const float4 a = kr[cc], qv = qr[cc], vv = vr[cc], wv = wr[cc];
-          ffma2x(a1[0], a1[1], a.x, a.y, qv.x, qv.y);
-          ffma2x(a1[2], a1[3], a.z, a.w, qv.z, qv.w);
-          ffma2x(a2[0], a2[1], vv.x, vv.y, wv.x, wv.y);
-          ffma2x(a2[2], a2[3], vv.z, vv.w, wv.z, wv.w);
-        }
-        d1 = (a1[0] + a1[1]) + (a1[2] + a1[3]);
-        d2 = (a2[0] + a2[1]) + (a2[2] + a2[3]);
-      }
-      // d1 = s log2e q·k̄: natural log score s q·k̄ + log1p(½ s² Σ q² var)
-      lsm[hh * kStageBlocksA + lane] = d1 * kLn2 + log1pf(d2);
-      // zero-order term of every block of the stage (log2 domain)
-      const float x = lane < rows ? d1 + bias2 : -INFINITY;
-      // the value of a pseudo-key is vsum / B: fold 1/B into its probability
-      const float p = head_add_logits(S[e], x) * inv_blk;
-#pragma unroll 4
-      for (int t = 0; t < rows; ++t) {
-        const float pt = __shfl_sync(0xffffffffu, p, t);
-        if (lane * 4 < D) {
-          const float4 v4 = *reinterpret_cast<const float4*>(vs + t * D + lane * 4);
-          ffma2x(S[e].acc[0], S[e].acc[1], pt, pt, v4.x, v4.y);
-          ffma2x(S[e].acc[2], S[e].acc[3], pt, pt, v4.z, v4.w);
+    for (int bi = 0; bi < kBatches; ++bi) {
+      const int jfirst = warp * kWarpBlocksA + bi * NBT;   // stage row of the batch's block 0
+      // partial sums, value index (jb G + h) 2 + kind (kind 0: q·k̄, 1: Σ q² Var)
+      float v[32];
+#pragma unroll
+      for (int jb = 0; jb < NBT; ++jb) {
+        const int jj = jfirst + jb;
+        float a[CPL], w[CPL];
+        const bool ok = jb < kWarpBlocksA - bi * NBT && jj < rows;
+        load_lane<CPL>(a, km + jj * D, lane, ok);
+        load_lane<CPL>(w, kv + jj * D, lane, ok);
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          float s1 = a[0] * qv[h][0], s2 = w[0] * wv[h][0];
+#pragma unroll
+          for (int c = 1; c < CPL; ++c) {
+            s1 = fmaf(a[c], qv[h][c], s1);
+            s2 = fmaf(w[c], wv[h][c], s2);
+          }
+          v[(jb * G + h) * 2] = s1;
+          v[(jb * G + h) * 2 + 1] = s2;
         }
       }
-    }
-    __syncthreads();
-    // group score of the stage's blocks: logsumexp over the g heads
-    if (warp == 0 && lane < rows) {
-      float mx = -INFINITY;
-      for (int hh = 0; hh < g; ++hh) mx = fmaxf(mx, lsm[hh * kStageBlocksA + lane]);
-      float sum = 0.f;
-      for (int hh = 0; hh < g; ++hh) sum += expf(lsm[hh * kStageBlocksA + lane] - mx);
-      scores[(size_t)pair * nb + j0 + lane] = mx + logf(sum);
+      // reduce-scatter: after the step of offset o, a lane keeps the half of
+      // its 2o values selected by bit o of its index; value `lane` remains
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) {
+        const bool up = (lane & o) != 0;
+#pragma unroll
+        for (int i = 0; i < o; ++i) {
+          const float send = up ? v[i] : v[i + o];
+          const float keep = up ? v[i + o] : v[i];
+          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+      }
+      const float other = __shfl_xor_sync(0xffffffffu, v[0], 1);
+      const float d1 = (lane & 1) ? other : v[0];           // s log2e q·k̄
+      const float d2 = (lane & 1) ? v[0] : other;           // ½ s² Σ q² Var
+      const int jj = jfirst + jbl;
+      const bool live = (lane & 1) == 0 && jbl < kWarpBlocksA - bi * NBT && jj < rows;
+      // group score of the block: logsumexp over its G heads (lanes 2 apart)
+      const float ls = live ? d1 * kLn2 + log1pf(d2) : -INFINITY;
+      float mx = ls;
+#pragma unroll
+      for (int o = 2; o < 2 * G; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      float se = live ? expf(ls - mx) : 0.f;
+#pragma unroll
+      for (int o = 2; o < 2 * G; o <<= 1) se += __shfl_xor_sync(0xffffffffu, se, o);
+      if (live && hl == 0) scores[(size_t)pair * nb + j0 + jj] = mx + logf(se);
+      // zero-order term: log2 weight of the pseudo-key (value vsum / B)
+      const float x = live ? d1 + bias2 : -INFINITY;
+      float bm = x;
+#pragma unroll
+      for (int o = 2 * G; o < 32; o <<= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
+      float mnew[G], corr[G];
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        mnew[h] = fmaxf(m[h], __shfl_sync(0xffffffffu, bm, 2 * h));
+        corr[h] = m[h] == -INFINITY ? 0.f : fast_exp2(m[h] - mnew[h]);
+      }
+      float mown = mnew[0];
+#pragma unroll
+      for (int h = 1; h < G; ++h)
+        if (hl == h) mown = mnew[h];
+      const float p = (live && mown != -INFINITY) ? fast_exp2(x - mown) : 0.f;
+      float ps = p;
+#pragma unroll
+      for (int o = 2 * G; o < 32; o <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        l[h] = l[h] * corr[h] + __shfl_sync(0xffffffffu, ps, 2 * h);
+        m[h] = mnew[h];
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) acc[h][c] *= corr[h];
+      }
+#pragma unroll
+      for (int jb = 0; jb < NBT; ++jb) {
+        const int jr = jfirst + jb;
+        const bool ok = jb < kWarpBlocksA - bi * NBT && jr < rows;
+        float vv[CPL];
+        load_lane<CPL>(vv, vs + jr * D, lane, ok);
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const float pw = __shfl_sync(0xffffffffu, p, (jb * G + h) * 2) * inv_blk;
+#pragma unroll
+          for (int c = 0; c < CPL; ++c) acc[h][c] = fmaf(pw, vv[c], acc[h][c]);
+        }
+      }
     }
     slot = (slot + 1) % kRingA;
-    // end of segment: write this segment's partial state for each head
-    if (++cur_sub >= stages_in(seg)) {
+    // end of segment: merge the warps' states per head and write them
+    const bool seg_end = ++cur_sub >= stages_in(seg);
+    if (seg_end) {
 #pragma unroll
-      for (int e = 0; e < 2; ++e)
-        if (warp + 4 * e < g)
-          head_store<D>(S[e], parta + (((size_t)b * Hq + kh * g + warp + 4 * e) * nsegA + sseg) * (D + 2), lane);
+      for (int h = 0; h < G; ++h) {
+        float* mw = mg + (warp * G + h) * (D + 2);
+        if (lane == 0) {
+          mw[0] = m[h];
+          mw[1] = l[h];
+        }
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) mw[2 + lane * CPL + c] = acc[h][c];
+      }
+    }
+    __syncthreads();   // the ring slot is reused by the next prefetch; the merge rows are complete
+    if (seg_end) {
+      for (int x = tid; x < G * D; x += kThrA) {
+        const int h = x / D, c = x % D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w2 = 0; w2 < kWarps; ++w2) M = fmaxf(M, mg[(w2 * G + h) * (D + 2)]);
+        float L = 0.f, A = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll
+          for (int w2 = 0; w2 < kWarps; ++w2) {
+            const float* mw = mg + (w2 * G + h) * (D + 2);
+            if (mw[0] == -INFINITY) continue;
+            const float f = fast_exp2(mw[0] - M);
+            L = fmaf(mw[1], f, L);
+            A = fmaf(mw[2 + c], f, A);
+          }
+        }
+        float* out = parta + (((size_t)b * Hq + kh * G + h) * nsegA + sseg) * (D + 2);
+        if (c == 0) {
+          out[0] = M;
+          out[1] = L;
+        }
+        out[2 + c] = A;
+      }
+      __syncthreads();   // the merge rows are rewritten at the next segment end
       cur_sub = 0;
       ++cur_seg_k;
     }
@@ -755,17 +840,27 @@ sa_status launch_decode(const void* q, const void* Kc, const void* Vc, const sa_
   const int sms = sm_count();
 
   // A
-  const size_t smemA = sizeof(float) * (2 * kMaxGroup * D + kMaxGroup * kStageBlocksA) +
-                       (size_t)kRingA * 3 * kStageBlocksA * D * 4;
-  if (cudaFuncSetAttribute(decode_stats_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smemA) !=
-      cudaSuccess)
-    return launch_status("cudaFuncSetAttribute(decode_stats_kernel)");
-  const long segsA = (long)npairs * L.nsegA;
-  const int gridA = (int)(segsA < 2 * sms ? segsA : 2 * sms);
-  decode_stats_kernel<D><<<gridA, kThrA, smemA, stream>>>(qb, st, s.Hq, s.Hkv, nb, s.block, scale,
-                                                                 L.nsegA, npairs, scores, parta);
-  sa_status r = launch_status("decode_stats_kernel");
-  if (r != SA_OK) return r;
+  {
+    const int g = s.Hq / s.Hkv;
+    const size_t smemA = sizeof(float) * 4 * g * (D + 2) + (size_t)kRingA * 3 * kStageBlocksA * D * 4;
+    const long segsA = (long)npairs * L.nsegA;
+    const int gridA = (int)(segsA < 2 * sms ? segsA : 2 * sms);
+    sa_status r0 = SA_OK;
+    auto run = [&](auto kern) {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smemA) != cudaSuccess) {
+        r0 = launch_status("cudaFuncSetAttribute(decode_stats_kernel)");
+        return;
+      }
+      kern<<<gridA, kThrA, smemA, stream>>>(qb, st, s.Hq, s.Hkv, nb, s.block, scale, L.nsegA, npairs, scores, parta);
+      r0 = launch_status("decode_stats_kernel");
+    };
+    if (g == 1) run(decode_stats_kernel<D, 1>);
+    else if (g == 2) run(decode_stats_kernel<D, 2>);
+    else if (g == 4) run(decode_stats_kernel<D, 4>);
+    else run(decode_stats_kernel<D, 8>);
+    if (r0 != SA_OK) return r0;
+  }
+  sa_status r = SA_OK;
 
   // B
   if (topk > 0) {
