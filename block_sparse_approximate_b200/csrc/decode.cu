@@ -40,6 +40,9 @@ constexpr int kRingA = 2;
 constexpr int kStageTokC = 64;
 constexpr int kSegC = 8;
 constexpr int kRingC = 4;
+// segments per CTA whose block indices are staged in shared memory (later
+// segments read theirs from global memory)
+constexpr int kItabSegs = 64;
 
 struct DecodeLayout {
   size_t scores_off, idx_off, parta_off, partc_off, total;
@@ -71,15 +74,6 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
-// (d0, d1) += (a0, a1) * (b0, b1) on two fp32 lanes at once (sm_100 packed FMA)
-__device__ __forceinline__ void ffma2x(float& d0, float& d1, float a0, float a1, float b0, float b1) {
-  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
-      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rd, {%0, %1};\n\t"
-      "fma.rn.f32x2 rd, ra, rb, rd;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-      : "+f"(d0), "+f"(d1)
-      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
 
 __device__ __forceinline__ uint32_t pack2bf16(float lo, float hi) {
@@ -524,8 +518,9 @@ decode_topk_kernel(const float* __restrict__ scores, int nb, int topk, int32_t* 
 // (m16n8k16, bf16 in, fp32 accumulate): S = Q Kᵀ with the group's g <= 8
 // query heads as the MMA rows, then O += P V.  Each warp keeps an online
 // softmax state per head; at the end of a segment the eight warps' states are
-// merged, the zero-order terms of the segment's blocks are subtracted, and one
-// partial state per head is written.
+// merged and one partial state per head is written.  The selected block
+// indices of all the CTA's segments are staged in shared memory once, so the
+// copy issue of a stage does not wait on a global load.
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a2, uint32_t b0) {
   // rows 8-15 of A and k 8-15 of B are zero (a1 = a3 = b1 = 0)
   asm volatile(
@@ -555,8 +550,8 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
 template <int D>
 __global__ void __launch_bounds__(kDecThreads, 1)
 decode_exact_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ Kc,
-                    const __nv_bfloat16* __restrict__ Vc, sa_block_stats st, int Hq, int Hkv, int N, int blk,
-                    const int32_t* __restrict__ idx, int topk, int zero_order, float scale, int nsegC, int npairs,
+                    const __nv_bfloat16* __restrict__ Vc, int Hq, int Hkv, int N, int blk,
+                    const int32_t* __restrict__ idx, int topk, float scale, int nsegC, int npairs,
                     float* __restrict__ partc) {
   constexpr int CH = D / 8;                         // 16-byte chunks per bf16 row
   constexpr int NT = D / 8;                         // n-tiles of 8 channels
@@ -565,31 +560,32 @@ decode_exact_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
   constexpr uint32_t kArrB = kStageTokC * kRowB;    // K (or V) of one stage
   constexpr uint32_t kStageB = 2 * kArrB;
   constexpr int kSegBlocksMax = kSegC * kStageTokC / 64;   // blocks of a segment (blk >= 64)
-  constexpr int kCenSlots = kRingC;                         // prefetch runs < kRingC segments ahead
   extern __shared__ __align__(16) uint8_t dsm[];
-  float* qs = reinterpret_cast<float*>(dsm);                         // [g][D]  s log2e q
-  float* mg = qs + kMaxGroup * D;                                    // [8 warps][g][D + 2] merge
-  float* cen = mg + kDecWarps * kMaxGroup * (D + 2);                 // [slots][blocks][kmean, vsum][D]
-  uint8_t* ring = reinterpret_cast<uint8_t*>(cen + kCenSlots * kSegBlocksMax * 2 * D);
+  float* mg = reinterpret_cast<float*>(dsm);                         // [8 warps][g][D + 2] merge
+  int* itab = reinterpret_cast<int*>(mg + kDecWarps * kMaxGroup * (D + 2));   // [segments][blocks]
+  uint8_t* ring = reinterpret_cast<uint8_t*>(itab + kItabSegs * kSegBlocksMax);
   const uint32_t ring_s = (uint32_t)__cvta_generic_to_shared(ring);
   const int g = Hq / Hkv;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int nb = N / blk;
   const int tok_pair = topk * blk;                  // exact tokens of one (sequence, KV head)
   const int nstage_pair = tok_pair / kStageTokC;    // blk is a multiple of 64
   const int total_segs = npairs * nsegC;
   const float scale2 = scale * kLog2e;
-  const float bias2 = log2f((float)blk);
-  const float inv_blk = 1.0f / blk;
   const int hrow = lane >> 2;                       // MMA row of this thread = query head
   const bool hvalid = hrow < g;
 
   auto seg_of = [&](int k_seg) { return (int)blockIdx.x + k_seg * (int)gridDim.x; };
   auto stages_in = [&](int seg) { return min(kSegC, nstage_pair - (seg % nsegC) * kSegC); };
-  auto issue = [&](int seg, int sub, int slot) {
+  // block slot `sl` (0 .. kSegBlocksMax) of the CTA's k-th segment
+  auto block_of = [&](int k, int seg, int sl) {
     const int pair = seg / nsegC, sseg = seg % nsegC;
-    const int t0 = (sseg * kSegC + sub) * kStageTokC;
-    const int tok0 = __ldg(idx + (size_t)pair * topk + t0 / blk) * blk + (t0 % blk);
+    const int si = sseg * kSegC * kStageTokC / blk + sl;
+    return k < kItabSegs ? itab[k * kSegBlocksMax + sl] : __ldg(idx + (size_t)pair * topk + si);
+  };
+  auto issue = [&](int k, int seg, int sub, int slot) {
+    const int pair = seg / nsegC;
+    const int tin = sub * kStageTokC;   // token offset inside the segment
+    const int tok0 = block_of(k, seg, tin / blk) * blk + (tin % blk);
     const size_t off = ((size_t)pair * N + tok0) * D;
     const uint8_t* ksrc = reinterpret_cast<const uint8_t*>(Kc + off);
     const uint8_t* vsrc = reinterpret_cast<const uint8_t*>(Vc + off);
@@ -601,28 +597,25 @@ decode_exact_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
       cp_async16(dst + kArrB + sw, vsrc + o * 16);
     }
   };
-  auto issue_centroids = [&](int seg, int cslot) {
-    float* cb = cen + cslot * kSegBlocksMax * 2 * D;
-    const int pair = seg / nsegC, sseg = seg % nsegC;
-    const int s0 = sseg * kSegC * kStageTokC / blk;
-    const int s1 = min(topk, ((sseg + 1) * kSegC * kStageTokC) / blk);
-    constexpr int R16 = D * 4 / 16;
-    for (int o = tid; o < (s1 - s0) * R16; o += kDecThreads) {
-      const int sidx = s0 + o / R16, c = o % R16;
-      const int j = __ldg(idx + (size_t)pair * topk + sidx);
-      const size_t row = ((size_t)pair * nb + j) * D;
-      cp_async16(cb + ((sidx - s0) * 2 + 0) * D + c * 4, st.kmean + row + c * 4);
-      cp_async16(cb + ((sidx - s0) * 2 + 1) * D + c * 4, st.vsum + row + c * 4);
-    }
-  };
-
   if (seg_of(0) >= total_segs) return;
+  // the selected blocks of the CTA's first kItabSegs segments
+  for (int x = tid; x < kItabSegs * kSegBlocksMax; x += kDecThreads) {
+    const int k = x / kSegBlocksMax, sl = x % kSegBlocksMax;
+    const int seg = seg_of(k);
+    int v = 0;
+    if (seg < total_segs) {
+      const int pair = seg / nsegC, sseg = seg % nsegC;
+      const int si = sseg * kSegC * kStageTokC / blk + sl;
+      if (si < topk) v = __ldg(idx + (size_t)pair * topk + si);
+    }
+    itab[x] = v;
+  }
+  __syncthreads();
   int pf_seg_k = 0, pf_sub = 0, pf_slot = 0;
   auto pf_valid = [&]() { return seg_of(pf_seg_k) < total_segs; };
   auto prefetch = [&]() {
     if (pf_valid()) {
-      if (zero_order && pf_sub == 0) issue_centroids(seg_of(pf_seg_k), pf_seg_k % kCenSlots);
-      issue(seg_of(pf_seg_k), pf_sub, pf_slot);
+      issue(pf_seg_k, seg_of(pf_seg_k), pf_sub, pf_slot);
       if (++pf_sub >= stages_in(seg_of(pf_seg_k))) {
         pf_sub = 0;
         ++pf_seg_k;
@@ -651,9 +644,6 @@ decode_exact_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
           qa0[kk] = hvalid ? lo : 0u;
           qa2[kk] = hvalid ? hi : 0u;
         }
-        __syncthreads();   // the previous pair's merge is done with qs
-        for (int x = tid; x < g * D; x += kDecThreads)
-          qs[x] = scale2 * __bfloat162float(q[((size_t)b * Hq + kh * g) * D + x]);
         cur_pair = pair;
       }
       m_run = -INFINITY;
@@ -726,52 +716,28 @@ decode_exact_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
         }
       }
       __syncthreads();
-      for (int hh = warp; hh < g; hh += kDecWarps) {
-        HeadState T;
+      for (int x = tid; x < g * D; x += kDecThreads) {
+        const int hh = x / D, c = x % D;
         float M = -INFINITY;
-        for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, mg[((size_t)w * kMaxGroup + hh) * (D + 2)]);
-        T.m = M;
-        T.l = 0.f;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) T.acc[c] = 0.f;
+        for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, mg[((size_t)w * kMaxGroup + hh) * (D + 2)]);
+        float L = 0.f, A = 0.f;
         if (M != -INFINITY) {
+#pragma unroll
           for (int w = 0; w < kDecWarps; ++w) {
             const float* mw = mg + ((size_t)w * kMaxGroup + hh) * (D + 2);
             if (mw[0] == -INFINITY) continue;
             const float f = fast_exp2(mw[0] - M);
-            if (lane == 0) T.l = fmaf(mw[1], f, T.l);
-            if (lane * 4 < D) {
-#pragma unroll
-              for (int c = 0; c < 4; ++c) T.acc[c] = fmaf(mw[2 + lane * 4 + c], f, T.acc[c]);
-            }
+            L = fmaf(mw[1], f, L);
+            A = fmaf(mw[2 + c], f, A);
           }
         }
-        if (zero_order) {
-          // subtract the zero-order term of each block of the segment
-          const int tb = sseg * kSegC * kStageTokC;
-          const int te = min(tok_pair, tb + kSegC * kStageTokC);
-          const float* qh = qs + hh * D;
-          const float* cb = cen + (cur_seg_k % kCenSlots) * kSegBlocksMax * 2 * D;
-          for (int sidx = tb / blk; sidx * blk < te; ++sidx) {
-            const float* kr = cb + ((sidx - tb / blk) * 2 + 0) * D;
-            const float* vr = cb + ((sidx - tb / blk) * 2 + 1) * D;
-            float d = 0.f;
-            for (int c = lane; c < D; c += 32) d = fmaf(qh[c], kr[c], d);
-            d = warp_sum(d);
-            const float cl = d + bias2;
-            const float m_new2 = fmaxf(T.m, cl);
-            const float corr2 = T.m == -INFINITY ? 0.f : fast_exp2(T.m - m_new2);
-            const float w = fast_exp2(cl - m_new2);
-            T.l = T.l * corr2 - (lane == 0 ? w : 0.f);
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              const float vv = lane * 4 < D ? vr[lane * 4 + c] * inv_blk : 0.f;
-              T.acc[c] = T.acc[c] * corr2 - w * vv;
-            }
-            T.m = m_new2;
-          }
+        float* out = partc + (((size_t)b * Hq + kh * g + hh) * nsegC + sseg) * (D + 2);
+        if (c == 0) {
+          out[0] = M;
+          out[1] = L;
         }
-        head_store<D>(T, partc + (((size_t)b * Hq + kh * g + hh) * nsegC + sseg) * (D + 2), lane);
+        out[2 + c] = A;
       }
       __syncthreads();
       cur_sub = 0;
@@ -782,35 +748,114 @@ decode_exact_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
 }
 
 // ---- D. merge ------------------------------------------------------------
+// One CTA of D threads per (query head, sequence), thread = channel.  It
+// merges the statistics pass's partial states (the zero-order term of every
+// block) with the exact pass's (the selected blocks token by token) under
+// their common maximum M, then subtracts the zero-order term of each
+// selected block (SPLA §2.2's subtraction applied to PISA's tail: the
+// statistics pass cannot know the selection), so that the tail holds the
+// unselected blocks only.  The subtraction cannot go below zero: for every
+// block Σ_n e^{x_n} ≥ B e^{mean x}, and M bounds every block's zero-order
+// logit, so no weight exceeds 1.
+// kParts x D threads: thread (part, channel); each part takes every
+// kParts-th partial state and selected block, and the parts' sums meet in
+// shared memory.  Shared memory (dynamic): per partial state its max, sum
+// and merge weight, per selected block its index and log2 zero-order
+// weight, then the parts' sums; loads that do not depend on one another are
+// issued together.
+constexpr int kParts = 4;
+
 template <int D>
-__global__ void decode_combine_kernel(const float* __restrict__ parta, int nsegA, const float* __restrict__ partc,
-                                      int nsegC, int use_tail, int Hq, __nv_bfloat16* __restrict__ O) {
-  const int h = blockIdx.x, b = blockIdx.y, c = threadIdx.x;
+__global__ void __launch_bounds__(kParts * D)
+decode_combine_kernel(const float* __restrict__ parta, int nsegA, const float* __restrict__ partc, int nsegC,
+                      int use_tail, const __nv_bfloat16* __restrict__ q, sa_block_stats st,
+                      const int32_t* __restrict__ idx, int topk, int nb, int blk, float scale, int Hq, int Hkv,
+                      __nv_bfloat16* __restrict__ O) {
+  constexpr int kT = kParts * D, kW = kT / 32;
+  extern __shared__ __align__(16) float csm[];
+  const int na = use_tail ? nsegA : 0, ns = na + nsegC;
+  const bool subtract = use_tail && nsegC > 0;
+  const int nsel = subtract ? topk : 0;
+  float* red = csm;                                        // [kParts][2][D] the parts' sums
+  float* hm = red + kParts * 2 * D;                        // [ns] partial maxima
+  float* hl = hm + ns;                                     // [ns] partial sums
+  float* hf = hl + ns;                                     // [ns] merge weights
+  float* xsel = hf + ns;                                   // [nsel] log2 zero-order weights
+  int* jsel = reinterpret_cast<int*>(xsel + nsel);         // [nsel] block indices
+  const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+  const int c = tid % D, pt = tid / D;
+  const int lane = tid & 31, warp = tid >> 5;
   const float* pa = parta + ((size_t)b * Hq + h) * nsegA * (D + 2);
   const float* pc = partc + ((size_t)b * Hq + h) * nsegC * (D + 2);
+  const int pair = b * Hkv + h / (Hq / Hkv);
+  auto part = [&](int sidx) { return sidx < na ? pa + (size_t)sidx * (D + 2) : pc + (size_t)(sidx - na) * (D + 2); };
+  for (int x = tid; x < ns; x += kT) {
+    const float* r = part(x);
+    hm[x] = r[0];
+    hl[x] = r[1];
+  }
+  for (int x = tid; x < nsel; x += kT) jsel[x] = __ldg(idx + (size_t)pair * topk + x);
+  __syncthreads();
   float M = -INFINITY;
-  if (use_tail)
-    for (int s = 0; s < nsegA; ++s) M = fmaxf(M, pa[s * (D + 2)]);
-  for (int s = 0; s < nsegC; ++s) M = fmaxf(M, pc[s * (D + 2)]);
-  float L = 0.f, A = 0.f;
-  if (M != -INFINITY) {
-    if (use_tail)
-      for (int s = 0; s < nsegA; ++s) {
-        const float* r = pa + s * (D + 2);
-        if (r[0] == -INFINITY) continue;
-        const float f = fast_exp2(r[0] - M);
-        L = fmaf(r[1], f, L);
-        A = fmaf(r[2 + c], f, A);
+  for (int x = 0; x < ns; ++x) M = fmaxf(M, hm[x]);
+  if (subtract && M != -INFINITY) {
+    // s log2e q·k̄_j + log2 B of the selected blocks: a warp per block, the
+    // rows of four blocks in flight at once
+    const float scale2 = scale * kLog2e, bias2 = log2f((float)blk);
+    float qv[D / 32];
+#pragma unroll
+    for (int e = 0; e < D / 32; ++e) qv[e] = scale2 * __bfloat162float(q[((size_t)b * Hq + h) * D + lane + 32 * e]);
+    for (int s0 = warp * 4; s0 < nsel; s0 += kW * 4) {
+      float kk[4][D / 32];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int si = min(s0 + u, nsel - 1);
+        const float* kr = st.kmean + ((size_t)pair * nb + jsel[si]) * D;
+#pragma unroll
+        for (int e = 0; e < D / 32; ++e) kk[u][e] = __ldg(kr + lane + 32 * e);
       }
-    for (int s = 0; s < nsegC; ++s) {
-      const float* r = pc + s * (D + 2);
-      if (r[0] == -INFINITY) continue;
-      const float f = fast_exp2(r[0] - M);
-      L = fmaf(r[1], f, L);
-      A = fmaf(r[2 + c], f, A);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        float d = 0.f;
+#pragma unroll
+        for (int e = 0; e < D / 32; ++e) d = fmaf(qv[e], kk[u][e], d);
+        d = warp_sum(d);
+        if (lane == 0 && s0 + u < nsel) xsel[s0 + u] = d + bias2;
+      }
     }
   }
-  O[((size_t)b * Hq + h) * D + c] = __float2bfloat16_rn(L > 0.f ? A / L : 0.f);
+  for (int x = tid; x < ns; x += kT) hf[x] = (M == -INFINITY || hm[x] == -INFINITY) ? 0.f : fast_exp2(hm[x] - M);
+  __syncthreads();
+  float L = 0.f, A = 0.f;
+  if (M != -INFINITY) {
+#pragma unroll 4
+    for (int x = pt; x < ns; x += kParts) {
+      const float f = hf[x];
+      L = fmaf(hl[x], f, L);
+      A = fmaf(part(x)[2 + c], f, A);
+    }
+    // subtract the zero-order term of each selected block (weight <= 1)
+    const float inv_blk = 1.0f / blk;
+#pragma unroll 8
+    for (int si = pt; si < nsel; si += kParts) {
+      const float w = fast_exp2(xsel[si] - M);
+      L -= w;
+      A = fmaf(-w * inv_blk, __ldg(st.vsum + ((size_t)pair * nb + jsel[si]) * D + c), A);
+    }
+  }
+  red[(pt * 2 + 0) * D + c] = L;
+  red[(pt * 2 + 1) * D + c] = A;
+  __syncthreads();
+  if (pt == 0) {
+    L = 0.f;
+    A = 0.f;
+#pragma unroll
+    for (int p2 = 0; p2 < kParts; ++p2) {
+      L += red[(p2 * 2 + 0) * D + c];
+      A += red[(p2 * 2 + 1) * D + c];
+    }
+    O[((size_t)b * Hq + h) * D + c] = __float2bfloat16_rn(L > 0.f ? A / L : 0.f);
+  }
 }
 
 int sm_count() {
@@ -871,8 +916,8 @@ sa_status launch_decode(const void* q, const void* Kc, const void* Vc, const sa_
 
   // C
   if (topk > 0) {
-    const size_t smemC = sizeof(float) * (kMaxGroup * D + kDecWarps * kMaxGroup * (D + 2) +
-                                          kRingC * (kSegC * kStageTokC / 64) * 2 * D) +
+    const size_t smemC = sizeof(float) * kDecWarps * kMaxGroup * (D + 2) +
+                         sizeof(int) * kItabSegs * (kSegC * kStageTokC / 64) +
                          (size_t)kRingC * 2 * kStageTokC * D * 2;
     if (cudaFuncSetAttribute(decode_exact_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smemC) !=
         cudaSuccess)
@@ -880,16 +925,26 @@ sa_status launch_decode(const void* q, const void* Kc, const void* Vc, const sa_
     const long segsC = (long)npairs * L.nsegC;   // < 2^31 for any supported shape
     const int gridC = (int)(segsC < sms ? segsC : sms);
     decode_exact_kernel<D><<<gridC, kDecThreads, smemC, stream>>>(
-        qb, static_cast<const __nv_bfloat16*>(Kc), static_cast<const __nv_bfloat16*>(Vc), st, s.Hq, s.Hkv, s.N,
-        s.block, idx, topk, tail == SA_TAIL_ZERO_ORDER, scale, L.nsegC, npairs, partc);
+        qb, static_cast<const __nv_bfloat16*>(Kc), static_cast<const __nv_bfloat16*>(Vc), s.Hq, s.Hkv, s.N,
+        s.block, idx, topk, scale, L.nsegC, npairs, partc);
     r = launch_status("decode_exact_kernel");
     if (r != SA_OK) return r;
   }
 
   // D
-  decode_combine_kernel<D><<<dim3(s.Hq, s.B), D, 0, stream>>>(parta, L.nsegA, partc, topk > 0 ? L.nsegC : 0,
-                                                             tail == SA_TAIL_ZERO_ORDER, s.Hq,
-                                                             static_cast<__nv_bfloat16*>(O));
+  {
+    const int use_tail = tail == SA_TAIL_ZERO_ORDER;
+    const int nsc = topk > 0 ? L.nsegC : 0;
+    const int ns = (use_tail ? L.nsegA : 0) + nsc;
+    const int nsel = (use_tail && nsc > 0) ? topk : 0;
+    const size_t smemD = sizeof(float) * (kParts * 2 * D + 3 * (size_t)ns + 2 * (size_t)nsel);
+    if (cudaFuncSetAttribute(decode_combine_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smemD) !=
+        cudaSuccess)
+      return launch_status("cudaFuncSetAttribute(decode_combine_kernel)");
+    decode_combine_kernel<D><<<dim3(s.Hq, s.B), kParts * D, smemD, stream>>>(
+        parta, L.nsegA, partc, nsc, use_tail, qb, st, idx, topk, nb, s.block, scale, s.Hq, s.Hkv,
+        static_cast<__nv_bfloat16*>(O));
+  }
   return launch_status("decode_combine_kernel");
 }
 
