@@ -7,157 +7,282 @@
 // u_i = P_k P_qᵀ q̄_i (x P is the row vector x times P), so no projected copy
 // of the key centroids is needed: u_i costs 2d² multiply-adds per query block.
 //
-// One CTA handles kRouteQB query blocks of one head (one warp each), so every
-// centroid tile it stages in shared memory serves kRouteQB score rows.  Scores
-// are computed with lane = KV block (a full dot product per lane against a
-// padded shared-memory row).  Selection: for small k each warp takes its k
-// winners by repeated warp arg-max over (score desc, index asc) keys, then
-// emits them in ascending order from a bitmap; for large k the CTA sorts each
-// row with a bitonic sort.
+// One CTA handles QB = 8 RPW query blocks of one head.  The scores of its QB
+// rows against all nb centroids are a small fp32 matrix product, done tile
+// by tile: TJ = 32 NCOL centroid rows are staged by cp.async into shared
+// memory rows padded to d + 4 floats (two buffers, so the next tile lands
+// while this one is used); warp w owns rows [w RPW, w RPW + RPW) and lane l
+// the centroids l, l + 32, ... of the tile, reading its centroid rows as
+// float4 without bank conflicts and the query rows as warp broadcasts.  The
+// proj vector u_i = P_k t_i (t_i = q̄_i P_q) takes the same path with the
+// rows of P_k in place of centroids.  Selection: for small k each warp finds
+// the key of the k-th best block of each of its rows by a radix select (one
+// bit per step, counted with a warp reduction), keeps the blocks above it
+// and the smallest indices among those equal to it, and emits them in
+// ascending order from a bitmap; for large k the CTA sorts each row with a
+// bitonic sort.
 #include "topk.cuh"
 
 namespace sa {
 namespace {
 
 constexpr int kRouteThreads = 256;
-constexpr int kRouteQB = kRouteThreads / 32;   // query blocks per CTA
-constexpr int kRouteTile = 32;                 // centroids per shared-memory tile
-constexpr int kWarpTopkMax = 64;               // largest k taken by the warp arg-max path
+constexpr int kRouteWarps = kRouteThreads / 32;
+constexpr int kWarpTopkMax = 64;               // largest k taken by the warp radix select
+constexpr int kRegKeys = 16;                   // keys per lane kept in registers (rows of <= 512 blocks)
+constexpr size_t kMaxSmemPerCta = 232448;      // opt-in shared memory of one CTA on sm_100
+constexpr size_t kSmemTwoPerSm = 115712;       // per CTA when two share an SM (233472 / 2 - 1 KB)
 
-__device__ __forceinline__ unsigned long long rank_key(float score, int j) {
-  // smaller key = better: higher score first, then smaller index
-  return ((unsigned long long)(~order_key(score)) << 32) | (unsigned)j;
+__device__ __forceinline__ void cp_async16r(float* smem_dst, const float* gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(smem_dst)),
+               "l"(gsrc)
+               : "memory");
 }
 
-__device__ __forceinline__ unsigned long long warp_min_u64(unsigned long long v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const unsigned long long w = __shfl_xor_sync(0xffffffffu, v, o);
-    v = w < v ? w : v;
+// Stages rows [r0, r0 + n) of a [rows][D] float array into `dst` (TJ rows
+// of D + 4 floats); rows past n are zero-filled.
+template <int D, int TJ>
+__device__ __forceinline__ void stage_rows(float* dst, const float* src, int r0, int n) {
+  constexpr int C4 = D / 4;
+  for (int x = threadIdx.x; x < TJ * C4; x += kRouteThreads) {
+    const int r = x / C4, c = x % C4;
+    float* d = dst + r * (D + 4) + 4 * c;
+    if (r < n) cp_async16r(d, src + (size_t)(r0 + r) * D + 4 * c);
+    else *reinterpret_cast<float4*>(d) = make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  return v;
 }
 
-template <int D>
+// out[r][n] = A[r]·T[lane + 32 n] for the warp's RPW rows of A ([.][D],
+// read as broadcasts) and the lane's NCOL rows of the tile T ([TJ][D + 4]).
+template <int D, int RPW, int NCOL>
+__device__ __forceinline__ void tile_dots(const float* A, const float* T, int lane, float (&out)[RPW][NCOL]) {
+#pragma unroll
+  for (int r = 0; r < RPW; ++r)
+#pragma unroll
+    for (int n = 0; n < NCOL; ++n) out[r][n] = 0.f;
+#pragma unroll 4
+  for (int c = 0; c < D; c += 4) {
+    float4 t[NCOL];
+#pragma unroll
+    for (int n = 0; n < NCOL; ++n) t[n] = *reinterpret_cast<const float4*>(T + (lane + 32 * n) * (D + 4) + c);
+#pragma unroll
+    for (int r = 0; r < RPW; ++r) {
+      const float4 a = *reinterpret_cast<const float4*>(A + r * D + c);
+#pragma unroll
+      for (int n = 0; n < NCOL; ++n) {
+        out[r][n] = fmaf(a.x, t[n].x, out[r][n]);
+        out[r][n] = fmaf(a.y, t[n].y, out[r][n]);
+        out[r][n] = fmaf(a.z, t[n].z, out[r][n]);
+        out[r][n] = fmaf(a.w, t[n].w, out[r][n]);
+      }
+    }
+  }
+}
+
+template <int D, int RPW, int NCOL>
 __global__ void __launch_bounds__(kRouteThreads)
 route_kernel(sa_block_stats st, int H, int nb, sa_route_mode mode, const float* __restrict__ Pq,
              const float* __restrict__ Pk, float scale, int topk, int32_t* __restrict__ block_idx,
              float* __restrict__ scores_out) {
-  constexpr int KS = D + 1;
+  constexpr int QB = kRouteWarps * RPW;          // query blocks per CTA
+  constexpr int TJ = 32 * NCOL;                  // centroids per tile
+  constexpr int TS = TJ * (D + 4);               // floats per staged tile
   const int h = blockIdx.y, b = blockIdx.z;
-  const int i0 = blockIdx.x * kRouteQB;
+  const int i0 = blockIdx.x * QB;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int i = i0 + warp;                       // this warp's query block
-  const bool has_row = i < nb;
   const size_t bh = (size_t)b * H + h;
   const bool t2 = mode == SA_ROUTE_TAYLOR2;
+  const int narr = t2 ? 2 : 1;                   // staged arrays per tile
 
-  extern __shared__ float rsm[];
-  float* u = rsm;                                // [QB][D]  query vector per warp
-  float* w = u + kRouteQB * D;                   // [QB][D]  ½ s² q̄² (taylor2) / scratch (proj)
-  float* kt = w + kRouteQB * D;                  // [TILE][KS] centroid tile
-  float* vt = kt + kRouteTile * KS;              // [TILE][KS] variance tile (taylor2)
+  extern __shared__ __align__(16) float rsm[];
+  float* u = rsm;                                // [QB][D]  query vectors
+  float* w = u + QB * D;                         // [QB][D]  ½ s² q̄² (taylor2) / q̄ P_q (proj)
+  float* tiles = w + QB * D;                     // [2 buffers][narr][TS]
   // the tile region doubles as the sort keys of the large-k path
-  int tile_floats = 2 * kRouteTile * KS;
+  size_t tile_floats = 2 * (size_t)narr * TS;
   if (topk > kWarpTopkMax) {
     int n2 = 1;
     while (n2 < nb) n2 <<= 1;
-    if (2 * n2 > tile_floats) tile_floats = 2 * n2;
+    if (2 * (size_t)n2 > tile_floats) tile_floats = 2 * (size_t)n2;
   }
-  float* sc = kt + tile_floats;                  // [QB][nb] scores
+  float* sc = tiles + tile_floats;               // [QB][nb] scores
   const int nwords = (nb + 31) >> 5;
-  uint32_t* bits = reinterpret_cast<uint32_t*>(sc + (size_t)kRouteQB * nb);   // [QB][nwords]
+  uint32_t* bits = reinterpret_cast<uint32_t*>(sc + (size_t)QB * nb);   // [QB][nwords]
 
-  // ---- query vectors (one warp per query block)
-  float* uw = u + warp * D;
-  float* ww = w + warp * D;
-  for (int c = lane; c < D; c += 32) {
-    const float q = has_row ? st.qmean[(bh * nb + i) * D + c] : 0.f;
-    uw[c] = t2 ? scale * q : q;
-    ww[c] = 0.5f * scale * scale * q * q;
+  // ---- query vectors
+  for (int x = tid; x < QB * D; x += kRouteThreads) {
+    const int r = x / D, c = x % D;
+    const int i = i0 + r;
+    const float q = i < nb ? st.qmean[(bh * nb + i) * D + c] : 0.f;
+    u[x] = t2 ? scale * q : q;
+    w[x] = 0.5f * scale * scale * q * q;
   }
-  __syncwarp();
+  __syncthreads();
   if (mode == SA_ROUTE_PROJ) {
-    // t = q̄ P_q (into ww), then u = P_k t
-    float tq[D / 32];
+    // t = q̄ P_q into w: rows of P_q staged as tiles; lane = output columns
+    // lane + 32 p, read from the tile rows without bank conflicts
+    float tq[RPW][D / 32];
 #pragma unroll
-    for (int p = 0; p < D / 32; ++p) {
-      const int c = lane + 32 * p;
-      float a = 0.f;
-      for (int r = 0; r < D; ++r) a = fmaf(uw[r], __ldg(Pq + (size_t)r * D + c), a);
-      tq[p] = a;
+    for (int r = 0; r < RPW; ++r)
+#pragma unroll
+      for (int p = 0; p < D / 32; ++p) tq[r][p] = 0.f;
+    for (int k0 = 0; k0 < D; k0 += TJ) {
+      __syncthreads();
+      stage_rows<D, TJ>(tiles, Pq, k0, min(TJ, D - k0));
+      asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+      __syncthreads();
+      for (int k = 0; k < TJ && k0 + k < D; ++k) {
+        const float* trow = tiles + k * (D + 4);
+#pragma unroll
+        for (int r = 0; r < RPW; ++r) {
+          const float a = u[(warp * RPW + r) * D + k0 + k];
+#pragma unroll
+          for (int p = 0; p < D / 32; ++p) tq[r][p] = fmaf(a, trow[lane + 32 * p], tq[r][p]);
+        }
+      }
     }
-    __syncwarp();
 #pragma unroll
-    for (int p = 0; p < D / 32; ++p) ww[lane + 32 * p] = tq[p];
-    __syncwarp();
+    for (int r = 0; r < RPW; ++r)
 #pragma unroll
-    for (int p = 0; p < D / 32; ++p) {
-      const int rr = lane + 32 * p;
-      const float* row = Pk + (size_t)rr * D;
-      float a = 0.f;
-      for (int e = 0; e < D; ++e) a = fmaf(__ldg(row + e), ww[e], a);
-      tq[p] = a;
+      for (int p = 0; p < D / 32; ++p) w[(warp * RPW + r) * D + lane + 32 * p] = tq[r][p];
+    __syncwarp();
+    // ... then u = P_k t, with the rows of P_k staged like centroid tiles
+    for (int r0 = 0; r0 < D; r0 += TJ) {
+      __syncthreads();
+      stage_rows<D, TJ>(tiles, Pk, r0, min(TJ, D - r0));
+      asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+      __syncthreads();
+      float o[RPW][NCOL];
+      tile_dots<D, RPW, NCOL>(w + warp * RPW * D, tiles, lane, o);
+#pragma unroll
+      for (int r = 0; r < RPW; ++r)
+#pragma unroll
+        for (int n = 0; n < NCOL; ++n)
+          if (r0 + lane + 32 * n < D) u[(warp * RPW + r) * D + r0 + lane + 32 * n] = o[r][n];
     }
-    __syncwarp();
-#pragma unroll
-    for (int p = 0; p < D / 32; ++p) uw[lane + 32 * p] = tq[p];
-    __syncwarp();
+    __syncthreads();
   }
 
-  // ---- scores: tiles of 32 centroids shared by the CTA's warps
+  // ---- scores: tiles of TJ centroids, two buffers
   const float* km = st.kmean + bh * (size_t)nb * D;
   const float* kv = t2 ? st.kvar + bh * (size_t)nb * D : nullptr;
-  float* scw = sc + (size_t)warp * nb;
-  for (int j0 = 0; j0 < nb; j0 += kRouteTile) {
-    __syncthreads();
-    for (int idx = tid; idx < kRouteTile * D; idx += kRouteThreads) {
-      const int n = idx / D, c = idx % D;
-      const int j = j0 + n;
-      kt[n * KS + c] = j < nb ? km[(size_t)j * D + c] : 0.f;
-      if (t2) vt[n * KS + c] = j < nb ? kv[(size_t)j * D + c] : 0.f;
+  const int ntiles = (nb + TJ - 1) / TJ;
+  auto stage = [&](int t, int buf) {
+    const int j0 = t * TJ, n = min(TJ, nb - j0);
+    stage_rows<D, TJ>(tiles + (size_t)buf * narr * TS, km, j0, n);
+    if (t2) stage_rows<D, TJ>(tiles + (size_t)buf * narr * TS + TS, kv, j0, n);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  stage(0, 0);
+  for (int t = 0; t < ntiles; ++t) {
+    if (t + 1 < ntiles) {
+      stage(t + 1, (t + 1) & 1);
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+    } else {
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
     }
     __syncthreads();
-    const int j = j0 + lane;
-    float s1 = 0.f, s2 = 0.f;
-    const float* kr = kt + lane * KS;
-#pragma unroll 8
-    for (int c = 0; c < D; ++c) s1 = fmaf(uw[c], kr[c], s1);
+    const float* tk = tiles + (size_t)(t & 1) * narr * TS;
+    float o[RPW][NCOL];
+    tile_dots<D, RPW, NCOL>(u + warp * RPW * D, tk, lane, o);
     if (t2) {
-      const float* vr = vt + lane * KS;
-#pragma unroll 8
-      for (int c = 0; c < D; ++c) s2 = fmaf(ww[c], vr[c], s2);
-      s1 += log1pf(s2);
+      float o2[RPW][NCOL];
+      tile_dots<D, RPW, NCOL>(w + warp * RPW * D, tk + TS, lane, o2);
+#pragma unroll
+      for (int r = 0; r < RPW; ++r)
+#pragma unroll
+        for (int n = 0; n < NCOL; ++n) o[r][n] += log1pf(o2[r][n]);
     }
-    if (j < nb) scw[j] = s1;
+#pragma unroll
+    for (int r = 0; r < RPW; ++r)
+#pragma unroll
+      for (int n = 0; n < NCOL; ++n) {
+        const int j = t * TJ + lane + 32 * n;
+        if (j < nb) sc[(size_t)(warp * RPW + r) * nb + j] = o[r][n];
+      }
+    __syncthreads();   // this buffer is restaged by the next iteration's prefetch
   }
-  __syncwarp();
-  if (has_row && scores_out) {
-    float* so = scores_out + (bh * nb + i) * (size_t)nb;
-    for (int j = lane; j < nb; j += 32) so[j] = scw[j];
+  if (scores_out) {
+    for (int r = warp * RPW; r < warp * RPW + RPW; ++r) {
+      const int i = i0 + r;
+      if (i >= nb) break;
+      float* so = scores_out + (bh * nb + i) * (size_t)nb;
+      for (int j = lane; j < nb; j += 32) so[j] = sc[(size_t)r * nb + j];
+    }
   }
 
   // ---- selection
   if (topk <= kWarpTopkMax) {
-    uint32_t* bw = bits + (size_t)warp * nwords;
-    for (int x = lane; x < nwords; x += 32) bw[x] = 0u;
-    __syncwarp();
-    if (has_row) {
-      // repeated arg-max: round r takes the best key strictly worse than the
-      // previous round's winner (keys are distinct: they carry the index)
-      unsigned long long prev = 0ull;
-      for (int r = 0; r < topk; ++r) {
-        unsigned long long mine = ~0ull;
-        for (int j = lane; j < nb; j += 32) {
-          const unsigned long long k = rank_key(scw[j], j);
-          if ((r == 0 || k > prev) && k < mine) mine = k;
+    for (int r = warp * RPW; r < warp * RPW + RPW; ++r) {
+      const int i = i0 + r;
+      if (i >= nb) break;
+      const float* scw = sc + (size_t)r * nb;
+      uint32_t* bw = bits + (size_t)r * nwords;
+      // radix select: the key T of the k-th best block, one bit at a time
+      // from the top.  `cand` counts the blocks whose high bits equal
+      // `prefix`, `want` the places left for them; once the two agree every
+      // candidate is kept and the bits below do not matter.  Rows of up to
+      // 512 blocks keep their keys in registers.
+      unsigned prefix = 0u, hi = 0u;
+      int want = topk, cand = nb;
+      if (nb <= 32 * kRegKeys) {
+        unsigned key[kRegKeys];
+#pragma unroll
+        for (int m = 0; m < kRegKeys; ++m) {
+          const int j = lane + 32 * m;
+          key[m] = j < nb ? order_key(scw[j]) : 0u;
         }
-        const unsigned long long best = warp_min_u64(mine);
-        if (lane == 0) {
-          const int jb = (int)(best & 0xffffffffu);
-          bw[jb >> 5] |= 1u << (jb & 31);
+        for (int bit = 31; bit >= 0; --bit) {
+          const unsigned bm = 1u << bit;
+          unsigned c = 0u;
+#pragma unroll
+          for (int m = 0; m < kRegKeys; ++m)
+            c += (lane + 32 * m < nb && (key[m] & hi) == prefix && (key[m] & bm)) ? 1u : 0u;
+          c = __reduce_add_sync(0xffffffffu, c);
+          if ((int)c >= want) {
+            prefix |= bm;
+            cand = (int)c;
+          } else {
+            want -= (int)c;
+            cand -= (int)c;
+          }
+          hi |= bm;
+          if (cand == want) break;
         }
-        prev = best;
+      } else {
+        for (int bit = 31; bit >= 0; --bit) {
+          const unsigned bm = 1u << bit;
+          unsigned c = 0u;
+          for (int j = lane; j < nb; j += 32) {
+            const unsigned key = order_key(scw[j]);
+            c += ((key & hi) == prefix && (key & bm)) ? 1u : 0u;
+          }
+          c = __reduce_add_sync(0xffffffffu, c);
+          if ((int)c >= want) {
+            prefix |= bm;
+            cand = (int)c;
+          } else {
+            want -= (int)c;
+            cand -= (int)c;
+          }
+          hi |= bm;
+          if (cand == want) break;
+        }
+      }
+      // keep every key above T and, of the keys equal to T, the smallest
+      // indices (after an early exit: every key whose high bits reach prefix)
+      const bool all_cand = cand == want;
+      for (int m = 0; m < nwords; ++m) {
+        const int j = 32 * m + lane;
+        const unsigned key = j < nb ? order_key(scw[j]) : 0u;
+        const bool eq = j < nb && key == prefix;
+        const unsigned eqb = __ballot_sync(0xffffffffu, eq);
+        const int before = __popc(eqb & ((1u << lane) - 1u));
+        const bool keep = all_cand ? (j < nb && (key & hi) >= prefix)
+                                   : ((j < nb && key > prefix) || (eq && before < want));
+        const unsigned take = __ballot_sync(0xffffffffu, keep);
+        if (lane == 0) bw[m] = take;
+        want -= min(want, __popc(eqb));
       }
       __syncwarp();
       // ascending emission from the bitmap
@@ -186,22 +311,52 @@ route_kernel(sa_block_stats st, int H, int nb, sa_route_mode mode, const float* 
   } else {
     // large k: each row in turn is sorted by the whole CTA
     __syncthreads();
-    unsigned long long* keys = reinterpret_cast<unsigned long long*>(kt);   // reuses the tile space
-    for (int q = 0; q < kRouteQB && i0 + q < nb; ++q)
-      block_topk_ascending(sc + (size_t)q * nb, nb, topk, keys,
-                           block_idx + (bh * nb + i0 + q) * (size_t)topk);
+    unsigned long long* keys = reinterpret_cast<unsigned long long*>(tiles);   // reuses the tile space
+    for (int r = 0; r < QB && i0 + r < nb; ++r)
+      block_topk_ascending(sc + (size_t)r * nb, nb, topk, keys,
+                           block_idx + (bh * nb + i0 + r) * (size_t)topk);
   }
 }
 
-size_t route_smem_bytes(int nb, int d, int topk) {
+struct RouteCfg {
+  int rpw, ncol;
+};
+
+size_t route_smem_bytes(int nb, int d, int topk, bool t2, RouteCfg c) {
+  const int qb = kRouteWarps * c.rpw;
   const int nwords = (nb + 31) / 32;
-  size_t tiles = 2 * (size_t)kRouteTile * (d + 1) * 4;
+  size_t tiles = 2 * (size_t)(t2 ? 2 : 1) * 32 * c.ncol * (d + 4);
   if (topk > kWarpTopkMax) {
     int n2 = 1;
     while (n2 < nb) n2 <<= 1;
-    if ((size_t)n2 * 8 > tiles) tiles = (size_t)n2 * 8;
+    if (2 * (size_t)n2 > tiles) tiles = 2 * (size_t)n2;
   }
-  return 2 * (size_t)kRouteQB * d * 4 + tiles + (size_t)kRouteQB * nb * 4 + (size_t)kRouteQB * nwords * 4;
+  return 4 * (2 * (size_t)qb * d + tiles + (size_t)qb * nb + (size_t)qb * nwords);
+}
+
+// Rows per warp and centroid columns per lane: the first of (2, 2), (2, 1),
+// (1, 2), (1, 1) that lets two CTAs share an SM, else the first that fits
+// in one CTA.
+RouteCfg route_cfg(int nb, int d, int topk, bool t2) {
+  const RouteCfg order[4] = {{2, 2}, {2, 1}, {1, 2}, {1, 1}};
+  for (const RouteCfg& c : order)
+    if (route_smem_bytes(nb, d, topk, t2, c) <= kSmemTwoPerSm) return c;
+  for (const RouteCfg& c : order)
+    if (route_smem_bytes(nb, d, topk, t2, c) <= kMaxSmemPerCta) return c;
+  return order[3];
+}
+
+template <int D, int RPW, int NCOL>
+sa_status launch_route(const sa_block_stats& st, sa_shape shape, int nb, sa_route_mode mode, const float* Pq,
+                       const float* Pk, float scale, int topk, int32_t* idx, float* scores, size_t smem,
+                       cudaStream_t s) {
+  auto kern = route_kernel<D, RPW, NCOL>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return launch_status("cudaFuncSetAttribute(route_kernel)");
+  constexpr int QB = kRouteWarps * RPW;
+  dim3 grid((nb + QB - 1) / QB, shape.H, shape.B);
+  kern<<<grid, kRouteThreads, smem, s>>>(st, shape.H, nb, mode, Pq, Pk, scale, topk, idx, scores);
+  return launch_status("route_kernel");
 }
 
 }  // namespace
@@ -228,19 +383,21 @@ extern "C" sa_status sa_route(const sa_block_stats* stats, sa_shape shape, sa_ro
   const void* ptrs[] = {stats->qmean, stats->kmean, stats->kvar, proj_q, proj_k, block_idx, scores};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return fail(SA_ERR_ALIGNMENT, "sa_route: pointers must be 16-byte aligned");
-  const size_t smem = route_smem_bytes(nb, shape.d, topk);
-  dim3 grid((nb + kRouteQB - 1) / kRouteQB, shape.H, shape.B);
+  const bool t2 = mode == SA_ROUTE_TAYLOR2;
+  const RouteCfg cfg = route_cfg(nb, shape.d, topk, t2);
+  const size_t smem = route_smem_bytes(nb, shape.d, topk, t2, cfg);
   cudaStream_t s = as_stream(stream);
-  if (shape.d == 128) {
-    if (cudaFuncSetAttribute(route_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-      return launch_status("cudaFuncSetAttribute(route_kernel)");
-    route_kernel<128><<<grid, kRouteThreads, smem, s>>>(*stats, shape.H, nb, mode, proj_q, proj_k,
-                                                        scale, topk, block_idx, scores);
-  } else {
-    if (cudaFuncSetAttribute(route_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-      return launch_status("cudaFuncSetAttribute(route_kernel)");
-    route_kernel<64><<<grid, kRouteThreads, smem, s>>>(*stats, shape.H, nb, mode, proj_q, proj_k,
-                                                       scale, topk, block_idx, scores);
+  const sa_block_stats& st = *stats;
+  const int key = (shape.d == 128 ? 4 : 0) + (cfg.rpw == 2 ? 2 : 0) + (cfg.ncol == 2 ? 1 : 0);
+  switch (key) {
+    case 7: return launch_route<128, 2, 2>(st, shape, nb, mode, proj_q, proj_k, scale, topk, block_idx, scores, smem, s);
+    case 6: return launch_route<128, 2, 1>(st, shape, nb, mode, proj_q, proj_k, scale, topk, block_idx, scores, smem, s);
+    case 5: return launch_route<128, 1, 2>(st, shape, nb, mode, proj_q, proj_k, scale, topk, block_idx, scores, smem, s);
+    case 4: return launch_route<128, 1, 1>(st, shape, nb, mode, proj_q, proj_k, scale, topk, block_idx, scores, smem, s);
+    case 3: return launch_route<64, 2, 2>(st, shape, nb, mode, proj_q, proj_k, scale, topk, block_idx, scores, smem, s);
+    case 2: return launch_route<64, 2, 1>(st, shape, nb, mode, proj_q, proj_k, scale, topk, block_idx, scores, smem, s);
+    case 1: return launch_route<64, 1, 2>(st, shape, nb, mode, proj_q, proj_k, scale, topk, block_idx, scores, smem, s);
+    default: return launch_route<64, 1, 1>(st, shape, nb, mode, proj_q, proj_k, scale, topk, block_idx, scores, smem, s);
   }
-  return launch_status("route_kernel");
 }
+
