@@ -201,15 +201,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   // selection bitmap, padded with 4 zero words so a tile's 4 words never run past it
   for (int w = threadIdx.x; w < nwords + 4; w += kTcThreads) selmask[w] = 0u;
   if (warp == 0) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
-  __syncthreads();
-  for (int s = threadIdx.x; s < topk; s += kTcThreads) {
-    const int j = sel[s];
-    atomicOr(&selmask[j >> 5], 1u << (j & 31));
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
+  // The producer and MMA warps start at once; the softmax warps fill the
+  // bitmap (read only by them, at the centroid tiles) under their own barrier.
 
   if (warp == kTmaWarp) {
     // ------------------------------------------------------------ producer
@@ -306,6 +303,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   } else {
     // ------------------------------------------------------------ softmax
     regs_inc<kSoftmaxRegs>();
+    for (int s = threadIdx.x; s < topk; s += 256) {
+      const int j = sel[s];
+      atomicOr(&selmask[j >> 5], 1u << (j & 31));
+    }
+    named_bar_softmax();                        // the bitmap is complete
     const int st = warp >> 2;                   // stream
     const int wq = warp & 3;                    // TMEM lane quarter
     const int r = wq * 32 + lane;               // query row
