@@ -254,18 +254,20 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     if (lane == 0 && T > 0) {
       constexpr uint32_t idS = F8 ? idesc_e4m3_f32(TB, TB, 0) : idesc_bf16_f32(TB, TB, 0, 0);
       constexpr uint32_t idO = F8 ? idesc_e4m3_f32(TB, TD, 1) : idesc_bf16_f32(TB, TD, 0, 1);
+      // descriptors are built once per operand tile and advanced per K step
+      const uint64_t qd0 = desc_sw128(sb, 16, 1024);
       // S(t) = Q K_tᵀ into the S columns of stream t % 2
       auto issue_s = [&](int t) -> bool {
         const int s = t % NS;
         if (!mbar_wait(bar(L::B_KF + s), (t / NS) & 1, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t ka = sb + kTile * (1 + 2 * s);
+        const uint64_t kd0 = desc_sw128(sb + kTile * (1 + 2 * s), 16, 1024);
         const uint32_t d = tbase + (uint32_t)(t & 1) * TB;
 #pragma unroll
         for (int k = 0; k < TD / kK; ++k) {
           // K step k: 32 bytes further along the row, next span every 4 steps
           const uint32_t koff = (k >> 2) * kSpan + (k & 3) * 32;
-          const uint64_t a = desc_sw128(sb + koff, 16, 1024), b = desc_sw128(ka + koff, 16, 1024);
+          const uint64_t a = desc_adv(qd0, koff), b = desc_adv(kd0, koff);
           if (F8) mma_ss_f8(d, a, b, idS, k > 0);
           else mma_ss(d, a, b, idS, k > 0);
         }
@@ -280,13 +282,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (!mbar_wait(bar(L::B_PR + st), u & 1, abort_flag)) break;
         if (!mbar_wait(bar(L::B_VF + su), (t / NS) & 1, abort_flag)) break;
         tc_fence_after();
-        const uint32_t va = sb + kTile * (2 + 2 * su);
+        const uint64_t vd0 = desc_sw128(sb + kTile * (2 + 2 * su), kSpan, 1024);
         const uint32_t pa = tbase + (uint32_t)st * TB;
         const uint32_t od = tbase + kColO + (uint32_t)st * TD;
 #pragma unroll
         for (int k = 0; k < TB / kK; ++k) {
           // K step k: kK keys = kK rows of 128 bytes further into V; 8 TMEM columns of P
-          const uint64_t b = desc_sw128(va + k * kK * 128, kSpan, 1024);
+          const uint64_t b = desc_adv(vd0, k * kK * 128);
           if (F8) mma_ts_f8(od, pa + k * 8, b, idO, (u > 0 || k > 0));
           else mma_ts(od, pa + k * 8, b, idO, (u > 0 || k > 0));
         }

@@ -139,6 +139,14 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr, uint32_t lbo, uin
   return d;
 }
 
+// The descriptor of the operand `bytes` further on: only the start-address
+// field (bits 0-13, 16-byte units) changes, and for shared-memory addresses
+// below 256 KB no carry leaves it, so one 32-bit add on the low word does.
+__device__ __forceinline__ uint64_t desc_adv(uint64_t d, uint32_t bytes) {
+  const uint32_t lo = (uint32_t)d + (bytes >> 4), hi = (uint32_t)(d >> 32);
+  return ((uint64_t)hi << 32) | lo;
+}
+
 // Instruction descriptor of kind::f16 with bf16 A/B and fp32 accumulation.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn_major, int b_mn_major) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn_major << 15) |
