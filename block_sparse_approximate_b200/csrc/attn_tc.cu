@@ -27,7 +27,8 @@
 //              by more than 2^8;
 //   warp 8     TMA producer: Q once, then K/V tiles into a 3-stage ring;
 //   warps 10-11 idle (they complete the producer warpgroup);
-//   warp 9     MMA issuer: S = Q·Kᵀ (both operands K-major in shared memory)
+//   warp 9     MMA issuer (the whole warp runs the loop, one elected lane
+//              issues): S = Q·Kᵀ (both operands K-major in shared memory)
 //              into the stream's S, and O_s += P·V with P read from TMEM and V
 //              as an MN-major shared-memory operand, alternating the streams
 //              so one group's softmax overlaps the other group's MMAs.
@@ -123,6 +124,37 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity) {
 __device__ __forceinline__ void named_bar_softmax() {
   // barrier 1 over the two softmax warpgroups (256 threads)
   asm volatile("bar.sync 1, 256;" ::: "memory");
+}
+
+// MMA issue from a converged warp: the whole MMA warp runs the issue loop
+// (its descriptors and addresses are warp-uniform) and elect.sync picks the
+// one lane that issues each tcgen05 instruction.  The same loop run by lane
+// 0 alone issued its instructions much more slowly while the softmax warps
+// kept the FMA pipes of its sub-partition busy (measured on B200: 7% of the
+// whole kernel).
+__device__ __forceinline__ void mma_ss_w(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile("{\n\t.reg .pred p, e;\n\telect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+               "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %5, %5, %5}, p;\n\t}"
+               ::"r"(d), "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(0u) : "memory");
+}
+__device__ __forceinline__ void mma_ts_w(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile("{\n\t.reg .pred p, e;\n\telect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+               "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %5, %5, %5}, p;\n\t}"
+               ::"r"(d), "r"(a), "l"(b), "r"(idesc), "r"(acc), "r"(0u) : "memory");
+}
+__device__ __forceinline__ void mma_ss_f8_w(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile("{\n\t.reg .pred p, e;\n\telect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+               "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, {%5, %5, %5, %5}, p;\n\t}"
+               ::"r"(d), "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(0u) : "memory");
+}
+__device__ __forceinline__ void mma_ts_f8_w(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile("{\n\t.reg .pred p, e;\n\telect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+               "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, {%5, %5, %5, %5}, p;\n\t}"
+               ::"r"(d), "r"(a), "l"(b), "r"(idesc), "r"(acc), "r"(0u) : "memory");
+}
+__device__ __forceinline__ void mma_commit_w(uint32_t bar) {
+  asm volatile("{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+               "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(bar) : "memory");
 }
 
 __device__ __forceinline__ void mma_ss_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
@@ -251,7 +283,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     regs_dec<kProducerRegs>();
-    if (lane == 0 && T > 0) {
+    if (T > 0) {
       constexpr uint32_t idS = F8 ? idesc_e4m3_f32(TB, TB, 0) : idesc_bf16_f32(TB, TB, 0, 0);
       constexpr uint32_t idO = F8 ? idesc_e4m3_f32(TB, TD, 1) : idesc_bf16_f32(TB, TD, 0, 1);
       // descriptors are built once per operand tile and advanced per K step
@@ -259,7 +291,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       // S(t) = Q K_tᵀ into the S columns of stream t % 2
       auto issue_s = [&](int t) -> bool {
         const int s = t % NS;
-        if (!mbar_wait(bar(L::B_KF + s), (t / NS) & 1, abort_flag)) return false;
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_KF + s), (t / NS) & 1, abort_flag))) return false;
         tc_fence_after();
         const uint64_t kd0 = desc_sw128(sb + kTile * (1 + 2 * s), 16, 1024);
         const uint32_t d = tbase + (uint32_t)(t & 1) * TB;
@@ -268,19 +300,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           // K step k: 32 bytes further along the row, next span every 4 steps
           const uint32_t koff = (k >> 2) * kSpan + (k & 3) * 32;
           const uint64_t a = desc_adv(qd0, koff), b = desc_adv(kd0, koff);
-          if (F8) mma_ss_f8(d, a, b, idS, k > 0);
-          else mma_ss(d, a, b, idS, k > 0);
+          if (F8) mma_ss_f8_w(d, a, b, idS, k > 0);
+          else mma_ss_w(d, a, b, idS, k > 0);
         }
-        mma_commit(bar(L::B_SF + (t & 1)));
+        mma_commit_w(bar(L::B_SF + (t & 1)));
         return true;
       };
-      bool ok = mbar_wait(bar(L::B_Q), 0, abort_flag);
+      bool ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_Q), 0, abort_flag));
       if (ok) ok = issue_s(0);
       if (ok && T > 1) ok = issue_s(1);
       for (int t = 0; ok && t < T; ++t) {
         const int st = t & 1, u = t >> 1, su = t % NS;
-        if (!mbar_wait(bar(L::B_PR + st), u & 1, abort_flag)) break;
-        if (!mbar_wait(bar(L::B_VF + su), (t / NS) & 1, abort_flag)) break;
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_PR + st), u & 1, abort_flag))) break;
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_VF + su), (t / NS) & 1, abort_flag))) break;
         tc_fence_after();
         const uint64_t vd0 = desc_sw128(sb + kTile * (2 + 2 * su), kSpan, 1024);
         const uint32_t pa = tbase + (uint32_t)st * TB;
@@ -289,15 +321,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         for (int k = 0; k < TB / kK; ++k) {
           // K step k: kK keys = kK rows of 128 bytes further into V; 8 TMEM columns of P
           const uint64_t b = desc_adv(vd0, k * kK * 128);
-          if (F8) mma_ts_f8(od, pa + k * 8, b, idO, (u > 0 || k > 0));
-          else mma_ts(od, pa + k * 8, b, idO, (u > 0 || k > 0));
+          if (F8) mma_ts_f8_w(od, pa + k * 8, b, idO, (u > 0 || k > 0));
+          else mma_ts_w(od, pa + k * 8, b, idO, (u > 0 || k > 0));
         }
-        mma_commit(bar(L::B_KE + su));
-        mma_commit(bar(L::B_OD + st));
+        mma_commit_w(bar(L::B_KE + su));
+        mma_commit_w(bar(L::B_OD + st));
         if (t + 2 < T && !issue_s(t + 2)) break;
       }
       // every MMA issued above has completed before TMEM is released
-      mma_commit(bar(L::B_FIN));
+      mma_commit_w(bar(L::B_FIN));
       wait_bounded(bar(L::B_FIN), 0);
     }
   } else if (warp >= 8) {
