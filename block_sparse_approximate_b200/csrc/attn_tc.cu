@@ -694,64 +694,64 @@ attn_tc_linmix_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     regs_dec<kProducerRegs>();
-    if (lane == 0) {
+    {   // the whole warp runs the loop; elect.sync picks the issuing lane
       constexpr uint32_t idS = idesc_bf16_f32(TB, TB, 0, 0);
       constexpr uint32_t idO = idesc_bf16_f32(TB, TD, 0, 1);
       constexpr uint32_t idA = idesc_bf16_f32(TD, TD, 1, 1);   // relu(K)ᵀ (MN-major) · V (MN-major)
       const uint32_t colO = tbase + 256, colA = tbase + kColA;
+      const uint64_t qd0 = desc_sw128(sb, 16, 1024);
       auto issue_s = [&](int t) -> bool {
         const int s = t % NS;
-        if (!mbar_wait(bar(L::B_KF + s), (t / NS) & 1, abort_flag)) return false;
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_KF + s), (t / NS) & 1, abort_flag))) return false;
         tc_fence_after();
-        const uint32_t ka = sb + kTile * (1 + 2 * s);
+        const uint64_t kd0 = desc_sw128(sb + kTile * (1 + 2 * s), 16, 1024);
         const uint32_t d = tbase + (uint32_t)(t & 1) * TB;
 #pragma unroll
         for (int k = 0; k < TD / 16; ++k) {
           const uint32_t koff = (k >> 2) * kSpan + (k & 3) * 32;
-          mma_ss(d, desc_sw128(sb + koff, 16, 1024), desc_sw128(ka + koff, 16, 1024), idS, k > 0);
+          mma_ss_w(d, desc_adv(qd0, koff), desc_adv(kd0, koff), idS, k > 0);
         }
-        mma_commit(bar(L::B_SF + (t & 1)));
+        mma_commit_w(bar(L::B_SF + (t & 1)));
         return true;
       };
-      bool ok = mbar_wait(bar(L::B_Q), 0, abort_flag);
+      bool ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_Q), 0, abort_flag));
       if (ok && T > 0) ok = issue_s(0);
       if (ok && T > 1) ok = issue_s(1);
       for (int t = 0; ok && t < T; ++t) {
         const int su = t % NS, b2 = t & 1;
-        const uint32_t ka = sb + kTile * (1 + 2 * su), va = ka + kTile;
+        const uint64_t kd0 = desc_sw128(sb + kTile * (1 + 2 * su), kSpan, 1024);
+        const uint64_t vd0 = desc_sw128(sb + kTile * (2 + 2 * su), kSpan, 1024);
         // A_i += relu(K_t)ᵀ V_t once warps 4-7 have applied the ReLU
-        if (!mbar_wait(bar(L::B_RL + b2), (t >> 1) & 1, abort_flag)) break;
-        if (!mbar_wait(bar(L::B_VF + su), (t / NS) & 1, abort_flag)) break;
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_RL + b2), (t >> 1) & 1, abort_flag))) break;
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_VF + su), (t / NS) & 1, abort_flag))) break;
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < TB / 16; ++k)
-          mma_ss(colA, desc_sw128(ka + k * 16 * 128, kSpan, 1024), desc_sw128(va + k * 16 * 128, kSpan, 1024),
-                 idA, (t > 0 || k > 0));
+          mma_ss_w(colA, desc_adv(kd0, k * 16 * 128), desc_adv(vd0, k * 16 * 128), idA, (t > 0 || k > 0));
         // O += P_t V_t
-        if (!mbar_wait(bar(L::B_PR + b2), (t >> 1) & 1, abort_flag)) break;
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_PR + b2), (t >> 1) & 1, abort_flag))) break;
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < TB / 16; ++k)
-          mma_ts(colO, tbase + (uint32_t)b2 * TB + k * 8, desc_sw128(va + k * 16 * 128, kSpan, 1024), idO,
-                 (t > 0 || k > 0));
-        mma_commit(bar(L::B_KE + su));
-        mma_commit(bar(L::B_OD));
+          mma_ts_w(colO, tbase + (uint32_t)b2 * TB + k * 8, desc_adv(vd0, k * 16 * 128), idO, (t > 0 || k > 0));
+        mma_commit_w(bar(L::B_KE + su));
+        mma_commit_w(bar(L::B_OD));
         if (t + 2 < T && !issue_s(t + 2)) break;
       }
-      mma_commit(bar(L::B_LAST));   // every MMA of the tile loop (or none) has completed
+      mma_commit_w(bar(L::B_LAST));   // every MMA of the tile loop (or none) has completed
       // epilogue: S0 = relu(Q) · (H_tot − A_i), operands prepared by warps 0-7
-      if (ok && mbar_wait(bar(L::B_EPI_IN), 0, abort_flag)) {
+      if (__all_sync(0xffffffffu, ok && mbar_wait(bar(L::B_EPI_IN), 0, abort_flag))) {
         tc_fence_after();
         const uint32_t dbase = sb + kTile;   // D tile in stage 0's K slot
 #pragma unroll
         for (int k = 0; k < TD / 16; ++k) {
           const uint32_t koff = (k >> 2) * kSpan + (k & 3) * 32;
-          mma_ss(tbase, desc_sw128(sb + koff, 16, 1024), desc_sw128(dbase + k * 16 * 128, kSpan, 1024),
-                 idO, k > 0);
+          mma_ss_w(tbase, desc_sw128(sb + koff, 16, 1024), desc_sw128(dbase + k * 16 * 128, kSpan, 1024),
+                   idO, k > 0);
         }
-        mma_commit(bar(L::B_EPI));
+        mma_commit_w(bar(L::B_EPI));
       }
-      mma_commit(bar(L::B_FIN));
+      mma_commit_w(bar(L::B_FIN));
       wait_bounded(bar(L::B_FIN), 0);
     }
   } else if (warp >= 8) {
