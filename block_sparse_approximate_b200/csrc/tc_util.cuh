@@ -192,6 +192,37 @@ __device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, 
       : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
 }
 
+// 2^x for two fp32 lanes on the FMA pipe instead of the MUFU unit (a share
+// of the softmax exponentials moves here so that the two pipes split the
+// work).  x = n + f with n = floor(x): adding 1.5·2^23 with rounding toward
+// -inf leaves n in the low mantissa bits; 2^f on [0, 1) is a degree-3
+// polynomial fitted here for minimax relative error (Lawson's iteratively
+// reweighted least squares; maximum relative error 7.5e-5, below the 2^-9
+// rounding of the bf16 P it feeds; the CPU tests check this bound from the
+// constants below); 2^n is added to the exponent field.  x is clamped at
+// -126 so the exponent never wraps: inputs below it give a value under
+// 2^-125 instead of 0.
+__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& y0, float& y1) {
+  constexpr float kC0 = 0.99992520f, kC1 = 0.69583370f, kC2 = 0.22606723f, kC3 = 0.07802423f;
+  constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23
+  x0 = fmaxf(x0, -126.0f);
+  x1 = fmaxf(x1, -126.0f);
+  float t0, t1, f0, f1, q0, q1;
+  asm("{\n\t.reg .b64 rx, rm, rt, rn, rf;\n\t"
+      "mov.b64 rx, {%4, %5};\n\tmov.b64 rm, {%6, %6};\n\t"
+      "add.rm.f32x2 rt, rx, rm;\n\t"
+      "sub.rn.f32x2 rn, rt, rm;\n\t"
+      "sub.rn.f32x2 rf, rx, rn;\n\t"
+      "mov.b64 {%0, %1}, rt;\n\tmov.b64 {%2, %3}, rf;\n\t}"
+      : "=f"(t0), "=f"(t1), "=f"(f0), "=f"(f1)
+      : "f"(x0), "f"(x1), "f"(kMagic));
+  ffma2(q0, q1, f0, f1, kC3, kC3, kC2, kC2);
+  ffma2(q0, q1, q0, q1, f0, f1, kC1, kC1);
+  ffma2(q0, q1, q0, q1, f0, f1, kC0, kC0);
+  y0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
+  y1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
+}
+
 // (d0, d1) += (a0, a1) on two fp32 lanes at once
 __device__ __forceinline__ void fadd2(float& d0, float& d1, float a0, float a1) {
   asm("{\n\t.reg .b64 ra, rd;\n\t"
