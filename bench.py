@@ -138,13 +138,28 @@ def _dist():
     return world, rank, local
 
 
-def _max_over_ranks(x: float, world: int) -> float:
+def _max_over_ranks(x: float, world: int, device: str = "cuda") -> float:
+    """The largest of the ranks' x (a device time): every rank calls it in the
+    same order.  ``device`` is where the one-element reduction tensor lives
+    (cuda for NCCL, cpu for gloo)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], device="cuda", dtype=torch.float64)
+    t = torch.tensor([x], device=device, dtype=torch.float64)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_workload(w, rank: int):
+    """Rank r's problem: the same shapes, seed + 1000 r (independent problems,
+    no exchange between ranks)."""
+    return wl.Workload(**{**w.__dict__, "seed": w.seed + 1000 * rank}) if rank else w
+
+
+def job_value(w, world: int, ms_step: float) -> float:
+    """Whole-job dense-equivalent TFLOPS: every rank ran one step of w in at
+    most ms_step (the max over ranks)."""
+    return world * dense_flops(w) / (ms_step * 1e-3) / 1e12
 
 
 def _barrier(world):
@@ -360,7 +375,7 @@ def run_ours(args, world, rank, local):
             print(json.dumps({"sla2_mix": time_sla2(args.steps, args.warmup)}), flush=True)
         return 0
     w = wl.WORKLOADS[WORKLOAD]
-    wr = wl.Workload(**{**w.__dict__, "seed": w.seed + 1000 * rank}) if rank else w
+    wr = rank_workload(w, rank)
     inp = wl.prefill_inputs(wr, "cuda")
     step = PrefillStep(wr, inp)
     clocks = ClockSampler(local) if rank == 0 else None
@@ -442,7 +457,7 @@ def run_ours(args, world, rank, local):
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = _max_over_ranks(e0.elapsed_time(e1) / n_e2e, world)
-        e2e = {"value": world * dense_flops(w) / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS",
+        e2e = {"value": job_value(w, world, e2e_ms), "unit": "TFLOPS",
                "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": sum(inp[n].numel() * inp[n].element_size() for n in ("Q", "K", "V")),
                "d2h_bytes_per_step": step.buf.out.numel() * step.buf.out.element_size()}
@@ -466,7 +481,7 @@ def run_ours(args, world, rank, local):
         inp_cpu = {n: inp[n].cpu() for n in ("Q", "K", "V")}
         cpu = cpu_baseline(w, inp_cpu)
     line = {
-        "metric": METRIC, "value": world * dense_flops(w) / (ms_step * 1e-3) / 1e12, "unit": "TFLOPS",
+        "metric": METRIC, "value": job_value(w, world, ms_step), "unit": "TFLOPS",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
