@@ -65,6 +65,48 @@ DecodeLayout decode_layout(const sa_decode_shape& s, int topk) {
   return L;
 }
 
+// Device-side error word of the decode kernels: set when a bounded wait gives
+// up; sa_device_error() reads and clears it with the attention kernels' word.
+static __device__ unsigned int g_decode_error = 0;
+constexpr long long kDecWaitCycles = 4000000000ll;   // ~2 s: far above any real wait
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void dbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void dbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+// Waits for the phase of parity `parity`; false after kDecWaitCycles (the
+// error word is set).
+__device__ __forceinline__ bool dbar_wait(uint32_t bar, uint32_t parity) {
+  const long long t0 = clock64();
+  for (;;) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    if (done) return true;
+    if (clock64() - t0 > kDecWaitCycles) {
+      atomicOr(&g_decode_error, 1u);
+      return false;
+    }
+  }
+}
+// One contiguous global -> shared copy of `bytes` (16-byte aligned, a
+// multiple of 16) completing on `bar`.
+__device__ __forceinline__ void bulk_copy(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(dst), "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
 __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(smem_dst)),
                "l"(gsrc)
@@ -103,9 +145,9 @@ __device__ __forceinline__ void head_store(const HeadState& S, float* out, int l
 }
 
 // ---- A. statistics pass --------------------------------------------------
-// Two CTAs of 4 warps per SM.  A stage (32 blocks of kmean, kvar and vsum
-// rows, 48 KB for d = 128) lands in shared memory by cp.async; warp w takes
-// blocks [8w, 8w + 8) of it.  Lane = a group of d/32 channels: it holds
+// Two CTAs of 8 warps per SM.  A stage (32 blocks of kmean, kvar and vsum
+// rows, 48 KB for d = 128) lands in shared memory by three bulk copies
+// issued by one thread; warp w takes blocks [4w, 4w + 4) of it.  Lane = a group of d/32 channels: it holds
 // s log2e q and ½ s² q² of the group's channels for all G heads in
 // registers and reads each stats row as one contiguous 512-byte row, so a
 // row costs four shared-memory wavefronts and is read by one warp only.
@@ -115,7 +157,7 @@ __device__ __forceinline__ void head_store(const HeadState& S, float* out, int l
 // terms of the batch then enter the warp's online state of each head
 // (max, sum, numerator channels of the lane); the four warps' states are
 // merged once per segment.
-constexpr int kThrA = 128;
+constexpr int kThrA = 256;
 
 // channels [lane CPL, lane CPL + CPL) of a shared-memory row, or zeros
 template <int CPL>
@@ -148,7 +190,8 @@ decode_stats_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int 
   constexpr int kWarps = kThrA / 32;
   extern __shared__ __align__(16) uint8_t dsm[];
   float* mg = reinterpret_cast<float*>(dsm);                 // [warps][G][D + 2] segment merge
-  uint8_t* ring = dsm + sizeof(float) * kWarps * G * (D + 2);
+  uint64_t* full = reinterpret_cast<uint64_t*>(dsm + sizeof(float) * kWarps * G * (D + 2));   // [kRingA]
+  uint8_t* ring = reinterpret_cast<uint8_t*>(full + 2 * kRingA);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nstage_pair = (nb + kStageBlocksA - 1) / kStageBlocksA;
   const int total_segs = npairs * nsegA;
@@ -159,26 +202,32 @@ decode_stats_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int 
   // the CTA's stage sequence: its segments in order, each segment's stages
   auto seg_of = [&](int k_seg) { return (int)blockIdx.x + k_seg * (int)gridDim.x; };
   auto stages_in = [&](int seg) { return min(kSegA, nstage_pair - (seg % nsegA) * kSegA); };
-  // issue the copies of stage `sub` of segment `seg` into ring slot `slot`
+  // thread 0 copies stage `sub` of segment `seg` into ring slot `slot`: the
+  // stage's rows of each array are contiguous, one bulk copy per array
   auto issue = [&](int seg, int sub, int slot) {
     const int pair = seg / nsegA, sseg = seg % nsegA;
     const int j0 = (sseg * kSegA + sub) * kStageBlocksA;
-    const int n16 = min(kStageBlocksA, nb - j0) * (int)(kRowB / 16);
+    const uint32_t bytes = (uint32_t)min(kStageBlocksA, nb - j0) * kRowB;
     const size_t goff = ((size_t)pair * nb + j0) * D;
-    uint8_t* dst = ring + slot * kStageB;
-    const uint8_t* src0 = reinterpret_cast<const uint8_t*>(st.kmean + goff);
-    const uint8_t* src1 = reinterpret_cast<const uint8_t*>(st.kvar + goff);
-    const uint8_t* src2 = reinterpret_cast<const uint8_t*>(st.vsum + goff);
-    for (int o = tid; o < n16; o += kThrA) {
-      cp_async16(dst + o * 16, src0 + o * 16);
-      cp_async16(dst + kArrB + o * 16, src1 + o * 16);
-      cp_async16(dst + 2 * kArrB + o * 16, src2 + o * 16);
-    }
+    const uint32_t dst = smem_addr(ring + slot * kStageB), fb = smem_addr(full + slot);
+    // the slot's previous contents were read by generic loads before the
+    // barrier that precedes this call; order them before the async writes
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    dbar_expect_tx(fb, 3 * bytes);
+    bulk_copy(dst, st.kmean + goff, bytes, fb);
+    bulk_copy(dst + kArrB, st.kvar + goff, bytes, fb);
+    bulk_copy(dst + 2 * kArrB, st.vsum + goff, bytes, fb);
   };
 
   if (seg_of(0) >= total_segs) return;
+  if (tid == 0) {
+    for (int r = 0; r < kRingA; ++r) dbar_init(smem_addr(full + r), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
   int cur_seg_k = 0, cur_sub = 0;
   int pf_seg_k = 0, pf_sub = 0, pf_slot = 0;
+  int issued = 0, consumed = 0;   // stages copied / used (ring phases)
   auto pf_valid = [&]() { return seg_of(pf_seg_k) < total_segs; };
   auto pf_advance = [&]() {
     if (++pf_sub >= stages_in(seg_of(pf_seg_k))) {
@@ -188,10 +237,10 @@ decode_stats_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int 
   };
   for (int r = 0; r < kRingA - 1; ++r) {
     if (pf_valid()) {
-      issue(seg_of(pf_seg_k), pf_sub, pf_slot);
+      if (tid == 0) issue(seg_of(pf_seg_k), pf_sub, pf_slot);
+      ++issued;
       pf_advance();
     }
-    cp_async_commit();
     pf_slot = (pf_slot + 1) % kRingA;
   }
 
@@ -223,15 +272,17 @@ decode_stats_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int 
         for (int c = 0; c < CPL; ++c) acc[h][c] = 0.f;
       }
     }
-    // prefetch one more stage, then wait for the current one
+    // prefetch one more stage (its slot was released by the previous
+    // stage's closing barrier), then wait for the current one
     if (pf_valid()) {
-      issue(seg_of(pf_seg_k), pf_sub, pf_slot);
+      if (tid == 0) issue(seg_of(pf_seg_k), pf_sub, pf_slot);
+      ++issued;
       pf_advance();
     }
-    cp_async_commit();
     pf_slot = (pf_slot + 1) % kRingA;
-    cp_async_wait<kRingA - 1>();
-    __syncthreads();
+    const bool landed = dbar_wait(smem_addr(full + slot), (consumed / kRingA) & 1);
+    ++consumed;
+    if (!__syncthreads_and(landed)) break;
 
     const uint8_t* stg = ring + slot * kStageB;
     const float* km = reinterpret_cast<const float*>(stg);
@@ -375,7 +426,9 @@ decode_stats_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int 
       ++cur_seg_k;
     }
   }
-  cp_async_wait<0>();
+  // after a give-up, let the copies still in flight land before exiting
+  if (tid == 0)
+    for (int q = consumed; q < issued; ++q) dbar_wait(smem_addr(full + q % kRingA), (q / kRingA) & 1);
 }
 
 // ---- B. top-k ------------------------------------------------------------
@@ -887,7 +940,8 @@ sa_status launch_decode(const void* q, const void* Kc, const void* Vc, const sa_
   // A
   {
     const int g = s.Hq / s.Hkv;
-    const size_t smemA = sizeof(float) * 4 * g * (D + 2) + (size_t)kRingA * 3 * kStageBlocksA * D * 4;
+    const size_t smemA = sizeof(float) * (kThrA / 32) * g * (D + 2) + 16 * kRingA +
+                         (size_t)kRingA * 3 * kStageBlocksA * D * 4;
     const long segsA = (long)npairs * L.nsegA;
     const int gridA = (int)(segsA < 2 * sms ? segsA : 2 * sms);
     sa_status r0 = SA_OK;
