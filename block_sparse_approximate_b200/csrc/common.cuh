@@ -36,6 +36,9 @@ inline size_t dtype_size(sa_dtype t) { return t == SA_FP32 ? 4 : 2; }
 // Host-side validation of a prefill shape; returns SA_OK or sets the error.
 sa_status check_shape(const sa_shape& s, const char* fn);
 
+// Reads and clears the decode kernels' device error word (decode.cu).
+uint32_t decode_error_take();
+
 // ---------------------------------------------------------------- device side
 
 template <typename T>

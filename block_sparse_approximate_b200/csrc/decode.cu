@@ -1020,6 +1020,16 @@ sa_status check_decode_shape(const sa_decode_shape& s, int topk) {
 }  // namespace
 }  // namespace sa
 
+namespace sa {
+uint32_t decode_error_take() {
+  unsigned int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_decode_error, sizeof(v)) != cudaSuccess ||
+      cudaMemcpyToSymbol(g_decode_error, &zero, sizeof(zero)) != cudaSuccess)
+    return 0u;
+  return v;
+}
+}  // namespace sa
+
 extern "C" size_t sa_decode_workspace_size(sa_decode_shape shape, int32_t topk) {
   using namespace sa;
   if (check_decode_shape(shape, topk) != SA_OK) return 0;
