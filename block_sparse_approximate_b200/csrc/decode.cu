@@ -118,6 +118,11 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start while its predecessor drains; it waits here
+// before touching anything the predecessor writes (a no-op otherwise).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ uint32_t pack2bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
@@ -441,6 +446,7 @@ constexpr int kTopkKPT = kMaxRouteBlocks / kDecThreads;   // keys per thread
 
 __global__ void __launch_bounds__(kDecThreads)
 decode_topk_kernel(const float* __restrict__ scores, int nb, int topk, int32_t* __restrict__ idx) {
+  pdl_wait();
   const int pair = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   __shared__ unsigned hist[256];
@@ -606,6 +612,7 @@ decode_exact_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
                     const __nv_bfloat16* __restrict__ Vc, int Hq, int Hkv, int N, int blk,
                     const int32_t* __restrict__ idx, int topk, float scale, int nsegC, int npairs,
                     float* __restrict__ partc) {
+  pdl_wait();
   constexpr int CH = D / 8;                         // 16-byte chunks per bf16 row
   constexpr int NT = D / 8;                         // n-tiles of 8 channels
   constexpr int KS = D / 16;                        // k steps of 16 channels
@@ -824,6 +831,7 @@ decode_combine_kernel(const float* __restrict__ parta, int nsegA, const float* _
                       int use_tail, const __nv_bfloat16* __restrict__ q, sa_block_stats st,
                       const int32_t* __restrict__ idx, int topk, int nb, int blk, float scale, int Hq, int Hkv,
                       __nv_bfloat16* __restrict__ O) {
+  pdl_wait();
   constexpr int kT = kParts * D, kW = kT / 32;
   extern __shared__ __align__(16) float csm[];
   const int na = use_tail ? nsegA : 0, ns = na + nsegC;
@@ -911,6 +919,26 @@ decode_combine_kernel(const float* __restrict__ parta, int nsegA, const float* _
   }
 }
 
+// Launch with programmatic stream serialization (the kernel calls pdl_wait()
+// before reading what the previous launch on the stream wrote).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+  if (e != cudaSuccess) cudaGetLastError();   // reported by the caller's status, not left pending
+  return e;
+}
+
 int sm_count() {
   static int n = 0;
   if (n == 0) {
@@ -963,7 +991,10 @@ sa_status launch_decode(const void* q, const void* Kc, const void* Vc, const sa_
 
   // B
   if (topk > 0) {
-    decode_topk_kernel<<<npairs, kDecThreads, 0, stream>>>(scores, nb, topk, idx);
+    {
+      const cudaError_t le = launch_pdl(decode_topk_kernel, dim3(npairs), dim3(kDecThreads), 0, stream, scores, nb, topk, idx);
+      if (le != cudaSuccess) return fail(SA_ERR_CUDA, std::string("decode_topk_kernel: ") + cudaGetErrorString(le));
+    }
     r = launch_status("decode_topk_kernel");
     if (r != SA_OK) return r;
   }
@@ -978,9 +1009,12 @@ sa_status launch_decode(const void* q, const void* Kc, const void* Vc, const sa_
       return launch_status("cudaFuncSetAttribute(decode_exact_kernel)");
     const long segsC = (long)npairs * L.nsegC;   // < 2^31 for any supported shape
     const int gridC = (int)(segsC < sms ? segsC : sms);
-    decode_exact_kernel<D><<<gridC, kDecThreads, smemC, stream>>>(
+    {
+      const cudaError_t le = launch_pdl(decode_exact_kernel<D>, dim3(gridC), dim3(kDecThreads), smemC, stream,
         qb, static_cast<const __nv_bfloat16*>(Kc), static_cast<const __nv_bfloat16*>(Vc), s.Hq, s.Hkv, s.N,
         s.block, idx, topk, scale, L.nsegC, npairs, partc);
+      if (le != cudaSuccess) return fail(SA_ERR_CUDA, std::string("decode_exact_kernel: ") + cudaGetErrorString(le));
+    }
     r = launch_status("decode_exact_kernel");
     if (r != SA_OK) return r;
   }
@@ -995,9 +1029,12 @@ sa_status launch_decode(const void* q, const void* Kc, const void* Vc, const sa_
     if (cudaFuncSetAttribute(decode_combine_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smemD) !=
         cudaSuccess)
       return launch_status("cudaFuncSetAttribute(decode_combine_kernel)");
-    decode_combine_kernel<D><<<dim3(s.Hq, s.B), kParts * D, smemD, stream>>>(
+    {
+      const cudaError_t le = launch_pdl(decode_combine_kernel<D>, dim3(s.Hq, s.B), dim3(kParts * D), smemD, stream,
         parta, L.nsegA, partc, nsc, use_tail, qb, st, idx, topk, nb, s.block, scale, s.Hq, s.Hkv,
         static_cast<__nv_bfloat16*>(O));
+      if (le != cudaSuccess) return fail(SA_ERR_CUDA, std::string("decode_combine_kernel: ") + cudaGetErrorString(le));
+    }
   }
   return launch_status("decode_combine_kernel");
 }
