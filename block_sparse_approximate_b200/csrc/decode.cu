@@ -857,6 +857,21 @@ decode_combine_kernel(const float* __restrict__ parta, int nsegA, const float* _
   }
   for (int x = tid; x < nsel; x += kT) jsel[x] = __ldg(idx + (size_t)pair * topk + x);
   __syncthreads();
+  // this thread's partial-state channels and selected-block vsum channels,
+  // loaded now (they do not depend on the maximum) so their latency overlaps
+  // the dot products below
+  constexpr int kPreP = 8, kPreV = 16;
+  float pv[kPreP], vv[kPreV];
+#pragma unroll
+  for (int e = 0; e < kPreP; ++e) {
+    const int x = pt + kParts * e;
+    pv[e] = x < ns ? part(x)[2 + c] : 0.f;
+  }
+#pragma unroll
+  for (int e = 0; e < kPreV; ++e) {
+    const int si = pt + kParts * e;
+    vv[e] = si < nsel ? __ldg(st.vsum + ((size_t)pair * nb + jsel[si]) * D + c) : 0.f;
+  }
   float M = -INFINITY;
   for (int x = 0; x < ns; ++x) M = fmaxf(M, hm[x]);
   if (subtract && M != -INFINITY) {
@@ -889,16 +904,30 @@ decode_combine_kernel(const float* __restrict__ parta, int nsegA, const float* _
   __syncthreads();
   float L = 0.f, A = 0.f;
   if (M != -INFINITY) {
-#pragma unroll 4
-    for (int x = pt; x < ns; x += kParts) {
-      const float f = hf[x];
-      L = fmaf(hl[x], f, L);
-      A = fmaf(part(x)[2 + c], f, A);
+#pragma unroll
+    for (int e = 0; e < kPreP; ++e) {
+      const int x = pt + kParts * e;
+      if (x < ns) {
+        L = fmaf(hl[x], hf[x], L);
+        A = fmaf(pv[e], hf[x], A);
+      }
+    }
+    for (int x = pt + kParts * kPreP; x < ns; x += kParts) {
+      L = fmaf(hl[x], hf[x], L);
+      A = fmaf(part(x)[2 + c], hf[x], A);
     }
     // subtract the zero-order term of each selected block (weight <= 1)
     const float inv_blk = 1.0f / blk;
-#pragma unroll 8
-    for (int si = pt; si < nsel; si += kParts) {
+#pragma unroll
+    for (int e = 0; e < kPreV; ++e) {
+      const int si = pt + kParts * e;
+      if (si < nsel) {
+        const float w = fast_exp2(xsel[si] - M);
+        L -= w;
+        A = fmaf(-w * inv_blk, vv[e], A);
+      }
+    }
+    for (int si = pt + kParts * kPreV; si < nsel; si += kParts) {
       const float w = fast_exp2(xsel[si] - M);
       L -= w;
       A = fmaf(-w * inv_blk, __ldg(st.vsum + ((size_t)pair * nb + jsel[si]) * D + c), A);
