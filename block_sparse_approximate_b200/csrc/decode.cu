@@ -36,10 +36,11 @@ constexpr int kMaxGroup = 8;
 constexpr int kStageBlocksA = 32;
 constexpr int kSegA = 4;
 constexpr int kRingA = 2;
-// C: a stage is 64 tokens of K and V; a segment is kSegC stages
-constexpr int kStageTokC = 64;
-constexpr int kSegC = 8;
-constexpr int kRingC = 4;
+// C: a stage is 128 selected tokens of K and V (two 64-token halves, each
+// inside one selected block); a segment is kSegC stages
+constexpr int kStageTokC = 128;
+constexpr int kSegC = 4;
+constexpr int kRingC = 3;
 // segments per CTA whose block indices are staged in shared memory (later
 // segments read theirs from global memory)
 constexpr int kItabSegs = 64;
@@ -107,9 +108,10 @@ __device__ __forceinline__ void bulk_copy(uint32_t dst, const void* src, uint32_
                : "memory");
 }
 
-__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(smem_dst)),
-               "l"(gsrc)
+// 16-byte cp.async reading `src_bytes` (16 or 0) and zero-filling the rest
+__device__ __forceinline__ void cp_async16z(void* smem_dst, const void* gsrc, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"((uint32_t)__cvta_generic_to_shared(smem_dst)),
+               "l"(gsrc), "r"(src_bytes)
                : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
@@ -570,24 +572,17 @@ decode_topk_kernel(const float* __restrict__ scores, int nb, int topk, int32_t* 
 }
 
 // ---- C. exact pass over the selected blocks --------------------------------
-// A stage is 64 consecutive tokens of one selected block (K and V rows staged
-// by cp.async with the 16-byte chunks of row r stored at chunk ^ (r & 7), so
-// ldmatrix reads are free of bank conflicts).  Warp w takes tokens
-// [8w, 8w + 8) of each stage and runs the small contractions on mma.sync
+// A stage is 128 selected tokens, two 64-token halves of selected blocks (K
+// and V rows staged by cp.async with the 16-byte chunks of row r stored at
+// chunk ^ (r & 7), so ldmatrix reads are free of bank conflicts).  Warp w
+// takes tokens [16w, 16w + 16) of each stage and runs the small contractions
+// on mma.sync
 // (m16n8k16, bf16 in, fp32 accumulate): S = Q Kᵀ with the group's g <= 8
 // query heads as the MMA rows, then O += P V.  Each warp keeps an online
 // softmax state per head; at the end of a segment the eight warps' states are
 // merged and one partial state per head is written.  The selected block
 // indices of all the CTA's segments are staged in shared memory once, so the
 // copy issue of a stage does not wait on a global load.
-__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a2, uint32_t b0) {
-  // rows 8-15 of A and k 8-15 of B are zero (a1 = a3 = b1 = 0)
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(0u));
-}
 __device__ __forceinline__ void mma16816_full(float (&d)[4], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
   asm volatile(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
@@ -628,7 +623,7 @@ decode_exact_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
   const int g = Hq / Hkv;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int tok_pair = topk * blk;                  // exact tokens of one (sequence, KV head)
-  const int nstage_pair = tok_pair / kStageTokC;    // blk is a multiple of 64
+  const int nstage_pair = (tok_pair + kStageTokC - 1) / kStageTokC;   // the last may hold 64
   const int total_segs = npairs * nsegC;
   const float scale2 = scale * kLog2e;
   const int hrow = lane >> 2;                       // MMA row of this thread = query head
@@ -642,19 +637,30 @@ decode_exact_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
     const int si = sseg * kSegC * kStageTokC / blk + sl;
     return k < kItabSegs ? itab[k * kSegBlocksMax + sl] : __ldg(idx + (size_t)pair * topk + si);
   };
+  // stage `sub` of segment `seg` into ring slot `slot`: two 64-token halves,
+  // each inside one selected block; a half past the pair's last selected
+  // token is zero-filled (it only occurs as the second half of a last stage)
   auto issue = [&](int k, int seg, int sub, int slot) {
-    const int pair = seg / nsegC;
-    const int tin = sub * kStageTokC;   // token offset inside the segment
-    const int tok0 = block_of(k, seg, tin / blk) * blk + (tin % blk);
-    const size_t off = ((size_t)pair * N + tok0) * D;
-    const uint8_t* ksrc = reinterpret_cast<const uint8_t*>(Kc + off);
-    const uint8_t* vsrc = reinterpret_cast<const uint8_t*>(Vc + off);
+    const int pair = seg / nsegC, sseg = seg % nsegC;
+    const int t0 = (sseg * kSegC + sub) * kStageTokC;
+    const int ntok = min(kStageTokC, tok_pair - t0);
+    const __nv_bfloat16* ks[2];
+    const __nv_bfloat16* vsrc[2];
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int tin = sub * kStageTokC + 64 * (hh < 1 || 64 < ntok ? hh : 0);   // token offset in the segment
+      const size_t off = ((size_t)pair * N + block_of(k, seg, tin / blk) * blk + (tin % blk)) * D;
+      ks[hh] = Kc + off;
+      vsrc[hh] = Vc + off;
+    }
     uint8_t* dst = ring + slot * kStageB;
     for (int o = tid; o < kStageTokC * CH; o += kDecThreads) {
-      const int r = o / CH, c = o % CH;
+      const int r = o / CH, c = o % CH, hh = r >> 6;
       const uint32_t sw = r * kRowB + ((c ^ (r & 7)) << 4);
-      cp_async16(dst + sw, ksrc + o * 16);
-      cp_async16(dst + kArrB + sw, vsrc + o * 16);
+      const size_t so = (size_t)(r & 63) * D + 8 * c;
+      const uint32_t nbytes = r < ntok ? 16u : 0u;   // 0: zero-fill
+      cp_async16z(dst + sw, ks[hh] + so, nbytes);
+      cp_async16z(dst + kArrB + sw, vsrc[hh] + so, nbytes);
     }
   };
   if (seg_of(0) >= total_segs) return;
@@ -718,41 +724,54 @@ decode_exact_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
     __syncthreads();
 
     const uint32_t kbase = ring_s + slot * kStageB, vbase = kbase + kArrB;
-    const int tokr = 8 * warp + (lane & 7);     // the row this lane addresses for ldmatrix
-    // S = Q Kᵀ for tokens [8 warp, 8 warp + 8)
-    float sacc[4] = {0.f, 0.f, 0.f, 0.f};
+    const int ntok = min(kStageTokC, tok_pair - (sseg * kSegC + cur_sub) * kStageTokC);
+    const int tb = 16 * warp;                   // this warp's tokens [tb, tb + 16) of the stage
+    const int tok0 = tb + (lane & 7), tok1 = tb + 8 + (lane & 7);   // rows this lane addresses
+    // S = Q Kᵀ for the warp's two 8-token n-tiles
+    float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int kp = 0; kp < KS / 2; ++kp) {
-      uint32_t kf[4];
+      uint32_t kf[4], kg[4];
       const int chunk = 4 * kp + (lane >> 3);
-      ldsm_x4(kf, kbase + tokr * kRowB + ((chunk ^ (tokr & 7)) << 4));
-      mma16816_full(sacc, qa0[2 * kp], qa2[2 * kp], kf[0], kf[1]);
-      mma16816_full(sacc, qa0[2 * kp + 1], qa2[2 * kp + 1], kf[2], kf[3]);
+      ldsm_x4(kf, kbase + tok0 * kRowB + ((chunk ^ (tok0 & 7)) << 4));
+      ldsm_x4(kg, kbase + tok1 * kRowB + ((chunk ^ (tok1 & 7)) << 4));
+      mma16816_full(s0, qa0[2 * kp], qa2[2 * kp], kf[0], kf[1]);
+      mma16816_full(s0, qa0[2 * kp + 1], qa2[2 * kp + 1], kf[2], kf[3]);
+      mma16816_full(s1, qa0[2 * kp], qa2[2 * kp], kg[0], kg[1]);
+      mma16816_full(s1, qa0[2 * kp + 1], qa2[2 * kp + 1], kg[2], kg[3]);
     }
-    // online softmax of this warp's 8 tokens for head hrow
-    const float x0 = sacc[0] * scale2, x1 = sacc[1] * scale2;
-    float tmax = fmaxf(x0, x1);
+    // online softmax of the warp's 16 tokens for head hrow (tokens past the
+    // stage's valid count are zero-filled rows: masked out)
+    const int tj = tb + 2 * (lane & 3);
+    const float x0 = tj < ntok ? s0[0] * scale2 : -INFINITY, x1 = tj + 1 < ntok ? s0[1] * scale2 : -INFINITY;
+    const float x2 = tj + 8 < ntok ? s1[0] * scale2 : -INFINITY, x3 = tj + 9 < ntok ? s1[1] * scale2 : -INFINITY;
+    float tmax = fmaxf(fmaxf(x0, x1), fmaxf(x2, x3));
     tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 1));
     tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 2));
     const float m_new = fmaxf(m_run, tmax);
-    const float corr = fast_exp2(m_run - m_new);
-    const float p0 = hvalid ? fast_exp2(x0 - m_new) : 0.f;
-    const float p1 = hvalid ? fast_exp2(x1 - m_new) : 0.f;
-    l_run = l_run * corr + p0 + p1;
+    const float corr = m_run == -INFINITY ? 0.f : fast_exp2(m_run - m_new);
+    const bool on = hvalid && m_new != -INFINITY;
+    const float p0 = on && x0 != -INFINITY ? fast_exp2(x0 - m_new) : 0.f;
+    const float p1 = on && x1 != -INFINITY ? fast_exp2(x1 - m_new) : 0.f;
+    const float p2 = on && x2 != -INFINITY ? fast_exp2(x2 - m_new) : 0.f;
+    const float p3 = on && x3 != -INFINITY ? fast_exp2(x3 - m_new) : 0.f;
+    l_run = l_run * corr + ((p0 + p1) + (p2 + p3));
     m_run = m_new;
-    const uint32_t pa = pack2bf16(p0, p1);
-    // O += P V for the 8 tokens (k 8-15 of the MMA are zero)
+    // P as the A fragment: k 0-7 = the first n-tile's tokens, k 8-15 the second's
+    const uint32_t pa0 = pack2bf16(p0, p1), pa2 = pack2bf16(p2, p3);
+    // O += P V over the 16 tokens
 #pragma unroll
     for (int nq = 0; nq < NT / 4; ++nq) {
-      uint32_t vf[4];
+      uint32_t vf[4], vg[4];
       const int chunk = 4 * nq + (lane >> 3);
-      ldsm_x4_t(vf, vbase + tokr * kRowB + ((chunk ^ (tokr & 7)) << 4));
+      ldsm_x4_t(vf, vbase + tok0 * kRowB + ((chunk ^ (tok0 & 7)) << 4));
+      ldsm_x4_t(vg, vbase + tok1 * kRowB + ((chunk ^ (tok1 & 7)) << 4));
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         float* oo = o[4 * nq + e];
         oo[0] *= corr;
         oo[1] *= corr;
-        mma16816(o[4 * nq + e], pa, 0u, vf[e]);
+        mma16816_full(o[4 * nq + e], pa0, pa2, vf[e], vg[e]);
       }
     }
     __syncthreads();
