@@ -33,6 +33,10 @@ Pins (the tests under ``tests/test_oracle_*.py``):
   block_pool          closed forms on ramps / constant blocks; brute force
   route_scores        brute-force loops; taylor2 == dot order when var == 0
   topk_from_scores    brute-force sort on tiny inputs, hand-made ties
+  first_order tail    H̄ = 0 (block-constant keys) -> zero_order; identical
+                      per-block deviations -> PISA's per-block first-order
+                      Taylor sum by brute force; error O(ε²) vs zero_order's
+                      O(ε) as the in-block deviations shrink
   sparse_attention    k = nb -> dense softmax attention (torch SDPA, fp64);
                       block size 1 / block-constant keys -> dense; V+c -> O+c;
                       hand-derived worked example (tests/golden); brute force
@@ -64,7 +68,7 @@ def _f64(x) -> np.ndarray:
 # ---------------------------------------------------------------------------
 
 def block_pool(Q, K, V, block: int, *, variance: bool = False,
-               linear: bool = False) -> dict:
+               linear: bool = False, first_order: bool = False) -> dict:
     """Per-block statistics of Q, K and V, all float64.
 
     Follows PISA "Implementação de Hardware", step "Pré-computação"
@@ -83,6 +87,9 @@ def block_pool(Q, K, V, block: int, *, variance: bool = False,
       ztot  [B,H,d]      sum over all tokens of relu(k)  (only with ``linear``)
       htot  [B,H,d,d]    sum over all tokens of relu(k_n) v_n^T
                          (only with ``linear``)
+      hbar  [B,H,d,d]    PISA's global first-order statistic H̄: the mean over
+                         the head's blocks of H_j = Σ_{n∈j} (k_n − k̄_j) v_nᵀ
+                         (only with ``first_order``)
     """
     K = _f64(K)
     V = _f64(V)
@@ -110,6 +117,11 @@ def block_pool(Q, K, V, block: int, *, variance: bool = False,
         out["ztot"] = out["zrelu"].sum(axis=2)
         Rt = np.maximum(K, 0.0)
         out["htot"] = np.einsum("bhnc,bhne->bhce", Rt, V)
+    if first_order:
+        # H_j = Σ_n (k_n − k̄_j) v_nᵀ for every block, then their mean
+        dev = Kb - kmean[:, :, :, None, :]
+        Hj = np.einsum("bhjnc,bhjne->bhjce", dev, Vb)
+        out["hbar"] = Hj.mean(axis=2)
     return out
 
 
@@ -206,13 +218,17 @@ def _block_tokens(blocks: Sequence[int], block: int) -> np.ndarray:
 
 def _attend_rows(q, K, V, sel: Sequence[int], nb: int, block: int, tail: str,
                  scale: float, alpha_h=None, eps: float = EPS_LINEAR,
-                 centroids=None) -> np.ndarray:
+                 centroids=None, hbar=None) -> np.ndarray:
     """Output rows o_t for query rows q [R, d] against one head's K, V [N, d].
 
     PISA "Algoritmo Central":  o_t = N_t / D_t with
       N_t = Σ_{j∈S} Σ_n e^{s q_t.k_{j,n}} v_{j,n} + Σ_{j∈U} e^{s q_t.k̄_j} Σ_n v_{j,n}
       D_t = Σ_{j∈S} Σ_n e^{s q_t.k_{j,n}}         + Σ_{j∈U} B e^{s q_t.k̄_j}
-    (zero_order; the first-order correction of PISA is not part of this path).
+    (zero_order).  "first_order" is PISA's hybrid order: the zero_order terms
+    plus the global first-order correction of the numerator,
+      N_t += (s q_t) H̄ Σ_{j∈U} e^{s q_t.k̄_j},
+    with H̄ the mean over all blocks of H_j = Σ_{n∈j} (k_n − k̄_j) v_nᵀ (the
+    first-order term of the denominator is zero: the deviations sum to zero).
     "drop" keeps only the S terms (the keep-or-drop baseline PISA and SPLA
     contrast with).  "linear_mix" is SLA2 §2A O = α⊙O_s + (1−α)⊙O_l with O_s
     the drop output and O_l the ReLU linear attention (SALAD §2) over U:
@@ -224,7 +240,7 @@ def _attend_rows(q, K, V, sel: Sequence[int], nb: int, block: int, tail: str,
     Ks, Vs = K[tok], V[tok]
     R, d = q.shape
     a = scale * (q @ Ks.T)                      # exact logits [R, |S|B]
-    if tail == "zero_order":
+    if tail in ("zero_order", "first_order"):
         if centroids is None:
             kbar = K.reshape(nb, block, d).mean(axis=1)[uns]      # [|U|, d]
             vsum = V.reshape(nb, block, d).sum(axis=1)[uns]       # [|U|, d]
@@ -241,6 +257,12 @@ def _attend_rows(q, K, V, sel: Sequence[int], nb: int, block: int, tail: str,
         wc = np.exp(c - m[:, None])
         num = wa @ Vs + wc @ vsum
         den = wa.sum(axis=1) + block * wc.sum(axis=1)
+        if tail == "first_order":
+            if hbar is None:
+                Kb = K.reshape(nb, block, d)
+                dev = Kb - Kb.mean(axis=1, keepdims=True)
+                hbar = np.einsum("jnc,jne->ce", dev, V.reshape(nb, block, d)) / nb
+            num = num + ((scale * q) @ _f64(hbar)) * wc.sum(axis=1)[:, None]
         return num / den[:, None]
     if tail in ("drop", "linear_mix"):
         if a.shape[1]:
@@ -286,11 +308,12 @@ def sparse_attention(Q, K, V, block_idx, block: int, tail: str, scale: float,
     if tail == "linear_mix" and alpha is None:
         raise ValueError("linear_mix needs alpha [H, d]")
 
-    def one(b, h, i):
-        q = _f64(Q[b, h, i * block:(i + 1) * block])
-        return _attend_rows(q, _f64(K[b, h]), _f64(V[b, h]), idx[b, h, i], nb,
-                            block, tail, scale,
-                            None if alpha is None else alpha[h], eps)
+    def hbar_of(Kh, Vh):
+        if tail != "first_order":
+            return None
+        Kb = Kh.reshape(nb, block, d)
+        dev = Kb - Kb.mean(axis=1, keepdims=True)
+        return np.einsum("jnc,jne->ce", dev, Vh.reshape(nb, block, d)) / nb
 
     if qblocks is not None:
         qb = list(qblocks)
@@ -299,22 +322,24 @@ def sparse_attention(Q, K, V, block_idx, block: int, tail: str, scale: float,
         for r, (b, h, i) in enumerate(qb):
             key = (b, h)
             if key not in cache:
-                cache = {key: (_f64(K[b, h]), _f64(V[b, h]))}
-            Kh, Vh = cache[key]
+                Kh, Vh = _f64(K[b, h]), _f64(V[b, h])
+                cache = {key: (Kh, Vh, hbar_of(Kh, Vh))}
+            Kh, Vh, Hb = cache[key]
             q = _f64(Q[b, h, i * block:(i + 1) * block])
             out[r] = _attend_rows(q, Kh, Vh, idx[b, h, i], nb, block, tail, scale,
-                                  None if alpha is None else alpha[h], eps)
+                                  None if alpha is None else alpha[h], eps, hbar=Hb)
         return out
 
     O = np.empty((Bsz, H, Q.shape[2], d))
     for b in range(Bsz):
         for h in range(H):
             Kh, Vh = _f64(K[b, h]), _f64(V[b, h])
+            Hb = hbar_of(Kh, Vh)
             for i in range(Q.shape[2] // block):
                 q = _f64(Q[b, h, i * block:(i + 1) * block])
                 O[b, h, i * block:(i + 1) * block] = _attend_rows(
                     q, Kh, Vh, idx[b, h, i], nb, block, tail, scale,
-                    None if alpha is None else alpha[h], eps)
+                    None if alpha is None else alpha[h], eps, hbar=Hb)
     return O
 
 
