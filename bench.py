@@ -79,9 +79,12 @@ def dense_flops(w) -> float:
 def algorithmic_attn_flops(w) -> float:
     """FLOPs the method performs in the attention kernel: every query row takes
     4·d FLOPs (QKᵀ and PV) per exact key (k blocks × block tokens) and per
-    zero-order pseudo-key (nb − k unselected blocks)."""
-    keys = w.k * w.block + ((w.nb - w.k) if w.tail == "zero_order" else 0)
-    return 4.0 * w.d * keys * w.B * w.H * float(w.N)
+    zero-order pseudo-key (nb − k unselected blocks); the first-order tail adds
+    the row's (s q)ᵀ H̄, 2·d² FLOPs."""
+    tail = w.tail in ("zero_order", "first_order")
+    keys = w.k * w.block + ((w.nb - w.k) if tail else 0)
+    fo = 2.0 * w.d * w.d if (w.tail == "first_order" and w.k < w.nb) else 0.0
+    return (4.0 * w.d * keys + fo) * w.B * w.H * float(w.N)
 
 
 class ClockSampler:
@@ -320,6 +323,30 @@ def time_fp8(steps: int = 10, warmup: int = 3):
     return out
 
 
+def time_first_order(steps: int = 10, warmup: int = 3):
+    """PISA's hybrid-order tail on the video_dit inputs (same seed): the step
+    (block_pool with H̄ + route + attention) and the attention launch alone."""
+    from block_sparse_approximate_b200 import binding as bd
+    from block_sparse_approximate_b200.pipeline import PrefillStep
+    w = wl.WORKLOADS["video_dit_fo"]
+    inp = wl.prefill_inputs(w, "cuda")
+    step = PrefillStep(w, inp)
+    step()
+    attn = lambda: bd.sparse_attn_fwd(inp["Q"], inp["K"], inp["V"], step.buf.block_idx, w.block, w.tail,
+                                      step.buf.stats, w.scale, out=step.buf.out)
+    ms_step, attn_ms = _time_prefill_variant(step, attn, steps, warmup)
+    _, bf16, _, src = _peaks()
+    fl = algorithmic_attn_flops(w)
+    ach = fl / (attn_ms * 1e-3) / 1e12
+    out = {"workload": w.name, "ms_per_step": ms_step, "attn_ms": attn_ms, "executed_tflops": ach,
+           "dense_equiv_tflops": dense_flops(w) / (ms_step * 1e-3) / 1e12,
+           "peak_tflops": bf16, "frac": ach / bf16, "peak_source": f"{src} bf16 burst",
+           "step": "block_pool (+ H̄ on the tensor cores) + route + sparse_attn_fwd (first_order)"}
+    del inp, step
+    torch.cuda.empty_cache()
+    return out
+
+
 def linear_mix_flops(w) -> float:
     """Per query block: exact softmax part 4·d·(k·B)·B, the A_i accumulation
     2·d²·(k·B) and the final relu(Q)(H_tot − A_i) 2·d²·B."""
@@ -373,6 +400,10 @@ def run_ours(args, world, rank, local):
     if args.only == "sla2":
         if rank == 0:
             print(json.dumps({"sla2_mix": time_sla2(args.steps, args.warmup)}), flush=True)
+        return 0
+    if args.only == "fo":
+        if rank == 0:
+            print(json.dumps({"first_order": time_first_order(args.steps, args.warmup)}), flush=True)
         return 0
     w = wl.WORKLOADS[WORKLOAD]
     wr = rank_workload(w, rank)
@@ -462,13 +493,14 @@ def run_ours(args, world, rank, local):
                "h2d_bytes_per_step": sum(inp[n].numel() * inp[n].element_size() for n in ("Q", "K", "V")),
                "d2h_bytes_per_step": step.buf.out.numel() * step.buf.out.element_size()}
 
-    decode = fp8 = sla2 = None
+    decode = fp8 = sla2 = first_order = None
     if rank == 0 and args.only == "all" and not args.no_decode:
         del step
         torch.cuda.empty_cache()
         decode = time_decode(batch=args.decode_batch)
         fp8 = time_fp8()
         sla2 = time_sla2()
+        first_order = time_first_order()
     ck = clocks.stop() if clocks else None
 
     if rank != 0:
@@ -502,6 +534,7 @@ def run_ours(args, world, rank, local):
         "decode": decode,
         "fp8": fp8,
         "sla2_mix": sla2,
+        "first_order": first_order,
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -520,8 +553,9 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
-    ap.add_argument("--only", choices=["all", "prefill", "decode", "fp8", "sla2"], default="all",
-                    help="prefill: the timed step only; decode / fp8 / sla2: only that workload's timing")
+    ap.add_argument("--only", choices=["all", "prefill", "decode", "fp8", "sla2", "fo"], default="all",
+                    help="prefill: the timed step only; decode / fp8 / sla2 / fo (first-order tail): "
+                         "only that workload's timing")
     ap.add_argument("--decode-batch", type=int, default=None,
                     help="sequences in the decode workload (default: the full 16)")
     args = ap.parse_args(argv)

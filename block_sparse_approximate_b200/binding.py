@@ -22,7 +22,7 @@ LIB_PATH = os.path.join(_HERE, "libsparseattn.so")
 SA_OK, SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED, SA_ERR_ALIGNMENT, SA_ERR_CUDA, SA_ERR_WORKSPACE = range(6)
 SA_FP32, SA_BF16 = 0, 1
 ROUTE = {"dot": 0, "proj": 1, "taylor2": 2}
-TAIL = {"drop": 0, "zero_order": 1, "linear_mix": 2}
+TAIL = {"drop": 0, "zero_order": 1, "linear_mix": 2, "first_order": 3}
 
 # every entry point declared in include/sparseattn.h
 EXPORTS = ("sa_block_pool", "sa_route", "sa_sparse_attn_fwd", "sa_decode_workspace_size",
@@ -46,7 +46,8 @@ class DecodeShape(ctypes.Structure):
                 ("N", ctypes.c_int32), ("d", ctypes.c_int32), ("block", ctypes.c_int32)]
 
 
-_STAT_FIELDS = ("qmean", "kmean", "vsum", "kvar", "zrelu", "htot", "ztot", "kmean_bf16", "vmean_bf16")
+_STAT_FIELDS = ("qmean", "kmean", "vsum", "kvar", "zrelu", "htot", "ztot", "kmean_bf16", "vmean_bf16",
+                "hbar", "hbarT_bf16")
 
 
 class BlockStats(ctypes.Structure):
@@ -141,7 +142,7 @@ def version() -> str:
 
 def block_pool(Q: Optional[torch.Tensor], K: torch.Tensor, V: torch.Tensor, block: int, *,
                variance: bool = False, linear: bool = False, centroids_bf16: bool = False,
-               stream=None) -> dict:
+               first_order: bool = False, stream=None) -> dict:
     """Block statistics of (Q,) K, V [B,H,N,d]; returns a dict of float32 tensors."""
     lib = load()
     Bsz, H, N, d = K.shape
@@ -160,6 +161,10 @@ def block_pool(Q: Optional[torch.Tensor], K: torch.Tensor, V: torch.Tensor, bloc
     if centroids_bf16:
         st["kmean_bf16"] = torch.empty(Bsz, H, nb, d, device=dev, dtype=torch.bfloat16)
         st["vmean_bf16"] = torch.empty(Bsz, H, nb, d, device=dev, dtype=torch.bfloat16)
+    if first_order:
+        st["hbar"] = torch.empty(Bsz, H, d, d, **f)
+        if centroids_bf16:
+            st["hbarT_bf16"] = torch.empty(Bsz, H, d, d, device=dev, dtype=torch.bfloat16)
     cst = _stats_struct(st)
     _check("sa_block_pool", lib.sa_block_pool(_ptr(Q), _ptr(K), _ptr(V), _dtype_code(K),
                                               Shape(Bsz, H, N, d, block), ctypes.byref(cst),

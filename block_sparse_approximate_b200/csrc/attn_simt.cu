@@ -9,6 +9,10 @@
 //                value vsum_j / B and log-weight ln B (B e^{x} = e^{x + ln B}),
 //                which puts exp(s q·k̄_j)·vsum_j in the numerator and
 //                B·exp(s q·k̄_j) in the denominator (PISA §2, N_t and D_t);
+//   first-order: the zero-order pass, with each row's sum of the pseudo-key
+//                weights Λ_t = Σ_{j∈U} e^{s q·k̄_j} (relative to the row's
+//                running maximum) kept beside the softmax state; the epilogue
+//                adds Λ_t (s q_t)ᵀ H̄ to the numerator (PISA's hybrid order);
 //   linear_mix:  O_s from the exact part; O_l = relu(q)ᵀ(H_tot − A_i) /
 //                (relu(q)·(z_tot − ζ_i) + eps) with A_i = Σ_{j∈S_i} relu(K_j)ᵀV_j
 //                accumulated here from the tiles already in shared memory
@@ -42,6 +46,7 @@ attn_simt_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __re
   const size_t head_off = bh * (size_t)N * D;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const bool linear = tail == SA_TAIL_LINEAR_MIX;
+  const bool fo = tail == SA_TAIL_FIRST_ORDER;
   const int nwords = (nb + 31) / 32;
   const size_t row0 = (size_t)i * BLK + (size_t)half * QROWS;   // first query row
 
@@ -50,7 +55,8 @@ attn_simt_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __re
   float* acc = qs + QROWS * D;                      // QROWS * D
   float* mrow = acc + QROWS * D;                    // QROWS
   float* lrow = mrow + QROWS;                       // QROWS
-  float* ks = lrow + QROWS;                         // KT * KS
+  float* lcrow = lrow + QROWS;                      // QROWS: Λ_t · BLK (first-order)
+  float* ks = lcrow + QROWS;                        // KT * KS
   float* vs = ks + KT * KS;                         // KT * D
   float* zeta = vs + KT * D;                        // D
   uint32_t* selmask = reinterpret_cast<uint32_t*>(zeta + D);           // nwords
@@ -64,6 +70,7 @@ attn_simt_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __re
   for (int r = tid; r < QROWS; r += kSimtThreads) {
     mrow[r] = -INFINITY;
     lrow[r] = 0.f;
+    lcrow[r] = 0.f;
   }
   for (int w = tid; w < nwords; w += kSimtThreads) selmask[w] = 0u;
   if (linear)
@@ -85,8 +92,9 @@ attn_simt_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __re
   const float scale2 = scale * kLog2e;
 
   // online-softmax update of this warp's rows with the KT keys in ks/vs;
-  // bias2 is added to every logit (log2 domain); key `lane` counts if `valid`
-  auto consume_tile = [&](float bias2, bool valid) {
+  // bias2 is added to every logit (log2 domain); key `lane` counts if `valid`;
+  // `pseudo` tiles also add their weights to lcrow
+  auto consume_tile = [&](float bias2, bool valid, bool pseudo) {
     for (int rr = 0; rr < RPW; ++rr) {
       const int r = warp * RPW + rr;
       float x = 0.f;
@@ -117,6 +125,7 @@ attn_simt_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __re
       if (lane == 0) {
         mrow[r] = m_new;
         lrow[r] = lrow[r] * corr + psum;
+        lcrow[r] = lcrow[r] * corr + (pseudo ? psum : 0.f);
       }
       __syncwarp();
     }
@@ -134,7 +143,7 @@ attn_simt_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __re
         vs[idx] = to_f<T>(V[g]);
       }
       __syncthreads();
-      consume_tile(0.f, true);
+      consume_tile(0.f, true, false);
       if (linear) {
         // A[c][e] += Σ_n relu(k_n[c]) v_n[e]; thread -> (c, 8-column chunks)
         for (int item = tid; item < D * (D / 8); item += kSimtThreads) {
@@ -155,7 +164,7 @@ attn_simt_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __re
   }
 
   // ---- zero-order tail: unselected blocks as pseudo-keys
-  if (tail == SA_TAIL_ZERO_ORDER) {
+  if (tail == SA_TAIL_ZERO_ORDER || fo) {
     const float bias2 = log2f((float)BLK);
     const float inv_blk = 1.0f / BLK;
     for (int j0 = 0; j0 < nb; j0 += KT) {
@@ -174,7 +183,7 @@ attn_simt_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __re
       __syncthreads();
       const int j = j0 + lane;
       const bool valid = j < nb && !((selmask[j >> 5] >> (j & 31)) & 1u);
-      consume_tile(bias2, valid);
+      consume_tile(bias2, valid, true);
     }
   }
   __syncthreads();
@@ -185,6 +194,24 @@ attn_simt_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __re
     const float l = lrow[r];
     const float inv_l = l > 0.f ? 1.0f / l : 0.f;
     T* orow = O + head_off + (row0 + r) * D;
+    if (fo) {
+      // + Λ_t (s q_t)ᵀ H̄, Λ_t = lcrow / BLK on the same running maximum as acc
+      const float* qr = qs + r * D;
+      const float* Hb = st.hbar + bh * (size_t)D * D;
+      float num[PER];
+#pragma unroll
+      for (int e = 0; e < PER; ++e) num[e] = 0.f;
+      for (int c = 0; c < D; ++c) {
+        const float qc = qr[c];
+#pragma unroll
+        for (int e = 0; e < PER; ++e) num[e] = fmaf(qc, Hb[(size_t)c * D + lane * PER + e], num[e]);
+      }
+      const float w = scale * lcrow[r] * (1.0f / BLK);
+#pragma unroll
+      for (int e = 0; e < PER; ++e)
+        orow[lane * PER + e] = from_f<T>(fmaf(w, num[e], acc[r * D + lane * PER + e]) * inv_l);
+      continue;
+    }
     if (!linear) {
 #pragma unroll
       for (int c = 0; c < PER; ++c) orow[lane * PER + c] = from_f<T>(acc[r * D + lane * PER + c] * inv_l);
@@ -238,7 +265,7 @@ sa_status launch_simt(const void* Q, const void* K, const void* V, const sa_shap
                       const sa_block_stats& st, float scale, void* O, cudaStream_t stream) {
   const int nb = s.N / BLK;
   const int nwords = (nb + 31) / 32;
-  size_t smem = sizeof(float) * (2 * (size_t)QROWS * D + 2 * QROWS + (size_t)KT * (D + 1) +
+  size_t smem = sizeof(float) * (2 * (size_t)QROWS * D + 3 * QROWS + (size_t)KT * (D + 1) +
                                  (size_t)KT * D + D) +
                 sizeof(uint32_t) * ((nwords + 3) & ~3);
   if (tail == SA_TAIL_LINEAR_MIX) smem += sizeof(float) * (size_t)D * D;

@@ -192,12 +192,14 @@ __device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float
   return lo | (hi << 16);
 }
 
-template <bool ZO, bool F8>
+template <bool ZO, bool F8, bool FO>
 __global__ void __launch_bounds__(kTcThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKb,
-               const __grid_constant__ CUtensorMap tmVb, const int32_t* __restrict__ block_idx, int nb,
-               int topk, float scale2, F8Scales f8, __nv_bfloat16* __restrict__ O, int N) {
+               const __grid_constant__ CUtensorMap tmVb, const __grid_constant__ CUtensorMap tmHb,
+               const int32_t* __restrict__ block_idx, int nb, int topk, float scale2, F8Scales f8,
+               __nv_bfloat16* __restrict__ O, int N) {
+  static_assert(!FO || (ZO && !F8), "the first-order tail extends the bf16 zero-order tail");
   using L = Layout<F8>;
   constexpr int NS = L::NS;
   constexpr uint32_t kTile = L::kTile;
@@ -216,6 +218,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const int nwords = (nb + 31) >> 5;
   const int ntail = (ZO && topk < nb) ? (nb + TB - 1) / TB : 0;
   const int T = topk + ntail;
+  // first-order tail: one more S MMA, S' = Q H̄ (tile T, K slot only), into
+  // the S columns of stream T % 2 once that stream's last P has been read
+  const bool fo = FO && ntail > 0;
+  const int Tx = T + (fo ? 1 : 0);
   const int32_t* sel = block_idx + ((size_t)bh * nb + i) * topk;
 
   if (threadIdx.x == 0) {
@@ -255,13 +261,23 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         prefetch_tmap(&tmKb);
         prefetch_tmap(&tmVb);
       }
+      if (FO) prefetch_tmap(&tmHb);
       mbar_expect_tx(bar(L::B_Q), kTile);
 #pragma unroll
       for (int h = 0; h < kSpans; ++h) tma_load_3d(sb + h * kSpan, &tmQ, 64 * h, i * TB, bh, bar(L::B_Q));
       int issued = 0;
-      for (int t = 0; t < T; ++t) {
+      for (int t = 0; t < Tx; ++t) {
         const int s = t % NS;
         if (t >= NS && !mbar_wait(bar(L::B_KE + s), ((t / NS) - 1) & 1, abort_flag)) break;
+        if (FO && t == T) {
+          // H̄ᵀ of this head [d rows = output channel e][d cols = c] as a K tile
+          const uint32_t ka = sb + kTile * (1 + 2 * s);
+          mbar_expect_tx(bar(L::B_KF + s), kTile);
+#pragma unroll
+          for (int h = 0; h < kSpans; ++h) tma_load_3d(ka + h * kSpan, &tmHb, 64 * h, 0, bh, bar(L::B_KF + s));
+          issued = t + 1;
+          break;
+        }
         const bool exact = t < topk;
         const CUtensorMap* mk = exact ? &tmK : &tmKb;
         const CUtensorMap* mv = exact ? &tmV : &tmVb;
@@ -280,7 +296,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         wait_bounded(bar(L::B_Q), 0);
         for (int t = issued > NS ? issued - NS : 0; t < issued; ++t) {
           wait_bounded(bar(L::B_KF + t % NS), (t / NS) & 1);
-          wait_bounded(bar(L::B_VF + t % NS), (t / NS) & 1);
+          if (t < T) wait_bounded(bar(L::B_VF + t % NS), (t / NS) & 1);
         }
       }
     }
@@ -312,7 +328,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       };
       bool ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_Q), 0, abort_flag));
       if (ok) ok = issue_s(0);
-      if (ok && T > 1) ok = issue_s(1);
+      if (ok && Tx > 1) ok = issue_s(1);
       for (int t = 0; ok && t < T; ++t) {
         const int st = t & 1, u = t >> 1, su = t % NS;
         if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_PR + st), u & 1, abort_flag))) break;
@@ -330,7 +346,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
         mma_commit_w(bar(L::B_KE + su));
         mma_commit_w(bar(L::B_OD + st));
-        if (t + 2 < T && !issue_s(t + 2)) break;
+        if (t + 2 < Tx && !issue_s(t + 2)) break;
       }
       // every MMA issued above has completed before TMEM is released
       mma_commit_w(bar(L::B_FIN));
@@ -363,6 +379,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       qs = f8.q[(size_t)bh * nb + i];
     }
     float m_used = -INFINITY, l = 0.f;
+    float lc = 0.f;   // first-order: the centroid tiles' share of l
     bool ok = true;
     for (int u = 0; u < U; ++u) {
       const int t = 2 * u + st;
@@ -452,6 +469,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       }
       const float sum = ((sm8[0] + sm8[1]) + (sm8[2] + sm8[3])) + ((sm8[4] + sm8[5]) + (sm8[6] + sm8[7]));
       l = l * factor + sum;
+      if (FO) lc = lc * factor + (centroid ? sum : 0.f);
       tmem_st32(lrow + s_col, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
       if (!F8) tmem_st32(lrow + s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
       tmem_wait_st();
@@ -481,11 +499,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     // both groups past their last PV: every MMA that reads Q has completed,
     // so the Q tile's shared memory can carry the (max, sum) exchange
     named_bar_softmax();
-    float* ex = reinterpret_cast<float*>(smem);   // [2 streams][2][128]
-    ex[st * 256 + r] = (U > 0) ? m_used : -INFINITY;
-    ex[st * 256 + 128 + r] = l;
+    constexpr int kEx = FO ? 384 : 256;
+    float* ex = reinterpret_cast<float*>(smem);   // [2 streams][2 or 3][128]
+    ex[st * kEx + r] = (U > 0) ? m_used : -INFINITY;
+    ex[st * kEx + 128 + r] = l;
+    if (FO) ex[st * kEx + 256 + r] = lc;
     named_bar_softmax();
-    const float m0 = ex[r], l0 = ex[128 + r], m1 = ex[256 + r], l1 = ex[384 + r];
+    const float m0 = ex[r], l0 = ex[128 + r], m1 = ex[kEx + r], l1 = ex[kEx + 128 + r];
     const int U0 = T > 0 ? (T + 1) / 2 : 0, U1 = T > 1 ? T / 2 : 0;
     const float M = fmaxf(m0, m1);
     const float f0 = (U0 > 0 && m0 != -INFINITY) ? fast_exp2(m0 - M) : 0.f;
@@ -493,6 +513,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const float L_ = l0 * f0 + l1 * f1;
     // e4m3: O accumulated Σ P σ_V V̂ · 448 / σ_Vmax
     const float inv = L_ > 0.f ? (F8 ? vmax / 448.0f : 1.0f) / L_ : 0.f;
+    // first-order: + Λ_t (s q_t)ᵀ H̄ with Λ_t = Σ_U e^{s q·k̄_j} on the merged
+    // maximum (the centroid tiles' sums carry the factor 128 = e^{ln 128})
+    float wfo = 0.f;
+    const uint32_t sp_col = (uint32_t)(T & 1) * TB + 64u * st;
+    if (FO && fo) {
+      const float lc0 = ex[256 + r], lc1 = ex[kEx + 256 + r];
+      wfo = scale2 * 0.6931471805599453f * (1.0f / 128.0f) * (lc0 * f0 + lc1 * f1);
+      // S' = Q H̄ is the (U_b + 1)-th completion of stream b = T % 2's S barrier
+      const int Ub = (T & 1) ? U1 : U0;
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_SF + (T & 1)), Ub & 1, abort_flag));
+    }
     ok = __all_sync(0xffffffffu, ok) && !*abort_flag;
     if (ok) {
       tc_fence_after();
@@ -507,6 +538,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (U1 > 0) {
           tmem_ld32(lrow + kColO + TD + 64 * st + 32 * c, b);
         }
+        uint32_t sp[32];
+        if (FO && fo) tmem_ld32(lrow + sp_col + 32 * c, sp);
         tmem_wait_ld();
         if (U0 == 0) {
 #pragma unroll
@@ -520,8 +553,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         for (int q = 0; q < 4; ++q) {
           float y[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            y[e] = (__uint_as_float(a[8 * q + e]) * f0 + __uint_as_float(b[8 * q + e]) * f1) * inv;
+          for (int e = 0; e < 8; ++e) {
+            float acc = __uint_as_float(a[8 * q + e]) * f0 + __uint_as_float(b[8 * q + e]) * f1;
+            if (FO && fo) acc = fmaf(wfo, __uint_as_float(sp[8 * q + e]), acc);
+            y[e] = acc * inv;
+          }
           uint4 w;
           w.x = pack_bf16(y[0], y[1]);
           w.y = pack_bf16(y[2], y[3]);
@@ -577,15 +613,19 @@ bool make_tmap_3d(CUtensorMap* map, const void* base, int elem, uint64_t cols, u
 
 template <bool F8>
 sa_status launch_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mkb,
-                    const CUtensorMap& mvb, bool zo, const sa_shape& s, const int32_t* block_idx, int topk,
-                    float scale, const F8Scales& f8, void* O, cudaStream_t stream) {
+                    const CUtensorMap& mvb, const CUtensorMap& mhb, bool zo, bool fo, const sa_shape& s,
+                    const int32_t* block_idx, int topk, float scale, const F8Scales& f8, void* O,
+                    cudaStream_t stream) {
   const int nb = s.N / TB;
   const size_t smem = Layout<F8>::smem_bytes(nb);
-  auto kern = zo ? attn_tc_kernel<true, F8> : attn_tc_kernel<false, F8>;
+  auto kern = zo ? attn_tc_kernel<true, F8, false> : attn_tc_kernel<false, F8, false>;
+  if constexpr (!F8) {
+    if (fo) kern = attn_tc_kernel<true, false, true>;
+  }
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return launch_status("cudaFuncSetAttribute(attn_tc_kernel)");
   dim3 grid(nb, (unsigned)((uint64_t)s.B * s.H));
-  kern<<<grid, kTcThreads, smem, stream>>>(mq, mk, mv, mkb, mvb, block_idx, nb, topk, scale * kLog2e, f8,
+  kern<<<grid, kTcThreads, smem, stream>>>(mq, mk, mv, mkb, mvb, mhb, block_idx, nb, topk, scale * kLog2e, f8,
                                            static_cast<__nv_bfloat16*>(O), s.N);
   return launch_status("attn_tc_kernel");
 }
@@ -974,12 +1014,17 @@ attn_tc_linmix_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
   }
 }
 
-// ---------------------------------------------------------------- H_tot
-// H_tot = Σ_n relu(k_n) v_nᵀ of one head (the total of SLA2's ReLU linear
-// branch, SALAD §2) on the tensor cores: a CTA takes a chunk of 128-token
-// tiles of one head, warps 2-5 apply ReLU in place to each K tile, warp 1
-// accumulates relu(K)ᵀ V in TMEM (MN-major × MN-major MMA), and the chunk's
-// d×d sum is added to htot with vector atomics.  Warp 0 is the TMA producer.
+// ---------------------------------------------------------------- H_tot, H̄
+// d×d outer-product sums Σ_n f(k_n) v_nᵀ of one head on the tensor cores:
+//   kmean == NULL: f = relu, H_tot (the total of SLA2's ReLU linear branch,
+//                  SALAD §2);
+//   kmean != NULL: f(k_n) = k_n − k̄_j with k̄_j the centroid of the 128-token
+//                  block that holds n, each chunk's sum scaled by oscale
+//                  (1/nb): PISA's mean first-order statistic H̄ (§2).
+// A CTA takes a chunk of 128-token tiles of one head, warps 2-5 apply f in
+// place to each K tile, warp 1 accumulates f(K)ᵀ V in TMEM (MN-major ×
+// MN-major MMA), and the chunk's d×d sum is added to `out` with vector
+// atomics.  Warp 0 is the TMA producer.
 constexpr int kHtThreads = 192;
 constexpr int kHtTiles = 32;          // tiles (of 128 tokens) per CTA
 struct HtLayout {
@@ -994,7 +1039,7 @@ struct HtLayout {
 
 __global__ void __launch_bounds__(kHtThreads, 1)
 htot_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, int N,
-               float* __restrict__ htot) {
+               const float* __restrict__ kmean, float oscale, float* __restrict__ htot) {
   using L = HtLayout;
   constexpr int NS = L::NS;
   constexpr uint32_t kTile = L::kTile;
@@ -1068,8 +1113,12 @@ htot_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
       wait_bounded(bar(L::B_DONE), 0);
     }
   } else {
-    // warps 2-5: ReLU of each K tile, then the epilogue (TMEM lane quarter w % 4)
+    // warps 2-5: f of each K tile, then the epilogue (TMEM lane quarter w % 4)
     const int tr = threadIdx.x - 64;
+    // 128-byte swizzle: the 16-byte vectors tr + 128 m of a tile all sit in
+    // row ≡ tr / 8 (mod 8) at physical chunk tr % 8, i.e. channels
+    // 64 (m / 8) + 8 ((tr % 8) ^ (tr / 8 % 8)) + [0, 8)
+    const int chunk8 = 8 * ((tr & 7) ^ ((tr >> 3) & 7));
     bool ok = true;
     for (int t = 0; t < T; ++t) {
       const int s = t % NS;
@@ -1078,14 +1127,37 @@ htot_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
         break;
       }
       uint4* kt = reinterpret_cast<uint4*>(smem + 2 * kTile * s);
-      const __nv_bfloat162 zero = __float2bfloat162_rn(0.f);
-#pragma unroll 4
-      for (int x = tr; x < (int)(kTile / 16); x += 128) {
-        uint4 u = kt[x];
-        __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+      if (kmean) {
+        const float* cen = kmean + ((size_t)bh * ntile_head + t0 + t) * TD + chunk8;
+        float c8[2][8];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) h[e] = __hmax2(h[e], zero);
-        kt[x] = u;
+        for (int h = 0; h < 2; ++h) {
+          const float4 a = *reinterpret_cast<const float4*>(cen + 64 * h);
+          const float4 b = *reinterpret_cast<const float4*>(cen + 64 * h + 4);
+          c8[h][0] = a.x; c8[h][1] = a.y; c8[h][2] = a.z; c8[h][3] = a.w;
+          c8[h][4] = b.x; c8[h][5] = b.y; c8[h][6] = b.z; c8[h][7] = b.w;
+        }
+#pragma unroll
+        for (int m = 0; m < (int)(kTile / 16) / 128; ++m) {
+          uint4 u = kt[tr + 128 * m];
+          __nv_bfloat162* hh = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(hh[e]);
+            hh[e] = __floats2bfloat162_rn(f.x - c8[m >> 3][2 * e], f.y - c8[m >> 3][2 * e + 1]);
+          }
+          kt[tr + 128 * m] = u;
+        }
+      } else {
+        const __nv_bfloat162 zero = __float2bfloat162_rn(0.f);
+#pragma unroll 4
+        for (int x = tr; x < (int)(kTile / 16); x += 128) {
+          uint4 u = kt[x];
+          __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) h[e] = __hmax2(h[e], zero);
+          kt[x] = u;
+        }
       }
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       mbar_arrive(bar(L::B_RL + s));
@@ -1104,8 +1176,9 @@ htot_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
         tmem_wait_ld();
 #pragma unroll
         for (int q4 = 0; q4 < 8; ++q4)
-          atomicAdd(hrow + 8 * cc + q4, make_float4(__uint_as_float(a[4 * q4]), __uint_as_float(a[4 * q4 + 1]),
-                                                    __uint_as_float(a[4 * q4 + 2]), __uint_as_float(a[4 * q4 + 3])));
+          atomicAdd(hrow + 8 * cc + q4,
+                    make_float4(__uint_as_float(a[4 * q4]) * oscale, __uint_as_float(a[4 * q4 + 1]) * oscale,
+                                __uint_as_float(a[4 * q4 + 2]) * oscale, __uint_as_float(a[4 * q4 + 3]) * oscale));
       }
     }
   }
@@ -1120,8 +1193,9 @@ htot_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
 
 }  // namespace
 
-sa_status htot_tc(const void* K, const void* V, const sa_shape& s, float* htot, cudaStream_t stream) {
-  if (s.d != TD || (s.N % TB)) return SA_ERR_UNSUPPORTED;
+sa_status kv_outer_tc(const void* K, const void* V, const sa_shape& s, const float* kmean, float oscale,
+                      float* out, cudaStream_t stream) {
+  if (s.d != TD || (s.N % TB) || (kmean && s.block != TB)) return SA_ERR_UNSUPPORTED;
   const uint64_t BH = (uint64_t)s.B * s.H;
   CUtensorMap mk, mv;
   if (!make_tmap_3d(&mk, K, 2, TD, s.N, BH) || !make_tmap_3d(&mv, V, 2, TD, s.N, BH))
@@ -1131,13 +1205,14 @@ sa_status htot_tc(const void* K, const void* V, const sa_shape& s, float* htot, 
     return launch_status("cudaFuncSetAttribute(htot_tc_kernel)");
   const int nt = s.N / TB;
   dim3 grid((nt + kHtTiles - 1) / kHtTiles, (unsigned)BH);
-  htot_tc_kernel<<<grid, kHtThreads, smem, stream>>>(mk, mv, s.N, htot);
+  htot_tc_kernel<<<grid, kHtThreads, smem, stream>>>(mk, mv, s.N, kmean, oscale, out);
   return launch_status("htot_tc_kernel");
 }
 
 bool attn_tc_supports(sa_dtype dtype, const sa_shape& s, sa_tail_mode tail) {
   return dtype == SA_BF16 && s.block == TB && s.d == TD &&
-         (tail == SA_TAIL_DROP || tail == SA_TAIL_ZERO_ORDER || tail == SA_TAIL_LINEAR_MIX);
+         (tail == SA_TAIL_DROP || tail == SA_TAIL_ZERO_ORDER || tail == SA_TAIL_LINEAR_MIX ||
+          tail == SA_TAIL_FIRST_ORDER);
 }
 
 sa_status attn_tc(const void* Q, const void* K, const void* V, const sa_shape& s, const int32_t* block_idx,
@@ -1160,7 +1235,9 @@ sa_status attn_tc(const void* Q, const void* K, const void* V, const sa_shape& s
                                                               static_cast<__nv_bfloat16*>(O), s.N);
     return launch_status("attn_tc_linmix_kernel");
   }
-  const bool zo = tail == SA_TAIL_ZERO_ORDER;
+  const bool fo = tail == SA_TAIL_FIRST_ORDER;
+  const bool zo = tail == SA_TAIL_ZERO_ORDER || fo;
+  CUtensorMap mhb = mk;
   if (zo) {
     if (!make_tmap_3d(&mkb, st.kmean_bf16, 2, TD, nb, BH) || !make_tmap_3d(&mvb, st.vmean_bf16, 2, TD, nb, BH))
       return fail(SA_ERR_CUDA, "sa_sparse_attn_fwd: cuTensorMapEncodeTiled failed for the block centroids");
@@ -1168,7 +1245,9 @@ sa_status attn_tc(const void* Q, const void* K, const void* V, const sa_shape& s
     mkb = mk;
     mvb = mv;
   }
-  return launch_tc<false>(mq, mk, mv, mkb, mvb, zo, s, block_idx, topk, scale, F8Scales{}, O, stream);
+  if (fo && !make_tmap_3d(&mhb, st.hbarT_bf16, 2, TD, TD, BH))
+    return fail(SA_ERR_CUDA, "sa_sparse_attn_fwd: cuTensorMapEncodeTiled failed for H̄ᵀ");
+  return launch_tc<false>(mq, mk, mv, mkb, mvb, mhb, zo, fo, s, block_idx, topk, scale, F8Scales{}, O, stream);
 }
 
 }  // namespace sa
@@ -1210,7 +1289,8 @@ extern "C" sa_status sa_sparse_attn_fwd_fp8(const sa_fp8_operands* ops, sa_shape
     mvb = mv;
   }
   F8Scales f8{ops->q_scale, ops->k_scale, ops->v_scale, ops->v_scale_max, ops->kbar_scale, ops->vbar_scale};
-  return launch_tc<true>(mq, mk, mv, mkb, mvb, zo, shape, block_idx, topk, scale, f8, O, as_stream(stream));
+  return launch_tc<true>(mq, mk, mv, mkb, mvb, mk, zo, false, shape, block_idx, topk, scale, f8, O,
+                         as_stream(stream));
 }
 
 extern "C" sa_status sa_device_error(uint32_t* code) {

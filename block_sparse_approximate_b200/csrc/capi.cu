@@ -41,7 +41,8 @@ extern "C" sa_status sa_sparse_attn_fwd(const void* Q, const void* K, const void
   const int nb = shape.N / shape.block;
   if (dtype != SA_FP32 && dtype != SA_BF16)
     return fail(SA_ERR_UNSUPPORTED, "sa_sparse_attn_fwd: dtype must be SA_FP32 or SA_BF16");
-  if (tail != SA_TAIL_DROP && tail != SA_TAIL_ZERO_ORDER && tail != SA_TAIL_LINEAR_MIX)
+  if (tail != SA_TAIL_DROP && tail != SA_TAIL_ZERO_ORDER && tail != SA_TAIL_LINEAR_MIX &&
+      tail != SA_TAIL_FIRST_ORDER)
     return fail(SA_ERR_INVALID_ARG, "sa_sparse_attn_fwd: unknown tail mode");
   if (shape.B == 0 || shape.H == 0 || shape.N == 0) return SA_OK;  // nothing to compute
   if (!Q || !K || !V || !O) return fail(SA_ERR_INVALID_ARG, "sa_sparse_attn_fwd: Q, K, V and O are required");
@@ -52,16 +53,21 @@ extern "C" sa_status sa_sparse_attn_fwd(const void* Q, const void* K, const void
   if (stats) st = *stats;
   if (tail == SA_TAIL_ZERO_ORDER && (!st.kmean || !st.vsum))
     return fail(SA_ERR_INVALID_ARG, "sa_sparse_attn_fwd: SA_TAIL_ZERO_ORDER needs stats->kmean and stats->vsum");
+  if (tail == SA_TAIL_FIRST_ORDER && (!st.kmean || !st.vsum || !st.hbar))
+    return fail(SA_ERR_INVALID_ARG,
+                "sa_sparse_attn_fwd: SA_TAIL_FIRST_ORDER needs stats->kmean, stats->vsum and stats->hbar");
   if (tail == SA_TAIL_LINEAR_MIX && (!alpha || !st.zrelu || !st.htot || !st.ztot))
     return fail(SA_ERR_INVALID_ARG,
                 "sa_sparse_attn_fwd: SA_TAIL_LINEAR_MIX needs alpha and stats->zrelu, htot, ztot");
   const void* ptrs[] = {Q, K, V, O, block_idx, alpha, st.kmean, st.vsum, st.zrelu, st.htot, st.ztot,
-                        st.kmean_bf16, st.vmean_bf16};
+                        st.kmean_bf16, st.vmean_bf16, st.hbar, st.hbarT_bf16};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return fail(SA_ERR_ALIGNMENT, "sa_sparse_attn_fwd: pointers must be 16-byte aligned");
   cudaStream_t s = as_stream(stream);
-  if (attn_tc_supports(dtype, shape, tail) &&
-      (tail != SA_TAIL_ZERO_ORDER || (st.kmean_bf16 && st.vmean_bf16)))
+  // the tensor-core kernel reads the tails' operands as bf16 tiles
+  const bool tc_operands = (tail != SA_TAIL_ZERO_ORDER && tail != SA_TAIL_FIRST_ORDER) ||
+                           (st.kmean_bf16 && st.vmean_bf16 && (tail == SA_TAIL_ZERO_ORDER || st.hbarT_bf16));
+  if (attn_tc_supports(dtype, shape, tail) && tc_operands)
     return attn_tc(Q, K, V, shape, block_idx, topk, tail, alpha, st, scale, O, s);
   return attn_simt(Q, K, V, dtype, shape, block_idx, topk, tail, alpha, st, scale, O, s);
 }

@@ -18,6 +18,8 @@ long-context LLM decoding; these synthetic inputs stand in for them):
 * ``sla2_mix``  B=1, H=40, N=65536 on a 16x64x64 grid, generated as
                 ``video_dit``; block 128; projected router with proj_q, proj_k
                 ~ N(0, 1/d); keep 5%; linear_mix with alpha ~ U(0.2, 0.9).
+* ``video_dit_fo``  ``video_dit`` (same seed, same inputs) with PISA's
+                first-order tail.
 * ``fp8``       ``video_dit`` shapes, e4m3 sparse branch; zero-order tail.
 * ``decode``    16 sequences, 32 query heads, 8 KV heads, d=128, bf16 cache of
                 131072 tokens: K, V ~ N(0,1) plus an N(0, 0.5) offset per
@@ -49,7 +51,7 @@ class Workload:
     dtype: str                 # "fp32" | "bf16"
     block: int
     route: str                 # "dot" | "proj" | "taylor2"
-    tail: str                  # "drop" | "zero_order" | "linear_mix"
+    tail: str                  # "drop" | "zero_order" | "first_order" | "linear_mix"
     seed: int
     topk: Optional[int] = None
     keep_pct: Optional[int] = None
@@ -86,6 +88,9 @@ WORKLOADS = {
     "sla2_mix": Workload("sla2_mix", B=1, H=40, N=16 * 64 * 64, d=128, dtype="bf16",
                          block=128, route="proj", tail="linear_mix", seed=2,
                          keep_pct=5, grid=(16, 64, 64)),
+    "video_dit_fo": Workload("video_dit_fo", B=1, H=12, N=8 * 64 * 64, d=128, dtype="bf16",
+                             block=128, route="dot", tail="first_order", seed=1,
+                             keep_pct=10, grid=(8, 64, 64)),
     "fp8": Workload("fp8", B=1, H=12, N=8 * 64 * 64, d=128, dtype="bf16",
                     block=128, route="dot", tail="zero_order", seed=3,
                     keep_pct=10, grid=(8, 64, 64), fp8=True),
@@ -175,6 +180,29 @@ def prefill_inputs(w: Workload, device="cpu", *, H: Optional[int] = None,
     if w.tail == "linear_mix":
         out["alpha"] = (0.2 + 0.7 * torch.rand(Hh, w.d, generator=gen, device=dev)).contiguous()
     return out
+
+
+def block_linear_inputs(B: int, H: int, nb: int, block: int, d: int, dtype, seed: int, device="cpu",
+                        dev_std: float = 0.5, mix: float = 4.0, noise: float = 0.1) -> dict:
+    """Q, K, V [B,H,nb*block,d] whose values follow the keys' in-block deviations.
+
+    Every key block j has a centroid c_j ~ N(0, I) and deviations
+    e_n ~ N(0, dev_std² I) shifted to zero mean over the block: k_n = c_j + e_n.
+    Values are v_n = e_n M + noise·N(0, I) with one M ~ N(0, mix²/d) per head,
+    so the blocks share a first-order statistic Σ_n e_n v_nᵀ of order
+    block·dev_std²·M; queries are N(0, I).
+    """
+    dev = torch.device(device)
+    gen = _gen(seed, dev)
+    N = nb * block
+    c = torch.randn(B, H, nb, 1, d, generator=gen, device=dev)
+    e = torch.randn(B, H, nb, block, d, generator=gen, device=dev) * dev_std
+    e = e - e.mean(dim=3, keepdim=True)
+    K = (c + e).reshape(B, H, N, d)
+    M = torch.randn(B, H, d, d, generator=gen, device=dev) * (mix / math.sqrt(d))
+    V = e.reshape(B, H, N, d) @ M + noise * torch.randn(B, H, N, d, generator=gen, device=dev)
+    Q = torch.randn(B, H, N, d, generator=gen, device=dev)
+    return {n: x.to(dtype).contiguous() for n, x in (("Q", Q), ("K", K), ("V", V))}
 
 
 def decode_inputs(w: Workload, device="cpu", *, B: Optional[int] = None,

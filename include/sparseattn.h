@@ -62,9 +62,13 @@ typedef enum {
   SA_TAIL_DROP = 0,        /* unselected blocks contribute nothing */
   SA_TAIL_ZERO_ORDER = 1,  /* PISA zero-order block term inside numerator
                               and denominator [PISA §2 "Algoritmo Central"] */
-  SA_TAIL_LINEAR_MIX = 2   /* O = α⊙O_s + (1−α)⊙O_l, O_l = ReLU linear
+  SA_TAIL_LINEAR_MIX = 2,  /* O = α⊙O_s + (1−α)⊙O_l, O_l = ReLU linear
                               attention over the unselected blocks
                               [SLA2 §2A, SALAD §2, SPLA §2.2] */
+  SA_TAIL_FIRST_ORDER = 3  /* PISA hybrid order: the zero-order terms plus
+                              the global first-order correction of the
+                              numerator, (s q) H̄ Σ_{j∈U} e^{s q·k̄_j}
+                              [PISA §2 "Algoritmo Central"] */
 } sa_tail_mode;
 
 /* Shape of a prefill problem: Q, K, V, O are [B, H, N, d]; query blocks and
@@ -94,13 +98,19 @@ typedef struct {
   float* ztot;      /* [B,H,d]     Σ_n relu(k_n) over all tokens             */
   uint16_t* kmean_bf16;  /* [B,H,nb,d] bf16 copy of kmean (tensor-core tail) */
   uint16_t* vmean_bf16;  /* [B,H,nb,d] bf16 of vsum / block (tensor-core tail) */
+  float* hbar;      /* [B,H,d,d]   H̄ = (1/nb) Σ_j Σ_{n∈j} (k_n − k̄_j) v_nᵀ, the
+                       mean first-order block statistic of PISA's hybrid
+                       order [PISA §2]; row c, column e                     */
+  uint16_t* hbarT_bf16;  /* [B,H,d,d] bf16 of H̄ᵀ (row e, column c; the
+                       tensor-core first-order tail)                        */
 } sa_block_stats;
 
 /* Block statistics of Q (optional), K and V.
  * Q: [B,H,N,d] or NULL (then stats->qmean is ignored); K, V: [B,H,N,d];
  * dtype: element type of Q, K, V.  Every non-NULL field of *stats is written;
- * kmean and vsum are required.  htot and ztot are sums over all tokens of a
- * head and are overwritten (no accumulation across calls).
+ * kmean and vsum are required.  htot, ztot and hbar are sums over all tokens
+ * of a head and are overwritten (no accumulation across calls); hbarT_bf16
+ * needs hbar.
  * Errors: SA_ERR_INVALID_ARG (null K/V/stats/kmean/vsum, bad shape),
  *         SA_ERR_UNSUPPORTED (d or block not supported), SA_ERR_ALIGNMENT. */
 sa_status sa_block_pool(const void* Q, const void* K, const void* V, sa_dtype dtype,
@@ -124,6 +134,11 @@ sa_status sa_route(const sa_block_stats* stats, sa_shape shape, sa_route_mode mo
  *   DROP:        o_t = Σ_{n∈S} e^{s q·k_n} v_n / Σ_{n∈S} e^{s q·k_n}  (0 if S empty)
  *   ZERO_ORDER:  o_t = (Σ_{n∈S} e^{s q·k_n} v_n + Σ_{j∈U} e^{s q·k̄_j} vsum_j)
  *                    / (Σ_{n∈S} e^{s q·k_n}     + Σ_{j∈U} block·e^{s q·k̄_j})
+ *   FIRST_ORDER: ZERO_ORDER with the numerator's first-order block term
+ *                added through the head's mean statistic H̄ (stats->hbar):
+ *                o_t = (N_t^ZO + (s q_t)ᵀ H̄ · Σ_{j∈U} e^{s q·k̄_j}) / D_t^ZO
+ *                (the denominator's first-order term is zero: a block's key
+ *                deviations from k̄_j sum to zero)
  *   LINEAR_MIX:  o_t = α_h ⊙ O_s + (1−α_h) ⊙ O_l,  O_s the DROP output,
  *                O_l = relu(q)ᵀ(H_tot − Σ_{j∈S} h_j) / (relu(q)·(z_tot − Σ_{j∈S} z_j) + 1e-6),
  *                h_j = Σ_{n∈j} relu(k_n) v_nᵀ (accumulated from the tiles the
@@ -133,6 +148,7 @@ sa_status sa_route(const sa_block_stats* stats, sa_shape shape, sa_route_mode mo
  * [B,H,nqb,topk] int32, each row ascending without repeats, entries in
  * [0, nb).  alpha: [H,d] float32 (LINEAR_MIX only).  stats: ZERO_ORDER needs
  * kmean, vsum (and kmean_bf16, vmean_bf16 for the bf16 tensor-core path);
+ * FIRST_ORDER needs those and hbar (+ hbarT_bf16 for the tensor-core path);
  * LINEAR_MIX needs zrelu, htot, ztot.
  * Errors: SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED, SA_ERR_ALIGNMENT. */
 sa_status sa_sparse_attn_fwd(const void* Q, const void* K, const void* V, sa_dtype dtype,

@@ -29,6 +29,22 @@ def test_exports_every_declared_symbol(lib):
     assert set(bd.EXPORTS) <= declared
 
 
+def _header():
+    return open(os.path.join(ROOT, "include", "sparseattn.h")).read()
+
+
+def test_binding_mirrors_header_layouts():
+    # the ctypes structs and enum maps follow the header's declarations
+    txt = _header()
+    body = re.search(r"typedef struct \{(.*?)\} sa_block_stats;", txt, flags=re.S).group(1)
+    fields = re.findall(r"^\s*(?:float|uint16_t)\*\s*(\w+);", body, flags=re.M)
+    assert tuple(fields) == bd._STAT_FIELDS
+    tails = dict((n.lower(), int(v)) for n, v in re.findall(r"SA_TAIL_(\w+)\s*=\s*(\d+)", txt))
+    assert tails == bd.TAIL
+    routes = dict((n.lower(), int(v)) for n, v in re.findall(r"SA_ROUTE_(\w+)\s*=\s*(\d+)", txt))
+    assert routes == bd.ROUTE
+
+
 def test_version(lib):
     assert "sm_100a" in bd.version()
 
@@ -53,6 +69,9 @@ def test_block_pool_validation(lib):
     assert "16-byte" in lib.sa_last_error().decode()
     # empty problem: nothing to launch
     assert lib.sa_block_pool(None, FAKE, FAKE, 1, bd.Shape(1, 1, 0, 128, 128), ctypes.byref(st), None) == bd.SA_OK
+    st2 = _stats(kmean=FAKE, vsum=FAKE, hbarT_bf16=FAKE)     # hbarT_bf16 without hbar
+    assert lib.sa_block_pool(None, FAKE, FAKE, 1, bd.Shape(1, 1, 256, 128, 128), ctypes.byref(st2), None) \
+        == bd.SA_ERR_INVALID_ARG
 
 
 def test_route_validation(lib):
@@ -82,6 +101,11 @@ def test_sparse_attn_validation(lib):
         == bd.SA_ERR_UNSUPPORTED            # unknown dtype
     assert f(FAKE, FAKE + 8, FAKE, 1, sh, FAKE, 2, 0, None, ctypes.byref(none), 0.1, FAKE, None) \
         == bd.SA_ERR_ALIGNMENT
+    zo = _stats(kmean=FAKE, vsum=FAKE)
+    assert f(FAKE, FAKE, FAKE, 1, sh, FAKE, 2, 3, None, ctypes.byref(zo), 0.1, FAKE, None) \
+        == bd.SA_ERR_INVALID_ARG            # first_order without hbar
+    assert f(FAKE, FAKE, FAKE, 1, sh, FAKE, 2, 4, None, ctypes.byref(zo), 0.1, FAKE, None) \
+        == bd.SA_ERR_INVALID_ARG            # unknown tail mode
 
 
 def test_decode_validation_and_workspace(lib):

@@ -26,7 +26,7 @@ def _sample_blocks(H, nqb, n, seed):
     return sorted(picks)
 
 
-@pytest.mark.parametrize("name", ["video_dit", "sla2_mix"])
+@pytest.mark.parametrize("name", ["video_dit", "video_dit_fo", "sla2_mix"])
 def test_prefill_full_size_sampled(lib, name):
     w = wl.WORKLOADS[name]
     inp = wl.prefill_inputs(w, DEV)

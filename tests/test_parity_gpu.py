@@ -40,6 +40,30 @@ def test_block_pool(lib, dtype, d, block, N):
     assert_stats_close(st["vmean_bf16"].float(), ref["vsum"] / block, "vmean_bf16", rtol=1e-2)
 
 
+@pytest.mark.parametrize("dtype,d,block,N", [(torch.float32, 64, 64, 1024), (torch.bfloat16, 128, 128, 4736),
+                                             (torch.bfloat16, 128, 64, 2048), (torch.bfloat16, 64, 128, 1024)])
+def test_block_pool_hbar(lib, dtype, d, block, N):
+    # PISA's H̄; bf16 with d = block = 128 takes the tensor-core path, whose
+    # key deviations k − k̄_j are rounded to bf16 (relative 2^-9) before the MMA
+    Q, K, V = _gauss(2, 3, N, d, dtype, 11)
+    st = bd.block_pool(Q, K, V, block, centroids_bf16=True, first_order=True)
+    ref = oracle.block_pool(np64(Q), np64(K), np64(V), block, first_order=True)
+    tc = dtype == torch.bfloat16 and d == 128 and block == 128
+    assert_stats_close(st["hbar"], ref["hbar"], "hbar", rtol=5e-3 if tc else 1e-4)
+    hT = np.swapaxes(ref["hbar"], -1, -2)
+    assert_stats_close(st["hbarT_bf16"].float(), hT, "hbarT_bf16", rtol=(5e-3 if tc else 0) + 2 ** -8)
+
+
+def test_block_pool_hbar_large_offset(lib):
+    # the deviation form: a large common key offset leaves H̄ unchanged
+    Q, K, V = _gauss(1, 2, 2048, 128, torch.float32, 12)
+    st0 = bd.block_pool(None, K, V, 128, first_order=True)
+    st1 = bd.block_pool(None, (K + 1000.0).contiguous(), V, 128, first_order=True)
+    ref = oracle.block_pool(None, np64(K), np64(V), 128, first_order=True)
+    assert_stats_close(st0["hbar"], ref["hbar"], "hbar", rtol=1e-4)
+    assert_stats_close(st1["hbar"], ref["hbar"], "hbar with offset", rtol=2e-3)
+
+
 def test_block_pool_large_offset_variance(lib):
     # two-pass variance: a large common offset must not destroy the variance
     Q, K, V = _gauss(1, 2, 2048, 128, torch.float32, 2)
@@ -97,7 +121,7 @@ def _prefill_case(Q, K, V, block, k, tail, mode="dot", alpha=None, seed=0, tol=B
     B, H, N, d = Q.shape
     s = 1 / math.sqrt(d)
     st = bd.block_pool(Q, K, V, block, linear=(tail == "linear_mix"),
-                       centroids_bf16=(Q.dtype == torch.bfloat16))
+                       centroids_bf16=(Q.dtype == torch.bfloat16), first_order=(tail == "first_order"))
     idx, sc = bd.route(st, (B, H, N, d, block), mode, k, want_scores=True)
     check_topk_exact(idx, sc, k)
     O = bd.sparse_attn_fwd(Q, K, V, idx, block, tail, st, s, alpha=alpha)
@@ -108,7 +132,7 @@ def _prefill_case(Q, K, V, block, k, tail, mode="dot", alpha=None, seed=0, tol=B
     return assert_tol(np64(O), ref, tol, f"{tail} k={k}")
 
 
-@pytest.mark.parametrize("tail", ["zero_order", "drop", "linear_mix"])
+@pytest.mark.parametrize("tail", ["zero_order", "drop", "linear_mix", "first_order"])
 def test_tiny_fp32(lib, tail):
     w = wl.WORKLOADS["tiny"]
     inp = wl.prefill_inputs(w, DEV)
@@ -116,7 +140,7 @@ def test_tiny_fp32(lib, tail):
     _prefill_case(inp["Q"], inp["K"], inp["V"], w.block, w.k, tail, alpha=alpha, tol=FP32_TOL)
 
 
-@pytest.mark.parametrize("tail", ["zero_order", "drop", "linear_mix"])
+@pytest.mark.parametrize("tail", ["zero_order", "drop", "linear_mix", "first_order"])
 @pytest.mark.parametrize("k", [0, 1, 4, 32])
 def test_video_small_bf16(lib, tail, k):
     w = wl.WORKLOADS["video_dit"]
@@ -125,7 +149,7 @@ def test_video_small_bf16(lib, tail, k):
     _prefill_case(inp["Q"], inp["K"], inp["V"], w.block, k, tail, alpha=alpha)
 
 
-@pytest.mark.parametrize("tail", ["zero_order", "drop", "linear_mix"])
+@pytest.mark.parametrize("tail", ["zero_order", "drop", "linear_mix", "first_order"])
 @pytest.mark.parametrize("dtype,d,block,nb,k", [
     (torch.bfloat16, 128, 128, 37, 5),     # ragged centroid tiles
     (torch.bfloat16, 128, 128, 133, 13),   # more than one 128-centroid tile, ragged
@@ -139,6 +163,31 @@ def test_shapes(lib, tail, dtype, d, block, nb, k):
     alpha = torch.rand(2, d, device=DEV) * 0.7 + 0.2 if tail == "linear_mix" else None
     tol = FP32_TOL if dtype == torch.float32 else BF16_TOL
     _prefill_case(Q, K, V, block, k, tail, alpha=alpha, tol=tol)
+
+
+@pytest.mark.parametrize("dtype,nb,k", [(torch.bfloat16, 37, 5), (torch.bfloat16, 133, 13),
+                                        (torch.float32, 37, 5), (torch.bfloat16, 9, 0)])
+def test_first_order_tail_matters(lib, dtype, nb, k):
+    # values tied to the keys' in-block deviations: the first-order term moves
+    # the output far beyond the tolerance, and the GPU's first-order minus
+    # zero-order difference matches the oracle's
+    block, d = 128, 128
+    inp = wl.block_linear_inputs(1, 2, nb, block, d, dtype, 21 + nb, DEV)
+    Q, K, V = inp["Q"], inp["K"], inp["V"]
+    tol = FP32_TOL if dtype == torch.float32 else BF16_TOL
+    s = 1 / math.sqrt(d)
+    st = bd.block_pool(Q, K, V, block, centroids_bf16=(dtype == torch.bfloat16), first_order=True)
+    idx, _ = bd.route(st, (1, 2, nb * block, d, block), "dot", k)
+    o_fo = bd.sparse_attn_fwd(Q, K, V, idx, block, "first_order", st, s)
+    o_zo = bd.sparse_attn_fwd(Q, K, V, idx, block, "zero_order", st, s)
+    torch.cuda.synchronize()
+    assert_no_device_error()
+    args = (np64(Q), np64(K), np64(V), idx.cpu().numpy(), block)
+    ref_fo = oracle.sparse_attention(*args, "first_order", s)
+    ref_zo = oracle.sparse_attention(*args, "zero_order", s)
+    assert np.abs(ref_fo - ref_zo).mean() > 10 * tol[1]
+    assert_tol(np64(o_fo), ref_fo, tol, "first_order")
+    assert_tol(np64(o_fo) - np64(o_zo), ref_fo - ref_zo, (2 * tol[0], 2 * tol[1]), "first_order - zero_order")
 
 
 def test_empty_problem_is_a_no_op(lib):
