@@ -25,6 +25,11 @@ design notes of the repository):
   the kept indices are returned in ascending order;
 * the SLA2 linear branch uses the ReLU feature map (SALAD), runs over the
   unselected blocks only, and adds eps = 1e-6 to its denominator;
+* PISA's covariance-aware routing: M_j = ‖H_j − H̄‖₂ is the spectral norm,
+  and the score adds the first-order error bound to the zero-order mass of the
+  block, s q̄.k̄_j + log1p(s ‖q̄_i‖ M_j / B) (the page says the score
+  "incorporates" both without a formula; this is the plainest combination the
+  error argument gives);
 * GQA decode shares one selection per (batch, KV head); the group's score for
   a block is the log of the sum over the group's query heads of each head's
   SPLA block mass (a logsumexp of the log-form scores).
@@ -37,6 +42,11 @@ Pins (the tests under ``tests/test_oracle_*.py``):
                       per-block deviations -> PISA's per-block first-order
                       Taylor sum by brute force; error O(ε²) vs zero_order's
                       O(ε) as the in-block deviations shrink
+  covnorm / "cov"     rank-one deviations H_j − H̄ = (γ_j − γ̄) u wᵀ -> closed
+                      form |γ_j − γ̄|·|u|·|w|; identical blocks -> M_j = 0 and
+                      "cov" = s·"dot"; the square root of the largest
+                      eigenvalue of AᵀA (a symmetric eigen-solver, not the
+                      SVD); brute-force score loops
   sparse_attention    k = nb -> dense softmax attention (torch SDPA, fp64);
                       block size 1 / block-constant keys -> dense; V+c -> O+c;
                       hand-derived worked example (tests/golden); brute force
@@ -68,7 +78,8 @@ def _f64(x) -> np.ndarray:
 # ---------------------------------------------------------------------------
 
 def block_pool(Q, K, V, block: int, *, variance: bool = False,
-               linear: bool = False, first_order: bool = False) -> dict:
+               linear: bool = False, first_order: bool = False,
+               covariance: bool = False) -> dict:
     """Per-block statistics of Q, K and V, all float64.
 
     Follows PISA "Implementação de Hardware", step "Pré-computação"
@@ -89,7 +100,11 @@ def block_pool(Q, K, V, block: int, *, variance: bool = False,
                          (only with ``linear``)
       hbar  [B,H,d,d]    PISA's global first-order statistic H̄: the mean over
                          the head's blocks of H_j = Σ_{n∈j} (k_n − k̄_j) v_nᵀ
-                         (only with ``first_order``)
+                         (only with ``first_order`` or ``covariance``)
+      covnorm [B,H,nb]   M_j = ‖H_j − H̄‖₂, the spectral norm (largest singular
+                         value) of each block's first-order deviation from the
+                         mean, PISA "Roteamento Consciente de Covariância"
+                         (only with ``covariance``)
     """
     K = _f64(K)
     V = _f64(V)
@@ -117,11 +132,14 @@ def block_pool(Q, K, V, block: int, *, variance: bool = False,
         out["ztot"] = out["zrelu"].sum(axis=2)
         Rt = np.maximum(K, 0.0)
         out["htot"] = np.einsum("bhnc,bhne->bhce", Rt, V)
-    if first_order:
+    if first_order or covariance:
         # H_j = Σ_n (k_n − k̄_j) v_nᵀ for every block, then their mean
         dev = Kb - kmean[:, :, :, None, :]
         Hj = np.einsum("bhjnc,bhjne->bhjce", dev, Vb)
         out["hbar"] = Hj.mean(axis=2)
+        if covariance:
+            # largest singular value of each d×d deviation matrix (LAPACK SVD)
+            out["covnorm"] = np.linalg.norm(Hj - out["hbar"][:, :, None], ord=2, axis=(-2, -1))
     return out
 
 
@@ -130,7 +148,8 @@ def block_pool(Q, K, V, block: int, *, variance: bool = False,
 # ---------------------------------------------------------------------------
 
 def route_scores(qmean, kmean, mode: str, *, proj_q=None, proj_k=None,
-                 kvar=None, scale: Optional[float] = None) -> np.ndarray:
+                 kvar=None, scale: Optional[float] = None, covnorm=None,
+                 block: Optional[int] = None) -> np.ndarray:
     """Block scores [B,H,nqb,nb] of the router.
 
     mode "dot":     q̄_i . k̄_j on mean-pooled blocks (SLA2 §2B, pooling of
@@ -140,6 +159,14 @@ def route_scores(qmean, kmean, mode: str, *, proj_q=None, proj_k=None,
     mode "taylor2": SPLA §2.1 score exp(q.k̄)(1 + ½ qᵀ diag(Var k) q) with the
                     scale folded into q (q' = s q̄_i), in log form
                     s q̄.k̄ + log1p(½ s² Σ_c q̄_c² var_c).
+    mode "cov":     PISA's covariance-aware score (§2 "Roteamento Consciente
+                    de Covariância"): the block's zero-order mass B e^{s q̄.k̄_j}
+                    plus the bound e^{s q̄.k̄_j} s‖q̄‖ M_j on the norm of the
+                    first-order term the hybrid order leaves out for it
+                    (‖α s qᵀ(H_j − H̄)‖ ≤ α s ‖q‖ M_j), in log form without
+                    the constant log B:
+                    s q̄.k̄_j + log1p(s ‖q̄_i‖ M_j / B).
+                    Needs covnorm (M_j), block (B) and scale.
     """
     qm = _f64(qmean)
     km = _f64(kmean)
@@ -156,6 +183,14 @@ def route_scores(qmean, kmean, mode: str, *, proj_q=None, proj_k=None,
         lin = s * np.einsum("bhic,bhjc->bhij", qm, km)
         quad = 0.5 * s * s * np.einsum("bhic,bhjc->bhij", qm * qm, _f64(kvar))
         return lin + np.log1p(quad)
+    if mode == "cov":
+        if covnorm is None or scale is None or block is None:
+            raise ValueError("cov needs covnorm, scale and block")
+        s = float(scale)
+        lin = s * np.einsum("bhic,bhjc->bhij", qm, km)
+        qn = np.sqrt((qm * qm).sum(axis=-1))                       # [B,H,nqb]
+        bound = s * qn[..., :, None] * _f64(covnorm)[..., None, :] / float(block)
+        return lin + np.log1p(bound)
     raise ValueError(f"unknown route mode {mode!r}")
 
 
