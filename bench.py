@@ -323,12 +323,13 @@ def time_fp8(steps: int = 10, warmup: int = 3):
     return out
 
 
-def time_first_order(steps: int = 10, warmup: int = 3):
-    """PISA's hybrid-order tail on the video_dit inputs (same seed): the step
-    (block_pool with H̄ + route + attention) and the attention launch alone."""
+def time_pisa(steps: int = 10, warmup: int = 3):
+    """PISA's full method on the video_dit inputs (same seed): covariance-aware
+    routing and the hybrid-order tail; the step (block_pool with H̄ and M_j +
+    route + attention) and the attention launch alone."""
     from block_sparse_approximate_b200 import binding as bd
     from block_sparse_approximate_b200.pipeline import PrefillStep
-    w = wl.WORKLOADS["video_dit_fo"]
+    w = wl.WORKLOADS["video_dit_pisa"]
     inp = wl.prefill_inputs(w, "cuda")
     step = PrefillStep(w, inp)
     step()
@@ -341,7 +342,7 @@ def time_first_order(steps: int = 10, warmup: int = 3):
     out = {"workload": w.name, "ms_per_step": ms_step, "attn_ms": attn_ms, "executed_tflops": ach,
            "dense_equiv_tflops": dense_flops(w) / (ms_step * 1e-3) / 1e12,
            "peak_tflops": bf16, "frac": ach / bf16, "peak_source": f"{src} bf16 burst",
-           "step": "block_pool (+ H̄ on the tensor cores) + route + sparse_attn_fwd (first_order)"}
+           "step": "block_pool (+ H̄ and M_j on the tensor cores) + route (cov) + sparse_attn_fwd (first_order)"}
     del inp, step
     torch.cuda.empty_cache()
     return out
@@ -401,9 +402,9 @@ def run_ours(args, world, rank, local):
         if rank == 0:
             print(json.dumps({"sla2_mix": time_sla2(args.steps, args.warmup)}), flush=True)
         return 0
-    if args.only == "fo":
+    if args.only == "pisa":
         if rank == 0:
-            print(json.dumps({"first_order": time_first_order(args.steps, args.warmup)}), flush=True)
+            print(json.dumps({"pisa": time_pisa(args.steps, args.warmup)}), flush=True)
         return 0
     w = wl.WORKLOADS[WORKLOAD]
     wr = rank_workload(w, rank)
@@ -493,14 +494,14 @@ def run_ours(args, world, rank, local):
                "h2d_bytes_per_step": sum(inp[n].numel() * inp[n].element_size() for n in ("Q", "K", "V")),
                "d2h_bytes_per_step": step.buf.out.numel() * step.buf.out.element_size()}
 
-    decode = fp8 = sla2 = first_order = None
+    decode = fp8 = sla2 = pisa = None
     if rank == 0 and args.only == "all" and not args.no_decode:
         del step
         torch.cuda.empty_cache()
         decode = time_decode(batch=args.decode_batch)
         fp8 = time_fp8()
         sla2 = time_sla2()
-        first_order = time_first_order()
+        pisa = time_pisa()
     ck = clocks.stop() if clocks else None
 
     if rank != 0:
@@ -534,7 +535,7 @@ def run_ours(args, world, rank, local):
         "decode": decode,
         "fp8": fp8,
         "sla2_mix": sla2,
-        "first_order": first_order,
+        "pisa": pisa,
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -553,9 +554,9 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
-    ap.add_argument("--only", choices=["all", "prefill", "decode", "fp8", "sla2", "fo"], default="all",
-                    help="prefill: the timed step only; decode / fp8 / sla2 / fo (first-order tail): "
-                         "only that workload's timing")
+    ap.add_argument("--only", choices=["all", "prefill", "decode", "fp8", "sla2", "pisa"], default="all",
+                    help="prefill: the timed step only; decode / fp8 / sla2 / pisa (covariance routing + "
+                         "first-order tail): only that workload's timing")
     ap.add_argument("--decode-batch", type=int, default=None,
                     help="sequences in the decode workload (default: the full 16)")
     args = ap.parse_args(argv)

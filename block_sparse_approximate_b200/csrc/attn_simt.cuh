@@ -25,9 +25,24 @@ bool attn_tc_supports(sa_dtype dtype, const sa_shape& s, sa_tail_mode tail);
 // added into `out`, which the caller zeroes first:
 //   kmean == NULL: H_tot = Σ_n relu(k_n) v_nᵀ (oscale 1);
 //   kmean != NULL: oscale · Σ_j Σ_{n∈j} (k_n − k̄_j) v_nᵀ over 128-token blocks
-//                  with centroids kmean [B,H,N/128,d] (H̄ with oscale = 1/nb).
+//                  with centroids kmean and value sums vsum [B,H,N/128,d]
+//                  (H̄ with oscale = 1/nb).
 // Returns SA_ERR_UNSUPPORTED (without setting an error) for other shapes.
-sa_status kv_outer_tc(const void* K, const void* V, const sa_shape& s, const float* kmean, float oscale,
-                      float* out, cudaStream_t stream);
+sa_status kv_outer_tc(const void* K, const void* V, const sa_shape& s, const float* kmean, const float* vsum,
+                      float oscale, float* out, cudaStream_t stream);
+
+// PISA's block covariance norms M_j = ‖H_j − H̄‖₂ on the tensor cores (bf16,
+// d = block = 128): covnorm [B,H,nb] from K, V and the statistics kmean,
+// vsum [B,H,nb,d] and hbar [B,H,d,d].  Returns SA_ERR_UNSUPPORTED (without
+// setting an error) for other shapes.
+sa_status covnorm_tc(const void* K, const void* V, const sa_shape& s, const float* kmean, const float* vsum,
+                     const float* hbar, float* covnorm, cudaStream_t stream);
+
+// Tensor maps and device error words shared by the tensor-core translation
+// units: a 3-D [outer][rows][cols] map with a {128 bytes, 128 rows, 1} box
+// and 128-byte swizzle (elem = 2 for bf16, 1 for e4m3), and the read-and-clear
+// of the covariance kernel's bounded-wait error word.
+bool make_tmap_128x128(void* map, const void* base, int elem, uint64_t cols, uint64_t rows, uint64_t outer);
+uint32_t covnorm_error_take();
 
 }  // namespace sa

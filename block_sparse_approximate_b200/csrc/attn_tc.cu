@@ -1020,13 +1020,18 @@ attn_tc_linmix_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
 //                  SALAD §2);
 //   kmean != NULL: f(k_n) = k_n − k̄_j with k̄_j the centroid of the 128-token
 //                  block that holds n, each chunk's sum scaled by oscale
-//                  (1/nb): PISA's mean first-order statistic H̄ (§2).
-// A CTA takes a chunk of 128-token tiles of one head, warps 2-5 apply f in
-// place to each K tile, warp 1 accumulates f(K)ᵀ V in TMEM (MN-major ×
-// MN-major MMA), and the chunk's d×d sum is added to `out` with vector
-// atomics.  Warp 0 is the TMA producer.
+//                  (1/nb): PISA's mean first-order statistic H̄ (§2).  The
+//                  MMAs accumulate the raw Kᵀ V of the chunk (bf16 products
+//                  are exact in fp32) and the epilogue subtracts
+//                  Σ_j k̄_j vsum_jᵀ over the chunk's blocks in fp32, which
+//                  equals Σ_j Σ_n (k_n − k̄_j) v_nᵀ without rounding the
+//                  deviations to bf16.
+// A CTA takes a chunk of 128-token tiles of one head, warps 2-5 apply the
+// ReLU in place to each K tile (H_tot only), warp 1 accumulates f(K)ᵀ V in
+// TMEM (MN-major × MN-major MMA), and the chunk's d×d sum is added to `out`
+// with vector atomics.  Warp 0 is the TMA producer.
 constexpr int kHtThreads = 192;
-constexpr int kHtTiles = 32;          // tiles (of 128 tokens) per CTA
+constexpr int kHtMinTiles = 4;        // fewest tiles (of 128 tokens) per CTA
 struct HtLayout {
   static constexpr int NS = 3;
   static constexpr uint32_t kTile = 2 * kSpan;
@@ -1039,7 +1044,8 @@ struct HtLayout {
 
 __global__ void __launch_bounds__(kHtThreads, 1)
 htot_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, int N,
-               const float* __restrict__ kmean, float oscale, float* __restrict__ htot) {
+               int tiles_per_cta, const float* __restrict__ kmean, const float* __restrict__ vsum, float oscale,
+               float* __restrict__ htot) {
   using L = HtLayout;
   constexpr int NS = L::NS;
   constexpr uint32_t kTile = L::kTile;
@@ -1052,8 +1058,8 @@ htot_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kSlotOff + 4);
   auto bar = [&](int k) { return sb + L::kBarOff + 8u * k; };
   const int ntile_head = N / TB;
-  const int t0 = chunk * kHtTiles;
-  const int T = min(kHtTiles, ntile_head - t0);
+  const int t0 = chunk * tiles_per_cta;
+  const int T = min(tiles_per_cta, ntile_head - t0);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
@@ -1113,12 +1119,9 @@ htot_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
       wait_bounded(bar(L::B_DONE), 0);
     }
   } else {
-    // warps 2-5: f of each K tile, then the epilogue (TMEM lane quarter w % 4)
+    // warps 2-5: ReLU of each K tile (H_tot), then the epilogue (TMEM lane
+    // quarter w % 4)
     const int tr = threadIdx.x - 64;
-    // 128-byte swizzle: the 16-byte vectors tr + 128 m of a tile all sit in
-    // row ≡ tr / 8 (mod 8) at physical chunk tr % 8, i.e. channels
-    // 64 (m / 8) + 8 ((tr % 8) ^ (tr / 8 % 8)) + [0, 8)
-    const int chunk8 = 8 * ((tr & 7) ^ ((tr >> 3) & 7));
     bool ok = true;
     for (int t = 0; t < T; ++t) {
       const int s = t % NS;
@@ -1126,29 +1129,8 @@ htot_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
         ok = false;
         break;
       }
-      uint4* kt = reinterpret_cast<uint4*>(smem + 2 * kTile * s);
-      if (kmean) {
-        const float* cen = kmean + ((size_t)bh * ntile_head + t0 + t) * TD + chunk8;
-        float c8[2][8];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const float4 a = *reinterpret_cast<const float4*>(cen + 64 * h);
-          const float4 b = *reinterpret_cast<const float4*>(cen + 64 * h + 4);
-          c8[h][0] = a.x; c8[h][1] = a.y; c8[h][2] = a.z; c8[h][3] = a.w;
-          c8[h][4] = b.x; c8[h][5] = b.y; c8[h][6] = b.z; c8[h][7] = b.w;
-        }
-#pragma unroll
-        for (int m = 0; m < (int)(kTile / 16) / 128; ++m) {
-          uint4 u = kt[tr + 128 * m];
-          __nv_bfloat162* hh = reinterpret_cast<__nv_bfloat162*>(&u);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 f = __bfloat1622float2(hh[e]);
-            hh[e] = __floats2bfloat162_rn(f.x - c8[m >> 3][2 * e], f.y - c8[m >> 3][2 * e + 1]);
-          }
-          kt[tr + 128 * m] = u;
-        }
-      } else {
+      if (!kmean) {
+        uint4* kt = reinterpret_cast<uint4*>(smem + 2 * kTile * s);
         const __nv_bfloat162 zero = __float2bfloat162_rn(0.f);
 #pragma unroll 4
         for (int x = tr; x < (int)(kTile / 16); x += 128) {
@@ -1174,6 +1156,23 @@ htot_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
         uint32_t a[32];
         tmem_ld32(lrow + 32 * cc, a);
         tmem_wait_ld();
+        if (kmean) {
+          // − Σ_j k̄_j[c] vsum_j[e] over the chunk's blocks
+          float* f = reinterpret_cast<float*>(a);
+          for (int t = 0; t < T; ++t) {
+            const size_t blk = (size_t)bh * ntile_head + t0 + t;
+            const float kc = kmean[blk * TD + c];
+            const float4* vs4 = reinterpret_cast<const float4*>(vsum + blk * TD + 32 * cc);
+#pragma unroll
+            for (int q4 = 0; q4 < 8; ++q4) {
+              const float4 v = vs4[q4];
+              f[4 * q4] = fmaf(-kc, v.x, f[4 * q4]);
+              f[4 * q4 + 1] = fmaf(-kc, v.y, f[4 * q4 + 1]);
+              f[4 * q4 + 2] = fmaf(-kc, v.z, f[4 * q4 + 2]);
+              f[4 * q4 + 3] = fmaf(-kc, v.w, f[4 * q4 + 3]);
+            }
+          }
+        }
 #pragma unroll
         for (int q4 = 0; q4 < 8; ++q4)
           atomicAdd(hrow + 8 * cc + q4,
@@ -1193,8 +1192,12 @@ htot_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
 
 }  // namespace
 
-sa_status kv_outer_tc(const void* K, const void* V, const sa_shape& s, const float* kmean, float oscale,
-                      float* out, cudaStream_t stream) {
+bool make_tmap_128x128(void* map, const void* base, int elem, uint64_t cols, uint64_t rows, uint64_t outer) {
+  return make_tmap_3d(static_cast<CUtensorMap*>(map), base, elem, cols, rows, outer);
+}
+
+sa_status kv_outer_tc(const void* K, const void* V, const sa_shape& s, const float* kmean, const float* vsum,
+                      float oscale, float* out, cudaStream_t stream) {
   if (s.d != TD || (s.N % TB) || (kmean && s.block != TB)) return SA_ERR_UNSUPPORTED;
   const uint64_t BH = (uint64_t)s.B * s.H;
   CUtensorMap mk, mv;
@@ -1204,8 +1207,28 @@ sa_status kv_outer_tc(const void* K, const void* V, const sa_shape& s, const flo
   if (cudaFuncSetAttribute(htot_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return launch_status("cudaFuncSetAttribute(htot_tc_kernel)");
   const int nt = s.N / TB;
-  dim3 grid((nt + kHtTiles - 1) / kHtTiles, (unsigned)BH);
-  htot_tc_kernel<<<grid, kHtThreads, smem, stream>>>(mk, mv, s.N, kmean, oscale, out);
+  // tiles per CTA: one CTA per SM (three 64 KB stages), so a wave of CTAs of
+  // c tiles takes about c + 2 tile-times (ring fill, the d×d atomic flush);
+  // pick the c with the fewest tile-times over all waves, at least
+  // kHtMinTiles
+  int sms = 148;
+  {
+    int dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  }
+  int tpc = kHtMinTiles;
+  long best = -1;
+  for (int c = kHtMinTiles; c <= std::max(kHtMinTiles, nt); ++c) {
+    const long ctas = (long)((nt + c - 1) / c) * (long)BH;
+    const long cost = ((ctas + sms - 1) / sms) * (long)(c + 2);
+    if (best < 0 || cost < best) {
+      best = cost;
+      tpc = c;
+    }
+    if (ctas <= sms) break;   // one wave: more tiles per CTA only add time
+  }
+  dim3 grid((nt + tpc - 1) / tpc, (unsigned)BH);
+  htot_tc_kernel<<<grid, kHtThreads, smem, stream>>>(mk, mv, s.N, tpc, kmean, vsum, oscale, out);
   return launch_status("htot_tc_kernel");
 }
 
@@ -1300,6 +1323,6 @@ extern "C" sa_status sa_device_error(uint32_t* code) {
   if (cudaMemcpyFromSymbol(&v, tc::g_device_error, sizeof(v)) != cudaSuccess ||
       cudaMemcpyToSymbol(tc::g_device_error, &zero, sizeof(zero)) != cudaSuccess)
     return launch_status("sa_device_error");
-  *code = v | decode_error_take();
+  *code = v | decode_error_take() | covnorm_error_take();
   return SA_OK;
 }

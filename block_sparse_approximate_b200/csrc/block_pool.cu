@@ -157,7 +157,7 @@ __global__ void __launch_bounds__(256)
 linear_totals_kernel(const T* __restrict__ K, const T* __restrict__ V, int H, int N,
                      float* __restrict__ htot, float* __restrict__ ztot,
                      const float* __restrict__ kmean = nullptr, float oscale = 1.f) {
-  static_assert(BLKDEV == 0 || kLinChunk % BLKDEV == 0, "a chunk holds whole blocks");
+  static_assert(kLinChunk % (BLKDEV ? BLKDEV : 1) == 0, "a chunk holds whole blocks");
   constexpr int kDevBlk = BLKDEV ? BLKDEV : 1;
   constexpr int TPR = 256 / D;       // threads per output row
   constexpr int CPT = D / TPR;       // columns per thread
@@ -225,6 +225,106 @@ __global__ void ztot_from_blocks_kernel(const float* __restrict__ zrelu, int H, 
   ztot[((size_t)b * H + h) * D + c] = acc;
 }
 
+// M_j = ‖H_j − H̄‖₂ of one block per CTA on CUDA cores (every shape; the
+// tensor-core kernel in cov_tc.cu takes bf16 with d = block = 128): the CTA
+// accumulates A = Σ_n (k_n − k̄_j) v_nᵀ − H̄ in shared memory (thread t owns
+// row t / (256/D) and D·D/256 of its columns), then runs the power iteration
+// x ← Aᵀ A x / ‖Aᵀ A x‖ until the Rayleigh quotient ‖A x‖² / ‖x‖² changes by
+// less than 1e-6 (relative) or 256 steps have run; M_j is its square root.
+constexpr int kCovSteps = 256;
+
+template <typename T, int D, int BLK>
+__global__ void __launch_bounds__(256)
+covnorm_simt_kernel(const T* __restrict__ K, const T* __restrict__ V, int H, int N,
+                    const float* __restrict__ kmean, const float* __restrict__ hbar, float* __restrict__ covnorm) {
+  constexpr int TPR = 256 / D;       // threads per row
+  constexpr int CPT = D / TPR;       // columns per thread
+  constexpr int AS = D + 1;          // padded row of A
+  const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int nb = N / BLK;
+  const size_t bh = (size_t)b * H + h;
+  const size_t head_off = bh * (size_t)N * D;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int c = tid / TPR, e0 = (tid % TPR) * CPT;
+  extern __shared__ float cs[];
+  float* A = cs;                          // [D][AS]
+  float* ks = A + D * AS;                 // [kLinTile][D]
+  float* vs = ks + kLinTile * D;          // [kLinTile][D]
+  float* x = vs + kLinTile * D;           // [D]
+  float* y = x + D;                       // [D]
+  float* red = y + D;                     // [2][8 warps][3]
+
+  const float* km = kmean + (bh * nb + j) * D;
+  float acc[CPT];
+#pragma unroll
+  for (int i = 0; i < CPT; ++i) acc[i] = 0.f;
+  for (int n0 = 0; n0 < BLK; n0 += kLinTile) {
+    __syncthreads();
+    for (int idx = tid; idx < kLinTile * D; idx += 256) {
+      const int r = idx / D, cc = idx % D;
+      const size_t g = head_off + ((size_t)j * BLK + n0 + r) * D + cc;
+      ks[idx] = to_f<T>(K[g]) - km[cc];
+      vs[idx] = to_f<T>(V[g]);
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int r = 0; r < kLinTile; ++r) {
+      const float kr = ks[r * D + c];
+#pragma unroll
+      for (int i = 0; i < CPT; ++i) acc[i] = fmaf(kr, vs[r * D + e0 + i], acc[i]);
+    }
+  }
+  const float* hb = hbar + (bh * D + c) * D;
+#pragma unroll
+  for (int i = 0; i < CPT; ++i) A[c * AS + e0 + i] = acc[i] - hb[e0 + i];
+  for (int i = tid; i < D; i += 256) x[i] = 0.5f + (float)((((uint32_t)i * 2654435761u) >> 24) & 0xffu) * (1.0f / 256.0f);
+  __syncthreads();
+
+  float lam = 0.f, lam_prev = -1.f;
+  for (int it = 0; it < kCovSteps; ++it) {
+    // y = A x (rows split over TPR adjacent lanes), with ‖y‖² and ‖x‖²
+    float py = 0.f;
+#pragma unroll
+    for (int i = 0; i < CPT; ++i) py = fmaf(A[c * AS + e0 + i], x[e0 + i], py);
+#pragma unroll
+    for (int o = TPR / 2; o > 0; o >>= 1) py += __shfl_xor_sync(0xffffffffu, py, o);
+    if (e0 == 0) y[c] = py;
+    float p1 = (e0 == 0) ? py * py : 0.f;
+    float p3 = (tid < D) ? x[tid] * x[tid] : 0.f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      p1 += __shfl_xor_sync(0xffffffffu, p1, o);
+      p3 += __shfl_xor_sync(0xffffffffu, p3, o);
+    }
+    const int rb = (it & 1) * 16;
+    if (lane == 0) {
+      red[rb + 2 * warp] = p1;
+      red[rb + 2 * warp + 1] = p3;
+    }
+    __syncthreads();
+    float S1 = 0.f, S3 = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      S1 += red[rb + 2 * w];
+      S3 += red[rb + 2 * w + 1];
+    }
+    lam = S3 > 0.f ? S1 / S3 : 0.f;
+    if (!(S1 > 0.f) || fabsf(lam - lam_prev) <= 1e-6f * lam) break;
+    lam_prev = lam;
+    // x = Aᵀ y / ‖Aᵀ y‖ scaled only by ‖y‖ (the quotient ignores the scale):
+    // column e of A over its D rows, thread t covering columns t, t + 256 ...
+    const float inv = rsqrtf(S1);
+    float z = 0.f;
+    if (tid < D) {
+      for (int r = 0; r < D; ++r) z = fmaf(A[r * AS + tid], y[r], z);
+    }
+    __syncthreads();
+    if (tid < D) x[tid] = z * inv;
+    __syncthreads();
+  }
+  if (tid == 0) covnorm[bh * nb + j] = sqrtf(fmaxf(lam, 0.f));
+}
+
 template <typename T, int D, int BLK>
 sa_status launch_pool(const void* Q, const void* K, const void* V, const sa_shape& s,
                       const sa_block_stats& st, cudaStream_t stream) {
@@ -241,7 +341,7 @@ sa_status launch_pool(const void* Q, const void* K, const void* V, const sa_shap
       return launch_status("cudaMemsetAsync(htot/ztot)");
     // bf16, d = 128: H_tot on the tensor cores and z_tot from the block sums
     if (sizeof(T) == 2 && D == 128 && st.zrelu &&
-        kv_outer_tc(K, V, s, nullptr, 1.f, st.htot, stream) == SA_OK) {
+        kv_outer_tc(K, V, s, nullptr, nullptr, 1.f, st.htot, stream) == SA_OK) {
       ztot_from_blocks_kernel<D><<<dim3(s.H, s.B), D, 0, stream>>>(st.zrelu, s.H, s.N / BLK, st.ztot);
       return launch_status("ztot_from_blocks_kernel");
     }
@@ -257,7 +357,7 @@ sa_status launch_pool(const void* Q, const void* K, const void* V, const sa_shap
     if (cudaMemsetAsync(st.hbar, 0, hbytes, stream) != cudaSuccess) return launch_status("cudaMemsetAsync(hbar)");
     const float inv_nb = 1.0f / (float)(s.N / BLK);
     if (!(sizeof(T) == 2 && D == 128 && BLK == 128 &&
-          kv_outer_tc(K, V, s, st.kmean, inv_nb, st.hbar, stream) == SA_OK)) {
+          kv_outer_tc(K, V, s, st.kmean, st.vsum, inv_nb, st.hbar, stream) == SA_OK)) {
       dim3 g2((s.N + kLinChunk - 1) / kLinChunk, s.H, s.B);
       linear_totals_kernel<T, D, BLK><<<g2, 256, 0, stream>>>(
           static_cast<const T*>(K), static_cast<const T*>(V), s.H, s.N, st.hbar, nullptr, st.kmean, inv_nb);
@@ -268,6 +368,20 @@ sa_status launch_pool(const void* Q, const void* K, const void* V, const sa_shap
       hbar_transpose_kernel<D><<<dim3(D / 32, D / 32, s.B * s.H), dim3(32, 8), 0, stream>>>(
           st.hbar, reinterpret_cast<__nv_bfloat16*>(st.hbarT_bf16));
       r = launch_status("hbar_transpose_kernel");
+      if (r != SA_OK) return r;
+    }
+    if (st.covnorm) {
+      // PISA's M_j from the H̄ just written (same stream)
+      if (sizeof(T) == 2 && D == 128 && BLK == 128 &&
+          covnorm_tc(K, V, s, st.kmean, st.vsum, st.hbar, st.covnorm, stream) == SA_OK)
+        return SA_OK;
+      const size_t smem = sizeof(float) * ((size_t)D * (D + 1) + 2 * (size_t)kLinTile * D + 2 * D + 32);
+      auto kern = covnorm_simt_kernel<T, D, BLK>;
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return launch_status("cudaFuncSetAttribute(covnorm_simt_kernel)");
+      kern<<<dim3(s.N / BLK, s.H, s.B), 256, smem, stream>>>(
+          static_cast<const T*>(K), static_cast<const T*>(V), s.H, s.N, st.kmean, st.hbar, st.covnorm);
+      r = launch_status("covnorm_simt_kernel");
     }
   }
   return r;
@@ -296,11 +410,11 @@ extern "C" sa_status sa_block_pool(const void* Q, const void* K, const void* V, 
     return fail(SA_ERR_INVALID_ARG, "sa_block_pool: K, V, stats, stats->kmean and stats->vsum are required");
   if ((stats->htot == nullptr) != (stats->ztot == nullptr))
     return fail(SA_ERR_INVALID_ARG, "sa_block_pool: htot and ztot go together");
-  if (stats->hbarT_bf16 && !stats->hbar)
-    return fail(SA_ERR_INVALID_ARG, "sa_block_pool: hbarT_bf16 needs hbar");
+  if ((stats->hbarT_bf16 || stats->covnorm) && !stats->hbar)
+    return fail(SA_ERR_INVALID_ARG, "sa_block_pool: hbarT_bf16 and covnorm need hbar");
   const void* ptrs[] = {Q, K, V, stats->qmean, stats->kmean, stats->vsum, stats->kvar,
                         stats->zrelu, stats->htot, stats->ztot, stats->kmean_bf16, stats->vmean_bf16,
-                        stats->hbar, stats->hbarT_bf16};
+                        stats->hbar, stats->hbarT_bf16, stats->covnorm};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return fail(SA_ERR_ALIGNMENT, "sa_block_pool: pointers must be 16-byte aligned");
   cudaStream_t s = as_stream(stream);

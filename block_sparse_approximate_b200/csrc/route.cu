@@ -3,6 +3,9 @@
 //   proj     (q̄_i P_q)·(k̄_j P_k)              (SLA2 §2B, learnable router)
 //   taylor2  s q̄_i·k̄_j + log1p(½ s² Σ q̄²var)  (SPLA §2.1, log of the
 //            second-order block score with diagonal covariance)
+//   cov      s q̄_i·k̄_j + log1p(s ‖q̄_i‖ M_j / B) (PISA §2, covariance-aware
+//            routing: zero-order mass plus the first-order error bound,
+//            M_j = ‖H_j − H̄‖₂ from block_pool)
 // The proj score (q̄_i P_q)·(k̄_j P_k) is evaluated as k̄_j·u_i with
 // u_i = P_k P_qᵀ q̄_i (x P is the row vector x times P), so no projected copy
 // of the key centroids is needed: u_i costs 2d² multiply-adds per query block.
@@ -82,7 +85,7 @@ __device__ __forceinline__ void tile_dots(const float* A, const float* T, int la
 template <int D, int RPW, int NCOL>
 __global__ void __launch_bounds__(kRouteThreads)
 route_kernel(sa_block_stats st, int H, int nb, sa_route_mode mode, const float* __restrict__ Pq,
-             const float* __restrict__ Pk, float scale, int topk, int32_t* __restrict__ block_idx,
+             const float* __restrict__ Pk, float scale, float inv_blk, int topk, int32_t* __restrict__ block_idx,
              float* __restrict__ scores_out) {
   constexpr int QB = kRouteWarps * RPW;          // query blocks per CTA
   constexpr int TJ = 32 * NCOL;                  // centroids per tile
@@ -92,6 +95,7 @@ route_kernel(sa_block_stats st, int H, int nb, sa_route_mode mode, const float* 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const size_t bh = (size_t)b * H + h;
   const bool t2 = mode == SA_ROUTE_TAYLOR2;
+  const bool cov = mode == SA_ROUTE_COV;
   const int narr = t2 ? 2 : 1;                   // staged arrays per tile
 
   extern __shared__ __align__(16) float rsm[];
@@ -114,7 +118,7 @@ route_kernel(sa_block_stats st, int H, int nb, sa_route_mode mode, const float* 
     const int r = x / D, c = x % D;
     const int i = i0 + r;
     const float q = i < nb ? st.qmean[(bh * nb + i) * D + c] : 0.f;
-    u[x] = t2 ? scale * q : q;
+    u[x] = (t2 || cov) ? scale * q : q;
     w[x] = 0.5f * scale * scale * q * q;
   }
   __syncthreads();
@@ -163,6 +167,23 @@ route_kernel(sa_block_stats st, int H, int nb, sa_route_mode mode, const float* 
     __syncthreads();
   }
 
+  // cov: ‖s q̄_r‖ / B of the warp's rows (every lane holds them)
+  float qnb[RPW];
+#pragma unroll
+  for (int r = 0; r < RPW; ++r) {
+    float ss = 0.f;
+    if (cov) {
+      for (int c = lane; c < D; c += 32) {
+        const float v = u[(warp * RPW + r) * D + c];
+        ss = fmaf(v, v, ss);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    }
+    qnb[r] = sqrtf(ss) * inv_blk;
+  }
+  const float* cvn = cov ? st.covnorm + bh * (size_t)nb : nullptr;
+
   // ---- scores: tiles of TJ centroids, two buffers
   const float* km = st.kmean + bh * (size_t)nb * D;
   const float* kv = t2 ? st.kvar + bh * (size_t)nb * D : nullptr;
@@ -192,6 +213,15 @@ route_kernel(sa_block_stats st, int H, int nb, sa_route_mode mode, const float* 
       for (int r = 0; r < RPW; ++r)
 #pragma unroll
         for (int n = 0; n < NCOL; ++n) o[r][n] += log1pf(o2[r][n]);
+    }
+    if (cov) {
+#pragma unroll
+      for (int n = 0; n < NCOL; ++n) {
+        const int j = t * TJ + lane + 32 * n;
+        const float m = j < nb ? cvn[j] : 0.f;
+#pragma unroll
+        for (int r = 0; r < RPW; ++r) o[r][n] += log1pf(qnb[r] * m);
+      }
     }
 #pragma unroll
     for (int r = 0; r < RPW; ++r)
@@ -348,14 +378,14 @@ RouteCfg route_cfg(int nb, int d, int topk, bool t2) {
 
 template <int D, int RPW, int NCOL>
 sa_status launch_route(const sa_block_stats& st, sa_shape shape, int nb, sa_route_mode mode, const float* Pq,
-                       const float* Pk, float scale, int topk, int32_t* idx, float* scores, size_t smem,
-                       cudaStream_t s) {
+                       const float* Pk, float scale, float inv_blk, int topk, int32_t* idx, float* scores,
+                       size_t smem, cudaStream_t s) {
   auto kern = route_kernel<D, RPW, NCOL>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return launch_status("cudaFuncSetAttribute(route_kernel)");
   constexpr int QB = kRouteWarps * RPW;
   dim3 grid((nb + QB - 1) / QB, shape.H, shape.B);
-  kern<<<grid, kRouteThreads, smem, s>>>(st, shape.H, nb, mode, Pq, Pk, scale, topk, idx, scores);
+  kern<<<grid, kRouteThreads, smem, s>>>(st, shape.H, nb, mode, Pq, Pk, scale, inv_blk, topk, idx, scores);
   return launch_status("route_kernel");
 }
 
@@ -372,15 +402,17 @@ extern "C" sa_status sa_route(const sa_block_stats* stats, sa_shape shape, sa_ro
   if (shape.N == 0 || shape.B == 0 || shape.H == 0) return SA_OK;  // nothing to compute
   if (!stats || !stats->qmean || !stats->kmean || (topk > 0 && !block_idx))
     return fail(SA_ERR_INVALID_ARG, "sa_route: stats->qmean, stats->kmean and block_idx are required");
-  if (mode != SA_ROUTE_DOT && mode != SA_ROUTE_PROJ && mode != SA_ROUTE_TAYLOR2)
+  if (mode != SA_ROUTE_DOT && mode != SA_ROUTE_PROJ && mode != SA_ROUTE_TAYLOR2 && mode != SA_ROUTE_COV)
     return fail(SA_ERR_INVALID_ARG, "sa_route: unknown route mode");
   if (mode == SA_ROUTE_PROJ && (!proj_q || !proj_k))
     return fail(SA_ERR_INVALID_ARG, "sa_route: SA_ROUTE_PROJ needs proj_q and proj_k");
   if (mode == SA_ROUTE_TAYLOR2 && !stats->kvar)
     return fail(SA_ERR_INVALID_ARG, "sa_route: SA_ROUTE_TAYLOR2 needs stats->kvar");
+  if (mode == SA_ROUTE_COV && !stats->covnorm)
+    return fail(SA_ERR_INVALID_ARG, "sa_route: SA_ROUTE_COV needs stats->covnorm");
   if (topk < 0 || topk > nb) return fail(SA_ERR_INVALID_ARG, "sa_route: topk must be in [0, N/block]");
   if (nb > kMaxRouteBlocks) return fail(SA_ERR_UNSUPPORTED, "sa_route: at most 4096 blocks per head");
-  const void* ptrs[] = {stats->qmean, stats->kmean, stats->kvar, proj_q, proj_k, block_idx, scores};
+  const void* ptrs[] = {stats->qmean, stats->kmean, stats->kvar, stats->covnorm, proj_q, proj_k, block_idx, scores};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return fail(SA_ERR_ALIGNMENT, "sa_route: pointers must be 16-byte aligned");
   const bool t2 = mode == SA_ROUTE_TAYLOR2;
@@ -388,16 +420,17 @@ extern "C" sa_status sa_route(const sa_block_stats* stats, sa_shape shape, sa_ro
   const size_t smem = route_smem_bytes(nb, shape.d, topk, t2, cfg);
   cudaStream_t s = as_stream(stream);
   const sa_block_stats& st = *stats;
+  const float inv_blk = 1.0f / (float)shape.block;
   const int key = (shape.d == 128 ? 4 : 0) + (cfg.rpw == 2 ? 2 : 0) + (cfg.ncol == 2 ? 1 : 0);
   switch (key) {
-    case 7: return launch_route<128, 2, 2>(st, shape, nb, mode, proj_q, proj_k, scale, topk, block_idx, scores, smem, s);
-    case 6: return launch_route<128, 2, 1>(st, shape, nb, mode, proj_q, proj_k, scale, topk, block_idx, scores, smem, s);
-    case 5: return launch_route<128, 1, 2>(st, shape, nb, mode, proj_q, proj_k, scale, topk, block_idx, scores, smem, s);
-    case 4: return launch_route<128, 1, 1>(st, shape, nb, mode, proj_q, proj_k, scale, topk, block_idx, scores, smem, s);
-    case 3: return launch_route<64, 2, 2>(st, shape, nb, mode, proj_q, proj_k, scale, topk, block_idx, scores, smem, s);
-    case 2: return launch_route<64, 2, 1>(st, shape, nb, mode, proj_q, proj_k, scale, topk, block_idx, scores, smem, s);
-    case 1: return launch_route<64, 1, 2>(st, shape, nb, mode, proj_q, proj_k, scale, topk, block_idx, scores, smem, s);
-    default: return launch_route<64, 1, 1>(st, shape, nb, mode, proj_q, proj_k, scale, topk, block_idx, scores, smem, s);
+    case 7: return launch_route<128, 2, 2>(st, shape, nb, mode, proj_q, proj_k, scale, inv_blk, topk, block_idx, scores, smem, s);
+    case 6: return launch_route<128, 2, 1>(st, shape, nb, mode, proj_q, proj_k, scale, inv_blk, topk, block_idx, scores, smem, s);
+    case 5: return launch_route<128, 1, 2>(st, shape, nb, mode, proj_q, proj_k, scale, inv_blk, topk, block_idx, scores, smem, s);
+    case 4: return launch_route<128, 1, 1>(st, shape, nb, mode, proj_q, proj_k, scale, inv_blk, topk, block_idx, scores, smem, s);
+    case 3: return launch_route<64, 2, 2>(st, shape, nb, mode, proj_q, proj_k, scale, inv_blk, topk, block_idx, scores, smem, s);
+    case 2: return launch_route<64, 2, 1>(st, shape, nb, mode, proj_q, proj_k, scale, inv_blk, topk, block_idx, scores, smem, s);
+    case 1: return launch_route<64, 1, 2>(st, shape, nb, mode, proj_q, proj_k, scale, inv_blk, topk, block_idx, scores, smem, s);
+    default: return launch_route<64, 1, 1>(st, shape, nb, mode, proj_q, proj_k, scale, inv_blk, topk, block_idx, scores, smem, s);
   }
 }
 

@@ -42,10 +42,12 @@ def alloc_prefill(w: Workload, Q: torch.Tensor, want_scores: bool = False) -> Pr
     if Q.dtype == torch.bfloat16 and w.tail in ("zero_order", "first_order"):
         st["kmean_bf16"] = torch.empty(B, H, nb, d, device=dev, dtype=torch.bfloat16)
         st["vmean_bf16"] = torch.empty(B, H, nb, d, device=dev, dtype=torch.bfloat16)
-    if w.tail == "first_order":
+    if w.tail == "first_order" or w.route == "cov":
         st["hbar"] = torch.empty(B, H, d, d, **f)
-        if Q.dtype == torch.bfloat16:
-            st["hbarT_bf16"] = torch.empty(B, H, d, d, device=dev, dtype=torch.bfloat16)
+    if w.tail == "first_order" and Q.dtype == torch.bfloat16:
+        st["hbarT_bf16"] = torch.empty(B, H, d, d, device=dev, dtype=torch.bfloat16)
+    if w.route == "cov":
+        st["covnorm"] = torch.empty(B, H, nb, **f)
     idx = torch.empty(B, H, nb, w.k, device=dev, dtype=torch.int32)
     sc = torch.empty(B, H, nb, nb, **f) if want_scores else None
     return PrefillBuffers(st, idx, sc, torch.empty_like(Q))

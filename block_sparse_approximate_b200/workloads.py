@@ -18,8 +18,8 @@ long-context LLM decoding; these synthetic inputs stand in for them):
 * ``sla2_mix``  B=1, H=40, N=65536 on a 16x64x64 grid, generated as
                 ``video_dit``; block 128; projected router with proj_q, proj_k
                 ~ N(0, 1/d); keep 5%; linear_mix with alpha ~ U(0.2, 0.9).
-* ``video_dit_fo``  ``video_dit`` (same seed, same inputs) with PISA's
-                first-order tail.
+* ``video_dit_pisa``  ``video_dit`` (same seed, same inputs) with PISA's
+                covariance-aware router and hybrid-order (first-order) tail.
 * ``fp8``       ``video_dit`` shapes, e4m3 sparse branch; zero-order tail.
 * ``decode``    16 sequences, 32 query heads, 8 KV heads, d=128, bf16 cache of
                 131072 tokens: K, V ~ N(0,1) plus an N(0, 0.5) offset per
@@ -50,7 +50,7 @@ class Workload:
     d: int
     dtype: str                 # "fp32" | "bf16"
     block: int
-    route: str                 # "dot" | "proj" | "taylor2"
+    route: str                 # "dot" | "proj" | "taylor2" | "cov"
     tail: str                  # "drop" | "zero_order" | "first_order" | "linear_mix"
     seed: int
     topk: Optional[int] = None
@@ -88,9 +88,9 @@ WORKLOADS = {
     "sla2_mix": Workload("sla2_mix", B=1, H=40, N=16 * 64 * 64, d=128, dtype="bf16",
                          block=128, route="proj", tail="linear_mix", seed=2,
                          keep_pct=5, grid=(16, 64, 64)),
-    "video_dit_fo": Workload("video_dit_fo", B=1, H=12, N=8 * 64 * 64, d=128, dtype="bf16",
-                             block=128, route="dot", tail="first_order", seed=1,
-                             keep_pct=10, grid=(8, 64, 64)),
+    "video_dit_pisa": Workload("video_dit_pisa", B=1, H=12, N=8 * 64 * 64, d=128, dtype="bf16",
+                               block=128, route="cov", tail="first_order", seed=1,
+                               keep_pct=10, grid=(8, 64, 64)),
     "fp8": Workload("fp8", B=1, H=12, N=8 * 64 * 64, d=128, dtype="bf16",
                     block=128, route="dot", tail="zero_order", seed=3,
                     keep_pct=10, grid=(8, 64, 64), fp8=True),

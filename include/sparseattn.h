@@ -54,8 +54,13 @@ typedef enum { SA_FP32 = 0, SA_BF16 = 1 } sa_dtype;
 typedef enum {
   SA_ROUTE_DOT = 0,      /* q̄_i · k̄_j on mean-pooled blocks [SLA2 §2B] */
   SA_ROUTE_PROJ = 1,     /* (q̄_i P_q) · (k̄_j P_k), learnable router [SLA2 §2B] */
-  SA_ROUTE_TAYLOR2 = 2   /* s q̄·k̄_j + log1p(½ s² Σ_c q̄_c² var_jc), the log of
+  SA_ROUTE_TAYLOR2 = 2,  /* s q̄·k̄_j + log1p(½ s² Σ_c q̄_c² var_jc), the log of
                             exp(q·k̄)(1 + ½ qᵀ diag(Var k) q) [SPLA §2.1] */
+  SA_ROUTE_COV = 3       /* s q̄·k̄_j + log1p(s ‖q̄_i‖ M_j / block): the block's
+                            zero-order mass plus the bound s‖q‖M_j on the
+                            first-order term the hybrid order leaves out,
+                            M_j = ‖H_j − H̄‖₂ (stats->covnorm)
+                            [PISA §2 "Roteamento Consciente de Covariância"] */
 } sa_route_mode;
 
 typedef enum {
@@ -103,6 +108,10 @@ typedef struct {
                        order [PISA §2]; row c, column e                     */
   uint16_t* hbarT_bf16;  /* [B,H,d,d] bf16 of H̄ᵀ (row e, column c; the
                        tensor-core first-order tail)                        */
+  float* covnorm;   /* [B,H,nb]    M_j = ‖H_j − H̄‖₂, the spectral norm of each
+                       block's first-order deviation from the mean (power
+                       iteration to 1e-6 relative on the Gram matrix)
+                       [PISA §2 "Roteamento Consciente de Covariância"]    */
 } sa_block_stats;
 
 /* Block statistics of Q (optional), K and V.
@@ -110,7 +119,7 @@ typedef struct {
  * dtype: element type of Q, K, V.  Every non-NULL field of *stats is written;
  * kmean and vsum are required.  htot, ztot and hbar are sums over all tokens
  * of a head and are overwritten (no accumulation across calls); hbarT_bf16
- * needs hbar.
+ * and covnorm need hbar.
  * Errors: SA_ERR_INVALID_ARG (null K/V/stats/kmean/vsum, bad shape),
  *         SA_ERR_UNSUPPORTED (d or block not supported), SA_ERR_ALIGNMENT. */
 sa_status sa_block_pool(const void* Q, const void* K, const void* V, sa_dtype dtype,
@@ -118,9 +127,10 @@ sa_status sa_block_pool(const void* Q, const void* K, const void* V, sa_dtype dt
 
 /* Router: scores every (query block i, KV block j) pair and keeps the topk
  * best KV blocks per query block [SLA2 §2B; PISA S_i; SPLA §2.1].
- * stats: needs qmean and kmean (+ kvar for TAYLOR2).  proj_q, proj_k: [d,d]
+ * stats: needs qmean and kmean (+ kvar for TAYLOR2, covnorm for COV).  proj_q, proj_k: [d,d]
  * float32 row-major (x P means Σ_r x_r P[r][c]); required for PROJ, ignored
- * otherwise.  scale: softmax scale s (used by TAYLOR2 only).
+ * otherwise.  scale: softmax scale s (used by TAYLOR2 and COV; COV also
+ * divides by shape.block).
  * block_idx: [B,H,nqb,topk] int32 output, ascending; a tie in score goes to
  * the smaller block index (may be NULL when topk == 0).  scores: [B,H,nqb,nb] float32 output or NULL.
  * Errors: SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED (nb > 4096), SA_ERR_ALIGNMENT. */

@@ -72,6 +72,9 @@ def test_block_pool_validation(lib):
     st2 = _stats(kmean=FAKE, vsum=FAKE, hbarT_bf16=FAKE)     # hbarT_bf16 without hbar
     assert lib.sa_block_pool(None, FAKE, FAKE, 1, bd.Shape(1, 1, 256, 128, 128), ctypes.byref(st2), None) \
         == bd.SA_ERR_INVALID_ARG
+    st3 = _stats(kmean=FAKE, vsum=FAKE, covnorm=FAKE)        # covnorm without hbar
+    assert lib.sa_block_pool(None, FAKE, FAKE, 1, bd.Shape(1, 1, 256, 128, 128), ctypes.byref(st3), None) \
+        == bd.SA_ERR_INVALID_ARG
 
 
 def test_route_validation(lib):
@@ -81,6 +84,8 @@ def test_route_validation(lib):
     assert lib.sa_route(ctypes.byref(st), sh, 1, None, None, 1.0, 2, FAKE, None, None) == bd.SA_ERR_INVALID_ARG
     assert lib.sa_route(ctypes.byref(st), sh, 2, None, None, 1.0, 2, FAKE, None, None) == bd.SA_ERR_INVALID_ARG
     assert lib.sa_route(ctypes.byref(st), sh, 7, None, None, 1.0, 2, FAKE, None, None) == bd.SA_ERR_INVALID_ARG
+    assert lib.sa_route(ctypes.byref(st), sh, 3, None, None, 1.0, 2, FAKE, None, None) \
+        == bd.SA_ERR_INVALID_ARG            # cov without covnorm
     big = bd.Shape(1, 1, 8192 * 64, 128, 64)
     assert lib.sa_route(ctypes.byref(st), big, 0, None, None, 1.0, 2, FAKE, None, None) == bd.SA_ERR_UNSUPPORTED
 

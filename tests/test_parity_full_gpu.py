@@ -26,7 +26,7 @@ def _sample_blocks(H, nqb, n, seed):
     return sorted(picks)
 
 
-@pytest.mark.parametrize("name", ["video_dit", "video_dit_fo", "sla2_mix"])
+@pytest.mark.parametrize("name", ["video_dit", "video_dit_pisa", "sla2_mix"])
 def test_prefill_full_size_sampled(lib, name):
     w = wl.WORKLOADS[name]
     inp = wl.prefill_inputs(w, DEV)
@@ -38,7 +38,9 @@ def test_prefill_full_size_sampled(lib, name):
     check_topk_exact(buf.block_idx, buf.scores, w.k)
     ref_sc = oracle.route_scores(np64(buf.stats["qmean"]), np64(buf.stats["kmean"]), w.route,
                                  proj_q=None if "proj_q" not in inp else np64(inp["proj_q"]),
-                                 proj_k=None if "proj_k" not in inp else np64(inp["proj_k"]))
+                                 proj_k=None if "proj_k" not in inp else np64(inp["proj_k"]),
+                                 covnorm=None if "covnorm" not in buf.stats else np64(buf.stats["covnorm"]),
+                                 scale=w.scale, block=w.block)
     assert selection_agreement(np64(buf.scores[0, :2]), ref_sc[0, :2], w.k) >= 0.95
     picks = _sample_blocks(w.H, w.nb, 12, 1)
     heads = sorted({h for _, h, _ in picks})

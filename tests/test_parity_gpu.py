@@ -43,15 +43,40 @@ def test_block_pool(lib, dtype, d, block, N):
 @pytest.mark.parametrize("dtype,d,block,N", [(torch.float32, 64, 64, 1024), (torch.bfloat16, 128, 128, 4736),
                                              (torch.bfloat16, 128, 64, 2048), (torch.bfloat16, 64, 128, 1024)])
 def test_block_pool_hbar(lib, dtype, d, block, N):
-    # PISA's H̄; bf16 with d = block = 128 takes the tensor-core path, whose
-    # key deviations k − k̄_j are rounded to bf16 (relative 2^-9) before the MMA
+    # PISA's H̄ (bf16 with d = block = 128 takes the tensor-core path) and the
+    # covariance norms M_j = ‖H_j − H̄‖₂ (power iteration to 1e-6 on λ)
     Q, K, V = _gauss(2, 3, N, d, dtype, 11)
-    st = bd.block_pool(Q, K, V, block, centroids_bf16=True, first_order=True)
-    ref = oracle.block_pool(np64(Q), np64(K), np64(V), block, first_order=True)
-    tc = dtype == torch.bfloat16 and d == 128 and block == 128
-    assert_stats_close(st["hbar"], ref["hbar"], "hbar", rtol=5e-3 if tc else 1e-4)
+    st = bd.block_pool(Q, K, V, block, centroids_bf16=True, first_order=True, covariance=True)
+    ref = oracle.block_pool(np64(Q), np64(K), np64(V), block, first_order=True, covariance=True)
+    assert_stats_close(st["hbar"], ref["hbar"], "hbar", rtol=1e-4)
     hT = np.swapaxes(ref["hbar"], -1, -2)
-    assert_stats_close(st["hbarT_bf16"].float(), hT, "hbarT_bf16", rtol=(5e-3 if tc else 0) + 2 ** -8)
+    assert_stats_close(st["hbarT_bf16"].float(), hT, "hbarT_bf16", rtol=2 ** -8)
+    got = np64(st["covnorm"])
+    np.testing.assert_allclose(got, ref["covnorm"], rtol=1e-3, atol=1e-4)
+
+
+@pytest.mark.parametrize("dtype,d,block", [(torch.bfloat16, 128, 128), (torch.float32, 64, 64)])
+def test_covnorm_rank_one(lib, dtype, d, block):
+    # keys k̄_j + a_n u, values b_n w + c_j: H_j − H̄ = (γ_j − γ̄) u wᵀ, so
+    # M_j = |γ_j − γ̄| |u| |w| (u, w, a, b chosen exactly representable in bf16)
+    g = torch.Generator(device="cpu")
+    g.manual_seed(13)
+    nb = 12
+    u = torch.randint(-4, 5, (d,), generator=g).double()
+    w = torch.randint(-4, 5, (d,), generator=g).double()
+    kbar = torch.randint(-8, 9, (nb, d), generator=g).double()
+    r = torch.randint(-3, 4, (nb, block // 2), generator=g).double()
+    a = torch.cat([r, -r], dim=1)                 # zero-mean deviations, small integers
+    bcoef = torch.randint(-3, 4, (nb, block), generator=g).double() / 4
+    cval = torch.randint(-8, 9, (nb, d), generator=g).double() / 8
+    K = (kbar[:, None, :] + a[:, :, None] * u[None, None, :]).reshape(1, 1, nb * block, d)
+    V = (bcoef[:, :, None] * w[None, None, :] + cval[:, None, :]).reshape(1, 1, nb * block, d)
+    gam = (a * bcoef).sum(dim=1)
+    expect = ((gam - gam.mean()).abs() * u.norm() * w.norm()).numpy()
+    Kd, Vd = K.to(dtype).to(DEV), V.to(dtype).to(DEV)
+    assert torch.equal(Kd.double().cpu(), K) and torch.equal(Vd.double().cpu(), V)
+    st = bd.block_pool(None, Kd, Vd, block, covariance=True)
+    np.testing.assert_allclose(np64(st["covnorm"])[0, 0], expect, rtol=1e-4, atol=1e-3)
 
 
 def test_block_pool_hbar_large_offset(lib):
@@ -77,7 +102,7 @@ def test_block_pool_large_offset_variance(lib):
 # router
 # --------------------------------------------------------------------------
 
-@pytest.mark.parametrize("mode", ["dot", "proj", "taylor2"])
+@pytest.mark.parametrize("mode", ["dot", "proj", "taylor2", "cov"])
 @pytest.mark.parametrize("nb,k", [(37, 5), (256, 26), (16, 0), (16, 16), (97, 64), (97, 65), (300, 100)])
 def test_route(lib, mode, nb, k):
     d, block = 128, 128
@@ -91,12 +116,13 @@ def test_route(lib, mode, nb, k):
     g.manual_seed(5)
     Pq = (torch.randn(d, d, generator=g, device=DEV) / math.sqrt(d)).contiguous()
     Pk = (torch.randn(d, d, generator=g, device=DEV) / math.sqrt(d)).contiguous()
-    st = bd.block_pool(Q, K, V, block, variance=True)
+    st = bd.block_pool(Q, K, V, block, variance=True, covariance=(mode == "cov"))
     s = 1 / math.sqrt(d)
     shape = (1, 2, nb * block, d, block)
     idx, sc = bd.route(st, shape, mode, k, proj_q=Pq, proj_k=Pk, scale=s, want_scores=True)
     ref = oracle.route_scores(np64(st["qmean"]), np64(st["kmean"]), mode, proj_q=np64(Pq),
-                              proj_k=np64(Pk), kvar=np64(st["kvar"]), scale=s)
+                              proj_k=np64(Pk), kvar=np64(st["kvar"]), scale=s,
+                              covnorm=np64(st["covnorm"]) if mode == "cov" else None, block=block)
     assert_stats_close(sc, ref, f"{mode} scores", rtol=2e-5)
     check_topk_exact(idx, sc, k)
     frac = selection_agreement(np64(sc), ref, k)
@@ -188,6 +214,33 @@ def test_first_order_tail_matters(lib, dtype, nb, k):
     assert np.abs(ref_fo - ref_zo).mean() > 10 * tol[1]
     assert_tol(np64(o_fo), ref_fo, tol, "first_order")
     assert_tol(np64(o_fo) - np64(o_zo), ref_fo - ref_zo, (2 * tol[0], 2 * tol[1]), "first_order - zero_order")
+
+
+@pytest.mark.parametrize("k", [1, 4, 26])
+def test_pisa_small(lib, k):
+    # PISA end to end: covariance-aware routing on the GPU's statistics (scores
+    # against the oracle's score of the same statistics, selection bit-exact
+    # against the oracle's top-k of the GPU scores, selection agreement with
+    # the oracle's statistics) and the hybrid-order tail on that selection
+    w = wl.WORKLOADS["video_dit_pisa"]
+    inp = wl.prefill_inputs(w, DEV, H=2, N=4096)
+    Q, K, V = inp["Q"], inp["K"], inp["V"]
+    B, H, N, d = Q.shape
+    s = w.scale
+    st = bd.block_pool(Q, K, V, w.block, centroids_bf16=True, first_order=True, covariance=True)
+    idx, sc = bd.route(st, (B, H, N, d, w.block), "cov", k, scale=s, want_scores=True)
+    check_topk_exact(idx, sc, k)
+    ref_st = oracle.block_pool(np64(Q), np64(K), np64(V), w.block, covariance=True)
+    ref_sc = oracle.route_scores(ref_st["qmean"], ref_st["kmean"], "cov", covnorm=ref_st["covnorm"],
+                                 scale=s, block=w.block)
+    # M_j comes from a power iteration stopped at 1e-6 on λ: scores within 2e-3
+    np.testing.assert_allclose(np64(sc), ref_sc, rtol=1e-4, atol=2e-3)
+    assert selection_agreement(np64(sc), ref_sc, k, gap_rel=5e-3) >= 0.9
+    O = bd.sparse_attn_fwd(Q, K, V, idx, w.block, "first_order", st, s)
+    torch.cuda.synchronize()
+    assert_no_device_error()
+    ref = oracle.sparse_attention(np64(Q), np64(K), np64(V), idx.cpu().numpy(), w.block, "first_order", s)
+    assert_tol(np64(O), ref, BF16_TOL, f"pisa k={k}")
 
 
 def test_empty_problem_is_a_no_op(lib):
