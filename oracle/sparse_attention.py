@@ -30,6 +30,14 @@ design notes of the repository):
   block, s q̄.k̄_j + log1p(s ‖q̄_i‖ M_j / B) (the page says the score
   "incorporates" both without a formula; this is the plainest combination the
   error argument gives);
+* SPLA's residual linear attention (decode tail "residual_linear"): the
+  feature map is φ(x) = exp(x) on the unscaled q and k, o_rla = ō − õ is the
+  difference of the UNNORMALISED linear attentions over all blocks and over
+  the selected ones (φ(q)ᵀ Σ_{n∈U} φ(k_n) v_nᵀ, the state that "accumulates
+  only the unselected blocks"), and the gated sum is o = o_sparse +
+  RMSNorm(o_rla) with unit gain (the RMS norm's scale is the only parameter
+  the page names; no trained value exists here) and eps = 1e-6; o_sparse is
+  the drop output;
 * GQA decode shares one selection per (batch, KV head); the group's score for
   a block is the log of the sum over the group's query heads of each head's
   SPLA block mass (a logsumexp of the log-form scores).
@@ -42,6 +50,9 @@ Pins (the tests under ``tests/test_oracle_*.py``):
                       per-block deviations -> PISA's per-block first-order
                       Taylor sum by brute force; error O(ε²) vs zero_order's
                       O(ε) as the in-block deviations shrink
+  residual_linear     all blocks selected -> drop (= dense); brute-force
+                      token loops; the subtraction form φ(q)ᵀ(S_all − S_sel)
+                      equals the direct sum; RMS-norm scale invariance
   covnorm / "cov"     rank-one deviations H_j − H̄ = (γ_j − γ̄) u wᵀ -> closed
                       form |γ_j − γ̄|·|u|·|w|; identical blocks -> M_j = 0 and
                       "cov" = s·"dot"; the square root of the largest
@@ -268,6 +279,9 @@ def _attend_rows(q, K, V, sel: Sequence[int], nb: int, block: int, tail: str,
     contrast with).  "linear_mix" is SLA2 §2A O = α⊙O_s + (1−α)⊙O_l with O_s
     the drop output and O_l the ReLU linear attention (SALAD §2) over U:
       O_l = φ(q)ᵀ Σ_{n∈U} φ(k_n) v_nᵀ / (φ(q)·Σ_{n∈U} φ(k_n) + eps).
+    "residual_linear" is SPLA's sparse plus residual linear attention
+    (§2.2-2.3): o = O_s + RMSNorm(o_rla) with o_rla = φ(q)ᵀ Σ_{n∈U} φ(k_n) v_nᵀ,
+    φ = exp elementwise, RMSNorm(x) = x / sqrt(mean(x²) + eps) (unit gain).
     """
     sel = sorted(int(j) for j in sel)
     uns = [j for j in range(nb) if j not in set(sel)]
@@ -299,7 +313,7 @@ def _attend_rows(q, K, V, sel: Sequence[int], nb: int, block: int, tail: str,
                 hbar = np.einsum("jnc,jne->ce", dev, V.reshape(nb, block, d)) / nb
             num = num + ((scale * q) @ _f64(hbar)) * wc.sum(axis=1)[:, None]
         return num / den[:, None]
-    if tail in ("drop", "linear_mix"):
+    if tail in ("drop", "linear_mix", "residual_linear"):
         if a.shape[1]:
             m = a.max(axis=1)
             wa = np.exp(a - m[:, None])
@@ -308,6 +322,15 @@ def _attend_rows(q, K, V, sel: Sequence[int], nb: int, block: int, tail: str,
             o_s = np.zeros((R, d))
         if tail == "drop":
             return o_s
+        if tail == "residual_linear":
+            # SPLA §2.2-2.3: the residual linear attention over the unselected
+            # tokens with the exponential feature map, φ(q)ᵀ Σ_{n∈U} φ(k_n) v_nᵀ
+            # (unnormalised: the RMS norm scales it), added to the exact part
+            # after an RMS norm of unit gain
+            tokU = _block_tokens(uns, block)
+            o_l = (np.exp(q) @ np.exp(K[tokU]).T) @ V[tokU]
+            rms = np.sqrt((o_l * o_l).mean(axis=1) + eps)
+            return o_s + o_l / rms[:, None]
         utok = _block_tokens(uns, block)
         phi_k = np.maximum(K[utok], 0.0)
         phi_q = np.maximum(q, 0.0)
@@ -388,7 +411,8 @@ def decode_attention(q, Kcache, Vcache, block: int, topk: int, scale: float, *,
     sums are computed from the cache, the group-shared taylor2 route picks
     ``topk`` blocks (unless ``block_idx`` [B,Hkv,topk] is given), and each of
     the group's query heads attends exactly to the selected blocks plus
-    PISA's zero-order term for the rest (or drops them).
+    PISA's zero-order term for the rest (or drops them, or adds SPLA's
+    residual linear attention over them: tail "residual_linear").
 
     Returns (o [B,Hq,d], block_idx [B,Hkv,topk], scores [B,Hkv,nb]).  With
     ``pairs`` (an iterable of (b, kv_head)) only those pairs are computed; the
