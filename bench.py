@@ -245,17 +245,19 @@ def run_reference(args, world, rank):
 # GPU arm
 # --------------------------------------------------------------------------
 
-def time_decode(steps: int = 50, warmup: int = 5, batch=None):
+def time_decode(steps: int = 50, warmup: int = 5, batch=None, name: str = "decode"):
     """Decode workload timing (separate from the prefill step): GB/s of the
     bytes the method moves per decode step.  ``batch`` shrinks the number of
-    sequences (for bounded profiler captures)."""
+    sequences (for bounded profiler captures).  ``decode_rla`` is the same
+    caches with SPLA's residual linear tail."""
     from block_sparse_approximate_b200 import binding as bd
     from block_sparse_approximate_b200.pipeline import DecodeStep
-    w = wl.WORKLOADS["decode"]
+    w = wl.WORKLOADS[name]
+    rla = w.tail == "residual_linear"
     if batch:
         w = wl.Workload(**{**w.__dict__, "B": int(batch)})
     inp = wl.decode_inputs(w, "cuda")
-    st = bd.block_pool(None, inp["Kcache"], inp["Vcache"], w.block, variance=True)
+    st = bd.block_pool(None, inp["Kcache"], inp["Vcache"], w.block, variance=True, residual=rla)
     step = DecodeStep(w, inp, st)
     for _ in range(warmup):
         step()
@@ -269,13 +271,15 @@ def time_decode(steps: int = 50, warmup: int = 5, batch=None):
     ms = s.elapsed_time(e) / steps
     B, Hkv, nb, d = w.B, w.Hkv, w.nb, w.d
     kv = 2.0 * B * Hkv * w.k * w.block * d * 2          # selected K and V, bf16
-    stats = 3.0 * B * Hkv * nb * d * 4                    # kmean, kvar, vsum fp32 (read once each)
+    # kmean, kvar (route) and vsum (zero-order tail) fp32, read once each; the
+    # residual linear tail reads S_all (d×d per KV head) instead of vsum
+    stats = (2.0 if rla else 3.0) * B * Hkv * nb * d * 4 + (4.0 * B * Hkv * d * d if rla else 0.0)
     qo = 2.0 * B * w.H * d * 2
     byts = kv + stats + qo
     hbm, _, _, src = _peaks()
     del inp, st, step
     torch.cuda.empty_cache()
-    return {"workload": "decode", "ms": ms, "bytes_per_step": byts, "gbs": byts / ms / 1e6,
+    return {"workload": name, "ms": ms, "bytes_per_step": byts, "gbs": byts / ms / 1e6,
             "hbm_peak_gbs": hbm, "frac": byts / ms / 1e6 / hbm, "peak_source": src}
 
 
@@ -390,9 +394,10 @@ def run_ours(args, world, rank, local):
     from block_sparse_approximate_b200.pipeline import PrefillStep
     torch.cuda.set_device(local)
     bd.load()
-    if args.only == "decode":
+    if args.only in ("decode", "decode_rla"):
         if rank == 0:
-            print(json.dumps({"decode": time_decode(args.steps, args.warmup, args.decode_batch)}), flush=True)
+            print(json.dumps({args.only: time_decode(args.steps, args.warmup, args.decode_batch, args.only)}),
+                  flush=True)
         return 0
     if args.only == "fp8":
         if rank == 0:
@@ -494,11 +499,12 @@ def run_ours(args, world, rank, local):
                "h2d_bytes_per_step": sum(inp[n].numel() * inp[n].element_size() for n in ("Q", "K", "V")),
                "d2h_bytes_per_step": step.buf.out.numel() * step.buf.out.element_size()}
 
-    decode = fp8 = sla2 = pisa = None
+    decode = decode_rla = fp8 = sla2 = pisa = None
     if rank == 0 and args.only == "all" and not args.no_decode:
         del step
         torch.cuda.empty_cache()
         decode = time_decode(batch=args.decode_batch)
+        decode_rla = time_decode(batch=args.decode_batch, name="decode_rla")
         fp8 = time_fp8()
         sla2 = time_sla2()
         pisa = time_pisa()
@@ -533,6 +539,7 @@ def run_ours(args, world, rank, local):
         "gpu_launches": args.steps * PrefillStepLaunches(w),
         "clocks": ck,
         "decode": decode,
+        "decode_rla": decode_rla,
         "fp8": fp8,
         "sla2_mix": sla2,
         "pisa": pisa,
@@ -554,7 +561,8 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
-    ap.add_argument("--only", choices=["all", "prefill", "decode", "fp8", "sla2", "pisa"], default="all",
+    ap.add_argument("--only", choices=["all", "prefill", "decode", "decode_rla", "fp8", "sla2", "pisa"],
+                    default="all",
                     help="prefill: the timed step only; decode / fp8 / sla2 / pisa (covariance routing + "
                          "first-order tail): only that workload's timing")
     ap.add_argument("--decode-batch", type=int, default=None,

@@ -22,7 +22,7 @@ LIB_PATH = os.path.join(_HERE, "libsparseattn.so")
 SA_OK, SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED, SA_ERR_ALIGNMENT, SA_ERR_CUDA, SA_ERR_WORKSPACE = range(6)
 SA_FP32, SA_BF16 = 0, 1
 ROUTE = {"dot": 0, "proj": 1, "taylor2": 2, "cov": 3}
-TAIL = {"drop": 0, "zero_order": 1, "linear_mix": 2, "first_order": 3}
+TAIL = {"drop": 0, "zero_order": 1, "linear_mix": 2, "first_order": 3, "residual_linear": 4}
 
 # every entry point declared in include/sparseattn.h
 EXPORTS = ("sa_block_pool", "sa_route", "sa_sparse_attn_fwd", "sa_decode_workspace_size",
@@ -47,7 +47,7 @@ class DecodeShape(ctypes.Structure):
 
 
 _STAT_FIELDS = ("qmean", "kmean", "vsum", "kvar", "zrelu", "htot", "ztot", "kmean_bf16", "vmean_bf16",
-                "hbar", "hbarT_bf16", "covnorm")
+                "hbar", "hbarT_bf16", "covnorm", "sexp")
 
 
 class BlockStats(ctypes.Structure):
@@ -142,7 +142,8 @@ def version() -> str:
 
 def block_pool(Q: Optional[torch.Tensor], K: torch.Tensor, V: torch.Tensor, block: int, *,
                variance: bool = False, linear: bool = False, centroids_bf16: bool = False,
-               first_order: bool = False, covariance: bool = False, stream=None) -> dict:
+               first_order: bool = False, covariance: bool = False, residual: bool = False,
+               stream=None) -> dict:
     """Block statistics of (Q,) K, V [B,H,N,d]; returns a dict of float32 tensors."""
     lib = load()
     Bsz, H, N, d = K.shape
@@ -167,6 +168,8 @@ def block_pool(Q: Optional[torch.Tensor], K: torch.Tensor, V: torch.Tensor, bloc
             st["hbarT_bf16"] = torch.empty(Bsz, H, d, d, device=dev, dtype=torch.bfloat16)
     if covariance:
         st["covnorm"] = torch.empty(Bsz, H, nb, **f)
+    if residual:
+        st["sexp"] = torch.empty(Bsz, H, d, d, **f)
     cst = _stats_struct(st)
     _check("sa_block_pool", lib.sa_block_pool(_ptr(Q), _ptr(K), _ptr(V), _dtype_code(K),
                                               Shape(Bsz, H, N, d, block), ctypes.byref(cst),

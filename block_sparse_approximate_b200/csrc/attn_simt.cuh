@@ -23,13 +23,16 @@ bool attn_tc_supports(sa_dtype dtype, const sa_shape& s, sa_tail_mode tail);
 
 // d×d sums per head on the tensor cores (bf16, d = 128, N a multiple of 128),
 // added into `out`, which the caller zeroes first:
-//   kmean == NULL: H_tot = Σ_n relu(k_n) v_nᵀ (oscale 1);
-//   kmean != NULL: oscale · Σ_j Σ_{n∈j} (k_n − k̄_j) v_nᵀ over 128-token blocks
-//                  with centroids kmean and value sums vsum [B,H,N/128,d]
-//                  (H̄ with oscale = 1/nb).
+//   kKvRelu:   H_tot = Σ_n relu(k_n) v_nᵀ (oscale 1);
+//   kKvCentre: oscale · Σ_j Σ_{n∈j} (k_n − k̄_j) v_nᵀ over 128-token blocks
+//              with centroids kmean and value sums vsum [B,H,N/128,d]
+//              (H̄ with oscale = 1/nb);
+//   kKvExp:    Σ_n φ(k_n) v_nᵀ with φ = phi_exp rounded to bf16 (SPLA's
+//              residual linear state; oscale 1).
 // Returns SA_ERR_UNSUPPORTED (without setting an error) for other shapes.
-sa_status kv_outer_tc(const void* K, const void* V, const sa_shape& s, const float* kmean, const float* vsum,
-                      float oscale, float* out, cudaStream_t stream);
+enum { kKvRelu = 0, kKvCentre = 1, kKvExp = 2 };
+sa_status kv_outer_tc(const void* K, const void* V, const sa_shape& s, int feature, const float* kmean,
+                      const float* vsum, float oscale, float* out, cudaStream_t stream);
 
 // PISA's block covariance norms M_j = ‖H_j − H̄‖₂ on the tensor cores (bf16,
 // d = block = 128): covnorm [B,H,nb] from K, V and the statistics kmean,

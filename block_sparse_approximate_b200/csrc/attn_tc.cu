@@ -1016,19 +1016,20 @@ attn_tc_linmix_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
 
 // ---------------------------------------------------------------- H_tot, H̄
 // d×d outer-product sums Σ_n f(k_n) v_nᵀ of one head on the tensor cores:
-//   kmean == NULL: f = relu, H_tot (the total of SLA2's ReLU linear branch,
-//                  SALAD §2);
-//   kmean != NULL: f(k_n) = k_n − k̄_j with k̄_j the centroid of the 128-token
-//                  block that holds n, each chunk's sum scaled by oscale
-//                  (1/nb): PISA's mean first-order statistic H̄ (§2).  The
-//                  MMAs accumulate the raw Kᵀ V of the chunk (bf16 products
-//                  are exact in fp32) and the epilogue subtracts
-//                  Σ_j k̄_j vsum_jᵀ over the chunk's blocks in fp32, which
-//                  equals Σ_j Σ_n (k_n − k̄_j) v_nᵀ without rounding the
-//                  deviations to bf16.
-// A CTA takes a chunk of 128-token tiles of one head, warps 2-5 apply the
-// ReLU in place to each K tile (H_tot only), warp 1 accumulates f(K)ᵀ V in
-// TMEM (MN-major × MN-major MMA), and the chunk's d×d sum is added to `out`
+//   kKvRelu:   f = relu, H_tot (the total of SLA2's ReLU linear branch,
+//              SALAD §2);
+//   kKvCentre: f(k_n) = k_n − k̄_j with k̄_j the centroid of the 128-token
+//              block that holds n, each chunk's sum scaled by oscale (1/nb):
+//              PISA's mean first-order statistic H̄ (§2).  The MMAs
+//              accumulate the raw Kᵀ V of the chunk (bf16 products are exact
+//              in fp32) and the epilogue subtracts Σ_j k̄_j vsum_jᵀ over the
+//              chunk's blocks in fp32, which equals Σ_j Σ_n (k_n − k̄_j) v_nᵀ
+//              without rounding the deviations to bf16;
+//   kKvExp:    f = φ = phi_exp rounded to bf16: SPLA's residual linear state
+//              Σ_n φ(k_n) v_nᵀ over all tokens (§2.2).
+// A CTA takes a chunk of 128-token tiles of one head, warps 2-5 apply f in
+// place to each K tile (relu, exp), warp 1 accumulates f(K)ᵀ V in TMEM
+// (MN-major × MN-major MMA), and the chunk's d×d sum is added to `out`
 // with vector atomics.  Warp 0 is the TMA producer.
 constexpr int kHtThreads = 192;
 constexpr int kHtMinTiles = 4;        // fewest tiles (of 128 tokens) per CTA
@@ -1044,8 +1045,8 @@ struct HtLayout {
 
 __global__ void __launch_bounds__(kHtThreads, 1)
 htot_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, int N,
-               int tiles_per_cta, const float* __restrict__ kmean, const float* __restrict__ vsum, float oscale,
-               float* __restrict__ htot) {
+               int tiles_per_cta, int feature, const float* __restrict__ kmean, const float* __restrict__ vsum,
+               float oscale, float* __restrict__ htot) {
   using L = HtLayout;
   constexpr int NS = L::NS;
   constexpr uint32_t kTile = L::kTile;
@@ -1129,7 +1130,7 @@ htot_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
         ok = false;
         break;
       }
-      if (!kmean) {
+      if (feature == kKvRelu) {
         uint4* kt = reinterpret_cast<uint4*>(smem + 2 * kTile * s);
         const __nv_bfloat162 zero = __float2bfloat162_rn(0.f);
 #pragma unroll 4
@@ -1138,6 +1139,19 @@ htot_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
           __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
 #pragma unroll
           for (int e = 0; e < 4; ++e) h[e] = __hmax2(h[e], zero);
+          kt[x] = u;
+        }
+      } else if (feature == kKvExp) {
+        uint4* kt = reinterpret_cast<uint4*>(smem + 2 * kTile * s);
+#pragma unroll 4
+        for (int x = tr; x < (int)(kTile / 16); x += 128) {
+          uint4 u = kt[x];
+          __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(h[e]);
+            h[e] = __floats2bfloat162_rn(phi_exp(f.x), phi_exp(f.y));
+          }
           kt[x] = u;
         }
       }
@@ -1156,7 +1170,7 @@ htot_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
         uint32_t a[32];
         tmem_ld32(lrow + 32 * cc, a);
         tmem_wait_ld();
-        if (kmean) {
+        if (feature == kKvCentre) {
           // − Σ_j k̄_j[c] vsum_j[e] over the chunk's blocks
           float* f = reinterpret_cast<float*>(a);
           for (int t = 0; t < T; ++t) {
@@ -1196,9 +1210,9 @@ bool make_tmap_128x128(void* map, const void* base, int elem, uint64_t cols, uin
   return make_tmap_3d(static_cast<CUtensorMap*>(map), base, elem, cols, rows, outer);
 }
 
-sa_status kv_outer_tc(const void* K, const void* V, const sa_shape& s, const float* kmean, const float* vsum,
-                      float oscale, float* out, cudaStream_t stream) {
-  if (s.d != TD || (s.N % TB) || (kmean && s.block != TB)) return SA_ERR_UNSUPPORTED;
+sa_status kv_outer_tc(const void* K, const void* V, const sa_shape& s, int feature, const float* kmean,
+                      const float* vsum, float oscale, float* out, cudaStream_t stream) {
+  if (s.d != TD || (s.N % TB) || (feature == kKvCentre && s.block != TB)) return SA_ERR_UNSUPPORTED;
   const uint64_t BH = (uint64_t)s.B * s.H;
   CUtensorMap mk, mv;
   if (!make_tmap_3d(&mk, K, 2, TD, s.N, BH) || !make_tmap_3d(&mv, V, 2, TD, s.N, BH))
@@ -1228,7 +1242,7 @@ sa_status kv_outer_tc(const void* K, const void* V, const sa_shape& s, const flo
     if (ctas <= sms) break;   // one wave: more tiles per CTA only add time
   }
   dim3 grid((nt + tpc - 1) / tpc, (unsigned)BH);
-  htot_tc_kernel<<<grid, kHtThreads, smem, stream>>>(mk, mv, s.N, tpc, kmean, vsum, oscale, out);
+  htot_tc_kernel<<<grid, kHtThreads, smem, stream>>>(mk, mv, s.N, tpc, feature, kmean, vsum, oscale, out);
   return launch_status("htot_tc_kernel");
 }
 

@@ -143,22 +143,25 @@ block_pool_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __r
 
 // One chunk of tokens per CTA adds its d×d outer-product sum Σ_n f(k_n) v_nᵀ
 // to out[b,h]:
-//   BLKDEV == 0: f(k) = relu(k), and ztot[b,h] += Σ relu(k_n) — the totals of
+//   kFeatRelu:   f(k) = relu(k), and ztot[b,h] += Σ relu(k_n) — the totals of
 //                the SLA2/SALAD linear branch;
-//   BLKDEV  > 0: f(k_n) = k_n − k̄_j for the block j of BLKDEV tokens that
-//                holds n, each chunk's sum scaled by oscale = 1/nb — PISA's
-//                mean first-order statistic H̄ (§2 "Algoritmo Central").
+//   kFeatCentre: f(k_n) = k_n − k̄_j for the block j of BLK tokens that holds
+//                n, each chunk's sum scaled by oscale = 1/nb — PISA's mean
+//                first-order statistic H̄ (§2 "Algoritmo Central");
+//   kFeatExp:    f(k) = exp(k) — the all-token state of SPLA's residual
+//                linear attention (§2.2-2.3).
 // Thread t owns row c = t / (256/D) of the d×d sum and D*D/256 of its columns.
 constexpr int kLinChunk = 1024;
 constexpr int kLinTile = 32;
 
-template <typename T, int D, int BLKDEV = 0>
+enum { kFeatRelu = 0, kFeatCentre = 1, kFeatExp = 2 };
+
+template <typename T, int D, int FEAT, int BLK = 1>
 __global__ void __launch_bounds__(256)
 linear_totals_kernel(const T* __restrict__ K, const T* __restrict__ V, int H, int N,
                      float* __restrict__ htot, float* __restrict__ ztot,
                      const float* __restrict__ kmean = nullptr, float oscale = 1.f) {
-  static_assert(kLinChunk % (BLKDEV ? BLKDEV : 1) == 0, "a chunk holds whole blocks");
-  constexpr int kDevBlk = BLKDEV ? BLKDEV : 1;
+  static_assert(kLinChunk % BLK == 0, "a chunk holds whole blocks");
   constexpr int TPR = 256 / D;       // threads per output row
   constexpr int CPT = D / TPR;       // columns per thread
   const int chunk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -182,24 +185,25 @@ linear_totals_kernel(const T* __restrict__ K, const T* __restrict__ V, int H, in
       if (n < n_end) {
         kv = to_f<T>(K[head_off + (size_t)n * D + cc]);
         vv = to_f<T>(V[head_off + (size_t)n * D + cc]);
-        if (BLKDEV) kv -= kmean[(((size_t)b * H + h) * (N / kDevBlk) + n / kDevBlk) * D + cc];
+        if (FEAT == kFeatCentre) kv -= kmean[(((size_t)b * H + h) * (N / BLK) + n / BLK) * D + cc];
+        if (FEAT == kFeatExp) kv = phi_exp(kv);
       }
-      ks[r][cc] = BLKDEV ? kv : fmaxf(kv, 0.f);
+      ks[r][cc] = FEAT == kFeatRelu ? fmaxf(kv, 0.f) : kv;
       vs[r][cc] = vv;
     }
     __syncthreads();
 #pragma unroll 4
     for (int r = 0; r < kLinTile; ++r) {
       const float kr = ks[r][c];
-      if (!BLKDEV && e0 == 0) z += kr;
+      if (FEAT == kFeatRelu && e0 == 0) z += kr;
 #pragma unroll
       for (int i = 0; i < CPT; ++i) acc[i] = fmaf(kr, vs[r][e0 + i], acc[i]);
     }
   }
   float* hp = htot + ((size_t)b * H + h) * D * D + (size_t)c * D + e0;
 #pragma unroll
-  for (int i = 0; i < CPT; ++i) atomicAdd(hp + i, BLKDEV ? acc[i] * oscale : acc[i]);
-  if (!BLKDEV && e0 == 0) atomicAdd(ztot + ((size_t)b * H + h) * D + c, z);
+  for (int i = 0; i < CPT; ++i) atomicAdd(hp + i, acc[i] * oscale);
+  if (FEAT == kFeatRelu && e0 == 0) atomicAdd(ztot + ((size_t)b * H + h) * D + c, z);
 }
 
 // bf16 copy of H̄ᵀ: out[b,h][e][c] = H̄[b,h][c][e] (the B operand of the
@@ -341,15 +345,27 @@ sa_status launch_pool(const void* Q, const void* K, const void* V, const sa_shap
       return launch_status("cudaMemsetAsync(htot/ztot)");
     // bf16, d = 128: H_tot on the tensor cores and z_tot from the block sums
     if (sizeof(T) == 2 && D == 128 && st.zrelu &&
-        kv_outer_tc(K, V, s, nullptr, nullptr, 1.f, st.htot, stream) == SA_OK) {
+        kv_outer_tc(K, V, s, kKvRelu, nullptr, nullptr, 1.f, st.htot, stream) == SA_OK) {
       ztot_from_blocks_kernel<D><<<dim3(s.H, s.B), D, 0, stream>>>(st.zrelu, s.H, s.N / BLK, st.ztot);
       return launch_status("ztot_from_blocks_kernel");
     }
     dim3 g2((s.N + kLinChunk - 1) / kLinChunk, s.H, s.B);
-    linear_totals_kernel<T, D><<<g2, 256, 0, stream>>>(
+    linear_totals_kernel<T, D, kFeatRelu><<<g2, 256, 0, stream>>>(
         static_cast<const T*>(K), static_cast<const T*>(V), s.H, s.N, st.htot, st.ztot);
     r = launch_status("linear_totals_kernel");
     if (r != SA_OK) return r;
+  }
+  if (st.sexp) {
+    // SPLA's all-token state Σ_n exp(k_n) v_nᵀ
+    const size_t hbytes = (size_t)s.B * s.H * s.d * s.d * sizeof(float);
+    if (cudaMemsetAsync(st.sexp, 0, hbytes, stream) != cudaSuccess) return launch_status("cudaMemsetAsync(sexp)");
+    if (!(sizeof(T) == 2 && D == 128 && kv_outer_tc(K, V, s, kKvExp, nullptr, nullptr, 1.f, st.sexp, stream) == SA_OK)) {
+      dim3 g2((s.N + kLinChunk - 1) / kLinChunk, s.H, s.B);
+      linear_totals_kernel<T, D, kFeatExp><<<g2, 256, 0, stream>>>(
+          static_cast<const T*>(K), static_cast<const T*>(V), s.H, s.N, st.sexp, nullptr);
+      r = launch_status("linear_totals_kernel(sexp)");
+      if (r != SA_OK) return r;
+    }
   }
   if (st.hbar) {
     // PISA's H̄ from the block centroids written above (same stream)
@@ -357,9 +373,9 @@ sa_status launch_pool(const void* Q, const void* K, const void* V, const sa_shap
     if (cudaMemsetAsync(st.hbar, 0, hbytes, stream) != cudaSuccess) return launch_status("cudaMemsetAsync(hbar)");
     const float inv_nb = 1.0f / (float)(s.N / BLK);
     if (!(sizeof(T) == 2 && D == 128 && BLK == 128 &&
-          kv_outer_tc(K, V, s, st.kmean, st.vsum, inv_nb, st.hbar, stream) == SA_OK)) {
+          kv_outer_tc(K, V, s, kKvCentre, st.kmean, st.vsum, inv_nb, st.hbar, stream) == SA_OK)) {
       dim3 g2((s.N + kLinChunk - 1) / kLinChunk, s.H, s.B);
-      linear_totals_kernel<T, D, BLK><<<g2, 256, 0, stream>>>(
+      linear_totals_kernel<T, D, kFeatCentre, BLK><<<g2, 256, 0, stream>>>(
           static_cast<const T*>(K), static_cast<const T*>(V), s.H, s.N, st.hbar, nullptr, st.kmean, inv_nb);
       r = launch_status("linear_totals_kernel(hbar)");
       if (r != SA_OK) return r;
@@ -414,7 +430,7 @@ extern "C" sa_status sa_block_pool(const void* Q, const void* K, const void* V, 
     return fail(SA_ERR_INVALID_ARG, "sa_block_pool: hbarT_bf16 and covnorm need hbar");
   const void* ptrs[] = {Q, K, V, stats->qmean, stats->kmean, stats->vsum, stats->kvar,
                         stats->zrelu, stats->htot, stats->ztot, stats->kmean_bf16, stats->vmean_bf16,
-                        stats->hbar, stats->hbarT_bf16, stats->covnorm};
+                        stats->hbar, stats->hbarT_bf16, stats->covnorm, stats->sexp};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return fail(SA_ERR_ALIGNMENT, "sa_block_pool: pointers must be 16-byte aligned");
   cudaStream_t s = as_stream(stream);

@@ -41,6 +41,8 @@ extern "C" sa_status sa_sparse_attn_fwd(const void* Q, const void* K, const void
   const int nb = shape.N / shape.block;
   if (dtype != SA_FP32 && dtype != SA_BF16)
     return fail(SA_ERR_UNSUPPORTED, "sa_sparse_attn_fwd: dtype must be SA_FP32 or SA_BF16");
+  if (tail == SA_TAIL_RESIDUAL_LINEAR)
+    return fail(SA_ERR_UNSUPPORTED, "sa_sparse_attn_fwd: SA_TAIL_RESIDUAL_LINEAR is a decode tail");
   if (tail != SA_TAIL_DROP && tail != SA_TAIL_ZERO_ORDER && tail != SA_TAIL_LINEAR_MIX &&
       tail != SA_TAIL_FIRST_ORDER)
     return fail(SA_ERR_INVALID_ARG, "sa_sparse_attn_fwd: unknown tail mode");

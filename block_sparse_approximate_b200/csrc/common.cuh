@@ -62,6 +62,12 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// SPLA's exponential feature map φ(x) = e^x (§2.3).  Every kernel that forms
+// Σ φ(k) vᵀ or φ(q)·φ(k) calls this one function, so the all-token state
+// and the selected blocks' correction that is subtracted from it use the
+// same values.
+__device__ __forceinline__ float phi_exp(float x) { return __expf(x); }
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

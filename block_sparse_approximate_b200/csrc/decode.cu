@@ -46,7 +46,7 @@ constexpr int kRingC = 3;
 constexpr int kItabSegs = 64;
 
 struct DecodeLayout {
-  size_t scores_off, idx_off, parta_off, partc_off, total;
+  size_t scores_off, idx_off, parta_off, partc_off, partr_off, total;
   int nsegA, nsegC;
 };
 
@@ -63,6 +63,17 @@ DecodeLayout decode_layout(const sa_decode_shape& s, int topk) {
   L.parta_off = L.idx_off + align256((size_t)s.B * s.Hkv * (topk > 0 ? topk : 1) * sizeof(int32_t));
   L.partc_off = L.parta_off + align256((size_t)s.B * s.Hq * (L.nsegA > 0 ? L.nsegA : 1) * part);
   L.total = L.partc_off + align256((size_t)s.B * s.Hq * (L.nsegC > 0 ? L.nsegC : 1) * part);
+  // residual linear tail: per (query head, exact segment) the selected
+  // tokens' Σ (φ(q)·φ(k_n)) v_n, over the statistics pass's partial states
+  // (which that tail does not read) when they fit there, else appended
+  const size_t partr = (size_t)s.B * s.Hq * (L.nsegC > 0 ? L.nsegC : 1) * s.d * sizeof(float);
+  const size_t parta = (size_t)s.B * s.Hq * (L.nsegA > 0 ? L.nsegA : 1) * part;
+  if (partr <= parta) {
+    L.partr_off = L.parta_off;
+  } else {
+    L.partr_off = L.total;
+    L.total += align256(partr);
+  }
   return L;
 }
 
@@ -128,6 +139,13 @@ __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;"
 __device__ __forceinline__ uint32_t pack2bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// SPLA's feature map φ = exp on both halves of a packed bf16 pair, rounded
+// back to bf16 (the same rounding as the all-token state in sa_block_pool)
+__device__ __forceinline__ uint32_t phi_bf16x2(uint32_t x) {
+  const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&x));
+  return pack2bf16(phi_exp(f.x), phi_exp(f.y));
 }
 
 // Partial online-softmax state of one query head in a warp: log2-domain max,
@@ -590,6 +608,16 @@ __device__ __forceinline__ void mma16816_full(float (&d)[4], uint32_t a0, uint32
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
 }
+// The same MMA when rows 8-15 of A are zero: only d0, d1 (row lane / 4) are
+// kept; the other two outputs go to scratch registers.
+__device__ __forceinline__ void mma16816_top(float (&d)[2], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
+  float x2, x3;
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%10,%10};"
+      : "+f"(d[0]), "+f"(d[1]), "=f"(x2), "=f"(x3)
+      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1), "f"(0.f));
+}
 __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
@@ -601,12 +629,12 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
                : "r"(addr));
 }
 
-template <int D>
+template <int D, bool RLA>
 __global__ void __launch_bounds__(kDecThreads, 1)
 decode_exact_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ Kc,
                     const __nv_bfloat16* __restrict__ Vc, int Hq, int Hkv, int N, int blk,
                     const int32_t* __restrict__ idx, int topk, float scale, int nsegC, int npairs,
-                    float* __restrict__ partc) {
+                    float* __restrict__ partc, float* __restrict__ partr) {
   pdl_wait();
   constexpr int CH = D / 8;                         // 16-byte chunks per bf16 row
   constexpr int NT = D / 8;                         // n-tiles of 8 channels
@@ -693,8 +721,10 @@ decode_exact_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
   for (int r = 0; r < kRingC - 1; ++r) prefetch();
 
   uint32_t qa0[KS], qa2[KS];                  // Q A-fragments (rows = heads)
+  uint32_t fa0[RLA ? KS : 1], fa2[RLA ? KS : 1];   // φ(Q) A-fragments (residual linear tail)
   float m_run = -INFINITY, l_run = 0.f;
-  float o[NT][4];
+  float o[NT][2];                             // rows 8-15 of the MMA are empty
+  float o2[RLA ? NT : 1][2];                  // Σ (φ(q)·φ(k_n)) v_n of the warp's tokens
   int cur_seg_k = 0, cur_sub = 0, cur_pair = -1, slot = 0;
   while (seg_of(cur_seg_k) < total_segs) {
     const int seg = seg_of(cur_seg_k);
@@ -709,6 +739,10 @@ decode_exact_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
           const uint32_t hi = *reinterpret_cast<const uint32_t*>(qrow + 16 * kk + 8 + 2 * (lane & 3));
           qa0[kk] = hvalid ? lo : 0u;
           qa2[kk] = hvalid ? hi : 0u;
+          if (RLA) {
+            fa0[kk] = hvalid ? phi_bf16x2(lo) : 0u;
+            fa2[kk] = hvalid ? phi_bf16x2(hi) : 0u;
+          }
         }
         cur_pair = pair;
       }
@@ -717,7 +751,13 @@ decode_exact_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) o[nt][e] = 0.f;
+        for (int e = 0; e < 2; ++e) o[nt][e] = 0.f;
+      if (RLA) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) o2[RLA ? nt : 0][e] = 0.f;
+      }
     }
     prefetch();
     cp_async_wait<kRingC - 1>();
@@ -729,6 +769,7 @@ decode_exact_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
     const int tok0 = tb + (lane & 7), tok1 = tb + 8 + (lane & 7);   // rows this lane addresses
     // S = Q Kᵀ for the warp's two 8-token n-tiles
     float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+    float w0[4] = {0.f, 0.f, 0.f, 0.f}, w1[4] = {0.f, 0.f, 0.f, 0.f};   // φ(q)·φ(k_n)
 #pragma unroll
     for (int kp = 0; kp < KS / 2; ++kp) {
       uint32_t kf[4], kg[4];
@@ -739,6 +780,20 @@ decode_exact_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
       mma16816_full(s0, qa0[2 * kp + 1], qa2[2 * kp + 1], kf[2], kf[3]);
       mma16816_full(s1, qa0[2 * kp], qa2[2 * kp], kg[0], kg[1]);
       mma16816_full(s1, qa0[2 * kp + 1], qa2[2 * kp + 1], kg[2], kg[3]);
+      if (RLA) {
+        // the same fragments through the feature map (zero-filled rows give
+        // φ = 1, but their V rows are zero)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          kf[e] = phi_bf16x2(kf[e]);
+          kg[e] = phi_bf16x2(kg[e]);
+        }
+        const int kq = RLA ? 2 * kp : 0;
+        mma16816_full(w0, fa0[kq], fa2[kq], kf[0], kf[1]);
+        mma16816_full(w0, fa0[kq + 1], fa2[kq + 1], kf[2], kf[3]);
+        mma16816_full(w1, fa0[kq], fa2[kq], kg[0], kg[1]);
+        mma16816_full(w1, fa0[kq + 1], fa2[kq + 1], kg[2], kg[3]);
+      }
     }
     // online softmax of the warp's 16 tokens for head hrow (tokens past the
     // stage's valid count are zero-filled rows: masked out)
@@ -759,6 +814,7 @@ decode_exact_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
     m_run = m_new;
     // P as the A fragment: k 0-7 = the first n-tile's tokens, k 8-15 the second's
     const uint32_t pa0 = pack2bf16(p0, p1), pa2 = pack2bf16(p2, p3);
+    const uint32_t wa0 = RLA ? pack2bf16(w0[0], w0[1]) : 0u, wa2 = RLA ? pack2bf16(w1[0], w1[1]) : 0u;
     // O += P V over the 16 tokens
 #pragma unroll
     for (int nq = 0; nq < NT / 4; ++nq) {
@@ -771,7 +827,8 @@ decode_exact_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
         float* oo = o[4 * nq + e];
         oo[0] *= corr;
         oo[1] *= corr;
-        mma16816_full(o[4 * nq + e], pa0, pa2, vf[e], vg[e]);
+        mma16816_top(o[4 * nq + e], pa0, pa2, vf[e], vg[e]);
+        if (RLA) mma16816_top(o2[RLA ? 4 * nq + e : 0], wa0, wa2, vf[e], vg[e]);
       }
     }
     __syncthreads();
@@ -819,6 +876,26 @@ decode_exact_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
         out[2 + c] = A;
       }
       __syncthreads();
+      if (RLA) {
+        // the residual linear sums add without a maximum: sum the warps'
+        if (hvalid) {
+          float* mw = mg + ((size_t)warp * kMaxGroup + hrow) * (D + 2);
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            mw[8 * nt + 2 * (lane & 3)] = o2[RLA ? nt : 0][0];
+            mw[8 * nt + 2 * (lane & 3) + 1] = o2[RLA ? nt : 0][1];
+          }
+        }
+        __syncthreads();
+        for (int x = tid; x < g * D; x += kDecThreads) {
+          const int hh = x / D, c = x % D;
+          float A = 0.f;
+#pragma unroll
+          for (int w = 0; w < kDecWarps; ++w) A += mg[((size_t)w * kMaxGroup + hh) * (D + 2) + c];
+          partr[(((size_t)b * Hq + kh * g + hh) * nsegC + sseg) * D + c] = A;
+        }
+        __syncthreads();
+      }
       cur_sub = 0;
       ++cur_seg_k;
     }
@@ -843,13 +920,14 @@ decode_exact_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
 // weight, then the parts' sums; loads that do not depend on one another are
 // issued together.
 constexpr int kParts = 4;
+constexpr float kRmsEps = 1e-6f;     // RMSNorm of SPLA's residual linear output
 
 template <int D>
 __global__ void __launch_bounds__(kParts * D)
 decode_combine_kernel(const float* __restrict__ parta, int nsegA, const float* __restrict__ partc, int nsegC,
-                      int use_tail, const __nv_bfloat16* __restrict__ q, sa_block_stats st,
-                      const int32_t* __restrict__ idx, int topk, int nb, int blk, float scale, int Hq, int Hkv,
-                      __nv_bfloat16* __restrict__ O) {
+                      int use_tail, const float* __restrict__ partr, const __nv_bfloat16* __restrict__ q,
+                      sa_block_stats st, const int32_t* __restrict__ idx, int topk, int nb, int blk, float scale,
+                      int Hq, int Hkv, __nv_bfloat16* __restrict__ O) {
   pdl_wait();
   constexpr int kT = kParts * D, kW = kT / 32;
   extern __shared__ __align__(16) float csm[];
@@ -862,6 +940,7 @@ decode_combine_kernel(const float* __restrict__ parta, int nsegA, const float* _
   float* hf = hl + ns;                                     // [ns] merge weights
   float* xsel = hf + ns;                                   // [nsel] log2 zero-order weights
   int* jsel = reinterpret_cast<int*>(xsel + nsel);         // [nsel] block indices
+  float* rr = reinterpret_cast<float*>(jsel + nsel);        // [kParts][D] residual parts, [D/32] squares
   const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
   const int c = tid % D, pt = tid / D;
   const int lane = tid & 31, warp = tid >> 5;
@@ -954,7 +1033,23 @@ decode_combine_kernel(const float* __restrict__ parta, int nsegA, const float* _
   }
   red[(pt * 2 + 0) * D + c] = L;
   red[(pt * 2 + 1) * D + c] = A;
+  if (partr) {
+    // SPLA's residual: this part's rows r of φ(q)ᵀ S_all (column c) minus its
+    // exact segments' Σ (φ(q)·φ(k_n)) v_n
+    float rpart = 0.f;
+    const float* sa = st.sexp + (size_t)pair * D * D;
+    const __nv_bfloat16* qh = q + ((size_t)b * Hq + h) * D;
+    // φ(q) rounded to bf16 as in the exact pass's operand, so that the two
+    // terms of the difference use the same feature values
+    for (int r = pt; r < D; r += kParts)
+      rpart = fmaf(__bfloat162float(__float2bfloat16_rn(phi_exp(__bfloat162float(qh[r])))), sa[(size_t)r * D + c],
+                   rpart);
+    const float* pr = partr + ((size_t)b * Hq + h) * nsegC * D;
+    for (int x = pt; x < nsegC; x += kParts) rpart -= pr[(size_t)x * D + c];
+    rr[pt * D + c] = rpart;
+  }
   __syncthreads();
+  float o_s = 0.f, res = 0.f;
   if (pt == 0) {
     L = 0.f;
     A = 0.f;
@@ -963,8 +1058,23 @@ decode_combine_kernel(const float* __restrict__ parta, int nsegA, const float* _
       L += red[(p2 * 2 + 0) * D + c];
       A += red[(p2 * 2 + 1) * D + c];
     }
-    O[((size_t)b * Hq + h) * D + c] = __float2bfloat16_rn(L > 0.f ? A / L : 0.f);
+    o_s = L > 0.f ? A / L : 0.f;
+    if (partr) {
+#pragma unroll
+      for (int p2 = 0; p2 < kParts; ++p2) res += rr[p2 * D + c];
+    }
   }
+  if (partr) {
+    // RMSNorm over the D channels (threads of part 0 = warps 0 .. D/32 - 1)
+    const float sq = warp_sum(res * res);
+    if (lane == 0 && warp < D / 32) rr[kParts * D + warp] = sq;
+    __syncthreads();
+    float tot = 0.f;
+#pragma unroll
+    for (int w = 0; w < D / 32; ++w) tot += rr[kParts * D + w];
+    res *= rsqrtf(tot / D + kRmsEps);
+  }
+  if (pt == 0) O[((size_t)b * Hq + h) * D + c] = __float2bfloat16_rn(o_s + res);
 }
 
 // Launch with programmatic stream serialization (the kernel calls pdl_wait()
@@ -1010,6 +1120,11 @@ sa_status launch_decode(const void* q, const void* Kc, const void* Vc, const sa_
   int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(ws + L.idx_off);
   float* parta = reinterpret_cast<float*>(ws + L.parta_off);
   float* partc = reinterpret_cast<float*>(ws + L.partc_off);
+  // residual linear tail: with every block selected U is empty and the
+  // residual is zero by definition (the difference S_all − S_sel would only
+  // hold rounding noise, which the RMS norm would blow up to unit size)
+  const bool rla = tail == SA_TAIL_RESIDUAL_LINEAR;
+  float* partr = rla ? reinterpret_cast<float*>(ws + L.partr_off) : nullptr;
   const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(q);
   const int sms = sm_count();
 
@@ -1052,15 +1167,15 @@ sa_status launch_decode(const void* q, const void* Kc, const void* Vc, const sa_
     const size_t smemC = sizeof(float) * kDecWarps * kMaxGroup * (D + 2) +
                          sizeof(int) * kItabSegs * (kSegC * kStageTokC / 64) +
                          (size_t)kRingC * 2 * kStageTokC * D * 2;
-    if (cudaFuncSetAttribute(decode_exact_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smemC) !=
-        cudaSuccess)
+    auto kern = rla ? decode_exact_kernel<D, true> : decode_exact_kernel<D, false>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smemC) != cudaSuccess)
       return launch_status("cudaFuncSetAttribute(decode_exact_kernel)");
     const long segsC = (long)npairs * L.nsegC;   // < 2^31 for any supported shape
     const int gridC = (int)(segsC < sms ? segsC : sms);
     {
-      const cudaError_t le = launch_pdl(decode_exact_kernel<D>, dim3(gridC), dim3(kDecThreads), smemC, stream,
+      const cudaError_t le = launch_pdl(kern, dim3(gridC), dim3(kDecThreads), smemC, stream,
         qb, static_cast<const __nv_bfloat16*>(Kc), static_cast<const __nv_bfloat16*>(Vc), s.Hq, s.Hkv, s.N,
-        s.block, idx, topk, scale, L.nsegC, npairs, partc);
+        s.block, idx, topk, scale, L.nsegC, npairs, partc, partr);
       if (le != cudaSuccess) return fail(SA_ERR_CUDA, std::string("decode_exact_kernel: ") + cudaGetErrorString(le));
     }
     r = launch_status("decode_exact_kernel");
@@ -1073,13 +1188,15 @@ sa_status launch_decode(const void* q, const void* Kc, const void* Vc, const sa_
     const int nsc = topk > 0 ? L.nsegC : 0;
     const int ns = (use_tail ? L.nsegA : 0) + nsc;
     const int nsel = (use_tail && nsc > 0) ? topk : 0;
-    const size_t smemD = sizeof(float) * (kParts * 2 * D + 3 * (size_t)ns + 2 * (size_t)nsel);
+    const size_t smemD = sizeof(float) * (kParts * 2 * D + 3 * (size_t)ns + 2 * (size_t)nsel +
+                                          (rla ? kParts * D + D / 32 : 0));
     if (cudaFuncSetAttribute(decode_combine_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smemD) !=
         cudaSuccess)
       return launch_status("cudaFuncSetAttribute(decode_combine_kernel)");
     {
       const cudaError_t le = launch_pdl(decode_combine_kernel<D>, dim3(s.Hq, s.B), dim3(kParts * D), smemD, stream,
-        parta, L.nsegA, partc, nsc, use_tail, qb, st, idx, topk, nb, s.block, scale, s.Hq, s.Hkv,
+        parta, L.nsegA, partc, nsc, use_tail, topk < nb ? partr : nullptr, qb, st, idx, topk, nb, s.block, scale,
+        s.Hq, s.Hkv,
         static_cast<__nv_bfloat16*>(O));
       if (le != cudaSuccess) return fail(SA_ERR_CUDA, std::string("decode_combine_kernel: ") + cudaGetErrorString(le));
     }
@@ -1130,11 +1247,15 @@ extern "C" sa_status sa_decode_fwd(const void* q, const void* Kcache, const void
   sa_status r = check_decode_shape(shape, topk);
   if (r != SA_OK) return r;
   if (dtype != SA_BF16) return fail(SA_ERR_UNSUPPORTED, "sa_decode_fwd: bf16 caches only");
-  if (tail != SA_TAIL_ZERO_ORDER && tail != SA_TAIL_DROP)
-    return fail(SA_ERR_UNSUPPORTED, "sa_decode_fwd: tail must be SA_TAIL_DROP or SA_TAIL_ZERO_ORDER");
+  if (tail != SA_TAIL_ZERO_ORDER && tail != SA_TAIL_DROP && tail != SA_TAIL_RESIDUAL_LINEAR)
+    return fail(SA_ERR_UNSUPPORTED,
+                "sa_decode_fwd: tail must be SA_TAIL_DROP, SA_TAIL_ZERO_ORDER or SA_TAIL_RESIDUAL_LINEAR");
   if (!q || !Kcache || !Vcache || !O || !stats || !stats->kmean || !stats->kvar || !stats->vsum)
     return fail(SA_ERR_INVALID_ARG, "sa_decode_fwd: q, caches, O and stats (kmean, kvar, vsum) are required");
-  const void* ptrs[] = {q, Kcache, Vcache, O, stats->kmean, stats->kvar, stats->vsum, block_idx_out, scores_out};
+  if (tail == SA_TAIL_RESIDUAL_LINEAR && !stats->sexp)
+    return fail(SA_ERR_INVALID_ARG, "sa_decode_fwd: SA_TAIL_RESIDUAL_LINEAR needs stats->sexp");
+  const void* ptrs[] = {q, Kcache, Vcache, O, stats->kmean, stats->kvar, stats->vsum, stats->sexp, block_idx_out,
+                        scores_out};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return fail(SA_ERR_ALIGNMENT, "sa_decode_fwd: pointers must be 16-byte aligned");
   const size_t need = decode_layout(shape, topk).total;

@@ -25,6 +25,9 @@ long-context LLM decoding; these synthetic inputs stand in for them):
                 131072 tokens: K, V ~ N(0,1) plus an N(0, 0.5) offset per
                 (64-token block, channel); q ~ N(0,1); block 64; taylor2 router,
                 top-64 blocks; zero-order tail.
+* ``decode_rla``  ``decode`` (same seed, same caches) with SPLA's residual
+                linear attention over the unselected blocks instead of the
+                zero-order tail.
 
 N(m, v) above names the variance v.
 """
@@ -97,6 +100,9 @@ WORKLOADS = {
     "decode": Workload("decode", B=16, H=32, N=131072, d=128, dtype="bf16",
                        block=64, route="taylor2", tail="zero_order", seed=4,
                        topk=64, decode=True, Hkv=8),
+    "decode_rla": Workload("decode_rla", B=16, H=32, N=131072, d=128, dtype="bf16",
+                           block=64, route="taylor2", tail="residual_linear", seed=4,
+                           topk=64, decode=True, Hkv=8),
 }
 
 _DT = {"fp32": torch.float32, "bf16": torch.bfloat16}

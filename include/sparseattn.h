@@ -70,10 +70,17 @@ typedef enum {
   SA_TAIL_LINEAR_MIX = 2,  /* O = α⊙O_s + (1−α)⊙O_l, O_l = ReLU linear
                               attention over the unselected blocks
                               [SLA2 §2A, SALAD §2, SPLA §2.2] */
-  SA_TAIL_FIRST_ORDER = 3  /* PISA hybrid order: the zero-order terms plus
+  SA_TAIL_FIRST_ORDER = 3, /* PISA hybrid order: the zero-order terms plus
                               the global first-order correction of the
                               numerator, (s q) H̄ Σ_{j∈U} e^{s q·k̄_j}
                               [PISA §2 "Algoritmo Central"] */
+  SA_TAIL_RESIDUAL_LINEAR = 4  /* decode only: o = O_s + RMSNorm(o_rla),
+                              O_s the DROP output, o_rla = φ(q)ᵀ Σ_{n∈U}
+                              φ(k_n) v_nᵀ with φ = exp, formed as
+                              φ(q)ᵀ S_all − Σ_{n∈S} (φ(q)·φ(k_n)) v_n from
+                              the tiles the exact pass loads; RMSNorm(x) =
+                              x / sqrt(mean(x²) + 1e-6), unit gain
+                              [SPLA §2.2 subtraction form, §2.3] */
 } sa_tail_mode;
 
 /* Shape of a prefill problem: Q, K, V, O are [B, H, N, d]; query blocks and
@@ -109,9 +116,13 @@ typedef struct {
   uint16_t* hbarT_bf16;  /* [B,H,d,d] bf16 of H̄ᵀ (row e, column c; the
                        tensor-core first-order tail)                        */
   float* covnorm;   /* [B,H,nb]    M_j = ‖H_j − H̄‖₂, the spectral norm of each
-                       block's first-order deviation from the mean (power
-                       iteration to 1e-6 relative on the Gram matrix)
+                       block's first-order deviation from the mean (Lanczos
+                       on the Gram matrix to 1e-6 relative)
                        [PISA §2 "Roteamento Consciente de Covariância"]    */
+  float* sexp;      /* [B,H,d,d]   S_all = Σ_n φ(k_n) v_nᵀ over all tokens, φ = exp
+                       (bf16-rounded on the tensor-core path, as the decode
+                       kernel rounds φ(k) of the selected blocks)
+                       [SPLA §2.2, the residual linear state]              */
 } sa_block_stats;
 
 /* Block statistics of Q (optional), K and V.

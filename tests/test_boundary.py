@@ -110,6 +110,8 @@ def test_sparse_attn_validation(lib):
     assert f(FAKE, FAKE, FAKE, 1, sh, FAKE, 2, 3, None, ctypes.byref(zo), 0.1, FAKE, None) \
         == bd.SA_ERR_INVALID_ARG            # first_order without hbar
     assert f(FAKE, FAKE, FAKE, 1, sh, FAKE, 2, 4, None, ctypes.byref(zo), 0.1, FAKE, None) \
+        == bd.SA_ERR_UNSUPPORTED            # residual_linear is a decode tail
+    assert f(FAKE, FAKE, FAKE, 1, sh, FAKE, 2, 5, None, ctypes.byref(zo), 0.1, FAKE, None) \
         == bd.SA_ERR_INVALID_ARG            # unknown tail mode
 
 
@@ -126,6 +128,11 @@ def test_decode_validation_and_workspace(lib):
         == bd.SA_ERR_UNSUPPORTED            # fp32 caches
     assert f(FAKE, FAKE, FAKE, 1, sh, ctypes.byref(st), 64, 0.1, 2, None, None, FAKE, FAKE, ws, None) \
         == bd.SA_ERR_UNSUPPORTED            # linear_mix decode
+    assert f(FAKE, FAKE, FAKE, 1, sh, ctypes.byref(st), 64, 0.1, 4, None, None, FAKE, FAKE, ws, None) \
+        == bd.SA_ERR_INVALID_ARG            # residual_linear without stats->sexp
+    # the residual partial sums fit over the statistics pass's partial states
+    # here, so the workspace (and the static scratch bound) does not grow
+    assert ws < 8 * 2 ** 20
     assert f(FAKE, FAKE, FAKE, 1, sh, ctypes.byref(st), 5000, 0.1, 1, None, None, FAKE, FAKE, ws, None) \
         == bd.SA_ERR_INVALID_ARG
     assert f(FAKE, FAKE, FAKE, 1, sh, ctypes.byref(st), 64, 0.1, 1, None, None, FAKE, FAKE + 16, ws, None) \

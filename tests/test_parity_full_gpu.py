@@ -54,10 +54,12 @@ def test_prefill_full_size_sampled(lib, name):
     assert_tol(got, ref, BF16_TOL, name)
 
 
-def test_decode_full_size_sampled(lib):
-    w = wl.WORKLOADS["decode"]
+@pytest.mark.parametrize("name", ["decode", "decode_rla"])
+def test_decode_full_size_sampled(lib, name):
+    w = wl.WORKLOADS[name]
     inp = wl.decode_inputs(w, DEV)
-    st = bd.block_pool(None, inp["Kcache"], inp["Vcache"], w.block, variance=True)
+    st = bd.block_pool(None, inp["Kcache"], inp["Vcache"], w.block, variance=True,
+                       residual=(w.tail == "residual_linear"))
     step = DecodeStep(w, inp, st)
     o = step()
     torch.cuda.synchronize()
@@ -69,7 +71,7 @@ def test_decode_full_size_sampled(lib):
         Kh = inp["Kcache"][b:b + 1, kh:kh + 1].cpu().float().numpy()
         Vh = inp["Vcache"][b:b + 1, kh:kh + 1].cpu().float().numpy()
         ref_o, _, ref_sc = oracle.decode_attention(q[b:b + 1, kh * g:(kh + 1) * g], Kh, Vh, w.block,
-                                                   w.k, w.scale,
+                                                   w.k, w.scale, tail=w.tail,
                                                    block_idx=step.idx[b:b + 1, kh:kh + 1].cpu().numpy())
         selection_agreement(np64(step.scores[b, kh]), ref_sc[0, 0], w.k)  # asserts on clear gaps
         assert_tol(np64(o[b, kh * g:(kh + 1) * g]), ref_o[0], BF16_TOL, f"decode b={b} g={kh}")

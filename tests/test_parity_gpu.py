@@ -269,7 +269,7 @@ def test_value_shift_on_gpu(lib):
 # decode
 # --------------------------------------------------------------------------
 
-@pytest.mark.parametrize("tail", ["zero_order", "drop"])
+@pytest.mark.parametrize("tail", ["zero_order", "drop", "residual_linear"])
 @pytest.mark.parametrize("B,Hq,Hkv,N,d,block,k", [
     (2, 8, 2, 8192, 128, 64, 16),
     (1, 4, 4, 4096, 128, 128, 5),
@@ -285,7 +285,7 @@ def test_decode(lib, tail, B, Hq, Hkv, N, d, block, k):
     Kc = (torch.randn(B, Hkv, N // block, block, d, generator=g, device=DEV)
           + 0.7 * torch.randn(B, Hkv, N // block, 1, d, generator=g, device=DEV)).reshape(B, Hkv, N, d).to(torch.bfloat16)
     Vc = torch.randn(B, Hkv, N, d, generator=g, device=DEV).to(torch.bfloat16)
-    st = bd.block_pool(None, Kc, Vc, block, variance=True)
+    st = bd.block_pool(None, Kc, Vc, block, variance=True, residual=(tail == "residual_linear"))
     s = 1 / math.sqrt(d)
     o, idx, sc = bd.decode_fwd(q, Kc, Vc, st, block, k, s, tail=tail)
     torch.cuda.synchronize()
@@ -295,7 +295,27 @@ def test_decode(lib, tail, B, Hq, Hkv, N, d, block, k):
     ref_o, _, _ = oracle.decode_attention(np64(q), np64(Kc), np64(Vc), block, k, s, tail=tail,
                                           block_idx=idx.cpu().numpy())
     assert_tol(np64(o), ref_o, BF16_TOL, f"decode {tail}")
+    assert_no_device_error()
     del w
+
+
+def test_block_pool_sexp(lib):
+    # SPLA's all-token state Σ_n exp(k_n) v_nᵀ: tensor-core path (bf16, d = 128,
+    # φ(k) rounded to bf16) and CUDA-core path (fp32)
+    for dtype, d, tol in ((torch.bfloat16, 128, 5e-3), (torch.float32, 64, 1e-5)):
+        Q, K, V = _gauss(2, 2, 1024, d, dtype, 17)
+        st = bd.block_pool(None, K, V, 64, residual=True)
+        ref = np.einsum("bhnc,bhne->bhce", np.exp(np64(K)), np64(V))
+        assert_stats_close(st["sexp"], ref, f"sexp {dtype}", rtol=tol)
+
+
+def test_residual_linear_prefill_is_rejected(lib):
+    Q = torch.zeros(1, 1, 256, 128, device=DEV, dtype=torch.bfloat16)
+    st = bd.block_pool(Q, Q, Q, 128, residual=True)
+    idx, _ = bd.route(st, (1, 1, 256, 128, 128), "dot", 1)
+    with pytest.raises(bd.SparseAttnError) as e:
+        bd.sparse_attn_fwd(Q, Q, Q, idx, 128, "residual_linear", st, 0.1)
+    assert e.value.status == bd.SA_ERR_UNSUPPORTED
 
 
 # --------------------------------------------------------------------------
