@@ -202,7 +202,9 @@ __device__ __forceinline__ void load_lane(float (&r)[CPL], const float* row, int
 
 constexpr int kWarpBlocksA = kStageBlocksA / (kThrA / 32);   // blocks of a stage per warp
 
-template <int D, int G>
+// ZT: the zero-order tail is wanted (its value sums are copied and its
+// online state kept); without it the pass only scores the blocks.
+template <int D, int G, bool ZT>
 __global__ void __launch_bounds__(kThrA, 2)
 decode_stats_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int Hq, int Hkv, int nb, int blk,
                     float scale, int nsegA, int npairs, float* __restrict__ scores, float* __restrict__ parta) {
@@ -238,10 +240,10 @@ decode_stats_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int 
     // the slot's previous contents were read by generic loads before the
     // barrier that precedes this call; order them before the async writes
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    dbar_expect_tx(fb, 3 * bytes);
+    dbar_expect_tx(fb, (ZT ? 3 : 2) * bytes);
     bulk_copy(dst, st.kmean + goff, bytes, fb);
     bulk_copy(dst + kArrB, st.kvar + goff, bytes, fb);
-    bulk_copy(dst + 2 * kArrB, st.vsum + goff, bytes, fb);
+    if (ZT) bulk_copy(dst + 2 * kArrB, st.vsum + goff, bytes, fb);
   };
 
   if (seg_of(0) >= total_segs) return;
@@ -366,6 +368,7 @@ decode_stats_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int 
 #pragma unroll
       for (int o = 2; o < 2 * G; o <<= 1) se += __shfl_xor_sync(0xffffffffu, se, o);
       if (live && hl == 0) scores[(size_t)pair * nb + j0 + jj] = mx + logf(se);
+      if (!ZT) continue;
       // zero-order term: log2 weight of the pseudo-key (value vsum / B)
       const float x = live ? d1 + bias2 : -INFINITY;
       float bm = x;
@@ -409,7 +412,7 @@ decode_stats_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int 
     slot = (slot + 1) % kRingA;
     // end of segment: merge the warps' states per head and write them
     const bool seg_end = ++cur_sub >= stages_in(seg);
-    if (seg_end) {
+    if (ZT && seg_end) {
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         float* mw = mg + (warp * G + h) * (D + 2);
@@ -423,7 +426,7 @@ decode_stats_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int 
     }
     __syncthreads();   // the ring slot is reused by the next prefetch; the merge rows are complete
     if (seg_end) {
-      for (int x = tid; x < G * D; x += kThrA) {
+      for (int x = tid; ZT && x < G * D; x += kThrA) {
         const int h = x / D, c = x % D;
         float M = -INFINITY;
 #pragma unroll
@@ -446,7 +449,7 @@ decode_stats_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int 
         }
         out[2 + c] = A;
       }
-      __syncthreads();   // the merge rows are rewritten at the next segment end
+      if (ZT) __syncthreads();   // the merge rows are rewritten at the next segment end
       cur_sub = 0;
       ++cur_seg_k;
     }
@@ -1144,10 +1147,11 @@ sa_status launch_decode(const void* q, const void* Kc, const void* Vc, const sa_
       kern<<<gridA, kThrA, smemA, stream>>>(qb, st, s.Hq, s.Hkv, nb, s.block, scale, L.nsegA, npairs, scores, parta);
       r0 = launch_status("decode_stats_kernel");
     };
-    if (g == 1) run(decode_stats_kernel<D, 1>);
-    else if (g == 2) run(decode_stats_kernel<D, 2>);
-    else if (g == 4) run(decode_stats_kernel<D, 4>);
-    else run(decode_stats_kernel<D, 8>);
+    const bool zt = tail == SA_TAIL_ZERO_ORDER;
+    if (g == 1) run(zt ? decode_stats_kernel<D, 1, true> : decode_stats_kernel<D, 1, false>);
+    else if (g == 2) run(zt ? decode_stats_kernel<D, 2, true> : decode_stats_kernel<D, 2, false>);
+    else if (g == 4) run(zt ? decode_stats_kernel<D, 4, true> : decode_stats_kernel<D, 4, false>);
+    else run(zt ? decode_stats_kernel<D, 8, true> : decode_stats_kernel<D, 8, false>);
     if (r0 != SA_OK) return r0;
   }
   sa_status r = SA_OK;
