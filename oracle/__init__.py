@@ -15,6 +15,7 @@ definitions on the pages it cites:
           Eficientes"
 * [SPLA]  "SPLA - Block Sparse Plus Linear Attention para Modelagem de
           Contexto Longo"
+* [SFA]   "Scaling Attention via Feature Sparsity" (feature_sparse.py)
 
 Pinning status of each public function (what fixes it other than itself) is
 listed in ``oracle.sparse_attention.__doc__``.
@@ -32,3 +33,4 @@ from .sparse_attention import (  # noqa: F401
     quantise_blocks_e4m3,
     fp8_attention,
 )
+from .feature_sparse import sfa_codes, sfa_densify, sfa_attention  # noqa: F401
