@@ -352,6 +352,53 @@ def time_pisa(steps: int = 10, warmup: int = 3):
     return out
 
 
+def time_sfa(steps: int = 10, warmup: int = 3):
+    """Sparse feature attention: top-16 feature codes of Q and K (zero-filled
+    rows written by the encoder) and the online-softmax attention over every
+    KV tile.  FLOPs counted as dense attention (4·N²·d per head): the tensor
+    cores run the zero-filled operands at full width."""
+    from block_sparse_approximate_b200 import binding as bd
+    w = wl.WORKLOADS["sfa"]
+    inp = wl.prefill_inputs(w, "cuda")
+    kf = w.extra["kf"]
+    Q, K, V = inp["Q"], inp["K"], inp["V"]
+    lib = bd.load()
+    shape = bd.Shape(w.B, w.H, w.N, w.d, w.block)
+    ws = torch.empty(max(int(lib.sa_sfa_workspace_size(shape)), 256), device="cuda", dtype=torch.uint8)
+    qv = torch.empty(Q.shape[:-1] + (kf,), device="cuda", dtype=torch.bfloat16)
+    qi = torch.empty(Q.shape[:-1] + (kf,), device="cuda", dtype=torch.uint8)
+    kv, ki = torch.empty_like(qv), torch.empty_like(qi)
+    Qs, Ks, O = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(Q)
+    rows = Q.numel() // w.d
+
+    def encode():
+        st = bd._stream(None)
+        bd._check("sa_sfa_encode", lib.sa_sfa_encode(Q.data_ptr(), rows, w.d, kf, qv.data_ptr(), qi.data_ptr(),
+                                                     Qs.data_ptr(), st))
+        bd._check("sa_sfa_encode", lib.sa_sfa_encode(K.data_ptr(), rows, w.d, kf, kv.data_ptr(), ki.data_ptr(),
+                                                     Ks.data_ptr(), st))
+
+    def attn():
+        bd._check("sa_sfa_attn_fwd", lib.sa_sfa_attn_fwd(Qs.data_ptr(), Ks.data_ptr(), V.data_ptr(), bd.SA_BF16,
+                                                         shape, float(w.scale), O.data_ptr(), ws.data_ptr(),
+                                                         ws.numel(), bd._stream(None)))
+
+    def step():
+        encode()
+        attn()
+
+    ms_step, attn_ms = _time_prefill_variant(step, attn, steps, warmup)
+    _, bf16, _, src = _peaks()
+    fl = dense_flops(w)
+    ach = fl / (attn_ms * 1e-3) / 1e12
+    out = {"workload": w.name, "kf": kf, "ms_per_step": ms_step, "attn_ms": attn_ms, "encode_ms": ms_step - attn_ms,
+           "executed_tflops": ach, "peak_tflops": bf16, "frac": ach / bf16, "peak_source": f"{src} bf16 burst",
+           "step": "sfa_encode (Q, K) + sfa_attn_fwd over every KV tile"}
+    del inp, Q, K, V, Qs, Ks, O
+    torch.cuda.empty_cache()
+    return out
+
+
 def linear_mix_flops(w) -> float:
     """Per query block: exact softmax part 4·d·(k·B)·B, the A_i accumulation
     2·d²·(k·B) and the final relu(Q)(H_tot − A_i) 2·d²·B."""
@@ -406,6 +453,10 @@ def run_ours(args, world, rank, local):
     if args.only == "sla2":
         if rank == 0:
             print(json.dumps({"sla2_mix": time_sla2(args.steps, args.warmup)}), flush=True)
+        return 0
+    if args.only == "sfa":
+        if rank == 0:
+            print(json.dumps({"sfa": time_sfa(args.steps, args.warmup)}), flush=True)
         return 0
     if args.only == "pisa":
         if rank == 0:
@@ -499,7 +550,7 @@ def run_ours(args, world, rank, local):
                "h2d_bytes_per_step": sum(inp[n].numel() * inp[n].element_size() for n in ("Q", "K", "V")),
                "d2h_bytes_per_step": step.buf.out.numel() * step.buf.out.element_size()}
 
-    decode = decode_rla = fp8 = sla2 = pisa = None
+    decode = decode_rla = fp8 = sla2 = pisa = sfa = None
     if rank == 0 and args.only == "all" and not args.no_decode:
         del step
         torch.cuda.empty_cache()
@@ -508,6 +559,7 @@ def run_ours(args, world, rank, local):
         fp8 = time_fp8()
         sla2 = time_sla2()
         pisa = time_pisa()
+        sfa = time_sfa()
     ck = clocks.stop() if clocks else None
 
     if rank != 0:
@@ -543,6 +595,7 @@ def run_ours(args, world, rank, local):
         "fp8": fp8,
         "sla2_mix": sla2,
         "pisa": pisa,
+        "sfa": sfa,
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -561,7 +614,7 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
-    ap.add_argument("--only", choices=["all", "prefill", "decode", "decode_rla", "fp8", "sla2", "pisa"],
+    ap.add_argument("--only", choices=["all", "prefill", "decode", "decode_rla", "fp8", "sla2", "pisa", "sfa"],
                     default="all",
                     help="prefill: the timed step only; decode / fp8 / sla2 / pisa (covariance routing + "
                          "first-order tail): only that workload's timing")

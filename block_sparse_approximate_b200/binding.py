@@ -27,6 +27,7 @@ TAIL = {"drop": 0, "zero_order": 1, "linear_mix": 2, "first_order": 3, "residual
 # every entry point declared in include/sparseattn.h
 EXPORTS = ("sa_block_pool", "sa_route", "sa_sparse_attn_fwd", "sa_decode_workspace_size",
            "sa_decode_fwd", "sa_decode_fwd_static", "sa_quantize_e4m3", "sa_sparse_attn_fwd_fp8",
+           "sa_sfa_encode", "sa_sfa_densify", "sa_sfa_workspace_size", "sa_sfa_attn_fwd",
            "sa_device_error", "sa_last_error", "sa_version")
 
 
@@ -86,8 +87,14 @@ def load():
                                          i32, f32, ctypes.c_int, vp, vp, vp, vp]
     lib.sa_quantize_e4m3.argtypes = [vp, ctypes.c_int64, i32, i32, i32, vp, vp, vp, vp]
     lib.sa_sparse_attn_fwd_fp8.argtypes = [ctypes.POINTER(Fp8Operands), Shape, vp, i32, ctypes.c_int, f32, vp, vp]
+    i64 = ctypes.c_int64
+    lib.sa_sfa_encode.argtypes = [vp, i64, i32, i32, vp, vp, vp, vp]
+    lib.sa_sfa_densify.argtypes = [vp, vp, i64, i32, i32, vp, vp]
+    lib.sa_sfa_workspace_size.argtypes = [Shape]
+    lib.sa_sfa_workspace_size.restype = sz
+    lib.sa_sfa_attn_fwd.argtypes = [vp, vp, vp, ctypes.c_int, Shape, f32, vp, vp, sz, vp]
     for fn in ("sa_block_pool", "sa_route", "sa_sparse_attn_fwd", "sa_decode_fwd", "sa_decode_fwd_static",
-               "sa_quantize_e4m3", "sa_sparse_attn_fwd_fp8"):
+               "sa_quantize_e4m3", "sa_sparse_attn_fwd_fp8", "sa_sfa_encode", "sa_sfa_densify", "sa_sfa_attn_fwd"):
         getattr(lib, fn).restype = ctypes.c_int
     lib.sa_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
     lib.sa_device_error.restype = ctypes.c_int
@@ -298,4 +305,43 @@ def sparse_attn_fwd_fp8(ops: dict, shape, block_idx, tail: str, scale: float, *,
            lib.sa_sparse_attn_fwd_fp8(ctypes.byref(cops), Shape(Bsz, H, N, d, block),
                                       _ptr(block_idx) if topk > 0 else None, int(topk), TAIL[tail],
                                       float(scale), _ptr(O), _stream(stream)))
+    return O
+
+
+def sfa_encode(X: torch.Tensor, kf: int, *, want_dense: bool = True, stream=None):
+    """Sparse feature codes of a bf16 tensor [..., d]: returns (vals bf16 [..., kf],
+    idx uint8 [..., kf], dense bf16 [..., d] zero-filled rows or None)."""
+    lib = load()
+    d = X.shape[-1]
+    rows = X.numel() // d
+    vals = torch.empty(X.shape[:-1] + (kf,), device=X.device, dtype=torch.bfloat16)
+    idx = torch.empty(X.shape[:-1] + (kf,), device=X.device, dtype=torch.uint8)
+    dense = torch.empty_like(X) if want_dense else None
+    _check("sa_sfa_encode", lib.sa_sfa_encode(_ptr(X), rows, d, int(kf), _ptr(vals), _ptr(idx), _ptr(dense),
+                                              _stream(stream)))
+    return vals, idx, dense
+
+
+def sfa_densify(vals: torch.Tensor, idx: torch.Tensor, d: int, *, stream=None) -> torch.Tensor:
+    """Zero-filled rows [..., d] bf16 from sparse feature codes."""
+    lib = load()
+    kf = vals.shape[-1]
+    rows = vals.numel() // kf
+    dense = torch.empty(vals.shape[:-1] + (d,), device=vals.device, dtype=torch.bfloat16)
+    _check("sa_sfa_densify", lib.sa_sfa_densify(_ptr(vals), _ptr(idx), rows, int(d), int(kf), _ptr(dense),
+                                                _stream(stream)))
+    return dense
+
+
+def sfa_attn_fwd(Qs, Ks, V, block: int, scale: float, *, workspace=None, out=None, stream=None) -> torch.Tensor:
+    """Sparse feature attention on zero-filled sparse Q, K [B,H,N,d] and dense V."""
+    lib = load()
+    Bsz, H, N, d = Qs.shape
+    shape = Shape(Bsz, H, N, d, block)
+    ws = int(lib.sa_sfa_workspace_size(shape))
+    if workspace is None:
+        workspace = torch.empty(max(ws, 256), device=Qs.device, dtype=torch.uint8)
+    O = out if out is not None else torch.empty_like(Qs)
+    _check("sa_sfa_attn_fwd", lib.sa_sfa_attn_fwd(_ptr(Qs), _ptr(Ks), _ptr(V), _dtype_code(Qs), shape, float(scale),
+                                                  _ptr(O), _ptr(workspace), workspace.numel(), _stream(stream)))
     return O

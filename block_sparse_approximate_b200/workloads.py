@@ -25,6 +25,11 @@ long-context LLM decoding; these synthetic inputs stand in for them):
                 131072 tokens: K, V ~ N(0,1) plus an N(0, 0.5) offset per
                 (64-token block, channel); q ~ N(0,1); block 64; taylor2 router,
                 top-64 blocks; zero-order tail.
+* ``sfa``       sparse feature attention ("Scaling Attention via Feature
+                Sparsity"): B=1, H=12, N=16384, d=128, bf16, Q,K,V ~ N(0,1),
+                seed 6; the top-16 of 128 features of every query and key
+                (the page's example k = 16, d = 128); every 128-token tile of
+                keys attends (non-causal).
 * ``decode_rla``  ``decode`` (same seed, same caches) with SPLA's residual
                 linear attention over the unselected blocks instead of the
                 zero-order tail.
@@ -100,6 +105,8 @@ WORKLOADS = {
     "decode": Workload("decode", B=16, H=32, N=131072, d=128, dtype="bf16",
                        block=64, route="taylor2", tail="zero_order", seed=4,
                        topk=64, decode=True, Hkv=8),
+    "sfa": Workload("sfa", B=1, H=12, N=16384, d=128, dtype="bf16", block=128, route="dot",
+                    tail="drop", seed=6, topk=128, extra={"kf": 16}),
     "decode_rla": Workload("decode_rla", B=16, H=32, N=131072, d=128, dtype="bf16",
                            block=64, route="taylor2", tail="residual_linear", seed=4,
                            topk=64, decode=True, Hkv=8),

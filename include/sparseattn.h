@@ -273,6 +273,41 @@ sa_status sa_decode_fwd_static(const void* q, const void* Kcache, const void* Vc
                                float scale, sa_tail_mode tail, int32_t* block_idx_out,
                                float* scores_out, void* O, void* stream);
 
+/* ---- Sparse feature attention ["Scaling Attention via Feature Sparsity",
+ * §2: top-k feature codes of Q and K; FlashSFA's exact online softmax over
+ * the overlap of the supports] ---------------------------------------------
+ *
+ * Sparse feature codes: for every row of X ([rows][d] bf16) the kf
+ * coordinates of largest |x|, a tie in magnitude going to the smaller
+ * channel index, in ascending channel order: vals [rows][kf] bf16 (signed
+ * values), idx [rows][kf] uint8 (channels).  dense: [rows][d] bf16 or NULL;
+ * when given, the zero-filled row (x at the kept channels, 0 elsewhere).
+ * d in {64, 128}; 1 <= kf <= min(d, 32).  X and dense 16-byte aligned.
+ * Errors: SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED, SA_ERR_ALIGNMENT. */
+sa_status sa_sfa_encode(const void* X, int64_t rows, int32_t d, int32_t kf, void* vals, uint8_t* idx,
+                        void* dense, void* stream);
+
+/* Zero-filled rows dense [rows][d] bf16 from codes (vals, idx) as written by
+ * sa_sfa_encode (e.g. a key cache kept as codes).  Same limits. */
+sa_status sa_sfa_densify(const void* vals, const uint8_t* idx, int64_t rows, int32_t d, int32_t kf,
+                         void* dense, void* stream);
+
+/* Bytes of workspace sa_sfa_attn_fwd needs (0 on a bad shape). */
+size_t sa_sfa_workspace_size(sa_shape shape);
+
+/* Sparse feature attention forward, non-causal: for every query row t,
+ *   o_t = Σ_n e^{s a_tn} v_n / Σ_n e^{s a_tn},  a_tn = Σ_{c ∈ supp(q_t) ∩ supp(k_n)} q_tc k_nc,
+ * which is the dot product of the zero-filled sparse rows.  Qs, Ks: the
+ * zero-filled codes of Q and K ([B,H,N,d], from sa_sfa_encode or
+ * sa_sfa_densify); V: [B,H,N,d] dense; all of `dtype`; O: [B,H,N,d] of
+ * `dtype`.  shape.block is the tile of the online softmax (128 with d = 128
+ * and bf16 takes the tensor-core kernel).  workspace: at least
+ * sa_sfa_workspace_size(shape) bytes, 16-byte aligned.
+ * Errors: SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED, SA_ERR_ALIGNMENT,
+ *         SA_ERR_WORKSPACE. */
+sa_status sa_sfa_attn_fwd(const void* Qs, const void* Ks, const void* V, sa_dtype dtype, sa_shape shape,
+                          float scale, void* O, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Reads and clears the library's device-side error word (synchronous: waits
  * for work already queued on the legacy default stream).  Non-zero means a
  * kernel gave up on an internal wait (bit 0: a bounded barrier wait timed

@@ -69,12 +69,15 @@ def sfa_densify(vals, idx, d: int) -> np.ndarray:
     return out
 
 
-def sfa_attention(Q, K, V, kf: int, scale: float) -> np.ndarray:
+def sfa_attention(Q, K, V, kf: int, scale: float, rows=None) -> np.ndarray:
     """SFA forward, [B,H,N,d] inputs, non-causal: softmax(s Q̃ K̃ᵀ) V with Q̃,
     K̃ the top-kf sparsified queries and keys (the support-overlap score is the
-    dot product of the zero-filled sparse vectors)."""
+    dot product of the zero-filled sparse vectors).  ``rows``: optional query
+    row indices (then only those rows are returned, [B,H,len(rows),d])."""
     Q, K, V = _f64(Q), _f64(K), _f64(V)
     d = Q.shape[-1]
+    if rows is not None:
+        Q = Q[:, :, np.asarray(rows, dtype=np.int64)]
     Qs = sfa_densify(*sfa_codes(Q, kf), d)
     Ks = sfa_densify(*sfa_codes(K, kf), d)
     a = scale * np.einsum("bhic,bhjc->bhij", Qs, Ks)

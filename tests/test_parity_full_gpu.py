@@ -103,3 +103,20 @@ def test_fp8_full_size_sampled(lib):
     err = np.abs(got - ref)
     print(f"fp8 vs unquantised float64 oracle: max-abs {err.max():.3e} mean-abs {err.mean():.3e}")
     assert err.mean() < 4e-2 and err.max() < 0.8
+
+
+def test_sfa_full_size_sampled(lib):
+    w = wl.WORKLOADS["sfa"]
+    inp = wl.prefill_inputs(w, DEV)
+    kf = w.extra["kf"]
+    _, _, Qs = bd.sfa_encode(inp["Q"], kf)
+    _, _, Ks = bd.sfa_encode(inp["K"], kf)
+    O = bd.sfa_attn_fwd(Qs, Ks, inp["V"], w.block, w.scale)
+    torch.cuda.synchronize()
+    assert_no_device_error()
+    rng = np.random.default_rng(5)
+    rows = np.sort(np.concatenate([[0, w.N - 1], rng.choice(w.N, 30, replace=False)]))
+    for h in (0, w.H - 1):
+        sub = {n: inp[n][:, h:h + 1].cpu().float().numpy() for n in ("Q", "K", "V")}
+        ref = oracle.sfa_attention(sub["Q"], sub["K"], sub["V"], kf, w.scale, rows=rows)
+        assert_tol(np64(O[:, h:h + 1, rows]), ref, BF16_TOL, f"sfa head {h}")

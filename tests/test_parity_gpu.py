@@ -379,3 +379,37 @@ def test_fp8_video_small(lib, tail, k):
 def test_fp8_ragged(lib, tail, nb, k):
     Q, K, V = _gauss(2, 2, nb * 128, 128, torch.bfloat16, 70 + nb)
     _fp8_case(Q, K, V, k, tail)
+
+
+# --------------------------------------------------------------------------
+# sparse feature attention
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("d,kf", [(128, 16), (128, 1), (64, 8), (128, 32)])
+def test_sfa_encode_bit_exact(lib, d, kf):
+    g = torch.Generator(device=DEV)
+    g.manual_seed(30 + kf)
+    # rounded to a coarse grid so that equal magnitudes (the tie rule) occur
+    X = (torch.randn(3, 257, d, generator=g, device=DEV) * 4).round().div(4).to(torch.bfloat16)
+    vals, idx, dense = bd.sfa_encode(X, kf)
+    torch.cuda.synchronize()
+    rv, ri = oracle.sfa_codes(np64(X), kf)
+    np.testing.assert_array_equal(idx.cpu().numpy().astype(np.int64), ri)
+    np.testing.assert_array_equal(np64(vals), rv)
+    np.testing.assert_array_equal(np64(dense), oracle.sfa_densify(rv, ri, d))
+    back = bd.sfa_densify(vals, idx, d)
+    torch.cuda.synchronize()
+    assert torch.equal(back, dense)
+
+
+@pytest.mark.parametrize("d,block,N,kf", [(128, 128, 1024, 16), (128, 128, 1152, 32), (64, 64, 640, 8)])
+def test_sfa_attention(lib, d, block, N, kf):
+    Q, K, V = _gauss(1, 2, N, d, torch.bfloat16, 40 + N)
+    _, _, Qs = bd.sfa_encode(Q, kf)
+    _, _, Ks = bd.sfa_encode(K, kf)
+    s = 1 / math.sqrt(d)
+    O = bd.sfa_attn_fwd(Qs, Ks, V, block, s)
+    torch.cuda.synchronize()
+    assert_no_device_error()
+    ref = oracle.sfa_attention(np64(Q), np64(K), np64(V), kf, s)
+    assert_tol(np64(O), ref, BF16_TOL, f"sfa d={d} kf={kf}")
