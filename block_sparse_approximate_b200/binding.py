@@ -28,6 +28,7 @@ TAIL = {"drop": 0, "zero_order": 1, "linear_mix": 2, "first_order": 3, "residual
 EXPORTS = ("sa_block_pool", "sa_route", "sa_sparse_attn_fwd", "sa_decode_workspace_size",
            "sa_decode_fwd", "sa_decode_fwd_static", "sa_quantize_e4m3", "sa_sparse_attn_fwd_fp8",
            "sa_sfa_encode", "sa_sfa_densify", "sa_sfa_workspace_size", "sa_sfa_attn_fwd",
+           "sa_sparse_attn_bwd_workspace_size", "sa_sparse_attn_bwd",
            "sa_device_error", "sa_last_error", "sa_version")
 
 
@@ -93,8 +94,13 @@ def load():
     lib.sa_sfa_workspace_size.argtypes = [Shape]
     lib.sa_sfa_workspace_size.restype = sz
     lib.sa_sfa_attn_fwd.argtypes = [vp, vp, vp, ctypes.c_int, Shape, f32, vp, vp, sz, vp]
+    lib.sa_sparse_attn_bwd_workspace_size.argtypes = [Shape, i32]
+    lib.sa_sparse_attn_bwd_workspace_size.restype = sz
+    lib.sa_sparse_attn_bwd.argtypes = [vp, vp, vp, vp, vp, ctypes.c_int, Shape, vp, i32, ctypes.c_int,
+                                       ctypes.POINTER(BlockStats), f32, vp, vp, vp, vp, sz, vp]
     for fn in ("sa_block_pool", "sa_route", "sa_sparse_attn_fwd", "sa_decode_fwd", "sa_decode_fwd_static",
-               "sa_quantize_e4m3", "sa_sparse_attn_fwd_fp8", "sa_sfa_encode", "sa_sfa_densify", "sa_sfa_attn_fwd"):
+               "sa_quantize_e4m3", "sa_sparse_attn_fwd_fp8", "sa_sfa_encode", "sa_sfa_densify", "sa_sfa_attn_fwd",
+               "sa_sparse_attn_bwd"):
         getattr(lib, fn).restype = ctypes.c_int
     lib.sa_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
     lib.sa_device_error.restype = ctypes.c_int
@@ -345,3 +351,24 @@ def sfa_attn_fwd(Qs, Ks, V, block: int, scale: float, *, workspace=None, out=Non
     _check("sa_sfa_attn_fwd", lib.sa_sfa_attn_fwd(_ptr(Qs), _ptr(Ks), _ptr(V), _dtype_code(Qs), shape, float(scale),
                                                   _ptr(O), _ptr(workspace), workspace.numel(), _stream(stream)))
     return O
+
+
+def sparse_attn_bwd(Q, K, V, O, dO, block_idx, block: int, tail: str, stats: dict, scale: float, *,
+                    workspace=None, stream=None):
+    """Backward of sparse_attn_fwd (drop, zero_order): returns float32 (dQ, dK, dV)."""
+    lib = load()
+    Bsz, H, N, d = Q.shape
+    topk = block_idx.shape[-1] if block_idx is not None else 0
+    shape = Shape(Bsz, H, N, d, block)
+    ws = int(lib.sa_sparse_attn_bwd_workspace_size(shape, int(topk)))
+    if workspace is None:
+        workspace = torch.empty(max(ws, 256), device=Q.device, dtype=torch.uint8)
+    f = dict(device=Q.device, dtype=torch.float32)
+    dQ, dK, dV = torch.empty(Q.shape, **f), torch.empty(K.shape, **f), torch.empty(V.shape, **f)
+    cst = _stats_struct(stats or {})
+    _check("sa_sparse_attn_bwd",
+           lib.sa_sparse_attn_bwd(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(dO), _dtype_code(Q), shape,
+                                  _ptr(block_idx) if topk > 0 else None, int(topk), TAIL[tail], ctypes.byref(cst),
+                                  float(scale), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(workspace), workspace.numel(),
+                                  _stream(stream)))
+    return dQ, dK, dV

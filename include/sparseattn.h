@@ -178,6 +178,31 @@ sa_status sa_sparse_attn_fwd(const void* Q, const void* K, const void* V, sa_dty
                              const sa_block_stats* stats, float scale, void* O,
                              void* stream);
 
+/* Bytes of workspace sa_sparse_attn_bwd needs (0 on bad arguments). */
+size_t sa_sparse_attn_bwd_workspace_size(sa_shape shape, int32_t topk);
+
+/* Backward of sa_sparse_attn_fwd for the DROP and ZERO_ORDER tails: given the
+ * forward's inputs, its output O and the output cotangent dO, writes
+ * dQ, dK, dV (float32 [B,H,N,d], overwritten).  The forward is softmax
+ * attention of query block i to its exact keys k_n (n in the selected
+ * blocks) and, for ZERO_ORDER, one pseudo-key per unselected block j (key
+ * k̄_j, value vsum_j / block, logit bias ln block), so with
+ * p = exp(s q·k + bias − lse), δ_t = dO_t·o_t and ds = p (dO·v − δ):
+ *   dQ = s Σ ds k,   dK_key = s Σ ds q,   dV_key = Σ p dO,
+ * and each pseudo-key's gradients are spread over its block's tokens
+ * divided by block (k̄ and vsum / block are means of the block's k and v).
+ * Q, K, V, O, dO of `dtype`; block_idx, topk, tail, stats (kmean, vsum for
+ * ZERO_ORDER) and scale as given to the forward.  workspace: at least
+ * sa_sparse_attn_bwd_workspace_size() bytes, 16-byte aligned.  CUDA-core
+ * kernels (fp32 arithmetic); the sums over query blocks run in a fixed
+ * order, so the result does not depend on scheduling.
+ * Errors: SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED (other tails), SA_ERR_ALIGNMENT,
+ *         SA_ERR_WORKSPACE. */
+sa_status sa_sparse_attn_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                             sa_dtype dtype, sa_shape shape, const int32_t* block_idx, int32_t topk,
+                             sa_tail_mode tail, const sa_block_stats* stats, float scale, float* dQ,
+                             float* dK, float* dV, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Per-block e4m3 quantisation [SLA2 §2C, low-precision sparse branch]:
  * X: bf16 [BH][N][d] (BH = batch x heads); codes: uint8 [BH][N][d] e4m3fn bit
  * patterns; scales: float [BH][ceil(N/block)] with σ = absmax/448 of each block

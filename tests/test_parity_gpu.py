@@ -413,3 +413,36 @@ def test_sfa_attention(lib, d, block, N, kf):
     assert_no_device_error()
     ref = oracle.sfa_attention(np64(Q), np64(K), np64(V), kf, s)
     assert_tol(np64(O), ref, BF16_TOL, f"sfa d={d} kf={kf}")
+
+
+# --------------------------------------------------------------------------
+# backward
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("tail", ["zero_order", "drop"])
+@pytest.mark.parametrize("dtype,d,block,nb,k", [
+    (torch.float32, 64, 64, 9, 2),
+    (torch.bfloat16, 128, 128, 12, 3),
+    (torch.bfloat16, 128, 64, 10, 0),
+    (torch.bfloat16, 64, 128, 6, 6),        # every block selected
+])
+def test_backward(lib, tail, dtype, d, block, nb, k):
+    B, H, N = 1, 2, nb * block
+    Q, K, V = _gauss(B, H, N, d, dtype, 60 + nb + k)
+    g = torch.Generator(device=DEV)
+    g.manual_seed(61)
+    dO = torch.randn(B, H, N, d, generator=g, device=DEV).to(dtype)
+    s = 1 / math.sqrt(d)
+    st = bd.block_pool(Q, K, V, block, centroids_bf16=(dtype == torch.bfloat16))
+    idx, _ = bd.route(st, (B, H, N, d, block), "dot", k)
+    O = bd.sparse_attn_fwd(Q, K, V, idx, block, tail, st, s)
+    dQ, dK, dV = bd.sparse_attn_bwd(Q, K, V, O, dO, idx, block, tail, st, s)
+    torch.cuda.synchronize()
+    assert_no_device_error()
+    # the oracle differentiates its own float64 forward at the same inputs;
+    # the GPU uses its (rounded) forward output O for δ = dO·O
+    rQ, rK, rV = oracle.sparse_attention_backward(np64(Q), np64(K), np64(V), idx.cpu().numpy(), block, tail, s,
+                                                  np64(dO))
+    tol = (1e-4, 1e-5) if dtype == torch.float32 else (3e-2, 2e-3)
+    for got, ref, name in ((dQ, rQ, "dQ"), (dK, rK, "dK"), (dV, rV, "dV")):
+        assert_tol(np64(got), ref, tol, f"backward {tail} {name}")
