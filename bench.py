@@ -399,6 +399,61 @@ def time_sfa(steps: int = 10, warmup: int = 3):
     return out
 
 
+def backward_flops(w) -> float:
+    """FLOPs of the backward over the exact and pseudo-keys of every query row:
+    recomputed scores (2·d) for the lse pass, then per (row, key) in the dQ
+    pass 2·d (scores) + 2·d (dP) + 2·d (dQ), and in the key-side passes again
+    2·d (scores) + 2·d (dP) + 2·d (dV) + 2·d (dK): 16·d per (row, key)."""
+    keys = w.k * w.block + ((w.nb - w.k) if w.tail in ("zero_order", "first_order") else 0)
+    return 16.0 * w.d * keys * w.B * w.H * float(w.N)
+
+
+def time_backward(steps: int = 3, warmup: int = 3):
+    """Backward of the video_dit prefill (zero-order tail): forward step once,
+    then sa_sparse_attn_bwd timed on the saved inputs, output and a random dO."""
+    import ctypes
+    from block_sparse_approximate_b200 import binding as bd
+    from block_sparse_approximate_b200.pipeline import PrefillStep
+    w = wl.WORKLOADS["video_dit"]
+    inp = wl.prefill_inputs(w, "cuda")
+    step = PrefillStep(w, inp)
+    O = step()
+    g = torch.Generator(device="cuda")
+    g.manual_seed(99)
+    dO = torch.randn(O.shape, generator=g, device="cuda").to(O.dtype)
+    lib = bd.load()
+    shape = bd.Shape(w.B, w.H, w.N, w.d, w.block)
+    ws = torch.empty(int(lib.sa_sparse_attn_bwd_workspace_size(shape, w.k)), device="cuda", dtype=torch.uint8)
+    f = dict(device="cuda", dtype=torch.float32)
+    dQ, dK, dV = torch.empty(O.shape, **f), torch.empty(O.shape, **f), torch.empty(O.shape, **f)
+    buf = step.buf
+
+    def bwd():
+        bd._check("sa_sparse_attn_bwd", lib.sa_sparse_attn_bwd(
+            inp["Q"].data_ptr(), inp["K"].data_ptr(), inp["V"].data_ptr(), O.data_ptr(), dO.data_ptr(),
+            bd.SA_BF16, shape, buf.block_idx.data_ptr(), int(w.k), bd.TAIL[w.tail], ctypes.byref(step.cst),
+            float(w.scale), dQ.data_ptr(), dK.data_ptr(), dV.data_ptr(), ws.data_ptr(), ws.numel(),
+            bd._stream(None)))
+
+    for _ in range(warmup):
+        bwd()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(steps):
+        bwd()
+    e.record()
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e) / steps
+    fl = backward_flops(w)
+    out = {"workload": w.name, "tail": w.tail, "ms": ms, "tflops": fl / (ms * 1e-3) / 1e12,
+           "kernels": "CUDA cores (fp32): lse/δ, dQ, key-major dK/dV, centroid gradients",
+           "flops_per_call": fl}
+    del inp, step, O, dO, dQ, dK, dV, ws
+    torch.cuda.empty_cache()
+    return out
+
+
 def linear_mix_flops(w) -> float:
     """Per query block: exact softmax part 4·d·(k·B)·B, the A_i accumulation
     2·d²·(k·B) and the final relu(Q)(H_tot − A_i) 2·d²·B."""
@@ -453,6 +508,10 @@ def run_ours(args, world, rank, local):
     if args.only == "sla2":
         if rank == 0:
             print(json.dumps({"sla2_mix": time_sla2(args.steps, args.warmup)}), flush=True)
+        return 0
+    if args.only == "backward":
+        if rank == 0:
+            print(json.dumps({"backward": time_backward(args.steps, args.warmup)}), flush=True)
         return 0
     if args.only == "sfa":
         if rank == 0:
@@ -550,7 +609,7 @@ def run_ours(args, world, rank, local):
                "h2d_bytes_per_step": sum(inp[n].numel() * inp[n].element_size() for n in ("Q", "K", "V")),
                "d2h_bytes_per_step": step.buf.out.numel() * step.buf.out.element_size()}
 
-    decode = decode_rla = fp8 = sla2 = pisa = sfa = None
+    decode = decode_rla = fp8 = sla2 = pisa = sfa = backward = None
     if rank == 0 and args.only == "all" and not args.no_decode:
         del step
         torch.cuda.empty_cache()
@@ -560,6 +619,7 @@ def run_ours(args, world, rank, local):
         sla2 = time_sla2()
         pisa = time_pisa()
         sfa = time_sfa()
+        backward = time_backward()
     ck = clocks.stop() if clocks else None
 
     if rank != 0:
@@ -596,6 +656,7 @@ def run_ours(args, world, rank, local):
         "sla2_mix": sla2,
         "pisa": pisa,
         "sfa": sfa,
+        "backward": backward,
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -614,7 +675,8 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
-    ap.add_argument("--only", choices=["all", "prefill", "decode", "decode_rla", "fp8", "sla2", "pisa", "sfa"],
+    ap.add_argument("--only", choices=["all", "prefill", "decode", "decode_rla", "fp8", "sla2", "pisa", "sfa",
+                                       "backward"],
                     default="all",
                     help="prefill: the timed step only; decode / fp8 / sla2 / pisa (covariance routing + "
                          "first-order tail): only that workload's timing")

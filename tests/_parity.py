@@ -28,7 +28,8 @@ def assert_tol(got, ref, tol, what=""):
     assert np.all(np.isfinite(got)), f"{what}: non-finite output"
     err = np.abs(got - ref)
     mx, mn = float(err.max()) if err.size else 0.0, float(err.mean()) if err.size else 0.0
-    assert mx <= tol[0] and mn <= tol[1], f"{what}: max-abs {mx:.3e} (tol {tol[0]}), mean-abs {mn:.3e} (tol {tol[1]})"
+    assert mx <= tol[0] and mn <= tol[1], (f"{what}: max-abs {mx:.3e} (tol {tol[0]}), mean-abs {mn:.3e} "
+                                           f"(tol {tol[1]}), max |ref| {float(np.abs(ref).max()):.3e}")
     return mx, mn
 
 

@@ -120,3 +120,32 @@ def test_sfa_full_size_sampled(lib):
         sub = {n: inp[n][:, h:h + 1].cpu().float().numpy() for n in ("Q", "K", "V")}
         ref = oracle.sfa_attention(sub["Q"], sub["K"], sub["V"], kf, w.scale, rows=rows)
         assert_tol(np64(O[:, h:h + 1, rows]), ref, BF16_TOL, f"sfa head {h}")
+
+
+def test_backward_full_size_heads(lib):
+    # the video_dit backward on the GPU (all 12 heads); the oracle recomputes
+    # two whole heads (every dQ, dK, dV entry of them)
+    w = wl.WORKLOADS["video_dit"]
+    inp = wl.prefill_inputs(w, DEV)
+    step = PrefillStep(w, inp)
+    O = step()
+    g = torch.Generator(device=DEV)
+    g.manual_seed(99)
+    dO = torch.randn(O.shape, generator=g, device=DEV).to(O.dtype)
+    dQ, dK, dV = bd.sparse_attn_bwd(inp["Q"], inp["K"], inp["V"], O, dO, step.buf.block_idx, w.block, w.tail,
+                                    step.buf.stats, w.scale)
+    torch.cuda.synchronize()
+    assert_no_device_error()
+    for h in (0, w.H - 1):
+        sl = slice(h, h + 1)
+        sub = {n: inp[n][:, sl].cpu().float().numpy() for n in ("Q", "K", "V")}
+        rQ, rK, rV = oracle.sparse_attention_backward(sub["Q"], sub["K"], sub["V"],
+                                                      step.buf.block_idx[:, sl].cpu().numpy(), w.block, w.tail,
+                                                      w.scale, np64(dO[:, sl]))
+        for got, ref, name in ((dQ, rQ, "dQ"), (dK, rK, "dK"), (dV, rV, "dV")):
+            # bf16 storage of O enters δ = dO·O (≈2^-9 relative per entry), and a
+            # key's dK / dV sums ds·q / p·dO over every row of every query block
+            # that selected it (thousands of rows here), so the bound scales with
+            # the gradient's own size
+            scale_ref = max(1.0, float(np.abs(ref).max()))
+            assert_tol(np64(got[:, sl]), ref, (2e-2 * scale_ref, 2e-3), f"backward head {h} {name}")
