@@ -27,13 +27,14 @@ constexpr int kBwdRpw = kBwdRows / kBwdWarps;   // rows per warp
 constexpr int kBwdKT = 32;                      // keys per staged tile
 
 // Stages a tile of kBwdKT keys (rows [row0, row0 + n) of src, [.][D] of T,
-// or fp32 statistics scaled by `mul`) into dst [kBwdKT][D + 1]; missing
+// or fp32 statistics scaled by `mul`) into dst [kBwdKT][D + 4] (the padding
+// keeps 16-byte rows and spreads the lanes' rows over the banks); missing
 // rows are zero.
 template <typename T, int D>
 __device__ __forceinline__ void stage_keys(float* dst, const T* src, int row0, int n, float mul = 1.f) {
   for (int x = threadIdx.x; x < kBwdKT * D; x += kBwdThreads) {
     const int r = x / D, c = x % D;
-    dst[r * (D + 1) + c] = r < n ? to_f<T>(src[(size_t)(row0 + r) * D + c]) * mul : 0.f;
+    dst[r * (D + 4) + c] = r < n ? to_f<T>(src[(size_t)(row0 + r) * D + c]) * mul : 0.f;
   }
 }
 
@@ -69,8 +70,8 @@ bwd_stats_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __re
   const int nwords = (nb + 31) >> 5;
   extern __shared__ float bsm[];
   float* qs = bsm;                                   // [64][D]
-  float* ks = qs + kBwdRows * D;                     // [KT][D + 1]
-  uint32_t* sel_bits = reinterpret_cast<uint32_t*>(ks + kBwdKT * (D + 1));
+  float* ks = qs + kBwdRows * D;                     // [KT][D + 4]
+  uint32_t* sel_bits = reinterpret_cast<uint32_t*>(ks + kBwdKT * (D + 4));
   for (int x = tid; x < kBwdRows * D; x += kBwdThreads) qs[x] = to_f<T>(Q[head + (size_t)row0 * D + x]);
   const int32_t* sel = block_idx + (bh * nb + i) * (size_t)topk;
   load_selection(sel_bits, nwords, sel, topk);
@@ -100,10 +101,16 @@ bwd_stats_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __re
 #pragma unroll
     for (int r = 0; r < kBwdRpw; ++r) {
       const float* qr = qs + (warp * kBwdRpw + r) * D;
-      const float* kr = ks + lane * (D + 1);
+      const float* kr = ks + lane * (D + 4);
       float x = 0.f;
 #pragma unroll 8
-      for (int c = 0; c < D; ++c) x = fmaf(qr[c], kr[c], x);
+      for (int c = 0; c < D; c += 4) {
+        const float4 a = *reinterpret_cast<const float4*>(qr + c), k4 = *reinterpret_cast<const float4*>(kr + c);
+        x = fmaf(a.x, k4.x, x);
+        x = fmaf(a.y, k4.y, x);
+        x = fmaf(a.z, k4.z, x);
+        x = fmaf(a.w, k4.w, x);
+      }
       x = valid ? fmaf(x, scale2, bias) : -INFINITY;
       const float tmax = warp_max(x);
       if (tmax == -INFINITY) continue;
@@ -190,9 +197,9 @@ bwd_dq_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __restr
   extern __shared__ float bsm[];
   float* qs = bsm;                                   // [64][D]
   float* gs = qs + kBwdRows * D;                     // [64][D] dO rows
-  float* ks = gs + kBwdRows * D;                     // [KT][D + 1]
-  float* vs = ks + kBwdKT * (D + 1);                 // [KT][D + 1]
-  uint32_t* sel_bits = reinterpret_cast<uint32_t*>(vs + kBwdKT * (D + 1));
+  float* ks = gs + kBwdRows * D;                     // [KT][D + 4]
+  float* vs = ks + kBwdKT * (D + 4);                 // [KT][D + 4]
+  uint32_t* sel_bits = reinterpret_cast<uint32_t*>(vs + kBwdKT * (D + 4));
   for (int x = tid; x < kBwdRows * D; x += kBwdThreads) {
     qs[x] = to_f<T>(Q[head + (size_t)row0 * D + x]);
     gs[x] = to_f<T>(dO[head + (size_t)row0 * D + x]);
@@ -232,13 +239,21 @@ bwd_dq_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __restr
     for (int r = 0; r < kBwdRpw; ++r) {
       const float* qr = qs + (warp * kBwdRpw + r) * D;
       const float* gr = gs + (warp * kBwdRpw + r) * D;
-      const float* kr = ks + lane * (D + 1);
-      const float* vr = vs + lane * (D + 1);
+      const float* kr = ks + lane * (D + 4);
+      const float* vr = vs + lane * (D + 4);
       float x = 0.f, dp = 0.f;
 #pragma unroll 8
-      for (int c = 0; c < D; ++c) {
-        x = fmaf(qr[c], kr[c], x);
-        dp = fmaf(gr[c], vr[c], dp);
+      for (int c = 0; c < D; c += 4) {
+        const float4 a = *reinterpret_cast<const float4*>(qr + c), k4 = *reinterpret_cast<const float4*>(kr + c);
+        const float4 gg = *reinterpret_cast<const float4*>(gr + c), v4 = *reinterpret_cast<const float4*>(vr + c);
+        x = fmaf(a.x, k4.x, x);
+        x = fmaf(a.y, k4.y, x);
+        x = fmaf(a.z, k4.z, x);
+        x = fmaf(a.w, k4.w, x);
+        dp = fmaf(gg.x, v4.x, dp);
+        dp = fmaf(gg.y, v4.y, dp);
+        dp = fmaf(gg.z, v4.z, dp);
+        dp = fmaf(gg.w, v4.w, dp);
       }
       const float p = valid ? fast_exp2(fmaf(x, scale2, bias) - l2[r]) : 0.f;
       const float ds = p * (dp - dl[r]);
@@ -246,7 +261,7 @@ bwd_dq_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __restr
       for (int t = 0; t < kBwdKT; ++t) {
         const float dst = __shfl_sync(0xffffffffu, ds, t);
 #pragma unroll
-        for (int c = 0; c < PER; ++c) acc[r][c] = fmaf(dst, ks[t * (D + 1) + lane * PER + c], acc[r][c]);
+        for (int c = 0; c < PER; ++c) acc[r][c] = fmaf(dst, ks[t * (D + 4) + lane * PER + c], acc[r][c]);
       }
     }
   }
@@ -260,7 +275,8 @@ bwd_dq_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __restr
 
 // ---- dK, dV of the exact keys ---------------------------------------------
 // One CTA per 64 keys of one KV block; thread = (key, part): four threads per
-// key, part p owning channels 4 i + p (conflict-free shared reads).  The
+// key, part p owning the 16-byte channel chunks 4 i + p (float4 shared reads
+// that the four parts take from four different chunks).  The
 // query rows of every query block that selected the block are staged 32 at a
 // time; s and dP are reduced over the four parts with two shuffles.
 constexpr int kKvKeys = 64;
@@ -281,14 +297,16 @@ bwd_dkv_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __rest
   const int tid = threadIdx.x, key = tid / kKvParts, part = tid % kKvParts;
   const int n = j * BLK + half * kKvKeys + key;       // this thread's key token
   const float scale2 = scale * kLog2e;
-  __shared__ float qs[kKvRows][D];
-  __shared__ float gs[kKvRows][D];
+  __shared__ __align__(16) float qs[kKvRows][D];
+  __shared__ __align__(16) float gs[kKvRows][D];
   __shared__ float ls[kKvRows], ds_[kKvRows];
+  // channel of element e: chunk kKvParts (e / 4) + part, lane e % 4 in it
+  auto ch = [&](int e) { return 4 * (kKvParts * (e >> 2) + part) + (e & 3); };
   float kr[CPT], vr[CPT], dk[CPT], dv[CPT];
 #pragma unroll
   for (int e = 0; e < CPT; ++e) {
-    kr[e] = to_f<T>(K[head + (size_t)n * D + kKvParts * e + part]);
-    vr[e] = to_f<T>(V[head + (size_t)n * D + kKvParts * e + part]);
+    kr[e] = to_f<T>(K[head + (size_t)n * D + ch(e)]);
+    vr[e] = to_f<T>(V[head + (size_t)n * D + ch(e)]);
     dk[e] = 0.f;
     dv[e] = 0.f;
   }
@@ -310,10 +328,19 @@ bwd_dkv_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __rest
 #pragma unroll 2
       for (int r = 0; r < kKvRows; ++r) {
         float x = 0.f, dp = 0.f;
+        float4 q4[CPT / 4], g4[CPT / 4];
 #pragma unroll
-        for (int e = 0; e < CPT; ++e) {
-          x = fmaf(qs[r][kKvParts * e + part], kr[e], x);
-          dp = fmaf(gs[r][kKvParts * e + part], vr[e], dp);
+        for (int e4 = 0; e4 < CPT / 4; ++e4) {
+          q4[e4] = *reinterpret_cast<const float4*>(&qs[r][ch(4 * e4)]);
+          g4[e4] = *reinterpret_cast<const float4*>(&gs[r][ch(4 * e4)]);
+          x = fmaf(q4[e4].x, kr[4 * e4], x);
+          x = fmaf(q4[e4].y, kr[4 * e4 + 1], x);
+          x = fmaf(q4[e4].z, kr[4 * e4 + 2], x);
+          x = fmaf(q4[e4].w, kr[4 * e4 + 3], x);
+          dp = fmaf(g4[e4].x, vr[4 * e4], dp);
+          dp = fmaf(g4[e4].y, vr[4 * e4 + 1], dp);
+          dp = fmaf(g4[e4].z, vr[4 * e4 + 2], dp);
+          dp = fmaf(g4[e4].w, vr[4 * e4 + 3], dp);
         }
 #pragma unroll
         for (int o = 1; o < kKvParts; o <<= 1) {
@@ -323,23 +350,29 @@ bwd_dkv_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __rest
         const float p = fast_exp2(fmaf(x, scale2, -ls[r]));
         const float d = p * (dp - ds_[r]);
 #pragma unroll
-        for (int e = 0; e < CPT; ++e) {
-          dv[e] = fmaf(p, gs[r][kKvParts * e + part], dv[e]);
-          dk[e] = fmaf(d, qs[r][kKvParts * e + part], dk[e]);
+        for (int e4 = 0; e4 < CPT / 4; ++e4) {
+          dv[4 * e4] = fmaf(p, g4[e4].x, dv[4 * e4]);
+          dv[4 * e4 + 1] = fmaf(p, g4[e4].y, dv[4 * e4 + 1]);
+          dv[4 * e4 + 2] = fmaf(p, g4[e4].z, dv[4 * e4 + 2]);
+          dv[4 * e4 + 3] = fmaf(p, g4[e4].w, dv[4 * e4 + 3]);
+          dk[4 * e4] = fmaf(d, q4[e4].x, dk[4 * e4]);
+          dk[4 * e4 + 1] = fmaf(d, q4[e4].y, dk[4 * e4 + 1]);
+          dk[4 * e4 + 2] = fmaf(d, q4[e4].z, dk[4 * e4 + 2]);
+          dk[4 * e4 + 3] = fmaf(d, q4[e4].w, dk[4 * e4 + 3]);
         }
       }
     }
   }
 #pragma unroll
   for (int e = 0; e < CPT; ++e) {
-    dK[head + (size_t)n * D + kKvParts * e + part] = scale * dk[e];
-    dV[head + (size_t)n * D + kKvParts * e + part] = dv[e];
+    dK[head + (size_t)n * D + ch(e)] = scale * dk[e];
+    dV[head + (size_t)n * D + ch(e)] = dv[e];
   }
 }
 
 // ---- zero-order tail: the centroids' gradients ----------------------------
 // One CTA per 32 centroids of a head, thread = (centroid, part) with eight
-// parts of strided channels; every query row of the head is visited (rows
+// parts owning the 16-byte channel chunks 8 i + part; every query row of the head is visited (rows
 // whose block selected a centroid get p = 0 for it).  At the end dk̄_j / B and
 // dv̄_j / B are added to every token of block j (dK, dV hold the exact part,
 // written by bwd_dkv_kernel earlier on the stream).
@@ -362,14 +395,15 @@ bwd_centroid_kernel(const T* __restrict__ Q, const T* __restrict__ dO, int H, in
   const int j = j0 + cj;
   const bool live = j < nb;
   const float scale2 = scale * kLog2e, bias = log2f((float)BLK), inv_blk = 1.0f / BLK;
-  __shared__ float qs[kCtRows][D];
-  __shared__ float gs[kCtRows][D];
+  __shared__ __align__(16) float qs[kCtRows][D];
+  __shared__ __align__(16) float gs[kCtRows][D];
   __shared__ float ls[kCtRows], ds_[kCtRows];
   __shared__ uint32_t selm;                          // bit c: centroid j0 + c selected by this query block
+  auto ch = [&](int e) { return 4 * (kCtParts * (e >> 2) + part) + (e & 3); };
   float kr[CPT], vr[CPT], dk[CPT], dv[CPT];
 #pragma unroll
   for (int e = 0; e < CPT; ++e) {
-    const size_t g = (bh * nb + (live ? j : 0)) * D + kCtParts * e + part;
+    const size_t g = (bh * nb + (live ? j : 0)) * D + ch(e);
     kr[e] = live ? kmean[g] : 0.f;
     vr[e] = live ? vsum[g] * inv_blk : 0.f;
     dk[e] = 0.f;
@@ -400,10 +434,19 @@ bwd_centroid_kernel(const T* __restrict__ Q, const T* __restrict__ dO, int H, in
 #pragma unroll 2
     for (int r = 0; r < kCtRows; ++r) {
       float x = 0.f, dp = 0.f;
+      float4 q4[CPT / 4], g4[CPT / 4];
 #pragma unroll
-      for (int e = 0; e < CPT; ++e) {
-        x = fmaf(qs[r][kCtParts * e + part], kr[e], x);
-        dp = fmaf(gs[r][kCtParts * e + part], vr[e], dp);
+      for (int e4 = 0; e4 < CPT / 4; ++e4) {
+        q4[e4] = *reinterpret_cast<const float4*>(&qs[r][ch(4 * e4)]);
+        g4[e4] = *reinterpret_cast<const float4*>(&gs[r][ch(4 * e4)]);
+        x = fmaf(q4[e4].x, kr[4 * e4], x);
+        x = fmaf(q4[e4].y, kr[4 * e4 + 1], x);
+        x = fmaf(q4[e4].z, kr[4 * e4 + 2], x);
+        x = fmaf(q4[e4].w, kr[4 * e4 + 3], x);
+        dp = fmaf(g4[e4].x, vr[4 * e4], dp);
+        dp = fmaf(g4[e4].y, vr[4 * e4 + 1], dp);
+        dp = fmaf(g4[e4].z, vr[4 * e4 + 2], dp);
+        dp = fmaf(g4[e4].w, vr[4 * e4 + 3], dp);
       }
 #pragma unroll
       for (int o = 1; o < kCtParts; o <<= 1) {
@@ -413,9 +456,15 @@ bwd_centroid_kernel(const T* __restrict__ Q, const T* __restrict__ dO, int H, in
       const float p = valid ? fast_exp2(fmaf(x, scale2, bias) - ls[r]) : 0.f;
       const float d = p * (dp - ds_[r]);
 #pragma unroll
-      for (int e = 0; e < CPT; ++e) {
-        dv[e] = fmaf(p, gs[r][kCtParts * e + part], dv[e]);
-        dk[e] = fmaf(d, qs[r][kCtParts * e + part], dk[e]);
+      for (int e4 = 0; e4 < CPT / 4; ++e4) {
+        dv[4 * e4] = fmaf(p, g4[e4].x, dv[4 * e4]);
+        dv[4 * e4 + 1] = fmaf(p, g4[e4].y, dv[4 * e4 + 1]);
+        dv[4 * e4 + 2] = fmaf(p, g4[e4].z, dv[4 * e4 + 2]);
+        dv[4 * e4 + 3] = fmaf(p, g4[e4].w, dv[4 * e4 + 3]);
+        dk[4 * e4] = fmaf(d, q4[e4].x, dk[4 * e4]);
+        dk[4 * e4 + 1] = fmaf(d, q4[e4].y, dk[4 * e4 + 1]);
+        dk[4 * e4 + 2] = fmaf(d, q4[e4].z, dk[4 * e4 + 2]);
+        dk[4 * e4 + 3] = fmaf(d, q4[e4].w, dk[4 * e4 + 3]);
       }
     }
   }
@@ -425,7 +474,7 @@ bwd_centroid_kernel(const T* __restrict__ Q, const T* __restrict__ dO, int H, in
     const size_t rowoff = head + ((size_t)j * BLK + t) * D;
 #pragma unroll
     for (int e = 0; e < CPT; ++e) {
-      const size_t g = rowoff + kCtParts * e + part;
+      const size_t g = rowoff + ch(e);
       dK[g] += scale * dk[e] * inv_blk;
       dV[g] += dv[e] * inv_blk;
     }
@@ -465,7 +514,7 @@ sa_status launch_bwd(const void* Q, const void* K, const void* V, const void* O,
   const int nwords = (nb + 31) / 32;
   const dim3 gq(s.N / kBwdRows, s.H, s.B);
   {
-    const size_t smem = sizeof(float) * ((size_t)kBwdRows * D + (size_t)kBwdKT * (D + 1)) +
+    const size_t smem = sizeof(float) * ((size_t)kBwdRows * D + (size_t)kBwdKT * (D + 4)) +
                         sizeof(uint32_t) * nwords;
     auto kern = bwd_stats_kernel<T, D, BLK>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
@@ -483,7 +532,7 @@ sa_status launch_bwd(const void* Q, const void* K, const void* V, const void* O,
     return launch_status("cudaMemsetAsync(bwd offsets)");
   }
   {
-    const size_t smem = sizeof(float) * (2 * (size_t)kBwdRows * D + 2 * (size_t)kBwdKT * (D + 1)) +
+    const size_t smem = sizeof(float) * (2 * (size_t)kBwdRows * D + 2 * (size_t)kBwdKT * (D + 4)) +
                         sizeof(uint32_t) * nwords;
     auto kern = bwd_dq_kernel<T, D, BLK>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
