@@ -446,8 +446,11 @@ def time_backward(steps: int = 3, warmup: int = 3):
     torch.cuda.synchronize()
     ms = s.elapsed_time(e) / steps
     fl = backward_flops(w)
-    out = {"workload": w.name, "tail": w.tail, "ms": ms, "tflops": fl / (ms * 1e-3) / 1e12,
-           "kernels": "CUDA cores (fp32): lse/δ, dQ, key-major dK/dV, centroid gradients",
+    _, bf16, _, src = _peaks()
+    ach = fl / (ms * 1e-3) / 1e12
+    out = {"workload": w.name, "tail": w.tail, "ms": ms, "tflops": ach, "peak_tflops": bf16, "frac": ach / bf16,
+           "peak_source": f"{src} bf16 burst",
+           "kernels": "mma.sync bf16: dQ (+ lse, δ), key-major dK/dV (exact keys, then centroids)",
            "flops_per_call": fl}
     del inp, step, O, dO, dQ, dK, dV, ws
     torch.cuda.empty_cache()

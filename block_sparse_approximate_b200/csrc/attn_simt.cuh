@@ -48,4 +48,14 @@ sa_status covnorm_tc(const void* K, const void* V, const sa_shape& s, const floa
 bool make_tmap_128x128(void* map, const void* base, int elem, uint64_t cols, uint64_t rows, uint64_t outer);
 uint32_t covnorm_error_take();
 
+// Backward of the sparse prefill on the tensor cores (bwd_mma.cu): bf16,
+// d = 128, block 64 or 128 (zero-order needs the bf16 centroids).  lse2,
+// delta [B·H·N] and the per-KV-block query lists offs/list come from the
+// caller's workspace (offs/list filled beforehand).
+bool bwd_tc_supports(sa_dtype dtype, const sa_shape& s, bool zo, const sa_block_stats& st);
+sa_status bwd_tc(const void* Q, const void* K, const void* V, const void* O, const void* dO, const sa_shape& s,
+                 const int32_t* block_idx, int topk, bool zo, const sa_block_stats& st, float scale, float* dQ,
+                 float* dK, float* dV, float* lse2, float* delta, const int32_t* offs, const int32_t* list,
+                 cudaStream_t stream);
+
 }  // namespace sa

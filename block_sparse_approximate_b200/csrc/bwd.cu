@@ -1,6 +1,7 @@
 // Backward of the sparse prefill for the drop and zero-order tails, on CUDA
 // cores (fp32 arithmetic; Q, K, V, O, dO of the forward's dtype; dQ, dK, dV
-// fp32).  The forward is softmax attention of query block i to the key list
+// fp32): the general path (fp32, d = 64), and the parity reference of the
+// tensor-core kernels in bwd_mma.cu, which take bf16 with d = 128.  The forward is softmax attention of query block i to the key list
 // [k_n, n ∈ S_i] + [k̄_j, j ∈ U_i] with logit biases 0 / ln B and values v_n /
 // v̄_j = vsum_j / B (PISA "Algoritmo Central"), so the gradients are
 //   p = exp(s q·k + bias − lse),  δ_t = dO_t·o_t,  ds = p (dO·v − δ),
@@ -513,6 +514,18 @@ sa_status launch_bwd(const void* Q, const void* K, const void* V, const void* O,
   const T* g = static_cast<const T*>(dO);
   const int nwords = (nb + 31) / 32;
   const dim3 gq(s.N / kBwdRows, s.H, s.B);
+  const sa_dtype dt = sizeof(T) == 2 ? SA_BF16 : SA_FP32;
+  if (bwd_tc_supports(dt, s, zo, st)) {
+    // tensor-core kernels: the per-KV-block query lists first
+    if (topk > 0) {
+      bwd_transpose_kernel<<<s.B * s.H, kBwdThreads, 0, stream>>>(block_idx, nb, topk, offs, list);
+      sa_status r = launch_status("bwd_transpose_kernel");
+      if (r != SA_OK) return r;
+    } else if (cudaMemsetAsync(offs, 0, (size_t)s.B * s.H * (nb + 1) * sizeof(int32_t), stream) != cudaSuccess) {
+      return launch_status("cudaMemsetAsync(bwd offsets)");
+    }
+    return bwd_tc(Q, K, V, O, dO, s, block_idx, topk, zo, st, scale, dQ, dK, dV, lse2, delta, offs, list, stream);
+  }
   {
     const size_t smem = sizeof(float) * ((size_t)kBwdRows * D + (size_t)kBwdKT * (D + 4)) +
                         sizeof(uint32_t) * nwords;
