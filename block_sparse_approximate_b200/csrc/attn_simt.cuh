@@ -56,6 +56,8 @@ bool bwd_tc_supports(sa_dtype dtype, const sa_shape& s, bool zo, const sa_block_
 sa_status bwd_tc(const void* Q, const void* K, const void* V, const void* O, const void* dO, const sa_shape& s,
                  const int32_t* block_idx, int topk, bool zo, const sa_block_stats& st, float scale, float* dQ,
                  float* dK, float* dV, float* lse2, float* delta, const int32_t* offs, const int32_t* list,
-                 cudaStream_t stream);
+                 float* part, cudaStream_t stream);
+// bytes of the centroid pass's partial sums (workspace)
+size_t bwd_tc_part_bytes(const sa_shape& s);
 
 }  // namespace sa

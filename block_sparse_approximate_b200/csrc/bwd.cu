@@ -483,7 +483,7 @@ bwd_centroid_kernel(const T* __restrict__ Q, const T* __restrict__ dO, int H, in
 }
 
 struct BwdLayout {
-  size_t lse_off, delta_off, offs_off, list_off, total;
+  size_t lse_off, delta_off, offs_off, list_off, part_off, total;
 };
 
 BwdLayout bwd_layout(const sa_shape& s, int topk) {
@@ -494,7 +494,9 @@ BwdLayout bwd_layout(const sa_shape& s, int topk) {
   L.delta_off = a256(BH * s.N * sizeof(float));
   L.offs_off = L.delta_off + a256(BH * s.N * sizeof(float));
   L.list_off = L.offs_off + a256(BH * (nb + 1) * sizeof(int32_t));
-  L.total = L.list_off + a256(BH * nb * (size_t)(topk > 0 ? topk : 1) * sizeof(int32_t));
+  L.part_off = L.list_off + a256(BH * nb * (size_t)(topk > 0 ? topk : 1) * sizeof(int32_t));
+  // the tensor-core centroid pass's partial sums (d = 128 shapes)
+  L.total = L.part_off + (s.d == 128 ? a256(bwd_tc_part_bytes(s)) : 0);
   return L;
 }
 
@@ -524,7 +526,8 @@ sa_status launch_bwd(const void* Q, const void* K, const void* V, const void* O,
     } else if (cudaMemsetAsync(offs, 0, (size_t)s.B * s.H * (nb + 1) * sizeof(int32_t), stream) != cudaSuccess) {
       return launch_status("cudaMemsetAsync(bwd offsets)");
     }
-    return bwd_tc(Q, K, V, O, dO, s, block_idx, topk, zo, st, scale, dQ, dK, dV, lse2, delta, offs, list, stream);
+    return bwd_tc(Q, K, V, O, dO, s, block_idx, topk, zo, st, scale, dQ, dK, dV, lse2, delta, offs, list,
+                  reinterpret_cast<float*>(ws + L.part_off), stream);
   }
   {
     const size_t smem = sizeof(float) * ((size_t)kBwdRows * D + (size_t)kBwdKT * (D + 4)) +

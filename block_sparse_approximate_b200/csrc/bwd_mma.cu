@@ -297,8 +297,11 @@ bwd_dq_mma_kernel(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __re
 // ---- dK, dV ---------------------------------------------------------------
 // CENT = false: 64 exact keys (block j, half `blockIdx.x % (BLK/64)`) over
 // the query blocks that selected block j (offs/list).  CENT = true: 64
-// centroids over every query row, masked where the row's block selected the
-// centroid; their gradients go ÷B to the tokens of their blocks.
+// centroids over one of kCentSplits ranges of the query rows (so that the
+// few centroid tiles still fill the GPU), masked where the row's block
+// selected the centroid; the partial dk̄, dv̄ go to `part`, which
+// bwd_centroid_scatter_kernel sums in order and spreads ÷B over the blocks.
+constexpr int kCentSplits = 8;
 template <int BLK, bool CENT>
 __global__ void __launch_bounds__(kMThreads)
 bwd_dkv_mma_kernel(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
@@ -306,7 +309,8 @@ bwd_dkv_mma_kernel(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __r
                    const __nv_bfloat16* __restrict__ kb16, const __nv_bfloat16* __restrict__ vb16, int H, int N,
                    const int32_t* __restrict__ block_idx, int topk, const int32_t* __restrict__ offs,
                    const int32_t* __restrict__ list, float scale, const float* __restrict__ lse2,
-                   const float* __restrict__ delta, float* __restrict__ dK, float* __restrict__ dV) {
+                   const float* __restrict__ delta, float* __restrict__ dK, float* __restrict__ dV,
+                   float* __restrict__ part) {
   const int nb = N / BLK;
   const size_t bh = (size_t)blockIdx.z * H + blockIdx.y;
   const size_t head = bh * (size_t)N * kMD;
@@ -321,8 +325,9 @@ bwd_dkv_mma_kernel(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __r
   float* lsd = reinterpret_cast<float*>(msm + 6 * kMTileB);   // [2 slots][lse 64, δ 64]
   // the CTA's keys: exact tokens or centroids
   int key0, nkeys, j = 0;
+  const int split = CENT ? (int)blockIdx.x % kCentSplits : 0;
   if (CENT) {
-    key0 = blockIdx.x * kMT;
+    key0 = ((int)blockIdx.x / kCentSplits) * kMT;
     nkeys = min(kMT, nb - key0);
     stage64(sK, kb16 + (bh * nb + key0) * (size_t)kMD, nkeys);
     stage64(sV, vb16 + (bh * nb + key0) * (size_t)kMD, nkeys);
@@ -339,8 +344,14 @@ bwd_dkv_mma_kernel(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __r
   const int32_t* off = offs + bh * (size_t)(nb + 1);
   const int32_t* lst = list + bh * (size_t)nb * topk;
   const int per_q = BLK / kMT;
-  const int nchunks = CENT ? N / kMT : (off[j + 1] - off[j]) * per_q;
-  auto chunk_row0 = [&](int c) { return CENT ? c * kMT : lst[off[j] + c / per_q] * BLK + (c % per_q) * kMT; };
+  // centroids: this split's range [c_lo, c_lo + nchunks) of the head's 64-row chunks
+  const int all_chunks = N / kMT;
+  const int c_lo = CENT ? (int)(((long)all_chunks * split) / kCentSplits) : 0;
+  const int nchunks = CENT ? (int)(((long)all_chunks * (split + 1)) / kCentSplits) - c_lo
+                           : (off[j + 1] - off[j]) * per_q;
+  auto chunk_row0 = [&](int c) {
+    return CENT ? (c_lo + c) * kMT : lst[off[j] + c / per_q] * BLK + (c % per_q) * kMT;
+  };
   auto issue = [&](int c, int slot) {
     const int r0 = chunk_row0(c);
     const uint32_t dq = sR0 + slot * 2 * kMTileB;
@@ -459,23 +470,15 @@ bwd_dkv_mma_kernel(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __r
     const int kr = rb + g + 8 * h;
     if (kr >= nkeys) continue;
     if (CENT) {
+      // partial sums of this split: part[2][split][bh][centroid][channel]
       const int jj = key0 + kr;
-      const float inv = 1.0f / BLK;
-      for (int t = 0; t < BLK; ++t) {
-        float* dkr = dK + head + ((size_t)jj * BLK + t) * kMD;
-        float* dvr = dV + head + ((size_t)jj * BLK + t) * kMD;
+      const size_t BHn = (size_t)gridDim.y * gridDim.z;
+      float* pk_ = part + (((size_t)split * BHn + bh) * nb + jj) * kMD;
+      float* pv_ = part + (((size_t)(kCentSplits + split) * BHn + bh) * nb + jj) * kMD;
 #pragma unroll
-        for (int n = 0; n < 16; ++n) {
-          float2* pk2 = reinterpret_cast<float2*>(dkr + 8 * n + 2 * tg);
-          float2* pv2 = reinterpret_cast<float2*>(dvr + 8 * n + 2 * tg);
-          float2 a = *pk2, b2 = *pv2;
-          a.x += scale * dk[n][2 * h] * inv;
-          a.y += scale * dk[n][2 * h + 1] * inv;
-          b2.x += dv[n][2 * h] * inv;
-          b2.y += dv[n][2 * h + 1] * inv;
-          *pk2 = a;
-          *pv2 = b2;
-        }
+      for (int n = 0; n < 16; ++n) {
+        *reinterpret_cast<float2*>(pk_ + 8 * n + 2 * tg) = make_float2(dk[n][2 * h], dk[n][2 * h + 1]);
+        *reinterpret_cast<float2*>(pv_ + 8 * n + 2 * tg) = make_float2(dv[n][2 * h], dv[n][2 * h + 1]);
       }
     } else {
       float* dkr = dK + head + (size_t)(key0 + kr) * kMD;
@@ -489,7 +492,35 @@ bwd_dkv_mma_kernel(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __r
   }
 }
 
+// dk̄_j, dv̄_j = the splits' partial sums in order; s dk̄_j / B and dv̄_j / B
+// added to each token of block j (one CTA per centroid, thread = channel).
+template <int BLK>
+__global__ void __launch_bounds__(kMD)
+bwd_centroid_scatter_kernel(const float* __restrict__ part, int H, int N, float scale, float* __restrict__ dK,
+                            float* __restrict__ dV) {
+  const int nb = N / BLK;
+  const int j = blockIdx.x, c = threadIdx.x;
+  const size_t bh = (size_t)blockIdx.z * H + blockIdx.y;
+  const size_t BHn = (size_t)gridDim.y * gridDim.z;
+  float sk = 0.f, sv = 0.f;
+  for (int sp = 0; sp < kCentSplits; ++sp) {
+    sk += part[(((size_t)sp * BHn + bh) * nb + j) * kMD + c];
+    sv += part[(((size_t)(kCentSplits + sp) * BHn + bh) * nb + j) * kMD + c];
+  }
+  sk *= scale / BLK;
+  sv *= 1.0f / BLK;
+  const size_t base = (bh * (size_t)N + (size_t)j * BLK) * kMD + c;
+  for (int t = 0; t < BLK; ++t) {
+    dK[base + (size_t)t * kMD] += sk;
+    dV[base + (size_t)t * kMD] += sv;
+  }
+}
+
 }  // namespace
+
+size_t bwd_tc_part_bytes(const sa_shape& s) {
+  return 2 * (size_t)kCentSplits * s.B * s.H * (size_t)(s.N / s.block) * kMD * sizeof(float);
+}
 
 bool bwd_tc_supports(sa_dtype dtype, const sa_shape& s, bool zo, const sa_block_stats& st) {
   return dtype == SA_BF16 && s.d == kMD && (s.block == 64 || s.block == 128) &&
@@ -500,7 +531,7 @@ template <int BLK>
 sa_status bwd_tc_launch(const void* Q, const void* K, const void* V, const void* O, const void* dO,
                         const sa_shape& s, const int32_t* block_idx, int topk, bool zo, const sa_block_stats& st,
                         float scale, float* dQ, float* dK, float* dV, float* lse2, float* delta,
-                        const int32_t* offs, const int32_t* list, cudaStream_t stream) {
+                        const int32_t* offs, const int32_t* list, float* part, cudaStream_t stream) {
   using bf = __nv_bfloat16;
   const int nb = s.N / BLK;
   const bf* q = static_cast<const bf*>(Q);
@@ -525,27 +556,31 @@ sa_status bwd_tc_launch(const void* Q, const void* K, const void* V, const void*
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
       return launch_status("cudaFuncSetAttribute(bwd_dkv_mma_kernel)");
     kern<<<dim3(nb * (BLK / kMT), s.H, s.B), kMThreads, smem, stream>>>(q, k, v, g, kb, vb, s.H, s.N, block_idx,
-                                                                       topk, offs, list, scale, lse2, delta, dK, dV);
+                                                                       topk, offs, list, scale, lse2, delta, dK, dV,
+                                                                       part);
     sa_status r = launch_status("bwd_dkv_mma_kernel");
     if (r != SA_OK || !zo) return r;
   }
   auto kern = bwd_dkv_mma_kernel<BLK, true>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return launch_status("cudaFuncSetAttribute(bwd_dkv_mma_kernel)");
-  kern<<<dim3((nb + kMT - 1) / kMT, s.H, s.B), kMThreads, smem, stream>>>(q, k, v, g, kb, vb, s.H, s.N, block_idx,
-                                                                         topk, offs, list, scale, lse2, delta, dK, dV);
-  return launch_status("bwd_dkv_mma_kernel(centroids)");
+  kern<<<dim3(((nb + kMT - 1) / kMT) * kCentSplits, s.H, s.B), kMThreads, smem, stream>>>(
+      q, k, v, g, kb, vb, s.H, s.N, block_idx, topk, offs, list, scale, lse2, delta, dK, dV, part);
+  sa_status r = launch_status("bwd_dkv_mma_kernel(centroids)");
+  if (r != SA_OK) return r;
+  bwd_centroid_scatter_kernel<BLK><<<dim3(nb, s.H, s.B), kMD, 0, stream>>>(part, s.H, s.N, scale, dK, dV);
+  return launch_status("bwd_centroid_scatter_kernel");
 }
 
 sa_status bwd_tc(const void* Q, const void* K, const void* V, const void* O, const void* dO, const sa_shape& s,
                  const int32_t* block_idx, int topk, bool zo, const sa_block_stats& st, float scale, float* dQ,
                  float* dK, float* dV, float* lse2, float* delta, const int32_t* offs, const int32_t* list,
-                 cudaStream_t stream) {
+                 float* part, cudaStream_t stream) {
   if (s.block == 128)
     return bwd_tc_launch<128>(Q, K, V, O, dO, s, block_idx, topk, zo, st, scale, dQ, dK, dV, lse2, delta, offs,
-                              list, stream);
+                              list, part, stream);
   return bwd_tc_launch<64>(Q, K, V, O, dO, s, block_idx, topk, zo, st, scale, dQ, dK, dV, lse2, delta, offs, list,
-                           stream);
+                           part, stream);
 }
 
 }  // namespace sa
