@@ -36,8 +36,9 @@
 //
 // e4m3 variant: Q, K, V (and the centroid tiles) are e4m3 codes with one
 // scale per 128-row block; S = σ_Q σ_K (Q̂·K̂ᵀ).  P is quantised to e4m3 as
-// P · 448 · σ_V(tile) / σ_Vmax (P ≤ 1: the running max is applied at once,
-// not lazily), so the MMA accumulates Σ P σ_V V̂ · 448 / σ_Vmax across tiles of
+// P · 112 · σ_V(tile) / σ_Vmax (P ≤ 4: the running max is applied lazily,
+// once it has grown by more than a factor 4, and 4 · 112 = 448 is the e4m3
+// maximum), so the MMA accumulates Σ P σ_V V̂ · 112 / σ_Vmax across tiles of
 // different V scales; the row sum uses the unquantised P.  σ_Vmax is the
 // largest V scale of the head (exact and centroid tiles).
 #include <mutex>
@@ -66,6 +67,11 @@ constexpr uint32_t kColO = 256;
 // (exp2_poly2) when bit n % 8 is set, else on MUFU.  Three of eight was the
 // fastest split measured on B200 for d = 128 tiles.
 constexpr uint32_t kExpFma = 0x49u;
+// e4m3 softmax: quad n of a row's 32 exponential quads runs on the FMA pipe
+// when bit n % 8 is set.  The e4m3 packing already loads the FMA pipe, so
+// only one quad in four moves there (measured on B200: 0, 1, 3, 4, 5 and 6 of
+// eight; 2 was the fastest, and 4 or more slower than none).
+constexpr uint32_t kExpFmaF8 = 0x11u;
 
 // Operand format of the kernel: spans per 128x128 tile, pipeline depth, MMA
 // K step (in elements), lazy-rescale threshold.
@@ -77,13 +83,17 @@ struct Fmt<false> {   // bf16
   static constexpr int NS = 3;
   static constexpr int kK = 16;                // K per MMA instruction
   static constexpr float kLazy = 8.0f;
+  static constexpr float kPScale = 1.0f;       // unused
 };
 template <>
 struct Fmt<true> {    // e4m3
   static constexpr int kSpans = 1;             // 128 bytes per row
   static constexpr int NS = 6;
   static constexpr int kK = 32;
-  static constexpr float kLazy = 0.0f;         // P <= 1 so that P·448 stays in range
+  // lazy rescale by up to 2^kLazy: P <= 2^kLazy, so P is quantised as
+  // P · kPScale with kPScale = 448 · 2^-kLazy (the e4m3 maximum is 448)
+  static constexpr float kLazy = 2.0f;
+  static constexpr float kPScale = 112.0f;
 };
 
 template <bool F8>
@@ -401,11 +411,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (centroid) {
           const int c = t - topk;
           tscale = scale2 * qs * f8.kbar[(size_t)bh * ntiles + c];
-          pscale = 448.0f * f8.vbar[(size_t)bh * ntiles + c] / vmax;
+          pscale = Fmt<true>::kPScale * f8.vbar[(size_t)bh * ntiles + c] / vmax;
         } else {
           const int j = sel[t];
           tscale = scale2 * qs * f8.k[(size_t)bh * nb + j];
-          pscale = 448.0f * f8.v[(size_t)bh * nb + j] / vmax;
+          pscale = Fmt<true>::kPScale * f8.v[(size_t)bh * nb + j] / vmax;
         }
       }
       if (centroid) {
@@ -451,7 +461,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           float a0, a1, a2, a3;
           ffma2(a0, a1, __uint_as_float(v[4 * n]), __uint_as_float(v[4 * n + 1]), sc2, sc2, ng, ng);
           ffma2(a2, a3, __uint_as_float(v[4 * n + 2]), __uint_as_float(v[4 * n + 3]), sc2, sc2, ng, ng);
-          const float p0 = fast_exp2(a0), p1 = fast_exp2(a1), p2 = fast_exp2(a2), p3 = fast_exp2(a3);
+          float p0, p1, p2, p3;
+          if ((kExpFmaF8 >> (n & 7)) & 1u) {
+            exp2_poly2(a0, a1, p0, p1);
+            exp2_poly2(a2, a3, p2, p3);
+          } else {
+            p0 = fast_exp2(a0); p1 = fast_exp2(a1); p2 = fast_exp2(a2); p3 = fast_exp2(a3);
+          }
           fadd2(sm8[2 * (n & 3)], sm8[2 * (n & 3) + 1], p0 + p2, p1 + p3);
           v[n] = pack_e4m3x4(p0 * pscale, p1 * pscale, p2 * pscale, p3 * pscale);
         }
@@ -511,8 +527,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const float f0 = (U0 > 0 && m0 != -INFINITY) ? fast_exp2(m0 - M) : 0.f;
     const float f1 = (U1 > 0 && m1 != -INFINITY) ? fast_exp2(m1 - M) : 0.f;
     const float L_ = l0 * f0 + l1 * f1;
-    // e4m3: O accumulated Σ P σ_V V̂ · 448 / σ_Vmax
-    const float inv = L_ > 0.f ? (F8 ? vmax / 448.0f : 1.0f) / L_ : 0.f;
+    // e4m3: O accumulated Σ P σ_V V̂ · kPScale / σ_Vmax
+    const float inv = L_ > 0.f ? (F8 ? vmax / Fmt<true>::kPScale : 1.0f) / L_ : 0.f;
     // first-order: + Λ_t (s q_t)ᵀ H̄ with Λ_t = Σ_U e^{s q·k̄_j} on the merged
     // maximum (the centroid tiles' sums carry the factor 128 = e^{ln 128})
     float wfo = 0.f;
