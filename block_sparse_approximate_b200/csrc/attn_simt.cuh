@@ -59,5 +59,12 @@ sa_status bwd_tc(const void* Q, const void* K, const void* V, const void* O, con
                  float* part, cudaStream_t stream);
 // bytes of the centroid pass's partial sums (workspace)
 size_t bwd_tc_part_bytes(const sa_shape& s);
+// dQ (with lse2 and delta) on tcgen05 (bwd_tc.cu): block 128, d = 128, at
+// least one tile per query block (topk > 0 or the zero-order tail); and the
+// read-and-clear of that kernel's bounded-wait error word.
+sa_status bwd_dq_tc(const void* Q, const void* K, const void* V, const void* O, const void* dO, const sa_shape& s,
+                    const int32_t* block_idx, int topk, bool zo, const sa_block_stats& st, float scale, float* lse2,
+                    float* delta, float* dQ, cudaStream_t stream);
+uint32_t bwd_error_take();
 
 }  // namespace sa

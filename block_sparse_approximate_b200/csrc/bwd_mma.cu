@@ -540,7 +540,10 @@ sa_status bwd_tc_launch(const void* Q, const void* K, const void* V, const void*
   const bf* g = static_cast<const bf*>(dO);
   const bf* kb = reinterpret_cast<const bf*>(st.kmean_bf16);
   const bf* vb = reinterpret_cast<const bf*>(st.vmean_bf16);
-  {
+  if (BLK == 128 && (topk > 0 || zo)) {
+    sa_status r = bwd_dq_tc(Q, K, V, O, dO, s, block_idx, topk, zo, st, scale, lse2, delta, dQ, stream);
+    if (r != SA_OK) return r;
+  } else {
     const size_t smem = 6 * (size_t)kMTileB + sizeof(uint32_t) * ((nb + 31) / 32);
     auto kern = bwd_dq_mma_kernel<BLK>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)

@@ -423,6 +423,9 @@ def test_sfa_attention(lib, d, block, N, kf):
 @pytest.mark.parametrize("dtype,d,block,nb,k", [
     (torch.float32, 64, 64, 9, 2),
     (torch.bfloat16, 128, 128, 12, 3),
+    (torch.bfloat16, 128, 128, 133, 13),    # two centroid tiles, the second ragged
+    (torch.bfloat16, 128, 128, 20, 0),      # zero-order: centroids only; drop: no key at all
+    (torch.bfloat16, 128, 128, 8, 8),       # every block selected: the centroid tile fully masked
     (torch.bfloat16, 128, 64, 10, 0),
     (torch.bfloat16, 64, 128, 6, 6),        # every block selected
 ])
