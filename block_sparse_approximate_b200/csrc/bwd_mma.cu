@@ -554,7 +554,10 @@ sa_status bwd_tc_launch(const void* Q, const void* K, const void* V, const void*
     if (r != SA_OK) return r;
   }
   const size_t smem = 6 * (size_t)kMTileB + 2 * 2 * kMT * sizeof(float);
-  {
+  if constexpr (BLK == 128) {
+    sa_status r = bwd_dkv_tc(Q, K, V, dO, s, topk, offs, list, scale, lse2, delta, dK, dV, stream);
+    if (r != SA_OK || !zo) return r;
+  } else {
     auto kern = bwd_dkv_mma_kernel<BLK, false>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
       return launch_status("cudaFuncSetAttribute(bwd_dkv_mma_kernel)");

@@ -437,6 +437,237 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   }
 }
 
+// ---- dK, dV of the exact keys --------------------------------------------
+// One CTA per 128-key block j, over the query blocks that selected it (the
+// transposed index offs/list, ascending), with the keys as the MMA rows:
+//   Sᵀ = K Q_cᵀ, dPᵀ = V dO_cᵀ, Pᵀ = 2^(s' Sᵀ − lse2), dSᵀ = Pᵀ ⊙ (dPᵀ − δ),
+//   dV += Pᵀ dO_c, dK += dSᵀ Q_c     (dK scaled by s at the end).
+// Warps 0-7: element-wise, group g = warp / 4 takes query rows 64 g .. + 63
+// (TMEM columns) of every chunk; warp 8: TMA (K, V once; a ring of two
+// (Q, dO, lse2, δ) chunks); warp 9: MMA.  TMEM: Sᵀ [0,128), dPᵀ [128,256),
+// dV [256,384), dK [384,512); Pᵀ (bf16) goes to Sᵀ's columns [32, 96) and
+// dSᵀ to dPᵀ's, each group inside the columns it read itself.
+constexpr int NR = 2;                          // query-chunk ring depth
+constexpr uint32_t kColST = 0, kColDPT = 128, kColDV = 256, kColDK = 384;
+
+struct KvLay {
+  static constexpr uint32_t kK = 0, kV = kTile, kR = 2 * kTile;     // ring stage: Q, dO
+  static constexpr uint32_t kLsd = kR + NR * 2 * kTile;             // [NR][lse2 128, δ 128] floats
+  static constexpr int B_KV = 0, B_RF = 1, B_RE = B_RF + NR, B_SF = B_RE + NR, B_EW = B_SF + 1,
+                       B_ACC = B_EW + 1, B_FIN = B_ACC + 1, NBAR = B_FIN + 1;
+  static constexpr uint32_t kBarOff = kLsd + NR * 2 * TB * 4;
+  static constexpr uint32_t kSlotOff = kBarOff + 8 * NBAR;
+  static constexpr size_t kSmem = 1024 + kSlotOff + 16;
+};
+
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmG,
+                  const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, int N, int topk,
+                  const int32_t* __restrict__ offs, const int32_t* __restrict__ list, float scale,
+                  const float* __restrict__ lse2, const float* __restrict__ delta, float* __restrict__ dK,
+                  float* __restrict__ dV) {
+  using L = KvLay;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(smem);
+  auto bar = [&](int k) { return sb + L::kBarOff + 8u * (uint32_t)k; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kSlotOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kSlotOff + 4);
+  const float* lsd = reinterpret_cast<const float*>(smem + L::kLsd);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nb = N / TB;
+  const int j = blockIdx.x;                    // key block
+  const int bh = blockIdx.y;
+  const int32_t* off = offs + (size_t)bh * (nb + 1);
+  const int32_t* lst = list + (size_t)bh * nb * topk + off[j];
+  const int C = off[j + 1] - off[j];           // query chunks (blocks that selected j)
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(L::B_KV), 1);
+    for (int s = 0; s < NR; ++s) {
+      mbar_init(bar(L::B_RF + s), 1);
+      mbar_init(bar(L::B_RE + s), 1);
+    }
+    mbar_init(bar(L::B_SF), 1);
+    mbar_init(bar(L::B_EW), 256);
+    mbar_init(bar(L::B_ACC), 1);
+    mbar_init(bar(L::B_FIN), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+
+  if (warp == kTmaWarp) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && C > 0) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmG);
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      mbar_expect_tx(bar(L::B_KV), 2 * kTile);
+      for (int h = 0; h < 2; ++h) {
+        tma_load_3d(sb + L::kK + h * kSpan, &tmK, 64 * h, j * TB, bh, bar(L::B_KV));
+        tma_load_3d(sb + L::kV + h * kSpan, &tmV, 64 * h, j * TB, bh, bar(L::B_KV));
+      }
+      int issued = 0;
+      for (int c = 0; c < C; ++c) {
+        const int s = c % NR;
+        if (c >= NR && !mbar_wait(bar(L::B_RE + s), ((c / NR) - 1) & 1, abort_flag)) break;
+        const int row0 = lst[c] * TB;
+        const uint32_t st = sb + L::kR + s * 2 * kTile;
+        mbar_expect_tx(bar(L::B_RF + s), 2 * kTile + 2 * TB * 4);
+        for (int h = 0; h < 2; ++h) {
+          tma_load_3d(st + h * kSpan, &tmQ, 64 * h, row0, bh, bar(L::B_RF + s));
+          tma_load_3d(st + kTile + h * kSpan, &tmG, 64 * h, row0, bh, bar(L::B_RF + s));
+        }
+        const uint32_t ls = sb + L::kLsd + s * 2 * TB * 4;
+        bulk_load(ls, lse2 + (size_t)bh * N + row0, TB * 4, bar(L::B_RF + s));
+        bulk_load(ls + TB * 4, delta + (size_t)bh * N + row0, TB * 4, bar(L::B_RF + s));
+        issued = c + 1;
+      }
+      if (*abort_flag) {
+        wait_bounded(bar(L::B_KV), 0);
+        for (int c = issued > NR ? issued - NR : 0; c < issued; ++c) wait_bounded(bar(L::B_RF + c % NR), (c / NR) & 1);
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    if (C > 0) {
+      constexpr uint32_t idS = idesc_bf16_f32(TB, TB, 0, 0);    // Sᵀ, dPᵀ: both operands K-major
+      constexpr uint32_t idA = idesc_bf16_f32(TB, TD, 0, 1);    // dV, dK: dO / Q as the MN-major operand
+      const uint64_t kd0 = desc_sw128(sb + L::kK, 16, 1024);
+      const uint64_t vd0 = desc_sw128(sb + L::kV, 16, 1024);
+      bool ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_KV), 0, abort_flag));
+      for (int c = 0; ok && c < C; ++c) {
+        const int s = c % NR;
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_RF + s), (c / NR) & 1, abort_flag))) break;
+        tc_fence_after();
+        const uint32_t st = sb + L::kR + s * 2 * kTile;
+        const uint64_t qd0 = desc_sw128(st, 16, 1024), gd0 = desc_sw128(st + kTile, 16, 1024);
+#pragma unroll
+        for (int k = 0; k < TD / 16; ++k) {
+          const uint32_t koff = (k >> 2) * kSpan + (k & 3) * 32;
+          mma_ss_w(tbase + kColST, desc_adv(kd0, koff), desc_adv(qd0, koff), idS, k > 0);
+        }
+#pragma unroll
+        for (int k = 0; k < TD / 16; ++k) {
+          const uint32_t koff = (k >> 2) * kSpan + (k & 3) * 32;
+          mma_ss_w(tbase + kColDPT, desc_adv(vd0, koff), desc_adv(gd0, koff), idS, k > 0);
+        }
+        mma_commit_w(bar(L::B_SF));
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_EW), c & 1, abort_flag))) break;
+        tc_fence_after();
+        const uint64_t qm0 = desc_sw128(st, kSpan, 1024), gm0 = desc_sw128(st + kTile, kSpan, 1024);
+#pragma unroll
+        for (int k = 0; k < TB / 16; ++k)
+          // K step k: 16 query rows = 16 rows of 128 bytes; 8 TMEM columns of Pᵀ
+          mma_ts_w(tbase + kColDV, tbase + kColST + 32 + 8 * k, desc_adv(gm0, k * 16 * 128), idA, (c > 0 || k > 0));
+#pragma unroll
+        for (int k = 0; k < TB / 16; ++k)
+          mma_ts_w(tbase + kColDK, tbase + kColDPT + 32 + 8 * k, desc_adv(qm0, k * 16 * 128), idA, (c > 0 || k > 0));
+        mma_commit_w(bar(L::B_RE + s));
+      }
+      mma_commit_w(bar(L::B_ACC));
+      mma_commit_w(bar(L::B_FIN));
+      wait_bounded(bar(L::B_FIN), 0);
+    }
+  } else if (warp < 8) {
+    // ------------------------------------------------------------ element-wise
+    const int grp = warp >> 2;                  // query-row half of every chunk
+    const int wq = warp & 3;                    // TMEM lane quarter
+    const int r = wq * 32 + lane;               // key within the block
+    const uint32_t lrow = tbase + ((uint32_t)(wq * 32) << 16);
+    const float scale2 = scale * kLog2e;
+    bool ok = true;
+    for (int c = 0; c < C; ++c) {
+      const int s = c % NR;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_SF), c & 1, abort_flag)) ||
+          !__all_sync(0xffffffffu, mbar_wait(bar(L::B_RF + s), (c / NR) & 1, abort_flag))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t v[64], p[64];
+      tmem_ld32(lrow + kColST + 64 * grp, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+      tmem_ld32(lrow + kColST + 64 * grp + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+      tmem_ld32(lrow + kColDPT + 64 * grp, *reinterpret_cast<uint32_t(*)[32]>(&p[0]));
+      tmem_ld32(lrow + kColDPT + 64 * grp + 32, *reinterpret_cast<uint32_t(*)[32]>(&p[32]));
+      tmem_wait_ld();
+      const float4* ls4 = reinterpret_cast<const float4*>(lsd + s * 2 * TB + 64 * grp);
+      const float4* dl4 = reinterpret_cast<const float4*>(lsd + s * 2 * TB + TB + 64 * grp);
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        const float4 la = ls4[q], da = dl4[q];
+        const float lq[4] = {la.x, la.y, la.z, la.w}, dq[4] = {da.x, da.y, da.z, da.w};
+        float pr[4], ds[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int cc = 4 * q + e;
+          pr[e] = fast_exp2(fmaf(__uint_as_float(v[cc]), scale2, -lq[e]));
+          ds[e] = pr[e] * (__uint_as_float(p[cc]) - dq[e]);
+        }
+        v[2 * q] = pack_bf16(pr[0], pr[1]);
+        v[2 * q + 1] = pack_bf16(pr[2], pr[3]);
+        p[2 * q] = pack_bf16(ds[0], ds[1]);
+        p[2 * q + 1] = pack_bf16(ds[2], ds[3]);
+      }
+      tmem_st32(lrow + kColST + 32 + 32 * grp, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+      tmem_st32(lrow + kColDPT + 32 + 32 * grp, *reinterpret_cast<uint32_t(*)[32]>(&p[0]));
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(L::B_EW));
+    }
+    ok = __all_sync(0xffffffffu, ok) && !*abort_flag;
+    if (ok && C > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_ACC), 0, abort_flag));
+    const size_t krow = ((size_t)bh * N + (size_t)j * TB + r) * TD + 64 * grp;
+    float4* ok4 = reinterpret_cast<float4*>(dK + krow);
+    float4* ov4 = reinterpret_cast<float4*>(dV + krow);
+    if (ok && C > 0) {
+      tc_fence_after();
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t a[32];
+        tmem_ld32(lrow + kColDV + 64 * grp + 32 * h, a);
+        tmem_wait_ld();
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          ov4[8 * h + q] = make_float4(__uint_as_float(a[4 * q]), __uint_as_float(a[4 * q + 1]),
+                                       __uint_as_float(a[4 * q + 2]), __uint_as_float(a[4 * q + 3]));
+        tmem_ld32(lrow + kColDK + 64 * grp + 32 * h, a);
+        tmem_wait_ld();
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          ok4[8 * h + q] = make_float4(scale * __uint_as_float(a[4 * q]), scale * __uint_as_float(a[4 * q + 1]),
+                                       scale * __uint_as_float(a[4 * q + 2]), scale * __uint_as_float(a[4 * q + 3]));
+      }
+    } else if (C == 0) {
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        ok4[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+        ov4[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tbase, kTmemCols);
+  }
+}
+
 }  // namespace
 
 sa_status bwd_dq_tc(const void* Q, const void* K, const void* V, const void* O, const void* dO, const sa_shape& s,
@@ -463,6 +694,23 @@ sa_status bwd_dq_tc(const void* Q, const void* K, const void* V, const void* O, 
       mq, mg, mk, mv, mkb, mvb, static_cast<const __nv_bfloat16*>(O), static_cast<const __nv_bfloat16*>(dO),
       block_idx, s.N, topk, zo ? 1 : 0, scale, lse2, delta, dQ);
   return launch_status("bwd_dq_tc_kernel");
+}
+
+sa_status bwd_dkv_tc(const void* Q, const void* K, const void* V, const void* dO, const sa_shape& s, int topk,
+                     const int32_t* offs, const int32_t* list, float scale, const float* lse2, const float* delta,
+                     float* dK, float* dV, cudaStream_t stream) {
+  const int nb = s.N / TB;
+  const uint64_t BH = (uint64_t)s.B * s.H;
+  alignas(64) CUtensorMap mq, mg, mk, mv;
+  if (!make_tmap_128x128(&mq, Q, 2, TD, s.N, BH) || !make_tmap_128x128(&mg, dO, 2, TD, s.N, BH) ||
+      !make_tmap_128x128(&mk, K, 2, TD, s.N, BH) || !make_tmap_128x128(&mv, V, 2, TD, s.N, BH))
+    return fail(SA_ERR_CUDA, "sa_sparse_attn_bwd: cuTensorMapEncodeTiled failed for Q/dO/K/V");
+  if (cudaFuncSetAttribute(bwd_dkv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)KvLay::kSmem) !=
+      cudaSuccess)
+    return launch_status("cudaFuncSetAttribute(bwd_dkv_tc_kernel)");
+  bwd_dkv_tc_kernel<<<dim3(nb, (unsigned)BH), kThreads, KvLay::kSmem, stream>>>(
+      mq, mg, mk, mv, s.N, topk, offs, list, scale, lse2, delta, dK, dV);
+  return launch_status("bwd_dkv_tc_kernel");
 }
 
 uint32_t bwd_error_take() {
