@@ -442,19 +442,23 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 // transposed index offs/list, ascending), with the keys as the MMA rows:
 //   Sᵀ = K Q_cᵀ, dPᵀ = V dO_cᵀ, Pᵀ = 2^(s' Sᵀ − lse2), dSᵀ = Pᵀ ⊙ (dPᵀ − δ),
 //   dV += Pᵀ dO_c, dK += dSᵀ Q_c     (dK scaled by s at the end).
-// Warps 0-7: element-wise, group g = warp / 4 takes query rows 64 g .. + 63
-// (TMEM columns) of every chunk; warp 8: TMA (K, V once; a ring of two
-// (Q, dO, lse2, δ) chunks); warp 9: MMA.  TMEM: Sᵀ [0,128), dPᵀ [128,256),
-// dV [256,384), dK [384,512); Pᵀ (bf16) goes to Sᵀ's columns [32, 96) and
-// dSᵀ to dPᵀ's, each group inside the columns it read itself.
+// Warps 0-7: element-wise, group h = warp / 4 owns query rows 64 h .. + 63
+// of every chunk (its half); warp 8: TMA (K, V once; a ring of two
+// (Q, dO, lse2, δ) chunks); warp 9: MMA.  Each half has its own Sᵀ and dPᵀ
+// (M = 128 keys, N = 64 rows), so while one group forms its Pᵀ and dSᵀ the
+// tensor pipe runs the other half's products: per chunk the MMA warp issues
+// dV, dK of half 0, then Sᵀ, dPᵀ of the next chunk's half 0, then the same
+// for half 1.  TMEM: half h at [128 h, 128 h + 128) (Sᵀ in the first 64
+// columns, dPᵀ in the next 64; Pᵀ and dSᵀ, bf16, overwrite the first 32 of
+// each), dV [256,384), dK [384,512).
 constexpr int NR = 2;                          // query-chunk ring depth
-constexpr uint32_t kColST = 0, kColDPT = 128, kColDV = 256, kColDK = 384;
+constexpr uint32_t kColDV = 256, kColDK = 384;
 
 struct KvLay {
   static constexpr uint32_t kK = 0, kV = kTile, kR = 2 * kTile;     // ring stage: Q, dO
   static constexpr uint32_t kLsd = kR + NR * 2 * kTile;             // [NR][lse2 128, δ 128] floats
-  static constexpr int B_KV = 0, B_RF = 1, B_RE = B_RF + NR, B_SF = B_RE + NR, B_EW = B_SF + 1,
-                       B_ACC = B_EW + 1, B_FIN = B_ACC + 1, NBAR = B_FIN + 1;
+  static constexpr int B_KV = 0, B_RF = 1, B_RE = B_RF + NR, B_SF = B_RE + NR, B_EW = B_SF + 2,
+                       B_ACC = B_EW + 2, B_FIN = B_ACC + 1, NBAR = B_FIN + 1;
   static constexpr uint32_t kBarOff = kLsd + NR * 2 * TB * 4;
   static constexpr uint32_t kSlotOff = kBarOff + 8 * NBAR;
   static constexpr size_t kSmem = 1024 + kSlotOff + 16;
@@ -495,8 +499,10 @@ bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
       mbar_init(bar(L::B_RF + s), 1);
       mbar_init(bar(L::B_RE + s), 1);
     }
-    mbar_init(bar(L::B_SF), 1);
-    mbar_init(bar(L::B_EW), 256);
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(bar(L::B_SF + h), 1);
+      mbar_init(bar(L::B_EW + h), 128);
+    }
     mbar_init(bar(L::B_ACC), 1);
     mbar_init(bar(L::B_FIN), 1);
     *abort_flag = 0;
@@ -544,39 +550,57 @@ bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (C > 0) {
-      constexpr uint32_t idS = idesc_bf16_f32(TB, TB, 0, 0);    // Sᵀ, dPᵀ: both operands K-major
+      constexpr uint32_t idS = idesc_bf16_f32(TB, 64, 0, 0);    // Sᵀ, dPᵀ of a half: both operands K-major
       constexpr uint32_t idA = idesc_bf16_f32(TB, TD, 0, 1);    // dV, dK: dO / Q as the MN-major operand
       const uint64_t kd0 = desc_sw128(sb + L::kK, 16, 1024);
       const uint64_t vd0 = desc_sw128(sb + L::kV, 16, 1024);
+      // Sᵀ and dPᵀ of half h of chunk c (rows 64 h .. + 63 start 8 KB into each span)
+      auto issue_s = [&](int c, int h) -> bool {
+        const int s = c % NR;
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_RF + s), (c / NR) & 1, abort_flag))) return false;
+        tc_fence_after();
+        const uint32_t st = sb + L::kR + s * 2 * kTile + 8192u * h;
+        const uint64_t qd0 = desc_sw128(st, 16, 1024), gd0 = desc_sw128(st + kTile, 16, 1024);
+        const uint32_t d = tbase + 128u * h;
+#pragma unroll
+        for (int k = 0; k < TD / 16; ++k) {
+          const uint32_t koff = (k >> 2) * kSpan + (k & 3) * 32;
+          mma_ss_w(d, desc_adv(kd0, koff), desc_adv(qd0, koff), idS, k > 0);
+        }
+#pragma unroll
+        for (int k = 0; k < TD / 16; ++k) {
+          const uint32_t koff = (k >> 2) * kSpan + (k & 3) * 32;
+          mma_ss_w(d + 64, desc_adv(vd0, koff), desc_adv(gd0, koff), idS, k > 0);
+        }
+        mma_commit_w(bar(L::B_SF + h));
+        return true;
+      };
       bool ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_KV), 0, abort_flag));
+      if (ok) ok = issue_s(0, 0);
+      if (ok) ok = issue_s(0, 1);
       for (int c = 0; ok && c < C; ++c) {
         const int s = c % NR;
-        if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_RF + s), (c / NR) & 1, abort_flag))) break;
-        tc_fence_after();
         const uint32_t st = sb + L::kR + s * 2 * kTile;
-        const uint64_t qd0 = desc_sw128(st, 16, 1024), gd0 = desc_sw128(st + kTile, 16, 1024);
-#pragma unroll
-        for (int k = 0; k < TD / 16; ++k) {
-          const uint32_t koff = (k >> 2) * kSpan + (k & 3) * 32;
-          mma_ss_w(tbase + kColST, desc_adv(kd0, koff), desc_adv(qd0, koff), idS, k > 0);
-        }
-#pragma unroll
-        for (int k = 0; k < TD / 16; ++k) {
-          const uint32_t koff = (k >> 2) * kSpan + (k & 3) * 32;
-          mma_ss_w(tbase + kColDPT, desc_adv(vd0, koff), desc_adv(gd0, koff), idS, k > 0);
-        }
-        mma_commit_w(bar(L::B_SF));
-        if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_EW), c & 1, abort_flag))) break;
-        tc_fence_after();
         const uint64_t qm0 = desc_sw128(st, kSpan, 1024), gm0 = desc_sw128(st + kTile, kSpan, 1024);
+        for (int h = 0; ok && h < 2; ++h) {
+          if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_EW + h), c & 1, abort_flag))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t pa = tbase + 128u * h;
 #pragma unroll
-        for (int k = 0; k < TB / 16; ++k)
-          // K step k: 16 query rows = 16 rows of 128 bytes; 8 TMEM columns of Pᵀ
-          mma_ts_w(tbase + kColDV, tbase + kColST + 32 + 8 * k, desc_adv(gm0, k * 16 * 128), idA, (c > 0 || k > 0));
+          for (int k = 0; k < 4; ++k)
+            // K step k: 16 query rows (64 h + 16 k ..) of 128 bytes; 8 TMEM columns of Pᵀ
+            mma_ts_w(tbase + kColDV, pa + 8 * k, desc_adv(gm0, (4 * h + k) * 16 * 128), idA,
+                     (c > 0 || h > 0 || k > 0));
 #pragma unroll
-        for (int k = 0; k < TB / 16; ++k)
-          mma_ts_w(tbase + kColDK, tbase + kColDPT + 32 + 8 * k, desc_adv(qm0, k * 16 * 128), idA, (c > 0 || k > 0));
-        mma_commit_w(bar(L::B_RE + s));
+          for (int k = 0; k < 4; ++k)
+            mma_ts_w(tbase + kColDK, pa + 64 + 8 * k, desc_adv(qm0, (4 * h + k) * 16 * 128), idA,
+                     (c > 0 || h > 0 || k > 0));
+          if (h == 1) mma_commit_w(bar(L::B_RE + s));
+          if (c + 1 < C) ok = issue_s(c + 1, h);
+        }
       }
       mma_commit_w(bar(L::B_ACC));
       mma_commit_w(bar(L::B_FIN));
@@ -584,7 +608,7 @@ bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     }
   } else if (warp < 8) {
     // ------------------------------------------------------------ element-wise
-    const int grp = warp >> 2;                  // query-row half of every chunk
+    const int grp = warp >> 2;                  // query-row half of every chunk (h)
     const int wq = warp & 3;                    // TMEM lane quarter
     const int r = wq * 32 + lane;               // key within the block
     const uint32_t lrow = tbase + ((uint32_t)(wq * 32) << 16);
@@ -592,17 +616,18 @@ bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     bool ok = true;
     for (int c = 0; c < C; ++c) {
       const int s = c % NR;
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_SF), c & 1, abort_flag)) ||
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_SF + grp), c & 1, abort_flag)) ||
           !__all_sync(0xffffffffu, mbar_wait(bar(L::B_RF + s), (c / NR) & 1, abort_flag))) {
         ok = false;
         break;
       }
       tc_fence_after();
+      const uint32_t hcol = lrow + 128u * grp;
       uint32_t v[64], p[64];
-      tmem_ld32(lrow + kColST + 64 * grp, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-      tmem_ld32(lrow + kColST + 64 * grp + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
-      tmem_ld32(lrow + kColDPT + 64 * grp, *reinterpret_cast<uint32_t(*)[32]>(&p[0]));
-      tmem_ld32(lrow + kColDPT + 64 * grp + 32, *reinterpret_cast<uint32_t(*)[32]>(&p[32]));
+      tmem_ld32(hcol, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+      tmem_ld32(hcol + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+      tmem_ld32(hcol + 64, *reinterpret_cast<uint32_t(*)[32]>(&p[0]));
+      tmem_ld32(hcol + 96, *reinterpret_cast<uint32_t(*)[32]>(&p[32]));
       tmem_wait_ld();
       const float4* ls4 = reinterpret_cast<const float4*>(lsd + s * 2 * TB + 64 * grp);
       const float4* dl4 = reinterpret_cast<const float4*>(lsd + s * 2 * TB + TB + 64 * grp);
@@ -622,11 +647,11 @@ bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         p[2 * q] = pack_bf16(ds[0], ds[1]);
         p[2 * q + 1] = pack_bf16(ds[2], ds[3]);
       }
-      tmem_st32(lrow + kColST + 32 + 32 * grp, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-      tmem_st32(lrow + kColDPT + 32 + 32 * grp, *reinterpret_cast<uint32_t(*)[32]>(&p[0]));
+      tmem_st32(hcol, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+      tmem_st32(hcol + 64, *reinterpret_cast<uint32_t(*)[32]>(&p[0]));
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar(L::B_EW));
+      mbar_arrive(bar(L::B_EW + grp));
     }
     ok = __all_sync(0xffffffffu, ok) && !*abort_flag;
     if (ok && C > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_ACC), 0, abort_flag));
