@@ -450,7 +450,7 @@ def time_backward(steps: int = 3, warmup: int = 3):
     ach = fl / (ms * 1e-3) / 1e12
     out = {"workload": w.name, "tail": w.tail, "ms": ms, "tflops": ach, "peak_tflops": bf16, "frac": ach / bf16,
            "peak_source": f"{src} bf16 burst",
-           "kernels": "bf16 tcgen05: dQ (+ lse, δ), key-major dK/dV of the exact keys; centroid dK/dV on mma.sync",
+           "kernels": "bf16 tcgen05: dQ (+ lse, δ); key-major dK/dV of the pseudo-keys (16 query ranges, reduced in order), then of the exact keys with the pseudo-key share added",
            "flops_per_call": fl}
     del inp, step, O, dO, dQ, dK, dV, ws
     torch.cuda.empty_cache()

@@ -65,11 +65,13 @@ size_t bwd_tc_part_bytes(const sa_shape& s);
 sa_status bwd_dq_tc(const void* Q, const void* K, const void* V, const void* O, const void* dO, const sa_shape& s,
                     const int32_t* block_idx, int topk, bool zo, const sa_block_stats& st, float scale, float* lse2,
                     float* delta, float* dQ, cudaStream_t stream);
-// dK, dV of the exact keys on tcgen05 (bwd_tc.cu), block 128, d = 128:
-// written for every key (zero where no query block selected its block).
-sa_status bwd_dkv_tc(const void* Q, const void* K, const void* V, const void* dO, const sa_shape& s, int topk,
-                     const int32_t* offs, const int32_t* list, float scale, const float* lse2, const float* delta,
-                     float* dK, float* dV, cudaStream_t stream);
+// dK, dV on tcgen05 (bwd_tc.cu), block 128, d = 128, written for every key:
+// the exact keys' sums plus, with the zero-order tail (zo), each block's
+// pseudo-key gradients ÷B (formed first in `part`, nsplit query ranges).
+sa_status bwd_dkv_tc(const void* Q, const void* K, const void* V, const void* dO, const sa_shape& s,
+                     const int32_t* block_idx, int topk, bool zo, const sa_block_stats& st, const int32_t* offs,
+                     const int32_t* list, float scale, const float* lse2, const float* delta, float* dK, float* dV,
+                     float* part, int nsplit, cudaStream_t stream);
 uint32_t bwd_error_take();
 
 }  // namespace sa

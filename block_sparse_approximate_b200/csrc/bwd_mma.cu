@@ -301,7 +301,7 @@ bwd_dq_mma_kernel(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __re
 // few centroid tiles still fill the GPU), masked where the row's block
 // selected the centroid; the partial dk̄, dv̄ go to `part`, which
 // bwd_centroid_scatter_kernel sums in order and spreads ÷B over the blocks.
-constexpr int kCentSplits = 8;
+constexpr int kCentSplits = 16;
 template <int BLK, bool CENT>
 __global__ void __launch_bounds__(kMThreads)
 bwd_dkv_mma_kernel(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
@@ -555,8 +555,8 @@ sa_status bwd_tc_launch(const void* Q, const void* K, const void* V, const void*
   }
   const size_t smem = 6 * (size_t)kMTileB + 2 * 2 * kMT * sizeof(float);
   if constexpr (BLK == 128) {
-    sa_status r = bwd_dkv_tc(Q, K, V, dO, s, topk, offs, list, scale, lse2, delta, dK, dV, stream);
-    if (r != SA_OK || !zo) return r;
+    return bwd_dkv_tc(Q, K, V, dO, s, block_idx, topk, zo, st, offs, list, scale, lse2, delta, dK, dV, part,
+                      kCentSplits, stream);
   } else {
     auto kern = bwd_dkv_mma_kernel<BLK, false>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)

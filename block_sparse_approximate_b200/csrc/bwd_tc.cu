@@ -470,12 +470,22 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
                : "memory");
 }
 
+// CENT = false: the keys of block j over the query blocks that selected it;
+// dK = s acc + (s / B) dk̄_j and dV = acc + dv̄_j / B, with dk̄_j, dv̄_j the
+// block's pseudo-key gradients (cent_k, cent_v; null without the tail).
+// CENT = true: 128 pseudo-keys (tmK, tmV over the bf16 centroids, bias
+// log2 B) over one of nsplit ranges of the head's query blocks, masked where
+// the query block selected the centroid's block; the unscaled sums go to
+// part[2][nsplit][BH][nb][d] for bwd_cent_reduce_kernel.
+template <bool CENT>
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmG,
                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, int N, int topk,
-                  const int32_t* __restrict__ offs, const int32_t* __restrict__ list, float scale,
-                  const float* __restrict__ lse2, const float* __restrict__ delta, float* __restrict__ dK,
-                  float* __restrict__ dV) {
+                  const int32_t* __restrict__ offs, const int32_t* __restrict__ list,
+                  const int32_t* __restrict__ block_idx, int nsplit, float scale, const float* __restrict__ lse2,
+                  const float* __restrict__ delta, const float* __restrict__ cent_k,
+                  const float* __restrict__ cent_v, float* __restrict__ dK, float* __restrict__ dV,
+                  float* __restrict__ part) {
   using L = KvLay;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -487,11 +497,21 @@ bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nb = N / TB;
-  const int j = blockIdx.x;                    // key block
   const int bh = blockIdx.y;
-  const int32_t* off = offs + (size_t)bh * (nb + 1);
-  const int32_t* lst = list + (size_t)bh * nb * topk + off[j];
-  const int C = off[j + 1] - off[j];           // query chunks (blocks that selected j)
+  // key tile j (exact: block j; centroids: centroids 128 j ..) and its query chunks
+  int j, C, qlo = 0, split = 0;
+  const int32_t* lst = nullptr;
+  if (CENT) {
+    j = blockIdx.x / nsplit;
+    split = blockIdx.x % nsplit;
+    qlo = (int)(((long)nb * split) / nsplit);
+    C = (int)(((long)nb * (split + 1)) / nsplit) - qlo;
+  } else {
+    j = blockIdx.x;
+    const int32_t* off = offs + (size_t)bh * (nb + 1);
+    lst = list + (size_t)bh * nb * topk + off[j];
+    C = off[j + 1] - off[j];                   // query blocks that selected block j
+  }
 
   if (threadIdx.x == 0) {
     mbar_init(bar(L::B_KV), 1);
@@ -530,7 +550,7 @@ bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
       for (int c = 0; c < C; ++c) {
         const int s = c % NR;
         if (c >= NR && !mbar_wait(bar(L::B_RE + s), ((c / NR) - 1) & 1, abort_flag)) break;
-        const int row0 = lst[c] * TB;
+        const int row0 = (CENT ? qlo + c : lst[c]) * TB;
         const uint32_t st = sb + L::kR + s * 2 * kTile;
         mbar_expect_tx(bar(L::B_RF + s), 2 * kTile + 2 * TB * 4);
         for (int h = 0; h < 2; ++h) {
@@ -631,6 +651,15 @@ bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
       tmem_wait_ld();
       const float4* ls4 = reinterpret_cast<const float4*>(lsd + s * 2 * TB + 64 * grp);
       const float4* dl4 = reinterpret_cast<const float4*>(lsd + s * 2 * TB + TB + 64 * grp);
+      // pseudo-keys: live unless past the head's blocks or selected by this query block
+      bool live = true;
+      if (CENT) {
+        const int jj = j * TB + r;
+        live = jj < nb;
+        const int32_t* sq = block_idx + ((size_t)bh * nb + qlo + c) * (size_t)topk;
+        for (int x = 0; x < topk; ++x) live &= __ldg(sq + x) != jj;
+      }
+      const float bias = CENT ? 7.0f : 0.f;   // log2 of the block size 128
 #pragma unroll
       for (int q = 0; q < 16; ++q) {
         const float4 la = ls4[q], da = dl4[q];
@@ -639,7 +668,7 @@ bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int cc = 4 * q + e;
-          pr[e] = fast_exp2(fmaf(__uint_as_float(v[cc]), scale2, -lq[e]));
+          pr[e] = live ? fast_exp2(fmaf(__uint_as_float(v[cc]), scale2, bias - lq[e])) : 0.f;
           ds[e] = pr[e] * (__uint_as_float(p[cc]) - dq[e]);
         }
         v[2 * q] = pack_bf16(pr[0], pr[1]);
@@ -655,32 +684,60 @@ bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     }
     ok = __all_sync(0xffffffffu, ok) && !*abort_flag;
     if (ok && C > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_ACC), 0, abort_flag));
-    const size_t krow = ((size_t)bh * N + (size_t)j * TB + r) * TD + 64 * grp;
-    float4* ok4 = reinterpret_cast<float4*>(dK + krow);
-    float4* ov4 = reinterpret_cast<float4*>(dV + krow);
+    // accumulators (zero without chunks), 64 channels of the thread's key
+    float acc_v[64], acc_k[64];
     if (ok && C > 0) {
       tc_fence_after();
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        uint32_t a[32];
-        tmem_ld32(lrow + kColDV + 64 * grp + 32 * h, a);
-        tmem_wait_ld();
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-          ov4[8 * h + q] = make_float4(__uint_as_float(a[4 * q]), __uint_as_float(a[4 * q + 1]),
-                                       __uint_as_float(a[4 * q + 2]), __uint_as_float(a[4 * q + 3]));
-        tmem_ld32(lrow + kColDK + 64 * grp + 32 * h, a);
-        tmem_wait_ld();
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-          ok4[8 * h + q] = make_float4(scale * __uint_as_float(a[4 * q]), scale * __uint_as_float(a[4 * q + 1]),
-                                       scale * __uint_as_float(a[4 * q + 2]), scale * __uint_as_float(a[4 * q + 3]));
+        tmem_ld32(lrow + kColDV + 64 * grp + 32 * h, *reinterpret_cast<uint32_t(*)[32]>(&acc_v[32 * h]));
+        tmem_ld32(lrow + kColDK + 64 * grp + 32 * h, *reinterpret_cast<uint32_t(*)[32]>(&acc_k[32 * h]));
       }
-    } else if (C == 0) {
+      tmem_wait_ld();
+    } else {
 #pragma unroll
-      for (int q = 0; q < 16; ++q) {
-        ok4[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-        ov4[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int e = 0; e < 64; ++e) acc_v[e] = acc_k[e] = 0.f;
+    }
+    if (ok || C == 0) {
+      if (CENT) {
+        const int jj = j * TB + r;
+        if (jj < nb) {
+          const size_t BHn = gridDim.y;
+          float4* pk4 = reinterpret_cast<float4*>(part + (((size_t)split * BHn + bh) * nb + jj) * TD + 64 * grp);
+          float4* pv4 =
+              reinterpret_cast<float4*>(part + (((size_t)(nsplit + split) * BHn + bh) * nb + jj) * TD + 64 * grp);
+#pragma unroll
+          for (int q = 0; q < 16; ++q) {
+            pk4[q] = make_float4(acc_k[4 * q], acc_k[4 * q + 1], acc_k[4 * q + 2], acc_k[4 * q + 3]);
+            pv4[q] = make_float4(acc_v[4 * q], acc_v[4 * q + 1], acc_v[4 * q + 2], acc_v[4 * q + 3]);
+          }
+        }
+      } else {
+        const size_t krow = ((size_t)bh * N + (size_t)j * TB + r) * TD + 64 * grp;
+        float4* ok4 = reinterpret_cast<float4*>(dK + krow);
+        float4* ov4 = reinterpret_cast<float4*>(dV + krow);
+        const size_t crow = ((size_t)bh * nb + j) * TD + 64 * grp;
+        const float sk = scale * (1.0f / TB), sv = 1.0f / TB;
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          float4 a = make_float4(scale * acc_k[4 * q], scale * acc_k[4 * q + 1], scale * acc_k[4 * q + 2],
+                                 scale * acc_k[4 * q + 3]);
+          float4 b = make_float4(acc_v[4 * q], acc_v[4 * q + 1], acc_v[4 * q + 2], acc_v[4 * q + 3]);
+          if (cent_k) {
+            const float4 ck = *reinterpret_cast<const float4*>(cent_k + crow + 4 * q);
+            const float4 cv = *reinterpret_cast<const float4*>(cent_v + crow + 4 * q);
+            a.x = fmaf(sk, ck.x, a.x);
+            a.y = fmaf(sk, ck.y, a.y);
+            a.z = fmaf(sk, ck.z, a.z);
+            a.w = fmaf(sk, ck.w, a.w);
+            b.x = fmaf(sv, cv.x, b.x);
+            b.y = fmaf(sv, cv.y, b.y);
+            b.z = fmaf(sv, cv.z, b.z);
+            b.w = fmaf(sv, cv.w, b.w);
+          }
+          ok4[q] = a;
+          ov4[q] = b;
+        }
       }
     }
   }
@@ -690,6 +747,19 @@ bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tbase, kTmemCols);
+  }
+}
+
+// dk̄_j, dv̄_j = the splits' partial sums in order, written over split 0
+// (one CTA per (centroid, head), thread = channel).
+__global__ void __launch_bounds__(TD)
+bwd_cent_reduce_kernel(float* __restrict__ part, int nb, int nsplit) {
+  const int j = blockIdx.x, c = threadIdx.x;
+  const size_t bh = blockIdx.y, BHn = gridDim.y;
+  for (int slot = 0; slot < 2; ++slot) {
+    float acc = 0.f;
+    for (int sp = 0; sp < nsplit; ++sp) acc += part[(((size_t)(slot * nsplit + sp) * BHn + bh) * nb + j) * TD + c];
+    part[(((size_t)(slot * nsplit) * BHn + bh) * nb + j) * TD + c] = acc;
   }
 }
 
@@ -721,20 +791,45 @@ sa_status bwd_dq_tc(const void* Q, const void* K, const void* V, const void* O, 
   return launch_status("bwd_dq_tc_kernel");
 }
 
-sa_status bwd_dkv_tc(const void* Q, const void* K, const void* V, const void* dO, const sa_shape& s, int topk,
-                     const int32_t* offs, const int32_t* list, float scale, const float* lse2, const float* delta,
-                     float* dK, float* dV, cudaStream_t stream) {
+sa_status bwd_dkv_tc(const void* Q, const void* K, const void* V, const void* dO, const sa_shape& s,
+                     const int32_t* block_idx, int topk, bool zo, const sa_block_stats& st, const int32_t* offs,
+                     const int32_t* list, float scale, const float* lse2, const float* delta, float* dK, float* dV,
+                     float* part, int nsplit, cudaStream_t stream) {
   const int nb = s.N / TB;
   const uint64_t BH = (uint64_t)s.B * s.H;
   alignas(64) CUtensorMap mq, mg, mk, mv;
   if (!make_tmap_128x128(&mq, Q, 2, TD, s.N, BH) || !make_tmap_128x128(&mg, dO, 2, TD, s.N, BH) ||
       !make_tmap_128x128(&mk, K, 2, TD, s.N, BH) || !make_tmap_128x128(&mv, V, 2, TD, s.N, BH))
     return fail(SA_ERR_CUDA, "sa_sparse_attn_bwd: cuTensorMapEncodeTiled failed for Q/dO/K/V");
-  if (cudaFuncSetAttribute(bwd_dkv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)KvLay::kSmem) !=
-      cudaSuccess)
+  const float* cent_k = nullptr;
+  const float* cent_v = nullptr;
+  if (zo) {
+    // the pseudo-keys first: partial sums per query-block range, reduced in order
+    alignas(64) CUtensorMap mkb, mvb;
+    if (!make_tmap_128x128(&mkb, st.kmean_bf16, 2, TD, nb, BH) ||
+        !make_tmap_128x128(&mvb, st.vmean_bf16, 2, TD, nb, BH))
+      return fail(SA_ERR_CUDA, "sa_sparse_attn_bwd: cuTensorMapEncodeTiled failed for the block centroids");
+    auto kc = bwd_dkv_tc_kernel<true>;
+    if (cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)KvLay::kSmem) != cudaSuccess)
+      return launch_status("cudaFuncSetAttribute(bwd_dkv_tc_kernel)");
+    const int ntc = (nb + TB - 1) / TB;
+    kc<<<dim3(ntc * nsplit, (unsigned)BH), kThreads, KvLay::kSmem, stream>>>(
+        mq, mg, mkb, mvb, s.N, topk, offs, list, block_idx, nsplit, scale, lse2, delta, nullptr, nullptr, dK, dV,
+        part);
+    sa_status r = launch_status("bwd_dkv_tc_kernel(centroids)");
+    if (r != SA_OK) return r;
+    bwd_cent_reduce_kernel<<<dim3(nb, (unsigned)BH), TD, 0, stream>>>(part, nb, nsplit);
+    r = launch_status("bwd_cent_reduce_kernel");
+    if (r != SA_OK) return r;
+    cent_k = part;
+    cent_v = part + (size_t)nsplit * BH * nb * TD;
+  }
+  auto ke = bwd_dkv_tc_kernel<false>;
+  if (cudaFuncSetAttribute(ke, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)KvLay::kSmem) != cudaSuccess)
     return launch_status("cudaFuncSetAttribute(bwd_dkv_tc_kernel)");
-  bwd_dkv_tc_kernel<<<dim3(nb, (unsigned)BH), kThreads, KvLay::kSmem, stream>>>(
-      mq, mg, mk, mv, s.N, topk, offs, list, scale, lse2, delta, dK, dV);
+  ke<<<dim3(nb, (unsigned)BH), kThreads, KvLay::kSmem, stream>>>(mq, mg, mk, mv, s.N, topk, offs, list, block_idx,
+                                                                 nsplit, scale, lse2, delta, cent_k, cent_v, dK, dV,
+                                                                 part);
   return launch_status("bwd_dkv_tc_kernel");
 }
 
