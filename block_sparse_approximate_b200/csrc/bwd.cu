@@ -177,6 +177,78 @@ bwd_transpose_kernel(const int32_t* __restrict__ block_idx, int nb, int topk, in
   }
 }
 
+// The same lists from a selection bitmap in shared memory (nb ≤ 1024: at
+// most 128 KB): bit (i, j) set for j ∈ S_i, then one thread per KV block j
+// counts its column, a warp scans the counts, and each thread writes its
+// column's query blocks in ascending order.
+constexpr int kTrThreads = 1024;
+constexpr int kTrMaxBlocks = 1024;
+__global__ void __launch_bounds__(kTrThreads)
+bwd_transpose_bitmap_kernel(const int32_t* __restrict__ block_idx, int nb, int topk, int32_t* __restrict__ offs,
+                            int32_t* __restrict__ list) {
+  extern __shared__ uint32_t trs[];
+  const int W = (nb + 31) >> 5;
+  uint32_t* bm = trs;                                                 // [nb][W]
+  int32_t* cnt = reinterpret_cast<int32_t*>(trs + (size_t)nb * W);    // [nb]
+  const size_t bh = blockIdx.x;
+  const int32_t* idx = block_idx + bh * (size_t)nb * topk;
+  int32_t* off = offs + bh * (size_t)(nb + 1);
+  int32_t* lst = list + bh * (size_t)nb * topk;
+  for (int x = threadIdx.x; x < nb * W; x += blockDim.x) bm[x] = 0u;
+  __syncthreads();
+  for (int e = threadIdx.x; e < nb * topk; e += blockDim.x) {
+    const int i = e / topk, j = idx[e];
+    if ((unsigned)j < (unsigned)nb) atomicOr(&bm[i * W + (j >> 5)], 1u << (j & 31));
+  }
+  __syncthreads();
+  for (int j = threadIdx.x; j < nb; j += blockDim.x) {
+    int c = 0;
+    for (int i = 0; i < nb; ++i) c += (bm[i * W + (j >> 5)] >> (j & 31)) & 1u;
+    cnt[j] = c;
+  }
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    // exclusive scan: lane l sums a contiguous chunk, the warp scans the sums
+    const int lane = threadIdx.x, per = (nb + 31) / 32;
+    const int a = min(nb, lane * per), b = min(nb, a + per);
+    int sum = 0;
+    for (int x = a; x < b; ++x) sum += cnt[x];
+    int incl = sum;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int run = incl - sum;
+    for (int x = a; x < b; ++x) {
+      const int c = cnt[x];
+      cnt[x] = run;
+      off[x] = run;
+      run += c;
+    }
+    if (lane == 31) off[nb] = incl;
+  }
+  __syncthreads();
+  for (int j = threadIdx.x; j < nb; j += blockDim.x) {
+    int p = cnt[j];
+    for (int i = 0; i < nb; ++i)
+      if ((bm[i * W + (j >> 5)] >> (j & 31)) & 1u) lst[p++] = i;
+  }
+}
+
+sa_status launch_transpose(const int32_t* block_idx, int nb, int topk, int32_t* offs, int32_t* list, int BH,
+                           cudaStream_t stream) {
+  if (nb <= kTrMaxBlocks) {
+    const size_t smem = sizeof(uint32_t) * ((size_t)nb * ((nb + 31) / 32) + nb);
+    if (cudaFuncSetAttribute(bwd_transpose_bitmap_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+      return launch_status("cudaFuncSetAttribute(bwd_transpose_bitmap_kernel)");
+    bwd_transpose_bitmap_kernel<<<BH, kTrThreads, smem, stream>>>(block_idx, nb, topk, offs, list);
+    return launch_status("bwd_transpose_bitmap_kernel");
+  }
+  bwd_transpose_kernel<<<BH, kBwdThreads, 0, stream>>>(block_idx, nb, topk, offs, list);
+  return launch_status("bwd_transpose_kernel");
+}
+
 // ---- dQ -------------------------------------------------------------------
 // One CTA per 64 query rows; per staged tile of 32 keys (exact or centroid)
 // every warp computes, for each of its rows, p and dP with lane = key, then
@@ -520,8 +592,7 @@ sa_status launch_bwd(const void* Q, const void* K, const void* V, const void* O,
   if (bwd_tc_supports(dt, s, zo, st)) {
     // tensor-core kernels: the per-KV-block query lists first
     if (topk > 0) {
-      bwd_transpose_kernel<<<s.B * s.H, kBwdThreads, 0, stream>>>(block_idx, nb, topk, offs, list);
-      sa_status r = launch_status("bwd_transpose_kernel");
+      sa_status r = launch_transpose(block_idx, nb, topk, offs, list, s.B * s.H, stream);
       if (r != SA_OK) return r;
     } else if (cudaMemsetAsync(offs, 0, (size_t)s.B * s.H * (nb + 1) * sizeof(int32_t), stream) != cudaSuccess) {
       return launch_status("cudaMemsetAsync(bwd offsets)");
@@ -541,8 +612,7 @@ sa_status launch_bwd(const void* Q, const void* K, const void* V, const void* O,
     if (r != SA_OK) return r;
   }
   if (topk > 0) {
-    bwd_transpose_kernel<<<s.B * s.H, kBwdThreads, 0, stream>>>(block_idx, nb, topk, offs, list);
-    sa_status r = launch_status("bwd_transpose_kernel");
+    sa_status r = launch_transpose(block_idx, nb, topk, offs, list, s.B * s.H, stream);
     if (r != SA_OK) return r;
   } else if (cudaMemsetAsync(offs, 0, (size_t)s.B * s.H * (nb + 1) * sizeof(int32_t), stream) != cudaSuccess) {
     return launch_status("cudaMemsetAsync(bwd offsets)");
