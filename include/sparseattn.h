@@ -193,9 +193,12 @@ size_t sa_sparse_attn_bwd_workspace_size(sa_shape shape, int32_t topk);
  * divided by block (k̄ and vsum / block are means of the block's k and v).
  * Q, K, V, O, dO of `dtype`; block_idx, topk, tail, stats (kmean, vsum for
  * ZERO_ORDER) and scale as given to the forward.  workspace: at least
- * sa_sparse_attn_bwd_workspace_size() bytes, 16-byte aligned.  CUDA-core
- * kernels (fp32 arithmetic); the sums over query blocks run in a fixed
- * order, so the result does not depend on scheduling.
+ * sa_sparse_attn_bwd_workspace_size() bytes, 16-byte aligned.  bf16 with
+ * d = 128 runs on the tensor cores (tcgen05 with TMEM accumulators for
+ * block 128, warp-level MMAs for block 64; p and ds rounded to bf16 for the
+ * second products, as the forward rounds p); fp32 and d = 64 run on CUDA
+ * cores in fp32.  The sums over query blocks run in a fixed order (no
+ * atomics), so the result does not depend on scheduling.
  * Errors: SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED (other tails), SA_ERR_ALIGNMENT,
  *         SA_ERR_WORKSPACE. */
 sa_status sa_sparse_attn_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
