@@ -399,18 +399,22 @@ def time_sfa(steps: int = 10, warmup: int = 3):
     return out
 
 
-def backward_flops(w) -> float:
-    """FLOPs of the backward over the exact and pseudo-keys of every query row:
-    recomputed scores (2·d) for the lse pass, then per (row, key) in the dQ
-    pass 2·d (scores) + 2·d (dP) + 2·d (dQ), and in the key-side passes again
-    2·d (scores) + 2·d (dP) + 2·d (dV) + 2·d (dK): 16·d per (row, key)."""
+def backward_flops(w, with_lse: bool = False) -> float:
+    """FLOPs the backward executes over the exact and pseudo-keys of every
+    query row: per (row, key) the dQ pass forms 2·d (scores) + 2·d (dP) +
+    2·d (dQ) and the key-side passes again 2·d (scores) + 2·d (dP) + 2·d (dV) +
+    2·d (dK); without the forward's log-sum-exp the dQ kernel first recomputes
+    the scores once more (2·d): 14·d or 16·d per (row, key)."""
     keys = w.k * w.block + ((w.nb - w.k) if w.tail in ("zero_order", "first_order") else 0)
-    return 16.0 * w.d * keys * w.B * w.H * float(w.N)
+    return (14.0 if with_lse else 16.0) * w.d * keys * w.B * w.H * float(w.N)
 
 
 def time_backward(steps: int = 3, warmup: int = 3):
-    """Backward of the video_dit prefill (zero-order tail): forward step once,
-    then sa_sparse_attn_bwd timed on the saved inputs, output and a random dO."""
+    """Backward of the video_dit prefill (zero-order tail): forward step once
+    (with the rows' log-sum-exp, sa_sparse_attn_fwd_lse), then
+    sa_sparse_attn_bwd_lse timed on the saved inputs, output, log-sum-exp and
+    a random dO; sa_sparse_attn_bwd (which recomputes the log-sum-exp) is
+    timed beside it."""
     import ctypes
     from block_sparse_approximate_b200 import binding as bd
     from block_sparse_approximate_b200.pipeline import PrefillStep
@@ -427,6 +431,16 @@ def time_backward(steps: int = 3, warmup: int = 3):
     f = dict(device="cuda", dtype=torch.float32)
     dQ, dK, dV = torch.empty(O.shape, **f), torch.empty(O.shape, **f), torch.empty(O.shape, **f)
     buf = step.buf
+    L = torch.empty(O.shape[:3], **f)
+    bd.sparse_attn_fwd(inp["Q"], inp["K"], inp["V"], buf.block_idx, w.block, w.tail, buf.stats, w.scale, out=O,
+                       lse=L)
+
+    def bwd_lse():
+        bd._check("sa_sparse_attn_bwd_lse", lib.sa_sparse_attn_bwd_lse(
+            inp["Q"].data_ptr(), inp["K"].data_ptr(), inp["V"].data_ptr(), O.data_ptr(), dO.data_ptr(),
+            L.data_ptr(), bd.SA_BF16, shape, buf.block_idx.data_ptr(), int(w.k), bd.TAIL[w.tail],
+            ctypes.byref(step.cst), float(w.scale), dQ.data_ptr(), dK.data_ptr(), dV.data_ptr(), ws.data_ptr(),
+            ws.numel(), bd._stream(None)))
 
     def bwd():
         bd._check("sa_sparse_attn_bwd", lib.sa_sparse_attn_bwd(
@@ -435,24 +449,30 @@ def time_backward(steps: int = 3, warmup: int = 3):
             float(w.scale), dQ.data_ptr(), dK.data_ptr(), dV.data_ptr(), ws.data_ptr(), ws.numel(),
             bd._stream(None)))
 
-    for _ in range(warmup):
-        bwd()
-    torch.cuda.synchronize()
-    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s.record()
-    for _ in range(steps):
-        bwd()
-    e.record()
-    torch.cuda.synchronize()
-    ms = s.elapsed_time(e) / steps
-    fl = backward_flops(w)
+    def timed(fn):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        for _ in range(steps):
+            fn()
+        e.record()
+        torch.cuda.synchronize()
+        return s.elapsed_time(e) / steps
+
+    ms_recompute = timed(bwd)
+    ms = timed(bwd_lse)
+    fl = backward_flops(w, with_lse=True)
     _, bf16, _, src = _peaks()
     ach = fl / (ms * 1e-3) / 1e12
     out = {"workload": w.name, "tail": w.tail, "ms": ms, "tflops": ach, "peak_tflops": bf16, "frac": ach / bf16,
-           "peak_source": f"{src} bf16 burst",
-           "kernels": "bf16 tcgen05: dQ (+ lse, δ); key-major dK/dV of the pseudo-keys (16 query ranges, reduced in order), then of the exact keys with the pseudo-key share added",
+           "peak_source": f"{src} bf16 burst", "entry": "sa_sparse_attn_bwd_lse (the forward's log-sum-exp given)",
+           "ms_recompute_lse": ms_recompute,
+           "tflops_recompute_lse": backward_flops(w) / (ms_recompute * 1e-3) / 1e12,
+           "kernels": "bf16 tcgen05: dQ (+ δ; the lse pass only without the forward's lse); key-major dK/dV of the pseudo-keys (16 query ranges, reduced in order), then of the exact keys with the pseudo-key share added",
            "flops_per_call": fl}
-    del inp, step, O, dO, dQ, dK, dV, ws
+    del inp, step, O, dO, dQ, dK, dV, ws, L
     torch.cuda.empty_cache()
     return out
 

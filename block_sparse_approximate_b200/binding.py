@@ -28,7 +28,8 @@ TAIL = {"drop": 0, "zero_order": 1, "linear_mix": 2, "first_order": 3, "residual
 EXPORTS = ("sa_block_pool", "sa_route", "sa_sparse_attn_fwd", "sa_decode_workspace_size",
            "sa_decode_fwd", "sa_decode_fwd_static", "sa_quantize_e4m3", "sa_sparse_attn_fwd_fp8",
            "sa_sfa_encode", "sa_sfa_densify", "sa_sfa_workspace_size", "sa_sfa_attn_fwd",
-           "sa_sparse_attn_bwd_workspace_size", "sa_sparse_attn_bwd",
+           "sa_sparse_attn_bwd_workspace_size", "sa_sparse_attn_bwd", "sa_sparse_attn_fwd_lse",
+           "sa_sparse_attn_bwd_lse",
            "sa_device_error", "sa_last_error", "sa_version")
 
 
@@ -98,9 +99,13 @@ def load():
     lib.sa_sparse_attn_bwd_workspace_size.restype = sz
     lib.sa_sparse_attn_bwd.argtypes = [vp, vp, vp, vp, vp, ctypes.c_int, Shape, vp, i32, ctypes.c_int,
                                        ctypes.POINTER(BlockStats), f32, vp, vp, vp, vp, sz, vp]
+    lib.sa_sparse_attn_fwd_lse.argtypes = [vp, vp, vp, ctypes.c_int, Shape, vp, i32, ctypes.c_int,
+                                           ctypes.POINTER(BlockStats), f32, vp, vp, vp]
+    lib.sa_sparse_attn_bwd_lse.argtypes = [vp, vp, vp, vp, vp, vp, ctypes.c_int, Shape, vp, i32, ctypes.c_int,
+                                           ctypes.POINTER(BlockStats), f32, vp, vp, vp, vp, sz, vp]
     for fn in ("sa_block_pool", "sa_route", "sa_sparse_attn_fwd", "sa_decode_fwd", "sa_decode_fwd_static",
                "sa_quantize_e4m3", "sa_sparse_attn_fwd_fp8", "sa_sfa_encode", "sa_sfa_densify", "sa_sfa_attn_fwd",
-               "sa_sparse_attn_bwd"):
+               "sa_sparse_attn_bwd", "sa_sparse_attn_fwd_lse", "sa_sparse_attn_bwd_lse"):
         getattr(lib, fn).restype = ctypes.c_int
     lib.sa_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
     lib.sa_device_error.restype = ctypes.c_int
@@ -207,13 +212,21 @@ def route(stats: dict, shape, mode: str, topk: int, *, proj_q=None, proj_k=None,
 
 
 def sparse_attn_fwd(Q, K, V, block_idx, block: int, tail: str, stats: dict, scale: float, *,
-                    alpha=None, out=None, stream=None) -> torch.Tensor:
-    """Sparse prefill forward; returns O with the shape and dtype of Q."""
+                    alpha=None, out=None, lse=None, stream=None) -> torch.Tensor:
+    """Sparse prefill forward; returns O with the shape and dtype of Q.  With
+    ``lse`` (float32 [B,H,N]) the rows' log2 log-sum-exp is written there
+    (sa_sparse_attn_fwd_lse)."""
     lib = load()
     Bsz, H, N, d = Q.shape
     O = out if out is not None else torch.empty_like(Q)
     topk = block_idx.shape[-1] if block_idx is not None else 0
     cst = _stats_struct(stats or {})
+    if lse is not None:
+        _check("sa_sparse_attn_fwd_lse",
+               lib.sa_sparse_attn_fwd_lse(_ptr(Q), _ptr(K), _ptr(V), _dtype_code(Q), Shape(Bsz, H, N, d, block),
+                                          _ptr(block_idx) if topk > 0 else None, int(topk), TAIL[tail],
+                                          ctypes.byref(cst), float(scale), _ptr(O), _ptr(lse), _stream(stream)))
+        return O
     _check("sa_sparse_attn_fwd",
            lib.sa_sparse_attn_fwd(_ptr(Q), _ptr(K), _ptr(V), _dtype_code(Q),
                                   Shape(Bsz, H, N, d, block),
@@ -354,8 +367,10 @@ def sfa_attn_fwd(Qs, Ks, V, block: int, scale: float, *, workspace=None, out=Non
 
 
 def sparse_attn_bwd(Q, K, V, O, dO, block_idx, block: int, tail: str, stats: dict, scale: float, *,
-                    workspace=None, stream=None):
-    """Backward of sparse_attn_fwd (drop, zero_order): returns float32 (dQ, dK, dV)."""
+                    lse=None, workspace=None, stream=None):
+    """Backward of sparse_attn_fwd (drop, zero_order): returns float32 (dQ, dK, dV).
+    ``lse``: the forward's log-sum-exp (sparse_attn_fwd(..., lse=...)), which
+    sa_sparse_attn_bwd_lse uses instead of recomputing it."""
     lib = load()
     Bsz, H, N, d = Q.shape
     topk = block_idx.shape[-1] if block_idx is not None else 0
@@ -366,6 +381,13 @@ def sparse_attn_bwd(Q, K, V, O, dO, block_idx, block: int, tail: str, stats: dic
     f = dict(device=Q.device, dtype=torch.float32)
     dQ, dK, dV = torch.empty(Q.shape, **f), torch.empty(K.shape, **f), torch.empty(V.shape, **f)
     cst = _stats_struct(stats or {})
+    if lse is not None:
+        _check("sa_sparse_attn_bwd_lse",
+               lib.sa_sparse_attn_bwd_lse(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(dO), _ptr(lse), _dtype_code(Q),
+                                          shape, _ptr(block_idx) if topk > 0 else None, int(topk), TAIL[tail],
+                                          ctypes.byref(cst), float(scale), _ptr(dQ), _ptr(dK), _ptr(dV),
+                                          _ptr(workspace), workspace.numel(), _stream(stream)))
+        return dQ, dK, dV
     _check("sa_sparse_attn_bwd",
            lib.sa_sparse_attn_bwd(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(dO), _dtype_code(Q), shape,
                                   _ptr(block_idx) if topk > 0 else None, int(topk), TAIL[tail], ctypes.byref(cst),

@@ -17,7 +17,7 @@ sa_status attn_simt(const void* Q, const void* K, const void* V, sa_dtype dtype,
 // requests it takes).
 sa_status attn_tc(const void* Q, const void* K, const void* V, const sa_shape& s,
                   const int32_t* block_idx, int topk, sa_tail_mode tail, const float* alpha,
-                  const sa_block_stats& st, float scale, void* O, cudaStream_t stream);
+                  const sa_block_stats& st, float scale, void* O, float* lse_out, cudaStream_t stream);
 
 bool attn_tc_supports(sa_dtype dtype, const sa_shape& s, sa_tail_mode tail);
 
@@ -55,16 +55,16 @@ uint32_t covnorm_error_take();
 bool bwd_tc_supports(sa_dtype dtype, const sa_shape& s, bool zo, const sa_block_stats& st);
 sa_status bwd_tc(const void* Q, const void* K, const void* V, const void* O, const void* dO, const sa_shape& s,
                  const int32_t* block_idx, int topk, bool zo, const sa_block_stats& st, float scale, float* dQ,
-                 float* dK, float* dV, float* lse2, float* delta, const int32_t* offs, const int32_t* list,
-                 float* part, cudaStream_t stream);
+                 float* dK, float* dV, const float* lse_in, float* lse2, float* delta, const int32_t* offs,
+                 const int32_t* list, float* part, cudaStream_t stream);
 // bytes of the centroid pass's partial sums (workspace)
 size_t bwd_tc_part_bytes(const sa_shape& s);
 // dQ (with lse2 and delta) on tcgen05 (bwd_tc.cu): block 128, d = 128, at
 // least one tile per query block (topk > 0 or the zero-order tail); and the
 // read-and-clear of that kernel's bounded-wait error word.
 sa_status bwd_dq_tc(const void* Q, const void* K, const void* V, const void* O, const void* dO, const sa_shape& s,
-                    const int32_t* block_idx, int topk, bool zo, const sa_block_stats& st, float scale, float* lse2,
-                    float* delta, float* dQ, cudaStream_t stream);
+                    const int32_t* block_idx, int topk, bool zo, const sa_block_stats& st, float scale,
+                    const float* lse_in, float* lse2, float* delta, float* dQ, cudaStream_t stream);
 // dK, dV on tcgen05 (bwd_tc.cu), block 128, d = 128, written for every key:
 // the exact keys' sums plus, with the zero-order tail (zo), each block's
 // pseudo-key gradients ÷B (formed first in `part`, nsplit query ranges).

@@ -208,7 +208,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKb,
                const __grid_constant__ CUtensorMap tmVb, const __grid_constant__ CUtensorMap tmHb,
                const int32_t* __restrict__ block_idx, int nb, int topk, float scale2, F8Scales f8,
-               __nv_bfloat16* __restrict__ O, int N) {
+               __nv_bfloat16* __restrict__ O, int N, float* __restrict__ lse_out) {
   static_assert(!FO || (ZO && !F8), "the first-order tail extends the bf16 zero-order tail");
   using L = Layout<F8>;
   constexpr int NS = L::NS;
@@ -529,6 +529,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const float L_ = l0 * f0 + l1 * f1;
     // e4m3: O accumulated Σ P σ_V V̂ · kPScale / σ_Vmax
     const float inv = L_ > 0.f ? (F8 ? vmax / Fmt<true>::kPScale : 1.0f) / L_ : 0.f;
+    // the row's log-sum-exp of its logits in log2 units (for the backward)
+    if (lse_out && st == 0) lse_out[(size_t)bh * N + (size_t)i * TB + r] = L_ > 0.f ? M + log2f(L_) : INFINITY;
     // first-order: + Λ_t (s q_t)ᵀ H̄ with Λ_t = Σ_U e^{s q·k̄_j} on the merged
     // maximum (the centroid tiles' sums carry the factor 128 = e^{ln 128})
     float wfo = 0.f;
@@ -631,7 +633,7 @@ template <bool F8>
 sa_status launch_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mkb,
                     const CUtensorMap& mvb, const CUtensorMap& mhb, bool zo, bool fo, const sa_shape& s,
                     const int32_t* block_idx, int topk, float scale, const F8Scales& f8, void* O,
-                    cudaStream_t stream) {
+                    float* lse_out, cudaStream_t stream) {
   const int nb = s.N / TB;
   const size_t smem = Layout<F8>::smem_bytes(nb);
   auto kern = zo ? attn_tc_kernel<true, F8, false> : attn_tc_kernel<false, F8, false>;
@@ -642,7 +644,7 @@ sa_status launch_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensor
     return launch_status("cudaFuncSetAttribute(attn_tc_kernel)");
   dim3 grid(nb, (unsigned)((uint64_t)s.B * s.H));
   kern<<<grid, kTcThreads, smem, stream>>>(mq, mk, mv, mkb, mvb, mhb, block_idx, nb, topk, scale * kLog2e, f8,
-                                           static_cast<__nv_bfloat16*>(O), s.N);
+                                           static_cast<__nv_bfloat16*>(O), s.N, lse_out);
   return launch_status("attn_tc_kernel");
 }
 
@@ -1270,7 +1272,7 @@ bool attn_tc_supports(sa_dtype dtype, const sa_shape& s, sa_tail_mode tail) {
 
 sa_status attn_tc(const void* Q, const void* K, const void* V, const sa_shape& s, const int32_t* block_idx,
                   int topk, sa_tail_mode tail, const float* alpha, const sa_block_stats& st, float scale,
-                  void* O, cudaStream_t stream) {
+                  void* O, float* lse_out, cudaStream_t stream) {
   const int nb = s.N / TB;
   const uint64_t BH = (uint64_t)s.B * s.H;
   CUtensorMap mq, mk, mv, mkb, mvb;
@@ -1300,7 +1302,8 @@ sa_status attn_tc(const void* Q, const void* K, const void* V, const sa_shape& s
   }
   if (fo && !make_tmap_3d(&mhb, st.hbarT_bf16, 2, TD, TD, BH))
     return fail(SA_ERR_CUDA, "sa_sparse_attn_fwd: cuTensorMapEncodeTiled failed for H̄ᵀ");
-  return launch_tc<false>(mq, mk, mv, mkb, mvb, mhb, zo, fo, s, block_idx, topk, scale, F8Scales{}, O, stream);
+  return launch_tc<false>(mq, mk, mv, mkb, mvb, mhb, zo, fo, s, block_idx, topk, scale, F8Scales{}, O, lse_out,
+                          stream);
 }
 
 }  // namespace sa
@@ -1342,7 +1345,7 @@ extern "C" sa_status sa_sparse_attn_fwd_fp8(const sa_fp8_operands* ops, sa_shape
     mvb = mv;
   }
   F8Scales f8{ops->q_scale, ops->k_scale, ops->v_scale, ops->v_scale_max, ops->kbar_scale, ops->vbar_scale};
-  return launch_tc<true>(mq, mk, mv, mkb, mvb, mk, zo, false, shape, block_idx, topk, scale, f8, O,
+  return launch_tc<true>(mq, mk, mv, mkb, mvb, mk, zo, false, shape, block_idx, topk, scale, f8, O, nullptr,
                          as_stream(stream));
 }
 

@@ -575,7 +575,8 @@ BwdLayout bwd_layout(const sa_shape& s, int topk) {
 template <typename T, int D, int BLK>
 sa_status launch_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
                      const sa_shape& s, const int32_t* block_idx, int topk, bool zo, const sa_block_stats& st,
-                     float scale, float* dQ, float* dK, float* dV, char* ws, cudaStream_t stream) {
+                     float scale, float* dQ, float* dK, float* dV, const float* lse_in, char* ws,
+                     cudaStream_t stream) {
   const BwdLayout L = bwd_layout(s, topk);
   const int nb = s.N / BLK;
   float* lse2 = reinterpret_cast<float*>(ws + L.lse_off);
@@ -597,7 +598,7 @@ sa_status launch_bwd(const void* Q, const void* K, const void* V, const void* O,
     } else if (cudaMemsetAsync(offs, 0, (size_t)s.B * s.H * (nb + 1) * sizeof(int32_t), stream) != cudaSuccess) {
       return launch_status("cudaMemsetAsync(bwd offsets)");
     }
-    return bwd_tc(Q, K, V, O, dO, s, block_idx, topk, zo, st, scale, dQ, dK, dV, lse2, delta, offs, list,
+    return bwd_tc(Q, K, V, O, dO, s, block_idx, topk, zo, st, scale, dQ, dK, dV, lse_in, lse2, delta, offs, list,
                   reinterpret_cast<float*>(ws + L.part_off), stream);
   }
   {
@@ -640,10 +641,12 @@ sa_status launch_bwd(const void* Q, const void* K, const void* V, const void* O,
 template <typename T>
 sa_status dispatch_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
                        const sa_shape& s, const int32_t* block_idx, int topk, bool zo, const sa_block_stats& st,
-                       float scale, float* dQ, float* dK, float* dV, char* ws, cudaStream_t stream) {
+                       float scale, float* dQ, float* dK, float* dV, const float* lse_in, char* ws,
+                       cudaStream_t stream) {
 #define SA_BWD_CASE(DD, BB)                                                                              \
   if (s.d == DD && s.block == BB)                                                                        \
-    return launch_bwd<T, DD, BB>(Q, K, V, O, dO, s, block_idx, topk, zo, st, scale, dQ, dK, dV, ws, stream);
+    return launch_bwd<T, DD, BB>(Q, K, V, O, dO, s, block_idx, topk, zo, st, scale, dQ, dK, dV, lse_in, ws,  \
+                                 stream);
   SA_BWD_CASE(128, 128)
   SA_BWD_CASE(128, 64)
   SA_BWD_CASE(64, 128)
@@ -661,12 +664,13 @@ extern "C" size_t sa_sparse_attn_bwd_workspace_size(sa_shape shape, int32_t topk
   return bwd_layout(shape, topk).total;
 }
 
-extern "C" sa_status sa_sparse_attn_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
-                                        sa_dtype dtype, sa_shape shape, const int32_t* block_idx, int32_t topk,
-                                        sa_tail_mode tail, const sa_block_stats* stats, float scale, float* dQ,
-                                        float* dK, float* dV, void* workspace, size_t workspace_bytes,
-                                        void* stream) {
-  using namespace sa;
+namespace sa {
+namespace {
+// lse_in: the forward's log-sum-exp (sa_sparse_attn_fwd_lse) or null
+sa_status bwd_entry(const void* Q, const void* K, const void* V, const void* O, const void* dO, sa_dtype dtype,
+                    sa_shape shape, const int32_t* block_idx, int32_t topk, sa_tail_mode tail,
+                    const sa_block_stats* stats, float scale, const float* lse_in, float* dQ, float* dK, float* dV,
+                    void* workspace, size_t workspace_bytes, void* stream) {
   sa_status r = check_shape(shape, "sa_sparse_attn_bwd");
   if (r != SA_OK) return r;
   const int nb = shape.N / shape.block;
@@ -688,12 +692,34 @@ extern "C" sa_status sa_sparse_attn_bwd(const void* Q, const void* K, const void
   const size_t need = bwd_layout(shape, topk).total;
   if (!workspace || workspace_bytes < need)
     return fail(SA_ERR_WORKSPACE, "sa_sparse_attn_bwd: workspace missing or smaller than the workspace size");
-  const void* ptrs[] = {Q, K, V, O, dO, dQ, dK, dV, workspace, block_idx, st.kmean, st.vsum};
+  const void* ptrs[] = {Q, K, V, O, dO, dQ, dK, dV, workspace, block_idx, st.kmean, st.vsum, lse_in};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return fail(SA_ERR_ALIGNMENT, "sa_sparse_attn_bwd: pointers must be 16-byte aligned");
   cudaStream_t s = as_stream(stream);
   char* ws = static_cast<char*>(workspace);
   if (dtype == SA_BF16)
-    return dispatch_bwd<__nv_bfloat16>(Q, K, V, O, dO, shape, block_idx, topk, zo, st, scale, dQ, dK, dV, ws, s);
-  return dispatch_bwd<float>(Q, K, V, O, dO, shape, block_idx, topk, zo, st, scale, dQ, dK, dV, ws, s);
+    return dispatch_bwd<__nv_bfloat16>(Q, K, V, O, dO, shape, block_idx, topk, zo, st, scale, dQ, dK, dV, lse_in,
+                                       ws, s);
+  return dispatch_bwd<float>(Q, K, V, O, dO, shape, block_idx, topk, zo, st, scale, dQ, dK, dV, lse_in, ws, s);
+}
+}  // namespace
+}  // namespace sa
+
+extern "C" sa_status sa_sparse_attn_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                                        sa_dtype dtype, sa_shape shape, const int32_t* block_idx, int32_t topk,
+                                        sa_tail_mode tail, const sa_block_stats* stats, float scale, float* dQ,
+                                        float* dK, float* dV, void* workspace, size_t workspace_bytes,
+                                        void* stream) {
+  return sa::bwd_entry(Q, K, V, O, dO, dtype, shape, block_idx, topk, tail, stats, scale, nullptr, dQ, dK, dV,
+                       workspace, workspace_bytes, stream);
+}
+
+extern "C" sa_status sa_sparse_attn_bwd_lse(const void* Q, const void* K, const void* V, const void* O,
+                                            const void* dO, const float* lse2, sa_dtype dtype, sa_shape shape,
+                                            const int32_t* block_idx, int32_t topk, sa_tail_mode tail,
+                                            const sa_block_stats* stats, float scale, float* dQ, float* dK,
+                                            float* dV, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!lse2) return sa::fail(SA_ERR_INVALID_ARG, "sa_sparse_attn_bwd_lse: lse2 is required");
+  return sa::bwd_entry(Q, K, V, O, dO, dtype, shape, block_idx, topk, tail, stats, scale, lse2, dQ, dK, dV,
+                       workspace, workspace_bytes, stream);
 }

@@ -15,7 +15,8 @@
 //              three and V tiles through a ring of two;
 //   warp 9     MMA issuer (converged; elect.sync picks the issuing lane).
 // Two passes over the row block's tiles (the selected blocks, then the
-// centroid tiles): pass 1 forms S = Q Kᵀ and the row's log-sum-exp; pass 2
+// centroid tiles): pass 1 forms S = Q Kᵀ and the row's log-sum-exp (skipped
+// when the forward's log-sum-exp is given); pass 2
 // forms S again, dP = dO Vᵀ, writes dS (bf16) into the S columns, and
 // accumulates dQ += dS · K with dS read from TMEM.
 // TMEM (512 columns): S₀ [0,128), S₁ [128,256) (tile g in S_{g mod 2}),
@@ -97,7 +98,8 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                  const __grid_constant__ CUtensorMap tmKb, const __grid_constant__ CUtensorMap tmVb,
                  const __nv_bfloat16* __restrict__ O, const __nv_bfloat16* __restrict__ dO,
                  const int32_t* __restrict__ block_idx, int N, int topk, int zo, float scale,
-                 float* __restrict__ lse2, float* __restrict__ delta, float* __restrict__ dQ) {
+                 const float* __restrict__ lse_in, float* __restrict__ lse2, float* __restrict__ delta,
+                 float* __restrict__ dQ) {
   using L = Lay;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -114,6 +116,9 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   const int nwords = (nb + 31) / 32;
   const int ntc = zo ? (nb + TB - 1) / TB : 0;  // centroid tiles
   const int T = topk + ntc;                    // tiles per pass
+  // pass-1 tiles: none when the forward's log-sum-exp is given; tile sequence
+  // g = 0 .. P1 + T - 1, the last T being pass 2
+  const int P1 = lse_in ? 0 : T, G = P1 + T;
   const int32_t* sel = block_idx + ((size_t)bh * nb + i) * (size_t)topk;
 
   if (threadIdx.x == 0) {
@@ -160,10 +165,10 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         tma_load_3d(sb + L::kQ + h * kSpan, &tmQ, 64 * h, i * TB, bh, bar(L::B_QG));
         tma_load_3d(sb + L::kG + h * kSpan, &tmG, 64 * h, i * TB, bh, bar(L::B_QG));
       }
-      // K loads n = 0 .. 2T-1 (tile n mod T); V loads of pass 2 follow their K
+      // K loads n = 0 .. G-1 (tile n, then n - P1 in pass 2); V loads of pass 2 follow their K
       int nk = 0, nv = 0;
-      for (int n = 0; n < 2 * T; ++n) {
-        const int t = n < T ? n : n - T;
+      for (int n = 0; n < G; ++n) {
+        const int t = n < P1 ? n : n - P1;
         const bool exact = t < topk;
         const int row = exact ? sel[t] * TB : (t - topk) * TB;
         {
@@ -175,7 +180,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                         bar(L::B_KF + s));
           nk = n + 1;
         }
-        if (n >= T) {
+        if (n >= P1) {
           const int s = t % NV;
           if (t >= NV && !mbar_wait(bar(L::B_VE + s), ((t / NV) - 1) & 1, abort_flag)) break;
           mbar_expect_tx(bar(L::B_VF + s), kTile);
@@ -212,7 +217,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
           mma_ss_w(d, desc_adv(qd0, koff), desc_adv(kd0, koff), idS, k > 0);
         }
         mma_commit_w(bar(L::B_SF + (g & 1)));
-        if (g < T) mma_commit_w(bar(L::B_KE + s));
+        if (g < P1) mma_commit_w(bar(L::B_KE + s));
         return true;
       };
       // dP(t) = dO V(t)ᵀ; releases the V stage
@@ -232,19 +237,19 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       };
       bool ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_QG), 0, abort_flag));
       if (ok) ok = issue_s(0);
-      if (ok && 2 * T > 1) ok = issue_s(1);
+      if (ok && G > 1) ok = issue_s(1);
       // pass 1: S only; a buffer is reissued once its S has been read
-      for (int g = 0; ok && g < T; ++g) {
+      for (int g = 0; ok && g < P1; ++g) {
         if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_SC + (g & 1)), (g >> 1) & 1, abort_flag))) {
           ok = false;
           break;
         }
-        if (g + 2 < 2 * T) ok = issue_s(g + 2);
+        if (g + 2 < G) ok = issue_s(g + 2);
       }
       // pass 2: dP one tile ahead, dQ += dS K once dS is in TMEM
       if (ok) ok = issue_dp(0);
-      for (int g = T; ok && g < 2 * T; ++g) {
-        const int t = g - T;
+      for (int g = P1; ok && g < G; ++g) {
+        const int t = g - P1;
         if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_SC + (g & 1)), (g >> 1) & 1, abort_flag))) {
           ok = false;
           break;
@@ -259,7 +264,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
           // K step k: 16 keys = 16 rows of 128 bytes into K; 8 TMEM columns of dS
           mma_ts_w(tbase + kColDQ, a0 + 8 * k, desc_adv(kd0, k * 16 * 128), idQ, (t > 0 || k > 0));
         mma_commit_w(bar(L::B_KE + s));
-        if (g + 2 < 2 * T) ok = issue_s(g + 2);
+        if (g + 2 < G) ok = issue_s(g + 2);
       }
       mma_commit_w(bar(L::B_DQ));
       // every MMA issued above has completed before TMEM is released
@@ -314,7 +319,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     bool ok = true;
     float m = -INFINITY, l = 0.f;
     // ---- pass 1: the row's running max and sum over its 64 keys of every tile
-    for (int g = 0; g < T; ++g) {
+    for (int g = 0; g < P1; ++g) {
       const int b = g & 1;
       if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_SF + b), (g >> 1) & 1, abort_flag))) {
         ok = false;
@@ -349,14 +354,20 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     // ---- the two groups' (max, sum) through the unused dQ columns
     ok = __all_sync(0xffffffffu, ok) && !*abort_flag;
     float lse = INFINITY;
-    if (ok) {
+    if (ok && P1 > 0) {
       tmem_st2(lrow + kColDQ + 2 * grp, __float_as_uint(m), __float_as_uint(l));
       tmem_wait_st();
     }
     tc_fence_before();
     named_bar_ew();
     tc_fence_after();
-    if (ok) {
+    if (ok && P1 == 0) {
+      lse = lse_in[row];
+      if (grp == 0) {
+        lse2[row] = lse;
+        delta[row] = dl;
+      }
+    } else if (ok) {
       uint32_t mo, lo;
       tmem_ld2(lrow + kColDQ + 2 * (1 - grp), mo, lo);
       tmem_wait_ld();
@@ -372,10 +383,10 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       }
     }
     // both groups have read the exchange before the first dQ MMA overwrites it
-    // (that MMA waits for every thread's arrival on the S barrier of tile T)
+    // (that MMA waits for every thread's arrival on the S barrier of tile P1)
     // ---- pass 2: dS = P (dP − δ) into the S columns [32, 96)
-    for (int g = T; ok && g < 2 * T; ++g) {
-      const int t = g - T, b = g & 1;
+    for (int g = P1; ok && g < G; ++g) {
+      const int t = g - P1, b = g & 1;
       if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_SF + b), (g >> 1) & 1, abort_flag)) ||
           !__all_sync(0xffffffffu, mbar_wait(bar(L::B_DPF), t & 1, abort_flag))) {
         ok = false;
@@ -766,8 +777,8 @@ bwd_cent_reduce_kernel(float* __restrict__ part, int nb, int nsplit) {
 }  // namespace
 
 sa_status bwd_dq_tc(const void* Q, const void* K, const void* V, const void* O, const void* dO, const sa_shape& s,
-                    const int32_t* block_idx, int topk, bool zo, const sa_block_stats& st, float scale, float* lse2,
-                    float* delta, float* dQ, cudaStream_t stream) {
+                    const int32_t* block_idx, int topk, bool zo, const sa_block_stats& st, float scale,
+                    const float* lse_in, float* lse2, float* delta, float* dQ, cudaStream_t stream) {
   const int nb = s.N / TB;
   const uint64_t BH = (uint64_t)s.B * s.H;
   alignas(64) CUtensorMap mq, mg, mk, mv, mkb, mvb;
@@ -787,7 +798,7 @@ sa_status bwd_dq_tc(const void* Q, const void* K, const void* V, const void* O, 
     return launch_status("cudaFuncSetAttribute(bwd_dq_tc_kernel)");
   bwd_dq_tc_kernel<<<dim3(nb, (unsigned)BH), kThreads, smem, stream>>>(
       mq, mg, mk, mv, mkb, mvb, static_cast<const __nv_bfloat16*>(O), static_cast<const __nv_bfloat16*>(dO),
-      block_idx, s.N, topk, zo ? 1 : 0, scale, lse2, delta, dQ);
+      block_idx, s.N, topk, zo ? 1 : 0, scale, lse_in, lse2, delta, dQ);
   return launch_status("bwd_dq_tc_kernel");
 }
 

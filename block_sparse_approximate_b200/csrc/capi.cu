@@ -29,13 +29,12 @@ extern "C" const char* sa_last_error(void) { return sa::g_last_error.c_str(); }
 
 extern "C" const char* sa_version(void) { return "libsparseattn 0.1 (sm_100a)"; }
 
-extern "C" sa_status sa_sparse_attn_fwd(const void* Q, const void* K, const void* V,
-                                        sa_dtype dtype, sa_shape shape,
-                                        const int32_t* block_idx, int32_t topk,
-                                        sa_tail_mode tail, const float* alpha,
-                                        const sa_block_stats* stats, float scale, void* O,
-                                        void* stream) {
-  using namespace sa;
+namespace sa {
+namespace {
+// lse2: the rows' log-sum-exp output (sa_sparse_attn_fwd_lse) or null
+sa_status fwd_entry(const void* Q, const void* K, const void* V, sa_dtype dtype, sa_shape shape,
+                    const int32_t* block_idx, int32_t topk, sa_tail_mode tail, const float* alpha,
+                    const sa_block_stats* stats, float scale, void* O, float* lse2, void* stream) {
   sa_status r = check_shape(shape, "sa_sparse_attn_fwd");
   if (r != SA_OK) return r;
   const int nb = shape.N / shape.block;
@@ -69,7 +68,33 @@ extern "C" sa_status sa_sparse_attn_fwd(const void* Q, const void* K, const void
   // the tensor-core kernel reads the tails' operands as bf16 tiles
   const bool tc_operands = (tail != SA_TAIL_ZERO_ORDER && tail != SA_TAIL_FIRST_ORDER) ||
                            (st.kmean_bf16 && st.vmean_bf16 && (tail == SA_TAIL_ZERO_ORDER || st.hbarT_bf16));
-  if (attn_tc_supports(dtype, shape, tail) && tc_operands)
-    return attn_tc(Q, K, V, shape, block_idx, topk, tail, alpha, st, scale, O, s);
+  const bool tc = attn_tc_supports(dtype, shape, tail) && tc_operands;
+  if (lse2) {
+    if (!tc || (tail != SA_TAIL_DROP && tail != SA_TAIL_ZERO_ORDER))
+      return fail(SA_ERR_UNSUPPORTED,
+                  "sa_sparse_attn_fwd_lse: the log-sum-exp comes from the bf16 tensor-core kernel (d = 128, "
+                  "block 128, SA_TAIL_DROP or SA_TAIL_ZERO_ORDER with the bf16 centroids)");
+    if (!aligned16(lse2)) return fail(SA_ERR_ALIGNMENT, "sa_sparse_attn_fwd_lse: lse2 must be 16-byte aligned");
+  }
+  if (tc) return attn_tc(Q, K, V, shape, block_idx, topk, tail, alpha, st, scale, O, lse2, s);
   return attn_simt(Q, K, V, dtype, shape, block_idx, topk, tail, alpha, st, scale, O, s);
+}
+}  // namespace
+}  // namespace sa
+
+extern "C" sa_status sa_sparse_attn_fwd(const void* Q, const void* K, const void* V,
+                                        sa_dtype dtype, sa_shape shape,
+                                        const int32_t* block_idx, int32_t topk,
+                                        sa_tail_mode tail, const float* alpha,
+                                        const sa_block_stats* stats, float scale, void* O,
+                                        void* stream) {
+  return sa::fwd_entry(Q, K, V, dtype, shape, block_idx, topk, tail, alpha, stats, scale, O, nullptr, stream);
+}
+
+extern "C" sa_status sa_sparse_attn_fwd_lse(const void* Q, const void* K, const void* V, sa_dtype dtype,
+                                            sa_shape shape, const int32_t* block_idx, int32_t topk,
+                                            sa_tail_mode tail, const sa_block_stats* stats, float scale,
+                                            void* O, float* lse2, void* stream) {
+  if (!lse2) return sa::fail(SA_ERR_INVALID_ARG, "sa_sparse_attn_fwd_lse: lse2 is required");
+  return sa::fwd_entry(Q, K, V, dtype, shape, block_idx, topk, tail, nullptr, stats, scale, O, lse2, stream);
 }

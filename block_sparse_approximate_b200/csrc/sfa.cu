@@ -222,6 +222,6 @@ extern "C" sa_status sa_sfa_attn_fwd(const void* Qs, const void* Ks, const void*
   if (r != SA_OK) return r;
   sa_block_stats st{};
   if (attn_tc_supports(dtype, shape, SA_TAIL_DROP))
-    return attn_tc(Qs, Ks, V, shape, idx, nb, SA_TAIL_DROP, nullptr, st, scale, O, s);
+    return attn_tc(Qs, Ks, V, shape, idx, nb, SA_TAIL_DROP, nullptr, st, scale, O, nullptr, s);
   return attn_simt(Qs, Ks, V, dtype, shape, idx, nb, SA_TAIL_DROP, nullptr, st, scale, O, s);
 }

@@ -178,6 +178,20 @@ sa_status sa_sparse_attn_fwd(const void* Q, const void* K, const void* V, sa_dty
                              const sa_block_stats* stats, float scale, void* O,
                              void* stream);
 
+/* sa_sparse_attn_fwd that also writes each query row's log-sum-exp of its
+ * logits in log2 units: lse2[b,h,t] = log2 Σ_key 2^(log2(e)·(s q_t·k + bias))
+ * over the row's exact keys and (ZERO_ORDER) pseudo-keys with bias ln block,
+ * +inf for a row without keys.  sa_sparse_attn_bwd_lse takes it to skip the
+ * recomputation of the row statistics.  lse2: float32 [B,H,N], caller-owned,
+ * 16-byte aligned.  Only the bf16 tensor-core kernel produces it: d = 128,
+ * block 128, SA_TAIL_DROP or SA_TAIL_ZERO_ORDER (with stats->kmean_bf16 and
+ * vmean_bf16); anything else returns SA_ERR_UNSUPPORTED.
+ * Errors: those of sa_sparse_attn_fwd; SA_ERR_INVALID_ARG without lse2. */
+sa_status sa_sparse_attn_fwd_lse(const void* Q, const void* K, const void* V, sa_dtype dtype,
+                                 sa_shape shape, const int32_t* block_idx, int32_t topk,
+                                 sa_tail_mode tail, const sa_block_stats* stats, float scale,
+                                 void* O, float* lse2, void* stream);
+
 /* Bytes of workspace sa_sparse_attn_bwd needs (0 on bad arguments). */
 size_t sa_sparse_attn_bwd_workspace_size(sa_shape shape, int32_t topk);
 
@@ -205,6 +219,17 @@ sa_status sa_sparse_attn_bwd(const void* Q, const void* K, const void* V, const 
                              sa_dtype dtype, sa_shape shape, const int32_t* block_idx, int32_t topk,
                              sa_tail_mode tail, const sa_block_stats* stats, float scale, float* dQ,
                              float* dK, float* dV, void* workspace, size_t workspace_bytes, void* stream);
+
+/* sa_sparse_attn_bwd given the forward's lse2 (sa_sparse_attn_fwd_lse, same
+ * inputs): the bf16 tensor-core path for block 128 then forms the scores
+ * once per tile instead of twice; other paths recompute the statistics and
+ * ignore lse2.  lse2: float32 [B,H,N], 16-byte aligned, required.
+ * Errors: those of sa_sparse_attn_bwd; SA_ERR_INVALID_ARG without lse2. */
+sa_status sa_sparse_attn_bwd_lse(const void* Q, const void* K, const void* V, const void* O,
+                                 const void* dO, const float* lse2, sa_dtype dtype, sa_shape shape,
+                                 const int32_t* block_idx, int32_t topk, sa_tail_mode tail,
+                                 const sa_block_stats* stats, float scale, float* dQ, float* dK,
+                                 float* dV, void* workspace, size_t workspace_bytes, void* stream);
 
 /* Per-block e4m3 quantisation [SLA2 §2C, low-precision sparse branch]:
  * X: bf16 [BH][N][d] (BH = batch x heads); codes: uint8 [BH][N][d] e4m3fn bit

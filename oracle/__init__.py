@@ -34,4 +34,4 @@ from .sparse_attention import (  # noqa: F401
     fp8_attention,
 )
 from .feature_sparse import sfa_codes, sfa_densify, sfa_attention  # noqa: F401
-from .backward import sparse_attention_backward  # noqa: F401
+from .backward import sparse_attention_backward, sparse_attention_lse  # noqa: F401

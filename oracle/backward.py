@@ -34,6 +34,37 @@ def _f64(x) -> np.ndarray:
     return np.asarray(x, dtype=np.float64)
 
 
+def sparse_attention_lse(Q, K, block_idx, block: int, tail: str, scale: float) -> np.ndarray:
+    """[B,H,N] float64: each query row's log-sum-exp of its logits in log2
+    units, log2 Σ exp(s q·k + bias) over the row's key list of
+    ``sparse_attention_backward`` (exact keys bias 0, pseudo-keys ln B); +inf
+    for a row without keys."""
+    if tail not in ("drop", "zero_order"):
+        raise ValueError("the log-sum-exp is defined for the drop and zero_order tails")
+    Q, K = _f64(Q), _f64(K)
+    Bsz, H, N, d = K.shape
+    nb = N // block
+    idx = np.asarray(block_idx)
+    out = np.full((Bsz, H, N), np.inf)
+    for b in range(Bsz):
+        for h in range(H):
+            Kh = K[b, h]
+            kbar = Kh.reshape(nb, block, d).mean(axis=1)
+            for i in range(N // block):
+                rows = slice(i * block, (i + 1) * block)
+                sel = sorted(int(j) for j in idx[b, h, i])
+                uns = [j for j in range(nb) if j not in set(sel)] if tail == "zero_order" else []
+                tok = [n for j in sel for n in range(j * block, (j + 1) * block)]
+                keys = np.concatenate([Kh[tok], kbar[uns]]) if tok or uns else np.zeros((0, d))
+                if keys.shape[0] == 0:
+                    continue
+                bias = np.concatenate([np.zeros(len(tok)), np.full(len(uns), np.log(block))])
+                a = scale * Q[b, h, rows] @ keys.T + bias
+                mx = a.max(axis=1, keepdims=True)
+                out[b, h, rows] = (mx[:, 0] + np.log(np.exp(a - mx).sum(axis=1))) / np.log(2.0)
+    return out
+
+
 def sparse_attention_backward(Q, K, V, block_idx, block: int, tail: str, scale: float, dO):
     """(dQ, dK, dV) [B,H,N,d] float64 of sparse_attention(tail) at (Q, K, V)
     for the output cotangent dO [B,H,N,d]; tail "drop" or "zero_order"."""

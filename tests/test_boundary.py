@@ -115,6 +115,33 @@ def test_sparse_attn_validation(lib):
         == bd.SA_ERR_INVALID_ARG            # unknown tail mode
 
 
+def test_lse_entry_validation(lib):
+    # the log-sum-exp entries: lse2 required, only the bf16 tensor-core forward produces it
+    sh = bd.Shape(1, 1, 1024, 128, 128)
+    none = _stats()
+    f = lib.sa_sparse_attn_fwd_lse
+    # every case returns before a launch (the pointers are never dereferenced)
+    assert f(FAKE, FAKE, FAKE, 1, sh, FAKE, 2, 0, ctypes.byref(none), 0.1, FAKE, None, None) \
+        == bd.SA_ERR_INVALID_ARG            # no lse2
+    assert f(FAKE, FAKE, FAKE, 0, sh, FAKE, 2, 0, ctypes.byref(none), 0.1, FAKE, FAKE, None) \
+        == bd.SA_ERR_UNSUPPORTED            # fp32 runs on the CUDA-core kernel
+    assert f(FAKE, FAKE, FAKE, 1, bd.Shape(1, 1, 1024, 64, 128), FAKE, 2, 0, ctypes.byref(none), 0.1, FAKE,
+             FAKE, None) == bd.SA_ERR_UNSUPPORTED   # d = 64
+    fo = _stats(kmean=FAKE, vsum=FAKE, hbar=FAKE, kmean_bf16=FAKE, vmean_bf16=FAKE, hbarT_bf16=FAKE)
+    assert f(FAKE, FAKE, FAKE, 1, sh, FAKE, 2, 3, ctypes.byref(fo), 0.1, FAKE, FAKE, None) \
+        == bd.SA_ERR_UNSUPPORTED            # first-order tail
+    assert f(FAKE, FAKE, FAKE, 1, sh, FAKE, 2, 0, ctypes.byref(none), 0.1, FAKE, FAKE + 4, None) \
+        == bd.SA_ERR_ALIGNMENT
+    g = lib.sa_sparse_attn_bwd_lse
+    big = 1 << 40
+    assert g(FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, sh, FAKE, 2, 0, ctypes.byref(none), 0.1, FAKE, FAKE, FAKE,
+             FAKE, big, None) == bd.SA_ERR_INVALID_ARG   # no lse2
+    assert g(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE + 4, 1, sh, FAKE, 2, 0, ctypes.byref(none), 0.1, FAKE, FAKE, FAKE,
+             FAKE, big, None) == bd.SA_ERR_ALIGNMENT
+    assert g(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, sh, FAKE, 2, 2, ctypes.byref(none), 0.1, FAKE, FAKE, FAKE,
+             FAKE, big, None) == bd.SA_ERR_UNSUPPORTED   # linear_mix has no backward
+
+
 def test_decode_validation_and_workspace(lib):
     sh = bd.DecodeShape(16, 32, 8, 131072, 128, 64)
     ws = lib.sa_decode_workspace_size(sh, 64)

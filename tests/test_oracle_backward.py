@@ -61,3 +61,38 @@ def test_drop_without_selection_has_no_gradient():
     idx = np.zeros((1, 2, 4, 0), dtype=np.int64)
     for g in oracle.sparse_attention_backward(Q, K, V, idx, blk, "drop", S, dO):
         assert not g.any()
+
+
+# ---- the rows' log-sum-exp (what sa_sparse_attn_fwd_lse writes) -------------
+
+@pytest.mark.parametrize("tail", ["zero_order", "drop"])
+def test_lse_every_block_selected_is_dense_logsumexp(tail):
+    # with every block selected there are no pseudo-keys: torch's logsumexp of
+    # the dense logits, in log2 units
+    rng = np.random.default_rng(21)
+    nb, blk, d = 4, 3, 4
+    Q, K = (rng.standard_normal((1, 2, nb * blk, d)) for _ in range(2))
+    idx = np.tile(np.arange(nb), (1, 2, nb, 1))
+    got = oracle.sparse_attention_lse(Q, K, idx, blk, tail, S)
+    ref = torch.logsumexp(S * torch.from_numpy(Q) @ torch.from_numpy(K).transpose(-1, -2), dim=-1) / np.log(2.0)
+    np.testing.assert_allclose(got, ref.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_lse_centroids_only():
+    # zero_order with nothing selected: log2 Σ_j B e^{s q·k̄_j} = log2 B +
+    # logsumexp_j(s q·k̄_j) / ln 2, the centroids taken with torch's mean
+    rng = np.random.default_rng(22)
+    nb, blk, d = 5, 4, 3
+    Q, K = (rng.standard_normal((1, 1, nb * blk, d)) for _ in range(2))
+    idx = np.zeros((1, 1, nb, 0), dtype=np.int64)
+    got = oracle.sparse_attention_lse(Q, K, idx, blk, "zero_order", S)
+    kbar = torch.from_numpy(K).reshape(1, 1, nb, blk, d).mean(dim=3)
+    ref = np.log2(blk) + torch.logsumexp(S * torch.from_numpy(Q) @ kbar.transpose(-1, -2), dim=-1) / np.log(2.0)
+    np.testing.assert_allclose(got, ref.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_lse_without_keys_is_infinite():
+    rng = np.random.default_rng(23)
+    Q, K = (rng.standard_normal((1, 1, 6, 2)) for _ in range(2))
+    got = oracle.sparse_attention_lse(Q, K, np.zeros((1, 1, 2, 0), dtype=np.int64), 3, "drop", S)
+    assert np.all(np.isinf(got)) and np.all(got > 0)

@@ -134,8 +134,15 @@ def test_backward_full_size_heads(lib):
     dO = torch.randn(O.shape, generator=g, device=DEV).to(O.dtype)
     dQ, dK, dV = bd.sparse_attn_bwd(inp["Q"], inp["K"], inp["V"], O, dO, step.buf.block_idx, w.block, w.tail,
                                     step.buf.stats, w.scale)
+    # the same through the forward's log-sum-exp (as bench.py times it)
+    L = torch.empty(O.shape[:3], device=DEV, dtype=torch.float32)
+    O2 = bd.sparse_attn_fwd(inp["Q"], inp["K"], inp["V"], step.buf.block_idx, w.block, w.tail, step.buf.stats,
+                            w.scale, lse=L)
+    grads_lse = bd.sparse_attn_bwd(inp["Q"], inp["K"], inp["V"], O2, dO, step.buf.block_idx, w.block, w.tail,
+                                   step.buf.stats, w.scale, lse=L)
     torch.cuda.synchronize()
     assert_no_device_error()
+    assert torch.equal(O2, O)
     for h in (0, w.H - 1):
         sl = slice(h, h + 1)
         sub = {n: inp[n][:, sl].cpu().float().numpy() for n in ("Q", "K", "V")}
@@ -149,3 +156,6 @@ def test_backward_full_size_heads(lib):
             # the gradient's own size
             scale_ref = max(1.0, float(np.abs(ref).max()))
             assert_tol(np64(got[:, sl]), ref, (2e-2 * scale_ref, 2e-3), f"backward head {h} {name}")
+        for got, ref, name in zip(grads_lse, (rQ, rK, rV), ("dQ", "dK", "dV")):
+            scale_ref = max(1.0, float(np.abs(ref).max()))
+            assert_tol(np64(got[:, sl]), ref, (2e-2 * scale_ref, 2e-3), f"backward (forward's lse) head {h} {name}")

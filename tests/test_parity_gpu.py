@@ -420,6 +420,39 @@ def test_sfa_attention(lib, d, block, N, kf):
 # --------------------------------------------------------------------------
 
 @pytest.mark.parametrize("tail", ["zero_order", "drop"])
+@pytest.mark.parametrize("nb,k", [(12, 3), (133, 13), (20, 0), (8, 8)])
+def test_forward_lse_and_backward_lse(lib, tail, nb, k):
+    # sa_sparse_attn_fwd_lse: O unchanged, lse2 against the oracle's row
+    # log-sum-exp; sa_sparse_attn_bwd_lse: gradients against the oracle
+    B, H, N, d, block = 1, 2, nb * 128, 128, 128
+    Q, K, V = _gauss(B, H, N, d, torch.bfloat16, 80 + nb + k)
+    g = torch.Generator(device=DEV)
+    g.manual_seed(81)
+    dO = torch.randn(B, H, N, d, generator=g, device=DEV).to(torch.bfloat16)
+    s = 1 / math.sqrt(d)
+    st = bd.block_pool(Q, K, V, block, centroids_bf16=True)
+    idx, _ = bd.route(st, (B, H, N, d, block), "dot", k)
+    O_plain = bd.sparse_attn_fwd(Q, K, V, idx, block, tail, st, s)
+    L = torch.empty(B, H, N, device=DEV, dtype=torch.float32)
+    O = bd.sparse_attn_fwd(Q, K, V, idx, block, tail, st, s, lse=L)
+    dQ, dK, dV = bd.sparse_attn_bwd(Q, K, V, O, dO, idx, block, tail, st, s, lse=L)
+    torch.cuda.synchronize()
+    assert_no_device_error()
+    assert torch.equal(O, O_plain)
+    ref_l = oracle.sparse_attention_lse(np64(Q), np64(K), idx.cpu().numpy(), block, tail, s)
+    got_l = L.cpu().numpy().astype(np.float64)
+    assert np.array_equal(np.isfinite(got_l), np.isfinite(ref_l))
+    fin = np.isfinite(ref_l)
+    # log2 units: the approximate exponentials (≤ 1e-4 relative per term) and
+    # the bf16 centroids move it by well under 2e-3
+    np.testing.assert_allclose(got_l[fin], ref_l[fin], rtol=0, atol=2e-3)
+    rQ, rK, rV = oracle.sparse_attention_backward(np64(Q), np64(K), np64(V), idx.cpu().numpy(), block, tail, s,
+                                                  np64(dO))
+    for got, ref, name in ((dQ, rQ, "dQ"), (dK, rK, "dK"), (dV, rV, "dV")):
+        assert_tol(np64(got), ref, (3e-2, 2e-3), f"backward with lse {tail} {name}")
+
+
+@pytest.mark.parametrize("tail", ["zero_order", "drop"])
 @pytest.mark.parametrize("dtype,d,block,nb,k", [
     (torch.float32, 64, 64, 9, 2),
     (torch.bfloat16, 128, 128, 12, 3),
