@@ -39,13 +39,6 @@ __device__ __forceinline__ void stage_keys(float* dst, const T* src, int row0, i
   }
 }
 
-// A tile of keys to visit for query block i: the exact blocks S_i in
-// 32-token pieces, then (zero-order) the centroids in pieces of 32.
-struct TileWalk {
-  int topk, blk, nb, pieces_exact, pieces_cent;
-  __device__ int count() const { return pieces_exact + pieces_cent; }
-};
-
 // selection bitmap of one query block into sel_bits (nwords words)
 __device__ __forceinline__ void load_selection(uint32_t* sel_bits, int nwords, const int32_t* sel, int topk) {
   for (int w = threadIdx.x; w < nwords; w += kBwdThreads) sel_bits[w] = 0u;

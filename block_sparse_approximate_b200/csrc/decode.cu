@@ -620,6 +620,8 @@ __device__ __forceinline__ void mma16816_top(float (&d)[2], uint32_t a0, uint32_
       "{%0,%1,%10,%10};"
       : "+f"(d[0]), "+f"(d[1]), "=f"(x2), "=f"(x3)
       : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1), "f"(0.f));
+  (void)x2;
+  (void)x3;
 }
 __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
