@@ -420,6 +420,31 @@ def test_sfa_attention(lib, d, block, N, kf):
 # --------------------------------------------------------------------------
 
 @pytest.mark.parametrize("tail", ["zero_order", "drop"])
+def test_backward_batched_heads(lib, tail):
+    # several sequences and heads: the (batch, head) indexing of the tensor
+    # maps, the query lists and the pseudo-key ranges of the tcgen05 backward
+    B, H, nb, k, d, block = 2, 3, 10, 3, 128, 128
+    N = nb * block
+    Q, K, V = _gauss(B, H, N, d, torch.bfloat16, 91)
+    g = torch.Generator(device=DEV)
+    g.manual_seed(92)
+    dO = torch.randn(B, H, N, d, generator=g, device=DEV).to(torch.bfloat16)
+    s = 1 / math.sqrt(d)
+    st = bd.block_pool(Q, K, V, block, centroids_bf16=True)
+    idx, _ = bd.route(st, (B, H, N, d, block), "dot", k)
+    L = torch.empty(B, H, N, device=DEV, dtype=torch.float32)
+    O = bd.sparse_attn_fwd(Q, K, V, idx, block, tail, st, s, lse=L)
+    grads = bd.sparse_attn_bwd(Q, K, V, O, dO, idx, block, tail, st, s)
+    grads_lse = bd.sparse_attn_bwd(Q, K, V, O, dO, idx, block, tail, st, s, lse=L)
+    torch.cuda.synchronize()
+    assert_no_device_error()
+    ref = oracle.sparse_attention_backward(np64(Q), np64(K), np64(V), idx.cpu().numpy(), block, tail, s, np64(dO))
+    for got_set, what in ((grads, "recomputed lse"), (grads_lse, "forward's lse")):
+        for got, r, name in zip(got_set, ref, ("dQ", "dK", "dV")):
+            assert_tol(np64(got), r, (3e-2, 2e-3), f"batched backward ({what}) {tail} {name}")
+
+
+@pytest.mark.parametrize("tail", ["zero_order", "drop"])
 @pytest.mark.parametrize("nb,k", [(12, 3), (133, 13), (20, 0), (8, 8)])
 def test_forward_lse_and_backward_lse(lib, tail, nb, k):
     # sa_sparse_attn_fwd_lse: O unchanged, lse2 against the oracle's row
