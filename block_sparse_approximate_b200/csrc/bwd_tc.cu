@@ -475,6 +475,12 @@ struct KvLay {
   static constexpr size_t kSmem = 1024 + kSlotOff + 16;
 };
 
+__device__ __forceinline__ float4 lds4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+  return v;
+}
+
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
                "l"(src), "r"(bytes), "r"(bar)
@@ -504,7 +510,6 @@ bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
   auto bar = [&](int k) { return sb + L::kBarOff + 8u * (uint32_t)k; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kSlotOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kSlotOff + 4);
-  const float* lsd = reinterpret_cast<const float*>(smem + L::kLsd);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nb = N / TB;
@@ -660,8 +665,9 @@ bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
       tmem_ld32(hcol + 64, *reinterpret_cast<uint32_t(*)[32]>(&p[0]));
       tmem_ld32(hcol + 96, *reinterpret_cast<uint32_t(*)[32]>(&p[32]));
       tmem_wait_ld();
-      const float4* ls4 = reinterpret_cast<const float4*>(lsd + s * 2 * TB + 64 * grp);
-      const float4* dl4 = reinterpret_cast<const float4*>(lsd + s * 2 * TB + TB + 64 * grp);
+      // the chunk's lse2 and δ of this group's 64 rows (shared-memory addresses)
+      const uint32_t ls_a = sb + L::kLsd + (uint32_t)(s * 2 * TB + 64 * grp) * 4u;
+      const uint32_t dl_a = ls_a + TB * 4u;
       // pseudo-keys: live unless past the head's blocks or selected by this query block
       bool live = true;
       if (CENT) {
@@ -673,7 +679,7 @@ bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
       const float bias = CENT ? 7.0f : 0.f;   // log2 of the block size 128
 #pragma unroll
       for (int q = 0; q < 16; ++q) {
-        const float4 la = ls4[q], da = dl4[q];
+        const float4 la = lds4(ls_a + 16u * q), da = lds4(dl_a + 16u * q);
         const float lq[4] = {la.x, la.y, la.z, la.w}, dq[4] = {da.x, da.y, da.z, da.w};
         float pr[4], ds[4];
 #pragma unroll
