@@ -82,6 +82,37 @@ __device__ __forceinline__ void tile_dots(const float* A, const float* T, int la
   }
 }
 
+// Radix select over a row of at most 32·KPL scores held KPL per lane in
+// registers: from the top bit down, counts (warp-wide) the keys whose high
+// bits equal `prefix` with the current bit set; `want` is the places left
+// among them, `cand` the keys still matching; stops once they agree.
+template <int KPL>
+__device__ __forceinline__ void radix_select_reg(const float* scw, int nb, int lane, unsigned& prefix, unsigned& hi,
+                                                 int& want, int& cand) {
+  unsigned key[KPL];
+#pragma unroll
+  for (int m = 0; m < KPL; ++m) {
+    const int j = lane + 32 * m;
+    key[m] = j < nb ? order_key(scw[j]) : 0u;
+  }
+  for (int bit = 31; bit >= 0; --bit) {
+    const unsigned bm = 1u << bit;
+    unsigned c = 0u;
+#pragma unroll
+    for (int m = 0; m < KPL; ++m) c += (lane + 32 * m < nb && (key[m] & hi) == prefix && (key[m] & bm)) ? 1u : 0u;
+    c = __reduce_add_sync(0xffffffffu, c);
+    if ((int)c >= want) {
+      prefix |= bm;
+      cand = (int)c;
+    } else {
+      want -= (int)c;
+      cand -= (int)c;
+    }
+    hi |= bm;
+    if (cand == want) break;
+  }
+}
+
 template <int D, int RPW, int NCOL>
 __global__ void __launch_bounds__(kRouteThreads)
 route_kernel(sa_block_stats st, int H, int nb, sa_route_mode mode, const float* __restrict__ Pq,
@@ -255,30 +286,10 @@ route_kernel(sa_block_stats st, int H, int nb, sa_route_mode mode, const float* 
       // 512 blocks keep their keys in registers.
       unsigned prefix = 0u, hi = 0u;
       int want = topk, cand = nb;
-      if (nb <= 32 * kRegKeys) {
-        unsigned key[kRegKeys];
-#pragma unroll
-        for (int m = 0; m < kRegKeys; ++m) {
-          const int j = lane + 32 * m;
-          key[m] = j < nb ? order_key(scw[j]) : 0u;
-        }
-        for (int bit = 31; bit >= 0; --bit) {
-          const unsigned bm = 1u << bit;
-          unsigned c = 0u;
-#pragma unroll
-          for (int m = 0; m < kRegKeys; ++m)
-            c += (lane + 32 * m < nb && (key[m] & hi) == prefix && (key[m] & bm)) ? 1u : 0u;
-          c = __reduce_add_sync(0xffffffffu, c);
-          if ((int)c >= want) {
-            prefix |= bm;
-            cand = (int)c;
-          } else {
-            want -= (int)c;
-            cand -= (int)c;
-          }
-          hi |= bm;
-          if (cand == want) break;
-        }
+      if (nb <= 32 * kRegKeys / 2) {
+        radix_select_reg<kRegKeys / 2>(scw, nb, lane, prefix, hi, want, cand);
+      } else if (nb <= 32 * kRegKeys) {
+        radix_select_reg<kRegKeys>(scw, nb, lane, prefix, hi, want, cand);
       } else {
         for (int bit = 31; bit >= 0; --bit) {
           const unsigned bm = 1u << bit;
