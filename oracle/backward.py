@@ -19,10 +19,15 @@ k̄_j = (1/B) Σ_n k_n and v̄_j = (1/B) Σ_n v_n: every token n of block j gets
 dk̄_j / B and dv̄_j / B (added to what it gets as an exact key of the query
 blocks that selected block j).
 
+The rows' log-sum-exp of that key list (``sparse_attention_lse``, log2
+units) is what the GPU forward can hand to its backward.
+
 Pins (``tests/test_oracle_backward.py``): central finite differences of the
 forward oracle on tiny inputs (both tails); with every block selected the
 gradients equal torch autograd of float64 softmax attention; drop with no
-selected block has zero gradients.
+selected block has zero gradients.  The log-sum-exp equals torch's
+``logsumexp`` of the dense logits when every block is selected, log2 B plus
+``logsumexp`` of the centroid logits when none is, and +inf without keys.
 """
 
 from __future__ import annotations
