@@ -179,9 +179,10 @@ sa_status sa_sparse_attn_fwd(const void* Q, const void* K, const void* V, sa_dty
                              void* stream);
 
 /* sa_sparse_attn_fwd that also writes each query row's log-sum-exp of its
- * logits in log2 units: lse2[b,h,t] = log2 Σ_key 2^(log2(e)·(s q_t·k + bias))
- * over the row's exact keys and (ZERO_ORDER) pseudo-keys with bias ln block,
- * +inf for a row without keys.  sa_sparse_attn_bwd_lse takes it to skip the
+ * logits in log2 units: lse2[b,h,t] = log2 D_t, D_t the denominator of PISA
+ * "Algoritmo Central" (Σ over the row's exact keys of e^{s q_t·k_n} plus,
+ * for ZERO_ORDER, Σ over the unselected blocks of block·e^{s q_t·k̄_j}; for
+ * DROP the first sum alone), +inf for a row without keys.  sa_sparse_attn_bwd_lse takes it to skip the
  * recomputation of the row statistics.  lse2: float32 [B,H,N], caller-owned,
  * 16-byte aligned.  Only the bf16 tensor-core kernel produces it: d = 128,
  * block 128, SA_TAIL_DROP or SA_TAIL_ZERO_ORDER (with stats->kmean_bf16 and
