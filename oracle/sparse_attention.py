@@ -67,7 +67,11 @@ Pins (the tests under ``tests/test_oracle_*.py``):
                       against torch.float8_e4m3fn
   quantise_blocks_e4m3  bounds of the format (|error| <= half an ulp)
   fp8_attention       on inputs already e4m3-exact per block the quantised
-                      forward equals sparse_attention (drop tail)
+                      forward equals sparse_attention (drop tail; zero-order
+                      tail with e4m3-exact block means over three centroid
+                      groups); a hand-quantised two-group worked example of
+                      the centroid path (bf16 then e4m3 ties, one scale per
+                      128 blocks, value means vsum/B)
 """
 
 from __future__ import annotations

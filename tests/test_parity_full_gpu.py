@@ -63,6 +63,7 @@ def test_decode_full_size_sampled(lib, name):
     step = DecodeStep(w, inp, st)
     o = step()
     torch.cuda.synchronize()
+    assert_no_device_error()
     check_topk_exact(step.idx, step.scores, w.k)
     pairs = [(0, 0), (7, 3), (15, 7)]
     g = w.H // w.Hkv
@@ -77,11 +78,7 @@ def test_decode_full_size_sampled(lib, name):
         assert_tol(np64(o[b, kh * g:(kh + 1) * g]), ref_o[0], BF16_TOL, f"decode b={b} g={kh}")
 
 
-def test_fp8_full_size_sampled(lib):
-    # e4m3 sparse branch against the oracle's quantised forward within the
-    # bound of P's e4m3 rounding (the pin); its distance to the unquantised
-    # float64 oracle is the format's own error on these inputs (reported, and
-    # only bounded loosely here)
+def _fp8_full_size_run():
     w = wl.WORKLOADS["fp8"]
     inp = wl.prefill_inputs(w, DEV)
     step = Fp8PrefillStep(w, inp)
@@ -95,14 +92,31 @@ def test_fp8_full_size_sampled(lib):
     sub = {n: inp[n][:, heads].cpu().float().numpy() for n in ("Q", "K", "V")}
     qb = [(b, hmap[h], i) for b, h, i in picks]
     got = np.stack([np64(O[b, h, i * w.block:(i + 1) * w.block]) for b, h, i in picks])
-    args = (sub["Q"], sub["K"], sub["V"], idx, w.block, w.tail, w.scale)
+    return w, got, (sub["Q"], sub["K"], sub["V"], idx, w.block, w.tail, w.scale), qb
+
+
+def test_fp8_full_size_sampled(lib):
+    # e4m3 sparse branch against the oracle's quantised forward, within the
+    # bound of P's e4m3 rounding and the bf16 store
+    _, got, args, qb = _fp8_full_size_run()
     emu = oracle.fp8_attention(*args, qblocks=qb)
     emu_abs = oracle.fp8_attention(*args, qblocks=qb, absolute_values=True)
     assert_fp8_bound(got, emu, emu_abs, "fp8 full size vs quantised forward")
-    ref = oracle.sparse_attention(sub["Q"], sub["K"], sub["V"], idx, w.block, w.tail, w.scale, qblocks=qb)
-    err = np.abs(got - ref)
-    print(f"fp8 vs unquantised float64 oracle: max-abs {err.max():.3e} mean-abs {err.mean():.3e}")
-    assert err.mean() < 4e-2 and err.max() < 0.8
+    ref = oracle.sparse_attention(*args, qblocks=qb)
+    err, err_emu = np.abs(got - ref), np.abs(emu - ref)
+    print(f"fp8 vs unquantised float64 oracle: max-abs {err.max():.3e} mean-abs {err.mean():.3e} "
+          f"(the exact e4m3 forward: {err_emu.max():.3e} / {err_emu.mean():.3e})")
+
+
+@pytest.mark.xfail(strict=True, reason="e4m3 format limit on these inputs: rounding Q, K, V to e4m3 with P "
+                   "kept exact already moves the output 0.34 max-abs / 0.020 mean-abs from the "
+                   "unquantised oracle (V alone: 0.10 / 0.004)")
+def test_fp8_full_size_within_fp8_tolerance_of_unquantised_oracle(lib):
+    # the e4m3 workload's stated tolerance against the unquantised float64
+    # oracle: max-abs 6e-2, mean-abs 6e-3
+    _, got, args, qb = _fp8_full_size_run()
+    ref = oracle.sparse_attention(*args, qblocks=qb)
+    assert_tol(got, ref, (6e-2, 6e-3), "fp8 full size vs unquantised oracle")
 
 
 def test_sfa_full_size_sampled(lib):
