@@ -20,7 +20,11 @@
 // A and C are persistent streaming kernels: each CTA walks a list of
 // 48 KB / 32 KB stages staged into shared memory with cp.async, three or four
 // stages deep, so the HBM stays busy while the previous stage is reduced.
+#include <cuda.h>
+
 #include <mutex>
+#include <utility>
+#include <vector>
 
 #include "topk.cuh"
 
@@ -1283,34 +1287,78 @@ extern "C" sa_status sa_decode_fwd(const void* q, const void* Kcache, const void
 // sa_decode_fwd_static runs the same kernels as sa_decode_fwd, with its
 // scratch (route scores, selected indices, per-split partial states) in this
 // file-scope device array instead of a caller workspace.  The array exists
-// once per device that loads the library and stays allocated until the
-// process exits.  Host code must not hand `g_decode_scratch` itself to a
-// kernel (on the host it names a shadow variable, not device memory); the
-// device address is looked up once per device with cudaGetSymbolAddress.
+// once per CUDA context that loads the library's module and stays allocated
+// until that context is destroyed (for the primary context: process exit or
+// cudaDeviceReset).  Host code must not hand `g_decode_scratch` itself to a
+// kernel (on the host it names a shadow variable, not device memory); its
+// device address is looked up with cudaGetSymbolAddress.
 static __device__ __align__(256) unsigned char g_decode_scratch[SA_DECODE_STATIC_SCRATCH_BYTES];
 
 namespace {
-constexpr int kMaxDevices = 64;
-std::mutex g_scratch_mu;
-void* g_scratch_addr[kMaxDevices] = {};
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
 
-// Device address of g_decode_scratch on the current device (looked up on the
-// first call per device, with that device current).
+struct CtxFns {
+  CtxGetCurrentFn get_current = nullptr;
+  CtxGetIdFn get_id = nullptr;
+};
+
+const CtxFns& ctx_fns() {
+  static CtxFns f;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      f.get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      f.get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  return f;
+}
+
+// Unique id of the current context (cuCtxGetId: ids are never reused within
+// a process, unlike context handles or device indices); 0 if none is current.
+unsigned long long current_ctx_id() {
+  const CtxFns& f = ctx_fns();
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!f.get_current || !f.get_id || f.get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  if (f.get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+std::mutex g_scratch_mu;
+// (context id, device address of g_decode_scratch in that context)
+std::vector<std::pair<unsigned long long, void*>> g_scratch_addr;
+
+// Device address of g_decode_scratch in the current context.  The address
+// belongs to the copy of the module loaded into one context, so it is cached
+// per context id: a context created by cudaDeviceReset, or a caller's own
+// context made current instead of the primary one, gets a lookup of its own.
+// The lookup (cudaGetSymbolAddress) also initialises the primary context
+// when none is current yet.
 sa_status static_scratch(void** out) {
   using namespace sa;
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess) return launch_status("sa_decode_fwd_static: cudaGetDevice");
-  if (dev < 0 || dev >= kMaxDevices) return fail(SA_ERR_UNSUPPORTED, "sa_decode_fwd_static: device index above 63");
+  unsigned long long id = current_ctx_id();
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_addr[dev] == nullptr) {
-    void* p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
-    if (e != cudaSuccess || p == nullptr)
-      return fail(SA_ERR_CUDA, std::string("sa_decode_fwd_static: cudaGetSymbolAddress failed: ") +
-                                   cudaGetErrorString(e));
-    g_scratch_addr[dev] = p;
-  }
-  *out = g_scratch_addr[dev];
+  if (id != 0)
+    for (const auto& e : g_scratch_addr)
+      if (e.first == id) {
+        *out = e.second;
+        return SA_OK;
+      }
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
+  if (e != cudaSuccess || p == nullptr)
+    return fail(SA_ERR_CUDA, std::string("sa_decode_fwd_static: cudaGetSymbolAddress failed: ") +
+                                 cudaGetErrorString(e));
+  if (id == 0) id = current_ctx_id();   // the lookup made the primary context current
+  if (id != 0) g_scratch_addr.emplace_back(id, p);
+  *out = p;
   return SA_OK;
 }
 }  // namespace

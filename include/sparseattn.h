@@ -312,9 +312,13 @@ sa_status sa_decode_fwd(const void* q, const void* Kcache, const void* Vcache, s
  *   - A problem whose sa_decode_workspace_size() exceeds
  *     SA_DECODE_STATIC_SCRATCH_BYTES is rejected with SA_ERR_WORKSPACE before
  *     anything runs.
- *   - The first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress, with that device current); make that first call
- *     before any stream capture.  Later calls do no set-up.
+ *   - The first call in each CUDA context looks up the array's device
+ *     address (cudaGetSymbolAddress, with that context current) and caches
+ *     it under the context's unique id (cuCtxGetId).  A device's primary
+ *     context is one such context; so is the new primary context after
+ *     cudaDeviceReset and any context the caller creates and makes current,
+ *     each with an array of its own.  Make the first call in a context before
+ *     any stream capture in it.  Later calls in that context do no set-up.
  *   - Every call on a device shares the one array and it keeps the last
  *     call's contents (nothing in it needs clearing: each call writes every
  *     entry before reading it).  Calls whose executions overlap on the GPU
