@@ -1,7 +1,10 @@
-"""Pins of the oracle's backward pass of the sparse prefill (drop and
-zero_order tails): central finite differences of the forward oracle, torch
-autograd of dense float64 attention when every block is selected, and zero
-gradients when nothing is attended."""
+"""Pins of the oracle's backward pass of the sparse prefill (every tail of
+the prefill): central finite differences of the forward oracle, torch
+autograd of dense float64 attention when every block is selected, torch
+autograd of float64 re-statements of PISA's hybrid order and of SLA2's
+mixture written with dense masks, the limits where the first-order and
+mixed tails reduce to the zero-order and drop ones, and zero gradients when
+nothing is attended."""
 
 import numpy as np
 import pytest
@@ -20,14 +23,18 @@ def _case(rng, nb=4, blk=3, d=4, H=2):
     return Q, K, V, idx, dO, blk
 
 
-@pytest.mark.parametrize("tail", ["zero_order", "drop"])
+ALPHA = np.array([[0.3, 0.8, 0.5, 0.6], [0.9, 0.2, 0.4, 0.7]])   # [H, d] of _case
+
+
+@pytest.mark.parametrize("tail", ["zero_order", "drop", "first_order", "linear_mix"])
 def test_finite_differences(tail):
     rng = np.random.default_rng(11)
     Q, K, V, idx, dO, blk = _case(rng)
-    dQ, dK, dV = oracle.sparse_attention_backward(Q, K, V, idx, blk, tail, S, dO)
+    alpha = ALPHA if tail == "linear_mix" else None
+    dQ, dK, dV = oracle.sparse_attention_backward(Q, K, V, idx, blk, tail, S, dO, alpha=alpha)
 
     def f(Qx, Kx, Vx):
-        return float((oracle.sparse_attention(Qx, Kx, Vx, idx, blk, tail, S) * dO).sum())
+        return float((oracle.sparse_attention(Qx, Kx, Vx, idx, blk, tail, S, alpha=alpha) * dO).sum())
 
     h = 1e-6
     for arr, grad, which in ((Q, dQ, 0), (K, dK, 1), (V, dV, 2)):
@@ -96,3 +103,119 @@ def test_lse_without_keys_is_infinite():
     Q, K = (rng.standard_normal((1, 1, 6, 2)) for _ in range(2))
     got = oracle.sparse_attention_lse(Q, K, np.zeros((1, 1, 2, 0), dtype=np.int64), 3, "drop", S)
     assert np.all(np.isinf(got)) and np.all(got > 0)
+
+
+# ---- PISA's hybrid order (first_order) ----------------------------------
+
+def _first_order_torch(Q, K, V, idx, blk, scale):
+    """PISA's hybrid order restated with dense masks over all tokens and all
+    block centroids (float64 torch, differentiable)."""
+    Bsz, H, N, d = Q.shape
+    nb = N // blk
+    Kb, Vb = K.reshape(Bsz, H, nb, blk, d), V.reshape(Bsz, H, nb, blk, d)
+    kbar, vsum = Kb.mean(dim=3), Vb.sum(dim=3)
+    hbar = torch.einsum("bhjnc,bhjne->bhce", Kb - kbar.unsqueeze(3), Vb) / nb
+    sel = torch.zeros(Bsz, H, nb, nb, dtype=torch.bool)             # [.., query block, key block]
+    for b in range(Bsz):
+        for h in range(H):
+            for i in range(nb):
+                sel[b, h, i, list(idx[b, h, i])] = True
+    sel_tok = sel.repeat_interleave(blk, dim=2).repeat_interleave(blk, dim=3)   # [.., N, N]
+    uns_row = (~sel).repeat_interleave(blk, dim=2)                               # [.., N, nb]
+    a = scale * Q @ K.transpose(-1, -2)
+    c = scale * Q @ kbar.transpose(-1, -2)
+    m = torch.maximum(a.masked_fill(~sel_tok, -1e300).amax(-1), c.masked_fill(~uns_row, -1e300).amax(-1))
+    wa = torch.exp(a - m[..., None]) * sel_tok
+    wc = torch.exp(c - m[..., None]) * uns_row
+    num = wa @ V + wc @ vsum + (scale * Q @ hbar) * wc.sum(-1, keepdim=True)
+    den = wa.sum(-1) + blk * wc.sum(-1)
+    return num / den[..., None]
+
+
+def test_first_order_matches_autograd_of_a_masked_restatement():
+    rng = np.random.default_rng(14)
+    Q, K, V, idx, dO, blk = _case(rng, nb=5, blk=3, d=4)
+    dQ, dK, dV = oracle.sparse_attention_backward(Q, K, V, idx, blk, "first_order", S, dO)
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (Q, K, V))
+    o = _first_order_torch(tq, tk, tv, idx, blk, S)
+    np.testing.assert_allclose(o.detach().numpy(), oracle.sparse_attention(Q, K, V, idx, blk, "first_order", S),
+                               rtol=1e-12, atol=1e-12)
+    o.backward(torch.tensor(dO))
+    for got, t in ((dQ, tq), (dK, tk), (dV, tv)):
+        np.testing.assert_allclose(got, t.grad.numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_first_order_with_block_constant_keys():
+    # constant keys inside every block give H̄ = 0: the output, dQ and dV are
+    # the zero-order ones; dK still differs, through H̄'s dependence on K
+    rng = np.random.default_rng(15)
+    Q, K, V, idx, dO, blk = _case(rng)
+    K = np.repeat(K[:, :, ::blk], blk, axis=2)
+    fo = oracle.sparse_attention_backward(Q, K, V, idx, blk, "first_order", S, dO)
+    zo = oracle.sparse_attention_backward(Q, K, V, idx, blk, "zero_order", S, dO)
+    np.testing.assert_allclose(fo[0], zo[0], rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(fo[2], zo[2], rtol=1e-12, atol=1e-13)
+    assert np.abs(fo[1] - zo[1]).max() > 1e-3
+
+
+# ---- SLA2's mixture (linear_mix) ------------------------------------------
+
+def _linear_mix_torch(Q, K, V, idx, blk, scale, alpha, eps=1e-6):
+    """SLA2's α⊙O_s + (1−α)⊙O_l restated with dense token masks."""
+    Bsz, H, N, d = Q.shape
+    nb = N // blk
+    sel = torch.zeros(Bsz, H, nb, nb, dtype=torch.bool)
+    for b in range(Bsz):
+        for h in range(H):
+            for i in range(nb):
+                sel[b, h, i, list(idx[b, h, i])] = True
+    sel_tok = sel.repeat_interleave(blk, dim=2).repeat_interleave(blk, dim=3)
+    a = (scale * Q @ K.transpose(-1, -2)).masked_fill(~sel_tok, float("-inf"))
+    has = sel_tok.any(-1, keepdim=True)
+    p = torch.softmax(torch.where(has, a, torch.zeros_like(a)), dim=-1) * has
+    o_s = p @ V
+    lin = torch.relu(Q) @ torch.relu(K).transpose(-1, -2) * (~sel_tok)
+    o_l = (lin @ V) / (lin.sum(-1, keepdim=True) + eps)
+    al = alpha[None, :, None, :]
+    return al * o_s + (1 - al) * o_l
+
+
+def test_linear_mix_matches_autograd_of_a_masked_restatement():
+    rng = np.random.default_rng(16)
+    Q, K, V, idx, dO, blk = _case(rng, nb=5, blk=3, d=4)
+    dQ, dK, dV = oracle.sparse_attention_backward(Q, K, V, idx, blk, "linear_mix", S, dO, alpha=ALPHA)
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (Q, K, V))
+    o = _linear_mix_torch(tq, tk, tv, idx, blk, S, torch.tensor(ALPHA))
+    np.testing.assert_allclose(o.detach().numpy(),
+                               oracle.sparse_attention(Q, K, V, idx, blk, "linear_mix", S, alpha=ALPHA),
+                               rtol=1e-12, atol=1e-12)
+    o.backward(torch.tensor(dO))
+    for got, t in ((dQ, tq), (dK, tk), (dV, tv)):
+        np.testing.assert_allclose(got, t.grad.numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_linear_mix_limits():
+    rng = np.random.default_rng(17)
+    Q, K, V, idx, dO, blk = _case(rng)
+    # α = 1: the drop backward
+    ones = np.ones_like(ALPHA)
+    lm = oracle.sparse_attention_backward(Q, K, V, idx, blk, "linear_mix", S, dO, alpha=ones)
+    dr = oracle.sparse_attention_backward(Q, K, V, idx, blk, "drop", S, dO)
+    for x, y in zip(lm, dr):
+        np.testing.assert_allclose(x, y, rtol=1e-12, atol=1e-13)
+    # every block selected: no linear branch; the drop backward of α⊙dO
+    nb = idx.shape[2]
+    full = np.tile(np.arange(nb), (1, 2, nb, 1))
+    lm = oracle.sparse_attention_backward(Q, K, V, full, blk, "linear_mix", S, dO, alpha=ALPHA)
+    dr = oracle.sparse_attention_backward(Q, K, V, full, blk, "drop", S, dO * ALPHA[None, :, None, :])
+    for x, y in zip(lm, dr):
+        np.testing.assert_allclose(x, y, rtol=1e-12, atol=1e-13)
+    # α = 0 and nothing selected: ReLU linear attention over all tokens (torch autograd)
+    empty = np.zeros((1, 2, nb, 0), dtype=np.int64)
+    lm = oracle.sparse_attention_backward(Q, K, V, empty, blk, "linear_mix", S, dO, alpha=np.zeros_like(ALPHA))
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (Q, K, V))
+    fq, fk = torch.relu(tq), torch.relu(tk)
+    o = (fq @ (fk.transpose(-1, -2) @ tv)) / (fq @ fk.sum(-2, keepdim=True).transpose(-1, -2) + 1e-6)
+    o.backward(torch.tensor(dO))
+    for got, t in zip(lm, (tq, tk, tv)):
+        np.testing.assert_allclose(got, t.grad.numpy(), rtol=1e-10, atol=1e-12)
