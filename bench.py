@@ -245,11 +245,13 @@ def run_reference(args, world, rank):
 # GPU arm
 # --------------------------------------------------------------------------
 
-def time_decode(steps: int = 50, warmup: int = 5, batch=None, name: str = "decode"):
+def time_decode(steps: int = 50, warmup: int = 5, batch=None, name: str = "decode", stats_dtype: str = "bf16"):
     """Decode workload timing (separate from the prefill step): GB/s of the
     bytes the method moves per decode step.  ``batch`` shrinks the number of
     sequences (for bounded profiler captures).  ``decode_rla`` is the same
-    caches with SPLA's residual linear tail."""
+    caches with SPLA's residual linear tail.  ``stats_dtype``: the block
+    statistics the decode reads, "bf16" (kmean, kvar, vsum / block as bf16
+    copies) or "f32"."""
     from block_sparse_approximate_b200 import binding as bd
     from block_sparse_approximate_b200.pipeline import DecodeStep
     w = wl.WORKLOADS[name]
@@ -257,8 +259,9 @@ def time_decode(steps: int = 50, warmup: int = 5, batch=None, name: str = "decod
     if batch:
         w = wl.Workload(**{**w.__dict__, "B": int(batch)})
     inp = wl.decode_inputs(w, "cuda")
-    st = bd.block_pool(None, inp["Kcache"], inp["Vcache"], w.block, variance=True, residual=rla)
-    step = DecodeStep(w, inp, st)
+    sb = stats_dtype == "bf16"
+    st = bd.block_pool(None, inp["Kcache"], inp["Vcache"], w.block, variance=True, residual=rla, centroids_bf16=sb)
+    step = DecodeStep(w, inp, bd.decode_stats_bf16(st) if sb else st)
     for _ in range(warmup):
         step()
     torch.cuda.synchronize()
@@ -271,15 +274,16 @@ def time_decode(steps: int = 50, warmup: int = 5, batch=None, name: str = "decod
     ms = s.elapsed_time(e) / steps
     B, Hkv, nb, d = w.B, w.Hkv, w.nb, w.d
     kv = 2.0 * B * Hkv * w.k * w.block * d * 2          # selected K and V, bf16
-    # kmean, kvar (route) and vsum (zero-order tail) fp32, read once each; the
-    # residual linear tail reads S_all (d×d per KV head) instead of vsum
-    stats = (2.0 if rla else 3.0) * B * Hkv * nb * d * 4 + (4.0 * B * Hkv * d * d if rla else 0.0)
+    # kmean, kvar (route) and vsum (zero-order tail), bf16 or fp32, read once
+    # each; the residual linear tail reads S_all (d×d fp32 per KV head) instead of vsum
+    esz = 2.0 if sb else 4.0
+    stats = (2.0 if rla else 3.0) * B * Hkv * nb * d * esz + (4.0 * B * Hkv * d * d if rla else 0.0)
     qo = 2.0 * B * w.H * d * 2
     byts = kv + stats + qo
     hbm, _, _, src = _peaks()
     del inp, st, step
     torch.cuda.empty_cache()
-    return {"workload": name, "ms": ms, "bytes_per_step": byts, "gbs": byts / ms / 1e6,
+    return {"workload": name, "stats": stats_dtype, "ms": ms, "bytes_per_step": byts, "gbs": byts / ms / 1e6,
             "hbm_peak_gbs": hbm, "frac": byts / ms / 1e6 / hbm, "peak_source": src}
 
 
@@ -521,8 +525,8 @@ def run_ours(args, world, rank, local):
     bd.load()
     if args.only in ("decode", "decode_rla"):
         if rank == 0:
-            print(json.dumps({args.only: time_decode(args.steps, args.warmup, args.decode_batch, args.only)}),
-                  flush=True)
+            print(json.dumps({args.only: time_decode(args.steps, args.warmup, args.decode_batch, args.only,
+                                                     args.decode_stats)}), flush=True)
         return 0
     if args.only == "fp8":
         if rank == 0:
@@ -632,11 +636,12 @@ def run_ours(args, world, rank, local):
                "h2d_bytes_per_step": sum(inp[n].numel() * inp[n].element_size() for n in ("Q", "K", "V")),
                "d2h_bytes_per_step": step.buf.out.numel() * step.buf.out.element_size()}
 
-    decode = decode_rla = fp8 = sla2 = pisa = sfa = backward = None
+    decode = decode_f32 = decode_rla = fp8 = sla2 = pisa = sfa = backward = None
     if rank == 0 and args.only == "all" and not args.no_decode:
         del step
         torch.cuda.empty_cache()
         decode = time_decode(batch=args.decode_batch)
+        decode_f32 = time_decode(batch=args.decode_batch, stats_dtype="f32")
         decode_rla = time_decode(batch=args.decode_batch, name="decode_rla")
         fp8 = time_fp8()
         sla2 = time_sla2()
@@ -674,6 +679,7 @@ def run_ours(args, world, rank, local):
         "gpu_launches": args.steps * PrefillStepLaunches(w),
         "clocks": ck,
         "decode": decode,
+        "decode_f32_stats": decode_f32,
         "decode_rla": decode_rla,
         "fp8": fp8,
         "sla2_mix": sla2,
@@ -703,6 +709,8 @@ def main(argv=None):
                     default="all",
                     help="prefill: the timed step only; decode / fp8 / sla2 / pisa (covariance routing + "
                          "first-order tail): only that workload's timing")
+    ap.add_argument("--decode-stats", choices=["bf16", "f32"], default="bf16",
+                    help="element type of the block statistics the decode reads (--only decode / decode_rla)")
     ap.add_argument("--decode-batch", type=int, default=None,
                     help="sequences in the decode workload (default: the full 16)")
     args = ap.parse_args(argv)

@@ -50,7 +50,7 @@ class DecodeShape(ctypes.Structure):
 
 
 _STAT_FIELDS = ("qmean", "kmean", "vsum", "kvar", "zrelu", "htot", "ztot", "kmean_bf16", "vmean_bf16",
-                "hbar", "hbarT_bf16", "covnorm", "sexp")
+                "hbar", "hbarT_bf16", "covnorm", "sexp", "kvar_bf16")
 
 
 class BlockStats(ctypes.Structure):
@@ -180,6 +180,8 @@ def block_pool(Q: Optional[torch.Tensor], K: torch.Tensor, V: torch.Tensor, bloc
     if centroids_bf16:
         st["kmean_bf16"] = torch.empty(Bsz, H, nb, d, device=dev, dtype=torch.bfloat16)
         st["vmean_bf16"] = torch.empty(Bsz, H, nb, d, device=dev, dtype=torch.bfloat16)
+        if variance:
+            st["kvar_bf16"] = torch.empty(Bsz, H, nb, d, device=dev, dtype=torch.bfloat16)
     if first_order or covariance:
         st["hbar"] = torch.empty(Bsz, H, d, d, **f)
         if centroids_bf16 and first_order:
@@ -234,6 +236,12 @@ def sparse_attn_fwd(Q, K, V, block_idx, block: int, tail: str, stats: dict, scal
                                   _ptr(alpha), ctypes.byref(cst), float(scale), _ptr(O),
                                   _stream(stream)))
     return O
+
+
+def decode_stats_bf16(stats: dict) -> dict:
+    """The view of block statistics that makes sa_decode_fwd read the bf16
+    copies (kmean_bf16, kvar_bf16, vmean_bf16; kmean left NULL), plus sexp."""
+    return {n: stats[n] for n in ("kmean_bf16", "kvar_bf16", "vmean_bf16", "sexp") if n in stats}
 
 
 def decode_workspace_size(B: int, Hq: int, Hkv: int, N: int, d: int, block: int, topk: int) -> int:

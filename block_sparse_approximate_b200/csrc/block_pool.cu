@@ -73,7 +73,7 @@ block_pool_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __r
         reinterpret_cast<__nv_bfloat16*>(st.kmean_bf16)[stat_off + tid] = __float2bfloat16_rn(m);
     }
     __syncthreads();
-    if (st.kvar) {
+    if (st.kvar || st.kvar_bf16) {
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         float s = 0.f;
@@ -85,7 +85,11 @@ block_pool_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __r
         acc[i] = s;
       }
       reduce_rows(acc);
-      if (tid < D) st.kvar[stat_off + tid] = mean_sh[tid] * inv;
+      if (tid < D) {
+        const float v = mean_sh[tid] * inv;
+        if (st.kvar) st.kvar[stat_off + tid] = v;
+        if (st.kvar_bf16) reinterpret_cast<__nv_bfloat16*>(st.kvar_bf16)[stat_off + tid] = __float2bfloat16_rn(v);
+      }
       __syncthreads();
     }
     if (st.zrelu) {
@@ -430,7 +434,7 @@ extern "C" sa_status sa_block_pool(const void* Q, const void* K, const void* V, 
     return fail(SA_ERR_INVALID_ARG, "sa_block_pool: hbarT_bf16 and covnorm need hbar");
   const void* ptrs[] = {Q, K, V, stats->qmean, stats->kmean, stats->vsum, stats->kvar,
                         stats->zrelu, stats->htot, stats->ztot, stats->kmean_bf16, stats->vmean_bf16,
-                        stats->hbar, stats->hbarT_bf16, stats->covnorm, stats->sexp};
+                        stats->hbar, stats->hbarT_bf16, stats->covnorm, stats->sexp, stats->kvar_bf16};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return fail(SA_ERR_ALIGNMENT, "sa_block_pool: pointers must be 16-byte aligned");
   cudaStream_t s = as_stream(stream);

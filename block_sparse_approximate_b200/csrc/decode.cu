@@ -203,31 +203,57 @@ __device__ __forceinline__ void load_lane(float (&r)[CPL], const float* row, int
     r[1] = x.y;
   }
 }
+template <int CPL>
+__device__ __forceinline__ void load_lane(float (&r)[CPL], const __nv_bfloat16* row, int lane, bool ok) {
+  if constexpr (CPL == 4) {
+    const uint2 x = ok ? *reinterpret_cast<const uint2*>(row + lane * 4) : make_uint2(0u, 0u);
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&x.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&x.y));
+    r[0] = a.x;
+    r[1] = a.y;
+    r[2] = b.x;
+    r[3] = b.y;
+  } else {
+    const uint32_t x = ok ? *reinterpret_cast<const uint32_t*>(row + lane * 2) : 0u;
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&x));
+    r[0] = a.x;
+    r[1] = a.y;
+  }
+}
+
+// Ring depth of the statistics pass: the same bytes in flight per CTA for
+// float32 and bf16 statistics (bf16 stages are half as large)
+template <typename TS>
+constexpr int ring_a() { return sizeof(TS) == 4 ? kRingA : 2 * kRingA - 1; }
 
 constexpr int kWarpBlocksA = kStageBlocksA / (kThrA / 32);   // blocks of a stage per warp
 
 // ZT: the zero-order tail is wanted (its value sums are copied and its
 // online state kept); without it the pass only scores the blocks.
-template <int D, int G, bool ZT>
+// TS: element type of the statistics, float (kmean, kvar, vsum) or bf16
+// (kmean, kvar and the value means vsum / blk); vmul turns a row of the
+// third array into the block's value mean (1 / blk for sums, 1 for means).
+template <int D, int G, bool ZT, typename TS>
 __global__ void __launch_bounds__(kThrA, 2)
-decode_stats_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int Hq, int Hkv, int nb, int blk,
-                    float scale, int nsegA, int npairs, float* __restrict__ scores, float* __restrict__ parta) {
+decode_stats_kernel(const __nv_bfloat16* __restrict__ q, const TS* __restrict__ kmean, const TS* __restrict__ kvar,
+                    const TS* __restrict__ vrow, float vmul, int Hq, int Hkv, int nb, int blk, float scale,
+                    int nsegA, int npairs, float* __restrict__ scores, float* __restrict__ parta) {
   constexpr int CPL = D / 32;                        // channels per lane
   constexpr int NBT = 16 / G;                        // blocks per batch: NBT x G x 2 = 32 sums
   constexpr int kBatches = (kWarpBlocksA + NBT - 1) / NBT;
-  constexpr uint32_t kRowB = D * 4;                  // bytes per stats row
+  constexpr int RING = ring_a<TS>();
+  constexpr uint32_t kRowB = D * sizeof(TS);         // bytes per stats row
   constexpr uint32_t kArrB = kStageBlocksA * kRowB;  // one array of one stage
   constexpr uint32_t kStageB = 3 * kArrB;
   constexpr int kWarps = kThrA / 32;
   extern __shared__ __align__(16) uint8_t dsm[];
   float* mg = reinterpret_cast<float*>(dsm);                 // [warps][G][D + 2] segment merge
-  uint64_t* full = reinterpret_cast<uint64_t*>(dsm + sizeof(float) * kWarps * G * (D + 2));   // [kRingA]
-  uint8_t* ring = reinterpret_cast<uint8_t*>(full + 2 * kRingA);
+  uint64_t* full = reinterpret_cast<uint64_t*>(dsm + sizeof(float) * kWarps * G * (D + 2));   // [RING]
+  uint8_t* ring = reinterpret_cast<uint8_t*>(full + 2 * RING);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nstage_pair = (nb + kStageBlocksA - 1) / kStageBlocksA;
   const int total_segs = npairs * nsegA;
   const float bias2 = log2f((float)blk);
-  const float inv_blk = 1.0f / blk;
   const int hl = (lane >> 1) % G, jbl = (lane >> 1) / G;   // the (block, head) of the sum lane ends with
 
   // the CTA's stage sequence: its segments in order, each segment's stages
@@ -245,14 +271,14 @@ decode_stats_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int 
     // barrier that precedes this call; order them before the async writes
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     dbar_expect_tx(fb, (ZT ? 3 : 2) * bytes);
-    bulk_copy(dst, st.kmean + goff, bytes, fb);
-    bulk_copy(dst + kArrB, st.kvar + goff, bytes, fb);
-    if (ZT) bulk_copy(dst + 2 * kArrB, st.vsum + goff, bytes, fb);
+    bulk_copy(dst, kmean + goff, bytes, fb);
+    bulk_copy(dst + kArrB, kvar + goff, bytes, fb);
+    if (ZT) bulk_copy(dst + 2 * kArrB, vrow + goff, bytes, fb);
   };
 
   if (seg_of(0) >= total_segs) return;
   if (tid == 0) {
-    for (int r = 0; r < kRingA; ++r) dbar_init(smem_addr(full + r), 1);
+    for (int r = 0; r < RING; ++r) dbar_init(smem_addr(full + r), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
@@ -266,13 +292,13 @@ decode_stats_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int 
       ++pf_seg_k;
     }
   };
-  for (int r = 0; r < kRingA - 1; ++r) {
+  for (int r = 0; r < RING - 1; ++r) {
     if (pf_valid()) {
       if (tid == 0) issue(seg_of(pf_seg_k), pf_sub, pf_slot);
       ++issued;
       pf_advance();
     }
-    pf_slot = (pf_slot + 1) % kRingA;
+    pf_slot = (pf_slot + 1) % RING;
   }
 
   float qv[G][CPL], wv[G][CPL];   // s log2e q and ½ s² q² of this lane's channels
@@ -310,15 +336,15 @@ decode_stats_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int 
       ++issued;
       pf_advance();
     }
-    pf_slot = (pf_slot + 1) % kRingA;
-    const bool landed = dbar_wait(smem_addr(full + slot), (consumed / kRingA) & 1);
+    pf_slot = (pf_slot + 1) % RING;
+    const bool landed = dbar_wait(smem_addr(full + slot), (consumed / RING) & 1);
     ++consumed;
     if (!__syncthreads_and(landed)) break;
 
     const uint8_t* stg = ring + slot * kStageB;
-    const float* km = reinterpret_cast<const float*>(stg);
-    const float* kv = reinterpret_cast<const float*>(stg + kArrB);
-    const float* vs = reinterpret_cast<const float*>(stg + 2 * kArrB);
+    const TS* km = reinterpret_cast<const TS*>(stg);
+    const TS* kv = reinterpret_cast<const TS*>(stg + kArrB);
+    const TS* vs = reinterpret_cast<const TS*>(stg + 2 * kArrB);
     const int j0 = (sseg * kSegA + cur_sub) * kStageBlocksA;
     const int rows = min(kStageBlocksA, nb - j0);
 
@@ -407,13 +433,13 @@ decode_stats_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int 
         load_lane<CPL>(vv, vs + jr * D, lane, ok);
 #pragma unroll
         for (int h = 0; h < G; ++h) {
-          const float pw = __shfl_sync(0xffffffffu, p, (jb * G + h) * 2) * inv_blk;
+          const float pw = __shfl_sync(0xffffffffu, p, (jb * G + h) * 2) * vmul;
 #pragma unroll
           for (int c = 0; c < CPL; ++c) acc[h][c] = fmaf(pw, vv[c], acc[h][c]);
         }
       }
     }
-    slot = (slot + 1) % kRingA;
+    slot = (slot + 1) % RING;
     // end of segment: merge the warps' states per head and write them
     const bool seg_end = ++cur_sub >= stages_in(seg);
     if (ZT && seg_end) {
@@ -460,7 +486,7 @@ decode_stats_kernel(const __nv_bfloat16* __restrict__ q, sa_block_stats st, int 
   }
   // after a give-up, let the copies still in flight land before exiting
   if (tid == 0)
-    for (int q = consumed; q < issued; ++q) dbar_wait(smem_addr(full + q % kRingA), (q / kRingA) & 1);
+    for (int q = consumed; q < issued; ++q) dbar_wait(smem_addr(full + q % RING), (q / RING) & 1);
 }
 
 // ---- B. top-k ------------------------------------------------------------
@@ -931,12 +957,18 @@ decode_exact_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
 constexpr int kParts = 4;
 constexpr float kRmsEps = 1e-6f;     // RMSNorm of SPLA's residual linear output
 
-template <int D>
+__device__ __forceinline__ float ld_stat(const float* p) { return __ldg(p); }
+__device__ __forceinline__ float ld_stat(const __nv_bfloat16* p) { return __bfloat162float(__ldg(p)); }
+
+// TS, kmean, vrow, vmul: the statistics as the statistics pass read them
+// (vmul turns a row of vrow into the block's value mean)
+template <int D, typename TS>
 __global__ void __launch_bounds__(kParts * D)
 decode_combine_kernel(const float* __restrict__ parta, int nsegA, const float* __restrict__ partc, int nsegC,
                       int use_tail, const float* __restrict__ partr, const __nv_bfloat16* __restrict__ q,
-                      sa_block_stats st, const int32_t* __restrict__ idx, int topk, int nb, int blk, float scale,
-                      int Hq, int Hkv, __nv_bfloat16* __restrict__ O) {
+                      const TS* __restrict__ kmean, const TS* __restrict__ vrow, float vmul,
+                      const float* __restrict__ sexp, const int32_t* __restrict__ idx, int topk, int nb, int blk,
+                      float scale, int Hq, int Hkv, __nv_bfloat16* __restrict__ O) {
   pdl_wait();
   constexpr int kT = kParts * D, kW = kT / 32;
   extern __shared__ __align__(16) float csm[];
@@ -977,7 +1009,7 @@ decode_combine_kernel(const float* __restrict__ parta, int nsegA, const float* _
 #pragma unroll
   for (int e = 0; e < kPreV; ++e) {
     const int si = pt + kParts * e;
-    vv[e] = si < nsel ? __ldg(st.vsum + ((size_t)pair * nb + jsel[si]) * D + c) : 0.f;
+    vv[e] = si < nsel ? ld_stat(vrow + ((size_t)pair * nb + jsel[si]) * D + c) : 0.f;
   }
   float M = -INFINITY;
   for (int x = 0; x < ns; ++x) M = fmaxf(M, hm[x]);
@@ -993,9 +1025,9 @@ decode_combine_kernel(const float* __restrict__ parta, int nsegA, const float* _
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int si = min(s0 + u, nsel - 1);
-        const float* kr = st.kmean + ((size_t)pair * nb + jsel[si]) * D;
+        const TS* kr = kmean + ((size_t)pair * nb + jsel[si]) * D;
 #pragma unroll
-        for (int e = 0; e < D / 32; ++e) kk[u][e] = __ldg(kr + lane + 32 * e);
+        for (int e = 0; e < D / 32; ++e) kk[u][e] = ld_stat(kr + lane + 32 * e);
       }
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
@@ -1024,20 +1056,19 @@ decode_combine_kernel(const float* __restrict__ parta, int nsegA, const float* _
       A = fmaf(part(x)[2 + c], hf[x], A);
     }
     // subtract the zero-order term of each selected block (weight <= 1)
-    const float inv_blk = 1.0f / blk;
 #pragma unroll
     for (int e = 0; e < kPreV; ++e) {
       const int si = pt + kParts * e;
       if (si < nsel) {
         const float w = fast_exp2(xsel[si] - M);
         L -= w;
-        A = fmaf(-w * inv_blk, vv[e], A);
+        A = fmaf(-w * vmul, vv[e], A);
       }
     }
     for (int si = pt + kParts * kPreV; si < nsel; si += kParts) {
       const float w = fast_exp2(xsel[si] - M);
       L -= w;
-      A = fmaf(-w * inv_blk, __ldg(st.vsum + ((size_t)pair * nb + jsel[si]) * D + c), A);
+      A = fmaf(-w * vmul, ld_stat(vrow + ((size_t)pair * nb + jsel[si]) * D + c), A);
     }
   }
   red[(pt * 2 + 0) * D + c] = L;
@@ -1046,7 +1077,7 @@ decode_combine_kernel(const float* __restrict__ parta, int nsegA, const float* _
     // SPLA's residual: this part's rows r of φ(q)ᵀ S_all (column c) minus its
     // exact segments' Σ (φ(q)·φ(k_n)) v_n
     float rpart = 0.f;
-    const float* sa = st.sexp + (size_t)pair * D * D;
+    const float* sa = sexp + (size_t)pair * D * D;
     const __nv_bfloat16* qh = q + ((size_t)b * Hq + h) * D;
     // φ(q) rounded to bf16 as in the exact pass's operand, so that the two
     // terms of the difference use the same feature values
@@ -1117,10 +1148,18 @@ int sm_count() {
   return n;
 }
 
-template <int D>
+// The statistics the decode reads: float32 kmean, kvar, vsum, or (when
+// kmean is NULL) their bf16 copies kmean_bf16, kvar_bf16, vmean_bf16.
+template <typename TS>
+struct DecodeStats {
+  const TS *kmean, *kvar, *vrow;
+  float vmul;   // vrow row -> block value mean
+};
+
+template <int D, typename TS>
 sa_status launch_decode(const void* q, const void* Kc, const void* Vc, const sa_decode_shape& s,
-                        const sa_block_stats& st, int topk, float scale, sa_tail_mode tail,
-                        int32_t* idx_out, float* scores_out, void* O, char* ws,
+                        const sa_block_stats& st, const DecodeStats<TS>& ds, int topk, float scale,
+                        sa_tail_mode tail, int32_t* idx_out, float* scores_out, void* O, char* ws,
                         cudaStream_t stream) {
   const DecodeLayout L = decode_layout(s, topk);
   const int nb = s.N / s.block;
@@ -1140,8 +1179,9 @@ sa_status launch_decode(const void* q, const void* Kc, const void* Vc, const sa_
   // A
   {
     const int g = s.Hq / s.Hkv;
-    const size_t smemA = sizeof(float) * (kThrA / 32) * g * (D + 2) + 16 * kRingA +
-                         (size_t)kRingA * 3 * kStageBlocksA * D * 4;
+    constexpr int RING = ring_a<TS>();
+    const size_t smemA = sizeof(float) * (kThrA / 32) * g * (D + 2) + 16 * RING +
+                         (size_t)RING * 3 * kStageBlocksA * D * sizeof(TS);
     const long segsA = (long)npairs * L.nsegA;
     const int gridA = (int)(segsA < 2 * sms ? segsA : 2 * sms);
     sa_status r0 = SA_OK;
@@ -1150,14 +1190,15 @@ sa_status launch_decode(const void* q, const void* Kc, const void* Vc, const sa_
         r0 = launch_status("cudaFuncSetAttribute(decode_stats_kernel)");
         return;
       }
-      kern<<<gridA, kThrA, smemA, stream>>>(qb, st, s.Hq, s.Hkv, nb, s.block, scale, L.nsegA, npairs, scores, parta);
+      kern<<<gridA, kThrA, smemA, stream>>>(qb, ds.kmean, ds.kvar, ds.vrow, ds.vmul, s.Hq, s.Hkv, nb, s.block,
+                                            scale, L.nsegA, npairs, scores, parta);
       r0 = launch_status("decode_stats_kernel");
     };
     const bool zt = tail == SA_TAIL_ZERO_ORDER;
-    if (g == 1) run(zt ? decode_stats_kernel<D, 1, true> : decode_stats_kernel<D, 1, false>);
-    else if (g == 2) run(zt ? decode_stats_kernel<D, 2, true> : decode_stats_kernel<D, 2, false>);
-    else if (g == 4) run(zt ? decode_stats_kernel<D, 4, true> : decode_stats_kernel<D, 4, false>);
-    else run(zt ? decode_stats_kernel<D, 8, true> : decode_stats_kernel<D, 8, false>);
+    if (g == 1) run(zt ? decode_stats_kernel<D, 1, true, TS> : decode_stats_kernel<D, 1, false, TS>);
+    else if (g == 2) run(zt ? decode_stats_kernel<D, 2, true, TS> : decode_stats_kernel<D, 2, false, TS>);
+    else if (g == 4) run(zt ? decode_stats_kernel<D, 4, true, TS> : decode_stats_kernel<D, 4, false, TS>);
+    else run(zt ? decode_stats_kernel<D, 8, true, TS> : decode_stats_kernel<D, 8, false, TS>);
     if (r0 != SA_OK) return r0;
   }
   sa_status r = SA_OK;
@@ -1200,13 +1241,13 @@ sa_status launch_decode(const void* q, const void* Kc, const void* Vc, const sa_
     const int nsel = (use_tail && nsc > 0) ? topk : 0;
     const size_t smemD = sizeof(float) * (kParts * 2 * D + 3 * (size_t)ns + 2 * (size_t)nsel +
                                           (rla ? kParts * D + D / 32 : 0));
-    if (cudaFuncSetAttribute(decode_combine_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smemD) !=
-        cudaSuccess)
+    if (cudaFuncSetAttribute(decode_combine_kernel<D, TS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smemD) != cudaSuccess)
       return launch_status("cudaFuncSetAttribute(decode_combine_kernel)");
     {
-      const cudaError_t le = launch_pdl(decode_combine_kernel<D>, dim3(s.Hq, s.B), dim3(kParts * D), smemD, stream,
-        parta, L.nsegA, partc, nsc, use_tail, topk < nb ? partr : nullptr, qb, st, idx, topk, nb, s.block, scale,
-        s.Hq, s.Hkv,
+      const cudaError_t le = launch_pdl(decode_combine_kernel<D, TS>, dim3(s.Hq, s.B), dim3(kParts * D), smemD,
+        stream, parta, L.nsegA, partc, nsc, use_tail, topk < nb ? partr : nullptr, qb, ds.kmean, ds.vrow, ds.vmul,
+        static_cast<const float*>(st.sexp), idx, topk, nb, s.block, scale, s.Hq, s.Hkv,
         static_cast<__nv_bfloat16*>(O));
       if (le != cudaSuccess) return fail(SA_ERR_CUDA, std::string("decode_combine_kernel: ") + cudaGetErrorString(le));
     }
@@ -1260,12 +1301,19 @@ extern "C" sa_status sa_decode_fwd(const void* q, const void* Kcache, const void
   if (tail != SA_TAIL_ZERO_ORDER && tail != SA_TAIL_DROP && tail != SA_TAIL_RESIDUAL_LINEAR)
     return fail(SA_ERR_UNSUPPORTED,
                 "sa_decode_fwd: tail must be SA_TAIL_DROP, SA_TAIL_ZERO_ORDER or SA_TAIL_RESIDUAL_LINEAR");
-  if (!q || !Kcache || !Vcache || !O || !stats || !stats->kmean || !stats->kvar || !stats->vsum)
-    return fail(SA_ERR_INVALID_ARG, "sa_decode_fwd: q, caches, O and stats (kmean, kvar, vsum) are required");
+  if (!q || !Kcache || !Vcache || !O || !stats)
+    return fail(SA_ERR_INVALID_ARG, "sa_decode_fwd: q, caches, O and stats are required");
+  const bool stats_bf16 = stats->kmean == nullptr;
+  if (!stats_bf16 && (!stats->kvar || !stats->vsum))
+    return fail(SA_ERR_INVALID_ARG, "sa_decode_fwd: float32 statistics need kmean, kvar and vsum");
+  if (stats_bf16 && (!stats->kmean_bf16 || !stats->kvar_bf16 || (tail == SA_TAIL_ZERO_ORDER && !stats->vmean_bf16)))
+    return fail(SA_ERR_INVALID_ARG,
+                "sa_decode_fwd: without stats->kmean the bf16 statistics kmean_bf16, kvar_bf16 (and vmean_bf16 "
+                "for SA_TAIL_ZERO_ORDER) are required");
   if (tail == SA_TAIL_RESIDUAL_LINEAR && !stats->sexp)
     return fail(SA_ERR_INVALID_ARG, "sa_decode_fwd: SA_TAIL_RESIDUAL_LINEAR needs stats->sexp");
   const void* ptrs[] = {q, Kcache, Vcache, O, stats->kmean, stats->kvar, stats->vsum, stats->sexp, block_idx_out,
-                        scores_out};
+                        scores_out, stats->kmean_bf16, stats->kvar_bf16, stats->vmean_bf16};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return fail(SA_ERR_ALIGNMENT, "sa_decode_fwd: pointers must be 16-byte aligned");
   const size_t need = decode_layout(shape, topk).total;
@@ -1276,11 +1324,24 @@ extern "C" sa_status sa_decode_fwd(const void* q, const void* Kcache, const void
   if (shape.B == 0 || shape.N == 0) return SA_OK;
   cudaStream_t s = as_stream(stream);
   char* ws = static_cast<char*>(workspace);
+  if (stats_bf16) {
+    typedef __nv_bfloat16 bf;
+    // vmean_bf16 may be NULL without the zero-order tail; the kernels then never read it
+    const DecodeStats<bf> ds{reinterpret_cast<const bf*>(stats->kmean_bf16),
+                             reinterpret_cast<const bf*>(stats->kvar_bf16),
+                             reinterpret_cast<const bf*>(stats->vmean_bf16), 1.0f};
+    if (shape.d == 128)
+      return launch_decode<128, bf>(q, Kcache, Vcache, shape, *stats, ds, topk, scale, tail, block_idx_out,
+                                    scores_out, O, ws, s);
+    return launch_decode<64, bf>(q, Kcache, Vcache, shape, *stats, ds, topk, scale, tail, block_idx_out,
+                                 scores_out, O, ws, s);
+  }
+  const DecodeStats<float> ds{stats->kmean, stats->kvar, stats->vsum, 1.0f / shape.block};
   if (shape.d == 128)
-    return launch_decode<128>(q, Kcache, Vcache, shape, *stats, topk, scale, tail, block_idx_out,
-                              scores_out, O, ws, s);
-  return launch_decode<64>(q, Kcache, Vcache, shape, *stats, topk, scale, tail, block_idx_out,
-                           scores_out, O, ws, s);
+    return launch_decode<128, float>(q, Kcache, Vcache, shape, *stats, ds, topk, scale, tail, block_idx_out,
+                                     scores_out, O, ws, s);
+  return launch_decode<64, float>(q, Kcache, Vcache, shape, *stats, ds, topk, scale, tail, block_idx_out,
+                                  scores_out, O, ws, s);
 }
 
 // ---- decode with library-owned scratch ---------------------------------------

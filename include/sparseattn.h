@@ -123,11 +123,15 @@ typedef struct {
                        (bf16-rounded on the tensor-core path, as the decode
                        kernel rounds φ(k) of the selected blocks)
                        [SPLA §2.2, the residual linear state]              */
+  uint16_t* kvar_bf16;   /* [B,H,nb,d] bf16 copy of kvar (the decode's bf16
+                       statistics; with kmean_bf16 and vmean_bf16 they are
+                       half the bytes of the float32 kmean, kvar, vsum)    */
 } sa_block_stats;
 
 /* Block statistics of Q (optional), K and V.
  * Q: [B,H,N,d] or NULL (then stats->qmean is ignored); K, V: [B,H,N,d];
- * dtype: element type of Q, K, V.  Every non-NULL field of *stats is written;
+ * dtype: element type of Q, K, V.  Every non-NULL field of *stats is written
+ * (the bf16 copies are the round-to-nearest-even bf16 of the float32 values);
  * kmean and vsum are required.  htot, ztot and hbar are sums over all tokens
  * of a head and are overwritten (no accumulation across calls); hbarT_bf16
  * and covnorm need hbar.
@@ -279,7 +283,13 @@ size_t sa_decode_workspace_size(sa_decode_shape shape, int32_t topk);
  * Split over the KV axis; partial (max, sum, acc) states are merged.
  * q: [B,Hq,d]; Kcache, Vcache: [B,Hkv,N,d], all of `dtype` (bf16 only);
  * the group Hq / Hkv is 1, 2, 4 or 8.
- * stats: kmean, kvar, vsum of the caches (sa_block_pool with Q = NULL).
+ * stats: the block statistics of the caches (sa_block_pool with Q = NULL),
+ * read in one of two precisions:
+ *   - float32: kmean, kvar and vsum (all three required);
+ *   - bf16, when stats->kmean is NULL: kmean_bf16, kvar_bf16 and, for
+ *     SA_TAIL_ZERO_ORDER, vmean_bf16 (= vsum / block).  Half the statistics
+ *     bytes; the scores and the tail are computed in float32 from the bf16
+ *     values.
  * block_idx_out: [B,Hkv,topk] int32 or NULL; scores_out: [B,Hkv,nb] float32
  * or NULL.  O: [B,Hq,d] of `dtype`.  workspace: device scratch of at least
  * sa_decode_workspace_size() bytes, 256-byte aligned; its contents on entry

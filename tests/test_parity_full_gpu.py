@@ -54,13 +54,14 @@ def test_prefill_full_size_sampled(lib, name):
     assert_tol(got, ref, BF16_TOL, name)
 
 
-@pytest.mark.parametrize("name", ["decode", "decode_rla"])
-def test_decode_full_size_sampled(lib, name):
+@pytest.mark.parametrize("name,stats_dtype", [("decode", "bf16"), ("decode", "f32"), ("decode_rla", "bf16")])
+def test_decode_full_size_sampled(lib, name, stats_dtype):
     w = wl.WORKLOADS[name]
     inp = wl.decode_inputs(w, DEV)
+    sb = stats_dtype == "bf16"
     st = bd.block_pool(None, inp["Kcache"], inp["Vcache"], w.block, variance=True,
-                       residual=(w.tail == "residual_linear"))
-    step = DecodeStep(w, inp, st)
+                       residual=(w.tail == "residual_linear"), centroids_bf16=sb)
+    step = DecodeStep(w, inp, bd.decode_stats_bf16(st) if sb else st)
     o = step()
     torch.cuda.synchronize()
     assert_no_device_error()
@@ -71,10 +72,18 @@ def test_decode_full_size_sampled(lib, name):
     for b, kh in pairs:
         Kh = inp["Kcache"][b:b + 1, kh:kh + 1].cpu().float().numpy()
         Vh = inp["Vcache"][b:b + 1, kh:kh + 1].cpu().float().numpy()
-        ref_o, _, ref_sc = oracle.decode_attention(q[b:b + 1, kh * g:(kh + 1) * g], Kh, Vh, w.block,
-                                                   w.k, w.scale, tail=w.tail,
+        qg = q[b:b + 1, kh * g:(kh + 1) * g]
+        ref_o, _, ref_sc = oracle.decode_attention(qg, Kh, Vh, w.block, w.k, w.scale, tail=w.tail,
                                                    block_idx=step.idx[b:b + 1, kh:kh + 1].cpu().numpy())
-        selection_agreement(np64(step.scores[b, kh]), ref_sc[0, 0], w.k)  # asserts on clear gaps
+        if sb:
+            # the scores of the bf16-rounded statistics; a float32 and a
+            # float64 mean can round to neighbouring bf16 values (~1e-4 in a score)
+            ost = oracle.block_pool(None, Kh, Vh, w.block, variance=True)
+            r16 = lambda x: torch.as_tensor(x).to(torch.bfloat16).to(torch.float64).numpy()
+            ref_sc = oracle.decode_route_scores(qg, r16(ost["kmean"]), r16(ost["kvar"]), w.scale)
+            selection_agreement(np64(step.scores[b, kh]), ref_sc[0, 0], w.k, gap_rel=1e-3)
+        else:
+            selection_agreement(np64(step.scores[b, kh]), ref_sc[0, 0], w.k)  # asserts on clear gaps
         assert_tol(np64(o[b, kh * g:(kh + 1) * g]), ref_o[0], BF16_TOL, f"decode b={b} g={kh}")
 
 

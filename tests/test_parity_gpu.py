@@ -299,6 +299,61 @@ def test_decode(lib, tail, B, Hq, Hkv, N, d, block, k):
     del w
 
 
+def _bf16_round(x: np.ndarray) -> np.ndarray:
+    return torch.as_tensor(x).to(torch.bfloat16).to(torch.float64).numpy()
+
+
+@pytest.mark.parametrize("tail", ["zero_order", "drop", "residual_linear"])
+@pytest.mark.parametrize("B,Hq,Hkv,N,d,block,k", [
+    (2, 8, 2, 8192, 128, 64, 16),
+    (1, 4, 4, 4096, 128, 128, 5),
+    (2, 8, 1, 2048, 64, 64, 3),
+    (3, 6, 3, 64 * 77, 128, 64, 7),         # ragged split ranges
+])
+def test_decode_bf16_stats(lib, tail, B, Hq, Hkv, N, d, block, k):
+    # the decode reading the bf16 copies of kmean, kvar and vsum / block: its
+    # scores against the oracle's taylor2 score of the bf16-rounded oracle
+    # statistics, the selection bit-exact against the oracle's top-k of the
+    # GPU's scores, the output against the float64 oracle (exact statistics)
+    g = torch.Generator(device=DEV)
+    g.manual_seed(300 + N + k)
+    q = torch.randn(B, Hq, d, generator=g, device=DEV).to(torch.bfloat16)
+    Kc = (torch.randn(B, Hkv, N // block, block, d, generator=g, device=DEV)
+          + 0.7 * torch.randn(B, Hkv, N // block, 1, d, generator=g, device=DEV)).reshape(B, Hkv, N, d).to(torch.bfloat16)
+    Vc = torch.randn(B, Hkv, N, d, generator=g, device=DEV).to(torch.bfloat16)
+    st = bd.block_pool(None, Kc, Vc, block, variance=True, centroids_bf16=True,
+                       residual=(tail == "residual_linear"))
+    s = 1 / math.sqrt(d)
+    o, idx, sc = bd.decode_fwd(q, Kc, Vc, bd.decode_stats_bf16(st), block, k, s, tail=tail)
+    torch.cuda.synchronize()
+    assert_no_device_error()
+    check_topk_exact(idx, sc, k)
+    ost = oracle.block_pool(None, np64(Kc), np64(Vc), block, variance=True)
+    ref_sc = oracle.decode_route_scores(np64(q), _bf16_round(ost["kmean"]), _bf16_round(ost["kvar"]), s)
+    # a float32 and a float64 mean can round to neighbouring bf16 values: one
+    # ulp (2^-8 relative) of one channel moves a score by ~1e-4
+    assert_stats_close(sc, ref_sc, "decode scores (bf16 statistics)", rtol=1e-4)
+    selection_agreement(np64(sc), ref_sc, k, gap_rel=1e-3)
+    ref_o, _, _ = oracle.decode_attention(np64(q), np64(Kc), np64(Vc), block, k, s, tail=tail,
+                                          block_idx=idx.cpu().numpy())
+    assert_tol(np64(o), ref_o, BF16_TOL, f"decode {tail} (bf16 statistics)")
+
+
+def test_decode_bf16_stats_requires_the_bf16_copies(lib):
+    q = torch.zeros(1, 4, 128, device=DEV, dtype=torch.bfloat16)
+    Kc = torch.zeros(1, 1, 1024, 128, device=DEV, dtype=torch.bfloat16)
+    st = bd.block_pool(None, Kc, Kc, 64, variance=True, centroids_bf16=True)
+    view = bd.decode_stats_bf16(st)
+    del view["vmean_bf16"]
+    with pytest.raises(bd.SparseAttnError) as e:
+        bd.decode_fwd(q, Kc, Kc, view, 64, 4, 0.1, tail="zero_order")
+    assert e.value.status == bd.SA_ERR_INVALID_ARG
+    # without the zero-order tail the value means are not needed
+    bd.decode_fwd(q, Kc, Kc, view, 64, 4, 0.1, tail="drop")
+    torch.cuda.synchronize()
+    assert_no_device_error()
+
+
 def test_block_pool_sexp(lib):
     # SPLA's all-token state Σ_n exp(k_n) v_nᵀ: tensor-core path (bf16, d = 128,
     # φ(k) rounded to bf16) and CUDA-core path (fp32)
