@@ -395,8 +395,16 @@ def time_sfa(steps: int = 10, warmup: int = 3):
     _, bf16, _, src = _peaks()
     fl = dense_flops(w)
     ach = fl / (attn_ms * 1e-3) / 1e12
+    # the method's own work ("Scaling Attention via Feature Sparsity" §2): the
+    # scores cost a (kf/d)² fraction of the dense scores (2·N²·kf²/d per
+    # head, the expected overlap of two random supports being kf²/d), the
+    # value product stays dense (2·N²·d per head)
+    method = 2.0 * w.B * w.H * float(w.N) ** 2 * (kf * kf / w.d + w.d)
     out = {"workload": w.name, "kf": kf, "ms_per_step": ms_step, "attn_ms": attn_ms, "encode_ms": ms_step - attn_ms,
            "executed_tflops": ach, "peak_tflops": bf16, "frac": ach / bf16, "peak_source": f"{src} bf16 burst",
+           "method_flops": method, "method_tflops": method / (attn_ms * 1e-3) / 1e12,
+           "note": "executed = dense-counted (zero-filled operands at full width); method = (kf/d)^2-counted scores "
+                   "+ dense P.V",
            "step": "sfa_encode (Q, K) + sfa_attn_fwd over every KV tile"}
     del inp, Q, K, V, Qs, Ks, O
     torch.cuda.empty_cache()
@@ -410,19 +418,24 @@ def backward_flops(w, with_lse: bool = False) -> float:
     2·d (dK); without the forward's log-sum-exp the dQ kernel first recomputes
     the scores once more (2·d): 14·d or 16·d per (row, key)."""
     keys = w.k * w.block + ((w.nb - w.k) if w.tail in ("zero_order", "first_order") else 0)
-    return (14.0 if with_lse else 16.0) * w.d * keys * w.B * w.H * float(w.N)
+    fl = (14.0 if with_lse else 16.0) * w.d * keys * w.B * w.H * float(w.N)
+    if w.tail == "first_order":
+        # PISA's first-order terms: H̄ dO_t (twice: for δ's shift and for dQ),
+        # G = s Σ λ q dOᵀ, and the dK, dV products with G: 5 × 2·d² per row
+        fl += 10.0 * w.d * w.d * w.B * w.H * float(w.N)
+    return fl
 
 
-def time_backward(steps: int = 3, warmup: int = 3):
-    """Backward of the video_dit prefill (zero-order tail): forward step once
-    (with the rows' log-sum-exp, sa_sparse_attn_fwd_lse), then
-    sa_sparse_attn_bwd_lse timed on the saved inputs, output, log-sum-exp and
-    a random dO; sa_sparse_attn_bwd (which recomputes the log-sum-exp) is
-    timed beside it."""
+def time_backward(steps: int = 3, warmup: int = 3, name: str = "video_dit"):
+    """Backward of the video_dit prefill (zero-order tail; "video_dit_pisa":
+    PISA's first-order tail): forward step once (with the rows' log-sum-exp,
+    sa_sparse_attn_fwd_lse), then sa_sparse_attn_bwd_lse timed on the saved
+    inputs, output, log-sum-exp and a random dO; sa_sparse_attn_bwd (which
+    recomputes the log-sum-exp) is timed beside it."""
     import ctypes
     from block_sparse_approximate_b200 import binding as bd
     from block_sparse_approximate_b200.pipeline import PrefillStep
-    w = wl.WORKLOADS["video_dit"]
+    w = wl.WORKLOADS[name]
     inp = wl.prefill_inputs(w, "cuda")
     step = PrefillStep(w, inp)
     O = step()
@@ -474,7 +487,7 @@ def time_backward(steps: int = 3, warmup: int = 3):
            "peak_source": f"{src} bf16 burst", "entry": "sa_sparse_attn_bwd_lse (the forward's log-sum-exp given)",
            "ms_recompute_lse": ms_recompute,
            "tflops_recompute_lse": backward_flops(w) / (ms_recompute * 1e-3) / 1e12,
-           "kernels": "bf16 tcgen05: dQ (+ δ; the lse pass only without the forward's lse); key-major dK/dV of the pseudo-keys (16 query ranges, reduced in order), then of the exact keys with the pseudo-key share added",
+           "kernels": "bf16 tcgen05: dQ (+ δ; the lse pass only without the forward's lse); key-major dK/dV of the pseudo-keys (16 query ranges, reduced in order), then of the exact keys with the pseudo-key share added" + ("; first-order terms through H̄ on mma.sync (δ shift, G = s Σ λ q dOᵀ in ordered partial sums, the dQ, dK, dV updates)" if w.tail == "first_order" else ""),
            "flops_per_call": fl}
     del inp, step, O, dO, dQ, dK, dV, ws, L
     torch.cuda.empty_cache()
@@ -538,7 +551,9 @@ def run_ours(args, world, rank, local):
         return 0
     if args.only == "backward":
         if rank == 0:
-            print(json.dumps({"backward": time_backward(args.steps, args.warmup)}), flush=True)
+            print(json.dumps({"backward": time_backward(args.steps, args.warmup),
+                              "backward_first_order": time_backward(args.steps, args.warmup, "video_dit_pisa")}),
+                  flush=True)
         return 0
     if args.only == "sfa":
         if rank == 0:
@@ -636,7 +651,7 @@ def run_ours(args, world, rank, local):
                "h2d_bytes_per_step": sum(inp[n].numel() * inp[n].element_size() for n in ("Q", "K", "V")),
                "d2h_bytes_per_step": step.buf.out.numel() * step.buf.out.element_size()}
 
-    decode = decode_f32 = decode_rla = fp8 = sla2 = pisa = sfa = backward = None
+    decode = decode_f32 = decode_rla = fp8 = sla2 = pisa = sfa = backward = backward_fo = None
     if rank == 0 and args.only == "all" and not args.no_decode:
         del step
         torch.cuda.empty_cache()
@@ -648,6 +663,7 @@ def run_ours(args, world, rank, local):
         pisa = time_pisa()
         sfa = time_sfa()
         backward = time_backward()
+        backward_fo = time_backward(name="video_dit_pisa")
     ck = clocks.stop() if clocks else None
 
     if rank != 0:
@@ -686,6 +702,7 @@ def run_ours(args, world, rank, local):
         "pisa": pisa,
         "sfa": sfa,
         "backward": backward,
+        "backward_first_order": backward_fo,
     }
     print(json.dumps(line), flush=True)
     return 0

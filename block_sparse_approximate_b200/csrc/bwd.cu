@@ -548,7 +548,7 @@ bwd_centroid_kernel(const T* __restrict__ Q, const T* __restrict__ dO, int H, in
 }
 
 struct BwdLayout {
-  size_t lse_off, delta_off, offs_off, list_off, part_off, total;
+  size_t lse_off, delta_off, offs_off, list_off, part_off, fo_off, total;
 };
 
 BwdLayout bwd_layout(const sa_shape& s, int topk) {
@@ -561,7 +561,9 @@ BwdLayout bwd_layout(const sa_shape& s, int topk) {
   L.list_off = L.offs_off + a256(BH * (nb + 1) * sizeof(int32_t));
   L.part_off = L.list_off + a256(BH * nb * (size_t)(topk > 0 ? topk : 1) * sizeof(int32_t));
   // the tensor-core centroid pass's partial sums (d = 128 shapes)
-  L.total = L.part_off + (s.d == 128 ? a256(bwd_tc_part_bytes(s)) : 0);
+  L.fo_off = L.part_off + (s.d == 128 ? a256(bwd_tc_part_bytes(s)) : 0);
+  // the first-order tail's per-row terms and partial H̄ gradients (d = block = 128)
+  L.total = L.fo_off + (s.d == 128 && s.block == 128 ? a256(bwd_fo_bytes(s)) : 0);
   return L;
 }
 
@@ -569,7 +571,7 @@ template <typename T, int D, int BLK>
 sa_status launch_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
                      const sa_shape& s, const int32_t* block_idx, int topk, bool zo, const sa_block_stats& st,
                      float scale, float* dQ, float* dK, float* dV, const float* lse_in, char* ws,
-                     cudaStream_t stream) {
+                     cudaStream_t stream, bool fo = false) {
   const BwdLayout L = bwd_layout(s, topk);
   const int nb = s.N / BLK;
   float* lse2 = reinterpret_cast<float*>(ws + L.lse_off);
@@ -591,9 +593,15 @@ sa_status launch_bwd(const void* Q, const void* K, const void* V, const void* O,
     } else if (cudaMemsetAsync(offs, 0, (size_t)s.B * s.H * (nb + 1) * sizeof(int32_t), stream) != cudaSuccess) {
       return launch_status("cudaMemsetAsync(bwd offsets)");
     }
+    if (fo)
+      return bwd_first_order(Q, K, V, O, dO, s, block_idx, topk, st, scale, dQ, dK, dV, lse_in, lse2, delta, offs,
+                             list, reinterpret_cast<float*>(ws + L.part_off), reinterpret_cast<float*>(ws + L.fo_off),
+                             stream);
     return bwd_tc(Q, K, V, O, dO, s, block_idx, topk, zo, st, scale, dQ, dK, dV, lse_in, lse2, delta, offs, list,
                   reinterpret_cast<float*>(ws + L.part_off), stream);
   }
+  if (fo) return fail(SA_ERR_UNSUPPORTED, "sa_sparse_attn_bwd: the first-order tail runs on the bf16 d = 128, "
+                                          "block 128 tensor-core path only");
   {
     const size_t smem = sizeof(float) * ((size_t)kBwdRows * D + (size_t)kBwdKT * (D + 4)) +
                         sizeof(uint32_t) * nwords;
@@ -635,11 +643,11 @@ template <typename T>
 sa_status dispatch_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
                        const sa_shape& s, const int32_t* block_idx, int topk, bool zo, const sa_block_stats& st,
                        float scale, float* dQ, float* dK, float* dV, const float* lse_in, char* ws,
-                       cudaStream_t stream) {
+                       cudaStream_t stream, bool fo) {
 #define SA_BWD_CASE(DD, BB)                                                                              \
   if (s.d == DD && s.block == BB)                                                                        \
     return launch_bwd<T, DD, BB>(Q, K, V, O, dO, s, block_idx, topk, zo, st, scale, dQ, dK, dV, lse_in, ws,  \
-                                 stream);
+                                 stream, fo);
   SA_BWD_CASE(128, 128)
   SA_BWD_CASE(128, 64)
   SA_BWD_CASE(64, 128)
@@ -669,31 +677,38 @@ sa_status bwd_entry(const void* Q, const void* K, const void* V, const void* O, 
   const int nb = shape.N / shape.block;
   if (dtype != SA_FP32 && dtype != SA_BF16)
     return fail(SA_ERR_UNSUPPORTED, "sa_sparse_attn_bwd: dtype must be SA_FP32 or SA_BF16");
-  if (tail != SA_TAIL_DROP && tail != SA_TAIL_ZERO_ORDER)
-    return fail(SA_ERR_UNSUPPORTED, "sa_sparse_attn_bwd: tail must be SA_TAIL_DROP or SA_TAIL_ZERO_ORDER");
+  if (tail != SA_TAIL_DROP && tail != SA_TAIL_ZERO_ORDER && tail != SA_TAIL_FIRST_ORDER)
+    return fail(SA_ERR_UNSUPPORTED,
+                "sa_sparse_attn_bwd: tail must be SA_TAIL_DROP, SA_TAIL_ZERO_ORDER or SA_TAIL_FIRST_ORDER");
   if (shape.B == 0 || shape.H == 0 || shape.N == 0) return SA_OK;
   if (!Q || !K || !V || !O || !dO || !dQ || !dK || !dV)
     return fail(SA_ERR_INVALID_ARG, "sa_sparse_attn_bwd: Q, K, V, O, dO, dQ, dK and dV are required");
   if (topk < 0 || topk > nb) return fail(SA_ERR_INVALID_ARG, "sa_sparse_attn_bwd: topk must be in [0, N/block]");
   if (topk > 0 && !block_idx) return fail(SA_ERR_INVALID_ARG, "sa_sparse_attn_bwd: block_idx is required");
   if (nb > kMaxAttnBlocks) return fail(SA_ERR_UNSUPPORTED, "sa_sparse_attn_bwd: at most 4096 blocks per head");
-  const bool zo = tail == SA_TAIL_ZERO_ORDER;
+  const bool fo = tail == SA_TAIL_FIRST_ORDER;
+  const bool zo = tail == SA_TAIL_ZERO_ORDER || fo;
   sa_block_stats st{};
   if (stats) st = *stats;
   if (zo && (!st.kmean || !st.vsum))
-    return fail(SA_ERR_INVALID_ARG, "sa_sparse_attn_bwd: SA_TAIL_ZERO_ORDER needs stats->kmean and stats->vsum");
+    return fail(SA_ERR_INVALID_ARG, "sa_sparse_attn_bwd: the zero-order tails need stats->kmean and stats->vsum");
+  if (fo && (dtype != SA_BF16 || shape.d != 128 || shape.block != 128))
+    return fail(SA_ERR_UNSUPPORTED, "sa_sparse_attn_bwd: SA_TAIL_FIRST_ORDER needs bf16, d = 128 and block 128");
+  if (fo && (!st.hbar || !st.kmean_bf16 || !st.vmean_bf16))
+    return fail(SA_ERR_INVALID_ARG,
+                "sa_sparse_attn_bwd: SA_TAIL_FIRST_ORDER needs stats->hbar, kmean_bf16 and vmean_bf16");
   const size_t need = bwd_layout(shape, topk).total;
   if (!workspace || workspace_bytes < need)
     return fail(SA_ERR_WORKSPACE, "sa_sparse_attn_bwd: workspace missing or smaller than the workspace size");
-  const void* ptrs[] = {Q, K, V, O, dO, dQ, dK, dV, workspace, block_idx, st.kmean, st.vsum, lse_in};
+  const void* ptrs[] = {Q, K, V, O, dO, dQ, dK, dV, workspace, block_idx, st.kmean, st.vsum, lse_in, st.hbar};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return fail(SA_ERR_ALIGNMENT, "sa_sparse_attn_bwd: pointers must be 16-byte aligned");
   cudaStream_t s = as_stream(stream);
   char* ws = static_cast<char*>(workspace);
   if (dtype == SA_BF16)
     return dispatch_bwd<__nv_bfloat16>(Q, K, V, O, dO, shape, block_idx, topk, zo, st, scale, dQ, dK, dV, lse_in,
-                                       ws, s);
-  return dispatch_bwd<float>(Q, K, V, O, dO, shape, block_idx, topk, zo, st, scale, dQ, dK, dV, lse_in, ws, s);
+                                       ws, s, fo);
+  return dispatch_bwd<float>(Q, K, V, O, dO, shape, block_idx, topk, zo, st, scale, dQ, dK, dV, lse_in, ws, s, fo);
 }
 }  // namespace
 }  // namespace sa

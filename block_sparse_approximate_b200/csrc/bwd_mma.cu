@@ -531,7 +531,8 @@ template <int BLK>
 sa_status bwd_tc_launch(const void* Q, const void* K, const void* V, const void* O, const void* dO,
                         const sa_shape& s, const int32_t* block_idx, int topk, bool zo, const sa_block_stats& st,
                         float scale, float* dQ, float* dK, float* dV, const float* lse_in, float* lse2,
-                        float* delta, const int32_t* offs, const int32_t* list, float* part, cudaStream_t stream) {
+                        float* delta, const int32_t* offs, const int32_t* list, float* part, cudaStream_t stream,
+                        const BwdFirstOrder* fo) {
   using bf = __nv_bfloat16;
   const int nb = s.N / BLK;
   const bf* q = static_cast<const bf*>(Q);
@@ -541,7 +542,7 @@ sa_status bwd_tc_launch(const void* Q, const void* K, const void* V, const void*
   const bf* kb = reinterpret_cast<const bf*>(st.kmean_bf16);
   const bf* vb = reinterpret_cast<const bf*>(st.vmean_bf16);
   if (BLK == 128 && (topk > 0 || zo)) {
-    sa_status r = bwd_dq_tc(Q, K, V, O, dO, s, block_idx, topk, zo, st, scale, lse_in, lse2, delta, dQ, stream);
+    sa_status r = bwd_dq_tc(Q, K, V, O, dO, s, block_idx, topk, zo, st, scale, lse_in, lse2, delta, dQ, stream, fo);
     if (r != SA_OK) return r;
   } else {
     const size_t smem = 6 * (size_t)kMTileB + sizeof(uint32_t) * ((nb + 31) / 32);
@@ -556,7 +557,7 @@ sa_status bwd_tc_launch(const void* Q, const void* K, const void* V, const void*
   const size_t smem = 6 * (size_t)kMTileB + 2 * 2 * kMT * sizeof(float);
   if constexpr (BLK == 128) {
     return bwd_dkv_tc(Q, K, V, dO, s, block_idx, topk, zo, st, offs, list, scale, lse2, delta, dK, dV, part,
-                      kCentSplits, stream);
+                      kCentSplits, stream, fo ? fo->delta_c : nullptr);
   } else {
     auto kern = bwd_dkv_mma_kernel<BLK, false>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
@@ -581,12 +582,13 @@ sa_status bwd_tc_launch(const void* Q, const void* K, const void* V, const void*
 sa_status bwd_tc(const void* Q, const void* K, const void* V, const void* O, const void* dO, const sa_shape& s,
                  const int32_t* block_idx, int topk, bool zo, const sa_block_stats& st, float scale, float* dQ,
                  float* dK, float* dV, const float* lse_in, float* lse2, float* delta, const int32_t* offs,
-                 const int32_t* list, float* part, cudaStream_t stream) {
+                 const int32_t* list, float* part, cudaStream_t stream, const BwdFirstOrder* fo) {
   if (s.block == 128)
     return bwd_tc_launch<128>(Q, K, V, O, dO, s, block_idx, topk, zo, st, scale, dQ, dK, dV, lse_in, lse2, delta,
-                              offs, list, part, stream);
+                              offs, list, part, stream, fo);
+  if (fo) return fail(SA_ERR_UNSUPPORTED, "sa_sparse_attn_bwd: the first-order tail needs block 128");
   return bwd_tc_launch<64>(Q, K, V, O, dO, s, block_idx, topk, zo, st, scale, dQ, dK, dV, lse_in, lse2, delta,
-                           offs, list, part, stream);
+                           offs, list, part, stream, nullptr);
 }
 
 }  // namespace sa

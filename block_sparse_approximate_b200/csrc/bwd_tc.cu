@@ -19,6 +19,11 @@
 // when the forward's log-sum-exp is given); pass 2
 // forms S again, dP = dO Vᵀ, writes dS (bf16) into the S columns, and
 // accumulates dQ += dS · K with dS read from TMEM.
+// PISA's first-order tail (doff non-null): a pseudo-key's value seen by row t
+// is v̄_j + f_t / B (f_t = s H̄ᵀ q_t), so the centroid tiles take
+// dS = P (dP − δ + doff_t) with doff_t = dO_t·f_t / B; the kernel also writes
+// that row's centroid δ (delta_c = δ − doff) for the centroid dK/dV pass and
+// each group's share of λ_t = Σ_{pseudo-keys} P / B (lam[grp · lam_stride + row]).
 // TMEM (512 columns): S₀ [0,128), S₁ [128,256) (tile g in S_{g mod 2}),
 // dP [256,384), dQ [384,512).  dS of tile g goes to columns [32, 96) of its S
 // buffer: group 0 writes [32, 64) and group 1 [64, 96), each inside the
@@ -99,7 +104,8 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                  const __nv_bfloat16* __restrict__ O, const __nv_bfloat16* __restrict__ dO,
                  const int32_t* __restrict__ block_idx, int N, int topk, int zo, float scale,
                  const float* __restrict__ lse_in, float* __restrict__ lse2, float* __restrict__ delta,
-                 float* __restrict__ dQ) {
+                 float* __restrict__ dQ, const float* __restrict__ doff, float* __restrict__ delta_c,
+                 float* __restrict__ lam, size_t lam_stride) {
   using L = Lay;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -361,6 +367,8 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     tc_fence_before();
     named_bar_ew();
     tc_fence_after();
+    const float dof = doff ? doff[row] : 0.f;
+    if (ok && grp == 0 && delta_c) delta_c[row] = dl - dof;
     if (ok && P1 == 0) {
       lse = lse_in[row];
       if (grp == 0) {
@@ -385,6 +393,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     // both groups have read the exchange before the first dQ MMA overwrites it
     // (that MMA waits for every thread's arrival on the S barrier of tile P1)
     // ---- pass 2: dS = P (dP − δ) into the S columns [32, 96)
+    float lam_part = 0.f;   // Σ P over this group's pseudo-keys
     for (int g = P1; ok && g < G; ++g) {
       const int t = g - P1, b = g & 1;
       if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_SF + b), (g >> 1) & 1, abort_flag)) ||
@@ -401,7 +410,10 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       tmem_wait_ld();
       uint32_t vb0, vb1;
       valid_bits(t, vb0, vb1);
-      const float nb2 = (t < topk ? 0.f : 7.0f) - lse;
+      const bool cent = t >= topk;
+      const float nb2 = (cent ? 7.0f : 0.f) - lse;
+      const float dlt = cent ? dl - dof : dl;
+      float psum = 0.f;
 #pragma unroll
       for (int c = 0; c < 32; ++c) {
         float ds[2];
@@ -410,16 +422,19 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
           const int cc = 2 * c + e;
           const bool ok_c = ((cc < 32 ? vb0 : vb1) >> (cc & 31)) & 1u;
           const float pr = ok_c ? fast_exp2(fmaf(__uint_as_float(v[cc]), scale2, nb2)) : 0.f;
-          ds[e] = pr * (__uint_as_float(p[cc]) - dl);
+          psum += pr;
+          ds[e] = pr * (__uint_as_float(p[cc]) - dlt);
         }
         v[c] = pack_bf16(ds[0], ds[1]);
       }
+      if (cent) lam_part += psum;
       tmem_st32(lrow + (uint32_t)b * TB + 32 + 32 * grp, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(L::B_SC + b));
     }
     ok = __all_sync(0xffffffffu, ok) && !*abort_flag;
+    if (ok && lam) lam[(size_t)grp * lam_stride + row] = lam_part * (1.0f / TB);   // ÷ B = 128
     if (ok && T > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_DQ), 0, abort_flag));
     float4* out = reinterpret_cast<float4*>(dQ + row * TD + 64 * grp);
     if (ok && T > 0) {
@@ -784,7 +799,8 @@ bwd_cent_reduce_kernel(float* __restrict__ part, int nb, int nsplit) {
 
 sa_status bwd_dq_tc(const void* Q, const void* K, const void* V, const void* O, const void* dO, const sa_shape& s,
                     const int32_t* block_idx, int topk, bool zo, const sa_block_stats& st, float scale,
-                    const float* lse_in, float* lse2, float* delta, float* dQ, cudaStream_t stream) {
+                    const float* lse_in, float* lse2, float* delta, float* dQ, cudaStream_t stream,
+                    const BwdFirstOrder* fo) {
   const int nb = s.N / TB;
   const uint64_t BH = (uint64_t)s.B * s.H;
   alignas(64) CUtensorMap mq, mg, mk, mv, mkb, mvb;
@@ -804,14 +820,15 @@ sa_status bwd_dq_tc(const void* Q, const void* K, const void* V, const void* O, 
     return launch_status("cudaFuncSetAttribute(bwd_dq_tc_kernel)");
   bwd_dq_tc_kernel<<<dim3(nb, (unsigned)BH), kThreads, smem, stream>>>(
       mq, mg, mk, mv, mkb, mvb, static_cast<const __nv_bfloat16*>(O), static_cast<const __nv_bfloat16*>(dO),
-      block_idx, s.N, topk, zo ? 1 : 0, scale, lse_in, lse2, delta, dQ);
+      block_idx, s.N, topk, zo ? 1 : 0, scale, lse_in, lse2, delta, dQ, fo ? fo->doff : nullptr,
+      fo ? fo->delta_c : nullptr, fo ? fo->lam : nullptr, (size_t)BH * s.N);
   return launch_status("bwd_dq_tc_kernel");
 }
 
 sa_status bwd_dkv_tc(const void* Q, const void* K, const void* V, const void* dO, const sa_shape& s,
                      const int32_t* block_idx, int topk, bool zo, const sa_block_stats& st, const int32_t* offs,
                      const int32_t* list, float scale, const float* lse2, const float* delta, float* dK, float* dV,
-                     float* part, int nsplit, cudaStream_t stream) {
+                     float* part, int nsplit, cudaStream_t stream, const float* delta_cent) {
   const int nb = s.N / TB;
   const uint64_t BH = (uint64_t)s.B * s.H;
   alignas(64) CUtensorMap mq, mg, mk, mv;
@@ -831,8 +848,8 @@ sa_status bwd_dkv_tc(const void* Q, const void* K, const void* V, const void* dO
       return launch_status("cudaFuncSetAttribute(bwd_dkv_tc_kernel)");
     const int ntc = (nb + TB - 1) / TB;
     kc<<<dim3(ntc * nsplit, (unsigned)BH), kThreads, KvLay::kSmem, stream>>>(
-        mq, mg, mkb, mvb, s.N, topk, offs, list, block_idx, nsplit, scale, lse2, delta, nullptr, nullptr, dK, dV,
-        part);
+        mq, mg, mkb, mvb, s.N, topk, offs, list, block_idx, nsplit, scale, lse2, delta_cent ? delta_cent : delta,
+        nullptr, nullptr, dK, dV, part);
     sa_status r = launch_status("bwd_dkv_tc_kernel(centroids)");
     if (r != SA_OK) return r;
     bwd_cent_reduce_kernel<<<dim3(nb, (unsigned)BH), TD, 0, stream>>>(part, nb, nsplit);

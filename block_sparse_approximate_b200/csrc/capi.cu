@@ -70,10 +70,10 @@ sa_status fwd_entry(const void* Q, const void* K, const void* V, sa_dtype dtype,
                            (st.kmean_bf16 && st.vmean_bf16 && (tail == SA_TAIL_ZERO_ORDER || st.hbarT_bf16));
   const bool tc = attn_tc_supports(dtype, shape, tail) && tc_operands;
   if (lse2) {
-    if (!tc || (tail != SA_TAIL_DROP && tail != SA_TAIL_ZERO_ORDER))
+    if (!tc || (tail != SA_TAIL_DROP && tail != SA_TAIL_ZERO_ORDER && tail != SA_TAIL_FIRST_ORDER))
       return fail(SA_ERR_UNSUPPORTED,
                   "sa_sparse_attn_fwd_lse: the log-sum-exp comes from the bf16 tensor-core kernel (d = 128, "
-                  "block 128, SA_TAIL_DROP or SA_TAIL_ZERO_ORDER with the bf16 centroids)");
+                  "block 128, SA_TAIL_DROP, SA_TAIL_ZERO_ORDER or SA_TAIL_FIRST_ORDER with the bf16 centroids)");
     if (!aligned16(lse2)) return fail(SA_ERR_ALIGNMENT, "sa_sparse_attn_fwd_lse: lse2 must be 16-byte aligned");
   }
   if (tc) return attn_tc(Q, K, V, shape, block_idx, topk, tail, alpha, st, scale, O, lse2, s);

@@ -189,8 +189,10 @@ sa_status sa_sparse_attn_fwd(const void* Q, const void* K, const void* V, sa_dty
  * DROP the first sum alone), +inf for a row without keys.  sa_sparse_attn_bwd_lse takes it to skip the
  * recomputation of the row statistics.  lse2: float32 [B,H,N], caller-owned,
  * 16-byte aligned.  Only the bf16 tensor-core kernel produces it: d = 128,
- * block 128, SA_TAIL_DROP or SA_TAIL_ZERO_ORDER (with stats->kmean_bf16 and
- * vmean_bf16); anything else returns SA_ERR_UNSUPPORTED.
+ * block 128, SA_TAIL_DROP, SA_TAIL_ZERO_ORDER or SA_TAIL_FIRST_ORDER (with
+ * stats->kmean_bf16 and vmean_bf16, + hbarT_bf16 for FIRST_ORDER; the
+ * first-order term changes the numerator only, so D_t is the zero-order one);
+ * anything else returns SA_ERR_UNSUPPORTED.
  * Errors: those of sa_sparse_attn_fwd; SA_ERR_INVALID_ARG without lse2. */
 sa_status sa_sparse_attn_fwd_lse(const void* Q, const void* K, const void* V, sa_dtype dtype,
                                  sa_shape shape, const int32_t* block_idx, int32_t topk,
@@ -200,9 +202,9 @@ sa_status sa_sparse_attn_fwd_lse(const void* Q, const void* K, const void* V, sa
 /* Bytes of workspace sa_sparse_attn_bwd needs (0 on bad arguments). */
 size_t sa_sparse_attn_bwd_workspace_size(sa_shape shape, int32_t topk);
 
-/* Backward of sa_sparse_attn_fwd for the DROP and ZERO_ORDER tails: given the
- * forward's inputs, its output O and the output cotangent dO, writes
- * dQ, dK, dV (float32 [B,H,N,d], overwritten).  The forward is softmax
+/* Backward of sa_sparse_attn_fwd for the DROP, ZERO_ORDER and FIRST_ORDER
+ * tails: given the forward's inputs, its output O and the output cotangent dO,
+ * writes dQ, dK, dV (float32 [B,H,N,d], overwritten).  The forward is softmax
  * attention of query block i to its exact keys k_n (n in the selected
  * blocks) and, for ZERO_ORDER, one pseudo-key per unselected block j (key
  * k̄_j, value vsum_j / block, logit bias ln block), so with
@@ -210,6 +212,14 @@ size_t sa_sparse_attn_bwd_workspace_size(sa_shape shape, int32_t topk);
  *   dQ = s Σ ds k,   dK_key = s Σ ds q,   dV_key = Σ p dO,
  * and each pseudo-key's gradients are spread over its block's tokens
  * divided by block (k̄ and vsum / block are means of the block's k and v).
+ * FIRST_ORDER [PISA §2 "Algoritmo Central", hybrid order] adds λ_t f_t to the
+ * zero-order output, f_t = s H̄ᵀ q_t, λ_t = Σ_{pseudo-keys} p / block: the
+ * pseudo-keys' value seen by row t is v̄_j + f_t / block, and with
+ * G = s Σ_t λ_t q_t dO_tᵀ the gradients gain dq_t += s λ_t H̄ dO_t,
+ * dk_m += G (v_m − v̄_j) / nb and dv_m += Gᵀ (k_m − k̄_j) / nb for every
+ * token m of block j (through H̄ = (1/nb) Σ_j Σ_{m∈j} (k_m − k̄_j) v_mᵀ); it
+ * runs for bf16, d = 128, block 128 only (SA_ERR_UNSUPPORTED otherwise) and
+ * needs stats->kmean, vsum, kmean_bf16, vmean_bf16 and hbar.
  * Q, K, V, O, dO of `dtype`; block_idx, topk, tail, stats (kmean, vsum for
  * ZERO_ORDER) and scale as given to the forward.  workspace: at least
  * sa_sparse_attn_bwd_workspace_size() bytes, 16-byte aligned.  bf16 with

@@ -71,9 +71,13 @@ def sparse_attention_lse(Q, K, block_idx, block: int, tail: str, scale: float) -
     """[B,H,N] float64: each query row's log-sum-exp of its logits in log2
     units, log2 Σ exp(s q·k + bias) over the row's key list of
     ``sparse_attention_backward`` (exact keys bias 0, pseudo-keys ln B); +inf
-    for a row without keys."""
-    if tail not in ("drop", "zero_order"):
-        raise ValueError("the log-sum-exp is defined for the drop and zero_order tails")
+    for a row without keys.  "first_order" has the zero-order denominator
+    (PISA's first-order term changes the numerator only), so its log-sum-exp
+    is the zero-order one."""
+    if tail not in ("drop", "zero_order", "first_order"):
+        raise ValueError("the log-sum-exp is defined for the drop, zero_order and first_order tails")
+    if tail == "first_order":
+        tail = "zero_order"
     Q, K = _f64(Q), _f64(K)
     Bsz, H, N, d = K.shape
     nb = N // block
@@ -99,11 +103,19 @@ def sparse_attention_lse(Q, K, block_idx, block: int, tail: str, scale: float) -
 
 
 def sparse_attention_backward(Q, K, V, block_idx, block: int, tail: str, scale: float, dO, *, alpha=None,
-                              eps: float = 1e-6):
+                              eps: float = 1e-6, o_forward=None):
     """(dQ, dK, dV) [B,H,N,d] float64 of sparse_attention(tail) at (Q, K, V)
     for the output cotangent dO [B,H,N,d]; tail "drop", "zero_order",
     "first_order" or "linear_mix" (with alpha [H,d] and the linear branch's
-    eps)."""
+    eps).
+
+    ``o_forward`` [B,H,N,d] (drop and zero_order): the output a quantised
+    forward produced.  SLA2 §2C runs the forward of its low-precision sparse
+    branch quantised and keeps the backward in 16 bits; read as a
+    straight-through estimator, the gradients are those above at the
+    unquantised operands, with δ_t = dO_t·o_t taken from the forward that
+    ran (the only quantity of the backward that comes from the forward's
+    output)."""
     if tail == "first_order":
         return _first_order_backward(Q, K, V, block_idx, block, scale, dO)
     if tail == "linear_mix":
@@ -113,6 +125,7 @@ def sparse_attention_backward(Q, K, V, block_idx, block: int, tail: str, scale: 
     if tail not in ("drop", "zero_order"):
         raise ValueError(f"no backward for tail {tail!r}")
     Q, K, V, dO = _f64(Q), _f64(K), _f64(V), _f64(dO)
+    Of = None if o_forward is None else _f64(o_forward)
     Bsz, H, N, d = K.shape
     nb = N // block
     idx = np.asarray(block_idx)
@@ -139,7 +152,7 @@ def sparse_attention_backward(Q, K, V, block_idx, block: int, tail: str, scale: 
                 a = scale * q @ keys.T + bias
                 p = np.exp(a - a.max(axis=1, keepdims=True))
                 p /= p.sum(axis=1, keepdims=True)
-                o = p @ vals
+                o = p @ vals if Of is None else Of[b, h, rows]
                 dvals = p.T @ g
                 dp = g @ vals.T
                 delta = (g * o).sum(axis=1, keepdims=True)

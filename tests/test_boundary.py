@@ -127,9 +127,12 @@ def test_lse_entry_validation(lib):
         == bd.SA_ERR_UNSUPPORTED            # fp32 runs on the CUDA-core kernel
     assert f(FAKE, FAKE, FAKE, 1, bd.Shape(1, 1, 1024, 64, 128), FAKE, 2, 0, ctypes.byref(none), 0.1, FAKE,
              FAKE, None) == bd.SA_ERR_UNSUPPORTED   # d = 64
-    fo = _stats(kmean=FAKE, vsum=FAKE, hbar=FAKE, kmean_bf16=FAKE, vmean_bf16=FAKE, hbarT_bf16=FAKE)
-    assert f(FAKE, FAKE, FAKE, 1, sh, FAKE, 2, 3, ctypes.byref(fo), 0.1, FAKE, FAKE, None) \
-        == bd.SA_ERR_UNSUPPORTED            # first-order tail
+    lin = _stats(zrelu=FAKE, htot=FAKE, ztot=FAKE)
+    assert f(FAKE, FAKE, FAKE, 1, sh, FAKE, 2, 2, ctypes.byref(lin), 0.1, FAKE, FAKE, None) \
+        == bd.SA_ERR_INVALID_ARG            # the linear mix (no alpha through this entry)
+    fo_cuda = _stats(kmean=FAKE, vsum=FAKE, hbar=FAKE)
+    assert f(FAKE, FAKE, FAKE, 1, sh, FAKE, 2, 3, ctypes.byref(fo_cuda), 0.1, FAKE, FAKE, None) \
+        == bd.SA_ERR_UNSUPPORTED            # first-order tail without the bf16 tiles: CUDA-core kernel
     assert f(FAKE, FAKE, FAKE, 1, sh, FAKE, 2, 0, ctypes.byref(none), 0.1, FAKE, FAKE + 4, None) \
         == bd.SA_ERR_ALIGNMENT
     g = lib.sa_sparse_attn_bwd_lse

@@ -219,3 +219,32 @@ def test_linear_mix_limits():
     o.backward(torch.tensor(dO))
     for got, t in zip(lm, (tq, tk, tv)):
         np.testing.assert_allclose(got, t.grad.numpy(), rtol=1e-10, atol=1e-12)
+
+
+# ---- the straight-through backward of a quantised forward (o_forward) ------
+
+@pytest.mark.parametrize("tail", ["zero_order", "drop"])
+def test_backward_with_the_forwards_own_output_is_unchanged(tail):
+    rng = np.random.default_rng(18)
+    Q, K, V, idx, dO, blk = _case(rng)
+    O = oracle.sparse_attention(Q, K, V, idx, blk, tail, S)
+    a = oracle.sparse_attention_backward(Q, K, V, idx, blk, tail, S, dO)
+    b = oracle.sparse_attention_backward(Q, K, V, idx, blk, tail, S, dO, o_forward=O)
+    for x, y in zip(a, b):
+        np.testing.assert_allclose(x, y, rtol=1e-12, atol=1e-14)
+
+
+def test_backward_shift_of_delta_closed_form():
+    # o_forward = O + E shifts δ by Δ_t = dO_t·E_t; dS = P (dP − δ) moves by
+    # −P Δ, so dQ moves by −s Δ_t Σ_k P_tk k_k = −s Δ_t · (attention of Q to K
+    # with the keys as values), and dV does not move
+    rng = np.random.default_rng(19)
+    Q, K, V, idx, dO, blk = _case(rng)
+    O = oracle.sparse_attention(Q, K, V, idx, blk, "zero_order", S)
+    E = 0.05 * rng.standard_normal(O.shape)
+    a = oracle.sparse_attention_backward(Q, K, V, idx, blk, "zero_order", S, dO)
+    b = oracle.sparse_attention_backward(Q, K, V, idx, blk, "zero_order", S, dO, o_forward=O + E)
+    shift = (dO * E).sum(axis=-1, keepdims=True)
+    pk = oracle.sparse_attention(Q, K, K, idx, blk, "zero_order", S)
+    np.testing.assert_allclose(b[0] - a[0], -S * shift * pk, rtol=1e-9, atol=1e-12)
+    np.testing.assert_allclose(b[2], a[2], rtol=1e-12, atol=1e-14)

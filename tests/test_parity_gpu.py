@@ -499,6 +499,82 @@ def test_backward_batched_heads(lib, tail):
             assert_tol(np64(got), r, (3e-2, 2e-3), f"batched backward ({what}) {tail} {name}")
 
 
+@pytest.mark.parametrize("B,H,nb,k", [(1, 2, 9, 3), (1, 2, 37, 5), (1, 1, 133, 13), (1, 2, 20, 0), (1, 2, 8, 8),
+                                      (2, 3, 10, 3)])
+def test_backward_first_order(lib, B, H, nb, k):
+    # PISA's hybrid order: inputs whose values follow the keys' in-block
+    # deviations, so the first-order terms move the gradients well past the
+    # tolerance (checked against the zero-order backward of the same inputs)
+    block, d = 128, 128
+    inp = wl.block_linear_inputs(B, H, nb, block, d, torch.bfloat16, 130 + nb + k, DEV)
+    Q, K, V = inp["Q"], inp["K"], inp["V"]
+    N = nb * block
+    g = torch.Generator(device=DEV)
+    g.manual_seed(131)
+    dO = torch.randn(B, H, N, d, generator=g, device=DEV).to(torch.bfloat16)
+    s = 1 / math.sqrt(d)
+    st = bd.block_pool(Q, K, V, block, centroids_bf16=True, first_order=True)
+    idx, _ = bd.route(st, (B, H, N, d, block), "dot", k)
+    L = torch.empty(B, H, N, device=DEV, dtype=torch.float32)
+    O = bd.sparse_attn_fwd(Q, K, V, idx, block, "first_order", st, s, lse=L)
+    grads = bd.sparse_attn_bwd(Q, K, V, O, dO, idx, block, "first_order", st, s)
+    grads_lse = bd.sparse_attn_bwd(Q, K, V, O, dO, idx, block, "first_order", st, s, lse=L)
+    torch.cuda.synchronize()
+    assert_no_device_error()
+    args = (np64(Q), np64(K), np64(V), idx.cpu().numpy(), block)
+    ref = oracle.sparse_attention_backward(*args, "first_order", s, np64(dO))
+    zo = oracle.sparse_attention_backward(*args, "zero_order", s, np64(dO))
+    # the centroid logits use the bf16 block means: up to s Σ_c |q_c k̄_c| 2^-9
+    # per logit, ~5e-3 in log2 units for these keys (centroids ~ N(0, 1))
+    np.testing.assert_allclose(np64(L), oracle.sparse_attention_lse(np64(Q), np64(K), idx.cpu().numpy(), block,
+                                                                    "first_order", s), rtol=0, atol=1e-2)
+    for got_set, what in ((grads, "recomputed lse"), (grads_lse, "forward's lse")):
+        for got, r, name in zip(got_set, ref, ("dQ", "dK", "dV")):
+            sc = max(1.0, float(np.abs(r).max()))
+            assert_tol(np64(got), r, (2e-2 * sc, 2e-3), f"first-order backward ({what}) {name}")
+    if k < nb:
+        assert max(float(np.abs(r - z).max()) for r, z in zip(ref, zo)) > 0.1
+
+
+def test_backward_of_the_e4m3_forward_straight_through(lib):
+    # SLA2 §2C: the forward of the sparse branch runs in e4m3, the backward in
+    # 16 bits.  Straight-through: the bf16 backward at the unquantised
+    # operands, δ = dO·O from the forward that ran.  The GPU backward given the
+    # oracle's e4m3 forward output matches the oracle's straight-through
+    # backward; dV (Pᵀ dO) does not depend on the forward's output at all.
+    B, H, nb, k, d, block = 1, 2, 12, 3, 128, 128
+    N = nb * block
+    Q, K, V = _gauss(B, H, N, d, torch.bfloat16, 140)
+    g = torch.Generator(device=DEV)
+    g.manual_seed(141)
+    dO = torch.randn(B, H, N, d, generator=g, device=DEV).to(torch.bfloat16)
+    s = 1 / math.sqrt(d)
+    st = bd.block_pool(Q, K, V, block, centroids_bf16=True)
+    idx, _ = bd.route(st, (B, H, N, d, block), "dot", k)
+    O8 = bd.sparse_attn_fwd_fp8(bd.fp8_operands(Q, K, V, st), (B, H, N, d, block), idx, "zero_order", s)
+    g8 = bd.sparse_attn_bwd(Q, K, V, O8, dO, idx, block, "zero_order", st, s)
+    args = (np64(Q), np64(K), np64(V), idx.cpu().numpy(), block)
+    emu = oracle.fp8_attention(*args, "zero_order", s)
+    Oe = torch.as_tensor(emu).to(DEV, torch.bfloat16)
+    ge = bd.sparse_attn_bwd(Q, K, V, Oe, dO, idx, block, "zero_order", st, s)
+    torch.cuda.synchronize()
+    assert_no_device_error()
+    ref = oracle.sparse_attention_backward(*args, "zero_order", s, np64(dO), o_forward=emu)
+    for got, r, name in zip(ge, ref, ("dQ", "dK", "dV")):
+        assert_tol(np64(got), r, (3e-2, 2e-3), f"straight-through backward {name}")
+    assert torch.equal(g8[2], ge[2])
+
+
+def test_backward_first_order_is_rejected_off_the_tensor_cores(lib):
+    Q, K, V = _gauss(1, 1, 512, 64, torch.float32, 132)
+    st = bd.block_pool(Q, K, V, 64, first_order=True)
+    idx, _ = bd.route(st, (1, 1, 512, 64, 64), "dot", 2)
+    O = bd.sparse_attn_fwd(Q, K, V, idx, 64, "first_order", st, 0.125)
+    with pytest.raises(bd.SparseAttnError) as e:
+        bd.sparse_attn_bwd(Q, K, V, O, O, idx, 64, "first_order", st, 0.125)
+    assert e.value.status == bd.SA_ERR_UNSUPPORTED
+
+
 @pytest.mark.parametrize("tail", ["zero_order", "drop"])
 @pytest.mark.parametrize("nb,k", [(12, 3), (133, 13), (20, 0), (8, 8)])
 def test_forward_lse_and_backward_lse(lib, tail, nb, k):
