@@ -531,6 +531,59 @@ def time_sla2(steps: int = 2, warmup: int = 1):
     return out
 
 
+def time_backward_linear_mix(steps: int = 2, warmup: int = 1):
+    """Backward of the SLA2 mix workload (H=40, N=65536, linear mix):
+    sa_sparse_attn_bwd_linear_mix on the step's inputs, output and a random dO.
+    FLOPs: the softmax branch's drop backward recomputing its log-sum-exp,
+    16·d per (row, selected key), plus the linear branch's products, 14·d² per
+    row (h_j; H_U·φ(q) twice; dH_U; the dq product; the dk, dv products)."""
+    import ctypes
+    from block_sparse_approximate_b200 import binding as bd
+    from block_sparse_approximate_b200.pipeline import PrefillStep
+    w = wl.WORKLOADS["sla2_mix"]
+    inp = wl.prefill_inputs(w, "cuda")
+    step = PrefillStep(w, inp)
+    O = step()
+    g = torch.Generator(device="cuda")
+    g.manual_seed(98)
+    dO = torch.randn(O.shape, generator=g, device="cuda").to(O.dtype)
+    lib = bd.load()
+    shape = bd.Shape(w.B, w.H, w.N, w.d, w.block)
+    ws = torch.empty(int(lib.sa_sparse_attn_bwd_linear_mix_workspace_size(shape, w.k)), device="cuda",
+                     dtype=torch.uint8)
+    f = dict(device="cuda", dtype=torch.float32)
+    dQ, dK, dV = torch.empty(O.shape, **f), torch.empty(O.shape, **f), torch.empty(O.shape, **f)
+    buf = step.buf
+
+    def bwd():
+        bd._check("sa_sparse_attn_bwd_linear_mix", lib.sa_sparse_attn_bwd_linear_mix(
+            inp["Q"].data_ptr(), inp["K"].data_ptr(), inp["V"].data_ptr(), O.data_ptr(), dO.data_ptr(), bd.SA_BF16,
+            shape, buf.block_idx.data_ptr(), int(w.k), inp["alpha"].data_ptr(), ctypes.byref(step.cst),
+            float(w.scale), dQ.data_ptr(), dK.data_ptr(), dV.data_ptr(), ws.data_ptr(), ws.numel(),
+            bd._stream(None)))
+
+    for _ in range(warmup):
+        bwd()
+    torch.cuda.synchronize()
+    s_, e_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s_.record()
+    for _ in range(steps):
+        bwd()
+    e_.record()
+    torch.cuda.synchronize()
+    ms = s_.elapsed_time(e_) / steps
+    fl = (16.0 * w.d * w.k * w.block + 14.0 * w.d * w.d) * w.B * w.H * float(w.N)
+    _, bf16, _, src = _peaks()
+    ach = fl / (ms * 1e-3) / 1e12
+    out = {"workload": w.name, "tail": w.tail, "ms": ms, "tflops": ach, "peak_tflops": bf16, "frac": ach / bf16,
+           "peak_source": f"{src} bf16 burst", "entry": "sa_sparse_attn_bwd_linear_mix", "flops_per_call": fl,
+           "kernels": "softmax branch: tcgen05 drop backward of alpha*dO with the branch's delta; linear branch on "
+                      "mma.sync (per-block h_j, per-query-block H_U, dH_U, key-major dh_j)"}
+    del inp, step, O, dO, dQ, dK, dV, ws
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args, world, rank, local):
     from block_sparse_approximate_b200 import binding as bd
     from block_sparse_approximate_b200.pipeline import PrefillStep
@@ -552,7 +605,8 @@ def run_ours(args, world, rank, local):
     if args.only == "backward":
         if rank == 0:
             print(json.dumps({"backward": time_backward(args.steps, args.warmup),
-                              "backward_first_order": time_backward(args.steps, args.warmup, "video_dit_pisa")}),
+                              "backward_first_order": time_backward(args.steps, args.warmup, "video_dit_pisa"),
+                              "backward_linear_mix": time_backward_linear_mix(min(args.steps, 2), 1)}),
                   flush=True)
         return 0
     if args.only == "sfa":
@@ -651,7 +705,7 @@ def run_ours(args, world, rank, local):
                "h2d_bytes_per_step": sum(inp[n].numel() * inp[n].element_size() for n in ("Q", "K", "V")),
                "d2h_bytes_per_step": step.buf.out.numel() * step.buf.out.element_size()}
 
-    decode = decode_f32 = decode_rla = fp8 = sla2 = pisa = sfa = backward = backward_fo = None
+    decode = decode_f32 = decode_rla = fp8 = sla2 = pisa = sfa = backward = backward_fo = backward_lm = None
     if rank == 0 and args.only == "all" and not args.no_decode:
         del step
         torch.cuda.empty_cache()
@@ -664,6 +718,7 @@ def run_ours(args, world, rank, local):
         sfa = time_sfa()
         backward = time_backward()
         backward_fo = time_backward(name="video_dit_pisa")
+        backward_lm = time_backward_linear_mix()
     ck = clocks.stop() if clocks else None
 
     if rank != 0:
@@ -703,6 +758,7 @@ def run_ours(args, world, rank, local):
         "sfa": sfa,
         "backward": backward,
         "backward_first_order": backward_fo,
+        "backward_linear_mix": backward_lm,
     }
     print(json.dumps(line), flush=True)
     return 0

@@ -53,18 +53,21 @@ uint32_t covnorm_error_take();
 // delta [B·H·N] and the per-KV-block query lists offs/list come from the
 // caller's workspace (offs/list filled beforehand).
 bool bwd_tc_supports(sa_dtype dtype, const sa_shape& s, bool zo, const sa_block_stats& st);
-// PISA's first-order tail in the backward (block 128 tensor-core path):
-// doff [B·H·N] = dO_t·f_t / B (input), delta_c [B·H·N] the centroid keys' δ and
-// lam [2][B·H·N] the two element-wise groups' shares of λ_t (outputs).
-struct BwdFirstOrder {
+// Tail terms of the block-128 tensor-core backward, each pointer optional:
+// PISA's first-order tail: doff [B·H·N] = dO_t·f_t / B (input), delta_c
+// [B·H·N] the centroid keys' δ and lam [2][B·H·N] the two element-wise groups'
+// shares of λ_t (outputs); SLA2's linear mix: delta_in [B·H·N] the rows' δ of
+// the softmax branch, used instead of dO·O (input).
+struct BwdTailTerms {
   const float* doff;
   float* delta_c;
   float* lam;
+  const float* delta_in;
 };
 sa_status bwd_tc(const void* Q, const void* K, const void* V, const void* O, const void* dO, const sa_shape& s,
                  const int32_t* block_idx, int topk, bool zo, const sa_block_stats& st, float scale, float* dQ,
                  float* dK, float* dV, const float* lse_in, float* lse2, float* delta, const int32_t* offs,
-                 const int32_t* list, float* part, cudaStream_t stream, const BwdFirstOrder* fo = nullptr);
+                 const int32_t* list, float* part, cudaStream_t stream, const BwdTailTerms* fo = nullptr);
 // bytes of the centroid pass's partial sums (workspace)
 size_t bwd_tc_part_bytes(const sa_shape& s);
 // dQ (with lse2 and delta) on tcgen05 (bwd_tc.cu): block 128, d = 128, at
@@ -73,7 +76,7 @@ size_t bwd_tc_part_bytes(const sa_shape& s);
 sa_status bwd_dq_tc(const void* Q, const void* K, const void* V, const void* O, const void* dO, const sa_shape& s,
                     const int32_t* block_idx, int topk, bool zo, const sa_block_stats& st, float scale,
                     const float* lse_in, float* lse2, float* delta, float* dQ, cudaStream_t stream,
-                    const BwdFirstOrder* fo = nullptr);
+                    const BwdTailTerms* fo = nullptr);
 // dK, dV on tcgen05 (bwd_tc.cu), block 128, d = 128, written for every key:
 // the exact keys' sums plus, with the zero-order tail (zo), each block's
 // pseudo-key gradients ÷B (formed first in `part`, nsplit query ranges);
@@ -87,6 +90,15 @@ uint32_t bwd_error_take();
 // the zero-order tensor-core backward with the pseudo-keys' δ shifted, then
 // the terms through H̄.  fo_ws: bwd_fo_bytes(s) of workspace.
 size_t bwd_fo_bytes(const sa_shape& s);
+// SLA2's linear mix in the backward (bwd_lin.cu; bf16, d = block = 128): the
+// drop backward of α⊙dO with the softmax branch's δ, then the linear branch.
+// lin_ws: bwd_lin_bytes(s) of workspace.
+size_t bwd_lin_bytes(const sa_shape& s);
+sa_status bwd_linear_mix(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                         const sa_shape& s, const int32_t* block_idx, int topk, const float* alpha,
+                         const sa_block_stats& st, float scale, float* dQ, float* dK, float* dV, float* lse2,
+                         float* delta, const int32_t* offs, const int32_t* list, float* part, char* lin_ws,
+                         cudaStream_t stream);
 sa_status bwd_first_order(const void* Q, const void* K, const void* V, const void* O, const void* dO,
                           const sa_shape& s, const int32_t* block_idx, int topk, const sa_block_stats& st, float scale,
                           float* dQ, float* dK, float* dV, const float* lse_in, float* lse2, float* delta,

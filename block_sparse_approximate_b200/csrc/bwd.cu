@@ -731,3 +731,68 @@ extern "C" sa_status sa_sparse_attn_bwd_lse(const void* Q, const void* K, const 
   return sa::bwd_entry(Q, K, V, O, dO, dtype, shape, block_idx, topk, tail, stats, scale, lse2, dQ, dK, dV,
                        workspace, workspace_bytes, stream);
 }
+
+// ---- SLA2's linear mix -----------------------------------------------------
+namespace sa {
+namespace {
+size_t lin_workspace_bytes(const sa_shape& s, int topk) {
+  auto a256 = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  return a256(bwd_layout(s, topk).total) + bwd_lin_bytes(s);
+}
+}  // namespace
+}  // namespace sa
+
+extern "C" size_t sa_sparse_attn_bwd_linear_mix_workspace_size(sa_shape shape, int32_t topk) {
+  using namespace sa;
+  if (check_shape(shape, "sa_sparse_attn_bwd_linear_mix_workspace_size") != SA_OK || topk < 0) return 0;
+  if (shape.d != 128 || shape.block != 128) return 0;
+  return lin_workspace_bytes(shape, topk);
+}
+
+extern "C" sa_status sa_sparse_attn_bwd_linear_mix(const void* Q, const void* K, const void* V, const void* O,
+                                                   const void* dO, sa_dtype dtype, sa_shape shape,
+                                                   const int32_t* block_idx, int32_t topk, const float* alpha,
+                                                   const sa_block_stats* stats, float scale, float* dQ, float* dK,
+                                                   float* dV, void* workspace, size_t workspace_bytes,
+                                                   void* stream) {
+  using namespace sa;
+  sa_status r = check_shape(shape, "sa_sparse_attn_bwd_linear_mix");
+  if (r != SA_OK) return r;
+  const int nb = shape.N / shape.block;
+  if (dtype != SA_BF16 || shape.d != 128 || shape.block != 128)
+    return fail(SA_ERR_UNSUPPORTED, "sa_sparse_attn_bwd_linear_mix: bf16, d = 128 and block 128 only");
+  if (shape.B == 0 || shape.H == 0 || shape.N == 0) return SA_OK;
+  if (!Q || !K || !V || !O || !dO || !dQ || !dK || !dV || !alpha || !stats)
+    return fail(SA_ERR_INVALID_ARG,
+                "sa_sparse_attn_bwd_linear_mix: Q, K, V, O, dO, alpha, stats, dQ, dK and dV are required");
+  if (topk < 0 || topk > nb)
+    return fail(SA_ERR_INVALID_ARG, "sa_sparse_attn_bwd_linear_mix: topk must be in [0, N/block]");
+  if (topk > 0 && !block_idx) return fail(SA_ERR_INVALID_ARG, "sa_sparse_attn_bwd_linear_mix: block_idx is required");
+  if (nb > kMaxAttnBlocks) return fail(SA_ERR_UNSUPPORTED, "sa_sparse_attn_bwd_linear_mix: at most 4096 blocks per head");
+  const sa_block_stats st = *stats;
+  if (!st.htot || !st.ztot || !st.zrelu)
+    return fail(SA_ERR_INVALID_ARG, "sa_sparse_attn_bwd_linear_mix: needs stats->htot, ztot and zrelu");
+  const size_t need = lin_workspace_bytes(shape, topk);
+  if (!workspace || workspace_bytes < need)
+    return fail(SA_ERR_WORKSPACE,
+                "sa_sparse_attn_bwd_linear_mix: workspace missing or smaller than its workspace size");
+  const void* ptrs[] = {Q, K, V, O, dO, dQ, dK, dV, workspace, block_idx, alpha, st.htot, st.ztot, st.zrelu};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p))
+      return fail(SA_ERR_ALIGNMENT, "sa_sparse_attn_bwd_linear_mix: pointers must be 16-byte aligned");
+  cudaStream_t s = as_stream(stream);
+  char* ws = static_cast<char*>(workspace);
+  const BwdLayout L = bwd_layout(shape, topk);
+  int32_t* offs = reinterpret_cast<int32_t*>(ws + L.offs_off);
+  int32_t* list = reinterpret_cast<int32_t*>(ws + L.list_off);
+  if (topk > 0) {
+    r = launch_transpose(block_idx, nb, topk, offs, list, shape.B * shape.H, s);
+    if (r != SA_OK) return r;
+  } else if (cudaMemsetAsync(offs, 0, (size_t)shape.B * shape.H * (nb + 1) * sizeof(int32_t), s) != cudaSuccess) {
+    return launch_status("cudaMemsetAsync(bwd offsets)");
+  }
+  auto a256 = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  return bwd_linear_mix(Q, K, V, O, dO, shape, block_idx, topk, alpha, st, scale, dQ, dK, dV,
+                        reinterpret_cast<float*>(ws + L.lse_off), reinterpret_cast<float*>(ws + L.delta_off), offs,
+                        list, reinterpret_cast<float*>(ws + L.part_off), ws + a256(L.total), s);
+}

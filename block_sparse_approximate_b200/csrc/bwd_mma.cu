@@ -532,7 +532,7 @@ sa_status bwd_tc_launch(const void* Q, const void* K, const void* V, const void*
                         const sa_shape& s, const int32_t* block_idx, int topk, bool zo, const sa_block_stats& st,
                         float scale, float* dQ, float* dK, float* dV, const float* lse_in, float* lse2,
                         float* delta, const int32_t* offs, const int32_t* list, float* part, cudaStream_t stream,
-                        const BwdFirstOrder* fo) {
+                        const BwdTailTerms* fo) {
   using bf = __nv_bfloat16;
   const int nb = s.N / BLK;
   const bf* q = static_cast<const bf*>(Q);
@@ -582,7 +582,7 @@ sa_status bwd_tc_launch(const void* Q, const void* K, const void* V, const void*
 sa_status bwd_tc(const void* Q, const void* K, const void* V, const void* O, const void* dO, const sa_shape& s,
                  const int32_t* block_idx, int topk, bool zo, const sa_block_stats& st, float scale, float* dQ,
                  float* dK, float* dV, const float* lse_in, float* lse2, float* delta, const int32_t* offs,
-                 const int32_t* list, float* part, cudaStream_t stream, const BwdFirstOrder* fo) {
+                 const int32_t* list, float* part, cudaStream_t stream, const BwdTailTerms* fo) {
   if (s.block == 128)
     return bwd_tc_launch<128>(Q, K, V, O, dO, s, block_idx, topk, zo, st, scale, dQ, dK, dV, lse_in, lse2, delta,
                               offs, list, part, stream, fo);

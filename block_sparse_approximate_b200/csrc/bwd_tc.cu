@@ -19,6 +19,7 @@
 // when the forward's log-sum-exp is given); pass 2
 // forms S again, dP = dO Vᵀ, writes dS (bf16) into the S columns, and
 // accumulates dQ += dS · K with dS read from TMEM.
+// SLA2's linear mix (delta_in non-null): the softmax branch's δ is given.
 // PISA's first-order tail (doff non-null): a pseudo-key's value seen by row t
 // is v̄_j + f_t / B (f_t = s H̄ᵀ q_t), so the centroid tiles take
 // dS = P (dP − δ + doff_t) with doff_t = dO_t·f_t / B; the kernel also writes
@@ -105,7 +106,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                  const int32_t* __restrict__ block_idx, int N, int topk, int zo, float scale,
                  const float* __restrict__ lse_in, float* __restrict__ lse2, float* __restrict__ delta,
                  float* __restrict__ dQ, const float* __restrict__ doff, float* __restrict__ delta_c,
-                 float* __restrict__ lam, size_t lam_stride) {
+                 float* __restrict__ lam, size_t lam_stride, const float* __restrict__ delta_in) {
   using L = Lay;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -290,9 +291,12 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     const size_t row = (size_t)bh * N + (size_t)i * TB + r;
     const uint32_t lrow = tbase + ((uint32_t)(wq * 32) << 16);
     const float scale2 = scale * kLog2e;
-    // δ = dO · O over the row's 128 channels (both groups, from the stored bf16 output)
+    // δ = dO · O over the row's 128 channels (both groups, from the stored bf16
+    // output), or the caller's δ (SLA2's linear mix: the softmax branch's own)
     float dl = 0.f;
-    {
+    if (delta_in) {
+      dl = delta_in[row];
+    } else {
       const uint4* go = reinterpret_cast<const uint4*>(dO + row * TD);
       const uint4* oo = reinterpret_cast<const uint4*>(O + row * TD);
 #pragma unroll 4
@@ -800,7 +804,7 @@ bwd_cent_reduce_kernel(float* __restrict__ part, int nb, int nsplit) {
 sa_status bwd_dq_tc(const void* Q, const void* K, const void* V, const void* O, const void* dO, const sa_shape& s,
                     const int32_t* block_idx, int topk, bool zo, const sa_block_stats& st, float scale,
                     const float* lse_in, float* lse2, float* delta, float* dQ, cudaStream_t stream,
-                    const BwdFirstOrder* fo) {
+                    const BwdTailTerms* fo) {
   const int nb = s.N / TB;
   const uint64_t BH = (uint64_t)s.B * s.H;
   alignas(64) CUtensorMap mq, mg, mk, mv, mkb, mvb;
@@ -821,7 +825,7 @@ sa_status bwd_dq_tc(const void* Q, const void* K, const void* V, const void* O, 
   bwd_dq_tc_kernel<<<dim3(nb, (unsigned)BH), kThreads, smem, stream>>>(
       mq, mg, mk, mv, mkb, mvb, static_cast<const __nv_bfloat16*>(O), static_cast<const __nv_bfloat16*>(dO),
       block_idx, s.N, topk, zo ? 1 : 0, scale, lse_in, lse2, delta, dQ, fo ? fo->doff : nullptr,
-      fo ? fo->delta_c : nullptr, fo ? fo->lam : nullptr, (size_t)BH * s.N);
+      fo ? fo->delta_c : nullptr, fo ? fo->lam : nullptr, (size_t)BH * s.N, fo ? fo->delta_in : nullptr);
   return launch_status("bwd_dq_tc_kernel");
 }
 

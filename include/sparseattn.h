@@ -246,6 +246,36 @@ sa_status sa_sparse_attn_bwd_lse(const void* Q, const void* K, const void* V, co
                                  const sa_block_stats* stats, float scale, float* dQ, float* dK,
                                  float* dV, void* workspace, size_t workspace_bytes, void* stream);
 
+/* Bytes of workspace sa_sparse_attn_bwd_linear_mix needs (0 on bad arguments
+ * or a shape it does not run: d and block must be 128). */
+size_t sa_sparse_attn_bwd_linear_mix_workspace_size(sa_shape shape, int32_t topk);
+
+/* Backward of sa_sparse_attn_fwd with SA_TAIL_LINEAR_MIX [SLA2 §2A; SALAD §2]:
+ * O = α⊙O_s + (1−α)⊙O_l, O_s the softmax attention over the selected blocks
+ * and O_l = φ(q)ᵀ H_U / (φ(q)·z_U + 1e-6) the ReLU linear attention over the
+ * unselected ones (H_U = H_tot − Σ_{j∈S} h_j, z_U likewise; O_l = 0 when
+ * every block is selected).  With g = dO_t and g_l = (1−α)⊙g:
+ *   softmax branch: the DROP backward of the cotangent α⊙g, its
+ *     δ_s = (α⊙g)·O_s = g·O − g_l·O_l formed from O and the recomputed O_l;
+ *   linear branch: dnum = g_l / den, dden = −(g_l·O_l) / den,
+ *     dq += 1[q > 0] ⊙ (H_U dnum + z_U dden), and per key block j, with
+ *     dh_j = Σ_{query blocks i not selecting j} Σ_{t∈i} φ(q_t) dnumᵀ (and dz_j
+ *     likewise), dk_n += 1[k_n > 0] ⊙ (dh_j v_n + dz_j), dv_n += dh_jᵀ φ(k_n).
+ * Q, K, V, O, dO: bf16 [B,H,N,d] (O the forward's output); block_idx, topk,
+ * alpha [H,d] and stats (htot, ztot, zrelu) as given to the forward.
+ * dQ, dK, dV: float32 [B,H,N,d], overwritten.  workspace: at least
+ * sa_sparse_attn_bwd_linear_mix_workspace_size() bytes, 16-byte aligned (it
+ * holds the per-block h_j and per-query-block dH_U as bf16 d x d tiles).
+ * bf16, d = 128, block 128 only (the softmax branch runs on the tcgen05
+ * backward, the linear branch on mma.sync); sums run in a fixed order.
+ * Errors: SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED, SA_ERR_ALIGNMENT,
+ *         SA_ERR_WORKSPACE. */
+sa_status sa_sparse_attn_bwd_linear_mix(const void* Q, const void* K, const void* V, const void* O,
+                                        const void* dO, sa_dtype dtype, sa_shape shape,
+                                        const int32_t* block_idx, int32_t topk, const float* alpha,
+                                        const sa_block_stats* stats, float scale, float* dQ, float* dK,
+                                        float* dV, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Per-block e4m3 quantisation [SLA2 §2C, low-precision sparse branch]:
  * X: bf16 [BH][N][d] (BH = batch x heads); codes: uint8 [BH][N][d] e4m3fn bit
  * patterns; scales: float [BH][ceil(N/block)] with σ = absmax/448 of each block

@@ -565,6 +565,34 @@ def test_backward_of_the_e4m3_forward_straight_through(lib):
     assert torch.equal(g8[2], ge[2])
 
 
+@pytest.mark.parametrize("B,H,nb,k", [(1, 2, 9, 3), (1, 1, 37, 5), (1, 2, 20, 0), (1, 2, 8, 8), (2, 3, 10, 3)])
+def test_backward_linear_mix(lib, B, H, nb, k):
+    # SLA2's mixture: α per head and channel in (0.2, 0.9); the linear branch's
+    # share of the gradients checked against the drop backward of α⊙dO
+    block, d = 128, 128
+    N = nb * block
+    Q, K, V = _gauss(B, H, N, d, torch.bfloat16, 150 + nb + k)
+    g = torch.Generator(device=DEV)
+    g.manual_seed(151)
+    dO = torch.randn(B, H, N, d, generator=g, device=DEV).to(torch.bfloat16)
+    alpha = (0.2 + 0.7 * torch.rand(H, d, generator=g, device=DEV)).contiguous()
+    s = 1 / math.sqrt(d)
+    st = bd.block_pool(Q, K, V, block, linear=True)
+    idx, _ = bd.route(st, (B, H, N, d, block), "dot", k)
+    O = bd.sparse_attn_fwd(Q, K, V, idx, block, "linear_mix", st, s, alpha=alpha)
+    grads = bd.sparse_attn_bwd_linear_mix(Q, K, V, O, dO, idx, block, alpha, st, s)
+    torch.cuda.synchronize()
+    assert_no_device_error()
+    args = (np64(Q), np64(K), np64(V), idx.cpu().numpy(), block)
+    ref = oracle.sparse_attention_backward(*args, "linear_mix", s, np64(dO), alpha=np64(alpha))
+    drop = oracle.sparse_attention_backward(*args, "drop", s, np64(dO) * np64(alpha)[None, :, None, :])
+    for got, r, name in zip(grads, ref, ("dQ", "dK", "dV")):
+        sc = max(1.0, float(np.abs(r).max()))
+        assert_tol(np64(got), r, (2e-2 * sc, 2e-3), f"linear-mix backward {name}")
+    if k < nb:
+        assert max(float(np.abs(r - z).max()) for r, z in zip(ref, drop)) > 0.05
+
+
 def test_backward_first_order_is_rejected_off_the_tensor_cores(lib):
     Q, K, V = _gauss(1, 1, 512, 64, torch.float32, 132)
     st = bd.block_pool(Q, K, V, 64, first_order=True)
