@@ -139,6 +139,10 @@ __device__ __forceinline__ void cp_async_wait() {
 // serialization may start while its predecessor drains; it waits here
 // before touching anything the predecessor writes (a no-op otherwise).
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Lets the next launch on the stream start its CTAs (up to their pdl_wait())
+// once every CTA of this grid has passed here; all of them are then resident,
+// so the waiting successors cannot hold back a CTA of this grid.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 __device__ __forceinline__ uint32_t pack2bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -491,49 +495,77 @@ decode_stats_kernel(const __nv_bfloat16* __restrict__ q, const TS* __restrict__ 
 
 // ---- B. top-k ------------------------------------------------------------
 // Radix select over the 32-bit order keys of the scores (higher score =
-// smaller key): four 8-bit histogram passes find the key T of the k-th best
-// block; every block with a smaller key is kept, and of the blocks whose key
-// equals T the ones with the smallest indices fill the remaining places.  The
-// kept indices are emitted in ascending order from a bitmap.
+// smaller key).  The keys of one row share their high bits (the scores span
+// a narrow range), so the select starts below the highest bit in which the
+// row's smallest and largest keys differ, and takes 8-bit digits from there:
+// each pass histograms the digit of the keys that still match the prefix
+// found so far, and the bin holding the k-th key extends the prefix.  Once
+// that bin holds exactly the places left, every key in it is kept and the
+// lower bits do not matter (usually after two passes); otherwise the passes
+// run down to bit 0 and, of the keys equal to the k-th, the smallest indices
+// fill the places left.  The kept indices are emitted in ascending order from
+// a bitmap.
 constexpr int kTopkKPT = kMaxRouteBlocks / kDecThreads;   // keys per thread
 
 __global__ void __launch_bounds__(kDecThreads)
 decode_topk_kernel(const float* __restrict__ scores, int nb, int topk, int32_t* __restrict__ idx) {
   pdl_wait();
+  pdl_trigger();
   const int pair = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   __shared__ unsigned hist[256];
   __shared__ uint32_t bits[kMaxRouteBlocks / 32];
-  __shared__ unsigned sh_prefix, sh_rank, sh_eq;
+  __shared__ unsigned sh_prefix, sh_rank, sh_cnt;
+  __shared__ unsigned sh_min[kDecWarps], sh_max[kDecWarps];
   const float* sc = scores + (size_t)pair * nb;
   int32_t* out = idx + (size_t)pair * topk;
   const int nwords = (nb + 31) / 32;
 
   uint32_t key[kTopkKPT];
+  unsigned kmin = 0xffffffffu, kmax = 0u;
 #pragma unroll
   for (int e = 0; e < kTopkKPT; ++e) {
     const int j = tid + e * kDecThreads;
     key[e] = j < nb ? ~order_key(sc[j]) : 0xffffffffu;
+    if (j < nb) {
+      kmin = min(kmin, key[e]);
+      kmax = max(kmax, key[e]);
+    }
   }
   for (int x = tid; x < nwords; x += kDecThreads) bits[x] = 0u;
-  if (tid == 0) {
-    sh_prefix = 0u;
-    sh_rank = (unsigned)topk;
+  kmin = __reduce_min_sync(0xffffffffu, kmin);
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
+  if (lane == 0) {
+    sh_min[warp] = kmin;
+    sh_max[warp] = kmax;
   }
-  unsigned mask = 0u;
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
+  __syncthreads();
+  kmin = sh_min[0];
+  kmax = sh_max[0];
+#pragma unroll
+  for (int w = 1; w < kDecWarps; ++w) {
+    kmin = min(kmin, sh_min[w]);
+    kmax = max(kmax, sh_max[w]);
+  }
+  // bits above `hi` are common to every key of the row
+  const unsigned diff = kmin ^ kmax;
+  int hi = diff ? 31 - __clz(diff) : -1;
+  unsigned mask = diff == 0u ? 0xffffffffu : (hi >= 31 ? 0u : ~((2u << hi) - 1u));
+  unsigned prefix = kmin & mask;
+  unsigned rank = (unsigned)topk, cnt = (unsigned)nb;
+  while (hi >= 0 && cnt != rank) {
+    const int lo = max(hi - 7, 0);
+    const unsigned dmask = (2u << (hi - lo)) - 1u;      // the digit's bits, shifted down
     for (int x = tid; x < 256; x += kDecThreads) hist[x] = 0u;
     __syncthreads();
-    const unsigned prefix = sh_prefix;
 #pragma unroll
     for (int e = 0; e < kTopkKPT; ++e) {
       const int j = tid + e * kDecThreads;
-      if (j < nb && (key[e] & mask) == prefix) atomicAdd(&hist[(key[e] >> shift) & 255u], 1u);
+      if (j < nb && (key[e] & mask) == prefix) atomicAdd(&hist[(key[e] >> lo) & dmask], 1u);
     }
     __syncthreads();
     if (warp == 0) {
-      // bucket holding the rank-th smallest key among those matching prefix
+      // the bin holding the rank-th smallest key among those matching prefix
       unsigned c[8], tot = 0;
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
@@ -546,50 +578,45 @@ decode_topk_kernel(const float* __restrict__ scores, int nb, int topk, int32_t* 
         const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= o) incl += y;
       }
-      const unsigned rank = sh_rank;
       const unsigned excl = incl - tot;
       if (excl < rank && rank <= incl) {
         unsigned run = excl;
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           if (run < rank && rank <= run + c[e]) {
-            sh_prefix = prefix | ((unsigned)(lane * 8 + e) << shift);
+            sh_prefix = prefix | ((unsigned)(lane * 8 + e) << lo);
             sh_rank = rank - run;
+            sh_cnt = c[e];
           }
           run += c[e];
         }
       }
     }
-    mask |= 255u << shift;
     __syncthreads();
+    prefix = sh_prefix;
+    rank = sh_rank;
+    cnt = sh_cnt;
+    mask |= dmask << lo;
+    hi = lo - 1;
   }
-  const unsigned T = sh_prefix;         // key of the k-th best block
-  const unsigned need_eq = sh_rank;     // how many blocks with key T are kept
-  if (tid == 0) sh_eq = 0u;
-  __syncthreads();
-  unsigned my_eq = 0;
+  // keep every key whose determined bits are below the prefix, and of the
+  // keys matching it: all of them when they fill the places left exactly,
+  // else (all bits determined: ties) the smallest indices
+  const bool all_eq = cnt == rank;
 #pragma unroll
   for (int e = 0; e < kTopkKPT; ++e) {
     const int j = tid + e * kDecThreads;
     if (j < nb) {
-      if (key[e] < T) atomicOr(&bits[j >> 5], 1u << (j & 31));
-      else if (key[e] == T) ++my_eq;
+      const unsigned km = key[e] & mask;
+      if (km < prefix || (all_eq && km == prefix)) atomicOr(&bits[j >> 5], 1u << (j & 31));
     }
   }
-  if (my_eq) atomicAdd(&sh_eq, my_eq);
-  __syncthreads();
-  if (sh_eq == need_eq) {
-#pragma unroll
-    for (int e = 0; e < kTopkKPT; ++e) {
-      const int j = tid + e * kDecThreads;
-      if (j < nb && key[e] == T) atomicOr(&bits[j >> 5], 1u << (j & 31));
-    }
-  } else if (warp == 0) {
-    // ties at the threshold: the smallest indices first
-    unsigned left = need_eq;
+  if (!all_eq && warp == 0) {
+    // ties at the threshold key (mask covers every bit): the smallest indices first
+    unsigned left = rank;
     for (int j0 = 0; j0 < nb && left > 0; j0 += 32) {
       const int j = j0 + lane;
-      const bool eq = j < nb && ~order_key(sc[j]) == T;
+      const bool eq = j < nb && ~order_key(sc[j]) == prefix;
       const unsigned bal = __ballot_sync(0xffffffffu, eq);
       const unsigned before = __popc(bal & ((1u << lane) - 1u));
       if (eq && before < left) atomicOr(&bits[j >> 5], 1u << (j & 31));
@@ -603,14 +630,14 @@ decode_topk_kernel(const float* __restrict__ scores, int nb, int topk, int32_t* 
     for (int x0 = 0; x0 < nwords; x0 += 32) {
       const int x = x0 + lane;
       const uint32_t word = x < nwords ? bits[x] : 0u;
-      const int cnt = __popc(word);
-      int pre = cnt;
+      const int cnt_w = __popc(word);
+      int pre = cnt_w;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int y = __shfl_up_sync(0xffffffffu, pre, o);
         if (lane >= o) pre += y;
       }
-      int pos = base + pre - cnt;
+      int pos = base + pre - cnt_w;
       uint32_t m = word;
       while (m) {
         const int bpos = __ffs(m) - 1;
@@ -671,6 +698,7 @@ decode_exact_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
                     const int32_t* __restrict__ idx, int topk, float scale, int nsegC, int npairs,
                     float* __restrict__ partc, float* __restrict__ partr) {
   pdl_wait();
+  pdl_trigger();
   constexpr int CH = D / 8;                         // 16-byte chunks per bf16 row
   constexpr int NT = D / 8;                         // n-tiles of 8 channels
   constexpr int KS = D / 16;                        // k steps of 16 channels
@@ -938,6 +966,254 @@ decode_exact_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
   cp_async_wait<0>();
 }
 
+// ---- A'. statistics pass on the tensor cores (bf16 statistics) ------------
+// The same outputs as decode_stats_kernel for bf16 kmean, kvar and value
+// means.  A stage is 64 blocks of the three arrays, staged by cp.async
+// (16-byte chunks of row r at chunk ^ (r & 7), as the exact pass stages K and
+// V) into a ring of four, so three stages (144 KB) are in flight while one is
+// reduced; a segment is two stages (128 blocks, the segments of
+// decode_stats_kernel).  Warp w takes blocks [8w, 8w + 8) of a stage.  The dot
+// products are mma.sync m16n8k16 contractions with the group's G <= 8 query
+// heads as the MMA rows and the warp's 8 blocks as the columns:
+// s log2e q·k̄_j (q and k̄ in bf16: exact products), and ½ s² Σ_c q_c² var_jc
+// with ½ s² q² split into two bf16 terms (hi + lo: q² of a bf16 q has 16
+// significant bits, so the split is exact).  The zero-order term of every
+// block enters the warp's online softmax per head, its value-mean product
+// P·v̄ on the tensor cores again (P in bf16, as the exact pass rounds its P;
+// the warp's 8 blocks fill the MMA's first 8 k rows, the other 8 carry P = 0).
+// At the end of a segment the warps' states are merged into one partial
+// state per head as in decode_stats_kernel.
+constexpr int kStageBlocksM = 64;
+constexpr int kSegM = (kStageBlocksA * kSegA) / kStageBlocksM;   // stages per segment (2)
+constexpr int kRingM = 4;
+
+template <int D, bool ZT>
+__global__ void __launch_bounds__(kDecThreads, 1)
+decode_stats_mma_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kmean,
+                        const __nv_bfloat16* __restrict__ kvar, const __nv_bfloat16* __restrict__ vmean, int Hq,
+                        int Hkv, int nb, int blk, float scale, int nsegA, int npairs, float* __restrict__ scores,
+                        float* __restrict__ parta) {
+  constexpr int CH = D / 8;                         // 16-byte chunks per bf16 row
+  constexpr int NT = D / 8;                         // n-tiles of 8 channels
+  constexpr int KS = D / 16;                        // k steps of 16 channels
+  constexpr uint32_t kRowB = D * 2;
+  constexpr uint32_t kArrB = kStageBlocksM * kRowB;
+  constexpr int NARR = ZT ? 3 : 2;
+  constexpr uint32_t kStageB = NARR * kArrB;
+  extern __shared__ __align__(16) uint8_t dsm[];
+  const int g = Hq / Hkv;
+  float* mg = reinterpret_cast<float*>(dsm);                         // [8 warps][g][D + 2] merge
+  uint8_t* ring = dsm + ((sizeof(float) * kDecWarps * g * (D + 2) + 127) & ~(size_t)127);
+  const uint32_t ring_s = (uint32_t)__cvta_generic_to_shared(ring);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int total_segs = npairs * nsegA;
+  const float scale2 = scale * kLog2e;
+  const float bias2 = log2f((float)blk);
+  const int hrow = lane >> 2;                       // MMA row of this thread = query head
+  const bool hvalid = hrow < g;
+  const int nstage_pair = (nb + kStageBlocksM - 1) / kStageBlocksM;
+
+  auto seg_of = [&](int k) { return (int)blockIdx.x + k * (int)gridDim.x; };
+  auto stages_in = [&](int seg) { return min(kSegM, nstage_pair - (seg % nsegA) * kSegM); };
+  // stage `sub` of segment `seg` into ring slot `slot`; rows past the pair's
+  // last block are zero-filled
+  auto issue = [&](int seg, int sub, int slot) {
+    const int pair = seg / nsegA, j0 = ((seg % nsegA) * kSegM + sub) * kStageBlocksM;
+    const int nrow = min(kStageBlocksM, nb - j0);
+    const size_t base = ((size_t)pair * nb + j0) * D;
+    uint8_t* dst = ring + slot * kStageB;
+    for (int o = tid; o < kStageBlocksM * CH; o += kDecThreads) {
+      const int r = o / CH, c = o % CH;
+      const uint32_t sw = r * kRowB + ((c ^ (r & 7)) << 4);
+      const size_t so = base + (size_t)(r < nrow ? r : 0) * D + 8 * c;
+      const uint32_t nbytes = r < nrow ? 16u : 0u;
+      cp_async16z(dst + sw, kmean + so, nbytes);
+      cp_async16z(dst + kArrB + sw, kvar + so, nbytes);
+      if (ZT) cp_async16z(dst + 2 * kArrB + sw, vmean + so, nbytes);
+    }
+  };
+  if (seg_of(0) >= total_segs) return;
+  int pf_k = 0, pf_sub = 0, pf_slot = 0;
+  auto prefetch = [&]() {
+    if (seg_of(pf_k) < total_segs) {
+      issue(seg_of(pf_k), pf_sub, pf_slot);
+      if (++pf_sub >= stages_in(seg_of(pf_k))) {
+        pf_sub = 0;
+        ++pf_k;
+      }
+    }
+    cp_async_commit();
+    pf_slot = (pf_slot + 1) % kRingM;
+  };
+  for (int r = 0; r < kRingM - 1; ++r) prefetch();
+
+  uint32_t qa0[KS], qa2[KS];                  // q (rows = heads)
+  uint32_t wh0[KS], wh2[KS], wl0[KS], wl2[KS];   // ½ s² q², hi and lo bf16 parts
+  float m_run = -INFINITY, l_run = 0.f;       // the warp's zero-order state of head hrow
+  float o[ZT ? NT : 1][2];
+  int cur_pair = -1, cur_k = 0, cur_sub = 0, slot = 0;
+  while (seg_of(cur_k) < total_segs) {
+    const int seg = seg_of(cur_k);
+    const int pair = seg / nsegA, sseg = seg % nsegA;
+    const int b = pair / Hkv, kh = pair % Hkv;
+    const int j0 = (sseg * kSegM + cur_sub) * kStageBlocksM;
+    if (pair != cur_pair) {
+      const __nv_bfloat16* qrow = q + ((size_t)b * Hq + kh * g + (hvalid ? hrow : 0)) * D;
+#pragma unroll
+      for (int kk = 0; kk < KS; ++kk) {
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const int c0 = 16 * kk + 8 * half + 2 * (lane & 3);
+          const uint32_t raw = *reinterpret_cast<const uint32_t*>(qrow + c0);
+          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw));
+          const float w0 = 0.5f * scale * scale * f.x * f.x, w1 = 0.5f * scale * scale * f.y * f.y;
+          const __nv_bfloat162 hi = __floats2bfloat162_rn(w0, w1);
+          const float2 hf = __bfloat1622float2(hi);
+          const uint32_t hiu = *reinterpret_cast<const uint32_t*>(&hi);
+          const uint32_t lou = pack2bf16(w0 - hf.x, w1 - hf.y);
+          if (half == 0) {
+            qa0[kk] = hvalid ? raw : 0u;
+            wh0[kk] = hvalid ? hiu : 0u;
+            wl0[kk] = hvalid ? lou : 0u;
+          } else {
+            qa2[kk] = hvalid ? raw : 0u;
+            wh2[kk] = hvalid ? hiu : 0u;
+            wl2[kk] = hvalid ? lou : 0u;
+          }
+        }
+      }
+      cur_pair = pair;
+    }
+    if (ZT && cur_sub == 0) {
+      m_run = -INFINITY;
+      l_run = 0.f;
+#pragma unroll
+      for (int nt = 0; nt < (ZT ? NT : 1); ++nt) o[nt][0] = o[nt][1] = 0.f;
+    }
+    prefetch();
+    cp_async_wait<kRingM - 1>();
+    __syncthreads();
+
+    const uint32_t kbase = ring_s + slot * kStageB, vbase = kbase + 2 * kArrB;
+    const int nrow = min(kStageBlocksM, nb - j0);
+    const int tb = 8 * warp;
+    const int r0 = tb + (lane & 7);             // the row this lane addresses
+    // four independent accumulator chains (even / odd k steps; hi / lo of ½ s² q²)
+    float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};   // q·k̄
+    float ta[4] = {0.f, 0.f, 0.f, 0.f}, tb4[4] = {0.f, 0.f, 0.f, 0.f};  // ½ s² Σ q² var
+#pragma unroll
+    for (int kp = 0; kp < KS / 2; ++kp) {
+      uint32_t kf[4], vf[4];
+      const int chunk = 4 * kp + (lane >> 3);
+      ldsm_x4(kf, kbase + r0 * kRowB + ((chunk ^ (r0 & 7)) << 4));
+      ldsm_x4(vf, kbase + kArrB + r0 * kRowB + ((chunk ^ (r0 & 7)) << 4));
+      mma16816_full(sa, qa0[2 * kp], qa2[2 * kp], kf[0], kf[1]);
+      mma16816_full(sb, qa0[2 * kp + 1], qa2[2 * kp + 1], kf[2], kf[3]);
+      mma16816_full(ta, wh0[2 * kp], wh2[2 * kp], vf[0], vf[1]);
+      mma16816_full(tb4, wh0[2 * kp + 1], wh2[2 * kp + 1], vf[2], vf[3]);
+      mma16816_full(ta, wl0[2 * kp], wl2[2 * kp], vf[0], vf[1]);
+      mma16816_full(tb4, wl0[2 * kp + 1], wl2[2 * kp + 1], vf[2], vf[3]);
+    }
+    // the lane's two (head hrow, block) values: blocks tj, tj + 1
+    const int tj = tb + 2 * (lane & 3);
+    float x[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const bool live = hvalid && tj + e < nrow;
+      const float d1 = (sa[e] + sb[e]) * scale2;   // s log2e q·k̄
+      const float d2 = ta[e] + tb4[e];             // ½ s² Σ q² var
+      // group score of the block, ln Σ_h e^{s q_h·k̄}(1 + d2_h) (the logsumexp
+      // of the heads' log scores), in log2 units over the lanes 4 apart
+      const float a = live ? d1 : -INFINITY;
+      float mx = a;
+#pragma unroll
+      for (int o2 = 4; o2 < 32; o2 <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o2));
+      float se = live ? fast_exp2(a - mx) * (1.0f + d2) : 0.f;
+#pragma unroll
+      for (int o2 = 4; o2 < 32; o2 <<= 1) se += __shfl_xor_sync(0xffffffffu, se, o2);
+      if (hrow == 0 && tj + e < nrow) scores[(size_t)pair * nb + j0 + tj + e] = (mx + __log2f(se)) * kLn2;
+      x[e] = live ? d1 + bias2 : -INFINITY;   // log2 weight of the block's pseudo-key
+    }
+    if (ZT) {
+      // the warp's 8 blocks of head hrow: max over the row's four lanes
+      float tmax = fmaxf(x[0], x[1]);
+      tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 1));
+      tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 2));
+      const float m_new = fmaxf(m_run, tmax);
+      const float corr = m_run == -INFINITY ? 0.f : fast_exp2(m_run - m_new);
+      const float p0 = x[0] != -INFINITY ? fast_exp2(x[0] - m_new) : 0.f;
+      const float p1 = x[1] != -INFINITY ? fast_exp2(x[1] - m_new) : 0.f;
+      l_run = l_run * corr + (p0 + p1);
+      m_run = m_new;
+      const uint32_t pa0 = pack2bf16(p0, p1);
+#pragma unroll
+      for (int nq = 0; nq < NT / 4; ++nq) {
+        uint32_t vv[4];
+        const int chunk = 4 * nq + (lane >> 3);
+        ldsm_x4_t(vv, vbase + r0 * kRowB + ((chunk ^ (r0 & 7)) << 4));
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float* oo = o[ZT ? 4 * nq + e : 0];
+          oo[0] *= corr;
+          oo[1] *= corr;
+          // k rows 8-15 carry P = 0 (their B operand repeats rows 0-7)
+          mma16816_top(o[ZT ? 4 * nq + e : 0], pa0, 0u, vv[e], vv[e]);
+        }
+      }
+    }
+    slot = (slot + 1) % kRingM;
+    const bool seg_end = ++cur_sub >= stages_in(seg);
+    if (ZT && seg_end) {
+      // the warp's state of head hrow for this segment, then the merge
+      float lq = l_run;
+      lq += __shfl_xor_sync(0xffffffffu, lq, 1);
+      lq += __shfl_xor_sync(0xffffffffu, lq, 2);
+      if (hvalid) {
+        float* mw = mg + ((size_t)warp * g + hrow) * (D + 2);
+        if ((lane & 3) == 0) {
+          mw[0] = m_run;
+          mw[1] = lq;
+        }
+#pragma unroll
+        for (int nt = 0; nt < (ZT ? NT : 1); ++nt) {
+          mw[2 + 8 * nt + 2 * (lane & 3)] = o[nt][0];
+          mw[2 + 8 * nt + 2 * (lane & 3) + 1] = o[nt][1];
+        }
+      }
+      __syncthreads();
+      for (int xi = tid; xi < g * D; xi += kDecThreads) {
+        const int hh = xi / D, c = xi % D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, mg[((size_t)w * g + hh) * (D + 2)]);
+        float Lm = 0.f, A = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll
+          for (int w = 0; w < kDecWarps; ++w) {
+            const float* mw = mg + ((size_t)w * g + hh) * (D + 2);
+            if (mw[0] == -INFINITY) continue;
+            const float f = fast_exp2(mw[0] - M);
+            Lm = fmaf(mw[1], f, Lm);
+            A = fmaf(mw[2 + c], f, A);
+          }
+        }
+        float* out = parta + (((size_t)b * Hq + kh * g + hh) * nsegA + sseg) * (D + 2);
+        if (c == 0) {
+          out[0] = M;
+          out[1] = Lm;
+        }
+        out[2 + c] = A;
+      }
+    }
+    __syncthreads();   // the slot is restaged by a later prefetch; the merge rows are free
+    if (seg_end) {
+      cur_sub = 0;
+      ++cur_k;
+    }
+  }
+  cp_async_wait<0>();
+}
+
 // ---- D. merge ------------------------------------------------------------
 // One CTA of D threads per (query head, sequence), thread = channel.  It
 // merges the statistics pass's partial states (the zero-order term of every
@@ -969,7 +1245,10 @@ decode_combine_kernel(const float* __restrict__ parta, int nsegA, const float* _
                       const TS* __restrict__ kmean, const TS* __restrict__ vrow, float vmul,
                       const float* __restrict__ sexp, const int32_t* __restrict__ idx, int topk, int nb, int blk,
                       float scale, int Hq, int Hkv, __nv_bfloat16* __restrict__ O) {
-  pdl_wait();
+  // Everything up to the pdl_wait() below comes from the earlier launches of
+  // the step (statistics pass, top-k), which had completed before the exact
+  // pass read the selection; only the exact pass's partial states (partc,
+  // partr) are read after it, so this prologue overlaps the exact pass's tail.
   constexpr int kT = kParts * D, kW = kT / 32;
   extern __shared__ __align__(16) float csm[];
   const int na = use_tail ? nsegA : 0, ns = na + nsegC;
@@ -989,7 +1268,7 @@ decode_combine_kernel(const float* __restrict__ parta, int nsegA, const float* _
   const float* pc = partc + ((size_t)b * Hq + h) * nsegC * (D + 2);
   const int pair = b * Hkv + h / (Hq / Hkv);
   auto part = [&](int sidx) { return sidx < na ? pa + (size_t)sidx * (D + 2) : pc + (size_t)(sidx - na) * (D + 2); };
-  for (int x = tid; x < ns; x += kT) {
+  for (int x = tid; x < na; x += kT) {
     const float* r = part(x);
     hm[x] = r[0];
     hl[x] = r[1];
@@ -1004,16 +1283,14 @@ decode_combine_kernel(const float* __restrict__ parta, int nsegA, const float* _
 #pragma unroll
   for (int e = 0; e < kPreP; ++e) {
     const int x = pt + kParts * e;
-    pv[e] = x < ns ? part(x)[2 + c] : 0.f;
+    pv[e] = x < na ? part(x)[2 + c] : 0.f;
   }
 #pragma unroll
   for (int e = 0; e < kPreV; ++e) {
     const int si = pt + kParts * e;
     vv[e] = si < nsel ? ld_stat(vrow + ((size_t)pair * nb + jsel[si]) * D + c) : 0.f;
   }
-  float M = -INFINITY;
-  for (int x = 0; x < ns; ++x) M = fmaxf(M, hm[x]);
-  if (subtract && M != -INFINITY) {
+  if (subtract) {
     // s log2e q·k̄_j + log2 B of the selected blocks: a warp per block, the
     // rows of four blocks in flight at once
     const float scale2 = scale * kLog2e, bias2 = log2f((float)blk);
@@ -1039,6 +1316,20 @@ decode_combine_kernel(const float* __restrict__ parta, int nsegA, const float* _
       }
     }
   }
+  pdl_wait();   // the exact pass's partial states from here on
+  for (int x = na + tid; x < ns; x += kT) {
+    const float* r = part(x);
+    hm[x] = r[0];
+    hl[x] = r[1];
+  }
+#pragma unroll
+  for (int e = 0; e < kPreP; ++e) {
+    const int x = pt + kParts * e;
+    if (x >= na && x < ns) pv[e] = part(x)[2 + c];
+  }
+  __syncthreads();
+  float M = -INFINITY;
+  for (int x = 0; x < ns; ++x) M = fmaxf(M, hm[x]);
   for (int x = tid; x < ns; x += kT) hf[x] = (M == -INFINITY || hm[x] == -INFINITY) ? 0.f : fast_exp2(hm[x] - M);
   __syncthreads();
   float L = 0.f, A = 0.f;
@@ -1195,7 +1486,18 @@ sa_status launch_decode(const void* q, const void* Kc, const void* Vc, const sa_
       r0 = launch_status("decode_stats_kernel");
     };
     const bool zt = tail == SA_TAIL_ZERO_ORDER;
-    if (g == 1) run(zt ? decode_stats_kernel<D, 1, true, TS> : decode_stats_kernel<D, 1, false, TS>);
+    if constexpr (sizeof(TS) == 2) {
+      // bf16 statistics: the tensor-core statistics pass, one CTA per SM
+      const size_t smemM = ((sizeof(float) * kDecWarps * g * (D + 2) + 127) & ~(size_t)127) +
+                           (size_t)kRingM * (zt ? 3 : 2) * kStageBlocksM * D * 2;
+      const int gridM = (int)(segsA < sms ? segsA : sms);
+      auto kern = zt ? decode_stats_mma_kernel<D, true> : decode_stats_mma_kernel<D, false>;
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smemM) != cudaSuccess)
+        return launch_status("cudaFuncSetAttribute(decode_stats_mma_kernel)");
+      kern<<<gridM, kDecThreads, smemM, stream>>>(qb, ds.kmean, ds.kvar, ds.vrow, s.Hq, s.Hkv, nb, s.block, scale,
+                                                  L.nsegA, npairs, scores, parta);
+      r0 = launch_status("decode_stats_mma_kernel");
+    } else if (g == 1) run(zt ? decode_stats_kernel<D, 1, true, TS> : decode_stats_kernel<D, 1, false, TS>);
     else if (g == 2) run(zt ? decode_stats_kernel<D, 2, true, TS> : decode_stats_kernel<D, 2, false, TS>);
     else if (g == 4) run(zt ? decode_stats_kernel<D, 4, true, TS> : decode_stats_kernel<D, 4, false, TS>);
     else run(zt ? decode_stats_kernel<D, 8, true, TS> : decode_stats_kernel<D, 8, false, TS>);
