@@ -531,7 +531,7 @@ def time_sla2(steps: int = 2, warmup: int = 1):
     return out
 
 
-def time_backward_linear_mix(steps: int = 2, warmup: int = 1):
+def time_backward_linear_mix(steps: int = 2, warmup: int = 3):
     """Backward of the SLA2 mix workload (H=40, N=65536, linear mix):
     sa_sparse_attn_bwd_linear_mix on the step's inputs, output and a random dO.
     FLOPs: the softmax branch's drop backward recomputing its log-sum-exp,
@@ -606,7 +606,7 @@ def run_ours(args, world, rank, local):
         if rank == 0:
             print(json.dumps({"backward": time_backward(args.steps, args.warmup),
                               "backward_first_order": time_backward(args.steps, args.warmup, "video_dit_pisa"),
-                              "backward_linear_mix": time_backward_linear_mix(min(args.steps, 2), 1)}),
+                              "backward_linear_mix": time_backward_linear_mix(min(args.steps, 2), 3)}),
                   flush=True)
         return 0
     if args.only == "sfa":

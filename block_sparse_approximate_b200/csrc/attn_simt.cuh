@@ -57,12 +57,14 @@ bool bwd_tc_supports(sa_dtype dtype, const sa_shape& s, bool zo, const sa_block_
 // PISA's first-order tail: doff [B·H·N] = dO_t·f_t / B (input), delta_c
 // [B·H·N] the centroid keys' δ and lam [2][B·H·N] the two element-wise groups'
 // shares of λ_t (outputs); SLA2's linear mix: delta_in [B·H·N] the rows' δ of
-// the softmax branch, used instead of dO·O (input).
+// the softmax branch, used instead of dO·O (input), and dq_add: the dQ kernel
+// adds to dQ instead of overwriting it.
 struct BwdTailTerms {
   const float* doff;
   float* delta_c;
   float* lam;
   const float* delta_in;
+  bool dq_add;
 };
 sa_status bwd_tc(const void* Q, const void* K, const void* V, const void* O, const void* dO, const sa_shape& s,
                  const int32_t* block_idx, int topk, bool zo, const sa_block_stats& st, float scale, float* dQ,

@@ -201,7 +201,7 @@ sa_status bwd_first_order(const void* Q, const void* K, const void* V, const voi
   sa_status r = launch_status("fo_pre_kernel");
   if (r != SA_OK) return r;
   // the zero-order backward with the pseudo-keys' shifted δ
-  const BwdTailTerms fo{doff, delta_c, lam, nullptr};
+  const BwdTailTerms fo{doff, delta_c, lam, nullptr, false};
   r = bwd_tc(Q, K, V, O, dO, s, block_idx, topk, true, st, scale, dQ, dK, dV, lse_in, lse2, delta, offs, list, part,
              stream, &fo);
   if (r != SA_OK) return r;

@@ -16,9 +16,9 @@
 // Kernels (mma.sync products on the tiles of mma_tile.cuh):
 //   lin_hblk_kernel  h_j of every block, bf16 (the query blocks read
 //                    Σ_{j∈S_i} h_j from them, a head's h_j staying in L2);
-//   lin_q_kernel     per query block: H_U, O_l, then (pass 0) δ_s, α⊙g,
-//                    dH_U,i, dz_U,i, or (pass 1) the dq term, added to the
-//                    softmax branch's dQ;
+//   lin_q_kernel     per query block: H_U, O_l, then δ_s, α⊙g, dH_U,i,
+//                    dz_U,i and the dq term, written to dQ (the softmax
+//                    branch's dQ kernel then adds its own);
 //   lin_tot_kernel   Σ_i dH_U,i and Σ_i dz_U,i per head, in order;
 //   lin_kv_kernel    per key block: dh_j, dz_j and the dk, dv terms.
 // No atomics: every sum runs in a fixed order.
@@ -35,6 +35,64 @@ __device__ __forceinline__ uint32_t relu_bf16x2(uint32_t x) {
   const __nv_bfloat162 z = __float2bfloat162_rn(0.f);
   const __nv_bfloat162 r = __hmax2(*reinterpret_cast<const __nv_bfloat162*>(&x), z);
   return *reinterpret_cast<const uint32_t*>(&r);
+}
+
+// a[e] (e < 64) = init[e] − Σ_{s < n} M_{ids[s]}[64 tid + e]: the thread's 64
+// entries of a sum of bf16 d x d matrices M_i = base + i d², the indices in
+// shared memory; two matrices' loads in flight at a time
+__device__ __forceinline__ void sub_matrices(float (&a)[64], const float* init, const __nv_bfloat16* base,
+                                             const int* ids, int n, int tid) {
+#pragma unroll
+  for (int e = 0; e < 64; e += 4) {
+    const float4 x = *reinterpret_cast<const float4*>(init + 64 * tid + e);
+    a[e] = x.x;
+    a[e + 1] = x.y;
+    a[e + 2] = x.z;
+    a[e + 3] = x.w;
+  }
+  auto sub8 = [&](const uint4 (&x)[8]) {
+#pragma unroll
+    for (int e8 = 0; e8 < 8; ++e8) {
+      const uint32_t xv[4] = {x[e8].x, x[e8].y, x[e8].z, x[e8].w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xv[u]));
+        a[8 * e8 + 2 * u] -= f.x;
+        a[8 * e8 + 2 * u + 1] -= f.y;
+      }
+    }
+  };
+  int s = 0;
+  for (; s + 2 <= n; s += 2) {
+    const uint4* m0 = reinterpret_cast<const uint4*>(base + (size_t)ids[s] * FD * FD + 64 * tid);
+    const uint4* m1 = reinterpret_cast<const uint4*>(base + (size_t)ids[s + 1] * FD * FD + 64 * tid);
+    uint4 x0[8], x1[8];
+#pragma unroll
+    for (int e8 = 0; e8 < 8; ++e8) x0[e8] = m0[e8];
+#pragma unroll
+    for (int e8 = 0; e8 < 8; ++e8) x1[e8] = m1[e8];
+    sub8(x0);
+    sub8(x1);
+  }
+  if (s < n) {
+    const uint4* m0 = reinterpret_cast<const uint4*>(base + (size_t)ids[s] * FD * FD + 64 * tid);
+    uint4 x0[8];
+#pragma unroll
+    for (int e8 = 0; e8 < 8; ++e8) x0[e8] = m0[e8];
+    sub8(x0);
+  }
+}
+
+// the thread's 64 entries (row tid / 2, columns 64 (tid & 1) ..) as a bf16 tile
+__device__ __forceinline__ void store_entries(uint8_t* tile, const float (&a)[64], int tid) {
+  const int r = tid >> 1;
+#pragma unroll
+  for (int c8 = 0; c8 < 8; ++c8) {
+    const int c = 8 * (tid & 1) + c8;
+    *reinterpret_cast<uint4*>(tile + swz(r, c)) =
+        make_uint4(fo_pack2(a[8 * c8], a[8 * c8 + 1]), fo_pack2(a[8 * c8 + 2], a[8 * c8 + 3]),
+                   fo_pack2(a[8 * c8 + 4], a[8 * c8 + 5]), fo_pack2(a[8 * c8 + 6], a[8 * c8 + 7]));
+  }
 }
 
 // a bf16 [128][128] tile of rows with ReLU applied, into shared memory
@@ -81,10 +139,9 @@ lin_hblk_kernel(const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __rest
   store_acc_bf16(hblk + ((size_t)bh * nb + j) * FD * FD, acc, ra, rb, lane);
 }
 
-// Per query block i (PASS 0: δ_s, α⊙g, dH_U,i, dz_U,i; PASS 1: dQ += the
-// linear branch's dq).  H_U = H_tot − Σ_{j∈S_i} h_j is formed in fp32 and
-// used as a bf16 tile.
-template <int PASS>
+// Per query block i: H_U = H_tot − Σ_{j∈S_i} h_j (fp32, used as a bf16 tile),
+// O_l, then δ_s, α⊙g, dH_U,i, dz_U,i and the linear branch's dq, written to dQ
+// (the softmax branch's dQ kernel adds its own term afterwards).
 __global__ void __launch_bounds__(kFoThreads)
 lin_q_kernel(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ O,
              const __nv_bfloat16* __restrict__ dO, const float* __restrict__ alpha, int H, int N,
@@ -103,67 +160,39 @@ lin_q_kernel(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restric
   float* zu = reinterpret_cast<float*>(fsm + 3 * kTileB);   // z_U [d]
   float* den = zu + FD;                       // [128]
   float* dden = den + FT;                     // [128]
+  int* ids = reinterpret_cast<int*>(dden + FT);             // [topk] the selected blocks
   const float* al = alpha + (size_t)h * FD;
   const int ra = 16 * warp + (lane >> 2), rb = ra + 8;
   const bool lin = topk < nb;                 // U_i is not empty
   if (!lin) {
-    // O_l = 0: the softmax branch takes δ = g·O and the cotangent α⊙g; nothing else
-    if (PASS == 0) {
-      for (int r = warp; r < FT; r += kFoThreads / 32) {
-        const __nv_bfloat16* gr = dO + (row0 + r) * FD;
-        const __nv_bfloat16* orow = O + (row0 + r) * FD;
-        float d = 0.f;
-        for (int c = lane; c < FD; c += 32) {
-          const float g = __bfloat162float(gr[c]);
-          d = fmaf(g, __bfloat162float(orow[c]), d);
-          dOs[(row0 + r) * FD + c] = __float2bfloat16_rn(al[c] * g);
-        }
-        d = warp_sum(d);
-        if (lane == 0) delta_s[row0 + r] = d;
+    // O_l = 0: δ_s = g·O, the cotangent α⊙g, no linear-branch terms
+    for (int r = warp; r < FT; r += kFoThreads / 32) {
+      const __nv_bfloat16* gr = dO + (row0 + r) * FD;
+      const __nv_bfloat16* orow = O + (row0 + r) * FD;
+      float d = 0.f;
+      for (int c = lane; c < FD; c += 32) {
+        const float g = __bfloat162float(gr[c]);
+        d = fmaf(g, __bfloat162float(orow[c]), d);
+        dOs[(row0 + r) * FD + c] = __float2bfloat16_rn(al[c] * g);
+        dQ[(row0 + r) * FD + c] = 0.f;
       }
-      for (int x = tid; x < FD * FD; x += kFoThreads) dHU[((size_t)bh * nb + i) * FD * FD + x] = __float2bfloat16_rn(0.f);
-      for (int x = tid; x < FD; x += kFoThreads) dzU[((size_t)bh * nb + i) * FD + x] = 0.f;
+      d = warp_sum(d);
+      if (lane == 0) delta_s[row0 + r] = d;
     }
+    for (int x = tid; x < FD * FD; x += kFoThreads) dHU[((size_t)bh * nb + i) * FD * FD + x] = __float2bfloat16_rn(0.f);
+    for (int x = tid; x < FD; x += kFoThreads) dzU[((size_t)bh * nb + i) * FD + x] = 0.f;
     return;
   }
-  // ---- H_U and z_U: thread tid owns entries [64 tid, 64 tid + 64) of the d x d matrix
+  for (int x = tid; x < topk; x += kFoThreads) ids[x] = sel[x];
+  __syncthreads();
+  // ---- H_U and z_U
   {
     float a[64];
-    const float* ht = htot + (size_t)bh * FD * FD + 64 * tid;
-#pragma unroll
-    for (int e = 0; e < 64; e += 4) {
-      const float4 x = *reinterpret_cast<const float4*>(ht + e);
-      a[e] = x.x;
-      a[e + 1] = x.y;
-      a[e + 2] = x.z;
-      a[e + 3] = x.w;
-    }
-    for (int s = 0; s < topk; ++s) {
-      const __nv_bfloat16* hj = hblk + ((size_t)bh * nb + sel[s]) * FD * FD + 64 * tid;
-#pragma unroll
-      for (int e = 0; e < 64; e += 8) {
-        const uint4 x = *reinterpret_cast<const uint4*>(hj + e);
-        const uint32_t xv[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xv[u]));
-          a[e + 2 * u] -= f.x;
-          a[e + 2 * u + 1] -= f.y;
-        }
-      }
-    }
-    // entry x = 64 tid + e is (row x / 128, column x % 128): row tid / 2, chunks 8 (tid & 1) ..
-    const int r = tid >> 1;
-#pragma unroll
-    for (int c8 = 0; c8 < 8; ++c8) {
-      const int c = 8 * (tid & 1) + c8;
-      *reinterpret_cast<uint4*>(hu + swz(r, c)) =
-          make_uint4(fo_pack2(a[8 * c8], a[8 * c8 + 1]), fo_pack2(a[8 * c8 + 2], a[8 * c8 + 3]),
-                     fo_pack2(a[8 * c8 + 4], a[8 * c8 + 5]), fo_pack2(a[8 * c8 + 6], a[8 * c8 + 7]));
-    }
+    sub_matrices(a, htot + (size_t)bh * FD * FD, hblk + (size_t)bh * nb * FD * FD, ids, topk, tid);
+    store_entries(hu, a, tid);
     if (tid < FD) {
       float z = ztot[(size_t)bh * FD + tid];
-      for (int s = 0; s < topk; ++s) z -= zrelu[((size_t)bh * nb + sel[s]) * FD + tid];
+      for (int s2 = 0; s2 < topk; ++s2) z -= zrelu[((size_t)bh * nb + ids[s2]) * FD + tid];
       zu[tid] = z;
     }
   }
@@ -191,7 +220,7 @@ lin_q_kernel(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restric
   const uint32_t hu_s = (uint32_t)__cvta_generic_to_shared(hu), pq_s = (uint32_t)__cvta_generic_to_shared(pq),
                  dn_s = (uint32_t)__cvta_generic_to_shared(dn);
   warp_gemm<kRowsMK, kRowsKM>(acc, pq_s, hu_s, 16 * warp, lane);
-  // O_l, g_l, dnum (into the dn tile), the rows' g_l·O_l and (pass 0) g·O
+  // O_l, g_l, dnum (into the dn tile), the rows' g_l·O_l and g·O, α⊙g
   const float ia = 1.0f / den[ra], ib = 1.0f / den[rb];
   float ga = 0.f, gb = 0.f, oa = 0.f, ob = 0.f;
 #pragma unroll
@@ -199,23 +228,21 @@ lin_q_kernel(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restric
     const int c = 8 * nt + 2 * (lane & 3);
     const float2 g0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(dO + (row0 + ra) * FD + c));
     const float2 g1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(dO + (row0 + rb) * FD + c));
+    const float2 o0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(O + (row0 + ra) * FD + c));
+    const float2 o1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(O + (row0 + rb) * FD + c));
     const float w0 = 1.0f - al[c], w1 = 1.0f - al[c + 1];
     const float la0 = acc[nt][0] * ia, la1 = acc[nt][1] * ia, lb0 = acc[nt][2] * ib, lb1 = acc[nt][3] * ib;
     const float gla0 = w0 * g0.x, gla1 = w1 * g0.y, glb0 = w0 * g1.x, glb1 = w1 * g1.y;
     ga = fmaf(gla0, la0, fmaf(gla1, la1, ga));
     gb = fmaf(glb0, lb0, fmaf(glb1, lb1, gb));
+    oa = fmaf(g0.x, o0.x, fmaf(g0.y, o0.y, oa));
+    ob = fmaf(g1.x, o1.x, fmaf(g1.y, o1.y, ob));
     // dnum[t][e] at chunk c / 8, element c % 8
     const int ch = c >> 3, el = c & 7;
     *reinterpret_cast<uint32_t*>(dn + swz(ra, ch) + 2 * el) = fo_pack2(gla0 * ia, gla1 * ia);
     *reinterpret_cast<uint32_t*>(dn + swz(rb, ch) + 2 * el) = fo_pack2(glb0 * ib, glb1 * ib);
-    if (PASS == 0) {
-      const float2 o0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(O + (row0 + ra) * FD + c));
-      const float2 o1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(O + (row0 + rb) * FD + c));
-      oa = fmaf(g0.x, o0.x, fmaf(g0.y, o0.y, oa));
-      ob = fmaf(g1.x, o1.x, fmaf(g1.y, o1.y, ob));
-      *reinterpret_cast<uint32_t*>(dOs + (row0 + ra) * FD + c) = fo_pack2(al[c] * g0.x, al[c + 1] * g0.y);
-      *reinterpret_cast<uint32_t*>(dOs + (row0 + rb) * FD + c) = fo_pack2(al[c] * g1.x, al[c + 1] * g1.y);
-    }
+    *reinterpret_cast<uint32_t*>(dOs + (row0 + ra) * FD + c) = fo_pack2(al[c] * g0.x, al[c + 1] * g0.y);
+    *reinterpret_cast<uint32_t*>(dOs + (row0 + rb) * FD + c) = fo_pack2(al[c] * g1.x, al[c + 1] * g1.y);
   }
 #pragma unroll
   for (int o = 1; o <= 2; o <<= 1) {
@@ -227,44 +254,35 @@ lin_q_kernel(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restric
   if ((lane & 3) == 0) {
     dden[ra] = -ga * ia;
     dden[rb] = -gb * ib;
-    if (PASS == 0) {
-      delta_s[row0 + ra] = oa - ga;   // g·O − g_l·O_l
-      delta_s[row0 + rb] = ob - gb;
-    }
+    delta_s[row0 + ra] = oa - ga;   // g·O − g_l·O_l
+    delta_s[row0 + rb] = ob - gb;
   }
   __syncthreads();
+  // dH_U,i[c][e] = Σ_t φq[t][c] dnum[t][e]: A[c][t] stored [t][c], B[t][e] stored [t][e]
   zero_acc(acc);
-  if (PASS == 0) {
-    // dH_U,i[c][e] = Σ_t φq[t][c] dnum[t][e]: A[c][t] stored [t][c], B[t][e] stored [t][e]
-    warp_gemm<kRowsKM, kRowsKM>(acc, pq_s, dn_s, 16 * warp, lane);
-    store_acc_bf16(dHU + ((size_t)bh * nb + i) * FD * FD, acc, ra, rb, lane);
-    // dz_U,i[c] = Σ_t φq[t][c] dden_t
-    if (tid < FD) {
-      float z = 0.f;
-      const int ch = tid >> 3, el = tid & 7;
-      for (int t = 0; t < FT; ++t)
-        z = fmaf(__bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(pq + swz(t, ch) + 2 * el)), dden[t], z);
-      dzU[((size_t)bh * nb + i) * FD + tid] = z;
-    }
-  } else {
-    // dφq[t][c] = Σ_e dnum[t][e] H_U[c][e] + z_U[c] dden_t: A = dnum [t][e], B[e][c] = H_U[c][e] stored [c][e]
-    warp_gemm<kRowsMK, kRowsMK>(acc, dn_s, hu_s, 16 * warp, lane);
-    const float da = dden[ra], db = dden[rb];
+  warp_gemm<kRowsKM, kRowsKM>(acc, pq_s, dn_s, 16 * warp, lane);
+  store_acc_bf16(dHU + ((size_t)bh * nb + i) * FD * FD, acc, ra, rb, lane);
+  // dz_U,i[c] = Σ_t φq[t][c] dden_t
+  if (tid < FD) {
+    float z = 0.f;
+    const int ch = tid >> 3, el = tid & 7;
+    for (int t = 0; t < FT; ++t)
+      z = fmaf(__bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(pq + swz(t, ch) + 2 * el)), dden[t], z);
+    dzU[((size_t)bh * nb + i) * FD + tid] = z;
+  }
+  // dφq[t][c] = Σ_e dnum[t][e] H_U[c][e] + z_U[c] dden_t: A = dnum [t][e], B[e][c] = H_U[c][e] stored [c][e]
+  zero_acc(acc);
+  warp_gemm<kRowsMK, kRowsMK>(acc, dn_s, hu_s, 16 * warp, lane);
+  const float da = dden[ra], db = dden[rb];
 #pragma unroll
-    for (int nt = 0; nt < 16; ++nt) {
-      const int c = 8 * nt + 2 * (lane & 3);
-      const float2 q0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(Q + (row0 + ra) * FD + c));
-      const float2 q1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(Q + (row0 + rb) * FD + c));
-      float2* pa = reinterpret_cast<float2*>(dQ + (row0 + ra) * FD + c);
-      float2* pb = reinterpret_cast<float2*>(dQ + (row0 + rb) * FD + c);
-      float2 xa = *pa, xb = *pb;
-      xa.x += q0.x > 0.f ? fmaf(zu[c], da, acc[nt][0]) : 0.f;
-      xa.y += q0.y > 0.f ? fmaf(zu[c + 1], da, acc[nt][1]) : 0.f;
-      xb.x += q1.x > 0.f ? fmaf(zu[c], db, acc[nt][2]) : 0.f;
-      xb.y += q1.y > 0.f ? fmaf(zu[c + 1], db, acc[nt][3]) : 0.f;
-      *pa = xa;
-      *pb = xb;
-    }
+  for (int nt = 0; nt < 16; ++nt) {
+    const int c = 8 * nt + 2 * (lane & 3);
+    const float2 q0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(Q + (row0 + ra) * FD + c));
+    const float2 q1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(Q + (row0 + rb) * FD + c));
+    *reinterpret_cast<float2*>(dQ + (row0 + ra) * FD + c) =
+        make_float2(q0.x > 0.f ? fmaf(zu[c], da, acc[nt][0]) : 0.f, q0.y > 0.f ? fmaf(zu[c + 1], da, acc[nt][1]) : 0.f);
+    *reinterpret_cast<float2*>(dQ + (row0 + rb) * FD + c) =
+        make_float2(q1.x > 0.f ? fmaf(zu[c], db, acc[nt][2]) : 0.f, q1.y > 0.f ? fmaf(zu[c + 1], db, acc[nt][3]) : 0.f);
   }
 }
 
@@ -302,43 +320,17 @@ lin_kv_kernel(const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __restri
   uint8_t* dh = fsm;                          // dh_j [c][e]
   uint8_t* at = fsm + kTileB;                 // V, then φ(K)
   float* dz = reinterpret_cast<float*>(fsm + 2 * kTileB);
+  int* ids = reinterpret_cast<int*>(dz + FD);   // [i1 - i0] the query blocks that selected j
   stage_bf16(at, V + row0 * FD);
+  for (int x = tid; x < i1 - i0; x += kFoThreads) ids[x] = lst[i0 + x];
+  __syncthreads();
   {
     float a[64];
-    const float* ht = dHtot + (size_t)bh * FD * FD + 64 * tid;
-#pragma unroll
-    for (int e = 0; e < 64; e += 4) {
-      const float4 x = *reinterpret_cast<const float4*>(ht + e);
-      a[e] = x.x;
-      a[e + 1] = x.y;
-      a[e + 2] = x.z;
-      a[e + 3] = x.w;
-    }
-    for (int s = i0; s < i1; ++s) {
-      const __nv_bfloat16* hi = dHU + ((size_t)bh * nb + lst[s]) * FD * FD + 64 * tid;
-#pragma unroll
-      for (int e = 0; e < 64; e += 8) {
-        const uint4 x = *reinterpret_cast<const uint4*>(hi + e);
-        const uint32_t xv[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xv[u]));
-          a[e + 2 * u] -= f.x;
-          a[e + 2 * u + 1] -= f.y;
-        }
-      }
-    }
-    const int r = tid >> 1;
-#pragma unroll
-    for (int c8 = 0; c8 < 8; ++c8) {
-      const int c = 8 * (tid & 1) + c8;
-      *reinterpret_cast<uint4*>(dh + swz(r, c)) =
-          make_uint4(fo_pack2(a[8 * c8], a[8 * c8 + 1]), fo_pack2(a[8 * c8 + 2], a[8 * c8 + 3]),
-                     fo_pack2(a[8 * c8 + 4], a[8 * c8 + 5]), fo_pack2(a[8 * c8 + 6], a[8 * c8 + 7]));
-    }
+    sub_matrices(a, dHtot + (size_t)bh * FD * FD, dHU + (size_t)bh * nb * FD * FD, ids, i1 - i0, tid);
+    store_entries(dh, a, tid);
     if (tid < FD) {
       float z = dztot[(size_t)bh * FD + tid];
-      for (int s = i0; s < i1; ++s) z -= dzU[((size_t)bh * nb + lst[s]) * FD + tid];
+      for (int s2 = 0; s2 < i1 - i0; ++s2) z -= dzU[((size_t)bh * nb + ids[s2]) * FD + tid];
       dz[tid] = z;
     }
   }
@@ -415,14 +407,11 @@ sa_status bwd_linear_mix(const void* Q, const void* K, const void* V, const void
   const bf* o = static_cast<const bf*>(O);
   const bf* g = static_cast<const bf*>(dO);
   const dim3 grid((unsigned)nb, (unsigned)BH);
-  const size_t smem2 = 2 * kTileB, smemq = 3 * kTileB + sizeof(float) * (FD + 2 * FT),
-               smemkv = 2 * kTileB + sizeof(float) * FD;
+  const size_t smem2 = 2 * kTileB, smemq = 3 * kTileB + sizeof(float) * (FD + 2 * FT) + sizeof(int) * nb,
+               smemkv = 2 * kTileB + sizeof(float) * FD + sizeof(int) * nb;
   if (cudaFuncSetAttribute(lin_hblk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2) !=
           cudaSuccess ||
-      cudaFuncSetAttribute(lin_q_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smemq) !=
-          cudaSuccess ||
-      cudaFuncSetAttribute(lin_q_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smemq) !=
-          cudaSuccess ||
+      cudaFuncSetAttribute(lin_q_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smemq) != cudaSuccess ||
       cudaFuncSetAttribute(lin_kv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smemkv) != cudaSuccess)
     return launch_status("cudaFuncSetAttribute(linear-mix backward kernels)");
   const bool lin = topk < (int)nb;
@@ -431,19 +420,23 @@ sa_status bwd_linear_mix(const void* Q, const void* K, const void* V, const void
     sa_status r = launch_status("lin_hblk_kernel");
     if (r != SA_OK) return r;
   }
-  lin_q_kernel<0><<<grid, kFoThreads, smemq, stream>>>(q, o, g, alpha, s.H, s.N, block_idx, topk, st.htot, st.ztot,
-                                                       st.zrelu, hblk, delta_s, dOs, dHU, dzU, dQ);
+  lin_q_kernel<<<grid, kFoThreads, smemq, stream>>>(q, o, g, alpha, s.H, s.N, block_idx, topk, st.htot, st.ztot,
+                                                    st.zrelu, hblk, delta_s, dOs, dHU, dzU, dQ);
   sa_status r = launch_status("lin_q_kernel");
   if (r != SA_OK) return r;
-  // the softmax branch: the drop backward of α⊙dO with δ_s
-  const BwdTailTerms tt{nullptr, nullptr, nullptr, delta_s};
-  r = bwd_tc(Q, K, V, O, dOs, s, block_idx, topk, false, st, scale, dQ, dK, dV, nullptr, lse2, delta, offs, list,
-             part, stream, &tt);
+  // the softmax branch: the drop backward of α⊙dO with δ_s, its dQ added to the
+  // linear branch's (without a selected block it has no keys and no gradients)
+  if (topk > 0) {
+    const BwdTailTerms tt{nullptr, nullptr, nullptr, delta_s, true};
+    r = bwd_tc(Q, K, V, O, dOs, s, block_idx, topk, false, st, scale, dQ, dK, dV, nullptr, lse2, delta, offs, list,
+               part, stream, &tt);
+  } else {
+    const size_t bytes = BH * s.N * FD * sizeof(float);
+    r = (cudaMemsetAsync(dK, 0, bytes, stream) == cudaSuccess && cudaMemsetAsync(dV, 0, bytes, stream) == cudaSuccess)
+            ? SA_OK
+            : launch_status("cudaMemsetAsync(dK, dV)");
+  }
   if (r != SA_OK || !lin) return r;
-  lin_q_kernel<1><<<grid, kFoThreads, smemq, stream>>>(q, o, g, alpha, s.H, s.N, block_idx, topk, st.htot, st.ztot,
-                                                       st.zrelu, hblk, delta_s, dOs, dHU, dzU, dQ);
-  r = launch_status("lin_q_kernel");
-  if (r != SA_OK) return r;
   lin_tot_kernel<<<dim3(FD * FD / 256, (unsigned)BH), 256, 0, stream>>>(dHU, dzU, (int)nb, dHtot, dztot);
   r = launch_status("lin_tot_kernel");
   if (r != SA_OK) return r;

@@ -19,7 +19,9 @@
 // when the forward's log-sum-exp is given); pass 2
 // forms S again, dP = dO Vᵀ, writes dS (bf16) into the S columns, and
 // accumulates dQ += dS · K with dS read from TMEM.
-// SLA2's linear mix (delta_in non-null): the softmax branch's δ is given.
+// SLA2's linear mix (delta_in non-null): the softmax branch's δ is given, and
+// with dq_add the kernel adds its dQ to what dQ already holds (the linear
+// branch's term, written first).
 // PISA's first-order tail (doff non-null): a pseudo-key's value seen by row t
 // is v̄_j + f_t / B (f_t = s H̄ᵀ q_t), so the centroid tiles take
 // dS = P (dP − δ + doff_t) with doff_t = dO_t·f_t / B; the kernel also writes
@@ -106,7 +108,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                  const int32_t* __restrict__ block_idx, int N, int topk, int zo, float scale,
                  const float* __restrict__ lse_in, float* __restrict__ lse2, float* __restrict__ delta,
                  float* __restrict__ dQ, const float* __restrict__ doff, float* __restrict__ delta_c,
-                 float* __restrict__ lam, size_t lam_stride, const float* __restrict__ delta_in) {
+                 float* __restrict__ lam, size_t lam_stride, const float* __restrict__ delta_in, int dq_add) {
   using L = Lay;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -449,11 +451,20 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         tmem_ld32(lrow + kColDQ + 64 * grp + 32 * h, a);
         tmem_wait_ld();
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
-          out[8 * h + q] = make_float4(scale * __uint_as_float(a[4 * q]), scale * __uint_as_float(a[4 * q + 1]),
-                                       scale * __uint_as_float(a[4 * q + 2]), scale * __uint_as_float(a[4 * q + 3]));
+        for (int q = 0; q < 8; ++q) {
+          float4 y = make_float4(scale * __uint_as_float(a[4 * q]), scale * __uint_as_float(a[4 * q + 1]),
+                                 scale * __uint_as_float(a[4 * q + 2]), scale * __uint_as_float(a[4 * q + 3]));
+          if (dq_add) {
+            const float4 x = out[8 * h + q];
+            y.x += x.x;
+            y.y += x.y;
+            y.z += x.z;
+            y.w += x.w;
+          }
+          out[8 * h + q] = y;
+        }
       }
-    } else if (T == 0) {
+    } else if (T == 0 && !dq_add) {
 #pragma unroll
       for (int q = 0; q < 16; ++q) out[q] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
@@ -825,7 +836,8 @@ sa_status bwd_dq_tc(const void* Q, const void* K, const void* V, const void* O, 
   bwd_dq_tc_kernel<<<dim3(nb, (unsigned)BH), kThreads, smem, stream>>>(
       mq, mg, mk, mv, mkb, mvb, static_cast<const __nv_bfloat16*>(O), static_cast<const __nv_bfloat16*>(dO),
       block_idx, s.N, topk, zo ? 1 : 0, scale, lse_in, lse2, delta, dQ, fo ? fo->doff : nullptr,
-      fo ? fo->delta_c : nullptr, fo ? fo->lam : nullptr, (size_t)BH * s.N, fo ? fo->delta_in : nullptr);
+      fo ? fo->delta_c : nullptr, fo ? fo->lam : nullptr, (size_t)BH * s.N, fo ? fo->delta_in : nullptr,
+      fo && fo->dq_add ? 1 : 0);
   return launch_status("bwd_dq_tc_kernel");
 }
 
