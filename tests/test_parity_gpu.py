@@ -103,7 +103,8 @@ def test_block_pool_large_offset_variance(lib):
 # --------------------------------------------------------------------------
 
 @pytest.mark.parametrize("mode", ["dot", "proj", "taylor2", "cov"])
-@pytest.mark.parametrize("nb,k", [(37, 5), (256, 26), (16, 0), (16, 16), (97, 64), (97, 65), (300, 100)])
+@pytest.mark.parametrize("nb,k", [(37, 5), (256, 26), (16, 0), (16, 16), (97, 64), (97, 65), (300, 100),
+                                  (600, 40), (1100, 64)])
 def test_route(lib, mode, nb, k):
     d, block = 128, 128
     w = wl.WORKLOADS["video_dit"]
@@ -127,6 +128,22 @@ def test_route(lib, mode, nb, k):
     check_topk_exact(idx, sc, k)
     frac = selection_agreement(np64(sc), ref, k)
     assert frac >= 0.95
+
+
+def test_route_tie_groups_cut_by_k(lib):
+    # 24 distinct key blocks, each repeated 4 times: every dot score comes in
+    # a group of 4 equal ones, and k = 10 keeps two groups and the two
+    # smallest indices of the third (the selection is the same for every
+    # score mode)
+    d, block, nb = 128, 128, 96
+    Q, K, V = _gauss(1, 1, nb * block, d, torch.float32, 7)
+    K = K.reshape(1, 1, nb, block, d)[:, :, ::4].repeat_interleave(4, dim=2).reshape(1, 1, nb * block, d)
+    st = bd.block_pool(Q, K.contiguous(), V, block)
+    idx, sc = bd.route(st, (1, 1, nb * block, d, block), "dot", 10, want_scores=True)
+    check_topk_exact(idx, sc, 10)
+    s = np64(sc)[0, 0]
+    assert (s.reshape(nb, 24, 4) == s.reshape(nb, 24, 4)[..., :1]).all()   # the groups do tie
+    assert (np.diff(idx.cpu().numpy(), axis=-1) > 0).all()
 
 
 def test_route_ties_pick_smaller_index(lib):
