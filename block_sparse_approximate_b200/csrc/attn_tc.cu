@@ -455,12 +455,20 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
       for (int k = 0; k < 8; ++k) sm8[k] = 0.f;
       const float sc2 = live ? tscale : 0.f, ng = live ? neg : -INFINITY;   // dead row: p = 0
+      float sum_scale = 1.f;
       if (F8) {
+        // the exponentials come out already scaled for the e4m3 store,
+        // p' = p·pscale = 2^(a + log2 pscale), and the row sum takes Σp'/pscale.
+        // pscale is floored at 2^-100: below it every p' rounds to e4m3 zero
+        // either way, and p' stays a normal fp32 number for the sum.
+        const float pse = fmaxf(pscale, 0x1p-100f);
+        const float ngp = ng + __log2f(pse);
+        sum_scale = 1.0f / pse;
 #pragma unroll
         for (int n = 0; n < TB / 4; ++n) {
           float a0, a1, a2, a3;
-          ffma2(a0, a1, __uint_as_float(v[4 * n]), __uint_as_float(v[4 * n + 1]), sc2, sc2, ng, ng);
-          ffma2(a2, a3, __uint_as_float(v[4 * n + 2]), __uint_as_float(v[4 * n + 3]), sc2, sc2, ng, ng);
+          ffma2(a0, a1, __uint_as_float(v[4 * n]), __uint_as_float(v[4 * n + 1]), sc2, sc2, ngp, ngp);
+          ffma2(a2, a3, __uint_as_float(v[4 * n + 2]), __uint_as_float(v[4 * n + 3]), sc2, sc2, ngp, ngp);
           float p0, p1, p2, p3;
           if ((kExpFmaF8 >> (n & 7)) & 1u) {
             exp2_poly2(a0, a1, p0, p1);
@@ -469,7 +477,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             p0 = fast_exp2(a0); p1 = fast_exp2(a1); p2 = fast_exp2(a2); p3 = fast_exp2(a3);
           }
           fadd2(sm8[2 * (n & 3)], sm8[2 * (n & 3) + 1], p0 + p2, p1 + p3);
-          v[n] = pack_e4m3x4(p0 * pscale, p1 * pscale, p2 * pscale, p3 * pscale);
+          v[n] = pack_e4m3x4(p0, p1, p2, p3);
         }
       } else {
 #pragma unroll
@@ -483,7 +491,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           v[n] = pack_bf16(p0, p1);
         }
       }
-      const float sum = ((sm8[0] + sm8[1]) + (sm8[2] + sm8[3])) + ((sm8[4] + sm8[5]) + (sm8[6] + sm8[7]));
+      const float sum =
+          (((sm8[0] + sm8[1]) + (sm8[2] + sm8[3])) + ((sm8[4] + sm8[5]) + (sm8[6] + sm8[7]))) * sum_scale;
       l = l * factor + sum;
       if (FO) lc = lc * factor + (centroid ? sum : 0.f);
       tmem_st32(lrow + s_col, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
