@@ -210,6 +210,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                const int32_t* __restrict__ block_idx, int nb, int topk, float scale2, F8Scales f8,
                __nv_bfloat16* __restrict__ O, int N, float* __restrict__ lse_out) {
   static_assert(!FO || (ZO && !F8), "the first-order tail extends the bf16 zero-order tail");
+  // launched with programmatic stream serialization: the block indices and
+  // statistics come from the previous launches on the stream
+  pdl_wait();
+  pdl_trigger();
   using L = Layout<F8>;
   constexpr int NS = L::NS;
   constexpr uint32_t kTile = L::kTile;
@@ -652,8 +656,9 @@ sa_status launch_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensor
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return launch_status("cudaFuncSetAttribute(attn_tc_kernel)");
   dim3 grid(nb, (unsigned)((uint64_t)s.B * s.H));
-  kern<<<grid, kTcThreads, smem, stream>>>(mq, mk, mv, mkb, mvb, mhb, block_idx, nb, topk, scale * kLog2e, f8,
-                                           static_cast<__nv_bfloat16*>(O), s.N, lse_out);
+  const cudaError_t le = launch_pdl(kern, grid, dim3(kTcThreads), smem, stream, mq, mk, mv, mkb, mvb, mhb, block_idx,
+                                    nb, topk, scale * kLog2e, f8, static_cast<__nv_bfloat16*>(O), s.N, lse_out);
+  if (le != cudaSuccess) return fail(SA_ERR_CUDA, std::string("attn_tc_kernel: ") + cudaGetErrorString(le));
   return launch_status("attn_tc_kernel");
 }
 
@@ -691,6 +696,8 @@ attn_tc_linmix_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
                       int topk, float scale2, const float* __restrict__ alpha, const float* __restrict__ zrelu,
                       const float* __restrict__ htot, const float* __restrict__ ztot, int H,
                       __nv_bfloat16* __restrict__ O, int N) {
+  pdl_wait();                                   // the block indices and statistics of the previous launches
+  pdl_trigger();
   using L = LinLayout;
   constexpr int NS = L::NS;
   constexpr uint32_t kTile = L::kTile;
@@ -1294,9 +1301,11 @@ sa_status attn_tc(const void* Q, const void* K, const void* V, const sa_shape& s
         cudaSuccess)
       return launch_status("cudaFuncSetAttribute(attn_tc_linmix_kernel)");
     dim3 grid(nb, (unsigned)BH);
-    attn_tc_linmix_kernel<<<grid, kTcThreads, smem, stream>>>(mq, mk, mv, block_idx, nb, topk, scale * kLog2e,
-                                                              alpha, st.zrelu, st.htot, st.ztot, s.H,
-                                                              static_cast<__nv_bfloat16*>(O), s.N);
+    const cudaError_t le = launch_pdl(attn_tc_linmix_kernel, grid, dim3(kTcThreads), smem, stream, mq, mk, mv,
+                                      block_idx, nb, topk, scale * kLog2e, alpha, st.zrelu, st.htot, st.ztot, s.H,
+                                      static_cast<__nv_bfloat16*>(O), s.N);
+    if (le != cudaSuccess)
+      return fail(SA_ERR_CUDA, std::string("attn_tc_linmix_kernel: ") + cudaGetErrorString(le));
     return launch_status("attn_tc_linmix_kernel");
   }
   const bool fo = tail == SA_TAIL_FIRST_ORDER;

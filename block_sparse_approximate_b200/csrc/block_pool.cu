@@ -28,6 +28,11 @@ block_pool_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __r
   const size_t head_off = ((size_t)b * H + h) * (size_t)N * D;
   const size_t row0 = (size_t)j * BLK;
   const size_t stat_off = (((size_t)b * H + h) * nb + j) * D;
+  // launched with programmatic stream serialization: wait for the previous
+  // launch (which may still read the statistics this kernel rewrites), then
+  // let the next launch on the stream (the router) schedule its CTAs
+  pdl_wait();
+  pdl_trigger();
 
   __shared__ float red[RPP][D];
   __shared__ float mean_sh[D];
@@ -337,8 +342,10 @@ template <typename T, int D, int BLK>
 sa_status launch_pool(const void* Q, const void* K, const void* V, const sa_shape& s,
                       const sa_block_stats& st, cudaStream_t stream) {
   dim3 grid(s.N / BLK, s.H, s.B);
-  block_pool_kernel<T, D, BLK><<<grid, kPoolThreads, 0, stream>>>(
-      static_cast<const T*>(Q), static_cast<const T*>(K), static_cast<const T*>(V), s.H, s.N, st);
+  const cudaError_t le = launch_pdl(block_pool_kernel<T, D, BLK>, grid, dim3(kPoolThreads), 0, stream,
+                                    static_cast<const T*>(Q), static_cast<const T*>(K), static_cast<const T*>(V),
+                                    s.H, s.N, st);
+  if (le != cudaSuccess) return fail(SA_ERR_CUDA, std::string("block_pool_kernel: ") + cudaGetErrorString(le));
   sa_status r = launch_status("block_pool_kernel");
   if (r != SA_OK) return r;
   if (st.htot || st.ztot) {

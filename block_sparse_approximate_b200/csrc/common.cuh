@@ -31,6 +31,27 @@ inline sa_status launch_status(const char* what) {
 
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
+// Launch with programmatic stream serialization: the kernel may be scheduled
+// while the previous launch on the stream drains, so it must call pdl_wait()
+// before it reads or writes anything that launch touches.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+  if (e != cudaSuccess) cudaGetLastError();   // reported by the caller's status, not left pending
+  return e;
+}
+
 inline size_t dtype_size(sa_dtype t) { return t == SA_FP32 ? 4 : 2; }
 
 // Host-side validation of a prefill shape; returns SA_OK or sets the error.
@@ -56,6 +77,15 @@ template <>
 __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
 
 // 2^x on the MUFU unit (PTX ex2.approx; flushes subnormal results to zero).
+// Programmatic dependent launch: a kernel launched by launch_pdl() may start
+// while its predecessor drains; it waits here before touching anything the
+// predecessor reads or writes (a no-op for a kernel launched without it).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Lets the next launch on the stream start its CTAs (up to their pdl_wait())
+// once every CTA of this grid has passed here; all of them are then resident,
+// so the waiting successors cannot hold back a CTA of this grid.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

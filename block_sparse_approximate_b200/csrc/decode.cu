@@ -135,15 +135,6 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// Programmatic dependent launch: a kernel launched with programmatic stream
-// serialization may start while its predecessor drains; it waits here
-// before touching anything the predecessor writes (a no-op otherwise).
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-// Lets the next launch on the stream start its CTAs (up to their pdl_wait())
-// once every CTA of this grid has passed here; all of them are then resident,
-// so the waiting successors cannot hold back a CTA of this grid.
-__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-
 __device__ __forceinline__ uint32_t pack2bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
@@ -1406,26 +1397,6 @@ decode_combine_kernel(const float* __restrict__ parta, int nsegA, const float* _
     res *= rsqrtf(tot / D + kRmsEps);
   }
   if (pt == 0) O[((size_t)b * Hq + h) * D + c] = __float2bfloat16_rn(o_s + res);
-}
-
-// Launch with programmatic stream serialization (the kernel calls pdl_wait()
-// before reading what the previous launch on the stream wrote).
-template <typename... KArgs, typename... Args>
-cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
-                       Args... args) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = block;
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
-  if (e != cudaSuccess) cudaGetLastError();   // reported by the caller's status, not left pending
-  return e;
 }
 
 int sm_count() {

@@ -223,6 +223,8 @@ route_kernel(sa_block_stats st, int H, int nb, sa_route_mode mode, const float* 
   const int nwords = (nb + 31) >> 5;
   uint32_t* bits = reinterpret_cast<uint32_t*>(sc + (size_t)QB * nb);   // [QB][nwords]
 
+  pdl_wait();                                     // the statistics come from the previous launch
+  pdl_trigger();
   // ---- query vectors
   for (int x = tid; x < QB * D; x += kRouteThreads) {
     const int r = x / D, c = x % D;
@@ -464,6 +466,8 @@ route_mma_kernel(sa_block_stats st, int H, int nb, sa_route_mode mode, const flo
   float* tiles = qw + (t2 ? kMQ * LD : 0);        // [2][narr][TS]; the row bitmaps after the scores
   float* sc = tiles + 2 * (size_t)narr * TS;      // [16][ldc] scores; T = q̄ P_q (proj) before them
 
+  pdl_wait();                                     // the statistics come from the previous launch
+  pdl_trigger();
   const float* qm = st.qmean + (bh * nb + i0) * D;
   const float* km = st.kmean + bh * (size_t)nb * D;
   const float* kv = t2 ? st.kvar + bh * (size_t)nb * D : nullptr;
@@ -603,7 +607,9 @@ sa_status launch_route_mma(const sa_block_stats& st, sa_shape shape, int nb, sa_
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return launch_status("cudaFuncSetAttribute(route_mma_kernel)");
   dim3 grid((nb + kMQ - 1) / kMQ, shape.H, shape.B);
-  kern<<<grid, kMmaThreads, smem, s>>>(st, shape.H, nb, mode, Pq, Pk, scale, inv_blk, topk, idx, scores);
+  const cudaError_t le = launch_pdl(kern, grid, dim3(kMmaThreads), smem, s, st, shape.H, nb, mode, Pq, Pk, scale,
+                                    inv_blk, topk, idx, scores);
+  if (le != cudaSuccess) return fail(SA_ERR_CUDA, std::string("route_mma_kernel: ") + cudaGetErrorString(le));
   return launch_status("route_mma_kernel");
 }
 
@@ -644,7 +650,9 @@ sa_status launch_route(const sa_block_stats& st, sa_shape shape, int nb, sa_rout
     return launch_status("cudaFuncSetAttribute(route_kernel)");
   constexpr int QB = kRouteWarps * RPW;
   dim3 grid((nb + QB - 1) / QB, shape.H, shape.B);
-  kern<<<grid, kRouteThreads, smem, s>>>(st, shape.H, nb, mode, Pq, Pk, scale, inv_blk, topk, idx, scores);
+  const cudaError_t le = launch_pdl(kern, grid, dim3(kRouteThreads), smem, s, st, shape.H, nb, mode, Pq, Pk, scale,
+                                    inv_blk, topk, idx, scores);
+  if (le != cudaSuccess) return fail(SA_ERR_CUDA, std::string("route_kernel: ") + cudaGetErrorString(le));
   return launch_status("route_kernel");
 }
 
