@@ -961,8 +961,9 @@ decode_exact_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
 // The same outputs as decode_stats_kernel for bf16 kmean, kvar and value
 // means.  A stage is 64 blocks of the three arrays, staged by cp.async
 // (16-byte chunks of row r at chunk ^ (r & 7), as the exact pass stages K and
-// V) into a ring of four, so three stages (144 KB) are in flight while one is
-// reduced; a segment is two stages (128 blocks, the segments of
+// V) into a ring (with the zero-order tail: four slots, three stages of
+// 48 KB in flight while one is reduced; without it: two CTAs per SM with two
+// slots each); a segment is two stages (128 blocks, the segments of
 // decode_stats_kernel).  Warp w takes blocks [8w, 8w + 8) of a stage.  The dot
 // products are mma.sync m16n8k16 contractions with the group's G <= 8 query
 // heads as the MMA rows and the warp's 8 blocks as the columns:
@@ -976,10 +977,18 @@ decode_exact_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
 // state per head as in decode_stats_kernel.
 constexpr int kStageBlocksM = 64;
 constexpr int kSegM = (kStageBlocksA * kSegA) / kStageBlocksM;   // stages per segment (2)
-constexpr int kRingM = 4;
+// ring slots and CTAs per SM: with the zero-order tail (three arrays and the
+// P·v̄ accumulators) one CTA per SM with four slots; without it (two arrays)
+// two CTAs per SM with two slots each (measured: 0.155 against 0.162 ms for
+// the residual-linear decode step; the zero-order variant spills at two per
+// SM and is slower)
+template <bool ZT>
+constexpr int ring_m() { return ZT ? 4 : 2; }
+template <bool ZT>
+constexpr int ctas_m() { return ZT ? 1 : 2; }
 
 template <int D, bool ZT>
-__global__ void __launch_bounds__(kDecThreads, 1)
+__global__ void __launch_bounds__(kDecThreads, ctas_m<ZT>())
 decode_stats_mma_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kmean,
                         const __nv_bfloat16* __restrict__ kvar, const __nv_bfloat16* __restrict__ vmean, int Hq,
                         int Hkv, int nb, int blk, float scale, int nsegA, int npairs, float* __restrict__ scores,
@@ -991,6 +1000,7 @@ decode_stats_mma_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16
   constexpr uint32_t kArrB = kStageBlocksM * kRowB;
   constexpr int NARR = ZT ? 3 : 2;
   constexpr uint32_t kStageB = NARR * kArrB;
+  constexpr int kRing = ring_m<ZT>();
   extern __shared__ __align__(16) uint8_t dsm[];
   const int g = Hq / Hkv;
   float* mg = reinterpret_cast<float*>(dsm);                         // [8 warps][g][D + 2] merge
@@ -1034,9 +1044,9 @@ decode_stats_mma_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16
       }
     }
     cp_async_commit();
-    pf_slot = (pf_slot + 1) % kRingM;
+    pf_slot = (pf_slot + 1) % kRing;
   };
-  for (int r = 0; r < kRingM - 1; ++r) prefetch();
+  for (int r = 0; r < kRing - 1; ++r) prefetch();
 
   uint32_t qa0[KS], qa2[KS];                  // q (rows = heads)
   uint32_t wh0[KS], wh2[KS], wl0[KS], wl2[KS];   // ½ s² q², hi and lo bf16 parts
@@ -1082,7 +1092,7 @@ decode_stats_mma_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16
       for (int nt = 0; nt < (ZT ? NT : 1); ++nt) o[nt][0] = o[nt][1] = 0.f;
     }
     prefetch();
-    cp_async_wait<kRingM - 1>();
+    cp_async_wait<kRing - 1>();
     __syncthreads();
 
     const uint32_t kbase = ring_s + slot * kStageB, vbase = kbase + 2 * kArrB;
@@ -1152,7 +1162,7 @@ decode_stats_mma_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16
         }
       }
     }
-    slot = (slot + 1) % kRingM;
+    slot = (slot + 1) % kRing;
     const bool seg_end = ++cur_sub >= stages_in(seg);
     if (ZT && seg_end) {
       // the warp's state of head hrow for this segment, then the merge
@@ -1458,10 +1468,11 @@ sa_status launch_decode(const void* q, const void* Kc, const void* Vc, const sa_
     };
     const bool zt = tail == SA_TAIL_ZERO_ORDER;
     if constexpr (sizeof(TS) == 2) {
-      // bf16 statistics: the tensor-core statistics pass, one CTA per SM
+      // bf16 statistics: the tensor-core statistics pass (one or two CTAs per SM)
       const size_t smemM = ((sizeof(float) * kDecWarps * g * (D + 2) + 127) & ~(size_t)127) +
-                           (size_t)kRingM * (zt ? 3 : 2) * kStageBlocksM * D * 2;
-      const int gridM = (int)(segsA < sms ? segsA : sms);
+                           (size_t)(zt ? ring_m<true>() : ring_m<false>()) * (zt ? 3 : 2) * kStageBlocksM * D * 2;
+      const int per_sm = zt ? ctas_m<true>() : ctas_m<false>();
+      const int gridM = (int)(segsA < per_sm * sms ? segsA : per_sm * sms);
       auto kern = zt ? decode_stats_mma_kernel<D, true> : decode_stats_mma_kernel<D, false>;
       if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smemM) != cudaSuccess)
         return launch_status("cudaFuncSetAttribute(decode_stats_mma_kernel)");

@@ -316,6 +316,36 @@ def test_decode(lib, tail, B, Hq, Hkv, N, d, block, k):
     del w
 
 
+@pytest.mark.parametrize("case", ["tie_groups", "all_equal", "long_row"])
+def test_decode_topk_edge_rows(lib, case):
+    # tie_groups: 12 distinct key blocks repeated 4 times, so the scores come
+    # in groups of 4 equal ones and k = 10 cuts the third group (the smallest
+    # indices win); all_equal: one key block everywhere; long_row: 4000 blocks
+    # per row (16 keys per thread of the top-k)
+    d, block = 128, 64
+    nb, k = {"tie_groups": (48, 10), "all_equal": (40, 5), "long_row": (4000, 64)}[case]
+    g = torch.Generator(device=DEV)
+    g.manual_seed(300 + nb)
+    q = torch.randn(1, 4, d, generator=g, device=DEV).to(torch.bfloat16)
+    Kb = torch.randn(1, 1, nb, block, d, generator=g, device=DEV)
+    if case == "tie_groups":
+        Kb = Kb[:, :, ::4].repeat_interleave(4, dim=2)
+    elif case == "all_equal":
+        Kb = Kb[:, :, :1].expand(1, 1, nb, block, d)
+    Kc = Kb.reshape(1, 1, nb * block, d).to(torch.bfloat16).contiguous()
+    Vc = torch.randn(1, 1, nb * block, d, generator=g, device=DEV).to(torch.bfloat16)
+    st = bd.block_pool(None, Kc, Vc, block, variance=True)
+    o, idx, sc = bd.decode_fwd(q, Kc, Vc, st, block, k, 1 / math.sqrt(d))
+    torch.cuda.synchronize()
+    assert_no_device_error()
+    check_topk_exact(idx, sc, k)
+    if case == "all_equal":
+        assert (idx.cpu().numpy().ravel() == np.arange(k)).all()
+    if case == "tie_groups":
+        s = np64(sc).ravel()
+        assert (s.reshape(12, 4) == s.reshape(12, 4)[:, :1]).all()   # the groups do tie
+
+
 def _bf16_round(x: np.ndarray) -> np.ndarray:
     return torch.as_tensor(x).to(torch.bfloat16).to(torch.float64).numpy()
 
