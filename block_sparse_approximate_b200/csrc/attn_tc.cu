@@ -392,11 +392,31 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         for (int c = 0; c < ntiles; ++c) vmax = fmaxf(vmax, f8.vbar[(size_t)bh * ntiles + c]);
       qs = f8.q[(size_t)bh * nb + i];
     }
+    const float inv_vmax = 1.0f / vmax;
+    // e4m3: the K and V scales of tile t (the block index, then the block's
+    // scales: two dependent loads), fetched one tile of this stream ahead so
+    // that they arrive during the previous tile's softmax
+    auto tile_scales = [&](int t, float& ks, float& vs) {
+      if (!F8 || t >= T) return;
+      const int ntiles = (nb + TB - 1) / TB;
+      if (t >= topk) {
+        ks = f8.kbar[(size_t)bh * ntiles + (t - topk)];
+        vs = f8.vbar[(size_t)bh * ntiles + (t - topk)];
+      } else {
+        const int j = sel[t];
+        ks = f8.k[(size_t)bh * nb + j];
+        vs = f8.v[(size_t)bh * nb + j];
+      }
+    };
+    float ks_cur = 1.f, vs_cur = 1.f;
+    if (F8 && U > 0) tile_scales(st, ks_cur, vs_cur);
     float m_used = -INFINITY, l = 0.f;
     float lc = 0.f;   // first-order: the centroid tiles' share of l
     bool ok = true;
     for (int u = 0; u < U; ++u) {
       const int t = 2 * u + st;
+      float ks_nxt = 1.f, vs_nxt = 1.f;
+      if (F8) tile_scales(t + 2, ks_nxt, vs_nxt);
       if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_SF + st), u & 1, abort_flag))) {
         ok = false;
         break;
@@ -411,16 +431,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       float bias = 0.f;
       float tscale = scale2, pscale = 1.f;
       if (F8) {
-        const int ntiles = (nb + TB - 1) / TB;
-        if (centroid) {
-          const int c = t - topk;
-          tscale = scale2 * qs * f8.kbar[(size_t)bh * ntiles + c];
-          pscale = Fmt<true>::kPScale * f8.vbar[(size_t)bh * ntiles + c] / vmax;
-        } else {
-          const int j = sel[t];
-          tscale = scale2 * qs * f8.k[(size_t)bh * nb + j];
-          pscale = Fmt<true>::kPScale * f8.v[(size_t)bh * nb + j] / vmax;
-        }
+        tscale = scale2 * qs * ks_cur;
+        pscale = Fmt<true>::kPScale * vs_cur * inv_vmax;
+        ks_cur = ks_nxt;
+        vs_cur = vs_nxt;
       }
       if (centroid) {
         // validity of the 128 pseudo-keys: inside the head and not selected
