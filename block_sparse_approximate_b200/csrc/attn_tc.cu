@@ -1388,6 +1388,6 @@ extern "C" sa_status sa_device_error(uint32_t* code) {
   if (cudaMemcpyFromSymbol(&v, tc::g_device_error, sizeof(v)) != cudaSuccess ||
       cudaMemcpyToSymbol(tc::g_device_error, &zero, sizeof(zero)) != cudaSuccess)
     return launch_status("sa_device_error");
-  *code = v | decode_error_take() | covnorm_error_take() | bwd_error_take();
+  *code = v | decode_error_take() | covnorm_error_take() | bwd_error_take() | decode_tc_error_take();
   return SA_OK;
 }

@@ -1468,17 +1468,23 @@ sa_status launch_decode(const void* q, const void* Kc, const void* Vc, const sa_
     };
     const bool zt = tail == SA_TAIL_ZERO_ORDER;
     if constexpr (sizeof(TS) == 2) {
-      // bf16 statistics: the tensor-core statistics pass (one or two CTAs per SM)
-      const size_t smemM = ((sizeof(float) * kDecWarps * g * (D + 2) + 127) & ~(size_t)127) +
-                           (size_t)(zt ? ring_m<true>() : ring_m<false>()) * (zt ? 3 : 2) * kStageBlocksM * D * 2;
-      const int per_sm = zt ? ctas_m<true>() : ctas_m<false>();
-      const int gridM = (int)(segsA < per_sm * sms ? segsA : per_sm * sms);
-      auto kern = zt ? decode_stats_mma_kernel<D, true> : decode_stats_mma_kernel<D, false>;
-      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smemM) != cudaSuccess)
-        return launch_status("cudaFuncSetAttribute(decode_stats_mma_kernel)");
-      kern<<<gridM, kDecThreads, smemM, stream>>>(qb, ds.kmean, ds.kvar, ds.vrow, s.Hq, s.Hkv, nb, s.block, scale,
-                                                  L.nsegA, npairs, scores, parta);
-      r0 = launch_status("decode_stats_mma_kernel");
+      if (D == 128 && g <= 16) {
+        // bf16 statistics, d = 128: the tcgen05 statistics pass (decode_tc.cu)
+        r0 = decode_stats_tc(qb, ds.kmean, ds.kvar, ds.vrow, s.B, s.Hq, s.Hkv, nb, s.block, scale, L.nsegA, zt,
+                             sms, scores, parta, stream);
+      } else {
+        // bf16 statistics otherwise: the mma.sync statistics pass (one or two CTAs per SM)
+        const size_t smemM = ((sizeof(float) * kDecWarps * g * (D + 2) + 127) & ~(size_t)127) +
+                             (size_t)(zt ? ring_m<true>() : ring_m<false>()) * (zt ? 3 : 2) * kStageBlocksM * D * 2;
+        const int per_sm = zt ? ctas_m<true>() : ctas_m<false>();
+        const int gridM = (int)(segsA < per_sm * sms ? segsA : per_sm * sms);
+        auto kern = zt ? decode_stats_mma_kernel<D, true> : decode_stats_mma_kernel<D, false>;
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smemM) != cudaSuccess)
+          return launch_status("cudaFuncSetAttribute(decode_stats_mma_kernel)");
+        kern<<<gridM, kDecThreads, smemM, stream>>>(qb, ds.kmean, ds.kvar, ds.vrow, s.Hq, s.Hkv, nb, s.block, scale,
+                                                    L.nsegA, npairs, scores, parta);
+        r0 = launch_status("decode_stats_mma_kernel");
+      }
     } else if (g == 1) run(zt ? decode_stats_kernel<D, 1, true, TS> : decode_stats_kernel<D, 1, false, TS>);
     else if (g == 2) run(zt ? decode_stats_kernel<D, 2, true, TS> : decode_stats_kernel<D, 2, false, TS>);
     else if (g == 4) run(zt ? decode_stats_kernel<D, 4, true, TS> : decode_stats_kernel<D, 4, false, TS>);
