@@ -64,10 +64,13 @@ uint32_t decode_error_take();
 // kmean, kvar (and, with the zero-order tail, value means) [B·Hkv][nb][128],
 // q bf16 [B][Hq][128] with Hq / Hkv <= 16; writes the group scores
 // [B·Hkv][nb] and the zero-order partial states [B][Hq][nsegA][130] (one per
-// 128 blocks).  decode_tc_error_take() reads and clears its device error word.
+// 128 blocks); when each CTA holds a whole row it also writes the row's top
+// `topk` indices to idx and sets *topk_done.  decode_tc_error_take() reads
+// and clears its device error word.
 sa_status decode_stats_tc(const __nv_bfloat16* q, const void* kmean, const void* kvar, const void* vmean, int B,
                           int Hq, int Hkv, int nb, int blk, float scale, int nsegA, bool zt, int sms,
-                          float* scores, float* parta, cudaStream_t stream);
+                          float* scores, float* parta, int topk, int32_t* idx, bool* topk_done,
+                          cudaStream_t stream);
 uint32_t decode_tc_error_take();
 
 // ---------------------------------------------------------------- device side

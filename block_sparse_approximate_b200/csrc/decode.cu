@@ -485,159 +485,14 @@ decode_stats_kernel(const __nv_bfloat16* __restrict__ q, const TS* __restrict__ 
 }
 
 // ---- B. top-k ------------------------------------------------------------
-// Radix select over the 32-bit order keys of the scores (higher score =
-// smaller key).  The keys of one row share their high bits (the scores span
-// a narrow range), so the select starts below the highest bit in which the
-// row's smallest and largest keys differ, and takes 8-bit digits from there:
-// each pass histograms the digit of the keys that still match the prefix
-// found so far, and the bin holding the k-th key extends the prefix.  Once
-// that bin holds exactly the places left, every key in it is kept and the
-// lower bits do not matter (usually after two passes); otherwise the passes
-// run down to bit 0 and, of the keys equal to the k-th, the smallest indices
-// fill the places left.  The kept indices are emitted in ascending order from
-// a bitmap.
-constexpr int kTopkKPT = kMaxRouteBlocks / kDecThreads;   // keys per thread
-
+// The top-k of each (sequence, KV head) row: radix_topk_cta (topk.cuh).
 __global__ void __launch_bounds__(kDecThreads)
 decode_topk_kernel(const float* __restrict__ scores, int nb, int topk, int32_t* __restrict__ idx) {
   pdl_wait();
   pdl_trigger();
+  __shared__ RadixTopkSmem sm;
   const int pair = blockIdx.x;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  __shared__ unsigned hist[256];
-  __shared__ uint32_t bits[kMaxRouteBlocks / 32];
-  __shared__ unsigned sh_prefix, sh_rank, sh_cnt;
-  __shared__ unsigned sh_min[kDecWarps], sh_max[kDecWarps];
-  const float* sc = scores + (size_t)pair * nb;
-  int32_t* out = idx + (size_t)pair * topk;
-  const int nwords = (nb + 31) / 32;
-
-  uint32_t key[kTopkKPT];
-  unsigned kmin = 0xffffffffu, kmax = 0u;
-#pragma unroll
-  for (int e = 0; e < kTopkKPT; ++e) {
-    const int j = tid + e * kDecThreads;
-    key[e] = j < nb ? ~order_key(sc[j]) : 0xffffffffu;
-    if (j < nb) {
-      kmin = min(kmin, key[e]);
-      kmax = max(kmax, key[e]);
-    }
-  }
-  for (int x = tid; x < nwords; x += kDecThreads) bits[x] = 0u;
-  kmin = __reduce_min_sync(0xffffffffu, kmin);
-  kmax = __reduce_max_sync(0xffffffffu, kmax);
-  if (lane == 0) {
-    sh_min[warp] = kmin;
-    sh_max[warp] = kmax;
-  }
-  __syncthreads();
-  kmin = sh_min[0];
-  kmax = sh_max[0];
-#pragma unroll
-  for (int w = 1; w < kDecWarps; ++w) {
-    kmin = min(kmin, sh_min[w]);
-    kmax = max(kmax, sh_max[w]);
-  }
-  // bits above `hi` are common to every key of the row
-  const unsigned diff = kmin ^ kmax;
-  int hi = diff ? 31 - __clz(diff) : -1;
-  unsigned mask = diff == 0u ? 0xffffffffu : (hi >= 31 ? 0u : ~((2u << hi) - 1u));
-  unsigned prefix = kmin & mask;
-  unsigned rank = (unsigned)topk, cnt = (unsigned)nb;
-  while (hi >= 0 && cnt != rank) {
-    const int lo = max(hi - 7, 0);
-    const unsigned dmask = (2u << (hi - lo)) - 1u;      // the digit's bits, shifted down
-    for (int x = tid; x < 256; x += kDecThreads) hist[x] = 0u;
-    __syncthreads();
-#pragma unroll
-    for (int e = 0; e < kTopkKPT; ++e) {
-      const int j = tid + e * kDecThreads;
-      if (j < nb && (key[e] & mask) == prefix) atomicAdd(&hist[(key[e] >> lo) & dmask], 1u);
-    }
-    __syncthreads();
-    if (warp == 0) {
-      // the bin holding the rank-th smallest key among those matching prefix
-      unsigned c[8], tot = 0;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        c[e] = hist[lane * 8 + e];
-        tot += c[e];
-      }
-      unsigned incl = tot;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      const unsigned excl = incl - tot;
-      if (excl < rank && rank <= incl) {
-        unsigned run = excl;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          if (run < rank && rank <= run + c[e]) {
-            sh_prefix = prefix | ((unsigned)(lane * 8 + e) << lo);
-            sh_rank = rank - run;
-            sh_cnt = c[e];
-          }
-          run += c[e];
-        }
-      }
-    }
-    __syncthreads();
-    prefix = sh_prefix;
-    rank = sh_rank;
-    cnt = sh_cnt;
-    mask |= dmask << lo;
-    hi = lo - 1;
-  }
-  // keep every key whose determined bits are below the prefix, and of the
-  // keys matching it: all of them when they fill the places left exactly,
-  // else (all bits determined: ties) the smallest indices
-  const bool all_eq = cnt == rank;
-#pragma unroll
-  for (int e = 0; e < kTopkKPT; ++e) {
-    const int j = tid + e * kDecThreads;
-    if (j < nb) {
-      const unsigned km = key[e] & mask;
-      if (km < prefix || (all_eq && km == prefix)) atomicOr(&bits[j >> 5], 1u << (j & 31));
-    }
-  }
-  if (!all_eq && warp == 0) {
-    // ties at the threshold key (mask covers every bit): the smallest indices first
-    unsigned left = rank;
-    for (int j0 = 0; j0 < nb && left > 0; j0 += 32) {
-      const int j = j0 + lane;
-      const bool eq = j < nb && ~order_key(sc[j]) == prefix;
-      const unsigned bal = __ballot_sync(0xffffffffu, eq);
-      const unsigned before = __popc(bal & ((1u << lane) - 1u));
-      if (eq && before < left) atomicOr(&bits[j >> 5], 1u << (j & 31));
-      const unsigned n = __popc(bal);
-      left = n >= left ? 0u : left - n;
-    }
-  }
-  __syncthreads();
-  if (warp == 0) {
-    int base = 0;
-    for (int x0 = 0; x0 < nwords; x0 += 32) {
-      const int x = x0 + lane;
-      const uint32_t word = x < nwords ? bits[x] : 0u;
-      const int cnt_w = __popc(word);
-      int pre = cnt_w;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, pre, o);
-        if (lane >= o) pre += y;
-      }
-      int pos = base + pre - cnt_w;
-      uint32_t m = word;
-      while (m) {
-        const int bpos = __ffs(m) - 1;
-        out[pos++] = x * 32 + bpos;
-        m &= m - 1;
-      }
-      base += __shfl_sync(0xffffffffu, pre, 31);
-    }
-  }
+  radix_topk_cta<kDecThreads>(scores + (size_t)pair * nb, nb, topk, idx + (size_t)pair * topk, sm);
 }
 
 // ---- C. exact pass over the selected blocks --------------------------------
@@ -1447,6 +1302,7 @@ sa_status launch_decode(const void* q, const void* Kc, const void* Vc, const sa_
   float* partr = rla ? reinterpret_cast<float*>(ws + L.partr_off) : nullptr;
   const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(q);
   const int sms = sm_count();
+  bool topk_done = false;   // the tensor-core statistics pass may select the blocks itself
 
   // A
   {
@@ -1471,7 +1327,7 @@ sa_status launch_decode(const void* q, const void* Kc, const void* Vc, const sa_
       if (D == 128 && g <= 16) {
         // bf16 statistics, d = 128: the tcgen05 statistics pass (decode_tc.cu)
         r0 = decode_stats_tc(qb, ds.kmean, ds.kvar, ds.vrow, s.B, s.Hq, s.Hkv, nb, s.block, scale, L.nsegA, zt,
-                             sms, scores, parta, stream);
+                             sms, scores, parta, topk, idx, &topk_done, stream);
       } else {
         // bf16 statistics otherwise: the mma.sync statistics pass (one or two CTAs per SM)
         const size_t smemM = ((sizeof(float) * kDecWarps * g * (D + 2) + 127) & ~(size_t)127) +
@@ -1493,8 +1349,8 @@ sa_status launch_decode(const void* q, const void* Kc, const void* Vc, const sa_
   }
   sa_status r = SA_OK;
 
-  // B
-  if (topk > 0) {
+  // B (unless the statistics pass selected the blocks already)
+  if (topk > 0 && !topk_done) {
     {
       const cudaError_t le = launch_pdl(decode_topk_kernel, dim3(npairs), dim3(kDecThreads), 0, stream, scores, nb, topk, idx);
       if (le != cudaSuccess) return fail(SA_ERR_CUDA, std::string("decode_topk_kernel: ") + cudaGetErrorString(le));

@@ -27,6 +27,7 @@
 // returns.
 #include "attn_simt.cuh"
 #include "tc_util.cuh"
+#include "topk.cuh"
 
 namespace sa {
 namespace {
@@ -42,6 +43,7 @@ constexpr uint32_t kStSpan = kStTile * 128;   // 128 rows of one 128-byte swizzl
 constexpr uint32_t kStArr = 2 * kStSpan;      // a 128 x 128 bf16 tile: 32 KB
 constexpr uint32_t kStBop = 2 * kStN * 128;   // a 16 x 128 bf16 operand (two spans): 4 KB
 constexpr uint32_t kStTmemCols = 128;         // two buffers of S1 (16), S2 (16), O (16 of 32)
+constexpr int kStTopkBlocks = 2048;           // rows up to this many blocks take their top-k here
 
 template <bool ZT>
 struct StLayout {
@@ -53,7 +55,9 @@ struct StLayout {
   static constexpr uint32_t kBar = kRed + 2 * 4 * kStN * 2 * 4;
   enum { B_FK = 0, B_EK = 2, B_FV = 4, B_EV = 6, B_SC = 8, B_PR = 10, B_OC = 12, B_TF = 14, B_FIN = 16, NBAR = 17 };
   static constexpr uint32_t kSlot = kBar + 8 * NBAR;          // tmem base, abort flag
-  static constexpr size_t bytes() { return 1024 + kSlot + 16; }
+  static constexpr uint32_t kScores = kSlot + 16;             // the row's scores (fused top-k)
+  static constexpr uint32_t kTopk = kScores + 4 * kStTopkBlocks;   // RadixTopkSmem
+  static constexpr size_t bytes() { return 1024 + kTopk + sizeof(RadixTopkSmem); }
 };
 
 // Byte offset of element (row h, column c) of a 16 x 128 bf16 operand in the
@@ -109,7 +113,7 @@ __global__ void __launch_bounds__(kStThreads, 1)
 decode_stats_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmVar,
                        const __grid_constant__ CUtensorMap tmV, const __nv_bfloat16* __restrict__ q, int Hq,
                        int Hkv, int nb, float scale, float bias2, int nsegA, int splits, float* __restrict__ scores,
-                       float* __restrict__ parta) {
+                       float* __restrict__ parta, int topk, int32_t* __restrict__ idx) {
   using L = StLayout<ZT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -122,6 +126,9 @@ decode_stats_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kSlot);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kSlot + 4);
+  // with `idx`, the CTA holds the whole row of its pair (one tile range per
+  // pair) and selects its top-k at the end
+  float* scs = reinterpret_cast<float*>(smem + L::kScores);
   auto bar = [&](int k) { return sb + L::kBar + 8u * k; };
 
   if (threadIdx.x == 0) {
@@ -325,7 +332,11 @@ decode_stats_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
 #pragma unroll
         for (int h = 0; h < kStN; ++h)
           if (h < g && valid) se += fast_exp2(x[h] - mx) * (1.0f + __uint_as_float(sv[16 + h]));
-        if (valid) scores[(size_t)pair * nb + j0 + j] = (mx + __log2f(se)) * kLn2;
+        if (valid) {
+          const float sc = (mx + __log2f(se)) * kLn2;
+          scores[(size_t)pair * nb + j0 + j] = sc;
+          if (idx) scs[j0 + j] = sc;
+        }
         if (!group_and(grp, true)) break;   // the heads' sums are in `red`
         if (j < g) {
           float* out = parta + (((size_t)b * Hq + kh * g + j) * nsegA + seg) * (kStD + 2);
@@ -357,7 +368,11 @@ decode_stats_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
 #pragma unroll
         for (int h = 0; h < kStN; ++h)
           if (h < g && valid) se += fast_exp2(x[h] - mx) * (1.0f + __uint_as_float(sv[16 + h]));
-        if (valid) scores[(size_t)pair * nb + j0 + j] = (mx + __log2f(se)) * kLn2;
+        if (valid) {
+          const float sc = (mx + __log2f(se)) * kLn2;
+          scores[(size_t)pair * nb + j0 + j] = sc;
+          if (idx) scs[j0 + j] = sc;
+        }
       }
       tc_fence_before();
       __syncwarp();
@@ -370,13 +385,17 @@ decode_stats_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
     tc_fence_after();
     tmem_dealloc(tbase, kStTmemCols);
   }
+  if (idx && !*abort_flag)
+    radix_topk_cta<kStThreads>(scs, nb, topk, idx + (size_t)pair * topk,
+                               *reinterpret_cast<RadixTopkSmem*>(smem + L::kTopk));
 }
 
 }  // namespace
 
 sa_status decode_stats_tc(const __nv_bfloat16* q, const void* kmean, const void* kvar, const void* vmean, int B,
                           int Hq, int Hkv, int nb, int blk, float scale, int nsegA, bool zt, int sms,
-                          float* scores, float* parta, cudaStream_t stream) {
+                          float* scores, float* parta, int topk, int32_t* idx, bool* topk_done,
+                          cudaStream_t stream) {
   const int npairs = B * Hkv;
   CUtensorMap mk, mvar, mv;
   if (!make_tmap_128x128(&mk, kmean, 2, kStD, (uint64_t)nb, (uint64_t)npairs) ||
@@ -387,12 +406,15 @@ sa_status decode_stats_tc(const __nv_bfloat16* q, const void* kmean, const void*
   int splits = npairs < sms ? sms / npairs : 1;
   if (splits > nsegA) splits = nsegA;
   const dim3 grid((unsigned)(npairs * splits));
+  // a CTA that holds a whole row of at most kStTopkBlocks blocks selects its top-k
+  const bool fuse = splits == 1 && nb <= kStTopkBlocks && topk > 0 && idx != nullptr;
+  *topk_done = fuse;
   const size_t smem = zt ? StLayout<true>::bytes() : StLayout<false>::bytes();
   auto kern = zt ? decode_stats_tc_kernel<true> : decode_stats_tc_kernel<false>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return launch_status("cudaFuncSetAttribute(decode_stats_tc_kernel)");
   kern<<<grid, kStThreads, smem, stream>>>(mk, mvar, mv, q, Hq, Hkv, nb, scale, log2f((float)blk), nsegA, splits,
-                                           scores, parta);
+                                           scores, parta, topk, fuse ? idx : nullptr);
   return launch_status("decode_stats_tc_kernel");
 }
 
