@@ -356,6 +356,9 @@ def _bf16_round(x: np.ndarray) -> np.ndarray:
     (1, 4, 4, 4096, 128, 128, 5),
     (2, 8, 1, 2048, 64, 64, 3),
     (3, 6, 3, 64 * 77, 128, 64, 7),         # ragged split ranges
+    (4, 32, 4, 8192, 128, 64, 16),          # 8 heads per KV head; whole rows per CTA (fused top-k)
+    (1, 8, 2, 64 * 300, 128, 64, 20),       # rows of three 128-block tiles, the last ragged
+    (40, 8, 2, 64 * 300, 128, 64, 20),      # the same rows held whole by one CTA each (fused top-k)
 ])
 def test_decode_bf16_stats(lib, tail, B, Hq, Hkv, N, d, block, k):
     # the decode reading the bf16 copies of kmean, kvar and vsum / block: its
