@@ -202,6 +202,29 @@ __device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float
   return lo | (hi << 16);
 }
 
+// L2 prefetch of the Q tile and the first `ntiles` selected K/V tiles of
+// the CTA one SM count further in launch order (grid x = query block,
+// y = batch·head), the one most likely to take this SM next.
+template <int kSpans>
+__device__ __forceinline__ void prefetch_next_cta(const CUtensorMap* tmQ, const CUtensorMap* tmK,
+                                                  const CUtensorMap* tmV, const int32_t* block_idx, int nb,
+                                                  int topk, int ntiles) {
+  const uint32_t nl = blockIdx.y * gridDim.x + blockIdx.x + sm_count_reg();
+  if (nl >= gridDim.x * gridDim.y) return;
+  const int ni = (int)(nl % gridDim.x), nbh = (int)(nl / gridDim.x);
+#pragma unroll
+  for (int h = 0; h < kSpans; ++h) tma_prefetch_3d(tmQ, 64 * h, ni * TB, nbh);
+  const int32_t* nsel = block_idx + ((size_t)nbh * nb + ni) * topk;
+  for (int u = 0; u < ntiles && u < topk; ++u) {
+    const int nr = nsel[u] * TB;
+#pragma unroll
+    for (int h = 0; h < kSpans; ++h) {
+      tma_prefetch_3d(tmK, 64 * h, nr, nbh);
+      tma_prefetch_3d(tmV, 64 * h, nr, nbh);
+    }
+  }
+}
+
 template <bool ZO, bool F8, bool FO>
 __global__ void __launch_bounds__(kTcThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -305,6 +328,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         for (int h = 0; h < kSpans; ++h) tma_load_3d(va + h * kSpan, mv, 64 * h, row, bh, bar(L::B_VF + s));
         issued = t + 1;
       }
+      // every load of this CTA is issued: warm L2 for the CTA that most
+      // likely takes this SM next, so its prologue reads L2, not HBM
+      prefetch_next_cta<kSpans>(&tmQ, &tmK, &tmV, block_idx, nb, topk, NS);
       if (*abort_flag) {
         // let the loads already in flight land before the CTA goes away
         wait_bounded(bar(L::B_Q), 0);
@@ -777,6 +803,7 @@ attn_tc_linmix_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
         tma_load_3d(va + kSpan, &tmV, 64, row, bh, bar(L::B_VF + s));
         issued = t + 1;
       }
+      prefetch_next_cta<2>(&tmQ, &tmK, &tmV, block_idx, nb, topk, NS);
       if (*abort_flag) {
         wait_bounded(bar(L::B_Q), 0);
         for (int t = issued > NS ? issued - NS : 0; t < issued; ++t) {
