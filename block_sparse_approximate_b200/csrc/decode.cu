@@ -537,6 +537,14 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
                : "r"(addr));
 }
 
+// floats of the exact pass's merge rows ([g][8 warps][D + 2]), rounded up to
+// 128 bytes; sized by the group rather than its maximum so that the pass
+// leaves room on the SM for a combine CTA, which then runs its prologue
+// while the pass streams
+__host__ __device__ constexpr int exact_merge_floats(int g, int D) {
+  return (kDecWarps * g * (D + 2) + 31) & ~31;
+}
+
 template <int D, bool RLA>
 __global__ void __launch_bounds__(kDecThreads, 1)
 decode_exact_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ Kc,
@@ -553,11 +561,11 @@ decode_exact_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
   constexpr uint32_t kStageB = 2 * kArrB;
   constexpr int kSegBlocksMax = kSegC * kStageTokC / 64;   // blocks of a segment (blk >= 64)
   extern __shared__ __align__(16) uint8_t dsm[];
-  float* mg = reinterpret_cast<float*>(dsm);                         // [8 warps][g][D + 2] merge
-  int* itab = reinterpret_cast<int*>(mg + kDecWarps * kMaxGroup * (D + 2));   // [segments][blocks]
+  const int g = Hq / Hkv;
+  float* mg = reinterpret_cast<float*>(dsm);                         // [g][8 warps][D + 2] merge
+  int* itab = reinterpret_cast<int*>(mg + exact_merge_floats(g, D));   // [segments][blocks]
   uint8_t* ring = reinterpret_cast<uint8_t*>(itab + kItabSegs * kSegBlocksMax);
   const uint32_t ring_s = (uint32_t)__cvta_generic_to_shared(ring);
-  const int g = Hq / Hkv;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int tok_pair = topk * blk;                  // exact tokens of one (sequence, KV head)
   const int nstage_pair = (tok_pair + kStageTokC - 1) / kStageTokC;   // the last may hold 64
@@ -749,7 +757,7 @@ decode_exact_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
       lq += __shfl_xor_sync(0xffffffffu, lq, 1);
       lq += __shfl_xor_sync(0xffffffffu, lq, 2);
       if (hvalid) {
-        float* mw = mg + ((size_t)warp * kMaxGroup + hrow) * (D + 2);
+        float* mw = mg + ((size_t)hrow * kDecWarps + warp) * (D + 2);
         if ((lane & 3) == 0) {
           mw[0] = m_run;
           mw[1] = lq;
@@ -765,12 +773,12 @@ decode_exact_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
         const int hh = x / D, c = x % D;
         float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, mg[((size_t)w * kMaxGroup + hh) * (D + 2)]);
+        for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, mg[((size_t)hh * kDecWarps + w) * (D + 2)]);
         float L = 0.f, A = 0.f;
         if (M != -INFINITY) {
 #pragma unroll
           for (int w = 0; w < kDecWarps; ++w) {
-            const float* mw = mg + ((size_t)w * kMaxGroup + hh) * (D + 2);
+            const float* mw = mg + ((size_t)hh * kDecWarps + w) * (D + 2);
             if (mw[0] == -INFINITY) continue;
             const float f = fast_exp2(mw[0] - M);
             L = fmaf(mw[1], f, L);
@@ -788,7 +796,7 @@ decode_exact_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
       if (RLA) {
         // the residual linear sums add without a maximum: sum the warps'
         if (hvalid) {
-          float* mw = mg + ((size_t)warp * kMaxGroup + hrow) * (D + 2);
+          float* mw = mg + ((size_t)hrow * kDecWarps + warp) * (D + 2);
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
             mw[8 * nt + 2 * (lane & 3)] = o2[RLA ? nt : 0][0];
@@ -800,7 +808,7 @@ decode_exact_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
           const int hh = x / D, c = x % D;
           float A = 0.f;
 #pragma unroll
-          for (int w = 0; w < kDecWarps; ++w) A += mg[((size_t)w * kMaxGroup + hh) * (D + 2) + c];
+          for (int w = 0; w < kDecWarps; ++w) A += mg[((size_t)hh * kDecWarps + w) * (D + 2) + c];
           partr[(((size_t)b * Hq + kh * g + hh) * nsegC + sseg) * D + c] = A;
         }
         __syncthreads();
@@ -1071,197 +1079,249 @@ decode_stats_mma_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16
 }
 
 // ---- D. merge ------------------------------------------------------------
-// One CTA of D threads per (query head, sequence), thread = channel.  It
-// merges the statistics pass's partial states (the zero-order term of every
-// block) with the exact pass's (the selected blocks token by token) under
-// their common maximum M, then subtracts the zero-order term of each
-// selected block (SPLA §2.2's subtraction applied to PISA's tail: the
-// statistics pass cannot know the selection), so that the tail holds the
-// unselected blocks only.  The subtraction cannot go below zero: for every
-// block Σ_n e^{x_n} ≥ B e^{mean x}, and M bounds every block's zero-order
-// logit, so no weight exceeds 1.
-// kParts x D threads: thread (part, channel); each part takes every
-// kParts-th partial state and selected block, and the parts' sums meet in
-// shared memory.  Shared memory (dynamic): per partial state its max, sum
-// and merge weight, per selected block its index and log2 zero-order
-// weight, then the parts' sums; loads that do not depend on one another are
-// issued together.
-constexpr int kParts = 4;
+// One CTA of D threads per (sequence, KV head), thread = channel, for the
+// group's G query heads.  It merges the statistics pass's partial states (the
+// zero-order term of every block) with the exact pass's (the selected blocks
+// token by token) under their common maximum, after subtracting the
+// zero-order term of each selected block (SPLA §2.2's subtraction applied to
+// PISA's tail: the statistics pass cannot know the selection), so that the
+// tail holds the unselected blocks only.  The subtraction cannot go below
+// zero: for every block Σ_n e^{x_n} ≥ B e^{mean x}, and the statistics
+// states' maximum M_A bounds every block's zero-order logit, so no weight
+// 2^{x_j − M_A} exceeds 1.
+// Everything but the exact pass's states is formed before the PDL wait: the
+// statistics states merged per head under M_A, the selected blocks' weights
+// (q·k̄_j, a warp per block) subtracted there, and with the residual linear
+// tail φ(q)ᵀ S_all.  The exact pass leaves room for one such CTA per SM, so
+// with at most one CTA per SM this work overlaps the pass and after it only
+// the exact states' merge remains.  States are merged a chunk at a time
+// (online, as the passes merge tokens): their (max, sum) pairs staged in
+// shared memory, the maxima and weights formed by a warp per head, and each
+// thread's channel values loaded in batches of 32 / G so that the loads of
+// a batch are in flight together.
 constexpr float kRmsEps = 1e-6f;     // RMSNorm of SPLA's residual linear output
+constexpr int kSelChunk = 64;        // selected blocks whose weights are staged at once
+constexpr int kStChunk = 128;        // (head, state) pairs staged at once
 
 __device__ __forceinline__ float ld_stat(const float* p) { return __ldg(p); }
 __device__ __forceinline__ float ld_stat(const __nv_bfloat16* p) { return __bfloat162float(__ldg(p)); }
 
+// shared memory of decode_combine_kernel (floats)
+__host__ __device__ constexpr int combine_smem_floats(int g, int D, bool rla) {
+  return g * D + (rla ? g * D : 0) + 2 * kStChunk + g * kSelChunk + kSelChunk + 3 * g + g * (D / 32);
+}
+
 // TS, kmean, vrow, vmul: the statistics as the statistics pass read them
 // (vmul turns a row of vrow into the block's value mean)
-template <int D, typename TS>
-__global__ void __launch_bounds__(kParts * D)
+template <int D, int G, typename TS>
+__global__ void __launch_bounds__(D, 640 / D)
 decode_combine_kernel(const float* __restrict__ parta, int nsegA, const float* __restrict__ partc, int nsegC,
                       int use_tail, const float* __restrict__ partr, const __nv_bfloat16* __restrict__ q,
                       const TS* __restrict__ kmean, const TS* __restrict__ vrow, float vmul,
                       const float* __restrict__ sexp, const int32_t* __restrict__ idx, int topk, int nb, int blk,
-                      float scale, int Hq, int Hkv, __nv_bfloat16* __restrict__ O) {
+                      float scale, int Hkv, __nv_bfloat16* __restrict__ O) {
   // Everything up to the pdl_wait() below comes from the earlier launches of
   // the step (statistics pass, top-k), which had completed before the exact
   // pass read the selection; only the exact pass's partial states (partc,
-  // partr) are read after it, so this prologue overlaps the exact pass's tail.
-  constexpr int kT = kParts * D, kW = kT / 32;
+  // partr) are read after it.
+  constexpr int kW = D / 32;
+  constexpr int kB = 32 / G;                                   // states per load batch
   extern __shared__ __align__(16) float csm[];
-  const int na = use_tail ? nsegA : 0, ns = na + nsegC;
-  const bool subtract = use_tail && nsegC > 0;
-  const int nsel = subtract ? topk : 0;
-  float* red = csm;                                        // [kParts][2][D] the parts' sums
-  float* hm = red + kParts * 2 * D;                        // [ns] partial maxima
-  float* hl = hm + ns;                                     // [ns] partial sums
-  float* hf = hl + ns;                                     // [ns] merge weights
-  float* xsel = hf + ns;                                   // [nsel] log2 zero-order weights
-  int* jsel = reinterpret_cast<int*>(xsel + nsel);         // [nsel] block indices
-  float* rr = reinterpret_cast<float*>(jsel + nsel);        // [kParts][D] residual parts, [D/32] squares
-  const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
-  const int c = tid % D, pt = tid / D;
-  const int lane = tid & 31, warp = tid >> 5;
-  const float* pa = parta + ((size_t)b * Hq + h) * nsegA * (D + 2);
-  const float* pc = partc + ((size_t)b * Hq + h) * nsegC * (D + 2);
-  const int pair = b * Hkv + h / (Hq / Hkv);
-  auto part = [&](int sidx) { return sidx < na ? pa + (size_t)sidx * (D + 2) : pc + (size_t)(sidx - na) * (D + 2); };
-  for (int x = tid; x < na; x += kT) {
-    const float* r = part(x);
-    hm[x] = r[0];
-    hl[x] = r[1];
+  const int Hq = Hkv * G;
+  const int pair = blockIdx.x, b = pair / Hkv;
+  const size_t row0 = (size_t)b * Hq + (size_t)(pair % Hkv) * G;   // the group's heads: rows row0 .. row0 + G - 1
+  const int c = threadIdx.x, lane = c & 31, warp = c >> 5;
+  const int na = use_tail ? nsegA : 0;
+  const int nsel = (use_tail && nsegC > 0) ? topk : 0;
+  const bool rla = partr != nullptr;
+  float* qs = csm;                                             // [G][D] s log2e q
+  float* fq = qs + G * D;                                      // [G][D] φ(q) in bf16 (residual linear)
+  float* sm = fq + (rla ? G * D : 0);                          // [kStChunk] state maxima, then weights
+  float* sl = sm + kStChunk;                                   // [kStChunk] state sums
+  float* wsel = sl + kStChunk;                                 // [G][kSelChunk] weights 2^{x_j − M_A}
+  int* jsel = reinterpret_cast<int*>(wsel + G * kSelChunk);    // [kSelChunk] block indices
+  float* hM = reinterpret_cast<float*>(jsel + kSelChunk);      // [G] running maximum per head
+  float* hL = hM + G;                                          // [G] running sum per head
+  float* hS = hL + G;                                          // [G] rescale of the last chunk
+  float* red = hS + G;                                         // [G][kW] RMS partial sums
+  const float scale2 = scale * kLog2e, bias2 = log2f((float)blk);
+  for (int x = c; x < G * D; x += D) {
+    const float qv = __bfloat162float(q[row0 * D + x]);
+    qs[x] = scale2 * qv;
+    // φ(q) rounded to bf16 as in the exact pass's operand, so that the two
+    // terms of the residual's difference use the same feature values
+    if (rla) fq[x] = __bfloat162float(__float2bfloat16_rn(phi_exp(qv)));
   }
-  for (int x = tid; x < nsel; x += kT) jsel[x] = __ldg(idx + (size_t)pair * topk + x);
-  __syncthreads();
-  // this thread's partial-state channels and selected-block vsum channels,
-  // loaded now (they do not depend on the maximum) so their latency overlaps
-  // the dot products below
-  constexpr int kPreP = 8, kPreV = 16;
-  float pv[kPreP], vv[kPreV];
-#pragma unroll
-  for (int e = 0; e < kPreP; ++e) {
-    const int x = pt + kParts * e;
-    pv[e] = x < na ? part(x)[2 + c] : 0.f;
+  if (c < G) {
+    hM[c] = -INFINITY;
+    hL[c] = 0.f;
   }
+  __syncthreads();   // qs, fq, hM, hL
+  float A[G];
 #pragma unroll
-  for (int e = 0; e < kPreV; ++e) {
-    const int si = pt + kParts * e;
-    vv[e] = si < nsel ? ld_stat(vrow + ((size_t)pair * nb + jsel[si]) * D + c) : 0.f;
-  }
-  if (subtract) {
-    // s log2e q·k̄_j + log2 B of the selected blocks: a warp per block, the
-    // rows of four blocks in flight at once
-    const float scale2 = scale * kLog2e, bias2 = log2f((float)blk);
-    float qv[D / 32];
+  for (int hh = 0; hh < G; ++hh) A[hh] = 0.f;
+
+  // merge states x ∈ [0, nst) of the group's heads (rows of D + 2 floats at
+  // base + ((row0 + hh) nst + x)(D + 2)) into (hM, hL) and A
+  auto merge_states = [&](const float* base, int nst) {
+    constexpr int per = kStChunk / G;
+    for (int x0 = 0; x0 < nst; x0 += per) {
+      const int n = min(per, nst - x0);
+      for (int z = c; z < G * n; z += D) {
+        const float* r = base + ((row0 + z / n) * nst + x0 + z % n) * (D + 2);
+        sm[z] = r[0];
+        sl[z] = r[1];
+      }
+      __syncthreads();
+      for (int hh = warp; hh < G; hh += kW) {
+        float cm = -INFINITY;
+        for (int x = lane; x < n; x += 32) cm = fmaxf(cm, sm[hh * n + x]);
+        cm = warp_max(cm);
+        const float mo = hM[hh], mn = fmaxf(mo, cm);
+        float ls = 0.f;
+        for (int x = lane; x < n; x += 32) {
+          const float m = sm[hh * n + x];
+          const float w = m == -INFINITY ? 0.f : fast_exp2(m - mn);
+          sm[hh * n + x] = w;
+          ls = fmaf(sl[hh * n + x], w, ls);
+        }
+        ls = warp_sum(ls);
+        if (lane == 0) {
+          const float so = mo == -INFINITY ? 0.f : fast_exp2(mo - mn);
+          hS[hh] = so;
+          hL[hh] = fmaf(hL[hh], so, ls);
+          hM[hh] = mn;
+        }
+      }
+      __syncthreads();
 #pragma unroll
-    for (int e = 0; e < D / 32; ++e) qv[e] = scale2 * __bfloat162float(q[((size_t)b * Hq + h) * D + lane + 32 * e]);
-    for (int s0 = warp * 4; s0 < nsel; s0 += kW * 4) {
-      float kk[4][D / 32];
+      for (int hh = 0; hh < G; ++hh) A[hh] *= hS[hh];
+      for (int x = 0; x < n; x += kB) {
+        float v[G][kB];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int si = min(s0 + u, nsel - 1);
-        const TS* kr = kmean + ((size_t)pair * nb + jsel[si]) * D;
+        for (int hh = 0; hh < G; ++hh)
+#pragma unroll
+          for (int u = 0; u < kB; ++u)
+            v[hh][u] = x + u < n ? base[((row0 + hh) * nst + x0 + x + u) * (D + 2) + 2 + c] : 0.f;
+#pragma unroll
+        for (int hh = 0; hh < G; ++hh)
+#pragma unroll
+          for (int u = 0; u < kB; ++u)
+            if (x + u < n) A[hh] = fmaf(v[hh][u], sm[hh * n + x + u], A[hh]);
+      }
+      __syncthreads();   // sm, sl are restaged by the next chunk
+    }
+  };
+
+  // the statistics pass's states (zero-order terms of every block) under M_A
+  merge_states(parta, na);
+
+  // subtract the zero-order term of each selected block (weight <= 1)
+  float lsub[G];
+#pragma unroll
+  for (int hh = 0; hh < G; ++hh) lsub[hh] = 0.f;
+  for (int s0 = 0; s0 < nsel; s0 += kSelChunk) {
+    const int n = min(kSelChunk, nsel - s0);
+    if (c < n) jsel[c] = __ldg(idx + (size_t)pair * topk + s0 + c);
+    __syncthreads();
+    // s log2e q_h·k̄_j + log2 B − M_A(h): a warp per block, eight blocks in flight
+    for (int u0 = warp * 8; u0 < n; u0 += kW * 8) {
+      float kk[8][D / 32];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const TS* kr = kmean + ((size_t)pair * nb + jsel[min(u0 + u, n - 1)]) * D;
 #pragma unroll
         for (int e = 0; e < D / 32; ++e) kk[u][e] = ld_stat(kr + lane + 32 * e);
       }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        float d = 0.f;
+      for (int hh = 0; hh < G; ++hh) {
+        const float ma = hM[hh];
 #pragma unroll
-        for (int e = 0; e < D / 32; ++e) d = fmaf(qv[e], kk[u][e], d);
-        d = warp_sum(d);
-        if (lane == 0 && s0 + u < nsel) xsel[s0 + u] = d + bias2;
+        for (int u = 0; u < 8; ++u) {
+          float d = 0.f;
+#pragma unroll
+          for (int e = 0; e < D / 32; ++e) d = fmaf(qs[hh * D + lane + 32 * e], kk[u][e], d);
+          d = warp_sum(d);
+          if (lane == 0 && u0 + u < n)
+            wsel[hh * kSelChunk + u0 + u] = ma == -INFINITY ? 0.f : fast_exp2(d + bias2 - ma);
+        }
       }
     }
-  }
-  pdl_wait();   // the exact pass's partial states from here on
-  for (int x = na + tid; x < ns; x += kT) {
-    const float* r = part(x);
-    hm[x] = r[0];
-    hl[x] = r[1];
-  }
-#pragma unroll
-  for (int e = 0; e < kPreP; ++e) {
-    const int x = pt + kParts * e;
-    if (x >= na && x < ns) pv[e] = part(x)[2 + c];
-  }
-  __syncthreads();
-  float M = -INFINITY;
-  for (int x = 0; x < ns; ++x) M = fmaxf(M, hm[x]);
-  for (int x = tid; x < ns; x += kT) hf[x] = (M == -INFINITY || hm[x] == -INFINITY) ? 0.f : fast_exp2(hm[x] - M);
-  __syncthreads();
-  float L = 0.f, A = 0.f;
-  if (M != -INFINITY) {
-#pragma unroll
-    for (int e = 0; e < kPreP; ++e) {
-      const int x = pt + kParts * e;
-      if (x < ns) {
-        L = fmaf(hl[x], hf[x], L);
-        A = fmaf(pv[e], hf[x], A);
-      }
-    }
-    for (int x = pt + kParts * kPreP; x < ns; x += kParts) {
-      L = fmaf(hl[x], hf[x], L);
-      A = fmaf(part(x)[2 + c], hf[x], A);
-    }
-    // subtract the zero-order term of each selected block (weight <= 1)
-#pragma unroll
-    for (int e = 0; e < kPreV; ++e) {
-      const int si = pt + kParts * e;
-      if (si < nsel) {
-        const float w = fast_exp2(xsel[si] - M);
-        L -= w;
-        A = fmaf(-w * vmul, vv[e], A);
-      }
-    }
-    for (int si = pt + kParts * kPreV; si < nsel; si += kParts) {
-      const float w = fast_exp2(xsel[si] - M);
-      L -= w;
-      A = fmaf(-w * vmul, ld_stat(vrow + ((size_t)pair * nb + jsel[si]) * D + c), A);
-    }
-  }
-  red[(pt * 2 + 0) * D + c] = L;
-  red[(pt * 2 + 1) * D + c] = A;
-  if (partr) {
-    // SPLA's residual: this part's rows r of φ(q)ᵀ S_all (column c) minus its
-    // exact segments' Σ (φ(q)·φ(k_n)) v_n
-    float rpart = 0.f;
-    const float* sa = sexp + (size_t)pair * D * D;
-    const __nv_bfloat16* qh = q + ((size_t)b * Hq + h) * D;
-    // φ(q) rounded to bf16 as in the exact pass's operand, so that the two
-    // terms of the difference use the same feature values
-    for (int r = pt; r < D; r += kParts)
-      rpart = fmaf(__bfloat162float(__float2bfloat16_rn(phi_exp(__bfloat162float(qh[r])))), sa[(size_t)r * D + c],
-                   rpart);
-    const float* pr = partr + ((size_t)b * Hq + h) * nsegC * D;
-    for (int x = pt; x < nsegC; x += kParts) rpart -= pr[(size_t)x * D + c];
-    rr[pt * D + c] = rpart;
-  }
-  __syncthreads();
-  float o_s = 0.f, res = 0.f;
-  if (pt == 0) {
-    L = 0.f;
-    A = 0.f;
-#pragma unroll
-    for (int p2 = 0; p2 < kParts; ++p2) {
-      L += red[(p2 * 2 + 0) * D + c];
-      A += red[(p2 * 2 + 1) * D + c];
-    }
-    o_s = L > 0.f ? A / L : 0.f;
-    if (partr) {
-#pragma unroll
-      for (int p2 = 0; p2 < kParts; ++p2) res += rr[p2 * D + c];
-    }
-  }
-  if (partr) {
-    // RMSNorm over the D channels (threads of part 0 = warps 0 .. D/32 - 1)
-    const float sq = warp_sum(res * res);
-    if (lane == 0 && warp < D / 32) rr[kParts * D + warp] = sq;
     __syncthreads();
-    float tot = 0.f;
+    for (int u0 = 0; u0 < n; u0 += 16) {
+      float v[16];
 #pragma unroll
-    for (int w = 0; w < D / 32; ++w) tot += rr[kParts * D + w];
-    res *= rsqrtf(tot / D + kRmsEps);
+      for (int u = 0; u < 16; ++u) v[u] = ld_stat(vrow + ((size_t)pair * nb + jsel[min(u0 + u, n - 1)]) * D + c);
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        if (u0 + u < n) {
+#pragma unroll
+          for (int hh = 0; hh < G; ++hh) {
+            const float w = wsel[hh * kSelChunk + u0 + u];
+            lsub[hh] += w;
+            A[hh] = fmaf(-w * vmul, v[u], A[hh]);
+          }
+        }
+      }
+    }
+    __syncthreads();   // jsel and wsel are restaged by the next chunk
   }
-  if (pt == 0) O[((size_t)b * Hq + h) * D + c] = __float2bfloat16_rn(o_s + res);
+  if (c == 0 && nsel > 0) {
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh) hL[hh] -= lsub[hh];
+  }
+
+  // SPLA's residual: φ(q)ᵀ S_all (column c) for each head of the group
+  float res[G];
+#pragma unroll
+  for (int hh = 0; hh < G; ++hh) res[hh] = 0.f;
+  if (rla) {
+    const float* sa = sexp + (size_t)pair * D * D;
+#pragma unroll 16
+    for (int r = 0; r < D; ++r) {
+      const float sv = __ldg(sa + (size_t)r * D + c);
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh) res[hh] = fmaf(fq[hh * D + r], sv, res[hh]);
+    }
+  }
+
+  pdl_wait();   // the exact pass's partial states from here on
+  merge_states(partc, nsegC);   // its first barrier orders thread 0's update of hL
+  if (rla) {
+    // minus the exact segments' Σ (φ(q)·φ(k_n)) v_n, then RMSNorm over the
+    // D channels of each head
+    for (int x = 0; x < nsegC; x += kB) {
+      float v[G][kB];
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh)
+#pragma unroll
+        for (int u = 0; u < kB; ++u) v[hh][u] = x + u < nsegC ? partr[((row0 + hh) * nsegC + x + u) * D + c] : 0.f;
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh)
+#pragma unroll
+        for (int u = 0; u < kB; ++u) res[hh] -= v[hh][u];
+    }
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh) {
+      const float sq = warp_sum(res[hh] * res[hh]);
+      if (lane == 0) red[hh * kW + warp] = sq;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh) {
+      float tot = 0.f;
+#pragma unroll
+      for (int w = 0; w < kW; ++w) tot += red[hh * kW + w];
+      res[hh] *= rsqrtf(tot / D + kRmsEps);
+    }
+  }
+  __syncthreads();   // hL
+#pragma unroll
+  for (int hh = 0; hh < G; ++hh) {
+    const float L = hL[hh];
+    const float o_s = L > 0.f ? A[hh] / L : 0.f;
+    O[(row0 + hh) * D + c] = __float2bfloat16_rn(o_s + res[hh]);
+  }
 }
 
 int sm_count() {
@@ -1361,7 +1421,7 @@ sa_status launch_decode(const void* q, const void* Kc, const void* Vc, const sa_
 
   // C
   if (topk > 0) {
-    const size_t smemC = sizeof(float) * kDecWarps * kMaxGroup * (D + 2) +
+    const size_t smemC = sizeof(float) * exact_merge_floats(s.Hq / s.Hkv, D) +
                          sizeof(int) * kItabSegs * (kSegC * kStageTokC / 64) +
                          (size_t)kRingC * 2 * kStageTokC * D * 2;
     auto kern = rla ? decode_exact_kernel<D, true> : decode_exact_kernel<D, false>;
@@ -1383,18 +1443,17 @@ sa_status launch_decode(const void* q, const void* Kc, const void* Vc, const sa_
   {
     const int use_tail = tail == SA_TAIL_ZERO_ORDER;
     const int nsc = topk > 0 ? L.nsegC : 0;
-    const int ns = (use_tail ? L.nsegA : 0) + nsc;
-    const int nsel = (use_tail && nsc > 0) ? topk : 0;
-    const size_t smemD = sizeof(float) * (kParts * 2 * D + 3 * (size_t)ns + 2 * (size_t)nsel +
-                                          (rla ? kParts * D + D / 32 : 0));
-    if (cudaFuncSetAttribute(decode_combine_kernel<D, TS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smemD) != cudaSuccess)
+    const float* pr = topk < nb ? partr : nullptr;
+    const int g = s.Hq / s.Hkv;
+    const size_t smemD = sizeof(float) * combine_smem_floats(g, D, pr != nullptr);
+    auto kern = g == 1 ? decode_combine_kernel<D, 1, TS> : g == 2 ? decode_combine_kernel<D, 2, TS>
+              : g == 4 ? decode_combine_kernel<D, 4, TS> : decode_combine_kernel<D, 8, TS>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smemD) != cudaSuccess)
       return launch_status("cudaFuncSetAttribute(decode_combine_kernel)");
     {
-      const cudaError_t le = launch_pdl(decode_combine_kernel<D, TS>, dim3(s.Hq, s.B), dim3(kParts * D), smemD,
-        stream, parta, L.nsegA, partc, nsc, use_tail, topk < nb ? partr : nullptr, qb, ds.kmean, ds.vrow, ds.vmul,
-        static_cast<const float*>(st.sexp), idx, topk, nb, s.block, scale, s.Hq, s.Hkv,
-        static_cast<__nv_bfloat16*>(O));
+      const cudaError_t le = launch_pdl(kern, dim3(npairs), dim3(D), smemD, stream, parta, L.nsegA, partc, nsc,
+        use_tail, pr, qb, ds.kmean, ds.vrow, ds.vmul, static_cast<const float*>(st.sexp), idx, topk, nb, s.block,
+        scale, s.Hkv, static_cast<__nv_bfloat16*>(O));
       if (le != cudaSuccess) return fail(SA_ERR_CUDA, std::string("decode_combine_kernel: ") + cudaGetErrorString(le));
     }
   }
