@@ -40,7 +40,7 @@ def _headers():
 
 # attn_tc_kernel and attn_tc_linmix_kernel reallocate registers with
 # setmaxnreg: their launch register count times 384 threads must cover the
-# split (256 x 216 + 128 x 40, and 128 x 216 + 128 x 96 + 128 x 40; see
+# split (256 x 216 + 128 x 40, and 128 x 216 + 128 x 96 + 128 x 56; see
 # attn_tc.cu), or setmaxnreg.inc would wait for registers that never come.
 TC_MIN_LAUNCH_REGS = 158
 
