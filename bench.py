@@ -56,7 +56,7 @@ def _peaks():
 # sources change the figure no longer describes the kernel and is reported as
 # null until it is captured again.
 ATTN_TRAFFIC = {"sources": ("csrc/attn_tc.cu", "csrc/tc_util.cuh", "csrc/common.cuh"),
-                "sha256": "1e586338 77c2c6eb 20b529c1", "bytes": 386.90e6}
+                "sha256": "d73ebb7f 77c2c6eb 20b529c1", "bytes": 386.42e6}
 
 
 def attn_traffic_bytes():
