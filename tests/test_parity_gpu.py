@@ -293,6 +293,10 @@ def test_value_shift_on_gpu(lib):
     (2, 8, 1, 2048, 64, 64, 0),
     (1, 4, 2, 2048, 128, 64, 32),           # every block selected
     (3, 6, 3, 64 * 77, 128, 64, 7),         # ragged split ranges
+    # 8 heads per KV head, 2304 blocks, top-160: the merge takes 18 statistics
+    # states and 20 exact states per head in chunks of 16, and the selected
+    # blocks' zero-order terms in chunks of 64
+    (1, 8, 1, 64 * 2304, 128, 64, 160),
 ])
 def test_decode(lib, tail, B, Hq, Hkv, N, d, block, k):
     w = wl.WORKLOADS["decode"]
@@ -359,6 +363,7 @@ def _bf16_round(x: np.ndarray) -> np.ndarray:
     (4, 32, 4, 8192, 128, 64, 16),          # 8 heads per KV head; whole rows per CTA (fused top-k)
     (1, 8, 2, 64 * 300, 128, 64, 20),       # rows of three 128-block tiles, the last ragged
     (40, 8, 2, 64 * 300, 128, 64, 20),      # the same rows held whole by one CTA each (fused top-k)
+    (1, 8, 1, 64 * 2304, 128, 64, 160),     # the merge's states and selected blocks in several chunks
 ])
 def test_decode_bf16_stats(lib, tail, B, Hq, Hkv, N, d, block, k):
     # the decode reading the bf16 copies of kmean, kvar and vsum / block: its
