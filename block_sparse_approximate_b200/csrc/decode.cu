@@ -3,23 +3,26 @@
 // SPLA §1-2 notes that decoding is bound by loading the KV cache and keeps
 // the IO profile of sparse decoding: only the selected blocks are read token
 // by token; every other block is represented by its precomputed statistics.
-// Four launches on the caller's stream:
-//   A. decode_stats_kernel  one pass over the block statistics (kmean, kvar,
-//        vsum, each read once): the SPLA §2.1 score of every block for each
-//        query head, summed over the GQA group (logsumexp) -> scores, and the
-//        PISA zero-order term of EVERY block -> per-segment partial states
-//        (max, sum, acc) per query head;
-//   B. decode_topk_kernel   top-k per (sequence, KV head) -> block_idx;
+// Up to four launches on the caller's stream, each started early by
+// programmatic dependent launch:
+//   A. the statistics pass (decode_stats_kernel for float32 statistics,
+//        decode_stats_mma_kernel for bf16 ones, decode_stats_tc_kernel in
+//        decode_tc.cu for bf16 ones with d = 128): one pass over kmean, kvar
+//        (and the value means), each read once: the SPLA §2.1 score of every
+//        block for each query head, summed over the GQA group (logsumexp)
+//        -> scores, and the PISA zero-order term of EVERY block -> per-segment
+//        partial states (max, sum, acc) per query head;
+//   B. decode_topk_kernel   top-k per (sequence, KV head) -> block_idx
+//        (skipped when the tensor-core statistics pass selected the blocks);
 //   C. decode_exact_kernel  the selected blocks token by token (exact online
-//        softmax), and for each selected block its own zero-order term with
-//        weight -1, so that A + C hold the zero-order term of the unselected
-//        blocks only (the subtraction form of SPLA §2.2 applied to PISA's
-//        tail; it cannot cancel below zero because Σ_n e^{x_n} ≥ B e^{mean x}
-//        for every block) -> per-segment partial states;
-//   D. decode_combine_kernel  merges the partial states -> o.
-// A and C are persistent streaming kernels: each CTA walks a list of
-// 48 KB / 32 KB stages staged into shared memory with cp.async, three or four
-// stages deep, so the HBM stays busy while the previous stage is reduced.
+//        softmax) -> per-segment partial states;
+//   D. decode_combine_kernel  merges A's states, subtracts each selected
+//        block's own zero-order term (the subtraction form of SPLA §2.2
+//        applied to PISA's tail; it cannot cancel below zero because
+//        Σ_n e^{x_n} ≥ B e^{mean x} for every block), merges C's states -> o.
+// A and C are persistent streaming kernels: each CTA walks a list of stages
+// staged into shared memory with cp.async (or TMA), several stages deep, so
+// the HBM stays busy while the previous stage is reduced.
 #include <cuda.h>
 
 #include <mutex>
